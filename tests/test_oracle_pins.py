@@ -1,0 +1,448 @@
+"""Pins of the CPU oracle to what the pages and the mathematics fix (no GPU).
+
+Each test states the fact it checks and where that fact comes from.  None of them re-types
+the oracle's own code: they use closed forms, invariants, special cases that reduce to a
+textbook result, and brute force with library routines on tiny inputs.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+from depth_recurrent_attention_b200 import configs, inputs
+
+RNG = np.random.default_rng(1234)
+
+
+def tiny_cfg(**kw):
+    return configs.TINY.with_(**kw)
+
+
+def rand_weights(cfg, seed=0, scale_o=1.0):
+    """Seeded fp32 weights for a small hand-made configuration."""
+    W = inputs.host_weights(cfg.with_(seed=seed))
+    if scale_o != 1.0:
+        W["w_o"] = (W["w_o"] * scale_o).astype(np.float32)
+    return W
+
+
+# ---------------------------------------------------------------------------------------
+# RMSNorm (papernotes "Overall framework": RMSNorm on the residual stream)
+
+def test_rmsnorm_worked_example():
+    # x = (3, 4): mean square 12.5, so x^ = (3, 4) / sqrt(12.5)
+    out = O.rmsnorm([3.0, 4.0], np.ones(2, np.float32), 0.0)
+    assert np.allclose(out, [3 / np.sqrt(12.5), 4 / np.sqrt(12.5)], rtol=0, atol=1e-15)
+
+
+def test_rmsnorm_unit_mean_square_and_scale_invariance():
+    x = RNG.normal(size=257) * 7.3
+    g = np.ones(257, np.float32)
+    eps = 1e-6
+    out = O.rmsnorm(x, g, eps)
+    ms = np.mean(x ** 2)
+    assert abs(np.mean(out ** 2) - ms / (ms + eps)) < 1e-12
+    out2 = O.rmsnorm(x * 1e3, g, 0.0)
+    assert np.allclose(out2, O.rmsnorm(x, g, 0.0), rtol=1e-13, atol=1e-13)
+    gg = RNG.normal(size=257).astype(np.float32)
+    assert np.allclose(O.rmsnorm(x, gg, eps), gg * out, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------------------
+# RoPE (rotate-half convention, Su et al. RoFormer) and depth RoPE with a reversed half
+# (papernotes "Key design 1"; gist.science "Methodology")
+
+def test_rope_two_dims_is_plain_rotation():
+    # n = 2: the single pair turns by pos * base^0 = pos radians
+    for pos in (0.0, 1.0, 2.5, 17.0):
+        v = O.rope([1.0, 0.0], pos)
+        assert np.allclose(v, [np.cos(pos), np.sin(pos)], atol=1e-15)
+        v = O.rope([0.0, 1.0], pos)
+        assert np.allclose(v, [-np.sin(pos), np.cos(pos)], atol=1e-15)
+
+
+def test_rope_pairing_and_ladder_special_values():
+    n = 16
+    for i in range(n // 2):
+        e = np.zeros(n)
+        e[i] = 1.0
+        v = O.rope(e, 3.0)
+        support = set(np.nonzero(np.abs(v) > 1e-15)[0].tolist())
+        assert support <= {i, i + n // 2}            # rotate-half pairs (i, i + n/2)
+    # n = 4, base 10^4: second pair turns 10^4^(-1/2) = 0.01 rad per position
+    e = np.array([0.0, 1.0, 0.0, 0.0])
+    v = O.rope(e, 1.0)
+    assert np.isclose(np.arctan2(v[3], v[1]), 0.01, atol=1e-15)
+
+
+def test_rope_norm_identity_and_relative_position():
+    d = 64
+    q, k = RNG.normal(size=d), RNG.normal(size=d)
+    assert np.allclose(O.rope(q, 0.0), q, atol=0)
+    assert np.isclose(np.linalg.norm(O.rope(q, 123.0)), np.linalg.norm(q), rtol=1e-14)
+    s1 = O.rope(q, 10.0) @ O.rope(k, 3.0)
+    s2 = O.rope(q, 57.0) @ O.rope(k, 50.0)
+    assert abs(s1 - s2) < 1e-11
+    # group property R_a R_b = R_{a+b}
+    assert np.allclose(O.rope(O.rope(q, 5.0), 9.0), O.rope(q, 14.0), atol=1e-12)
+
+
+def test_depth_rope_forward_half_depends_on_depth_difference_only():
+    d, L = 64, 16
+    q, k = RNG.normal(size=d), RNG.normal(size=d)
+    h2 = d // 2
+    for (l, j, c) in [(5, 2, 3), (7, 0, 6), (4, 4, 9)]:
+        a = O.depth_rope(q, l, L)[:h2] @ O.depth_rope(k, j, L)[:h2]
+        b = O.depth_rope(q, l + c, L)[:h2] @ O.depth_rope(k, j + c, L)[:h2]
+        assert abs(a - b) < 1e-11
+
+
+def test_depth_rope_reversed_half():
+    d, L = 64, 16
+    q, k = RNG.normal(size=d), RNG.normal(size=d)
+    h2 = d // 2
+    # second half sits at L-1-l: its score depends on j - l, i.e. the same shift reversed
+    a = O.depth_rope(q, 5, L)[h2:] @ O.depth_rope(k, 2, L)[h2:]
+    b = O.depth_rope(q, 8, L)[h2:] @ O.depth_rope(k, 5, L)[h2:]
+    assert abs(a - b) < 1e-11
+    # at depth 0 the first half is untouched and the second half turns to position L-1
+    v0 = O.depth_rope(q, 0, L)
+    assert np.array_equal(v0[:h2], q[:h2])
+    assert np.allclose(v0[h2:], O.rope(q[h2:], L - 1), atol=1e-15)
+    # at the last depth the roles swap
+    vL = O.depth_rope(q, L - 1, L)
+    assert np.allclose(vL[:h2], O.rope(q[:h2], L - 1), atol=1e-15)
+    assert np.array_equal(vL[h2:], q[h2:])
+    # and the two halves are not rotated alike at depths other than the middle one
+    assert not np.allclose(O.depth_rope(q, 2, L)[:h2] @ q[:h2],
+                           O.depth_rope(q, 2, L)[h2:] @ q[h2:])
+    assert np.isclose(np.linalg.norm(O.depth_rope(q, 3, L)), np.linalg.norm(q), rtol=1e-14)
+
+
+# ---------------------------------------------------------------------------------------
+# scaled dot-product attention / softmax
+
+def test_softmax_rows_sum_to_one_and_closed_forms():
+    d = 16
+    q = RNG.normal(size=d)
+    K = RNG.normal(size=(37, d))
+    V = RNG.normal(size=(37, d))
+    out, p = O.attend(q, K, V)
+    assert abs(p.sum() - 1.0) < 1e-12 * 37
+    # one key: the output is that key's value exactly (DA at depth 0 equals its V)
+    out1, p1 = O.attend(q, K[:1], V[:1])
+    assert np.array_equal(out1, V[0]) and p1[0] == 1.0
+    # identical keys: uniform weights, output is the mean of the values
+    Ke = np.repeat(K[:1], 5, axis=0)
+    oute, pe = O.attend(q, Ke, V[:5])
+    assert np.allclose(pe, 0.2, atol=1e-15) and np.allclose(oute, V[:5].mean(0), atol=1e-14)
+    # two keys: weight of key 1 is sigmoid(s1 - s0), scores scaled by 1/sqrt(d)
+    s = K[:2] @ q / np.sqrt(d)
+    _, p2 = O.attend(q, K[:2], V[:2])
+    assert np.isclose(p2[1], 1 / (1 + np.exp(-(s[1] - s[0]))), rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------------------
+# routing sigma(x) = norm(TopK(sigmoid(x), x + b, k))   (papernotes "Key design 2")
+
+def test_topk_matches_sort_with_index_tiebreak():
+    for E, k in [(16, 2), (256, 4), (1024, 8), (33, 33)]:
+        z = RNG.normal(size=E)
+        b = RNG.uniform(-0.1, 0.1, size=E).astype(np.float32)
+        idx, w, margin = O.topk(z, b, k)
+        key = z + b.astype(np.float64)
+        order = sorted(range(E), key=lambda e: (-key[e], e))
+        assert list(idx) == order[:k]
+        assert abs(w.sum() - 1.0) < 1e-12
+        sg = 1 / (1 + np.exp(-z[idx]))
+        assert np.allclose(w, sg / sg.sum(), rtol=1e-13)
+        if k < E:
+            assert np.isclose(margin, key[order[k - 1]] - key[order[k]], atol=1e-15)
+        else:
+            assert margin == np.inf
+
+
+def test_topk_zero_bias_equals_topk_of_sigmoid():
+    z = RNG.normal(size=300) * 3
+    idx, _, _ = O.topk(z, np.zeros(300, np.float32), 7)
+    s = 1 / (1 + np.exp(-z))
+    assert set(idx.tolist()) == set(np.argsort(-s, kind="stable")[:7].tolist())
+
+
+def test_topk_bias_chooses_but_does_not_weight():
+    z = np.array([0.0, 0.1, 0.2, 0.3])
+    b = np.array([5.0, 0.0, 0.0, 0.0], np.float32)
+    idx, w, _ = O.topk(z, b, 2)
+    assert list(idx) == [0, 3]                       # bias lifts expert 0 into the picks
+    s = 1 / (1 + np.exp(-np.array([0.0, 0.3])))
+    assert np.allclose(w, s / s.sum())               # weights come from sigmoid(z), not z+b
+
+
+def test_topk_ties_go_to_lower_index():
+    idx, w, margin = O.topk(np.zeros(10), np.zeros(10, np.float32), 3)
+    assert list(idx) == [0, 1, 2] and margin == 0.0 and np.allclose(w, 1 / 3)
+
+
+def test_bias_update_closed_form():
+    # N = (1, 5, 3, 3) summed over depths -> sorted (1, 3, 3, 5), lower median 3
+    counts = np.array([[1, 2, 1, 2], [0, 3, 2, 1]], np.int32)
+    b = O.bias_update(counts, 0.01, np.zeros(4))
+    assert np.allclose(b, [0.01, -0.01, 0.0, 0.0])
+
+
+# ---------------------------------------------------------------------------------------
+# linear-MoE projection with the absorbed shared expert (papernotes "Key design 3")
+
+def test_absorbed_shared_expert_identity():
+    Wp = RNG.normal(size=(48, 80)).astype(np.float32)
+    Ws = RNG.normal(size=(48, 80)).astype(np.float32)
+    x = RNG.normal(size=48)
+    for sigma in (0.51, 0.93):
+        a = O.linear_moe(x, Wp, Ws, sigma)
+        b = O.linear_moe(x, Wp, Ws, sigma, absorbed=True)
+        assert np.allclose(a, b, rtol=1e-12, atol=1e-12)
+        assert np.allclose(a, sigma * (x @ Wp.astype(np.float64)) + sigma * (x @ Ws.astype(np.float64)),
+                           rtol=1e-12, atol=1e-12)
+
+
+def test_expert_ffn_scalar_case():
+    # h = 1, m = 1: SiLU(y w1) w2
+    y, w1, w2 = 0.7, 1.3, -2.1
+    u = y * w1
+    out = O.expert(np.array([y]), np.array([[w1]], np.float32), np.array([[w2]], np.float32))
+    w1f, w2f = np.float32(w1), np.float32(w2)
+    u = y * float(w1f)
+    assert np.isclose(out[0], u / (1 + np.exp(-u)) * float(w2f), rtol=1e-14)
+
+
+# ---------------------------------------------------------------------------------------
+# whole block
+
+def _closed_form_single_token(cfg, W, x0):
+    """L = 1, s = 1, E = k: SA over one key returns v_SA, DA at depth 0 returns v_DA,
+    all experts are picked.  Everything reduces to plain matrix products."""
+    h, dr = cfg.hidden, cfg.router_dim
+    f = lambda a: np.asarray(a, np.float64)
+    x = f(x0)
+    xh = x / np.sqrt(np.mean(x ** 2, axis=-1, keepdims=True) + cfg.rms_eps) * f(W["g"])
+    P = cfg.n_proj_experts
+    if P > 0:
+        # single projection expert: p* = 0, sigma = sigmoid(q_P . k~_P / sqrt(d_r))
+        kP = O.depth_rope(f(W["k_P"][0]), 0, 1)
+        z = (xh @ f(W["w_qP"])) @ kP / np.sqrt(dr)
+        sig = (1 / (1 + np.exp(-z)))[:, None]
+        Wqkv = sig[:, :, None] * (f(W["w_qkv"][0]) + f(W["w_qkv_shared"]))[None]
+        Wo = sig[:, :, None] * (f(W["w_o"][0]) + f(W["w_o_shared"]))[None]
+        qkv = np.einsum("ti,tij->tj", xh, Wqkv)
+    else:
+        qkv = xh @ f(W["w_qkv"][0])
+        Wo = None
+    v_sa, v_da = qkv[:, 2 * h:3 * h], qkv[:, 5 * h:6 * h]
+    cat = np.concatenate([v_sa, v_da], axis=1)
+    o = np.einsum("ti,tij->tj", cat, Wo) if Wo is not None else cat @ f(W["w_o"][0])
+    y = xh + o
+    kE = np.stack([O.depth_rope(f(k), 0, 1) for k in W["k_E"]])
+    z = (y @ f(W["w_qE"])) @ kE.T / np.sqrt(dr)
+    s = 1 / (1 + np.exp(-z))
+    w = s / s.sum(1, keepdims=True)
+    out = y.copy()
+    for e in range(cfg.n_experts):
+        u = y @ f(W["w1"][e])
+        out += w[:, e:e + 1] * ((u / (1 + np.exp(-u))) @ f(W["w2"][e]))
+    return out
+
+
+@pytest.mark.parametrize("P", [0, 1])
+def test_block_reduces_to_closed_form(P):
+    cfg = tiny_cfg(batch=3, seq=1, depth=1, n_experts=3, top_k=3, n_proj_experts=P)
+    W = rand_weights(cfg, seed=11)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    r = O.Oracle(cfg, W, threads=1).forward(x0)
+    ref = _closed_form_single_token(cfg, W, x0)
+    assert np.allclose(r["x_out"], ref, rtol=1e-11, atol=1e-11)
+
+
+def test_da_reshape_equals_explicit_loops():
+    cfg = configs.TINY
+    W = inputs.host_weights(cfg)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    o = O.Oracle(cfg, W, threads=2)
+    a = o.forward(x0)
+    b = o.forward(x0, da_loops=True)
+    assert np.allclose(a["x_out"], b["x_out"], rtol=1e-12, atol=1e-12)
+    assert np.array_equal(a["idx"], b["idx"])
+
+
+def test_da_at_depth_zero_returns_its_value():
+    # SA rows of W_O zero, DA rows identity, experts off: x_1 = x^ + v_DA(x^)
+    cfg = tiny_cfg(depth=1, n_experts=2, top_k=1)
+    W = rand_weights(cfg, seed=3)
+    h = cfg.hidden
+    W["w_o"] = np.zeros_like(W["w_o"])
+    W["w_o"][0, h:, :] = np.eye(h, dtype=np.float32)
+    W["w2"] = np.zeros_like(W["w2"])
+    x0 = inputs.host_inputs(cfg)["x0"]
+    r = O.Oracle(cfg, W, threads=1).forward(x0)
+    x = x0.astype(np.float64)
+    xh = x / np.sqrt(np.mean(x ** 2, 1, keepdims=True) + cfg.rms_eps)
+    v_da = xh @ W["w_qkv"][0][:, 5 * h:6 * h].astype(np.float64)
+    assert np.allclose(r["x_out"], xh + v_da, rtol=1e-12, atol=1e-12)
+
+
+def test_sa_causality_and_single_token():
+    cfg = tiny_cfg(batch=2, seq=8, depth=2)
+    W = rand_weights(cfg, seed=5)
+    x0 = inputs.host_inputs(cfg)["x0"].copy()
+    o = O.Oracle(cfg, W, threads=1)
+    a = o.forward(x0)["x_out"]
+    x1 = x0.copy()
+    x1[5] += 1.0                        # token 5 of sequence 0
+    b = o.forward(x1)["x_out"]
+    assert np.array_equal(a[:5], b[:5])          # earlier tokens bit-identical
+    assert not np.allclose(a[5:8], b[5:8])
+    assert np.array_equal(a[8:], b[8:])          # other sequence untouched
+
+
+def test_batch_permutation_equivariance():
+    cfg = tiny_cfg(batch=3, seq=4, depth=2)
+    W = rand_weights(cfg, seed=6)
+    x0 = inputs.host_inputs(cfg)["x0"].reshape(3, 4, -1)
+    o = O.Oracle(cfg, W, threads=1)
+    a = o.forward(x0.reshape(12, -1))["x_out"].reshape(3, 4, -1)
+    b = o.forward(x0[[2, 0, 1]].reshape(12, -1))["x_out"].reshape(3, 4, -1)
+    assert np.array_equal(a[[2, 0, 1]], b)
+
+
+def test_counts_are_histogram_of_indices():
+    cfg = configs.TINY
+    W = inputs.host_weights(cfg)
+    r = O.Oracle(cfg, W, threads=1).forward(inputs.host_inputs(cfg)["x0"])
+    T, k, L, E = cfg.tokens, cfg.top_k, cfg.depth, cfg.n_experts
+    assert np.all(r["counts"].sum(1) == T * k)
+    for l in range(L):
+        assert np.array_equal(r["counts"][l], np.bincount(r["idx"][l].ravel(), minlength=E))
+        for t in range(T):
+            assert len(set(r["idx"][l, t].tolist())) == k
+    assert np.allclose(r["w"].sum(-1), 1.0, atol=1e-12)
+
+
+def test_depth_range_composes():
+    """Running depths [0, 2) then [2, L) through the DA buffer equals [0, L)."""
+    cfg = configs.TINY
+    W = inputs.host_weights(cfg)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    o = O.Oracle(cfg, W, threads=1)
+    full = o.forward(x0)
+    a = o.forward(x0, 0, 2)
+    b = o.forward(a["x_out"].astype(np.float32), 2, cfg.depth, da_kv=a["da_kv"])
+    # the middle state passes through float32, so compare loosely
+    assert np.allclose(b["x_out"], full["x_out"], rtol=1e-5, atol=1e-5)
+
+
+@pytest.mark.parametrize("variant", [0, 2])
+def test_step_tokens_equals_forward_rows(variant):
+    cfg = tiny_cfg(batch=2, seq=8, depth=3, variant=variant)
+    W = rand_weights(cfg, seed=8)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    o = O.Oracle(cfg, W, threads=1)
+    full = o.forward(x0, 0, 2)
+    x2 = full["x_out"].astype(np.float32)
+    ref = o.forward(x2, 2, 3, da_kv=full["da_kv"])
+    seq = 1
+    pos = np.array([0, 3, 7], np.int32)
+    toks = seq * cfg.seq + pos
+    st = o.step_tokens(2, x2[seq * cfg.seq:(seq + 1) * cfg.seq], full["da_kv"][toks], pos)
+    assert np.allclose(st["x_out"], ref["x_out"][toks], rtol=1e-12, atol=1e-12)
+    assert np.array_equal(st["idx"], ref["idx"][2][toks])
+
+
+@pytest.mark.parametrize("P,variant", [(0, 0), (2, 0), (0, 1), (0, 2)])
+def test_decode_equals_last_row_of_longer_prefill(P, variant):
+    cfg = tiny_cfg(batch=1, seq=6, depth=3, n_proj_experts=P, variant=variant)
+    W = rand_weights(cfg, seed=9)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    o = O.Oracle(cfg, W, threads=1)
+    full = o.forward(x0)                       # prefill of s + 1 = 6 tokens
+    L, H, d, h = cfg.depth, cfg.n_heads, cfg.head_dim, cfg.hidden
+    s = 5
+    cap = 8
+    kc = np.zeros((L, H, cap, d))
+    vc = np.zeros((L, H, cap, d))
+    for l in range(L):
+        kc[l, :, :s] = full["sa_k"][l, :s].reshape(s, H, d).transpose(1, 0, 2)
+        vc[l, :, :s] = full["sa_v"][l, :s].reshape(s, H, d).transpose(1, 0, 2)
+    dec = o.decode_seq(x0[s], kc, vc, s)
+    assert np.allclose(dec["x_out"], full["x_out"][s], rtol=1e-12, atol=1e-12)
+    assert np.array_equal(dec["idx"].reshape(L, -1), full["idx"][:, s])
+    # the decode step wrote the new token's keys at slot s
+    for l in range(L):
+        assert np.allclose(kc[l, :, s], full["sa_k"][l, s].reshape(H, d), atol=1e-12)
+
+
+def test_decode_empty_cache_single_depth_is_one_token_block():
+    cfg = tiny_cfg(batch=1, seq=1, depth=1)
+    W = rand_weights(cfg, seed=10)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    o = O.Oracle(cfg, W, threads=1)
+    ref = o.forward(x0)["x_out"][0]
+    kc = np.zeros((1, cfg.n_heads, 4, cfg.head_dim))
+    vc = np.zeros_like(kc)
+    dec = o.decode_seq(x0[0], kc, vc, 0)
+    assert np.allclose(dec["x_out"], ref, rtol=1e-13, atol=1e-13)
+
+
+def test_serial_layout_closed_form():
+    """Serial DA -> SA -> EA at L = 1, s = 1, E = k: u = x^ + v_DA W_O^DA;
+    v = u + v_SA(u) W_O^SA; x_1 = v + mixture(v)."""
+    cfg = tiny_cfg(batch=2, seq=1, depth=1, n_experts=2, top_k=2, variant=1)
+    W = rand_weights(cfg, seed=12)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    r = O.Oracle(cfg, W, threads=1).forward(x0)
+    h, dr = cfg.hidden, cfg.router_dim
+    f = lambda a: np.asarray(a, np.float64)
+    x = f(x0)
+    xh = x / np.sqrt(np.mean(x ** 2, 1, keepdims=True) + cfg.rms_eps)
+    Wq, Wo = f(W["w_qkv"][0]), f(W["w_o"][0])
+    u = xh + (xh @ Wq[:, 5 * h:]) @ Wo[h:]
+    v = u + (u @ Wq[:, 2 * h:3 * h]) @ Wo[:h]
+    kE = np.stack([O.depth_rope(f(k), 0, 1) for k in W["k_E"]])
+    z = (v @ f(W["w_qE"])) @ kE.T / np.sqrt(dr)
+    s = 1 / (1 + np.exp(-z))
+    w = s / s.sum(1, keepdims=True)
+    out = v.copy()
+    for e in range(2):
+        a = v @ f(W["w1"][e])
+        out += w[:, e:e + 1] * ((a / (1 + np.exp(-a))) @ f(W["w2"][e]))
+    assert np.allclose(r["x_out"], out, rtol=1e-11, atol=1e-11)
+
+
+def test_fully_parallel_layout_routes_normed_state():
+    """Fully parallel DA + SA + EA: with W_O = 0 the output is x^ + mixture(x^)."""
+    cfg = tiny_cfg(batch=1, seq=3, depth=1, n_experts=4, top_k=4, variant=2)
+    W = rand_weights(cfg, seed=13)
+    W["w_o"] = np.zeros_like(W["w_o"])
+    x0 = inputs.host_inputs(cfg)["x0"]
+    r = O.Oracle(cfg, W, threads=1).forward(x0)
+    f = lambda a: np.asarray(a, np.float64)
+    x = f(x0)
+    xh = x / np.sqrt(np.mean(x ** 2, 1, keepdims=True) + cfg.rms_eps)
+    kE = np.stack([O.depth_rope(f(k), 0, 1) for k in W["k_E"]])
+    z = (xh @ f(W["w_qE"])) @ kE.T / np.sqrt(cfg.router_dim)
+    s = 1 / (1 + np.exp(-z))
+    w = s / s.sum(1, keepdims=True)
+    out = xh.copy()
+    for e in range(4):
+        a = xh @ f(W["w1"][e])
+        out += w[:, e:e + 1] * ((a / (1 + np.exp(-a))) @ f(W["w2"][e]))
+    assert np.allclose(r["x_out"], out, rtol=1e-11, atol=1e-11)
+
+
+def test_route_entry_matches_forward_trace():
+    cfg = configs.TINY
+    W = inputs.host_weights(cfg)
+    o = O.Oracle(cfg, W, threads=1)
+    full = o.forward(inputs.host_inputs(cfg)["x0"])
+    y1 = full["y"][1].astype(np.float32)
+    r = o.route(1, y1)
+    # routing from the float32-rounded y picks the same experts except at near ties
+    same = np.all(np.sort(r["idx"], 1) == np.sort(full["idx"][1], 1), axis=1)
+    assert np.all(same | (full["margin"][1] < 1e-5))
