@@ -1,0 +1,660 @@
+// libdreamer: C ABI of the Dreamer depth-recurrent core forward on B200 (sm_100a).
+// The depth step (papernotes.org notes on "Depth-Recurrent Attention Mixtures", section
+// "Overall framework", flowchart): RMSNorm -> [DA || SA] -> residual -> EA -> next depth.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <vector>
+
+#include "../../include/dreamer.h"
+#include "common.cuh"
+#include "kernels_simt.cuh"
+
+using namespace dreamer;
+
+struct dreamer_handle {
+  dreamer_config cfg;
+  int T;        // token capacity of the workspace
+  int esz;      // element size
+  int max_pos;  // RoPE table rows
+  int ldz;      // router score row stride (E rounded up to 8)
+  int ldzp;     // projection router score row stride
+  // weights in kernel layouts ([N][K], K contiguous)
+  void *g = nullptr, *wqkv_t = nullptr, *wo_t = nullptr, *wqE_t = nullptr, *wqP_t = nullptr;
+  void *w1_t = nullptr, *w2_t = nullptr;
+  void *kE_raw = nullptr;        // [E][dr] dtype (unrotated)
+  float *bias = nullptr;         // [E]
+  float *kE_rot = nullptr;       // [L][E][dr]
+  float *kP_rot = nullptr;       // [L][P][dr]
+  float2 *rope_tok = nullptr;    // [max_pos][d/2]
+  float2 *rope_dep = nullptr;    // [L][d/2]
+  float2 *rope_dr = nullptr;     // [L][dr/2] depth RoPE table of the router key dim
+  // workspace
+  void *xh = nullptr, *qkv_sa = nullptr, *q_da = nullptr, *attn = nullptr, *y = nullptr;
+  void *u = nullptr, *da_kv_int = nullptr, *Hbuf = nullptr, *qsplit = nullptr;
+  float *acc = nullptr, *zbuf = nullptr, *qbuf = nullptr, *psig = nullptr, *ew = nullptr;
+  int *pidx = nullptr, *eidx = nullptr, *counts = nullptr, *ecnt = nullptr, *eoffs = nullptr;
+  int *etiles_a = nullptr, *etiles_b = nullptr, *ecursor = nullptr, *erows = nullptr;
+  int *pcnt = nullptr, *poffs = nullptr, *ptiles_a = nullptr, *ptiles_b = nullptr;
+  int *pcursor = nullptr, *prows = nullptr, *pinv = nullptr;
+  int *err = nullptr;
+  int use_tc = 1;  // bf16 contractions on tcgen05 (0: CUDA cores, for cross-checks)
+  std::vector<void *> allocs;
+};
+
+#include "tc_kernels.cuh"
+
+#define CK(call)                                                  \
+  do {                                                            \
+    cudaError_t e_ = (call);                                      \
+    if (e_ != cudaSuccess) {                                      \
+      fprintf(stderr, "libdreamer: %s failed: %s\n", #call,      \
+              cudaGetErrorString(e_));                            \
+      return e_ == cudaErrorMemoryAllocation ? DREAMER_ERR_OOM    \
+                                             : DREAMER_ERR_CUDA;  \
+    }                                                             \
+  } while (0)
+
+static int dalloc(dreamer_handle *h, void **p, size_t bytes) {
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    *p = nullptr;
+    return e == cudaErrorMemoryAllocation ? DREAMER_ERR_OOM : DREAMER_ERR_CUDA;
+  }
+  h->allocs.push_back(*p);
+  return DREAMER_OK;
+}
+#define DALLOC(ptr, bytes)                                     \
+  do {                                                         \
+    int rc_ = dalloc(h, (void **)&(ptr), (size_t)(bytes));     \
+    if (rc_ != DREAMER_OK) return rc_;                         \
+  } while (0)
+
+static inline int cdiv(long a, long b) { return (int)((a + b - 1) / b); }
+static inline int round8(int v) { return (v + 7) / 8 * 8; }
+
+extern "C" const char *dreamer_strerror(int code) {
+  switch (code) {
+    case DREAMER_OK: return "ok";
+    case DREAMER_ERR_ARG: return "invalid argument";
+    case DREAMER_ERR_UNSUPPORTED: return "unsupported configuration";
+    case DREAMER_ERR_CUDA: return "CUDA runtime error";
+    case DREAMER_ERR_OOM: return "out of device memory";
+    case DREAMER_ERR_TIMEOUT: return "device wait timed out";
+    case DREAMER_ERR_STATE: return "call not valid for this handle";
+    default: return "unknown error";
+  }
+}
+
+static int validate(const dreamer_config *c) {
+  if (!c) return DREAMER_ERR_ARG;
+  if (c->batch < 1 || c->seq < 1 || c->depth < 1 || c->n_heads < 1 || c->head_dim < 1)
+    return DREAMER_ERR_ARG;
+  if (c->hidden != c->n_heads * c->head_dim) return DREAMER_ERR_ARG;
+  if (c->top_k < 1 || c->top_k > c->n_experts) return DREAMER_ERR_ARG;
+  if (c->dtype != 0 && c->dtype != 1) return DREAMER_ERR_ARG;
+  if (c->n_proj_experts < 0 || c->max_cache_len < 0) return DREAMER_ERR_ARG;
+  if (c->variant < 0 || c->variant > 2) return DREAMER_ERR_ARG;
+  if (!(c->rope_base > 0.f) || !(c->rms_eps >= 0.f)) return DREAMER_ERR_ARG;
+  const int d = c->head_dim;
+  if (d != 16 && d != 32 && d != 64 && d != 128) return DREAMER_ERR_UNSUPPORTED;
+  if (c->top_k > 16 || c->n_experts > 65536 || c->n_proj_experts > 64) return DREAMER_ERR_UNSUPPORTED;
+  if (c->expert_hidden % 16 || c->router_dim % 16 || c->router_dim > 256 || c->hidden % 64)
+    return DREAMER_ERR_UNSUPPORTED;
+  if (c->depth > 1024) return DREAMER_ERR_UNSUPPORTED;
+  return DREAMER_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// host-side tables
+// RoPE rotate-half tables in double, stored as float2 (cos, sin).
+static void rope_table(std::vector<float2> &t, int rows, int n, double base) {
+  // rows positions x n/2 pairs, angle pos * base^(-2i/n)
+  t.resize((size_t)rows * (n / 2));
+  for (int p = 0; p < rows; p++)
+    for (int i = 0; i < n / 2; i++) {
+      double th = (double)p * pow(base, -2.0 * i / (double)n);
+      t[(size_t)p * (n / 2) + i] = make_float2((float)cos(th), (float)sin(th));
+    }
+}
+// depth table [L][n/2]: first n/4 entries at position l over n/2 dims, next n/4 at L-1-l.
+static void depth_table(std::vector<float2> &t, int L, int n, double base) {
+  t.resize((size_t)L * (n / 2));
+  const int q = n / 4;
+  for (int l = 0; l < L; l++)
+    for (int half = 0; half < 2; half++)
+      for (int i = 0; i < q; i++) {
+        double pos = half == 0 ? l : (L - 1 - l);
+        double th = pos * pow(base, -2.0 * i / (double)(n / 2));
+        t[(size_t)l * (n / 2) + half * q + i] = make_float2((float)cos(th), (float)sin(th));
+      }
+}
+
+static float host_to_f(const void *p, size_t i, int dtype) {
+  if (dtype == 0) return ((const float *)p)[i];
+  uint16_t b = ((const uint16_t *)p)[i];
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+// keys [n][dr] (dtype, device) -> rotated fp32 [L][n][dr] by the depth RoPE of each depth.
+static int rotated_keys(dreamer_handle *h, const void *keys_dev, int n, float **out) {
+  const dreamer_config &c = h->cfg;
+  const int dr = c.router_dim, L = c.depth;
+  std::vector<uint8_t> raw((size_t)n * dr * h->esz);
+  CK(cudaMemcpy(raw.data(), keys_dev, raw.size(), cudaMemcpyDeviceToHost));
+  std::vector<float> rot((size_t)L * n * dr);
+  const int half = dr / 2, q = dr / 4;
+  for (int l = 0; l < L; l++)
+    for (int e = 0; e < n; e++) {
+      std::vector<double> v(dr);
+      for (int i = 0; i < dr; i++) v[i] = host_to_f(raw.data(), (size_t)e * dr + i, c.dtype);
+      for (int hh = 0; hh < 2; hh++) {
+        double pos = hh == 0 ? l : (L - 1 - l);
+        for (int i = 0; i < q; i++) {
+          double th = pos * pow((double)c.rope_base, -2.0 * i / (double)half);
+          double cs = cos(th), sn = sin(th);
+          double a = v[hh * half + i], b = v[hh * half + i + q];
+          v[hh * half + i] = a * cs - b * sn;
+          v[hh * half + i + q] = b * cs + a * sn;
+        }
+      }
+      for (int i = 0; i < dr; i++) rot[((size_t)l * n + e) * dr + i] = (float)v[i];
+    }
+  DALLOC(*out, rot.size() * sizeof(float));
+  CK(cudaMemcpy(*out, rot.data(), rot.size() * sizeof(float), cudaMemcpyHostToDevice));
+  return DREAMER_OK;
+}
+
+template <typename T>
+static void launch_transpose(const void *src, const void *sh, void *dst, int rows, int cols,
+                             int G, cudaStream_t s) {
+  dim3 grid(cdiv(cols, 32), cdiv(rows, 32), G), block(32, 8);
+  transpose_absorb_kernel<T><<<grid, block, 0, s>>>((const T *)src, (const T *)sh, (T *)dst,
+                                                     rows, cols, G);
+}
+
+extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
+                            dreamer_stream stream, dreamer_handle **out) {
+  if (!out) return DREAMER_ERR_ARG;
+  *out = nullptr;
+  int rc = validate(cfg);
+  if (rc) return rc;
+  if (!w || !w->rms_gain || !w->w_qkv || !w->w_o || !w->w_qE || !w->k_E || !w->bias_E ||
+      !w->w1 || !w->w2)
+    return DREAMER_ERR_ARG;
+  if (cfg->n_proj_experts > 0 &&
+      (!w->w_qkv_shared || !w->w_o_shared || !w->w_qP || !w->k_P))
+    return DREAMER_ERR_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  dreamer_handle *h = new dreamer_handle();
+  h->cfg = *cfg;
+  rc = [&]() -> int {
+    const dreamer_config &c = h->cfg;
+    const int hd = c.hidden, E = c.n_experts, m = c.expert_hidden, dr = c.router_dim;
+    const int P = c.n_proj_experts, G = P > 0 ? P : 1, L = c.depth, d = c.head_dim;
+    h->esz = c.dtype == 0 ? 4 : 2;
+    h->T = c.batch * c.seq > c.batch ? c.batch * c.seq : c.batch;
+    h->max_pos = c.seq > c.max_cache_len ? c.seq : c.max_cache_len;
+    h->ldz = round8(E);
+    h->ldzp = round8(P > 0 ? P : 1);
+    const size_t es = h->esz;
+    const long T = h->T;
+    if (const char *ev = getenv("DREAMER_NO_TC")) h->use_tc = atoi(ev) ? 0 : 1;
+    // ---- weights
+    DALLOC(h->g, hd * es);
+    CK(cudaMemcpyAsync(h->g, w->rms_gain, hd * es, cudaMemcpyDeviceToDevice, s));
+    DALLOC(h->wqkv_t, (size_t)G * hd * 6 * hd * es);
+    DALLOC(h->wo_t, (size_t)G * 2 * hd * hd * es);
+    DALLOC(h->wqE_t, (size_t)hd * dr * es);
+    DALLOC(h->w1_t, (size_t)E * hd * m * es);
+    DALLOC(h->w2_t, (size_t)E * hd * m * es);
+    DALLOC(h->kE_raw, (size_t)E * dr * es);
+    CK(cudaMemcpyAsync(h->kE_raw, w->k_E, (size_t)E * dr * es, cudaMemcpyDeviceToDevice, s));
+    DALLOC(h->bias, E * sizeof(float));
+    CK(cudaMemcpyAsync(h->bias, w->bias_E, E * sizeof(float), cudaMemcpyDeviceToDevice, s));
+    auto tr = c.dtype == 0 ? launch_transpose<float> : launch_transpose<bf16>;
+    // W_qkv [G][h][6h] (+ shared) -> [G][6h][h]; W_o [G][2h][h] -> [G][h][2h]
+    tr(w->w_qkv, P > 0 ? w->w_qkv_shared : nullptr, h->wqkv_t, hd, 6 * hd, G, s);
+    tr(w->w_o, P > 0 ? w->w_o_shared : nullptr, h->wo_t, 2 * hd, hd, G, s);
+    tr(w->w_qE, nullptr, h->wqE_t, hd, dr, 1, s);
+    tr(w->w1, nullptr, h->w1_t, hd, m, E, s);     // [E][h][m] -> [E][m][h]
+    tr(w->w2, nullptr, h->w2_t, m, hd, E, s);     // [E][m][h] -> [E][h][m]
+    if (P > 0) {
+      DALLOC(h->wqP_t, (size_t)hd * dr * es);
+      tr(w->w_qP, nullptr, h->wqP_t, hd, dr, 1, s);
+    }
+    CK(cudaGetLastError());
+    CK(cudaStreamSynchronize(s));
+    int r2 = rotated_keys(h, w->k_E, E, &h->kE_rot);
+    if (r2) return r2;
+    if (P > 0) {
+      r2 = rotated_keys(h, w->k_P, P, &h->kP_rot);
+      if (r2) return r2;
+    }
+    std::vector<float2> tt, td, tq;
+    rope_table(tt, h->max_pos + 1, d, c.rope_base);
+    depth_table(td, L, d, c.rope_base);
+    depth_table(tq, L, dr, c.rope_base);
+    DALLOC(h->rope_tok, tt.size() * sizeof(float2));
+    DALLOC(h->rope_dep, td.size() * sizeof(float2));
+    DALLOC(h->rope_dr, tq.size() * sizeof(float2));
+    CK(cudaMemcpy(h->rope_tok, tt.data(), tt.size() * sizeof(float2), cudaMemcpyHostToDevice));
+    CK(cudaMemcpy(h->rope_dep, td.data(), td.size() * sizeof(float2), cudaMemcpyHostToDevice));
+    CK(cudaMemcpy(h->rope_dr, tq.data(), tq.size() * sizeof(float2), cudaMemcpyHostToDevice));
+    // ---- workspace
+    const long Tk = T * c.top_k;
+    DALLOC(h->xh, T * hd * es);
+    DALLOC(h->u, T * hd * es);
+    DALLOC(h->qkv_sa, T * 3 * hd * es);
+    DALLOC(h->q_da, T * hd * es);
+    DALLOC(h->attn, T * 2 * hd * es);
+    DALLOC(h->y, T * hd * es);
+    DALLOC(h->acc, T * hd * sizeof(float));
+    DALLOC(h->da_kv_int, (size_t)T * L * 2 * hd * es);
+    DALLOC(h->Hbuf, (Tk + 128) * m * es);
+    DALLOC(h->qsplit, T * 3 * dr * 2);
+    DALLOC(h->zbuf, (size_t)T * (h->ldz > h->ldzp ? h->ldz : h->ldzp) * sizeof(float));
+    DALLOC(h->qbuf, T * dr * sizeof(float));
+    DALLOC(h->psig, T * sizeof(float));
+    DALLOC(h->pidx, T * sizeof(int));
+    DALLOC(h->ew, Tk * sizeof(float));
+    DALLOC(h->eidx, Tk * sizeof(int));
+    DALLOC(h->counts, (size_t)L * E * sizeof(int));
+    DALLOC(h->ecnt, E * sizeof(int));
+    DALLOC(h->eoffs, (E + 1) * sizeof(int));
+    DALLOC(h->etiles_a, (E + 1) * sizeof(int));
+    DALLOC(h->etiles_b, (E + 1) * sizeof(int));
+    DALLOC(h->ecursor, E * sizeof(int));
+    DALLOC(h->erows, Tk * sizeof(int));
+    DALLOC(h->pcnt, (G + 1) * sizeof(int));
+    DALLOC(h->poffs, (G + 1) * sizeof(int));
+    DALLOC(h->ptiles_a, (G + 1) * sizeof(int));
+    DALLOC(h->ptiles_b, (G + 1) * sizeof(int));
+    DALLOC(h->pcursor, (G + 1) * sizeof(int));
+    DALLOC(h->prows, T * sizeof(int));
+    DALLOC(h->pinv, T * sizeof(int));
+    DALLOC(h->err, sizeof(int));
+    CK(cudaMemset(h->err, 0, sizeof(int)));
+    CK(cudaMemset(h->counts, 0, (size_t)L * E * sizeof(int)));
+    int r3 = tc_init(h);
+    if (r3) return r3;
+    CK(cudaDeviceSynchronize());
+    return DREAMER_OK;
+  }();
+  if (rc != DREAMER_OK) {
+    dreamer_destroy(h);
+    return rc;
+  }
+  *out = h;
+  return DREAMER_OK;
+}
+
+extern "C" void dreamer_destroy(dreamer_handle *h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  tc_destroy(h);
+  for (void *p : h->allocs) cudaFree(p);
+  delete h;
+}
+
+// ---------------------------------------------------------------------------------------
+// launch helpers
+template <typename TA, typename TB, int SEG, class Epi>
+static void gemm_simt(const GemmArgs &a, int max_tiles, const Epi &epi, cudaStream_t s) {
+  dim3 grid(max_tiles, cdiv(a.N, 128));
+  gemm_simt_kernel<TA, TB, SEG, Epi><<<grid, 256, 0, s>>>(a, epi);
+}
+
+static GemmArgs dense_args(int M, int N, int K, const void *A, long lda, const void *B,
+                           long ldb) {
+  GemmArgs a{};
+  a.N = N; a.K = K; a.G = 1; a.M = M; a.goffs = nullptr; a.tile_offs = nullptr;
+  a.arow = nullptr; a.arow_div = 1; a.A = A; a.lda = lda; a.B = B; a.ldb = ldb; a.bgstride = 0;
+  return a;
+}
+
+template <typename T>
+static void launch_attn(const AttnArgs &a, int d, cudaStream_t s) {
+  const int warps = a.n_q * a.H;
+  const int blocks = cdiv(warps, 8);
+  switch (d) {
+    case 16: attn_warp_kernel<T, 16><<<blocks, 256, 0, s>>>(a); break;
+    case 32: attn_warp_kernel<T, 32><<<blocks, 256, 0, s>>>(a); break;
+    case 64: attn_warp_kernel<T, 64><<<blocks, 256, 0, s>>>(a); break;
+    default: attn_warp_kernel<T, 128><<<blocks, 256, 0, s>>>(a); break;
+  }
+}
+
+template <typename T, int SEG>
+static void gemm_qkv(dreamer_handle *h, const GemmArgs &a, int max_tiles, const EpiQKV<T> &e,
+                     cudaStream_t s) {
+  gemm_simt<T, T, SEG>(a, max_tiles, e, s);
+}
+
+// Routing of n rows X [n][h] at depth l (router query projection, scores against the
+// depth-RoPE'd keys, top-k).  mode 0: expert attention; mode 1: projection router.
+template <typename T>
+static void route_rows(dreamer_handle *h, int mode, int l, const void *X, int n, int *idx,
+                       float *wout, int *counts_a, int *counts_b, cudaStream_t s) {
+  const dreamer_config &c = h->cfg;
+  const int dr = c.router_dim, hd = c.hidden;
+  const int E = mode == 0 ? c.n_experts : c.n_proj_experts;
+  const int ldz = mode == 0 ? h->ldz : h->ldzp;
+  const void *Wq = mode == 0 ? h->wqE_t : h->wqP_t;
+  const float *krot = (mode == 0 ? h->kE_rot : h->kP_rot) + (size_t)l * E * dr;
+  if (mode == 0 && h->use_tc && c.dtype == 1 && tc_route_ok(h)) {
+    tc_route(h, l, X, n, idx, wout, counts_a, counts_b, s);
+    return;
+  }
+  // q = X W_q (fp32 accumulation), z = q . k~ (fp32), on CUDA cores
+  GemmArgs a = dense_args(n, dr, hd, X, hd, Wq, hd);
+  gemm_simt<T, T, 8>(a, cdiv(n, 64), EpiStoreF32{h->qbuf, dr, dr}, s);
+  GemmArgs b = dense_args(n, E, dr, h->qbuf, dr, krot, dr);
+  gemm_simt<float, float, 8>(b, cdiv(n, 64), EpiStoreF32{h->zbuf, ldz, E}, s);
+  TopkArgs t{};
+  t.n_tok = n; t.E = E; t.k = mode == 0 ? c.top_k : 1; t.mode = mode;
+  t.z = h->zbuf; t.ldz = ldz; t.zscale = 1.0f / sqrtf((float)dr);
+  t.bias = mode == 0 ? h->bias : nullptr;
+  t.idx = idx; t.w = wout; t.counts_a = counts_a; t.counts_b = counts_b;
+  topk_kernel<<<cdiv(n, 8), 256, 0, s>>>(t);
+}
+
+struct DepthIO {
+  int mode;               // 0 prefill, 1 decode
+  int n_tok;
+  const void *x_in;       // first depth only
+  void *da_kv;
+  void *k_cache, *v_cache;
+  const int *cache_len;
+};
+
+// One depth step for all n_tok tokens.
+template <typename T>
+static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, cudaStream_t s) {
+  const dreamer_config &c = h->cfg;
+  const int hd = c.hidden, d = c.head_dim, L = c.depth, E = c.n_experts, k = c.top_k;
+  const int m = c.expert_hidden, P = c.n_proj_experts, G = P > 0 ? P : 1;
+  const int n = io.n_tok;
+  const bool tc = h->use_tc && c.dtype == 1;
+
+  // 1. RMSNorm of the residual stream (x_0 on the first depth, else the fp32 accumulator)
+  rmsnorm_kernel<T><<<cdiv(n, 8), 256, 0, s>>>(first ? (const T *)io.x_in : nullptr,
+                                               first ? nullptr : h->acc, (const T *)h->g,
+                                               (T *)h->xh, nullptr, n, hd, c.rms_eps);
+  // 2. projection router and token grouping (linear-MoE QKV/O)
+  const int *prow = nullptr;
+  const float *psig = nullptr;
+  if (P > 0) {
+    cudaMemsetAsync(h->pcnt, 0, (G + 1) * sizeof(int), s);
+    route_rows<T>(h, 1, l, h->xh, n, h->pidx, h->psig, nullptr, h->pcnt, s);
+    scan_kernel<<<1, 1024, 0, s>>>(h->pcnt, G, h->poffs, h->ptiles_a, 64, h->ptiles_b, 128,
+                                   h->pcursor);
+    scatter_kernel<<<cdiv(n, 256), 256, 0, s>>>(h->pidx, n, h->pcursor, h->prows, h->pinv);
+    prow = h->prows;
+    psig = h->psig;
+  }
+  auto grouped = [&](int N, int K, const void *A, long lda, const void *B, long bgs) {
+    GemmArgs a{};
+    a.N = N; a.K = K; a.G = G; a.M = n;
+    a.goffs = P > 0 ? h->poffs : nullptr;
+    a.tile_offs = P > 0 ? h->ptiles_a : nullptr;
+    a.arow = prow; a.arow_div = 1; a.A = A; a.lda = lda; a.B = B; a.ldb = K; a.bgstride = bgs;
+    return a;
+  };
+  const int ptiles = cdiv(n, 64) + (P > 0 ? G : 0);
+
+  EpiQKV<T> eq{};
+  eq.h = hd; eq.d = d; eq.L = L; eq.l = l; eq.S = c.seq; eq.mode = io.mode; eq.col_lo = 0;
+  eq.psig = psig; eq.rope_tok = h->rope_tok; eq.rope_dep = h->rope_dep;
+  eq.qkv_sa = (T *)h->qkv_sa; eq.q_da = (T *)h->q_da; eq.da_kv = (T *)io.da_kv;
+  eq.k_cache = (T *)io.k_cache; eq.v_cache = (T *)io.v_cache; eq.cache_len = io.cache_len;
+  eq.B = c.batch; eq.cap = c.max_cache_len; eq.err = h->err;
+
+  AttnArgs da{};
+  da.mode = 0; da.n_q = n; da.H = c.n_heads; da.d = d; da.h = hd;
+  da.q = h->q_da; da.ldq = hd; da.kv = io.da_kv; da.L = L; da.l = l;
+  da.out = h->attn; da.ldo = 2 * hd; da.col0 = hd;
+  AttnArgs sa{};
+  sa.mode = io.mode == 0 ? 1 : 2; sa.n_q = n; sa.H = c.n_heads; sa.d = d; sa.h = hd;
+  sa.q = h->qkv_sa; sa.ldq = 3 * hd; sa.kv = io.mode == 0 ? h->qkv_sa : io.k_cache;
+  sa.vc = io.v_cache; sa.L = L; sa.l = l; sa.S = c.seq; sa.B = c.batch;
+  sa.cap = c.max_cache_len; sa.cache_len = io.cache_len; sa.err = h->err;
+  sa.out = h->attn; sa.ldo = 2 * hd; sa.col0 = 0;
+
+  auto qkv_gemm = [&](const void *A, int col0, int ncols) {
+    // columns [col0, col0 + ncols) of the fused QKV projection
+    GemmArgs a = grouped(ncols, hd, A, hd, (const T *)h->wqkv_t + (size_t)col0 * hd,
+                         (long)6 * hd * hd);
+    EpiQKV<T> e2 = eq;
+    e2.col_lo = col0;
+    if (tc && tc_gemm_ok(h, a)) {
+      tc_gemm_qkv(h, a, e2, s);
+      return;
+    }
+    switch (d) {
+      case 16: gemm_qkv<T, 16>(h, a, ptiles, e2, s); break;
+      case 32: gemm_qkv<T, 32>(h, a, ptiles, e2, s); break;
+      case 64: gemm_qkv<T, 64>(h, a, ptiles, e2, s); break;
+      default: gemm_qkv<T, 128>(h, a, ptiles, e2, s); break;
+    }
+  };
+  auto o_gemm = [&](const void *A, int row0, int nrows, const void *resid) {
+    // O projection over input rows [row0, row0 + nrows) of W_O ([a_SA | a_DA] order)
+    GemmArgs a = grouped(hd, nrows, A, 2 * hd, (const T *)h->wo_t + row0, (long)2 * hd * hd);
+    a.ldb = 2 * hd;
+    EpiO<T> eo{hd, psig, (const T *)resid, (T *)h->y, h->acc};
+    if (tc && tc_gemm_ok(h, a)) {
+      tc_gemm_o(h, a, eo, s);
+      return;
+    }
+    gemm_simt<T, T, 16>(a, ptiles, eo, s);
+  };
+
+  if (c.variant == 1) {
+    // serial DA -> SA -> EA: DA on x^, then SA on u = x^ + DA-part of O, then EA
+    qkv_gemm(h->xh, 3 * hd, 3 * hd);
+    launch_attn<T>(da, d, s);
+    {
+      GemmArgs a = grouped(hd, hd, (const T *)h->attn + hd, 2 * hd,
+                           (const T *)h->wo_t + hd, (long)2 * hd * hd);
+      a.ldb = 2 * hd;
+      EpiO<T> eo{hd, psig, (const T *)h->xh, (T *)h->u, nullptr};
+      gemm_simt<T, T, 16>(a, ptiles, eo, s);
+    }
+    qkv_gemm(h->u, 0, 3 * hd);
+    if (io.mode == 0 && tc && tc_sa_ok(h)) tc_sa(h, s); else launch_attn<T>(sa, d, s);
+    o_gemm(h->attn, 0, hd, h->u);
+  } else {
+    // 3. fused QKV projection with RoPE / depth RoPE epilogue, DA KV write
+    qkv_gemm(h->xh, 0, 6 * hd);
+    // 4. DA || SA (papernotes "Key design 1": run in parallel for throughput)
+    launch_attn<T>(da, d, s);
+    if (io.mode == 0 && tc && tc_sa_ok(h)) tc_sa(h, s); else launch_attn<T>(sa, d, s);
+    // 5. O projection, residual y = x^ + DA + SA
+    o_gemm(h->attn, 0, 2 * hd, h->xh);
+  }
+  // 6. expert attention routing on y (fully parallel layout: on x^)
+  const void *ein = c.variant == 2 ? h->xh : h->y;
+  cudaMemsetAsync(h->ecnt, 0, E * sizeof(int), s);
+  route_rows<T>(h, 0, l, ein, n, h->eidx, h->ew, h->counts + (size_t)l * E, h->ecnt, s);
+  scan_kernel<<<1, 1024, 0, s>>>(h->ecnt, E, h->eoffs, h->etiles_a, 64, h->etiles_b, 128,
+                                 h->ecursor);
+  scatter_kernel<<<cdiv((long)n * k, 256), 256, 0, s>>>(h->eidx, n * k, h->ecursor, h->erows,
+                                                         nullptr);
+  // 7. expert FFNs: H = SiLU(X W1_e), acc[token] += w * H W2_e
+  if (tc && tc_expert_ok(h)) {
+    tc_expert(h, ein, n, s);
+  } else {
+    const int etiles = cdiv((long)n * k, 64) + E;
+    GemmArgs up{};
+    up.N = m; up.K = hd; up.G = E; up.M = n * k; up.goffs = h->eoffs; up.tile_offs = h->etiles_a;
+    up.arow = h->erows; up.arow_div = k; up.A = ein; up.lda = hd; up.B = h->w1_t; up.ldb = hd;
+    up.bgstride = (long)m * hd;
+    gemm_simt<T, T, 16>(up, etiles, EpiUp<T>{m, (T *)h->Hbuf}, s);
+    GemmArgs dn{};
+    dn.N = hd; dn.K = m; dn.G = E; dn.M = n * k; dn.goffs = h->eoffs; dn.tile_offs = h->etiles_a;
+    dn.arow = nullptr; dn.arow_div = 1; dn.A = h->Hbuf; dn.lda = m; dn.B = h->w2_t; dn.ldb = m;
+    dn.bgstride = (long)m * hd;
+    gemm_simt<T, T, 16>(dn, etiles, EpiDown{hd, k, h->erows, h->ew, h->acc}, s);
+  }
+}
+
+static int check_dev_error(dreamer_handle *h) {
+  int e = 0;
+  if (cudaMemcpy(&e, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DREAMER_ERR_CUDA;
+  if (e) {
+    cudaMemset(h->err, 0, sizeof(int));
+    return e == DEV_TIMEOUT ? DREAMER_ERR_TIMEOUT : DREAMER_ERR_ARG;
+  }
+  return DREAMER_OK;
+}
+
+static void trace_depth(dreamer_handle *h, const dreamer_trace *tr, int l, int n, bool prefill,
+                        cudaStream_t s) {
+  if (!tr) return;
+  const dreamer_config &c = h->cfg;
+  const size_t es = h->esz, hd = c.hidden, k = c.top_k;
+  const size_t off = (size_t)l * n;
+  if (tr->xhat) cudaMemcpyAsync((char *)tr->xhat + off * hd * es, h->xh, n * hd * es, cudaMemcpyDeviceToDevice, s);
+  if (tr->y) cudaMemcpyAsync((char *)tr->y + off * hd * es, c.variant == 2 ? h->xh : h->y, n * hd * es, cudaMemcpyDeviceToDevice, s);
+  if (tr->idx) cudaMemcpyAsync(tr->idx + off * k, h->eidx, n * k * sizeof(int), cudaMemcpyDeviceToDevice, s);
+  if (tr->w) cudaMemcpyAsync(tr->w + off * k, h->ew, n * k * sizeof(float), cudaMemcpyDeviceToDevice, s);
+  if (prefill && tr->sa_k)
+    cudaMemcpy2DAsync((char *)tr->sa_k + off * hd * es, hd * es, (char *)h->qkv_sa + hd * es,
+                      3 * hd * es, hd * es, n, cudaMemcpyDeviceToDevice, s);
+  if (prefill && tr->sa_v)
+    cudaMemcpy2DAsync((char *)tr->sa_v + off * hd * es, hd * es, (char *)h->qkv_sa + 2 * hd * es,
+                      3 * hd * es, hd * es, n, cudaMemcpyDeviceToDevice, s);
+  if (c.n_proj_experts > 0) {
+    if (tr->pidx) cudaMemcpyAsync(tr->pidx + off, h->pidx, n * sizeof(int), cudaMemcpyDeviceToDevice, s);
+    if (tr->psig) cudaMemcpyAsync(tr->psig + off, h->psig, n * sizeof(float), cudaMemcpyDeviceToDevice, s);
+  }
+}
+
+static bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
+
+template <typename T>
+static int forward_impl(dreamer_handle *h, const void *x_in, void *x_out, int l0, int l1,
+                        void *da_kv, const dreamer_trace *tr, cudaStream_t s) {
+  const dreamer_config &c = h->cfg;
+  const int n = c.batch * c.seq;
+  CK(cudaMemsetAsync(h->counts, 0, (size_t)c.depth * c.n_experts * sizeof(int), s));
+  DepthIO io{};
+  io.mode = 0; io.n_tok = n; io.x_in = x_in; io.da_kv = da_kv ? da_kv : h->da_kv_int;
+  for (int l = l0; l < l1; l++) {
+    run_depth<T>(h, l, l == l0, io, s);
+    trace_depth(h, tr, l, n, true, s);
+  }
+  if (l1 > l0) {
+    long tot = (long)n * c.hidden;
+    finish_kernel<T><<<cdiv(tot / 8, 256), 256, 0, s>>>(h->acc, (T *)x_out, tot);
+  } else if (x_out != x_in) {
+    CK(cudaMemcpyAsync(x_out, x_in, (size_t)n * c.hidden * h->esz, cudaMemcpyDeviceToDevice, s));
+  }
+  CK(cudaGetLastError());
+  return DREAMER_OK;
+}
+
+extern "C" int dreamer_core_forward(dreamer_handle *h, const void *x_in, void *x_out,
+                                    int depth_begin, int depth_end, void *da_kv,
+                                    const dreamer_trace *trace, dreamer_stream stream) {
+  if (!h || !x_in || !x_out) return DREAMER_ERR_ARG;
+  const dreamer_config &c = h->cfg;
+  if (depth_begin < 0 || depth_end > c.depth || depth_begin > depth_end) return DREAMER_ERR_ARG;
+  if (!da_kv && depth_begin != 0) return DREAMER_ERR_ARG;
+  if (!aligned16(x_in) || !aligned16(x_out) || (da_kv && !aligned16(da_kv))) return DREAMER_ERR_ARG;
+  int e = check_dev_error(h);
+  if (e) return e;
+  cudaStream_t s = (cudaStream_t)stream;
+  return c.dtype == 0 ? forward_impl<float>(h, x_in, x_out, depth_begin, depth_end, da_kv, trace, s)
+                      : forward_impl<bf16>(h, x_in, x_out, depth_begin, depth_end, da_kv, trace, s);
+}
+
+template <typename T>
+static int decode_impl(dreamer_handle *h, const void *x_new, void *kc, void *vc,
+                       const int32_t *len, void *x_out, const dreamer_trace *tr, cudaStream_t s) {
+  const dreamer_config &c = h->cfg;
+  const int n = c.batch;
+  CK(cudaMemsetAsync(h->counts, 0, (size_t)c.depth * c.n_experts * sizeof(int), s));
+  DepthIO io{};
+  io.mode = 1; io.n_tok = n; io.x_in = x_new; io.da_kv = h->da_kv_int;
+  io.k_cache = kc; io.v_cache = vc; io.cache_len = len;
+  for (int l = 0; l < c.depth; l++) {
+    run_depth<T>(h, l, l == 0, io, s);
+    trace_depth(h, tr, l, n, false, s);
+  }
+  long tot = (long)n * c.hidden;
+  finish_kernel<T><<<cdiv(tot / 8, 256), 256, 0, s>>>(h->acc, (T *)x_out, tot);
+  CK(cudaGetLastError());
+  return DREAMER_OK;
+}
+
+extern "C" int dreamer_decode_step(dreamer_handle *h, const void *x_new, void *k_cache,
+                                   void *v_cache, const int32_t *cache_len, void *x_out,
+                                   const dreamer_trace *trace, dreamer_stream stream) {
+  if (!h || !x_new || !k_cache || !v_cache || !cache_len || !x_out) return DREAMER_ERR_ARG;
+  if (h->cfg.max_cache_len < 1) return DREAMER_ERR_STATE;
+  if (!aligned16(x_new) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(x_out))
+    return DREAMER_ERR_ARG;
+  int e = check_dev_error(h);
+  if (e) return e;
+  cudaStream_t s = (cudaStream_t)stream;
+  return h->cfg.dtype == 0
+             ? decode_impl<float>(h, x_new, k_cache, v_cache, cache_len, x_out, trace, s)
+             : decode_impl<bf16>(h, x_new, k_cache, v_cache, cache_len, x_out, trace, s);
+}
+
+extern "C" int dreamer_route_counts(dreamer_handle *h, int32_t *counts, int on_host,
+                                    dreamer_stream stream) {
+  if (!h || !counts) return DREAMER_ERR_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t bytes = (size_t)h->cfg.depth * h->cfg.n_experts * sizeof(int);
+  if (on_host) {
+    CK(cudaMemcpyAsync(counts, h->counts, bytes, cudaMemcpyDeviceToHost, s));
+    CK(cudaStreamSynchronize(s));
+    return check_dev_error(h);
+  }
+  CK(cudaMemcpyAsync(counts, h->counts, bytes, cudaMemcpyDeviceToDevice, s));
+  return DREAMER_OK;
+}
+
+extern "C" int dreamer_route_experts(dreamer_handle *h, int depth, const void *y, int n_tokens,
+                                     int32_t *idx, float *w, int32_t *counts,
+                                     dreamer_stream stream) {
+  if (!h || !y || !idx || !w) return DREAMER_ERR_ARG;
+  if (depth < 0 || depth >= h->cfg.depth || n_tokens < 0 || n_tokens > h->T) return DREAMER_ERR_ARG;
+  if (!aligned16(y)) return DREAMER_ERR_ARG;
+  if (n_tokens == 0) return DREAMER_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (counts) CK(cudaMemsetAsync(counts, 0, h->cfg.n_experts * sizeof(int), s));
+  if (h->cfg.dtype == 0)
+    route_rows<float>(h, 0, depth, y, n_tokens, idx, w, counts, nullptr, s);
+  else
+    route_rows<bf16>(h, 0, depth, y, n_tokens, idx, w, counts, nullptr, s);
+  CK(cudaGetLastError());
+  return DREAMER_OK;
+}
+
+extern "C" int dreamer_bias_update(dreamer_handle *h, float lambda, float *bias_out,
+                                   dreamer_stream stream) {
+  if (!h) return DREAMER_ERR_ARG;
+  const int E = h->cfg.n_experts;
+  int n2 = 1;
+  while (n2 < E) n2 <<= 1;
+  const size_t smem = (size_t)(n2 + E) * sizeof(int);
+  if (smem > 200 * 1024) return DREAMER_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (smem > 48 * 1024)
+    CK(cudaFuncSetAttribute(bias_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  bias_update_kernel<<<1, 1024, smem, s>>>(h->counts, h->cfg.depth, E, lambda, h->bias, bias_out);
+  CK(cudaGetLastError());
+  return DREAMER_OK;
+}

@@ -166,9 +166,20 @@ def input_specs(cfg: DreamerConfig) -> list[TensorSpec]:
     return specs
 
 
-def draw(spec: TensorSpec, seed: int, start: int = 0, n: int | None = None) -> np.ndarray:
-    """Flat elements [start, start+n) of a tensor, as float32 values of spec.dtype."""
+def draw(spec: TensorSpec, seed: int, start: int = 0, n: int | None = None,
+         use_c: bool = True) -> np.ndarray:
+    """Flat elements [start, start+n) of a tensor, as float32 values of spec.dtype.
+
+    Uses the C copy of the generator (libdreamer_inputs.so, OpenMP) when it is built, else
+    the numpy definition below."""
     n = spec.numel - start if n is None else n
+    if use_c and _lib_available():
+        out = np.empty(n, np.float32)
+        _lib().dri_fill_host(out.ctypes.data_as(ctypes.c_void_p),
+                             ctypes.c_uint64(stream_key(seed, spec.tid)), ctypes.c_uint64(start),
+                             ctypes.c_uint64(n), KIND_CODE[spec.kind], float(spec.param),
+                             DTYPE_CODE[spec.dtype])
+        return out
     if spec.kind == "ones":
         v = np.ones(n, np.float64)
     elif spec.kind == "normal":
@@ -210,6 +221,10 @@ _LIB = None
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
 
+def _lib_available() -> bool:
+    return os.path.exists(os.path.join(_HERE, "libdreamer_inputs.so"))
+
+
 def _lib():
     global _LIB
     if _LIB is None:
@@ -221,6 +236,10 @@ def _lib():
         lib.dri_fill.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint64,
                                  ctypes.c_uint64, ctypes.c_int, ctypes.c_double,
                                  ctypes.c_int, ctypes.c_void_p]
+        lib.dri_fill_host.restype = ctypes.c_int
+        lib.dri_fill_host.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint64,
+                                      ctypes.c_uint64, ctypes.c_int, ctypes.c_double,
+                                      ctypes.c_int]
         _LIB = lib
     return _LIB
 
@@ -238,3 +257,28 @@ def fill_device(ptr: int, spec: TensorSpec, seed: int, stream: int = 0,
                          float(spec.param), DTYPE_CODE[spec.dtype], ctypes.c_void_p(stream))
     if rc != 0:
         raise RuntimeError(f"dri_fill failed with CUDA error {rc}")
+
+
+def device_tensor(spec: TensorSpec, seed: int, stream=None):
+    """A torch CUDA tensor drawn in place by the device copy of the generator."""
+    import torch
+    dt = torch.float32 if spec.dtype == "fp32" else torch.bfloat16
+    t = torch.empty(spec.shape, dtype=dt, device="cuda")
+    s = stream if stream is not None else torch.cuda.current_stream()
+    fill_device(t.data_ptr(), spec, seed, stream=s.cuda_stream)
+    return t
+
+
+def device_weights(cfg: DreamerConfig) -> dict:
+    return {s.name: device_tensor(s, cfg.seed) for s in weight_specs(cfg)}
+
+
+def device_inputs(cfg: DreamerConfig) -> dict:
+    return {s.name: device_tensor(s, cfg.seed) for s in input_specs(cfg)}
+
+
+def to_device(arr: np.ndarray, dtype: str):
+    """Upload float32 host values (exact in dtype) as a CUDA tensor of dtype."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(arr, np.float32))
+    return t.to("cuda").to(torch.float32 if dtype == "fp32" else torch.bfloat16)

@@ -1,0 +1,170 @@
+/*
+ * libdreamer — B200 (sm_100a) forward pass of Dreamer's single depth-recurrent layer.
+ *
+ * Method (web pages about arXiv 2601.21582, "Depth-Recurrent Attention Mixtures: Giving
+ * Latent Reasoning the Attention it Deserves"; [notes] = papernotes.org notes, [gist] =
+ * gist.science technical summary):
+ *   one shared layer is applied for depths l = 0 .. L-1 ([notes] "Overall framework",
+ *   flowchart).  Each depth:
+ *     x^_l   = RMSNorm(x_l)                                      ([notes] flowchart)
+ *     y_l    = x^_l + DA(x^_0..l) + SA(x^_l)                     ([notes] "Key design 1")
+ *     x_l+1  = y_l + sum_{e in TopK} w_e FFN_e(y_l)               ([notes] "Key design 2")
+ *   with DA attending over the token's own depth states under a depth RoPE whose second
+ *   half is reversed, SA causal over tokens, expert selection
+ *   sigma(x) = norm(TopK(sigmoid(x), x + b, k)) against depth-RoPE'd expert keys, and
+ *   (optionally) top-1 linear-MoE QKV/O projections whose shared expert is absorbed into
+ *   each routed expert ([notes] "Key design 3": sigma x W + max(sigma^) x W_shared =
+ *   sigma x (W + W_shared)).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers unless stated, row-major, densely packed,
+ *     16-byte aligned, of the element type given by dreamer_config.dtype ("dtype" below:
+ *     0 = float32, 1 = bfloat16).  Routing weights, biases and counts have fixed types.
+ *   - Weight matrices use the x @ W convention: W[in][out].
+ *   - The caller owns every buffer it passes; the library never frees them.
+ *   - Calls are asynchronous on the given stream (0 = legacy default stream) and return
+ *     DREAMER_OK or a negative code.  A device-side error (a bounded wait that expired)
+ *     is reported by the next call on the handle and by dreamer_route_counts(on_host=1),
+ *     which synchronises.
+ *   - One handle per stream: calls on one handle must not overlap.
+ */
+#ifndef DREAMER_H
+#define DREAMER_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DREAMER_OK 0
+#define DREAMER_ERR_ARG (-1)         /* null/misaligned pointer, inconsistent config     */
+#define DREAMER_ERR_UNSUPPORTED (-2) /* shape outside what the kernels implement         */
+#define DREAMER_ERR_CUDA (-3)        /* a CUDA runtime call failed                        */
+#define DREAMER_ERR_OOM (-4)         /* device allocation failed                          */
+#define DREAMER_ERR_TIMEOUT (-5)     /* a kernel's bounded wait expired                   */
+#define DREAMER_ERR_STATE (-6)       /* call not valid for this handle's configuration   */
+
+typedef struct dreamer_handle dreamer_handle;
+typedef void *dreamer_stream; /* a cudaStream_t */
+
+typedef struct {
+  int batch;          /* b: sequences (prefill) or decode sequences                       */
+  int seq;            /* s: tokens per sequence for core_forward (1 for decode-only)       */
+  int hidden;         /* h = n_heads * head_dim                                           */
+  int n_heads;        /* H                                                                */
+  int head_dim;       /* d, multiple of 16                                                */
+  int depth;          /* L: number of depth steps (unrolled applications of the layer)    */
+  int n_experts;      /* E: expert-attention experts                                      */
+  int top_k;          /* k <= E, k <= 16                                                  */
+  int expert_hidden;  /* m: expert FFN hidden size, multiple of 16                        */
+  int router_dim;     /* d_r: expert/projection router key dim, multiple of 16            */
+  int n_proj_experts; /* P: 0 = dense QKV/O; else top-1 linear-MoE QKV/O with P experts   */
+  int dtype;          /* 0 = float32, 1 = bfloat16 (weights, activations, caches)         */
+  float rope_base;    /* 10000                                                            */
+  float rms_eps;      /* 1e-6                                                             */
+  int max_cache_len;  /* decode: SA cache capacity per sequence (0 = no decode)           */
+  int variant;        /* block layout ([notes] ablation table): 0 DA||SA then EA (default),
+                         1 serial DA->SA->EA, 2 fully parallel DA+SA+EA                   */
+} dreamer_config;
+
+typedef struct {
+  const void *rms_gain;     /* [h]                                                          */
+  const void *w_qkv;        /* [max(P,1)][h][6h]: columns qSA|kSA|vSA|qDA|kDA|vDA, each
+                               h wide and head-major (head j at columns j*d .. j*d+d-1)      */
+  const void *w_qkv_shared; /* [h][6h] shared expert, P > 0 only (NULL otherwise)           */
+  const void *w_o;          /* [max(P,1)][2h][h]: rows 0..h-1 take a_SA, rows h..2h-1 a_DA   */
+  const void *w_o_shared;   /* [2h][h], P > 0 only                                          */
+  const void *w_qP;         /* [h][d_r] projection-router query, P > 0 only                 */
+  const void *k_P;          /* [P][d_r] projection-expert keys, P > 0 only                  */
+  const void *w_qE;         /* [h][d_r] expert-router query                                 */
+  const void *k_E;          /* [E][d_r] expert keys (depth RoPE applied per depth inside)   */
+  const float *bias_E;      /* [E] float32 selection bias b                                 */
+  const void *w1;           /* [E][h][m] expert up-projections                              */
+  const void *w2;           /* [E][m][h] expert down-projections                            */
+} dreamer_weights;
+
+/* Optional per-depth dumps for checking and analysis; any member may be NULL.
+ * Layout [L][T][...] with T = batch*seq (forward) or batch (decode); only the depths a
+ * call runs are written.                                                                  */
+typedef struct {
+  void *xhat;      /* [L][T][h] dtype: RMSNorm output                                      */
+  void *y;         /* [L][T][h] dtype: input of expert attention                            */
+  int32_t *idx;    /* [L][T][k]: selected experts                                          */
+  float *w;        /* [L][T][k]: routing weights                                           */
+  void *sa_k;      /* [L][T][h] dtype: post-RoPE SA keys (forward only)                    */
+  void *sa_v;      /* [L][T][h] dtype: SA values (forward only)                            */
+  int32_t *pidx;   /* [L][T]: projection expert p* (P > 0)                                 */
+  float *psig;     /* [L][T]: projection weight sigma (P > 0)                              */
+} dreamer_trace;
+
+/* Create a handle: validates the configuration, copies the weights (device pointers) into
+ * handle-owned buffers in the kernels' layouts, absorbs the shared projection expert into
+ * every routed one (W~_p = round(W_p + W_shared), [notes] "Key design 3"), precomputes the
+ * RoPE tables and allocates the workspace for batch*seq tokens.  Synchronises `stream`.
+ * Returns DREAMER_ERR_ARG / _UNSUPPORTED / _OOM / _CUDA on failure (*out = NULL).         */
+int dreamer_init(const dreamer_config *cfg, const dreamer_weights *weights,
+                 dreamer_stream stream, dreamer_handle **out);
+
+/* Prefill forward over depths [depth_begin, depth_end) for all batch*seq tokens
+ * ([notes] "Overall framework" flowchart; "Key design 1" residual equation).
+ *   x_in   [T][h] dtype: residual stream x at depth_begin (x_0 when depth_begin = 0).
+ *   x_out  [T][h] dtype: residual stream at depth_end (no final norm).
+ *   da_kv  [T][L][2][h] dtype or NULL.  The depth KV buffer: slot [t][j][0] holds the
+ *          post-depth-RoPE DA key of token t at depth j, [t][j][1] its value.  Depths below
+ *          depth_begin are read, depths depth_begin .. depth_end-1 are written.  NULL uses
+ *          a handle-owned buffer and then requires depth_begin == 0.
+ *   trace  NULL or dump pointers.
+ * Route counts of the run depths are kept in the handle (zeroed at the start of the call).
+ * x_in and x_out may alias.                                                               */
+int dreamer_core_forward(dreamer_handle *h, const void *x_in, void *x_out, int depth_begin,
+                         int depth_end, void *da_kv, const dreamer_trace *trace,
+                         dreamer_stream stream);
+
+/* One decode step: one new token for each of the `batch` sequences through all L depths
+ * ([notes] "Overall framework": the SA KV cache persists across tokens while the DA KV
+ * cache is overwritten for the next token).
+ *   x_new   [B][h] dtype: the new tokens' embeddings.
+ *   k_cache, v_cache [L][B][H][max_cache_len][d] dtype: per-depth SA caches holding
+ *           post-RoPE keys and values of past tokens.  Slot cache_len[b] of every depth is
+ *           written with the new token's key/value; the call attends over cache_len[b]+1
+ *           keys.  The caller advances cache_len afterwards.
+ *   cache_len [B] int32, device: past tokens per sequence (< max_cache_len).
+ *   x_out   [B][h] dtype.                                                                 */
+int dreamer_decode_step(dreamer_handle *h, const void *x_new, void *k_cache, void *v_cache,
+                        const int32_t *cache_len, void *x_out, const dreamer_trace *trace,
+                        dreamer_stream stream);
+
+/* Route counts N[l][e] of the last forward/decode call ([notes] "Key design 2": the usage
+ * counts the bias update balances).  counts: [L][E] int32, device pointer (on_host = 0) or
+ * host pointer (on_host = 1; the call then synchronises `stream` and also reports any
+ * device-side error).  Depths the call did not run hold 0.                                 */
+int dreamer_route_counts(dreamer_handle *h, int32_t *counts, int on_host,
+                         dreamer_stream stream);
+
+/* Expert routing alone on given states ([notes] "Key design 2", routing equation):
+ * z_e = (y W_qE) . (depth-RoPE_l k_e) / sqrt(d_r); pick the k experts with the largest
+ * z_e + b_e (ties to the lower index); w_e = sigmoid(z_e) / sum over picks.
+ *   y [n_tokens][h] dtype; idx [n_tokens][k] int32; w [n_tokens][k] float32;
+ *   counts [E] int32 (overwritten with this call's histogram) or NULL.
+ * n_tokens <= batch*seq (or batch for a decode-only handle).                              */
+int dreamer_route_experts(dreamer_handle *h, int depth, const void *y, int n_tokens,
+                          int32_t *idx, float *w, int32_t *counts, dreamer_stream stream);
+
+/* Bias balance update from the handle's last route counts ([notes] "Key design 2"):
+ * b_e <- b_e + lambda * sign(median(N) - N_e), N_e = sum over depths, lower median for an
+ * even E.  Updates the handle's bias; if bias_out is not NULL also copies the new bias
+ * ([E] float32, device) there.                                                            */
+int dreamer_bias_update(dreamer_handle *h, float lambda, float *bias_out,
+                        dreamer_stream stream);
+
+/* Free the handle and everything it owns (synchronises the device).                      */
+void dreamer_destroy(dreamer_handle *h);
+
+/* Static description of an error code.                                                    */
+const char *dreamer_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DREAMER_H */

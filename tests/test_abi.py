@@ -1,0 +1,60 @@
+"""The C-ABI library loads and exports every entry point include/dreamer.h declares (no GPU
+calls)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+PKG = os.path.join(ROOT, "depth_recurrent_attention_b200")
+
+
+@pytest.fixture(scope="module")
+def built():
+    from depth_recurrent_attention_b200 import build
+    return build.build()
+
+
+def declared(header):
+    txt = open(os.path.join(ROOT, "include", header)).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(dreamer_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared("dreamer.h")
+    for n in ("dreamer_init", "dreamer_core_forward", "dreamer_decode_step",
+              "dreamer_route_counts", "dreamer_route_experts", "dreamer_bias_update",
+              "dreamer_destroy", "dreamer_strerror"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(built):
+    lib = ctypes.CDLL(os.path.join(PKG, "libdreamer.so"))
+    for header in os.listdir(os.path.join(ROOT, "include")):
+        for n in declared(header):
+            assert hasattr(lib, n), f"{n} declared in {header} but not exported"
+    out = subprocess.run(["nm", "-D", "--defined-only", os.path.join(PKG, "libdreamer.so")],
+                         capture_output=True, text=True).stdout
+    for n in declared("dreamer.h"):
+        assert re.search(rf"\bT {n}\b", out), n
+
+
+def test_strerror_without_gpu(built):
+    lib = ctypes.CDLL(os.path.join(PKG, "libdreamer.so"))
+    lib.dreamer_strerror.restype = ctypes.c_char_p
+    assert lib.dreamer_strerror(0) == b"ok"
+    assert lib.dreamer_strerror(-1) == b"invalid argument"
+    assert lib.dreamer_strerror(-5) == b"device wait timed out"
+
+
+def test_product_does_not_reference_the_oracle():
+    for dirpath, _, files in os.walk(PKG):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in txt.lower() or f == "inputs.py", f
+    lib_txt = open(os.path.join(PKG, "dreamer.py")).read()
+    assert "import oracle" not in lib_txt

@@ -1,0 +1,305 @@
+"""GPU parity of libdreamer (through the C ABI) against the CPU oracle on seeded inputs.
+
+Tolerances are the contract's (see tests/parity.py).  Inputs for the oracle and for the GPU
+come from the same seeded generator; nothing the GPU computes is fed to the oracle.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+import parity as PY
+from depth_recurrent_attention_b200 import configs, inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def upload(cfg, arrays: dict):
+    return {k: inputs.to_device(v, "fp32" if k == "bias" else cfg.dtype) for k, v in arrays.items()}
+
+
+def make_handle(cfg, W_host, **kw):
+    from depth_recurrent_attention_b200.dreamer import Dreamer
+    return Dreamer(cfg, upload(cfg, W_host), **kw)
+
+
+def trace_buffers(cfg, n_tok, with_sa=False):
+    torch = _torch()
+    L, h, k = cfg.depth, cfg.hidden, cfg.top_k
+    dt = torch.float32 if cfg.dtype == "fp32" else torch.bfloat16
+    tr = dict(y=torch.zeros((L, n_tok, h), dtype=dt, device="cuda"),
+              xhat=torch.zeros((L, n_tok, h), dtype=dt, device="cuda"),
+              idx=torch.zeros((L, n_tok, k), dtype=torch.int32, device="cuda"),
+              w=torch.zeros((L, n_tok, k), dtype=torch.float32, device="cuda"))
+    if cfg.n_proj_experts > 0:
+        tr["pidx"] = torch.zeros((L, n_tok), dtype=torch.int32, device="cuda")
+        tr["psig"] = torch.zeros((L, n_tok), dtype=torch.float32, device="cuda")
+    if with_sa:
+        tr["sa_k"] = torch.zeros((L, n_tok, h), dtype=dt, device="cuda")
+        tr["sa_v"] = torch.zeros((L, n_tok, h), dtype=dt, device="cuda")
+    return tr
+
+
+# ---------------------------------------------------------------------------------------
+# tiny, float32, free-running end to end
+
+@pytest.mark.parametrize("variant", [0, 1, 2])
+def test_tiny_forward_fp32(cuda, variant):
+    torch = _torch()
+    cfg = configs.TINY.with_(variant=variant)
+    W = inputs.host_weights(cfg)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    ref = O.Oracle(cfg, W).forward(x0)
+    dev = make_handle(cfg, W)
+    tr = trace_buffers(cfg, cfg.tokens)
+    out = dev.forward(inputs.to_device(x0, "fp32"), trace=tr)
+    torch.cuda.synchronize()
+    for l in range(cfg.depth):
+        same, flips = PY.check_routing(cfg, W, l, tr["idx"][l].cpu().numpy(), ref["idx"][l],
+                                       ref["margin"][l], strict=True)
+        assert flips == 0, "a near tie flipped; later depths are not comparable"
+        assert np.allclose(PY.to_np(tr["w"][l]), ref["w"][l], atol=1e-5)
+        PY.check_hidden(PY.to_np(tr["y"][l]), ref["y"][l], False, f"y depth {l}")
+    PY.check_hidden(PY.to_np(out), ref["x_out"], False, "x_L")
+    counts = dev.route_counts(on_host=True).numpy()
+    assert np.array_equal(counts, ref["counts"])
+
+
+def test_tiny_depth_ranges_compose(cuda):
+    torch = _torch()
+    cfg = configs.TINY
+    W = inputs.host_weights(cfg)
+    x0 = inputs.to_device(inputs.host_inputs(cfg)["x0"], "fp32")
+    dev = make_handle(cfg, W)
+    full = dev.forward(x0).clone()
+    da = torch.zeros((cfg.tokens, cfg.depth, 2, cfg.hidden), device="cuda")
+    mid = dev.forward(x0, depth_begin=0, depth_end=2, da_kv=da)
+    out = dev.forward(mid, depth_begin=2, depth_end=cfg.depth, da_kv=da)
+    assert torch.allclose(out, full, atol=1e-5, rtol=0)
+
+
+# ---------------------------------------------------------------------------------------
+# router on identical inputs: strict index parity
+
+@pytest.mark.parametrize("name,l", [("tiny", 1), ("small", 0), ("small", 5)])
+def test_router_strict(cuda, name, l):
+    cfg = configs.CONFIGS[name]
+    W = inputs.host_weights(cfg)
+    y = inputs.extra_normal(cfg, 3000 + l, (cfg.tokens, cfg.hidden), 1.0)
+    ref = O.Oracle(cfg, W).route(l, y)
+    dev = make_handle(cfg, W)
+    idx, w, counts = dev.route_experts(l, inputs.to_device(y, cfg.dtype))
+    idx = idx.cpu().numpy()
+    same, flips = PY.check_routing(cfg, W, l, idx, ref["idx"], ref["margin"], strict=True)
+    near = int((ref["margin"] <= PY.NEAR_TIE).sum())
+    print(f"router {name} depth {l}: {flips} flips at {near} near ties")
+    assert np.allclose(PY.to_np(w)[same], ref["w"][same], atol=1e-5)
+    c = counts.cpu().numpy()
+    assert np.array_equal(c, np.bincount(idx.ravel(), minlength=cfg.n_experts))
+    if flips == 0:
+        assert np.array_equal(c, ref["counts"])
+
+
+# ---------------------------------------------------------------------------------------
+# small, bf16: one depth at a time from seeded states (every depth)
+
+def step_inputs(cfg, l):
+    T, L, h = cfg.tokens, cfg.depth, cfg.hidden
+    x = inputs.extra_normal(cfg, 1000 + l, (T, h), 1.0)
+    hist = np.zeros((T, L, 2, h), np.float32)
+    if l > 0:
+        hist[:, :l] = inputs.extra_normal(cfg, 2000 + l, (T, l, 2, h), 1.0)
+    return x, hist
+
+
+def run_step_and_compare(cfg, W, dev, l, toks=None, orc=None):
+    torch = _torch()
+    x, hist = step_inputs(cfg, l)
+    tr = trace_buffers(cfg, cfg.tokens)
+    xd = inputs.to_device(x, cfg.dtype)
+    hd = inputs.to_device(hist, cfg.dtype)
+    out = dev.forward(xd, depth_begin=l, depth_end=l + 1, da_kv=hd, trace=tr)
+    torch.cuda.synchronize()
+    g_x, g_y = PY.to_np(out), PY.to_np(tr["y"][l])
+    g_idx = tr["idx"][l].cpu().numpy()
+    o = orc or O.Oracle(cfg, W)
+    if toks is None:
+        r = o.forward(x, l, l + 1, da_kv=hist.astype(np.float64))
+        rx, ry, ridx, rmg = r["x_out"], r["y"][l], r["idx"][l], r["margin"][l]
+        sel = slice(None)
+        g_da = PY.to_np(hd[:, l])
+        assert np.allclose(g_da, r["da_kv"][:, l], atol=PY.TOL_BF16_ABS * 2)
+    else:
+        seq, pos = toks
+        S = cfg.seq
+        tk = seq * S + np.asarray(pos)
+        r = o.step_tokens(l, x[seq * S:(seq + 1) * S], hist[tk].astype(np.float64), pos)
+        rx, ry, ridx, rmg = r["x_out"], r["y"], r["idx"], r["margin"]
+        sel = tk
+    bf = cfg.dtype == "bf16"
+    PY.check_hidden(g_y[sel], ry, bf, f"y depth {l}")
+    same, flips = PY.check_routing(cfg, W, l, g_idx[sel], ridx, rmg, g_y[sel], ry)
+    PY.check_hidden(g_x[sel][same], rx[same], bf, f"x depth {l}")
+    return flips, int(np.size(same))
+
+
+def test_small_every_depth_bf16(cuda):
+    cfg = configs.SMALL
+    W = inputs.host_weights(cfg)
+    dev = make_handle(cfg, W)
+    orc = O.Oracle(cfg, W)
+    tot = 0
+    for l in range(cfg.depth):
+        flips, n = run_step_and_compare(cfg, W, dev, l, orc=orc)
+        print(f"small depth {l}: {flips}/{n} routing flips explained by bf16 rounding of y")
+        assert flips <= 0.05 * n
+        tot += flips
+
+
+@pytest.mark.parametrize("variant", [1, 2])
+def test_small_layout_variants_bf16(cuda, variant):
+    cfg = configs.SMALL.with_(variant=variant, depth=3)
+    W = inputs.host_weights(cfg)
+    dev = make_handle(cfg, W)
+    if variant == 1:
+        # the serial layout needs every token's DA; run the whole (short) forward
+        torch = _torch()
+        x0 = inputs.host_inputs(cfg)["x0"]
+        ref = O.Oracle(cfg, W).forward(x0, 0, 1)
+        tr = trace_buffers(cfg, cfg.tokens)
+        out = dev.forward(inputs.to_device(x0, "bf16"), depth_end=1, trace=tr)
+        torch.cuda.synchronize()
+        gy = PY.to_np(tr["y"][0])
+        PY.check_hidden(gy, ref["y"][0], True, "y serial")
+        same, flips = PY.check_routing(cfg, W, 0, tr["idx"][0].cpu().numpy(), ref["idx"][0],
+                                       ref["margin"][0], gy, ref["y"][0])
+        PY.check_hidden(PY.to_np(out)[same], ref["x_out"][same], True, "x serial")
+    else:
+        for l in (0, 2):
+            run_step_and_compare(cfg, W, dev, l)
+
+
+def test_small_free_running_drift_reported(cuda):
+    """Free-running bf16 through all 8 depths: routing flips compound, so the drift is
+    reported, not gated; only a gross failure (rel-L2 > 0.5) fails."""
+    cfg = configs.SMALL
+    W = inputs.host_weights(cfg)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    ref = O.Oracle(cfg, W).forward(x0, trace=False)
+    dev = make_handle(cfg, W)
+    out = PY.to_np(dev.forward(inputs.to_device(x0, "bf16")))
+    rl = PY.rel_l2(out, ref["x_out"])
+    print(f"small free-running bf16 drift: rel-L2 {rl:.3e}, max-abs "
+          f"{np.max(np.abs(out - ref['x_out'])):.3e}")
+    assert rl < 0.5
+
+
+# ---------------------------------------------------------------------------------------
+# decode
+
+def decode_case(cfg, lens):
+    B, L, H, d = cfg.batch, cfg.depth, cfg.n_heads, cfg.head_dim
+    cap = cfg.cache_len + 1
+    kc = inputs.extra_normal(cfg, 4001, (L, B, H, cap, d), 1.0)
+    vc = inputs.extra_normal(cfg, 4002, (L, B, H, cap, d), 1.0)
+    x = inputs.extra_normal(cfg, 4003, (B, cfg.hidden), 1.0)
+    return x, kc, vc, np.asarray(lens, np.int32)
+
+
+@pytest.mark.parametrize("base,lens", [("tiny", [12, 5, 0]), ("small", [300, 1, 77, 299])])
+def test_decode_step(cuda, base, lens):
+    torch = _torch()
+    cfg = configs.CONFIGS[base].with_(batch=len(lens), seq=1, cache_len=max(lens) + 1)
+    W = inputs.host_weights(cfg)
+    x, kc, vc, ln = decode_case(cfg, lens)
+    dev = make_handle(cfg, W)
+    kd, vd = inputs.to_device(kc, cfg.dtype), inputs.to_device(vc, cfg.dtype)
+    tr = trace_buffers(cfg, cfg.batch)
+    out = dev.decode_step(inputs.to_device(x, cfg.dtype), kd, vd,
+                          torch.from_numpy(ln).cuda(), trace=tr)
+    torch.cuda.synchronize()
+    o = O.Oracle(cfg, W)
+    bf = cfg.dtype == "bf16"
+    g = PY.to_np(out)
+    kd_np, vd_np = PY.to_np(kd), PY.to_np(vd)
+    for b in range(cfg.batch):
+        kcb = kc[:, b].astype(np.float64).copy()
+        vcb = vc[:, b].astype(np.float64).copy()
+        r = o.decode_seq(x[b], kcb, vcb, int(ln[b]))
+        # the new token's key/value went to slot cache_len of every depth
+        PY.check_hidden(kd_np[:, b, :, ln[b]], kcb[:, :, ln[b]], bf, f"k slot seq {b}")
+        PY.check_hidden(vd_np[:, b, :, ln[b]], vcb[:, :, ln[b]], bf, f"v slot seq {b}")
+        if not bf:
+            for l in range(cfg.depth):
+                same, flips = PY.check_routing(cfg, W, l, tr["idx"][l, b:b + 1].cpu().numpy(),
+                                               r["idx"][l:l + 1], r["margin"][l:l + 1],
+                                               strict=True)
+                assert flips == 0
+            PY.check_hidden(g[b], r["x_out"], False, f"x_out seq {b}")
+        else:
+            # first depth is comparable token by token; later depths drift by routing flips
+            gy = PY.to_np(tr["y"][0, b])
+            PY.check_hidden(gy, r["y"][0], True, f"y depth 0 seq {b}")
+
+
+# ---------------------------------------------------------------------------------------
+# bias balance update, error handling, generator
+
+def test_bias_update_matches_oracle(cuda):
+    torch = _torch()
+    cfg = configs.TINY
+    W = inputs.host_weights(cfg)
+    dev = make_handle(cfg, W)
+    dev.forward(inputs.to_device(inputs.host_inputs(cfg)["x0"], "fp32"))
+    counts = dev.route_counts(on_host=True).numpy()
+    new_b = dev.bias_update(0.01).cpu().numpy()
+    ref = O.bias_update(counts, 0.01, W["bias"].astype(np.float64))
+    assert np.allclose(new_b, ref, atol=1e-7)
+
+
+def test_errors_are_returned_not_faulted(cuda):
+    torch = _torch()
+    from depth_recurrent_attention_b200.dreamer import Dreamer, DreamerError, ERR_ARG, \
+        ERR_UNSUPPORTED, ERR_STATE
+    cfg = configs.TINY
+    W = upload(cfg, inputs.host_weights(cfg))
+    with pytest.raises(DreamerError) as e:
+        Dreamer(cfg.with_(hidden=65), W)
+    assert e.value.code == ERR_ARG
+    with pytest.raises(DreamerError) as e:
+        Dreamer(cfg.with_(top_k=17, n_experts=32), W)
+    assert e.value.code == ERR_UNSUPPORTED
+    with pytest.raises(DreamerError) as e:
+        Dreamer(cfg.with_(head_dim=8, n_heads=8), W)
+    assert e.value.code == ERR_UNSUPPORTED
+    dev = Dreamer(cfg, W)
+    x = torch.zeros((cfg.tokens, cfg.hidden), device="cuda")
+    with pytest.raises(DreamerError) as e:          # no DA buffer for a later start depth
+        dev.forward(x, depth_begin=1)
+    assert e.value.code == ERR_ARG
+    with pytest.raises(DreamerError) as e:          # misaligned pointer
+        xm = x.view(-1)[1:1 + (cfg.tokens - 1) * cfg.hidden].view(cfg.tokens - 1, cfg.hidden)
+        dev.forward(xm)
+    assert e.value.code == ERR_ARG
+    with pytest.raises(DreamerError) as e:          # decode on a handle without a cache
+        dev.decode_step(x[:1], x, x, torch.zeros(1, dtype=torch.int32, device="cuda"))
+    assert e.value.code == ERR_STATE
+    # the context is still usable
+    dev.forward(x)
+    torch.cuda.synchronize()
+
+
+def test_device_generator_matches_host(cuda):
+    torch = _torch()
+    cfg = configs.SMALL
+    for spec in inputs.weight_specs(cfg):
+        t = inputs.device_tensor(spec, cfg.seed)
+        n = min(spec.numel, 1 << 20)
+        host = inputs.draw(spec, cfg.seed, 0, n)
+        dev = t.float().view(-1)[:n].cpu().numpy()
+        mism = int((host != dev).sum())
+        assert mism <= max(1, n // 1_000_000), (spec.name, mism)
