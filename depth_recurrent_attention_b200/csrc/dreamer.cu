@@ -36,16 +36,17 @@ struct dreamer_handle {
   void *xh = nullptr, *qkv_sa = nullptr, *q_da = nullptr, *attn = nullptr, *y = nullptr;
   void *u = nullptr, *da_kv_int = nullptr, *Hbuf = nullptr, *qsplit = nullptr;
   float *acc = nullptr, *zbuf = nullptr, *qbuf = nullptr, *psig = nullptr, *ew = nullptr;
+  float *inv_rms = nullptr;      // [T] 1/rms of the current depth's residual
   int *pidx = nullptr, *eidx = nullptr, *counts = nullptr, *ecnt = nullptr, *eoffs = nullptr;
   int *etiles_a = nullptr, *etiles_b = nullptr, *ecursor = nullptr, *erows = nullptr;
   int *pcnt = nullptr, *poffs = nullptr, *ptiles_a = nullptr, *ptiles_b = nullptr;
   int *pcursor = nullptr, *prows = nullptr, *pinv = nullptr;
   int *err = nullptr;
+  void *k3 = nullptr;            // [E][3 d_r] bf16: router keys repeated for split scores
+  int num_sms = 148;
   int use_tc = 1;  // bf16 contractions on tcgen05 (0: CUDA cores, for cross-checks)
   std::vector<void *> allocs;
 };
-
-#include "tc_kernels.cuh"
 
 #define CK(call)                                                  \
   do {                                                            \
@@ -75,6 +76,9 @@ static int dalloc(dreamer_handle *h, void **p, size_t bytes) {
   } while (0)
 
 static inline int cdiv(long a, long b) { return (int)((a + b - 1) / b); }
+
+#include "tc_kernels.cuh"
+
 static inline int round8(int v) { return (v + 7) / 8 * 8; }
 
 extern "C" const char *dreamer_strerror(int code) {
@@ -257,6 +261,7 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     DALLOC(h->attn, T * 2 * hd * es);
     DALLOC(h->y, T * hd * es);
     DALLOC(h->acc, T * hd * sizeof(float));
+    DALLOC(h->inv_rms, T * sizeof(float));
     DALLOC(h->da_kv_int, (size_t)T * L * 2 * hd * es);
     DALLOC(h->Hbuf, (Tk + 128) * m * es);
     DALLOC(h->qsplit, T * 3 * dr * 2);
@@ -349,10 +354,9 @@ static void route_rows(dreamer_handle *h, int mode, int l, const void *X, int n,
   const int ldz = mode == 0 ? h->ldz : h->ldzp;
   const void *Wq = mode == 0 ? h->wqE_t : h->wqP_t;
   const float *krot = (mode == 0 ? h->kE_rot : h->kP_rot) + (size_t)l * E * dr;
-  if (mode == 0 && h->use_tc && c.dtype == 1 && tc_route_ok(h)) {
-    tc_route(h, l, X, n, idx, wout, counts_a, counts_b, s);
+  if (mode == 0 && h->use_tc && c.dtype == 1 && tc_route_ok(h) &&
+      tc_route(h, l, X, n, idx, wout, counts_a, counts_b, s))
     return;
-  }
   // q = X W_q (fp32 accumulation), z = q . k~ (fp32), on CUDA cores
   GemmArgs a = dense_args(n, dr, hd, X, hd, Wq, hd);
   gemm_simt<T, T, 8>(a, cdiv(n, 64), EpiStoreF32{h->qbuf, dr, dr}, s);
@@ -387,7 +391,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
   // 1. RMSNorm of the residual stream (x_0 on the first depth, else the fp32 accumulator)
   rmsnorm_kernel<T><<<cdiv(n, 8), 256, 0, s>>>(first ? (const T *)io.x_in : nullptr,
                                                first ? nullptr : h->acc, (const T *)h->g,
-                                               (T *)h->xh, nullptr, n, hd, c.rms_eps);
+                                               (T *)h->xh, h->inv_rms, n, hd, c.rms_eps);
   // 2. projection router and token grouping (linear-MoE QKV/O)
   const int *prow = nullptr;
   const float *psig = nullptr;
@@ -434,10 +438,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
                          (long)6 * hd * hd);
     EpiQKV<T> e2 = eq;
     e2.col_lo = col0;
-    if (tc && tc_gemm_ok(h, a)) {
-      tc_gemm_qkv(h, a, e2, s);
-      return;
-    }
+    if (tc && tc_gemm_ok(h, a) && tc_gemm_qkv(h, a, e2, s)) return;
     switch (d) {
       case 16: gemm_qkv<T, 16>(h, a, ptiles, e2, s); break;
       case 32: gemm_qkv<T, 32>(h, a, ptiles, e2, s); break;
@@ -445,15 +446,16 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
       default: gemm_qkv<T, 128>(h, a, ptiles, e2, s); break;
     }
   };
-  auto o_gemm = [&](const void *A, int row0, int nrows, const void *resid) {
+  // residual source of the O epilogue: x^ rebuilt from x_l (first depth: the input,
+  // else the fp32 accumulator rounded to dtype) or, for the serial layout's second half, u
+  const int res_xhat = first ? 0 : 1;
+  auto o_gemm = [&](const void *A, int row0, int nrows, int res_mode, void *yout) {
     // O projection over input rows [row0, row0 + nrows) of W_O ([a_SA | a_DA] order)
     GemmArgs a = grouped(hd, nrows, A, 2 * hd, (const T *)h->wo_t + row0, (long)2 * hd * hd);
     a.ldb = 2 * hd;
-    EpiO<T> eo{hd, psig, (const T *)resid, (T *)h->y, h->acc};
-    if (tc && tc_gemm_ok(h, a)) {
-      tc_gemm_o(h, a, eo, s);
-      return;
-    }
+    EpiO<T> eo{hd, psig, res_mode, (const T *)io.x_in, h->inv_rms, (const T *)h->g,
+               (T *)yout, h->acc};
+    if (tc && tc_gemm_ok(h, a) && tc_gemm_o(h, a, eo, s)) return;
     gemm_simt<T, T, 16>(a, ptiles, eo, s);
   };
 
@@ -461,16 +463,10 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
     // serial DA -> SA -> EA: DA on x^, then SA on u = x^ + DA-part of O, then EA
     qkv_gemm(h->xh, 3 * hd, 3 * hd);
     launch_attn<T>(da, d, s);
-    {
-      GemmArgs a = grouped(hd, hd, (const T *)h->attn + hd, 2 * hd,
-                           (const T *)h->wo_t + hd, (long)2 * hd * hd);
-      a.ldb = 2 * hd;
-      EpiO<T> eo{hd, psig, (const T *)h->xh, (T *)h->u, nullptr};
-      gemm_simt<T, T, 16>(a, ptiles, eo, s);
-    }
+    o_gemm((const T *)h->attn + hd, hd, hd, res_xhat, h->u);   // u = x^ + DA part (acc = u)
     qkv_gemm(h->u, 0, 3 * hd);
     if (io.mode == 0 && tc && tc_sa_ok(h)) tc_sa(h, s); else launch_attn<T>(sa, d, s);
-    o_gemm(h->attn, 0, hd, h->u);
+    o_gemm(h->attn, 0, hd, 2, h->y);                            // y = u + SA part
   } else {
     // 3. fused QKV projection with RoPE / depth RoPE epilogue, DA KV write
     qkv_gemm(h->xh, 0, 6 * hd);
@@ -478,7 +474,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
     launch_attn<T>(da, d, s);
     if (io.mode == 0 && tc && tc_sa_ok(h)) tc_sa(h, s); else launch_attn<T>(sa, d, s);
     // 5. O projection, residual y = x^ + DA + SA
-    o_gemm(h->attn, 0, 2 * hd, h->xh);
+    o_gemm(h->attn, 0, 2 * hd, res_xhat, h->y);
   }
   // 6. expert attention routing on y (fully parallel layout: on x^)
   const void *ein = c.variant == 2 ? h->xh : h->y;
@@ -489,9 +485,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
   scatter_kernel<<<cdiv((long)n * k, 256), 256, 0, s>>>(h->eidx, n * k, h->ecursor, h->erows,
                                                          nullptr);
   // 7. expert FFNs: H = SiLU(X W1_e), acc[token] += w * H W2_e
-  if (tc && tc_expert_ok(h)) {
-    tc_expert(h, ein, n, s);
-  } else {
+  if (!(tc && tc_expert_ok(h) && tc_expert(h, ein, n, s))) {
     const int etiles = cdiv((long)n * k, 64) + E;
     GemmArgs up{};
     up.N = m; up.K = hd; up.G = E; up.M = n * k; up.goffs = h->eoffs; up.tile_offs = h->etiles_a;
@@ -524,7 +518,7 @@ static void trace_depth(dreamer_handle *h, const dreamer_trace *tr, int l, int n
   const size_t es = h->esz, hd = c.hidden, k = c.top_k;
   const size_t off = (size_t)l * n;
   if (tr->xhat) cudaMemcpyAsync((char *)tr->xhat + off * hd * es, h->xh, n * hd * es, cudaMemcpyDeviceToDevice, s);
-  if (tr->y) cudaMemcpyAsync((char *)tr->y + off * hd * es, c.variant == 2 ? h->xh : h->y, n * hd * es, cudaMemcpyDeviceToDevice, s);
+  if (tr->y) cudaMemcpyAsync((char *)tr->y + off * hd * es, h->y, n * hd * es, cudaMemcpyDeviceToDevice, s);
   if (tr->idx) cudaMemcpyAsync(tr->idx + off * k, h->eidx, n * k * sizeof(int), cudaMemcpyDeviceToDevice, s);
   if (tr->w) cudaMemcpyAsync(tr->w + off * k, h->ew, n * k * sizeof(float), cudaMemcpyDeviceToDevice, s);
   if (prefill && tr->sa_k)

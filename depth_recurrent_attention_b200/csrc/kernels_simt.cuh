@@ -93,24 +93,44 @@ template <typename T> struct EpiQKV {
 };
 
 // O projection epilogue: y = x^ + sigma [a_SA | a_DA] W~_O (papernotes "Key design 1"
-// residual equation); also seeds the fp32 accumulator of x_{l+1} with y.
+// residual equation).  The residual is carried in fp32: x^ is rebuilt from the residual x_l
+// (dtype: the input on the first depth, else the fp32 accumulator rounded to dtype), the gain
+// and the token's 1/rms, so the only rounding of y is its own store.  acc receives the fp32 y
+// (the base that the expert outputs are added to); y itself is stored in dtype for the
+// router and the experts.
+//   res_mode 0: residual x^ from xin;  1: x^ from round(acc);  2: residual = acc as is
+//   (the serial layout's u).
 template <typename T> struct EpiO {
   int h;
   const float *psig;
-  const T *resid;   // [T][h] x^ (or u in the serial layout)
-  T *y;             // [T][h]
-  float *acc;       // [T][h]
+  int res_mode;
+  const T *xin;
+  const float *inv_rms;
+  const T *gain;
+  T *y;             // [T][h] or null
+  float *acc;       // [T][h] read (res_mode 1, 2) and written
   template <int SEG>
   __device__ __forceinline__ void operator()(int r, int token, int g, int n0, float *v) const {
     const float s = psig ? psig[token] : 1.0f;
+    const float ir = res_mode == 2 ? 0.f : inv_rms[token];
 #pragma unroll
     for (int i = 0; i < SEG; i += 8) {
-      float xr[8], o[8];
-      load8(resid + (long)token * h + n0 + i, xr);
+      float xr[8], gv[8], o[8];
+      float *ap = acc + (long)token * h + n0 + i;
+      if (res_mode == 0) load8(xin + (long)token * h + n0 + i, xr);
+      else load8(ap, xr);
+      if (res_mode != 2) {
+        load8(gain + n0 + i, gv);
 #pragma unroll
-      for (int j = 0; j < 8; j++) o[j] = to_f(from_f<T>(xr[j] + s * v[i + j]));
-      store8(y + (long)token * h + n0 + i, o);
-      if (acc) store8(acc + (long)token * h + n0 + i, o);
+        for (int j = 0; j < 8; j++) {
+          const float xv = res_mode == 1 ? to_f(from_f<T>(xr[j])) : xr[j];
+          xr[j] = gv[j] * xv * ir;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; j++) o[j] = xr[j] + s * v[i + j];
+      if (y) store8(y + (long)token * h + n0 + i, o);
+      store8(ap, o);
     }
   }
 };
@@ -274,7 +294,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a, Epi epi) {
 // =======================================================================================
 template <typename T>
 __global__ void rmsnorm_kernel(const T *x_in, const float *acc, const T *gain, T *xh,
-                               T *x_store, int n_tok, int h, float eps) {
+                               float *inv_rms, int n_tok, int h, float eps) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= n_tok) return;
@@ -293,13 +313,13 @@ __global__ void rmsnorm_kernel(const T *x_in, const float *acc, const T *gain, T
   }
   ss = warp_sum(ss);
   const float r = rsqrtf(ss / (float)h + eps);
+  if (lane == 0 && inv_rms) inv_rms[warp] = r;
   for (int c = lane * 8; c < h; c += 256) {
     float v[8], gv[8], o[8];
     if (acc) {
       load8(acc + (long)warp * h + c, v);
 #pragma unroll
       for (int j = 0; j < 8; j++) v[j] = to_f(from_f<T>(v[j]));
-      if (x_store) store8(x_store + (long)warp * h + c, v);
     } else {
       load8(x_in + (long)warp * h + c, v);
     }

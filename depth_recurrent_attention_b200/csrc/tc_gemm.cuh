@@ -1,0 +1,247 @@
+// Persistent grouped GEMM on the 5th-generation tensor cores (tcgen05), bf16 in, fp32
+// accumulated in TMEM:  C[r][n] = sum_k A[row(r)][k] * B_g[n][k]  for the sorted rows r of
+// group g, B_g = rows g*b_group_rows + b_row0 .. of B (K contiguous).
+//
+// Roles (one CTA per SM, tiles of 128 x BN, K-blocks of BK):
+//   warp 0      TMA producer: B tile (and A tile unless rows are gathered) per stage
+//   warp 1      TMEM allocator + single-thread MMA issuer (tcgen05.mma, commit to barriers)
+//   warps 2-5   epilogue: tcgen05.ld of the 128 x BN accumulator, row r per thread, then the
+//               caller's epilogue functor on column segments of SEG values
+//   warps 6-9   (GATHER only) A producers: 16-byte cp.async of gathered rows into the
+//               128B-swizzled layout TMA would have written
+// Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap the MMAs of
+// tile i+1.  Every wait is bounded (tc::mbar_wait); on expiry the CTA winds down and the
+// device error flag is set.
+#pragma once
+#include "tc_common.cuh"
+
+namespace dreamer {
+namespace tc {
+
+struct TcGemmArgs {
+  int N, K, G, M;
+  const int *goffs;   // [G+1] sorted-row offsets or null (single group of M rows)
+  const int *tiles;   // [G+1] cumulative 128-row tiles per group or null
+  const int *arow;    // gathered source row of sorted row r (A row = arow[r] / arow_div)
+  int arow_div;
+  const bf16 *A;      // gather source [*][lda]
+  long lda;
+  int b_group_rows, b_row0;
+  int *err;
+};
+
+__device__ __forceinline__ bool tc_tile_rows(const TcGemmArgs &a, int mt, int &g, int &m0,
+                                             int &m1) {
+  if (!a.goffs) {
+    g = 0;
+    m0 = mt * 128;
+    m1 = min(m0 + 128, a.M);
+    return m0 < m1;
+  }
+  int lo = 0, hi = a.G - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (a.tiles[mid] <= mt) lo = mid; else hi = mid - 1;
+  }
+  g = lo;
+  m0 = a.goffs[g] + (mt - a.tiles[g]) * 128;
+  m1 = min(m0 + 128, a.goffs[g + 1]);
+  return m0 < m1;
+}
+
+template <int BN, int BK, int STAGES, bool GATHER>
+struct TcGemmCfg {
+  static constexpr int A_BYTES = 128 * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int THREADS = GATHER ? 320 : 192;
+  // at least 120 KB so that a second CTA never shares the SM (and its 512 TMEM columns)
+  static constexpr int SMEM_USED = STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*bars*/;
+  static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
+  static_assert(SMEM_USED <= 227 * 1024, "shared memory");
+  static constexpr uint32_t IDESC = idesc_bf16_m128(BN);
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "N tile");
+  static_assert(BK == 16 || BK == 32 || BK == 64, "K block");
+  static_assert(!GATHER || BK == 64, "gathered rows use 128-byte K blocks");
+};
+
+template <int BN, int BK, int STAGES, bool GATHER, int SEG, class Epi>
+__global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   TcGemmArgs a, Epi epi) {
+  using C = TcGemmCfg<BN, BK, STAGES, GATHER>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * C::A_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + STAGES * C::B_BYTES);
+  uint64_t *full = bars, *empty = bars + STAGES, *tfull = bars + 2 * STAGES, *tempty = tfull + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NT = a.N / BN;
+  const int mtiles = a.goffs ? a.tiles[a.G] : (a.M + 127) / 128;
+  const int total = mtiles * NT;
+  const int KB = a.K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; s++) {
+      mbar_init(smem_u32(&full[s]), GATHER ? 1 + 128 : 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int i = 0; i < 2; i++) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmB);
+    if (!GATHER) prefetch_tmap(&tmA);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int issued_ph[STAGES];
+      for (int i = 0; i < STAGES; i++) issued_ph[i] = -1;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        int g, m0, m1;
+        const int mt = t / NT, n0 = (t % NT) * BN;
+        tc_tile_rows(a, mt, g, m0, m1);
+        const int brow = g * a.b_group_rows + a.b_row0 + n0;
+        for (int kb = 0; kb < KB; kb++) {
+          if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag, a.err)) { ok = false; break; }
+          const uint32_t fb = smem_u32(&full[s]);
+          mbar_expect_tx(fb, GATHER ? C::B_BYTES : C::A_BYTES + C::B_BYTES);
+          if (!GATHER) tma_load_2d(smem_u32(sA + s * C::A_BYTES), &tmA, fb, kb * BK, m0);
+          tma_load_2d(smem_u32(sB + s * C::B_BYTES), &tmB, fb, kb * BK, brow);
+          issued_ph[s] = (int)ph;
+          if (++s == STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+      if (!ok) {  // let copies already in flight land before the CTA exits
+        for (int i = 0; i < STAGES; i++)
+          if (issued_ph[i] >= 0) {
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(smem_u32(&full[i]), (uint32_t)issued_ph[i]) &&
+                   globaltimer() - t0 < WAIT_LIMIT_NS) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, it++) {
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait(smem_u32(&tempty[acc]), aph ^ 1, abort_flag, a.err)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + acc * BN;
+        for (int kb = 0; kb < KB; kb++) {
+          if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag, a.err)) { ok = false; break; }
+          tc_fence_after();
+          if (GATHER) fence_proxy_async();
+          const uint32_t a0 = smem_u32(sA + s * C::A_BYTES), b0 = smem_u32(sB + s * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; k++)
+            mma_bf16(d, smem_desc(a0 + k * 32, BK * 2), smem_desc(b0 + k * 32, BK * 2), C::IDESC,
+                     (kb | k) != 0);
+          mma_commit(smem_u32(&empty[s]));
+          if (++s == STAGES) { s = 0; ph ^= 1; }
+        }
+        if (ok) mma_commit(smem_u32(&tfull[acc]));
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    int it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, it++) {
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      if (!mbar_wait(smem_u32(&tfull[acc]), aph, abort_flag, a.err)) break;
+      tc_fence_after();
+      int g, m0, m1;
+      const int mt = t / NT, n0 = (t % NT) * BN;
+      tc_tile_rows(a, mt, g, m0, m1);
+      const int r = m0 + row;
+      const bool valid = r < m1;
+      const int token = valid ? (a.arow ? a.arow[r] / a.arow_div : r) : 0;
+      const uint32_t base = tmem + acc * BN + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+      for (int sg = 0; sg < BN / SEG; sg++) {
+        float v[SEG];
+        if (SEG >= 32) {
+#pragma unroll
+          for (int c = 0; c < SEG; c += 32) tmem_ld32(base + sg * SEG + c, v + c);
+        } else {
+          tmem_ld16(base + sg * SEG, v);
+        }
+        if (valid) epi.template operator()<SEG>(r, token, g, n0 + sg * SEG, v);
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&tempty[acc]));
+    }
+  } else if (GATHER) {
+    // ------------------------------------------------------------- gathered A producers
+    const int tid = threadIdx.x - 192;  // 0..127
+    const int c = tid & 7;              // 16-byte chunk of the 128-byte row slice
+    const int rsub = tid >> 3;          // 0..15
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      int g, m0, m1;
+      const int mt = t / NT;
+      tc_tile_rows(a, mt, g, m0, m1);
+      const bf16 *src[8];
+      uint32_t bytes[8];
+#pragma unroll
+      for (int p = 0; p < 8; p++) {
+        const int rr = p * 16 + rsub, r = m0 + rr;
+        const bool v = r < m1;
+        src[p] = a.A + (v ? (long)(a.arow[r] / a.arow_div) * a.lda : 0) + c * 8;
+        bytes[p] = v ? 16u : 0u;
+      }
+      for (int kb = 0; kb < KB; kb++) {
+        if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag, a.err)) { ok = false; break; }
+        const uint32_t dst0 = smem_u32(sA + s * C::A_BYTES);
+#pragma unroll
+        for (int p = 0; p < 8; p++) {
+          const int rr = p * 16 + rsub;
+          cp_async16(dst0 + rr * 128 + ((c ^ (rr & 7)) << 4), src[p] + kb * 64, bytes[p]);
+        }
+        cp_async_arrive(smem_u32(&full[s]));
+        if (++s == STAGES) { s = 0; ph ^= 1; }
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace tc
+}  // namespace dreamer

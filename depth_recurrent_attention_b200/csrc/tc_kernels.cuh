@@ -1,19 +1,302 @@
-// tcgen05 / TMA kernels (bf16 contractions).  Included after the handle definition.
+// Host side of the tcgen05 path: tensor maps, launch shapes and the bf16 contraction steps
+// of the depth step (QKV / O projections, router scores, expert FFNs).  Included by
+// dreamer.cu after the handle definition.
 #pragma once
+#include <cuda.h>
 
-static int tc_init(dreamer_handle *h) { return 0; }
+#include "tc_attn.cuh"
+#include "tc_gemm.cuh"
+
+namespace dreamer {
+
+// Router query epilogue (papernotes "Key design 2", reading R8): the thread holds the full
+// fp32 row q = y W_qE.  z_e = q . (R_l k_e) = (R_l^T q) . k_e, so the query is turned back by
+// the depth rotation of depth l (k_e then enters the contraction exactly as stored, bf16) and
+// split into three bf16 parts hi + mid + lo that carry q to float32 precision; the score
+// contraction against [k | k | k] then runs on the tensor cores with fp32 accumulation.
+struct EpiRouterQ {
+  int dr;
+  const float2 *rope;  // depth-RoPE table row of depth l over d_r dims
+  bf16 *qs;            // [n][3 d_r]
+  template <int SEG>
+  __device__ __forceinline__ void operator()(int r, int token, int g, int n0, float *v) const {
+    const int q4 = SEG / 4;
+#pragma unroll
+    for (int half = 0; half < 2; half++) {
+#pragma unroll
+      for (int i = 0; i < q4; i++) {
+        const float c = rope[half * q4 + i].x, s = rope[half * q4 + i].y;
+        const float a = v[half * (SEG / 2) + i], b = v[half * (SEG / 2) + i + q4];
+        v[half * (SEG / 2) + i] = a * c + b * s;
+        v[half * (SEG / 2) + i + q4] = b * c - a * s;
+      }
+    }
+    bf16 *row = qs + (long)r * 3 * SEG;
+#pragma unroll
+    for (int i = 0; i < SEG; i += 8) {
+      float hi[8], mid[8], lo[8];
+#pragma unroll
+      for (int j = 0; j < 8; j++) {
+        hi[j] = __bfloat162float(__float2bfloat16_rn(v[i + j]));
+        const float r1 = v[i + j] - hi[j];
+        mid[j] = __bfloat162float(__float2bfloat16_rn(r1));
+        lo[j] = r1 - mid[j];
+      }
+      store8(row + i, hi);
+      store8(row + SEG + i, mid);
+      store8(row + 2 * SEG + i, lo);
+    }
+  }
+};
+
+// Expert down-projection epilogue with 16-byte vector reductions: acc[token] += w (H W2_e).
+struct EpiDownVec {
+  int h, k;
+  const int *rows;
+  const float *wts;
+  float *acc;
+  template <int SEG>
+  __device__ __forceinline__ void operator()(int r, int token, int g, int n0, float *v) const {
+    const int slot = rows[r];
+    const float w = wts[slot];
+    float *dst = acc + (long)(slot / k) * h + n0;
+#pragma unroll
+    for (int i = 0; i < SEG; i += 4)
+      asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + i),
+                   "f"(w * v[i]), "f"(w * v[i + 1]), "f"(w * v[i + 2]), "f"(w * v[i + 3])
+                   : "memory");
+  }
+};
+
+}  // namespace dreamer
+
+typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                      const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                      const cuuint32_t *, CUtensorMapInterleave,
+                                      CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                      CUtensorMapFloatOOBfill);
+static PFN_encodeTiled_t g_encode_tiled = nullptr;
+
+// 2-D bf16 tensor map: `rows` rows of `inner` elements at `pitch_bytes`, box box_inner x
+// box_rows, swizzle = box_inner * 2 bytes (32, 64 or 128).
+static bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows,
+                      uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_rows) {
+  if (!g_encode_tiled || ((uintptr_t)base & 15) || (pitch_bytes & 15) || rows == 0) return false;
+  const uint32_t sw_bytes = box_inner * 2;
+  CUtensorMapSwizzle sw = sw_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : sw_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                          : sw_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                           : CU_TENSOR_MAP_SWIZZLE_NONE;
+  if (sw == CU_TENSOR_MAP_SWIZZLE_NONE) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base),
+                              dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static int tc_init(dreamer_handle *h) {
+  const dreamer_config &c = h->cfg;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (!g_encode_tiled) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode_tiled = (PFN_encodeTiled_t)fn;
+  }
+  if (c.dtype == 1) {
+    // [E][3 d_r] = [k | k | k] for the split-precision score contraction
+    const int E = c.n_experts, dr = c.router_dim;
+    if (dalloc(h, &h->k3, (size_t)E * 3 * dr * 2)) return DREAMER_ERR_OOM;
+    for (int i = 0; i < 3; i++)
+      if (cudaMemcpy2D((char *)h->k3 + i * dr * 2, 3 * dr * 2, h->kE_raw, dr * 2, dr * 2, E,
+                       cudaMemcpyDeviceToDevice) != cudaSuccess)
+        return DREAMER_ERR_CUDA;
+  }
+  return tc_attn_init(h);
+}
+
 static void tc_destroy(dreamer_handle *h) {}
-static bool tc_route_ok(dreamer_handle *h) { return false; }
-static void tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, float *w,
-                     int *counts_a, int *counts_b, cudaStream_t s) {}
-static bool tc_gemm_ok(dreamer_handle *h, const dreamer::GemmArgs &a) { return false; }
+
+template <int BN, int BK, int ST, bool GATHER, int SEG, class Epi>
+static void tc_launch(dreamer_handle *h, const dreamer::tc::TcGemmArgs &a, const CUtensorMap &ta,
+                      const CUtensorMap &tb, long max_tiles, const Epi &epi, cudaStream_t s) {
+  using Cfg = dreamer::tc::TcGemmCfg<BN, BK, ST, GATHER>;
+  auto kern = dreamer::tc::tc_gemm_kernel<BN, BK, ST, GATHER, SEG, Epi>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    attr_set = true;
+  }
+  long grid = max_tiles < h->num_sms ? max_tiles : h->num_sms;
+  if (grid < 1) grid = 1;
+  kern<<<(int)grid, Cfg::THREADS, Cfg::SMEM, s>>>(ta, tb, a, epi);
+}
+
+// Build engine arguments and tensor maps from the generic GEMM description.  B rows of group
+// g start at g * (bgstride / ldb); A is TMA-loaded unless rows are gathered.
+template <int BN, int BK>
+static bool tc_prepare(dreamer_handle *h, const dreamer::GemmArgs &a, const int *tiles,
+                       long a_rows, dreamer::tc::TcGemmArgs &t, CUtensorMap &ta, CUtensorMap &tb,
+                       long &max_tiles) {
+  if (a.N % BN || a.K % BK) return false;
+  const bool gather = a.arow != nullptr;
+  const long bgr = a.G > 1 ? a.bgstride / a.ldb : 0;
+  if (!make_tmap(&tb, a.B, a.K, (uint64_t)((a.G - 1) * bgr + a.N), a.ldb * 2, BK, BN)) return false;
+  if (!gather) {
+    if (!make_tmap(&ta, a.A, a.K, (uint64_t)a_rows, a.lda * 2, BK, 128)) return false;
+  } else {
+    ta = tb;  // unused
+    if (((uintptr_t)a.A & 15) || (a.lda * 2) % 16) return false;
+  }
+  t.N = a.N; t.K = a.K; t.G = a.G; t.M = a.M;
+  t.goffs = a.goffs; t.tiles = a.goffs ? tiles : nullptr;
+  t.arow = a.arow; t.arow_div = a.arow_div;
+  t.A = (const dreamer::bf16 *)a.A; t.lda = a.lda;
+  t.b_group_rows = (int)bgr; t.b_row0 = 0;
+  t.err = h->err;
+  max_tiles = ((a.M + 127) / 128 + (a.goffs ? a.G : 0)) * (long)(a.N / BN);
+  return true;
+}
+
+static bool tc_gemm_ok(dreamer_handle *h, const dreamer::GemmArgs &a) {
+  if (!g_encode_tiled) return false;
+  const int d = h->cfg.head_dim;
+  return a.N % 256 == 0 && a.K % 64 == 0 && (d == 64 || d == 128);
+}
+
 template <typename T>
-static void tc_gemm_qkv(dreamer_handle *h, const dreamer::GemmArgs &a,
-                        const dreamer::EpiQKV<T> &e, cudaStream_t s) {}
+static bool tc_gemm_qkv(dreamer_handle *h, const dreamer::GemmArgs &a, const dreamer::EpiQKV<T> &e,
+                        cudaStream_t s) {
+  if constexpr (sizeof(T) == 2) {
+    dreamer::tc::TcGemmArgs t{};
+    CUtensorMap ta, tb;
+    long mt;
+    const int *tiles = h->ptiles_b;
+    if (!tc_prepare<256, 64>(h, a, tiles, a.M, t, ta, tb, mt)) return false;
+    const bool gather = a.arow != nullptr;
+    if (h->cfg.head_dim == 64) {
+      if (gather) tc_launch<256, 64, 4, true, 64>(h, t, ta, tb, mt, e, s);
+      else tc_launch<256, 64, 4, false, 64>(h, t, ta, tb, mt, e, s);
+    } else {
+      if (gather) tc_launch<256, 64, 4, true, 128>(h, t, ta, tb, mt, e, s);
+      else tc_launch<256, 64, 4, false, 128>(h, t, ta, tb, mt, e, s);
+    }
+    return true;
+  }
+  return false;
+}
+
 template <typename T>
-static void tc_gemm_o(dreamer_handle *h, const dreamer::GemmArgs &a, const dreamer::EpiO<T> &e,
-                      cudaStream_t s) {}
-static bool tc_sa_ok(dreamer_handle *h) { return false; }
-static void tc_sa(dreamer_handle *h, cudaStream_t s) {}
-static bool tc_expert_ok(dreamer_handle *h) { return false; }
-static void tc_expert(dreamer_handle *h, const void *X, int n, cudaStream_t s) {}
+static bool tc_gemm_o(dreamer_handle *h, const dreamer::GemmArgs &a, const dreamer::EpiO<T> &e,
+                      cudaStream_t s) {
+  if constexpr (sizeof(T) == 2) {
+    dreamer::tc::TcGemmArgs t{};
+    CUtensorMap ta, tb;
+    long mt;
+    if (!tc_prepare<256, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
+    if (a.arow) tc_launch<256, 64, 4, true, 32>(h, t, ta, tb, mt, e, s);
+    else tc_launch<256, 64, 4, false, 32>(h, t, ta, tb, mt, e, s);
+    return true;
+  }
+  return false;
+}
+
+static bool tc_route_ok(dreamer_handle *h) {
+  const dreamer_config &c = h->cfg;
+  return g_encode_tiled && h->k3 && c.n_experts % 256 == 0 &&
+         (c.router_dim == 64 || c.router_dim == 128) && c.hidden % 64 == 0;
+}
+
+static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, float *w,
+                     int *counts_a, int *counts_b, cudaStream_t s) {
+  using namespace dreamer;
+  const dreamer_config &c = h->cfg;
+  const int dr = c.router_dim, hd = c.hidden, E = c.n_experts;
+  // q = X W_qE, turned back by the depth rotation and split into hi/mid/lo bf16
+  GemmArgs qa{};
+  qa.N = dr; qa.K = hd; qa.G = 1; qa.M = n; qa.arow_div = 1;
+  qa.A = X; qa.lda = hd; qa.B = h->wqE_t; qa.ldb = hd; qa.bgstride = 0;
+  tc::TcGemmArgs t{}, t2{};
+  CUtensorMap ta, tb, ta2, tb2;
+  long mt, mt2;
+  EpiRouterQ eq{dr, h->rope_dr + (size_t)l * (dr / 2), (bf16 *)h->qsplit};
+  // z = [q_hi | q_mid | q_lo] . [k | k | k]
+  GemmArgs za{};
+  za.N = E; za.K = 3 * dr; za.G = 1; za.M = n; za.arow_div = 1;
+  za.A = h->qsplit; za.lda = 3 * dr; za.B = h->k3; za.ldb = 3 * dr; za.bgstride = 0;
+  if (!tc_prepare<256, 64>(h, za, nullptr, n, t2, ta2, tb2, mt2)) return false;
+  if (dr == 64) {
+    if (!tc_prepare<64, 64>(h, qa, nullptr, n, t, ta, tb, mt)) return false;
+    tc_launch<64, 64, 6, false, 64>(h, t, ta, tb, mt, eq, s);
+  } else {
+    if (!tc_prepare<128, 64>(h, qa, nullptr, n, t, ta, tb, mt)) return false;
+    tc_launch<128, 64, 6, false, 128>(h, t, ta, tb, mt, eq, s);
+  }
+  tc_launch<256, 64, 4, false, 32>(h, t2, ta2, tb2, mt2, EpiStoreF32{h->zbuf, h->ldz, E}, s);
+  TopkArgs k{};
+  k.n_tok = n; k.E = E; k.k = c.top_k; k.mode = 0;
+  k.z = h->zbuf; k.ldz = h->ldz; k.zscale = 1.0f / sqrtf((float)dr);
+  k.bias = h->bias; k.idx = idx; k.w = w; k.counts_a = counts_a; k.counts_b = counts_b;
+  topk_kernel<<<(n + 7) / 8, 256, 0, s>>>(k);
+  return true;
+}
+
+static bool tc_expert_ok(dreamer_handle *h) {
+  const dreamer_config &c = h->cfg;
+  const int m = c.expert_hidden;
+  return g_encode_tiled && (m == 16 || m == 32 || m == 64) && c.hidden % 256 == 0;
+}
+
+static bool tc_expert(dreamer_handle *h, const void *X, int n, cudaStream_t s) {
+  using namespace dreamer;
+  const dreamer_config &c = h->cfg;
+  const int hd = c.hidden, m = c.expert_hidden, k = c.top_k, E = c.n_experts;
+  const long rows = (long)n * k;
+  // up: H = SiLU(X_gathered W1_e)
+  GemmArgs up{};
+  up.N = m; up.K = hd; up.G = E; up.M = (int)rows; up.goffs = h->eoffs; up.tile_offs = h->etiles_b;
+  up.arow = h->erows; up.arow_div = k; up.A = X; up.lda = hd; up.B = h->w1_t; up.ldb = hd;
+  up.bgstride = (long)m * hd;
+  // down: acc[token] += w * H W2_e
+  GemmArgs dn{};
+  dn.N = hd; dn.K = m; dn.G = E; dn.M = (int)rows; dn.goffs = h->eoffs; dn.tile_offs = h->etiles_b;
+  dn.arow = nullptr; dn.arow_div = 1; dn.A = h->Hbuf; dn.lda = m; dn.B = h->w2_t; dn.ldb = m;
+  dn.bgstride = (long)m * hd;
+  tc::TcGemmArgs tu{}, td{};
+  CUtensorMap tau, tbu, tad, tbd;
+  long mtu, mtd;
+  EpiUp<bf16> eu{m, (bf16 *)h->Hbuf};
+  EpiDownVec ed{hd, k, h->erows, h->ew, h->acc};
+  switch (m) {
+    case 16:
+      if (!tc_prepare<16, 64>(h, up, h->etiles_b, rows, tu, tau, tbu, mtu) ||
+          !tc_prepare<256, 16>(h, dn, h->etiles_b, rows + 128, td, tad, tbd, mtd))
+        return false;
+      tc_launch<16, 64, 8, true, 16>(h, tu, tau, tbu, mtu, eu, s);
+      tc_launch<256, 16, 8, false, 32>(h, td, tad, tbd, mtd, ed, s);
+      return true;
+    case 32:
+      if (!tc_prepare<32, 64>(h, up, h->etiles_b, rows, tu, tau, tbu, mtu) ||
+          !tc_prepare<256, 32>(h, dn, h->etiles_b, rows + 128, td, tad, tbd, mtd))
+        return false;
+      tc_launch<32, 64, 8, true, 16>(h, tu, tau, tbu, mtu, eu, s);
+      tc_launch<256, 32, 6, false, 32>(h, td, tad, tbd, mtd, ed, s);
+      return true;
+    default:
+      if (!tc_prepare<64, 64>(h, up, h->etiles_b, rows, tu, tau, tbu, mtu) ||
+          !tc_prepare<256, 64>(h, dn, h->etiles_b, rows + 128, td, tad, tbd, mtd))
+        return false;
+      tc_launch<64, 64, 8, true, 16>(h, tu, tau, tbu, mtu, eu, s);
+      tc_launch<256, 64, 4, false, 32>(h, td, tad, tbd, mtd, ed, s);
+      return true;
+  }
+}

@@ -89,7 +89,8 @@ typedef struct {
  * call runs are written.                                                                  */
 typedef struct {
   void *xhat;      /* [L][T][h] dtype: RMSNorm output                                      */
-  void *y;         /* [L][T][h] dtype: input of expert attention                            */
+  void *y;         /* [L][T][h] dtype: y_l = x^_l + DA + SA, the state entering expert
+                      attention (the fully parallel layout routes x^_l instead)             */
   int32_t *idx;    /* [L][T][k]: selected experts                                          */
   float *w;        /* [L][T][k]: routing weights                                           */
   void *sa_k;      /* [L][T][h] dtype: post-RoPE SA keys (forward only)                    */

@@ -116,6 +116,10 @@ def step_inputs(cfg, l):
     return x, hist
 
 
+def router_input(cfg, tr, l):
+    return PY.to_np(tr["xhat"][l] if cfg.variant == 2 else tr["y"][l])
+
+
 def run_step_and_compare(cfg, W, dev, l, toks=None, orc=None):
     torch = _torch()
     x, hist = step_inputs(cfg, l)
@@ -125,11 +129,13 @@ def run_step_and_compare(cfg, W, dev, l, toks=None, orc=None):
     out = dev.forward(xd, depth_begin=l, depth_end=l + 1, da_kv=hd, trace=tr)
     torch.cuda.synchronize()
     g_x, g_y = PY.to_np(out), PY.to_np(tr["y"][l])
+    g_ein = router_input(cfg, tr, l)
     g_idx = tr["idx"][l].cpu().numpy()
     o = orc or O.Oracle(cfg, W)
     if toks is None:
         r = o.forward(x, l, l + 1, da_kv=hist.astype(np.float64))
         rx, ry, ridx, rmg = r["x_out"], r["y"][l], r["idx"][l], r["margin"][l]
+        rein = r["xhat"][l] if cfg.variant == 2 else ry
         sel = slice(None)
         g_da = PY.to_np(hd[:, l])
         assert np.allclose(g_da, r["da_kv"][:, l], atol=PY.TOL_BF16_ABS * 2)
@@ -139,10 +145,11 @@ def run_step_and_compare(cfg, W, dev, l, toks=None, orc=None):
         tk = seq * S + np.asarray(pos)
         r = o.step_tokens(l, x[seq * S:(seq + 1) * S], hist[tk].astype(np.float64), pos)
         rx, ry, ridx, rmg = r["x_out"], r["y"], r["idx"], r["margin"]
+        rein = r["xhat"] if cfg.variant == 2 else ry
         sel = tk
     bf = cfg.dtype == "bf16"
     PY.check_hidden(g_y[sel], ry, bf, f"y depth {l}")
-    same, flips = PY.check_routing(cfg, W, l, g_idx[sel], ridx, rmg, g_y[sel], ry)
+    same, flips = PY.check_routing(cfg, W, l, g_idx[sel], ridx, rmg, g_ein[sel], rein)
     PY.check_hidden(g_x[sel][same], rx[same], bf, f"x depth {l}")
     return flips, int(np.size(same))
 
@@ -158,6 +165,15 @@ def test_small_every_depth_bf16(cuda):
         print(f"small depth {l}: {flips}/{n} routing flips explained by bf16 rounding of y")
         assert flips <= 0.05 * n
         tot += flips
+
+
+def test_small_linear_moe_step_bf16(cuda):
+    """Top-1 linear-MoE QKV/O with 8 projection experts (grouped GEMMs over p*)."""
+    cfg = configs.SMALL.with_(n_proj_experts=8, depth=4)
+    W = inputs.host_weights(cfg)
+    dev = make_handle(cfg, W)
+    for l in (0, 3):
+        run_step_and_compare(cfg, W, dev, l)
 
 
 @pytest.mark.parametrize("variant", [1, 2])
@@ -199,6 +215,34 @@ def test_small_free_running_drift_reported(cuda):
 
 
 # ---------------------------------------------------------------------------------------
+# bf16 through every depth, free-running, where no routing decision can flip
+
+@pytest.mark.parametrize("kw", [dict(n_experts=4, top_k=4, depth=4),
+                                dict(n_experts=8, top_k=8, depth=3, n_proj_experts=1),
+                                dict(n_experts=4, top_k=4, depth=3, variant=1),
+                                dict(n_experts=4, top_k=4, depth=3, variant=2)])
+def test_small_flip_free_all_depths_bf16(cuda, kw):
+    torch = _torch()
+    cfg = configs.SMALL.with_(**kw)
+    W = inputs.host_weights(cfg)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    ref = O.Oracle(cfg, W).forward(x0)
+    dev = make_handle(cfg, W)
+    tr = trace_buffers(cfg, cfg.tokens)
+    out = dev.forward(inputs.to_device(x0, "bf16"), trace=tr)
+    torch.cuda.synchronize()
+    for l in range(cfg.depth):
+        PY.check_hidden(PY.to_np(tr["y"][l]), ref["y"][l], True, f"y depth {l}")
+        assert np.allclose(PY.to_np(tr["w"][l])[np.arange(cfg.tokens)[:, None],
+                                               np.argsort(tr["idx"][l].cpu().numpy(), 1)],
+                           ref["w"][l][np.arange(cfg.tokens)[:, None],
+                                       np.argsort(ref["idx"][l], 1)], atol=5e-3)
+    e, rl = PY.check_hidden(PY.to_np(out), ref["x_out"], True, "x_L")
+    print(f"flip-free {kw}: x_L max-abs {e:.3g} rel-L2 {rl:.3g}")
+    assert np.array_equal(dev.route_counts().numpy(), ref["counts"])
+
+
+# ---------------------------------------------------------------------------------------
 # decode
 
 def decode_case(cfg, lens):
@@ -210,10 +254,21 @@ def decode_case(cfg, lens):
     return x, kc, vc, np.asarray(lens, np.int32)
 
 
-@pytest.mark.parametrize("base,lens", [("tiny", [12, 5, 0]), ("small", [300, 1, 77, 299])])
-def test_decode_step(cuda, base, lens):
+def flip_free(cfg):
+    """E = k and P <= 1: no routing decision can flip, so bf16 runs stay comparable with the
+    oracle through every depth."""
+    return cfg.n_experts == cfg.top_k and cfg.n_proj_experts <= 1
+
+
+@pytest.mark.parametrize("base,lens,kw", [
+    ("tiny", [12, 5, 0], {}),
+    ("small", [300, 1, 77, 299], {}),
+    ("small", [300, 1, 77, 299], dict(n_experts=4, top_k=4, depth=4)),
+    ("small", [40, 0, 17], dict(n_experts=4, top_k=4, depth=3, n_proj_experts=1)),
+])
+def test_decode_step(cuda, base, lens, kw):
     torch = _torch()
-    cfg = configs.CONFIGS[base].with_(batch=len(lens), seq=1, cache_len=max(lens) + 1)
+    cfg = configs.CONFIGS[base].with_(batch=len(lens), seq=1, cache_len=max(lens) + 1, **kw)
     W = inputs.host_weights(cfg)
     x, kc, vc, ln = decode_case(cfg, lens)
     dev = make_handle(cfg, W)
@@ -230,16 +285,19 @@ def test_decode_step(cuda, base, lens):
         kcb = kc[:, b].astype(np.float64).copy()
         vcb = vc[:, b].astype(np.float64).copy()
         r = o.decode_seq(x[b], kcb, vcb, int(ln[b]))
-        # the new token's key/value went to slot cache_len of every depth
-        PY.check_hidden(kd_np[:, b, :, ln[b]], kcb[:, :, ln[b]], bf, f"k slot seq {b}")
-        PY.check_hidden(vd_np[:, b, :, ln[b]], vcb[:, :, ln[b]], bf, f"v slot seq {b}")
-        if not bf:
+        # the new token's key/value went to slot cache_len of every depth (bf16 with real
+        # routing: depth 0 only, later depths drift through routing flips)
+        dl = slice(None) if (not bf or flip_free(cfg)) else slice(0, 1)
+        PY.check_hidden(kd_np[dl, b, :, ln[b]], kcb[dl, :, ln[b]], bf, f"k slot seq {b}")
+        PY.check_hidden(vd_np[dl, b, :, ln[b]], vcb[dl, :, ln[b]], bf, f"v slot seq {b}")
+        if not bf or flip_free(cfg):
             for l in range(cfg.depth):
                 same, flips = PY.check_routing(cfg, W, l, tr["idx"][l, b:b + 1].cpu().numpy(),
                                                r["idx"][l:l + 1], r["margin"][l:l + 1],
                                                strict=True)
                 assert flips == 0
-            PY.check_hidden(g[b], r["x_out"], False, f"x_out seq {b}")
+                PY.check_hidden(PY.to_np(tr["y"][l, b]), r["y"][l], bf, f"y depth {l} seq {b}")
+            PY.check_hidden(g[b], r["x_out"], bf, f"x_out seq {b}")
         else:
             # first depth is comparable token by token; later depths drift by routing flips
             gy = PY.to_np(tr["y"][0, b])
