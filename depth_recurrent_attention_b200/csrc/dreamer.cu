@@ -465,14 +465,14 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
     launch_attn<T>(da, d, s);
     o_gemm((const T *)h->attn + hd, hd, hd, res_xhat, h->u);   // u = x^ + DA part (acc = u)
     qkv_gemm(h->u, 0, 3 * hd);
-    if (io.mode == 0 && tc && tc_sa_ok(h)) tc_sa(h, s); else launch_attn<T>(sa, d, s);
+    if (!(io.mode == 0 && tc && tc_sa_ok(h) && tc_sa(h, s))) launch_attn<T>(sa, d, s);
     o_gemm(h->attn, 0, hd, 2, h->y);                            // y = u + SA part
   } else {
     // 3. fused QKV projection with RoPE / depth RoPE epilogue, DA KV write
     qkv_gemm(h->xh, 0, 6 * hd);
     // 4. DA || SA (papernotes "Key design 1": run in parallel for throughput)
     launch_attn<T>(da, d, s);
-    if (io.mode == 0 && tc && tc_sa_ok(h)) tc_sa(h, s); else launch_attn<T>(sa, d, s);
+    if (!(io.mode == 0 && tc && tc_sa_ok(h) && tc_sa(h, s))) launch_attn<T>(sa, d, s);
     // 5. O projection, residual y = x^ + DA + SA
     o_gemm(h->attn, 0, 2 * hd, res_xhat, h->y);
   }

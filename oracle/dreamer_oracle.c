@@ -34,6 +34,7 @@
 #include "dreamer_oracle.h"
 
 #include <math.h>
+#include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 #ifdef _OPENMP
@@ -49,6 +50,18 @@ void orc_set_threads(int n) {
 }
 
 static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/* Round to bfloat16 (nearest even, through float32): the precision in which the bf16 path
+ * stores the states its routers read.  Where a float decides an integer (an argmax, a
+ * top-k) both sides take the decision on the same stored input.                         */
+static double round_bf16(double v) {
+  float f = (float)v;
+  uint32_t b;
+  memcpy(&b, &f, 4);
+  b = (b + 0x7FFFu + ((b >> 16) & 1u)) & 0xFFFF0000u;
+  memcpy(&f, &b, 4);
+  return (double)f;
+}
 
 static void *xcalloc(size_t n, size_t sz) {
   void *p = calloc(n ? n : 1, sz);
@@ -243,8 +256,10 @@ static void proj_route(const orc_cfg *c, const orc_weights *W, const double *kro
   double q[1024];
   double z[256] = {0.0};
   for (int j = 0; j < dr; j++) q[j] = 0.0;
-  for (int i = 0; i < c->h; i++)
-    for (int j = 0; j < dr; j++) q[j] += xh[i] * (double)W->w_qP[(long)i * dr + j];
+  for (int i = 0; i < c->h; i++) {
+    const double xi = c->route_bf16 ? round_bf16(xh[i]) : xh[i];
+    for (int j = 0; j < dr; j++) q[j] += xi * (double)W->w_qP[(long)i * dr + j];
+  }
   for (int p = 0; p < P; p++) {
     double s = 0.0;
     for (int j = 0; j < dr; j++) s += q[j] * krotP[(long)p * dr + j];
@@ -267,8 +282,10 @@ static void ea_scores(const orc_cfg *c, const orc_weights *W, const double *krot
   int dr = c->dr;
   double q[1024];
   for (int j = 0; j < dr; j++) q[j] = 0.0;
-  for (int i = 0; i < c->h; i++)
-    for (int j = 0; j < dr; j++) q[j] += x[i] * (double)W->w_qE[(long)i * dr + j];
+  for (int i = 0; i < c->h; i++) {
+    const double xi = c->route_bf16 ? round_bf16(x[i]) : x[i];
+    for (int j = 0; j < dr; j++) q[j] += xi * (double)W->w_qE[(long)i * dr + j];
+  }
   for (int e = 0; e < c->E; e++) {
     double s = 0.0;
     for (int j = 0; j < dr; j++) s += q[j] * krotE[(long)e * dr + j];

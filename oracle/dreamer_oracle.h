@@ -36,6 +36,8 @@ typedef struct {
   int P;           /* projection experts (0 = dense QKV/O)                            */
   double rope_base, eps;
   int variant;     /* block layout: 0 DA||SA then EA; 1 serial DA->SA->EA; 2 all parallel */
+  int route_bf16;  /* 1: routing decisions read their input rounded to bf16, the precision
+                      the bf16 kernels store it in (the decision itself stays float64)     */
 } orc_cfg;
 
 typedef struct {

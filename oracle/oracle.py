@@ -25,7 +25,8 @@ i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
 
 class OrcCfg(C.Structure):
     _fields_ = [(n, C.c_int) for n in ("B", "S", "h", "H", "d", "L", "E", "k", "m", "dr", "P")] + \
-               [("rope_base", C.c_double), ("eps", C.c_double), ("variant", C.c_int)]
+               [("rope_base", C.c_double), ("eps", C.c_double), ("variant", C.c_int),
+                ("route_bf16", C.c_int)]
 
 
 _WNAMES = ("g", "w_qkv", "w_qkv_sh", "w_o", "w_o_sh", "w_qP", "k_P", "w_qE", "k_E", "bias",
@@ -84,12 +85,16 @@ class Oracle:
     """The oracle bound to one configuration and one weight set (float32 arrays holding
     exact bf16/fp32 values)."""
 
-    def __init__(self, cfg, weights: dict, threads: int | None = None):
+    def __init__(self, cfg, weights: dict, threads: int | None = None,
+                 route_bf16: bool | None = None):
+        """route_bf16 (default: the config is bf16) makes routing decisions read their input
+        rounded to bf16, as the bf16 kernels store it."""
         self.cfg = cfg
+        rb = (cfg.dtype == "bf16") if route_bf16 is None else route_bf16
         self.c = OrcCfg(cfg.batch, cfg.seq, cfg.hidden, cfg.n_heads, cfg.head_dim, cfg.depth,
                         cfg.n_experts, cfg.top_k, cfg.expert_hidden, cfg.router_dim,
                         cfg.n_proj_experts, float(cfg.rope_base), float(cfg.rms_eps),
-                        int(cfg.variant))
+                        int(cfg.variant), int(rb))
         self._keep = {}
         ptrs = {}
         alias = {"w_qkv_sh": "w_qkv_shared", "w_o_sh": "w_o_shared"}

@@ -137,8 +137,14 @@ def run_step_and_compare(cfg, W, dev, l, toks=None, orc=None):
         rx, ry, ridx, rmg = r["x_out"], r["y"][l], r["idx"][l], r["margin"][l]
         rein = r["xhat"][l] if cfg.variant == 2 else ry
         sel = slice(None)
+        if cfg.n_proj_experts > 0:
+            # projection argmax: same decision except at near ties (both read bf16 x^)
+            gp = tr["pidx"][l].cpu().numpy()
+            pm = gp == r["pidx"][l]
+            assert np.all(pm | (r["pmargin"][l] <= 1e-3)), "projection routing mismatch"
+            assert pm.all(), f"{int((~pm).sum())} projection near-tie flips"
         g_da = PY.to_np(hd[:, l])
-        assert np.allclose(g_da, r["da_kv"][:, l], atol=PY.TOL_BF16_ABS * 2)
+        PY.check_hidden(g_da, r["da_kv"][:, l], cfg.dtype == "bf16", f"DA kv depth {l}")
     else:
         seq, pos = toks
         S = cfg.seq

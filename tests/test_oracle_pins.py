@@ -446,3 +446,16 @@ def test_route_entry_matches_forward_trace():
     # routing from the float32-rounded y picks the same experts except at near ties
     same = np.all(np.sort(r["idx"], 1) == np.sort(full["idx"][1], 1), axis=1)
     assert np.all(same | (full["margin"][1] < 1e-5))
+
+
+def test_route_on_bf16_input_changes_only_near_ties():
+    """Taking the routing decision on the bf16-rounded state moves a selection only where
+    the float64 margin is below the effect of that rounding."""
+    cfg = configs.SMALL.with_(batch=1, seq=64, depth=2)
+    W = inputs.host_weights(cfg)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    a = O.Oracle(cfg, W, threads=2, route_bf16=False).forward(x0, 0, 1)
+    b = O.Oracle(cfg, W, threads=2, route_bf16=True).forward(x0, 0, 1)
+    assert np.array_equal(a["y"], b["y"])                      # states are untouched
+    same = np.all(np.sort(a["idx"][0], 1) == np.sort(b["idx"][0], 1), axis=1)
+    assert np.all(same | (a["margin"][0] < 0.05))
