@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""Throughput of the Dreamer depth-recurrent core forward on B200.
+
+Metric: token-depth-steps per second (one unit = one token through one depth step) of the
+full L-depth forward, bf16, and its fraction of the roofline
+T_roof = max(F_alg / tensor peak, B_alg / HBM peak) with both peaks measured on this machine.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config small|medium|large|decode]
+  python bench.py --impl reference ...     # the CPU oracle, timed on the host cores
+
+N > 1 runs one replica per GPU (torchrun, one rank per GPU): sequences are independent,
+each rank runs the whole configured batch (weak scaling), nothing crosses ranks on the data
+path; the timed region is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from depth_recurrent_attention_b200 import configs, inputs  # noqa: E402
+
+METRIC = "Dreamer core fwd token·depth-steps/s (bf16, 1×B200) and % of roofline"
+UNIT = "token-depth-steps/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ----------------------------------------------------------------------------------------
+# roofline accounting (algorithmic work of one forward)
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), tc=float(p["bf16_tflops"]),
+                    tc_sust=float(p["bf16_tflops_sustained"]), source="measured")
+    except Exception:
+        return dict(hbm=6650.0, tc=1590.0, tc_sust=1400.0, source="fallback")
+
+
+def algorithmic(cfg, counts=None):
+    """Per-stage algorithmic FLOPs and HBM bytes of one full forward (or decode step).
+
+    FLOPs: every multiply-add of a contraction counted twice (SA causal half only, the router
+    at its plain 2 h d_r + 2 E d_r per token).  Bytes: weights read once per depth (routed
+    experts only: those the run's route counts touch), activations read and written once,
+    DA keys/values written once and re-read for every later depth, SA keys/values (prefill)
+    written and read once, the decode cache read once.  bf16 = 2 bytes."""
+    b, s, h, L = cfg.batch, cfg.seq, cfg.hidden, cfg.depth
+    E, k, m, dr, P = cfg.n_experts, cfg.top_k, cfg.expert_hidden, cfg.router_dim, cfg.n_proj_experts
+    T = cfg.tokens
+    es = 2 if cfg.dtype == "bf16" else 4
+    G = max(P, 1)
+    st = {}
+
+    def add(name, fl, by):
+        f0, b0 = st.get(name, (0.0, 0.0))
+        st[name] = (f0 + fl, b0 + by)
+
+    for l in range(L):
+        add("norm", 0.0, T * h * (es + es))                      # x in, x^ out
+        if P > 0:
+            add("proj_route", 2.0 * T * h * dr + 2.0 * T * P * dr, T * h * es)
+        add("qkv", 2.0 * T * h * 6 * h, T * h * es + G * 6 * h * h * es + T * 6 * h * es)
+        ctx = (l + 1)
+        add("da", 4.0 * T * h * ctx, T * h * es + T * 2 * h * es * l + T * h * es)
+        if cfg.is_decode:
+            n_ctx = cfg.cache_len + 1
+            add("sa", 4.0 * T * h * n_ctx, 2.0 * T * h * es * n_ctx + 2 * T * h * es)
+        else:
+            add("sa", 4.0 * h * b * s * (s + 1) / 2, 4.0 * T * h * es)
+        add("o_proj", 2.0 * T * 2 * h * h, T * 2 * h * es + G * 2 * h * h * es + T * h * (es + 4))
+        add("ea_route", 2.0 * T * h * dr + 2.0 * T * E * dr, T * h * es + h * dr * es + E * dr * es)
+        touched = E
+        if counts is not None:
+            touched = int((np.asarray(counts)[l] > 0).sum())
+        add("experts", 4.0 * T * k * h * m,
+            2.0 * touched * h * m * es + T * h * es + T * h * 4 * 2)
+    tot_f = sum(v[0] for v in st.values())
+    tot_b = sum(v[1] for v in st.values())
+    return st, tot_f, tot_b
+
+
+# ----------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[5 + i].lower() in ("active", "1")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------------------
+# our arm
+
+def device_setup(cfg, torch, rank):
+    W = inputs.device_weights(cfg)
+    X = inputs.device_inputs(cfg)
+    if rank:
+        # each rank draws its own batch (the next seed), weights are shared
+        X = {s.name: inputs.device_tensor(s, cfg.seed + 1000 * rank) for s in inputs.input_specs(cfg)}
+    return W, X
+
+
+def run_ours(args, cfg, rank, world, torch, dist):
+    from depth_recurrent_attention_b200.dreamer import Dreamer
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    W, X = device_setup(cfg, torch, rank)
+    model = Dreamer(cfg, W)
+    x_in = X["x0"]
+    x_out = torch.empty_like(x_in)
+    decode = cfg.is_decode
+    if decode:
+        lens = torch.full((cfg.batch,), cfg.cache_len, dtype=torch.int32, device=dev)
+        kc, vc = X["k_cache"], X["v_cache"]
+
+    def step(xi=x_in, xo=x_out):
+        if decode:
+            model.decode_step(xi, kc, vc, lens, x_out=xo)
+        else:
+            model.forward(xi, x_out=xo)
+
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    resident = (sum(t.numel() * t.element_size() for t in W.values()) +
+                sum(t.numel() * t.element_size() for t in X.values()))
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # ---- timed region: K steps, L2 flushed before each (flush not timed)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    model.stats(reset=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            starts[i].record()
+            step()
+            ends[i].record()
+        torch.cuda.synchronize()
+    barrier()
+    launches = model.stats(reset=True)["launches"]
+    ms_steps = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms_total = float(sum(ms_steps))
+    if dist is not None:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    units = cfg.units * world
+    value = units / (ms_step / 1e3)
+    clocks = clk.summary()
+
+    # ---- per-stage device times (same workload, profiling events on, separate run)
+    model.set_profiling(True)
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        step()
+    st = model.stats(reset=True)
+    model.set_profiling(False)
+    counts = model.route_counts(on_host=True).numpy()
+    stage_alg, F, B = algorithmic(cfg, counts)
+    pk = peaks()
+    t_roof = max(F / (pk["tc"] * 1e12), B / (pk["hbm"] * 1e9))
+    per_stage = {}
+    for name, ms in st["ms"].items():
+        n = max(st["count"][name], 1)
+        per_stage[name] = ms / max(args.steps, 1)
+    dominant = max(per_stage, key=lambda k: per_stage[k])
+    fl, by = stage_alg.get(dominant, (0.0, 0.0))
+    t_dom = per_stage[dominant] / 1e3  # s per forward
+    bound_tensor = fl / (pk["tc"] * 1e12) > by / (pk["hbm"] * 1e9)
+    launches_per_fwd = max(st["count"][dominant] // max(args.steps, 1), 1)
+    if bound_tensor:
+        achieved = fl / t_dom / 1e12
+        roof = dict(bound="tensor", achieved=achieved, peak=pk["tc"], unit="TFLOP/s",
+                    frac=achieved / pk["tc"])
+    else:
+        achieved = by / t_dom / 1e9
+        roof = dict(bound="hbm", achieved=achieved, peak=pk["hbm"], unit="GB/s",
+                    frac=achieved / pk["hbm"])
+    roof.update(kernel=dominant, launches_per_step=launches_per_fwd, traffic=None,
+                peak_source=pk["source"] + " (MEASURED_PEAKS.json burst figure)")
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not decode:
+        host_in = torch.empty(x_in.shape, dtype=x_in.dtype, pin_memory=True)
+        host_in.copy_(x_in)
+        host_out = torch.empty(x_in.shape, dtype=x_in.dtype, pin_memory=True)
+        xi = torch.empty_like(x_in)
+        for _ in range(2):
+            xi.copy_(host_in, non_blocking=True)
+            step(xi, x_out)
+            host_out.copy_(x_out, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(args.steps):
+            xi.copy_(host_in, non_blocking=True)
+            step(xi, x_out)
+            host_out.copy_(x_out, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        ms_e2e = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        nbytes = x_in.numel() * x_in.element_size()
+        e2e = {"value": units / (ms_e2e / args.steps / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+               "note": "includes the L2-resident reuse of weights across steps"}
+    else:
+        # decode: new token embeddings in, outputs out
+        host_in = torch.empty(x_in.shape, dtype=x_in.dtype, pin_memory=True)
+        host_in.copy_(x_in)
+        host_out = torch.empty(x_in.shape, dtype=x_in.dtype, pin_memory=True)
+        xi = torch.empty_like(x_in)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(args.steps):
+            xi.copy_(host_in, non_blocking=True)
+            step(xi, x_out)
+            host_out.copy_(x_out, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        ms_e2e = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        nbytes = x_in.numel() * x_in.element_size()
+        e2e = {"value": units / (ms_e2e / args.steps / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
+
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded N(0,1) inputs, N(0,1/fan_in) weights)",
+        "config": {"workload": workload_name(cfg), "global_batch": cfg.batch * world,
+                   "seq_len": cfg.seq, "depth": cfg.depth, "hidden": cfg.hidden,
+                   "heads": f"{cfg.n_heads}x{cfg.head_dim}", "experts": cfg.n_experts,
+                   "top_k": cfg.top_k, "expert_hidden": cfg.expert_hidden,
+                   "proj_experts": cfg.n_proj_experts,
+                   "units_per_step": cfg.units * world, "parallelism": f"dp{world} (replicas)",
+                   "l2": "flushed before every timed step (256 MB write, not timed)",
+                   "resident_bytes_per_gpu": resident},
+        "roofline": roof,
+        "roofline_step": {"t_roof_ms": t_roof * 1e3, "t_meas_ms": ms_step,
+                          "frac": t_roof * 1e3 / ms_step, "F_alg": F, "B_alg": B,
+                          "peaks": {"tensor_tflops": pk["tc"], "hbm_gbs": pk["hbm"],
+                                    "source": pk["source"]}},
+        "stage_ms_per_step": per_stage,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    return out, model
+
+
+def workload_name(cfg):
+    base = f"{cfg.name}: b={cfg.batch} s={cfg.seq} h={cfg.hidden} {cfg.n_heads}x{cfg.head_dim} " \
+           f"L={cfg.depth} E={cfg.n_experts} k={cfg.top_k} m={cfg.expert_hidden} P={cfg.n_proj_experts}"
+    if cfg.is_decode:
+        base += f" decode cache={cfg.cache_len}"
+    return base
+
+
+# ----------------------------------------------------------------------------------------
+# the oracle on the host cores (cpu_baseline leg and the --impl reference arm)
+
+def oracle_sample(cfg, seconds_hint=20.0, threads=None):
+    """Time the oracle on a bounded sample of the workload: one sequence (or, for decode,
+    one sequence's step) through a few depths; returns units/s and a description."""
+    sys.path.insert(0, os.path.join(ROOT, "oracle"))
+    import oracle as O
+    threads = threads or os.cpu_count() or 1
+    W = inputs.host_weights(cfg)
+    if cfg.is_decode:
+        one = cfg.with_(batch=1)
+        o = O.Oracle(one, W, threads=threads)
+        L, H, d = cfg.depth, cfg.n_heads, cfg.head_dim
+        cap = cfg.cache_len + 1
+        spec_k = [s for s in inputs.input_specs(cfg) if s.name == "k_cache"][0]
+        kc = np.zeros((L, H, cap, d))
+        vc = np.zeros((L, H, cap, d))
+        x = inputs.host_inputs(one)["x0"][0] if False else inputs.draw(
+            [s for s in inputs.input_specs(cfg) if s.name == "x0"][0], cfg.seed, 0, cfg.hidden)
+        t0 = time.perf_counter()
+        o.decode_seq(x, kc, vc, cfg.cache_len)
+        dt = time.perf_counter() - t0
+        return 1 * cfg.depth / dt, f"one sequence's decode step (all {cfg.depth} depths, cache " \
+                                   f"{cfg.cache_len}), zero cache contents", threads
+    # prefill: one sequence of S tokens, first depths until ~seconds_hint
+    one = cfg.with_(batch=1)
+    o = O.Oracle(one, W, threads=threads)
+    x = inputs.host_inputs(one)["x0"]
+    t0 = time.perf_counter()
+    depths = 0
+    da = np.zeros((one.tokens, cfg.depth, 2, cfg.hidden))
+    while depths < cfg.depth:
+        r = o.forward(x, depths, depths + 1, da_kv=da, trace=False)
+        x = r["x_out"].astype(np.float32)
+        da = r["da_kv"]
+        depths += 1
+        if time.perf_counter() - t0 > seconds_hint:
+            break
+    dt = time.perf_counter() - t0
+    return one.tokens * depths / dt, f"one sequence ({one.tokens} tokens) through depths " \
+                                     f"0..{depths - 1} of {cfg.depth}", threads
+
+
+def run_reference(args, cfg):
+    v, sample, cores = oracle_sample(cfg, seconds_hint=max(5.0, 20.0 / max(args.steps, 1)))
+    vals = [v]
+    for _ in range(max(args.steps, 1) - 1):
+        vv, _, _ = oracle_sample(cfg, seconds_hint=max(5.0, 20.0 / max(args.steps, 1)))
+        vals.append(vv)
+    value = statistics.median(vals)
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": workload_name(cfg)},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="small", choices=["small", "medium", "large", "decode"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = configs.CONFIGS[args.config]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, cfg)))
+        return 0
+
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    out, model = run_ours(args, cfg, rank, world, torch, dist)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            v, sample, cores = oracle_sample(cfg)
+            out["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                   "sample": sample}
+        print(json.dumps(out))
+    model.close()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

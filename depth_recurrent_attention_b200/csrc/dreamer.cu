@@ -46,7 +46,30 @@ struct dreamer_handle {
   int num_sms = 148;
   int use_tc = 1;  // bf16 contractions on tcgen05 (0: CUDA cores, for cross-checks)
   std::vector<void *> allocs;
+  // instrumentation
+  uint64_t launches = 0;
+  int prof = 0;
+  std::vector<cudaEvent_t> ev;
+  std::vector<int> ev_stage;
+  size_t ev_used = 0;
+  double stage_ms[DREAMER_N_STAGES] = {0};
+  uint64_t stage_count[DREAMER_N_STAGES] = {0};
 };
+
+// stage boundary: with profiling on, an event tagged with the stage that starts here
+static void mark(dreamer_handle *h, cudaStream_t s, int stage) {
+  if (!h->prof) return;
+  if (h->ev_used == h->ev.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return;
+    h->ev.push_back(e);
+    h->ev_stage.push_back(0);
+  }
+  cudaEventRecord(h->ev[h->ev_used], s);
+  h->ev_stage[h->ev_used] = stage;
+  h->ev_used++;
+}
+#define LAUNCHED(n) (h->launches += (n))
 
 #define CK(call)                                                  \
   do {                                                            \
@@ -301,10 +324,47 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
   return DREAMER_OK;
 }
 
+extern "C" int dreamer_set_profiling(dreamer_handle *h, int enable) {
+  if (!h) return DREAMER_ERR_ARG;
+  h->prof = enable ? 1 : 0;
+  return DREAMER_OK;
+}
+
+extern "C" int dreamer_get_stats(dreamer_handle *h, dreamer_stats *out, int reset) {
+  if (!h || !out) return DREAMER_ERR_ARG;
+  if (h->ev_used > 1) {
+    CK(cudaEventSynchronize(h->ev[h->ev_used - 1]));
+    for (size_t i = 0; i + 1 < h->ev_used; i++) {
+      const int st = h->ev_stage[i];
+      if (st >= DREAMER_N_STAGES) continue;  // end of a call: the next mark starts a new one
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, h->ev[i], h->ev[i + 1]) == cudaSuccess) {
+        h->stage_ms[st] += ms;
+        h->stage_count[st] += 1;
+      }
+    }
+  }
+  h->ev_used = 0;
+  out->launches = h->launches;
+  for (int i = 0; i < DREAMER_N_STAGES; i++) {
+    out->ms[i] = h->stage_ms[i];
+    out->count[i] = h->stage_count[i];
+  }
+  if (reset) {
+    h->launches = 0;
+    for (int i = 0; i < DREAMER_N_STAGES; i++) {
+      h->stage_ms[i] = 0;
+      h->stage_count[i] = 0;
+    }
+  }
+  return DREAMER_OK;
+}
+
 extern "C" void dreamer_destroy(dreamer_handle *h) {
   if (!h) return;
   cudaDeviceSynchronize();
   tc_destroy(h);
+  for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
   for (void *p : h->allocs) cudaFree(p);
   delete h;
 }
@@ -389,6 +449,8 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
   const bool tc = h->use_tc && c.dtype == 1;
 
   // 1. RMSNorm of the residual stream (x_0 on the first depth, else the fp32 accumulator)
+  mark(h, s, DREAMER_STAGE_NORM);
+  LAUNCHED(1);
   rmsnorm_kernel<T><<<cdiv(n, 8), 256, 0, s>>>(first ? (const T *)io.x_in : nullptr,
                                                first ? nullptr : h->acc, (const T *)h->g,
                                                (T *)h->xh, h->inv_rms, n, hd, c.rms_eps);
@@ -396,6 +458,8 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
   const int *prow = nullptr;
   const float *psig = nullptr;
   if (P > 0) {
+    mark(h, s, DREAMER_STAGE_PROJ_ROUTE);
+    LAUNCHED(2);
     cudaMemsetAsync(h->pcnt, 0, (G + 1) * sizeof(int), s);
     route_rows<T>(h, 1, l, h->xh, n, h->pidx, h->psig, nullptr, h->pcnt, s);
     scan_kernel<<<1, 1024, 0, s>>>(h->pcnt, G, h->poffs, h->ptiles_a, 64, h->ptiles_b, 128,
@@ -434,6 +498,8 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
 
   auto qkv_gemm = [&](const void *A, int col0, int ncols) {
     // columns [col0, col0 + ncols) of the fused QKV projection
+    mark(h, s, DREAMER_STAGE_QKV);
+    LAUNCHED(1);
     GemmArgs a = grouped(ncols, hd, A, hd, (const T *)h->wqkv_t + (size_t)col0 * hd,
                          (long)6 * hd * hd);
     EpiQKV<T> e2 = eq;
@@ -451,6 +517,8 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
   const int res_xhat = first ? 0 : 1;
   auto o_gemm = [&](const void *A, int row0, int nrows, int res_mode, void *yout) {
     // O projection over input rows [row0, row0 + nrows) of W_O ([a_SA | a_DA] order)
+    mark(h, s, DREAMER_STAGE_O);
+    LAUNCHED(1);
     GemmArgs a = grouped(hd, nrows, A, 2 * hd, (const T *)h->wo_t + row0, (long)2 * hd * hd);
     a.ldb = 2 * hd;
     EpiO<T> eo{hd, psig, res_mode, (const T *)io.x_in, h->inv_rms, (const T *)h->g,
@@ -462,29 +530,41 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
   if (c.variant == 1) {
     // serial DA -> SA -> EA: DA on x^, then SA on u = x^ + DA-part of O, then EA
     qkv_gemm(h->xh, 3 * hd, 3 * hd);
+    mark(h, s, DREAMER_STAGE_DA);
+    LAUNCHED(1);
     launch_attn<T>(da, d, s);
     o_gemm((const T *)h->attn + hd, hd, hd, res_xhat, h->u);   // u = x^ + DA part (acc = u)
     qkv_gemm(h->u, 0, 3 * hd);
+    mark(h, s, DREAMER_STAGE_SA);
+    LAUNCHED(1);
     if (!(io.mode == 0 && tc && tc_sa_ok(h) && tc_sa(h, s))) launch_attn<T>(sa, d, s);
     o_gemm(h->attn, 0, hd, 2, h->y);                            // y = u + SA part
   } else {
     // 3. fused QKV projection with RoPE / depth RoPE epilogue, DA KV write
     qkv_gemm(h->xh, 0, 6 * hd);
     // 4. DA || SA (papernotes "Key design 1": run in parallel for throughput)
+    mark(h, s, DREAMER_STAGE_DA);
+    LAUNCHED(2);
     launch_attn<T>(da, d, s);
+    mark(h, s, DREAMER_STAGE_SA);
     if (!(io.mode == 0 && tc && tc_sa_ok(h) && tc_sa(h, s))) launch_attn<T>(sa, d, s);
     // 5. O projection, residual y = x^ + DA + SA
     o_gemm(h->attn, 0, 2 * hd, res_xhat, h->y);
   }
   // 6. expert attention routing on y (fully parallel layout: on x^)
   const void *ein = c.variant == 2 ? h->xh : h->y;
+  mark(h, s, DREAMER_STAGE_EA_ROUTE);
+  LAUNCHED(5);
   cudaMemsetAsync(h->ecnt, 0, E * sizeof(int), s);
   route_rows<T>(h, 0, l, ein, n, h->eidx, h->ew, h->counts + (size_t)l * E, h->ecnt, s);
+  mark(h, s, DREAMER_STAGE_PERMUTE);
   scan_kernel<<<1, 1024, 0, s>>>(h->ecnt, E, h->eoffs, h->etiles_a, 64, h->etiles_b, 128,
                                  h->ecursor);
   scatter_kernel<<<cdiv((long)n * k, 256), 256, 0, s>>>(h->eidx, n * k, h->ecursor, h->erows,
                                                          nullptr);
   // 7. expert FFNs: H = SiLU(X W1_e), acc[token] += w * H W2_e
+  mark(h, s, DREAMER_STAGE_EXPERTS);
+  LAUNCHED(2);
   if (!(tc && tc_expert_ok(h) && tc_expert(h, ein, n, s))) {
     const int etiles = cdiv((long)n * k, 64) + E;
     GemmArgs up{};
@@ -547,12 +627,15 @@ static int forward_impl(dreamer_handle *h, const void *x_in, void *x_out, int l0
     run_depth<T>(h, l, l == l0, io, s);
     trace_depth(h, tr, l, n, true, s);
   }
+  mark(h, s, DREAMER_STAGE_FINISH);
   if (l1 > l0) {
+    LAUNCHED(1);
     long tot = (long)n * c.hidden;
     finish_kernel<T><<<cdiv(tot / 8, 256), 256, 0, s>>>(h->acc, (T *)x_out, tot);
   } else if (x_out != x_in) {
     CK(cudaMemcpyAsync(x_out, x_in, (size_t)n * c.hidden * h->esz, cudaMemcpyDeviceToDevice, s));
   }
+  mark(h, s, DREAMER_N_STAGES);
   CK(cudaGetLastError());
   return DREAMER_OK;
 }
@@ -585,8 +668,11 @@ static int decode_impl(dreamer_handle *h, const void *x_new, void *kc, void *vc,
     run_depth<T>(h, l, l == 0, io, s);
     trace_depth(h, tr, l, n, false, s);
   }
+  mark(h, s, DREAMER_STAGE_FINISH);
+  LAUNCHED(1);
   long tot = (long)n * c.hidden;
   finish_kernel<T><<<cdiv(tot / 8, 256), 256, 0, s>>>(h->acc, (T *)x_out, tot);
+  mark(h, s, DREAMER_N_STAGES);
   CK(cudaGetLastError());
   return DREAMER_OK;
 }

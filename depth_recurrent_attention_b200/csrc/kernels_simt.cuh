@@ -98,7 +98,7 @@ template <typename T> struct EpiQKV {
 // and the token's 1/rms, so the only rounding of y is its own store.  acc receives the fp32 y
 // (the base that the expert outputs are added to); y itself is stored in dtype for the
 // router and the experts.
-//   res_mode 0: residual x^ from xin;  1: x^ from round(acc);  2: residual = acc as is
+//   res_mode 0: residual x^ from xin;  1: x^ from acc (fp32 x_l);  2: residual = acc as is
 //   (the serial layout's u).
 template <typename T> struct EpiO {
   int h;
@@ -123,8 +123,7 @@ template <typename T> struct EpiO {
         load8(gain + n0 + i, gv);
 #pragma unroll
         for (int j = 0; j < 8; j++) {
-          const float xv = res_mode == 1 ? to_f(from_f<T>(xr[j])) : xr[j];
-          xr[j] = gv[j] * xv * ir;
+          xr[j] = gv[j] * xr[j] * ir;
         }
       }
 #pragma unroll
@@ -289,8 +288,9 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a, Epi epi) {
 // =======================================================================================
 // RMSNorm (papernotes "Overall framework": RMSNorm on the residual stream; R1: one norm per
 // depth, the stream continues from x^).  One warp per token.  The input is either the
-// dtype residual x (first depth) or the fp32 accumulator of the previous depth, which is
-// first rounded to dtype (the residual stream is carried in dtype between depths).
+// dtype residual x (first depth of a call) or the fp32 accumulator of the previous depth:
+// inside a call the residual stream stays in fp32, it is rounded to dtype only when it
+// leaves the call.
 // =======================================================================================
 template <typename T>
 __global__ void rmsnorm_kernel(const T *x_in, const float *acc, const T *gain, T *xh,
@@ -301,13 +301,8 @@ __global__ void rmsnorm_kernel(const T *x_in, const float *acc, const T *gain, T
   float ss = 0.f;
   for (int c = lane * 8; c < h; c += 256) {
     float v[8];
-    if (acc) {
-      load8(acc + (long)warp * h + c, v);
-#pragma unroll
-      for (int j = 0; j < 8; j++) v[j] = to_f(from_f<T>(v[j]));
-    } else {
-      load8(x_in + (long)warp * h + c, v);
-    }
+    if (acc) load8(acc + (long)warp * h + c, v);
+    else load8(x_in + (long)warp * h + c, v);
 #pragma unroll
     for (int j = 0; j < 8; j++) ss += v[j] * v[j];
   }
@@ -316,13 +311,8 @@ __global__ void rmsnorm_kernel(const T *x_in, const float *acc, const T *gain, T
   if (lane == 0 && inv_rms) inv_rms[warp] = r;
   for (int c = lane * 8; c < h; c += 256) {
     float v[8], gv[8], o[8];
-    if (acc) {
-      load8(acc + (long)warp * h + c, v);
-#pragma unroll
-      for (int j = 0; j < 8; j++) v[j] = to_f(from_f<T>(v[j]));
-    } else {
-      load8(x_in + (long)warp * h + c, v);
-    }
+    if (acc) load8(acc + (long)warp * h + c, v);
+    else load8(x_in + (long)warp * h + c, v);
     load8(gain + c, gv);
 #pragma unroll
     for (int j = 0; j < 8; j++) o[j] = gv[j] * v[j] * r;

@@ -45,6 +45,15 @@ class WeightsC(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in WEIGHT_FIELDS]
 
 
+STAGES = ("norm", "proj_route", "qkv", "da", "sa", "o_proj", "ea_route", "permute",
+          "experts", "finish")
+
+
+class StatsC(C.Structure):
+    _fields_ = [("launches", C.c_uint64), ("ms", C.c_double * len(STAGES)),
+                ("count", C.c_uint64 * len(STAGES))]
+
+
 TRACE_FIELDS = ("xhat", "y", "idx", "w", "sa_k", "sa_v", "pidx", "psig")
 
 
@@ -65,12 +74,15 @@ def lib():
         L.dreamer_route_counts.argtypes = [vp, vp, i, vp]
         L.dreamer_route_experts.argtypes = [vp, i, vp, i, vp, vp, vp, vp]
         L.dreamer_bias_update.argtypes = [vp, C.c_float, vp, vp]
+        L.dreamer_set_profiling.argtypes = [vp, i]
+        L.dreamer_get_stats.argtypes = [vp, C.POINTER(StatsC), i]
         L.dreamer_destroy.argtypes = [vp]
         L.dreamer_destroy.restype = None
         L.dreamer_strerror.argtypes = [i]
         L.dreamer_strerror.restype = C.c_char_p
         for f in ("dreamer_init", "dreamer_core_forward", "dreamer_decode_step",
-                  "dreamer_route_counts", "dreamer_route_experts", "dreamer_bias_update"):
+                  "dreamer_route_counts", "dreamer_route_experts", "dreamer_bias_update",
+                  "dreamer_set_profiling", "dreamer_get_stats"):
             getattr(L, f).restype = i
         _lib = L
     return _lib
@@ -193,3 +205,13 @@ class Dreamer:
         _check(lib().dreamer_bias_update(self.h, float(lam), _ptr(out), _stream(stream)),
                "dreamer_bias_update")
         return out
+
+    def set_profiling(self, enable: bool):
+        _check(lib().dreamer_set_profiling(self.h, int(bool(enable))), "dreamer_set_profiling")
+
+    def stats(self, reset: bool = True) -> dict:
+        st = StatsC()
+        _check(lib().dreamer_get_stats(self.h, C.byref(st), int(bool(reset))), "dreamer_get_stats")
+        return dict(launches=int(st.launches),
+                    ms={n: float(st.ms[i]) for i, n in enumerate(STAGES)},
+                    count={n: int(st.count[i]) for i, n in enumerate(STAGES)})

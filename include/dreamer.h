@@ -159,6 +159,34 @@ int dreamer_route_experts(dreamer_handle *h, int depth, const void *y, int n_tok
 int dreamer_bias_update(dreamer_handle *h, float lambda, float *bias_out,
                         dreamer_stream stream);
 
+/* Instrumentation.  Stages of the depth step, in launch order: */
+enum {
+  DREAMER_STAGE_NORM = 0,     /* RMSNorm of the residual stream                          */
+  DREAMER_STAGE_PROJ_ROUTE,   /* projection router + grouping (linear-MoE QKV/O)         */
+  DREAMER_STAGE_QKV,          /* fused QKV projection, RoPE / depth RoPE, DA KV write    */
+  DREAMER_STAGE_DA,           /* depth attention                                         */
+  DREAMER_STAGE_SA,           /* causal sequence attention (prefill) / cache attention   */
+  DREAMER_STAGE_O,            /* O projection + residual                                 */
+  DREAMER_STAGE_EA_ROUTE,     /* expert router: query, scores, top-k, counts             */
+  DREAMER_STAGE_PERMUTE,      /* counting sort of routed slots by expert                 */
+  DREAMER_STAGE_EXPERTS,      /* expert FFNs with weighted scatter-add                   */
+  DREAMER_STAGE_FINISH,       /* final residual store and call overhead                  */
+  DREAMER_N_STAGES
+};
+typedef struct {
+  uint64_t launches;                 /* kernels launched by the library since the reset    */
+  double ms[DREAMER_N_STAGES];       /* device time per stage (profiling enabled only)     */
+  uint64_t count[DREAMER_N_STAGES];  /* timed stage executions                             */
+} dreamer_stats;
+
+/* Enable (1) or disable (0) per-stage CUDA-event timing on the streams of later calls.
+ * Timing adds one event record per stage boundary; it is meant for measurement runs.     */
+int dreamer_set_profiling(dreamer_handle *h, int enable);
+
+/* Read the launch counter and the per-stage times accumulated since the last reset
+ * (synchronises the device when profiling is on); reset = 1 clears them afterwards.      */
+int dreamer_get_stats(dreamer_handle *h, dreamer_stats *out, int reset);
+
 /* Free the handle and everything it owns (synchronises the device).                      */
 void dreamer_destroy(dreamer_handle *h);
 

@@ -5,9 +5,9 @@ Tolerances (the stated bounds of the Dreamer core-forward contract):
     oracle's k-th and (k+1)-th biased scores lie within 1e-5 (counted, reported).
   * bfloat16 mode: hidden states max-abs <= 3e-2 and relative L2 <= 1e-2.
   * route counts exact.
-A bfloat16 output is its value rounded to bf16: for |x| >= 8 that rounding alone can reach
-1/32 > 3e-2, so each element's bound is 3e-2 plus the part of its own half-ulp above 1/64
-(the half-ulp of the [4, 8) binade); below 8 the bound is exactly 3e-2.
+A bfloat16 output is its exact value rounded to the nearest bf16 number; that rounding (up
+to half an ulp: 1/64 for |x| in [4, 8), 1/32 in [8, 16)) is not arithmetic error.  Each
+element's bound is therefore 3e-2 plus its own half-ulp; relative L2 <= 1e-2 applies as is.
 In bfloat16 mode the router reads the bf16-rounded state y, which differs from the oracle's
 float64 y by rounding; a selection may then legitimately differ from the oracle's where the
 oracle's selection margin is below what that difference in y can move the scores:
@@ -77,7 +77,7 @@ def bf16_half_ulp(x) -> np.ndarray:
 
 
 def bf16_abs_bound(ref) -> np.ndarray:
-    return TOL_BF16_ABS + np.maximum(0.0, bf16_half_ulp(ref) - 1.0 / 64)
+    return TOL_BF16_ABS + bf16_half_ulp(ref)
 
 
 def check_hidden(got, ref, bf16: bool, what: str):
