@@ -46,6 +46,23 @@ struct dreamer_handle {
   int num_sms = 148;
   int use_tc = 1;  // bf16 contractions on tcgen05 (0: CUDA cores, for cross-checks)
   std::vector<void *> allocs;
+  int *err_host = nullptr;       // pinned copy of the device error flag (async)
+  cudaStream_t side = nullptr;   // second stream: DA runs beside SA
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  int use_graph = 1;
+  struct GraphEntry {
+    int kind;                    // 0 forward, 1 decode
+    const void *key[5];
+    int l0, l1, prof;
+    int captured;                // 0: seen once (ran directly), 1: graph ready
+    cudaGraphExec_t exec;
+    uint64_t launches;
+    std::vector<cudaEvent_t> evs;
+    std::vector<int> stages;
+    uint64_t last_use;
+  };
+  std::vector<GraphEntry> graphs;
+  uint64_t use_clock = 0;
   // instrumentation
   uint64_t launches = 0;
   int prof = 0;
@@ -70,6 +87,21 @@ static void mark(dreamer_handle *h, cudaStream_t s, int stage) {
   h->ev_used++;
 }
 #define LAUNCHED(n) (h->launches += (n))
+
+static void accumulate_marks(dreamer_handle *h, const std::vector<cudaEvent_t> &evs,
+                             const std::vector<int> &stages) {
+  for (size_t i = 0; i + 1 < evs.size(); i++) {
+    const int st = stages[i];
+    if (st >= DREAMER_N_STAGES) continue;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, evs[i], evs[i + 1]) == cudaSuccess) {
+      h->stage_ms[st] += ms;
+      h->stage_count[st] += 1;
+    }
+  }
+}
+
+
 
 #define CK(call)                                                  \
   do {                                                            \
@@ -234,6 +266,12 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     const size_t es = h->esz;
     const long T = h->T;
     if (const char *ev = getenv("DREAMER_NO_TC")) h->use_tc = atoi(ev) ? 0 : 1;
+    if (const char *ev = getenv("DREAMER_NO_GRAPH")) h->use_graph = atoi(ev) ? 0 : 1;
+    CK(cudaHostAlloc((void **)&h->err_host, sizeof(int), cudaHostAllocDefault));
+    *h->err_host = 0;
+    CK(cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
+    CK(cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming));
     // ---- weights
     DALLOC(h->g, hd * es);
     CK(cudaMemcpyAsync(h->g, w->rms_gain, hd * es, cudaMemcpyDeviceToDevice, s));
@@ -334,15 +372,9 @@ extern "C" int dreamer_get_stats(dreamer_handle *h, dreamer_stats *out, int rese
   if (!h || !out) return DREAMER_ERR_ARG;
   if (h->ev_used > 1) {
     CK(cudaEventSynchronize(h->ev[h->ev_used - 1]));
-    for (size_t i = 0; i + 1 < h->ev_used; i++) {
-      const int st = h->ev_stage[i];
-      if (st >= DREAMER_N_STAGES) continue;  // end of a call: the next mark starts a new one
-      float ms = 0.f;
-      if (cudaEventElapsedTime(&ms, h->ev[i], h->ev[i + 1]) == cudaSuccess) {
-        h->stage_ms[st] += ms;
-        h->stage_count[st] += 1;
-      }
-    }
+    std::vector<cudaEvent_t> evs(h->ev.begin(), h->ev.begin() + h->ev_used);
+    std::vector<int> st(h->ev_stage.begin(), h->ev_stage.begin() + h->ev_used);
+    accumulate_marks(h, evs, st);
   }
   h->ev_used = 0;
   out->launches = h->launches;
@@ -365,6 +397,14 @@ extern "C" void dreamer_destroy(dreamer_handle *h) {
   cudaDeviceSynchronize();
   tc_destroy(h);
   for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+  for (auto &g : h->graphs) {
+    if (g.captured) cudaGraphExecDestroy(g.exec);
+    for (cudaEvent_t e : g.evs) cudaEventDestroy(e);
+  }
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
+  if (h->side) cudaStreamDestroy(h->side);
+  if (h->err_host) cudaFreeHost(h->err_host);
   for (void *p : h->allocs) cudaFree(p);
   delete h;
 }
@@ -542,12 +582,22 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
   } else {
     // 3. fused QKV projection with RoPE / depth RoPE epilogue, DA KV write
     qkv_gemm(h->xh, 0, 6 * hd);
-    // 4. DA || SA (papernotes "Key design 1": run in parallel for throughput)
-    mark(h, s, DREAMER_STAGE_DA);
+    // 4. DA || SA (papernotes "Key design 1": run in parallel for throughput).  DA runs
+    // on the side stream beside SA (two branches of the captured graph); with stage
+    // profiling on they run one after the other so each stage's time is its own.
     LAUNCHED(2);
-    launch_attn<T>(da, d, s);
+    if (h->prof) {
+      mark(h, s, DREAMER_STAGE_DA);
+      launch_attn<T>(da, d, s);
+    } else {
+      cudaEventRecord(h->ev_fork, s);
+      cudaStreamWaitEvent(h->side, h->ev_fork, 0);
+      launch_attn<T>(da, d, h->side);
+      cudaEventRecord(h->ev_join, h->side);
+    }
     mark(h, s, DREAMER_STAGE_SA);
     if (!(io.mode == 0 && tc && tc_sa_ok(h) && tc_sa(h, s))) launch_attn<T>(sa, d, s);
+    if (!h->prof) cudaStreamWaitEvent(s, h->ev_join, 0);
     // 5. O projection, residual y = x^ + DA + SA
     o_gemm(h->attn, 0, 2 * hd, res_xhat, h->y);
   }
@@ -580,13 +630,28 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
   }
 }
 
+// The device error flag is copied to pinned host memory at the end of every call; the next
+// call reads that copy without synchronising (errors of calls still running show up one call
+// later, or at dreamer_route_counts(on_host = 1), which synchronises and reads it exactly).
+static int dev_error_code(int e) { return e == DEV_TIMEOUT ? DREAMER_ERR_TIMEOUT : DREAMER_ERR_ARG; }
 static int check_dev_error(dreamer_handle *h) {
+  const int e = *(volatile int *)h->err_host;
+  if (e) {
+    cudaDeviceSynchronize();
+    cudaMemset(h->err, 0, sizeof(int));
+    *h->err_host = 0;
+    return dev_error_code(e);
+  }
+  return DREAMER_OK;
+}
+static int check_dev_error_sync(dreamer_handle *h) {
   int e = 0;
   if (cudaMemcpy(&e, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return DREAMER_ERR_CUDA;
   if (e) {
     cudaMemset(h->err, 0, sizeof(int));
-    return e == DEV_TIMEOUT ? DREAMER_ERR_TIMEOUT : DREAMER_ERR_ARG;
+    *h->err_host = 0;
+    return dev_error_code(e);
   }
   return DREAMER_OK;
 }
@@ -615,6 +680,87 @@ static void trace_depth(dreamer_handle *h, const dreamer_trace *tr, int l, int n
 
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
 
+// ---------------------------------------------------------------------------------------
+// CUDA graphs: the whole call (every depth, ~10 kernels each) is captured once per set of
+// argument pointers and replayed, so the host enqueues one graph instead of ~10 L kernels.
+// A pointer set runs directly the first time it is seen (this also sets every kernel's
+// attributes outside capture) and is captured on its second use.  Calls with a trace run
+// directly.  Up to 8 graphs are cached per handle (least recently used evicted).
+template <class F>
+static int run_graphed(dreamer_handle *h, int kind, const void *const key[5], int l0, int l1,
+                       cudaStream_t s, F &&enqueue) {
+  if (!h->use_graph) return enqueue();
+  dreamer_handle::GraphEntry *e = nullptr;
+  for (auto &g : h->graphs)
+    if (g.kind == kind && g.l0 == l0 && g.l1 == l1 && g.prof == h->prof &&
+        !memcmp(g.key, key, sizeof(g.key))) {
+      e = &g;
+      break;
+    }
+  if (!e) {
+    if (h->graphs.size() >= 8) {
+      size_t old = 0;
+      for (size_t i = 1; i < h->graphs.size(); i++)
+        if (h->graphs[i].last_use < h->graphs[old].last_use) old = i;
+      auto &g = h->graphs[old];
+      if (g.captured) cudaGraphExecDestroy(g.exec);
+      for (cudaEvent_t ev : g.evs) cudaEventDestroy(ev);
+      h->graphs.erase(h->graphs.begin() + old);
+    }
+    dreamer_handle::GraphEntry g{};
+    g.kind = kind;
+    memcpy(g.key, key, sizeof(g.key));
+    g.l0 = l0; g.l1 = l1; g.prof = h->prof; g.captured = 0;
+    g.last_use = ++h->use_clock;
+    h->graphs.push_back(g);
+    return enqueue();  // first use: direct
+  }
+  e->last_use = ++h->use_clock;
+  if (!e->captured) {
+    const size_t ev0 = h->ev_used;
+    const uint64_t l_before = h->launches;
+    cudaGraph_t graph = nullptr;
+    if (cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+      cudaGetLastError();
+      return enqueue();
+    }
+    int rc = enqueue();
+    cudaError_t ce = cudaStreamEndCapture(s, &graph);
+    const uint64_t n_launch = h->launches - l_before;
+    h->launches = l_before;
+    if (rc != DREAMER_OK || ce != cudaSuccess || !graph) {
+      if (graph) cudaGraphDestroy(graph);
+      cudaGetLastError();
+      h->ev_used = ev0;
+      h->use_graph = 0;  // capture is not available here: run directly from now on
+      return rc != DREAMER_OK ? rc : enqueue();
+    }
+    cudaError_t ie = cudaGraphInstantiate(&e->exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (ie != cudaSuccess) {
+      cudaGetLastError();
+      h->ev_used = ev0;
+      h->use_graph = 0;
+      return enqueue();
+    }
+    e->captured = 1;
+    e->launches = n_launch;
+    // the graph records into the events its marks captured: they now belong to it
+    e->evs.assign(h->ev.begin() + ev0, h->ev.begin() + h->ev_used);
+    e->stages.assign(h->ev_stage.begin() + ev0, h->ev_stage.begin() + h->ev_used);
+    h->ev.erase(h->ev.begin() + ev0, h->ev.begin() + h->ev_used);
+    h->ev_stage.erase(h->ev_stage.begin() + ev0, h->ev_stage.begin() + h->ev_used);
+    h->ev_used = ev0;
+  }
+  CK(cudaGraphLaunch(e->exec, s));
+  h->launches += e->launches;
+  if (e->prof && !e->evs.empty()) {
+    CK(cudaStreamSynchronize(s));
+    accumulate_marks(h, e->evs, e->stages);
+  }
+  return DREAMER_OK;
+}
+
 template <typename T>
 static int forward_impl(dreamer_handle *h, const void *x_in, void *x_out, int l0, int l1,
                         void *da_kv, const dreamer_trace *tr, cudaStream_t s) {
@@ -635,6 +781,7 @@ static int forward_impl(dreamer_handle *h, const void *x_in, void *x_out, int l0
   } else if (x_out != x_in) {
     CK(cudaMemcpyAsync(x_out, x_in, (size_t)n * c.hidden * h->esz, cudaMemcpyDeviceToDevice, s));
   }
+  CK(cudaMemcpyAsync(h->err_host, h->err, sizeof(int), cudaMemcpyDeviceToHost, s));
   mark(h, s, DREAMER_N_STAGES);
   CK(cudaGetLastError());
   return DREAMER_OK;
@@ -651,8 +798,13 @@ extern "C" int dreamer_core_forward(dreamer_handle *h, const void *x_in, void *x
   int e = check_dev_error(h);
   if (e) return e;
   cudaStream_t s = (cudaStream_t)stream;
-  return c.dtype == 0 ? forward_impl<float>(h, x_in, x_out, depth_begin, depth_end, da_kv, trace, s)
-                      : forward_impl<bf16>(h, x_in, x_out, depth_begin, depth_end, da_kv, trace, s);
+  auto enqueue = [&]() -> int {
+    return c.dtype == 0 ? forward_impl<float>(h, x_in, x_out, depth_begin, depth_end, da_kv, trace, s)
+                        : forward_impl<bf16>(h, x_in, x_out, depth_begin, depth_end, da_kv, trace, s);
+  };
+  if (trace) return enqueue();
+  const void *key[5] = {x_in, x_out, da_kv, nullptr, nullptr};
+  return run_graphed(h, 0, key, depth_begin, depth_end, s, enqueue);
 }
 
 template <typename T>
@@ -672,6 +824,7 @@ static int decode_impl(dreamer_handle *h, const void *x_new, void *kc, void *vc,
   LAUNCHED(1);
   long tot = (long)n * c.hidden;
   finish_kernel<T><<<cdiv(tot / 8, 256), 256, 0, s>>>(h->acc, (T *)x_out, tot);
+  CK(cudaMemcpyAsync(h->err_host, h->err, sizeof(int), cudaMemcpyDeviceToHost, s));
   mark(h, s, DREAMER_N_STAGES);
   CK(cudaGetLastError());
   return DREAMER_OK;
@@ -687,9 +840,14 @@ extern "C" int dreamer_decode_step(dreamer_handle *h, const void *x_new, void *k
   int e = check_dev_error(h);
   if (e) return e;
   cudaStream_t s = (cudaStream_t)stream;
-  return h->cfg.dtype == 0
-             ? decode_impl<float>(h, x_new, k_cache, v_cache, cache_len, x_out, trace, s)
-             : decode_impl<bf16>(h, x_new, k_cache, v_cache, cache_len, x_out, trace, s);
+  auto enqueue = [&]() -> int {
+    return h->cfg.dtype == 0
+               ? decode_impl<float>(h, x_new, k_cache, v_cache, cache_len, x_out, trace, s)
+               : decode_impl<bf16>(h, x_new, k_cache, v_cache, cache_len, x_out, trace, s);
+  };
+  if (trace) return enqueue();
+  const void *key[5] = {x_new, k_cache, v_cache, cache_len, x_out};
+  return run_graphed(h, 1, key, 0, h->cfg.depth, s, enqueue);
 }
 
 extern "C" int dreamer_route_counts(dreamer_handle *h, int32_t *counts, int on_host,
@@ -700,7 +858,7 @@ extern "C" int dreamer_route_counts(dreamer_handle *h, int32_t *counts, int on_h
   if (on_host) {
     CK(cudaMemcpyAsync(counts, h->counts, bytes, cudaMemcpyDeviceToHost, s));
     CK(cudaStreamSynchronize(s));
-    return check_dev_error(h);
+    return check_dev_error_sync(h);
   }
   CK(cudaMemcpyAsync(counts, h->counts, bytes, cudaMemcpyDeviceToDevice, s));
   return DREAMER_OK;

@@ -226,18 +226,25 @@ void orc_bias_update(int L, int E, const int32_t *counts, double lambda, double 
 
 /* out[j] = sum_i x[i] * W[(row0 + i) * ld + col0 + j] for j < ncol, over the routed
  * expert's matrix Wp and, for the linear MoE, plus the shared matrix, both scaled by
- * sigma (R12 with the identity of "Key design 3").  Dense projections: Wsh == NULL.     */
+ * sigma (R12 with the identity of "Key design 3").  Dense projections: Wsh == NULL.
+ * Loops run over the rows of W (i outer) so W streams once; every out[j] is still the sum
+ * over i = 0, 1, ... in that order.                                                       */
 static void proj(const double *x, int nin, const float *Wp, const float *Wsh, long ld, int row0,
                  int col0, int ncol, double sigma, double *out) {
-  for (int j = 0; j < ncol; j++) {
-    double ap = 0.0, as = 0.0;
-    for (int i = 0; i < nin; i++) {
-      double xi = x[i];
-      ap += xi * (double)Wp[(long)(row0 + i) * ld + col0 + j];
-      if (Wsh) as += xi * (double)Wsh[(long)(row0 + i) * ld + col0 + j];
+  double *ap = (double *)xcalloc((size_t)ncol, sizeof(double));
+  double *as = Wsh ? (double *)xcalloc((size_t)ncol, sizeof(double)) : NULL;
+  for (int i = 0; i < nin; i++) {
+    const double xi = x[i];
+    const float *wr = Wp + (long)(row0 + i) * ld + col0;
+    for (int j = 0; j < ncol; j++) ap[j] += xi * (double)wr[j];
+    if (Wsh) {
+      const float *sr = Wsh + (long)(row0 + i) * ld + col0;
+      for (int j = 0; j < ncol; j++) as[j] += xi * (double)sr[j];
     }
-    out[j] = Wsh ? (sigma * ap + sigma * as) : ap;
   }
+  for (int j = 0; j < ncol; j++) out[j] = Wsh ? (sigma * ap[j] + sigma * as[j]) : ap[j];
+  free(ap);
+  free(as);
 }
 
 /* depth-RoPE'd key table for depth l: rot[e][:] = R_l key[e][:] (R6, R8)               */
