@@ -119,3 +119,10 @@ def check_drift(got, ref, what: str, gate_abs: bool):
         return check_hidden(got, ref, True, what)
     assert rl <= TOL_BF16_REL, f"{what}: rel-L2 {rl:.3g} (<= {TOL_BF16_REL}); max-abs {err:.3g}"
     return err, rl
+
+
+def weights_by_expert(idx, w) -> np.ndarray:
+    """Routing weights reordered by expert index (the pick order of two nearly equal
+    scores may differ between the two sides; the (expert, weight) pairs may not)."""
+    o = np.argsort(idx, axis=-1)
+    return np.take_along_axis(np.asarray(w, np.float64), o, axis=-1)

@@ -102,7 +102,8 @@ def test_fullsize_router_strict(cuda, name, l):
     same, flips = PY.check_routing(cfg, W, l, idx, ref["idx"], ref["margin"], strict=True)
     print(f"router {name} depth {l}: {flips} flips at "
           f"{int((ref['margin'] <= PY.NEAR_TIE).sum())} near ties over {cfg.tokens} tokens")
-    assert np.allclose(PY.to_np(w)[same], ref["w"][same], atol=1e-5)
+    assert np.allclose(PY.weights_by_expert(idx, PY.to_np(w))[same],
+                       PY.weights_by_expert(ref["idx"], ref["w"])[same], atol=1e-5)
     c = counts.cpu().numpy()
     assert np.array_equal(c, np.bincount(idx.ravel(), minlength=cfg.n_experts))
     if flips == 0:
