@@ -32,7 +32,8 @@ def build(force: bool = False, verbose: bool = False) -> list:
     lib = os.path.join(HERE, "libdreamer.so")
     deps = [p for p in _sources() if not p.endswith("inputs_gen.cu")]
     if force or not _newer(lib, deps):
-        cmd = ["nvcc", *ARCH, *FLAGS, "-o", lib, os.path.join(CSRC, "dreamer.cu")]
+        cmd = ["nvcc", *ARCH, *FLAGS, "-o", lib, os.path.join(CSRC, "dreamer.cu"),
+               os.path.join(CSRC, "route_noalloc.cu")]
         if verbose:
             print(" ".join(cmd))
         subprocess.run(cmd, check=True)

@@ -152,6 +152,30 @@ int dreamer_route_counts(dreamer_handle *h, int32_t *counts, int on_host,
 int dreamer_route_experts(dreamer_handle *h, int depth, const void *y, int n_tokens,
                           int32_t *idx, float *w, int32_t *counts, dreamer_stream stream);
 
+/* Expert routing that allocates no device memory and needs no handle.  The pages have no
+ * counterpart of this entry point: it exists for callers that cannot call cudaMalloc where
+ * they route — a host application that gives all device memory to its own pool and allows no
+ * outside allocation, a real-time loop where an allocation (which can synchronise the
+ * device) is not acceptable, a plugin that only receives buffers from its host.
+ * Computes the same routing as dreamer_route_experts, on CUDA cores.
+ *   cfg      hidden, depth (L), n_experts (E), top_k (k <= 16), router_dim (d_r = 32, 64 or
+ *            128), dtype and rope_base are read; other fields are ignored.
+ *   y        [n_tokens][h] dtype, w_qE [h][d_r] dtype, k_E [E][d_r] dtype (unrotated),
+ *            bias_E [E] float32: inputs, device pointers, caller-owned.
+ *   idx      [n_tokens][k] int32, w [n_tokens][k] float32: outputs.  counts [E] int32 or
+ *            NULL: cleared, then the histogram of idx.
+ * Scratch: a fixed array of 4 MiB (1,048,576 floats) inside the library holds the expert keys
+ * turned by the depth RoPE of `depth`; E * d_r above 1,048,576 returns
+ * DREAMER_ERR_UNSUPPORTED before anything runs.  Every GPU that loads the library keeps the
+ * array until the process exits.  All calls share it and it keeps the last call's contents,
+ * so calls that overlap on the GPU (other streams, other host threads) race: serialise them.
+ * The first call on a device looks up the array's device address and caches it; make that
+ * first call before any stream capture on the device.                                      */
+int dreamer_route_experts_noalloc(const dreamer_config *cfg, int depth, const void *y,
+                                  int n_tokens, const void *w_qE, const void *k_E,
+                                  const float *bias_E, int32_t *idx, float *w,
+                                  int32_t *counts, dreamer_stream stream);
+
 /* Bias balance update from the handle's last route counts ([notes] "Key design 2"):
  * b_e <- b_e + lambda * sign(median(N) - N_e), N_e = sum over depths, lower median for an
  * even E.  Updates the handle's bias; if bias_out is not NULL also copies the new bias
