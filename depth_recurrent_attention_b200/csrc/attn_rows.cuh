@@ -1,0 +1,200 @@
+// Attention of one query row over a run of key/value rows, HBM-bound form (bf16 / fp32).
+// Used for depth attention (the token's own depth states 0..l; papernotes "Key design 1":
+// DA looks back over the token's earlier depth states) and for decode attention over the
+// per-depth SA cache (split over key ranges, then merged).
+//
+// Layout of the work inside a warp: a key row of D elements is CH = D / VEC chunks of 16
+// bytes; lane = r * CH + c owns chunk c of row r of a group of RPW = 32 / CH rows.  A warp
+// issues U groups of K and V loads (2U independent 16-byte loads per lane) before using any
+// of them, reduces the partial dot products over the CH lanes of a row with shuffles, keeps an
+// online softmax over groups, and reduces the output chunks over the RPW rows at the end.
+#pragma once
+#include "common.cuh"
+
+namespace dreamer {
+
+template <typename T> struct VecOf;
+template <> struct VecOf<bf16> { static constexpr int N = 8; };
+template <> struct VecOf<float> { static constexpr int N = 4; };
+
+__device__ __forceinline__ void ld16(const bf16 *p, float *o) { load8(p, o); }
+__device__ __forceinline__ void ld16(const float *p, float *o) {
+  float4 a = *reinterpret_cast<const float4 *>(p);
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+}
+__device__ __forceinline__ void st16(bf16 *p, const float *v) { store8(p, v); }
+__device__ __forceinline__ void st16(float *p, const float *v) {
+  *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+
+struct RowsArgs {
+  int mode;            // 0 depth attention, 2 decode attention (split)
+  int n_q, H, h, L, l;
+  const void *q;       // [n_q][ldq], head at column head * D
+  long ldq;
+  const void *kv;      // mode 0: da_kv [T][L][2][h]; mode 2: k cache [L][B][H][cap][D]
+  const void *vc;      // mode 2: v cache
+  int B, cap, nsplit;
+  const int *cache_len;
+  int *err;
+  void *out;           // mode 0: attn [n_q][ldo] at column col0 + head * D
+  long ldo;
+  int col0;
+  float *part;         // mode 2: [n_q][H][nsplit][D + 2] partial (o, m, l)
+};
+
+template <typename T, int D, int U>
+__global__ void __launch_bounds__(256) attn_rows_kernel(RowsArgs a) {
+  constexpr int VEC = VecOf<T>::N;
+  constexpr int CH = D / VEC;
+  static_assert(CH >= 1 && CH <= 32 && (32 % CH) == 0, "chunking");
+  constexpr int RPW = 32 / CH;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int c = lane % CH, r = lane / CH;
+  const int splits = a.mode == 2 ? a.nsplit : 1;
+  if (gw >= a.n_q * a.H * splits) return;
+  const int sp = gw % splits;
+  const int qh = gw / splits;
+  const int qi = qh / a.H, head = qh % a.H;
+
+  const T *Kb, *Vb;
+  long ldk;
+  int j0, j1;
+  if (a.mode == 0) {
+    const T *base = reinterpret_cast<const T *>(a.kv);
+    Kb = base + ((long)qi * a.L * 2) * a.h + head * D;
+    Vb = Kb + a.h;
+    ldk = 2L * a.h;
+    j0 = 0;
+    j1 = a.l + 1;
+  } else {
+    const int len = a.cache_len[qi];
+    if (len < 0 || len >= a.cap) {  // slot outside the cache: report, attend to nothing
+      if (lane == 0) raise_dev_error(a.err, DEV_BAD_INDEX);
+      return;
+    }
+    const long off = ((((long)a.l * a.B + qi) * a.H + head) * a.cap) * D;
+    Kb = reinterpret_cast<const T *>(a.kv) + off;
+    Vb = reinterpret_cast<const T *>(a.vc) + off;
+    ldk = D;
+    const int nk = len + 1;
+    const int per = (nk + splits - 1) / splits;
+    j0 = sp * per;
+    j1 = min(nk, j0 + per);
+  }
+  float q[VEC];
+  ld16(reinterpret_cast<const T *>(a.q) + (long)qi * a.ldq + head * D + c * VEC, q);
+  const float sl2 = 1.4426950408889634f * rsqrtf((float)D);
+#pragma unroll
+  for (int i = 0; i < VEC; i++) q[i] *= sl2;  // scores in log2 units
+
+  float m = -INFINITY, lsum = 0.f;
+  float o[VEC];
+#pragma unroll
+  for (int i = 0; i < VEC; i++) o[i] = 0.f;
+
+  for (int g = j0; g < j1; g += U * RPW) {
+    float kv[U][VEC], vv[U][VEC];
+    bool ok[U];
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const int j = g + u * RPW + r;
+      ok[u] = j < j1;
+      if (ok[u]) {
+        ld16(Kb + (long)j * ldk + c * VEC, kv[u]);
+        ld16(Vb + (long)j * ldk + c * VEC, vv[u]);
+      }
+    }
+    float s[U];
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      float p = 0.f;
+#pragma unroll
+      for (int i = 0; i < VEC; i++) p = fmaf(q[i], ok[u] ? kv[u][i] : 0.f, p);
+#pragma unroll
+      for (int o2 = 1; o2 < CH; o2 <<= 1) p += __shfl_xor_sync(0xffffffffu, p, o2);
+      s[u] = ok[u] ? p : -INFINITY;
+    }
+    float gm = s[0];
+#pragma unroll
+    for (int u = 1; u < U; u++) gm = fmaxf(gm, s[u]);
+    gm = warp_max(gm);
+    const float mn = fmaxf(m, gm);
+    const float alpha = exp2f(m - mn);
+    float ps = 0.f;
+#pragma unroll
+    for (int i = 0; i < VEC; i++) o[i] *= alpha;
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const float p = ok[u] ? exp2f(s[u] - mn) : 0.f;
+      ps += p;
+#pragma unroll
+      for (int i = 0; i < VEC; i++) o[i] = fmaf(p, ok[u] ? vv[u][i] : 0.f, o[i]);
+    }
+    // row sums: each row's p sits on its CH lanes, count it once
+    ps = warp_sum(c == 0 ? ps : 0.f);
+    lsum = lsum * alpha + ps;
+    m = mn;
+  }
+  // reduce the output chunks over the RPW rows of the warp
+#pragma unroll
+  for (int o2 = CH; o2 < 32; o2 <<= 1)
+#pragma unroll
+    for (int i = 0; i < VEC; i++) o[i] += __shfl_xor_sync(0xffffffffu, o[i], o2);
+  if (a.mode == 0) {
+    if (r == 0) {
+      const float inv = 1.0f / lsum;
+#pragma unroll
+      for (int i = 0; i < VEC; i++) o[i] *= inv;
+      st16(reinterpret_cast<T *>(a.out) + (long)qi * a.ldo + a.col0 + head * D + c * VEC, o);
+    }
+  } else {
+    float *pp = a.part + ((long)qh * splits + sp) * (D + 2);
+    if (r == 0) {
+#pragma unroll
+      for (int i = 0; i < VEC; i++) pp[c * VEC + i] = o[i];
+    }
+    if (lane == 0) {
+      pp[D] = m;
+      pp[D + 1] = lsum;
+    }
+  }
+}
+
+// Merge the split partials of decode attention: o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) attn_merge_kernel(RowsArgs a) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= a.n_q * a.H) return;
+  const int qi = gw / a.H, head = gw % a.H;
+  const float *pp = a.part + (long)gw * a.nsplit * (D + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < a.nsplit; s++) M = fmaxf(M, pp[s * (D + 2) + D]);
+  float den = 0.f;
+  constexpr int PER = (D + 31) / 32;
+  float acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; i++) acc[i] = 0.f;
+  for (int s = 0; s < a.nsplit; s++) {
+    const float ms = pp[s * (D + 2) + D];
+    if (ms == -INFINITY) continue;  // empty split
+    const float f = exp2f(ms - M);
+    den += f * pp[s * (D + 2) + D + 1];
+#pragma unroll
+    for (int i = 0; i < PER; i++) {
+      const int dd = lane + 32 * i;
+      if (dd < D) acc[i] = fmaf(f, pp[s * (D + 2) + dd], acc[i]);
+    }
+  }
+  T *dst = reinterpret_cast<T *>(a.out) + (long)qi * a.ldo + a.col0 + head * D;
+  const float inv = 1.0f / den;
+#pragma unroll
+  for (int i = 0; i < PER; i++) {
+    const int dd = lane + 32 * i;
+    if (dd < D) dst[dd] = from_f<T>(acc[i] * inv);
+  }
+}
+
+}  // namespace dreamer

@@ -12,6 +12,7 @@
 #include "../../include/dreamer.h"
 #include "common.cuh"
 #include "kernels_simt.cuh"
+#include "attn_rows.cuh"
 
 using namespace dreamer;
 
@@ -37,6 +38,8 @@ struct dreamer_handle {
   void *u = nullptr, *da_kv_int = nullptr, *Hbuf = nullptr, *qsplit = nullptr;
   float *acc = nullptr, *zbuf = nullptr, *qbuf = nullptr, *psig = nullptr, *ew = nullptr;
   float *inv_rms = nullptr;      // [T] 1/rms of the current depth's residual
+  float *part = nullptr;         // decode attention split partials [B][H][nsplit][d + 2]
+  int nsplit = 1;
   int *pidx = nullptr, *eidx = nullptr, *counts = nullptr, *ecnt = nullptr, *eoffs = nullptr;
   int *etiles_a = nullptr, *etiles_b = nullptr, *ecursor = nullptr, *erows = nullptr;
   int *pcnt = nullptr, *poffs = nullptr, *ptiles_a = nullptr, *ptiles_b = nullptr;
@@ -86,7 +89,8 @@ static void mark(dreamer_handle *h, cudaStream_t s, int stage) {
   h->ev_stage[h->ev_used] = stage;
   h->ev_used++;
 }
-#define LAUNCHED(n) (h->launches += (n))
+// kernels launched by this thread through the library (read as deltas around each call)
+#define LAUNCHED(n) ((void)0)
 
 static void accumulate_marks(dreamer_handle *h, const std::vector<cudaEvent_t> &evs,
                              const std::vector<int> &stages) {
@@ -131,6 +135,8 @@ static int dalloc(dreamer_handle *h, void **p, size_t bytes) {
   } while (0)
 
 static inline int cdiv(long a, long b) { return (int)((a + b - 1) / b); }
+// kernels launched by this thread through the library (read as deltas around each call)
+static thread_local uint64_t g_launches = 0;
 
 #include "tc_kernels.cuh"
 
@@ -235,6 +241,7 @@ template <typename T>
 static void launch_transpose(const void *src, const void *sh, void *dst, int rows, int cols,
                              int G, cudaStream_t s) {
   dim3 grid(cdiv(cols, 32), cdiv(rows, 32), G), block(32, 8);
+  ++g_launches;
   transpose_absorb_kernel<T><<<grid, block, 0, s>>>((const T *)src, (const T *)sh, (T *)dst,
                                                      rows, cols, G);
 }
@@ -347,6 +354,11 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     DALLOC(h->prows, T * sizeof(int));
     DALLOC(h->pinv, T * sizeof(int));
     DALLOC(h->err, sizeof(int));
+    if (c.max_cache_len > 0) {
+      h->nsplit = (c.max_cache_len + 255) / 256;
+      if (h->nsplit > 64) h->nsplit = 64;
+      DALLOC(h->part, (size_t)c.batch * c.n_heads * h->nsplit * (d + 2) * sizeof(float));
+    }
     CK(cudaMemset(h->err, 0, sizeof(int)));
     CK(cudaMemset(h->counts, 0, (size_t)L * E * sizeof(int)));
     int r3 = tc_init(h);
@@ -414,6 +426,7 @@ extern "C" void dreamer_destroy(dreamer_handle *h) {
 template <typename TA, typename TB, int SEG, class Epi>
 static void gemm_simt(const GemmArgs &a, int max_tiles, const Epi &epi, cudaStream_t s) {
   dim3 grid(max_tiles, cdiv(a.N, 128));
+  ++g_launches;
   gemm_simt_kernel<TA, TB, SEG, Epi><<<grid, 256, 0, s>>>(a, epi);
 }
 
@@ -430,10 +443,32 @@ static void launch_attn(const AttnArgs &a, int d, cudaStream_t s) {
   const int warps = a.n_q * a.H;
   const int blocks = cdiv(warps, 8);
   switch (d) {
-    case 16: attn_warp_kernel<T, 16><<<blocks, 256, 0, s>>>(a); break;
-    case 32: attn_warp_kernel<T, 32><<<blocks, 256, 0, s>>>(a); break;
-    case 64: attn_warp_kernel<T, 64><<<blocks, 256, 0, s>>>(a); break;
-    default: attn_warp_kernel<T, 128><<<blocks, 256, 0, s>>>(a); break;
+    case 16: ++g_launches; attn_warp_kernel<T, 16><<<blocks, 256, 0, s>>>(a); break;
+    case 32: ++g_launches; attn_warp_kernel<T, 32><<<blocks, 256, 0, s>>>(a); break;
+    case 64: ++g_launches; attn_warp_kernel<T, 64><<<blocks, 256, 0, s>>>(a); break;
+    default: ++g_launches; attn_warp_kernel<T, 128><<<blocks, 256, 0, s>>>(a); break;
+  }
+}
+
+// depth attention (mode 0) or split decode attention + merge (mode 2)
+template <typename T>
+static void launch_rows(const RowsArgs &a, int d, cudaStream_t s) {
+  const long warps = (long)a.n_q * a.H * (a.mode == 2 ? a.nsplit : 1);
+  const int blocks = cdiv(warps, 8);
+  switch (d) {
+    case 16: ++g_launches; attn_rows_kernel<T, 16, 4><<<blocks, 256, 0, s>>>(a); break;
+    case 32: ++g_launches; attn_rows_kernel<T, 32, 4><<<blocks, 256, 0, s>>>(a); break;
+    case 64: ++g_launches; attn_rows_kernel<T, 64, 4><<<blocks, 256, 0, s>>>(a); break;
+    default: ++g_launches; attn_rows_kernel<T, 128, 4><<<blocks, 256, 0, s>>>(a); break;
+  }
+  if (a.mode == 2) {
+    const int mb = cdiv((long)a.n_q * a.H, 8);
+    switch (d) {
+      case 16: ++g_launches; attn_merge_kernel<T, 16><<<mb, 256, 0, s>>>(a); break;
+      case 32: ++g_launches; attn_merge_kernel<T, 32><<<mb, 256, 0, s>>>(a); break;
+      case 64: ++g_launches; attn_merge_kernel<T, 64><<<mb, 256, 0, s>>>(a); break;
+      default: ++g_launches; attn_merge_kernel<T, 128><<<mb, 256, 0, s>>>(a); break;
+    }
   }
 }
 
@@ -467,6 +502,7 @@ static void route_rows(dreamer_handle *h, int mode, int l, const void *X, int n,
   t.z = h->zbuf; t.ldz = ldz; t.zscale = 1.0f / sqrtf((float)dr);
   t.bias = mode == 0 ? h->bias : nullptr;
   t.idx = idx; t.w = wout; t.counts_a = counts_a; t.counts_b = counts_b;
+  ++g_launches;
   topk_kernel<<<cdiv(n, 8), 256, 0, s>>>(t);
 }
 
@@ -491,6 +527,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
   // 1. RMSNorm of the residual stream (x_0 on the first depth, else the fp32 accumulator)
   mark(h, s, DREAMER_STAGE_NORM);
   LAUNCHED(1);
+  ++g_launches;
   rmsnorm_kernel<T><<<cdiv(n, 8), 256, 0, s>>>(first ? (const T *)io.x_in : nullptr,
                                                first ? nullptr : h->acc, (const T *)h->g,
                                                (T *)h->xh, h->inv_rms, n, hd, c.rms_eps);
@@ -501,9 +538,12 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
     mark(h, s, DREAMER_STAGE_PROJ_ROUTE);
     LAUNCHED(2);
     cudaMemsetAsync(h->pcnt, 0, (G + 1) * sizeof(int), s);
-    route_rows<T>(h, 1, l, h->xh, n, h->pidx, h->psig, nullptr, h->pcnt, s);
+    if (!(tc && tc_proj_route(h, l, h->xh, n, s)))
+      route_rows<T>(h, 1, l, h->xh, n, h->pidx, h->psig, nullptr, h->pcnt, s);
+    ++g_launches;
     scan_kernel<<<1, 1024, 0, s>>>(h->pcnt, G, h->poffs, h->ptiles_a, 64, h->ptiles_b, 128,
                                    h->pcursor);
+    ++g_launches;
     scatter_kernel<<<cdiv(n, 256), 256, 0, s>>>(h->pidx, n, h->pcursor, h->prows, h->pinv);
     prow = h->prows;
     psig = h->psig;
@@ -525,10 +565,15 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
   eq.k_cache = (T *)io.k_cache; eq.v_cache = (T *)io.v_cache; eq.cache_len = io.cache_len;
   eq.B = c.batch; eq.cap = c.max_cache_len; eq.err = h->err;
 
-  AttnArgs da{};
-  da.mode = 0; da.n_q = n; da.H = c.n_heads; da.d = d; da.h = hd;
-  da.q = h->q_da; da.ldq = hd; da.kv = io.da_kv; da.L = L; da.l = l;
-  da.out = h->attn; da.ldo = 2 * hd; da.col0 = hd;
+  RowsArgs da{};
+  da.mode = 0; da.n_q = n; da.H = c.n_heads; da.h = hd; da.L = L; da.l = l;
+  da.q = h->q_da; da.ldq = hd; da.kv = io.da_kv;
+  da.out = h->attn; da.ldo = 2 * hd; da.col0 = hd; da.err = h->err;
+  RowsArgs sd{};  // decode: attention over the per-depth SA cache, split over key ranges
+  sd.mode = 2; sd.n_q = n; sd.H = c.n_heads; sd.h = hd; sd.L = L; sd.l = l;
+  sd.q = h->qkv_sa; sd.ldq = 3 * hd; sd.kv = io.k_cache; sd.vc = io.v_cache;
+  sd.B = c.batch; sd.cap = c.max_cache_len; sd.nsplit = h->nsplit; sd.cache_len = io.cache_len;
+  sd.err = h->err; sd.out = h->attn; sd.ldo = 2 * hd; sd.col0 = 0; sd.part = h->part;
   AttnArgs sa{};
   sa.mode = io.mode == 0 ? 1 : 2; sa.n_q = n; sa.H = c.n_heads; sa.d = d; sa.h = hd;
   sa.q = h->qkv_sa; sa.ldq = 3 * hd; sa.kv = io.mode == 0 ? h->qkv_sa : io.k_cache;
@@ -536,6 +581,15 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
   sa.cap = c.max_cache_len; sa.cache_len = io.cache_len; sa.err = h->err;
   sa.out = h->attn; sa.ldo = 2 * hd; sa.col0 = 0;
 
+  // SA: tcgen05 flash kernel for bf16 prefill, split decode attention for decode, the warp
+  // kernel for float32 prefill
+  auto run_sa = [&](cudaStream_t st) {
+    if (io.mode == 1) {
+      launch_rows<T>(sd, d, st);
+      return;
+    }
+    if (!(tc && tc_sa_ok(h) && tc_sa(h, st))) launch_attn<T>(sa, d, st);
+  };
   auto qkv_gemm = [&](const void *A, int col0, int ncols) {
     // columns [col0, col0 + ncols) of the fused QKV projection
     mark(h, s, DREAMER_STAGE_QKV);
@@ -572,12 +626,12 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
     qkv_gemm(h->xh, 3 * hd, 3 * hd);
     mark(h, s, DREAMER_STAGE_DA);
     LAUNCHED(1);
-    launch_attn<T>(da, d, s);
+    launch_rows<T>(da, d, s);
     o_gemm((const T *)h->attn + hd, hd, hd, res_xhat, h->u);   // u = x^ + DA part (acc = u)
     qkv_gemm(h->u, 0, 3 * hd);
     mark(h, s, DREAMER_STAGE_SA);
-    LAUNCHED(1);
-    if (!(io.mode == 0 && tc && tc_sa_ok(h) && tc_sa(h, s))) launch_attn<T>(sa, d, s);
+    LAUNCHED(io.mode == 1 ? 2 : 1);
+    run_sa(s);
     o_gemm(h->attn, 0, hd, 2, h->y);                            // y = u + SA part
   } else {
     // 3. fused QKV projection with RoPE / depth RoPE epilogue, DA KV write
@@ -585,18 +639,18 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
     // 4. DA || SA (papernotes "Key design 1": run in parallel for throughput).  DA runs
     // on the side stream beside SA (two branches of the captured graph); with stage
     // profiling on they run one after the other so each stage's time is its own.
-    LAUNCHED(2);
+    LAUNCHED(io.mode == 1 ? 3 : 2);
     if (h->prof) {
       mark(h, s, DREAMER_STAGE_DA);
-      launch_attn<T>(da, d, s);
+      launch_rows<T>(da, d, s);
     } else {
       cudaEventRecord(h->ev_fork, s);
       cudaStreamWaitEvent(h->side, h->ev_fork, 0);
-      launch_attn<T>(da, d, h->side);
+      launch_rows<T>(da, d, h->side);
       cudaEventRecord(h->ev_join, h->side);
     }
     mark(h, s, DREAMER_STAGE_SA);
-    if (!(io.mode == 0 && tc && tc_sa_ok(h) && tc_sa(h, s))) launch_attn<T>(sa, d, s);
+    run_sa(s);
     if (!h->prof) cudaStreamWaitEvent(s, h->ev_join, 0);
     // 5. O projection, residual y = x^ + DA + SA
     o_gemm(h->attn, 0, 2 * hd, res_xhat, h->y);
@@ -608,8 +662,10 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
   cudaMemsetAsync(h->ecnt, 0, E * sizeof(int), s);
   route_rows<T>(h, 0, l, ein, n, h->eidx, h->ew, h->counts + (size_t)l * E, h->ecnt, s);
   mark(h, s, DREAMER_STAGE_PERMUTE);
+  ++g_launches;
   scan_kernel<<<1, 1024, 0, s>>>(h->ecnt, E, h->eoffs, h->etiles_a, 64, h->etiles_b, 128,
                                  h->ecursor);
+  ++g_launches;
   scatter_kernel<<<cdiv((long)n * k, 256), 256, 0, s>>>(h->eidx, n * k, h->ecursor, h->erows,
                                                          nullptr);
   // 7. expert FFNs: H = SiLU(X W1_e), acc[token] += w * H W2_e
@@ -718,7 +774,7 @@ static int run_graphed(dreamer_handle *h, int kind, const void *const key[5], in
   e->last_use = ++h->use_clock;
   if (!e->captured) {
     const size_t ev0 = h->ev_used;
-    const uint64_t l_before = h->launches;
+    const uint64_t l_before = g_launches;
     cudaGraph_t graph = nullptr;
     if (cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
       cudaGetLastError();
@@ -726,9 +782,10 @@ static int run_graphed(dreamer_handle *h, int kind, const void *const key[5], in
     }
     int rc = enqueue();
     cudaError_t ce = cudaStreamEndCapture(s, &graph);
-    const uint64_t n_launch = h->launches - l_before;
-    h->launches = l_before;
+    const uint64_t n_launch = g_launches - l_before;
+    g_launches = l_before;  // captured kernels run when the graph is launched
     if (rc != DREAMER_OK || ce != cudaSuccess || !graph) {
+      g_launches = l_before;
       if (graph) cudaGraphDestroy(graph);
       cudaGetLastError();
       h->ev_used = ev0;
@@ -753,7 +810,7 @@ static int run_graphed(dreamer_handle *h, int kind, const void *const key[5], in
     h->ev_used = ev0;
   }
   CK(cudaGraphLaunch(e->exec, s));
-  h->launches += e->launches;
+  g_launches += e->launches;
   if (e->prof && !e->evs.empty()) {
     CK(cudaStreamSynchronize(s));
     accumulate_marks(h, e->evs, e->stages);
@@ -777,6 +834,7 @@ static int forward_impl(dreamer_handle *h, const void *x_in, void *x_out, int l0
   if (l1 > l0) {
     LAUNCHED(1);
     long tot = (long)n * c.hidden;
+    ++g_launches;
     finish_kernel<T><<<cdiv(tot / 8, 256), 256, 0, s>>>(h->acc, (T *)x_out, tot);
   } else if (x_out != x_in) {
     CK(cudaMemcpyAsync(x_out, x_in, (size_t)n * c.hidden * h->esz, cudaMemcpyDeviceToDevice, s));
@@ -802,9 +860,16 @@ extern "C" int dreamer_core_forward(dreamer_handle *h, const void *x_in, void *x
     return c.dtype == 0 ? forward_impl<float>(h, x_in, x_out, depth_begin, depth_end, da_kv, trace, s)
                         : forward_impl<bf16>(h, x_in, x_out, depth_begin, depth_end, da_kv, trace, s);
   };
-  if (trace) return enqueue();
-  const void *key[5] = {x_in, x_out, da_kv, nullptr, nullptr};
-  return run_graphed(h, 0, key, depth_begin, depth_end, s, enqueue);
+  const uint64_t l0c = g_launches;
+  int rc;
+  if (trace) {
+    rc = enqueue();
+  } else {
+    const void *key[5] = {x_in, x_out, da_kv, nullptr, nullptr};
+    rc = run_graphed(h, 0, key, depth_begin, depth_end, s, enqueue);
+  }
+  h->launches += g_launches - l0c;
+  return rc;
 }
 
 template <typename T>
@@ -823,6 +888,7 @@ static int decode_impl(dreamer_handle *h, const void *x_new, void *kc, void *vc,
   mark(h, s, DREAMER_STAGE_FINISH);
   LAUNCHED(1);
   long tot = (long)n * c.hidden;
+  ++g_launches;
   finish_kernel<T><<<cdiv(tot / 8, 256), 256, 0, s>>>(h->acc, (T *)x_out, tot);
   CK(cudaMemcpyAsync(h->err_host, h->err, sizeof(int), cudaMemcpyDeviceToHost, s));
   mark(h, s, DREAMER_N_STAGES);
@@ -845,9 +911,16 @@ extern "C" int dreamer_decode_step(dreamer_handle *h, const void *x_new, void *k
                ? decode_impl<float>(h, x_new, k_cache, v_cache, cache_len, x_out, trace, s)
                : decode_impl<bf16>(h, x_new, k_cache, v_cache, cache_len, x_out, trace, s);
   };
-  if (trace) return enqueue();
-  const void *key[5] = {x_new, k_cache, v_cache, cache_len, x_out};
-  return run_graphed(h, 1, key, 0, h->cfg.depth, s, enqueue);
+  const uint64_t l0c = g_launches;
+  int rc;
+  if (trace) {
+    rc = enqueue();
+  } else {
+    const void *key[5] = {x_new, k_cache, v_cache, cache_len, x_out};
+    rc = run_graphed(h, 1, key, 0, h->cfg.depth, s, enqueue);
+  }
+  h->launches += g_launches - l0c;
+  return rc;
 }
 
 extern "C" int dreamer_route_counts(dreamer_handle *h, int32_t *counts, int on_host,
@@ -892,6 +965,7 @@ extern "C" int dreamer_bias_update(dreamer_handle *h, float lambda, float *bias_
   cudaStream_t s = (cudaStream_t)stream;
   if (smem > 48 * 1024)
     CK(cudaFuncSetAttribute(bias_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  ++g_launches;
   bias_update_kernel<<<1, 1024, smem, s>>>(h->counts, h->cfg.depth, E, lambda, h->bias, bias_out);
   CK(cudaGetLastError());
   return DREAMER_OK;

@@ -30,6 +30,11 @@ struct TcGemmArgs {
   int *err;
 };
 
+// per-row epilogue state: Epi::State for row-pass epilogues, nothing otherwise
+struct NoEpiState {};
+template <class Epi, bool ROWPASS> struct EpiState { using type = NoEpiState; };
+template <class Epi> struct EpiState<Epi, true> { using type = typename Epi::State; };
+
 __device__ __forceinline__ bool tc_tile_rows(const TcGemmArgs &a, int mt, int &g, int &m0,
                                              int &m1) {
   if (!a.goffs) {
@@ -64,7 +69,10 @@ struct TcGemmCfg {
   static_assert(!GATHER || BK == 64, "gathered rows use 128-byte K blocks");
 };
 
-template <int BN, int BK, int STAGES, bool GATHER, int SEG, class Epi>
+// ROWPASS: a CTA takes row tiles mt = blockIdx.x, blockIdx.x + gridDim.x, ... and runs all
+// N tiles of each in order, so the epilogue can carry per-row state across the N tiles
+// (Epi::State with row_begin / row_apply / row_end); otherwise tiles are strided over CTAs.
+template <int BN, int BK, int STAGES, bool GATHER, int SEG, class Epi, bool ROWPASS = false>
 __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    TcGemmArgs a, Epi epi) {
@@ -83,6 +91,18 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
   const int mtiles = a.goffs ? a.tiles[a.G] : (a.M + 127) / 128;
   const int total = mtiles * NT;
   const int KB = a.K / BK;
+  // the i-th tile of this CTA (identical sequence in every role); false past the last one
+  auto tile_at = [&](int i, int &mt, int &nt) -> bool {
+    if (ROWPASS) {
+      mt = blockIdx.x + (i / NT) * gridDim.x;
+      nt = i % NT;
+      return mt < mtiles;
+    }
+    const int t = blockIdx.x + i * gridDim.x;
+    mt = t / NT;
+    nt = t % NT;
+    return t < total;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; s++) {
@@ -115,9 +135,10 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
       int issued_ph[STAGES];
       for (int i = 0; i < STAGES; i++) issued_ph[i] = -1;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      int mt, nt;
+      for (int i = 0; ok && tile_at(i, mt, nt); i++) {
         int g, m0, m1;
-        const int mt = t / NT, n0 = (t % NT) * BN;
+        const int n0 = nt * BN;
         tc_tile_rows(a, mt, g, m0, m1);
         const int brow = g * a.b_group_rows + a.b_row0 + n0;
         for (int kb = 0; kb < KB; kb++) {
@@ -145,9 +166,9 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
-      int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, it++) {
+      int mt, nt;
+      for (int it = 0; ok && tile_at(it, mt, nt); it++) {
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         if (!mbar_wait(smem_u32(&tempty[acc]), aph ^ 1, abort_flag, a.err)) break;
@@ -172,19 +193,23 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
     // ------------------------------------------------------------- epilogue
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    int it = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, it++) {
+    int mt, nt;
+    typename EpiState<Epi, ROWPASS>::type st;
+    for (int it = 0; tile_at(it, mt, nt); it++) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       if (!mbar_wait(smem_u32(&tfull[acc]), aph, abort_flag, a.err)) break;
       tc_fence_after();
       int g, m0, m1;
-      const int mt = t / NT, n0 = (t % NT) * BN;
+      const int n0 = nt * BN;
       tc_tile_rows(a, mt, g, m0, m1);
       const int r = m0 + row;
       const bool valid = r < m1;
       const int token = valid ? (a.arow ? a.arow[r] / a.arow_div : r) : 0;
       const uint32_t base = tmem + acc * BN + ((uint32_t)(q * 32) << 16);
+      if constexpr (ROWPASS) {
+        if (nt == 0) epi.row_begin(st);
+      }
 #pragma unroll 1
       for (int sg = 0; sg < BN / SEG; sg++) {
         float v[SEG];
@@ -194,10 +219,16 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
         } else {
           tmem_ld16(base + sg * SEG, v);
         }
-        if (valid) epi.template operator()<SEG>(r, token, g, n0 + sg * SEG, v);
+        if (valid) {
+          if constexpr (ROWPASS) epi.template row_apply<SEG>(st, r, token, g, n0 + sg * SEG, v);
+          else epi.template operator()<SEG>(r, token, g, n0 + sg * SEG, v);
+        }
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&tempty[acc]));
+      if constexpr (ROWPASS) {
+        if (nt == NT - 1 && valid) epi.row_end(st, r, token);
+      }
     }
   } else if (GATHER) {
     // ------------------------------------------------------------- gathered A producers

@@ -68,6 +68,108 @@ struct EpiDownVec {
   }
 };
 
+// Expert-attention top-k fused into the score GEMM (row-pass epilogue): each thread owns one
+// token's row, walks all E scores tile by tile and keeps its best KT by z + b (lower expert
+// index on exact ties) in registers (papernotes "Key design 2": sigma(x) = norm(TopK(
+// sigmoid(x), x + b, k))); at the row's end it writes the picks, the weights
+// sigmoid(z) / sum over the picks, and the two histograms (per-depth counts, per-call expert
+// sizes for the permutation).
+template <int KT>
+struct EpiTopK {
+  int E;
+  float zscale;
+  const float *bias;
+  int *idx;
+  float *w;
+  int *counts_a, *counts_b;
+  struct State {
+    float v[KT], z[KT];
+    int e[KT];
+  };
+  __device__ __forceinline__ static bool better(float v1, int e1, float v2, int e2) {
+    return v1 > v2 || (v1 == v2 && e1 < e2);
+  }
+  __device__ __forceinline__ void row_begin(State &s) const {
+#pragma unroll
+    for (int i = 0; i < KT; i++) {
+      s.v[i] = -INFINITY;
+      s.z[i] = 0.f;
+      s.e[i] = 0x7fffffff;
+    }
+  }
+  template <int SEG>
+  __device__ __forceinline__ void row_apply(State &s, int r, int token, int g, int n0,
+                                            const float *vals) const {
+#pragma unroll
+    for (int i = 0; i < SEG; i++) {
+      const int e = n0 + i;
+      float z = vals[i] * zscale;
+      float v = z + bias[e];
+      if (v != v) v = -INFINITY;
+      if (!better(v, e, s.v[KT - 1], s.e[KT - 1])) continue;
+      int ce = e;
+      float cv = v, cz = z;
+#pragma unroll
+      for (int j = 0; j < KT; j++) {  // insertion by compare-and-swap down the sorted list
+        if (better(cv, ce, s.v[j], s.e[j])) {
+          const float tv = s.v[j], tz = s.z[j];
+          const int te = s.e[j];
+          s.v[j] = cv; s.z[j] = cz; s.e[j] = ce;
+          cv = tv; cz = tz; ce = te;
+        }
+      }
+    }
+  }
+  __device__ __forceinline__ void row_end(State &s, int r, int token) const {
+    float sg[KT], sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < KT; i++) {
+      sg[i] = 1.0f / (1.0f + __expf(-s.z[i]));
+      sum += sg[i];
+    }
+    const float inv = 1.0f / sum;
+#pragma unroll
+    for (int i = 0; i < KT; i++) {
+      idx[(long)r * KT + i] = s.e[i];
+      w[(long)r * KT + i] = sg[i] * inv;
+      if (counts_a) atomicAdd(counts_a + s.e[i], 1);
+      if (counts_b) atomicAdd(counts_b + s.e[i], 1);
+    }
+  }
+};
+
+// Projection router fused into its query GEMM epilogue (papernotes "Key design 3", reading
+// R12): the thread holds q_P = x^ W_qP (fp32) of its token, scores it against the P
+// depth-rotated projection keys, takes the argmax (lower index on ties), sigma = sigmoid(max)
+// and counts the token into its group.
+struct EpiProjRoute {
+  int P, dr;
+  float zscale;
+  const float *keys;   // [P][d_r] fp32, rotated to the current depth
+  int *pidx;
+  float *psig;
+  int *pcount;
+  template <int SEG>
+  __device__ __forceinline__ void operator()(int r, int token, int g, int n0, float *v) const {
+    float best = -INFINITY;
+    int bi = 0;
+    for (int p = 0; p < P; p++) {
+      const float *kr = keys + (long)p * SEG;
+      float z = 0.f;
+#pragma unroll
+      for (int i = 0; i < SEG; i++) z = fmaf(v[i], kr[i], z);
+      z *= zscale;
+      if (z > best) {  // strict: the lower index keeps ties
+        best = z;
+        bi = p;
+      }
+    }
+    pidx[r] = bi;
+    psig[r] = 1.0f / (1.0f + __expf(-best));
+    atomicAdd(pcount + bi, 1);
+  }
+};
+
 }  // namespace dreamer
 
 typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -126,11 +228,12 @@ static int tc_init(dreamer_handle *h) {
 
 static void tc_destroy(dreamer_handle *h) {}
 
-template <int BN, int BK, int ST, bool GATHER, int SEG, class Epi>
+template <int BN, int BK, int ST, bool GATHER, int SEG, class Epi, bool ROWPASS = false>
 static void tc_launch(dreamer_handle *h, const dreamer::tc::TcGemmArgs &a, const CUtensorMap &ta,
                       const CUtensorMap &tb, long max_tiles, const Epi &epi, cudaStream_t s) {
   using Cfg = dreamer::tc::TcGemmCfg<BN, BK, ST, GATHER>;
-  auto kern = dreamer::tc::tc_gemm_kernel<BN, BK, ST, GATHER, SEG, Epi>;
+  auto kern = dreamer::tc::tc_gemm_kernel<BN, BK, ST, GATHER, SEG, Epi, ROWPASS>;
+  if (ROWPASS) max_tiles /= (a.N / BN);  // one unit of work per row tile
   static bool attr_set = false;
   if (!attr_set) {
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
@@ -138,6 +241,7 @@ static void tc_launch(dreamer_handle *h, const dreamer::tc::TcGemmArgs &a, const
   }
   long grid = max_tiles < h->num_sms ? max_tiles : h->num_sms;
   if (grid < 1) grid = 1;
+  ++g_launches;
   kern<<<(int)grid, Cfg::THREADS, Cfg::SMEM, s>>>(ta, tb, a, epi);
 }
 
@@ -241,12 +345,59 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
     if (!tc_prepare<128, 64>(h, qa, nullptr, n, t, ta, tb, mt)) return false;
     tc_launch<128, 64, 6, false, 128>(h, t, ta, tb, mt, eq, s);
   }
+  const float zs = 1.0f / sqrtf((float)dr);
+  // The fused top-k gives each 128-row tile to one CTA for all E columns: worth it only when
+  // there are enough row tiles to fill the GPU; otherwise scores go through memory and the
+  // warp top-k spreads the rows over every SM.
+  const int k_fused = (n + 127) / 128 >= h->num_sms / 2 ? c.top_k : 0;
+  switch (k_fused) {  // top-k fused into the score GEMM
+    case 4:
+      tc_launch<256, 64, 4, false, 32, EpiTopK<4>, true>(
+          h, t2, ta2, tb2, mt2, EpiTopK<4>{E, zs, h->bias, idx, w, counts_a, counts_b}, s);
+      return true;
+    case 8:
+      tc_launch<256, 64, 4, false, 32, EpiTopK<8>, true>(
+          h, t2, ta2, tb2, mt2, EpiTopK<8>{E, zs, h->bias, idx, w, counts_a, counts_b}, s);
+      return true;
+    case 16:
+      tc_launch<256, 64, 4, false, 32, EpiTopK<16>, true>(
+          h, t2, ta2, tb2, mt2, EpiTopK<16>{E, zs, h->bias, idx, w, counts_a, counts_b}, s);
+      return true;
+    default:
+      break;
+  }
   tc_launch<256, 64, 4, false, 32>(h, t2, ta2, tb2, mt2, EpiStoreF32{h->zbuf, h->ldz, E}, s);
   TopkArgs k{};
   k.n_tok = n; k.E = E; k.k = c.top_k; k.mode = 0;
   k.z = h->zbuf; k.ldz = h->ldz; k.zscale = 1.0f / sqrtf((float)dr);
   k.bias = h->bias; k.idx = idx; k.w = w; k.counts_a = counts_a; k.counts_b = counts_b;
+  ++g_launches;
   topk_kernel<<<(n + 7) / 8, 256, 0, s>>>(k);
+  return true;
+}
+
+// Projection router: q_P = x^ W_qP on the tensor cores, argmax over the P keys in the
+// epilogue.  Needs d_r in {64, 128} (the thread holds the whole query row).
+static bool tc_proj_route(dreamer_handle *h, int l, const void *X, int n, cudaStream_t s) {
+  using namespace dreamer;
+  const dreamer_config &c = h->cfg;
+  const int dr = c.router_dim, hd = c.hidden, P = c.n_proj_experts;
+  if (!g_encode_tiled || !(dr == 64 || dr == 128) || hd % 64) return false;
+  GemmArgs qa{};
+  qa.N = dr; qa.K = hd; qa.G = 1; qa.M = n; qa.arow_div = 1;
+  qa.A = X; qa.lda = hd; qa.B = h->wqP_t; qa.ldb = hd; qa.bgstride = 0;
+  tc::TcGemmArgs t{};
+  CUtensorMap ta, tb;
+  long mt;
+  EpiProjRoute e{P, dr, 1.0f / sqrtf((float)dr), h->kP_rot + (size_t)l * P * dr, h->pidx,
+                 h->psig, h->pcnt};
+  if (dr == 64) {
+    if (!tc_prepare<64, 64>(h, qa, nullptr, n, t, ta, tb, mt)) return false;
+    tc_launch<64, 64, 6, false, 64>(h, t, ta, tb, mt, e, s);
+  } else {
+    if (!tc_prepare<128, 64>(h, qa, nullptr, n, t, ta, tb, mt)) return false;
+    tc_launch<128, 64, 6, false, 128>(h, t, ta, tb, mt, e, s);
+  }
   return true;
 }
 
