@@ -197,4 +197,203 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(RowsArgs a) {
   }
 }
 
+
+// =======================================================================================
+// Depth attention, one CTA per token: the token's depth KV rows 0..l for all heads are one
+// contiguous run of the [T][L][2][h] buffer ((l + 1) * 2h elements), so thread 0 streams it
+// into shared memory with 1-D bulk TMA copies in chunks of CHUNK depths (two buffers), and
+// warp `head` attends over its head's slice of every row: score over d with a warp sum,
+// online softmax across rows, output chunk per lane (papernotes "Key design 1": DA attends
+// over the same token's states at depths 0..l).
+// =======================================================================================
+namespace tcda {
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ bool try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+}  // namespace tcda
+
+struct DaBulkArgs {
+  int n_tok, H, h, L, l, chunk;  // chunk: depths per shared-memory buffer
+  const void *q;                 // q_DA [T][h]
+  const void *kv;                // [T][L][2][h]
+  void *out;                     // attn [T][ldo], DA part at column col0
+  long ldo;
+  int col0;
+  int *err;
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
+  extern __shared__ __align__(128) uint8_t dsm[];
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ int abort_flag;
+  const int tok = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nrow = a.l + 1;
+  const long row_el = 2L * a.h;                        // elements of one depth row (K then V)
+  const uint32_t chunk_bytes = (uint32_t)(a.chunk * row_el * sizeof(T));
+  T *buf[2] = {reinterpret_cast<T *>(dsm), reinterpret_cast<T *>(dsm + chunk_bytes)};
+  const T *src = reinterpret_cast<const T *>(a.kv) + (long)tok * a.L * row_el;
+  const int nchunks = (nrow + a.chunk - 1) / a.chunk;
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tcda::smem_u32(&bars[0])) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tcda::smem_u32(&bars[1])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    abort_flag = 0;
+  }
+  __syncthreads();
+  auto issue = [&](int c) {
+    const int r0 = c * a.chunk, nr = min(a.chunk, nrow - r0);
+    const uint32_t bytes = (uint32_t)(nr * row_el * sizeof(T));
+    const uint32_t bar = tcda::smem_u32(&bars[c & 1]);
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+                 "r"(bytes)
+                 : "memory");
+    tcda::bulk_load(tcda::smem_u32(buf[c & 1]), src + (long)r0 * row_el, bytes, bar);
+  };
+  int issued = 0;  // chunks issued (thread 0's count)
+  if (threadIdx.x == 0) {
+    issue(0);
+    issued = 1;
+    if (nchunks > 1) {
+      issue(1);
+      issued = 2;
+    }
+  }
+  // row-group layout: CH lanes of 16 bytes cover a row, RPW rows per warp step
+  constexpr int VEC = VecOf<T>::N;
+  constexpr int CH = D / VEC;
+  constexpr int RPW = 32 / CH;
+  constexpr int U = 2;  // row groups per iteration (one max / sum reduction for U * RPW rows)
+  const int cc = lane % CH, rr = lane / CH;
+  const int head = warp;
+  const bool active = head < a.H;
+  float q[VEC], o[VEC];
+  const float sl2 = 1.4426950408889634f * rsqrtf((float)D);
+  if (active) ld16(reinterpret_cast<const T *>(a.q) + (long)tok * a.h + head * D + cc * VEC, q);
+#pragma unroll
+  for (int i = 0; i < VEC; i++) {
+    q[i] = active ? q[i] * sl2 : 0.f;
+    o[i] = 0.f;
+  }
+  float m = -INFINITY, lsum = 0.f;
+  int consumed = 0;
+  for (int c = 0; c < nchunks; c++) {
+    // wait for chunk c (bounded; on expiry every thread leaves the loop)
+    const uint32_t bar = tcda::smem_u32(&bars[c & 1]);
+    const uint32_t par = (c >> 1) & 1;
+    if (!tcda::try_wait(bar, par)) {
+      const uint64_t t0 = tcda::gtimer();
+      while (!tcda::try_wait(bar, par)) {
+        if (abort_flag) break;
+        if (tcda::gtimer() - t0 > 2000000000ull) {
+          abort_flag = 1;
+          raise_dev_error(a.err, DEV_TIMEOUT);
+          break;
+        }
+      }
+    }
+    if (abort_flag) break;
+    consumed = c + 1;
+    const T *bk = buf[c & 1];
+    const int nr = min(a.chunk, nrow - c * a.chunk);
+    if (active) {
+      for (int g = 0; g < nr; g += U * RPW) {
+        float s[U], vv[U][VEC];
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+          const int j = g + u * RPW + rr;
+          s[u] = -INFINITY;
+          if (j < nr) {
+            float kv[VEC];
+            const T *kr = bk + (long)j * row_el + head * D + cc * VEC;
+            ld16(kr, kv);
+            ld16(kr + a.h, vv[u]);
+            float p = 0.f;
+#pragma unroll
+            for (int i = 0; i < VEC; i++) p = fmaf(q[i], kv[i], p);
+            s[u] = p;
+          } else {
+#pragma unroll
+            for (int i = 0; i < VEC; i++) vv[u][i] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+          float p = s[u] == -INFINITY ? 0.f : s[u];
+#pragma unroll
+          for (int o2 = 1; o2 < CH; o2 <<= 1) p += __shfl_xor_sync(0xffffffffu, p, o2);
+          if (s[u] != -INFINITY) s[u] = p;
+        }
+        float gm = s[0];
+#pragma unroll
+        for (int u = 1; u < U; u++) gm = fmaxf(gm, s[u]);
+        gm = warp_max(gm);
+        const float mn = fmaxf(m, gm);
+        const float alpha = exp2f(m - mn);
+        float ps = 0.f;
+#pragma unroll
+        for (int i = 0; i < VEC; i++) o[i] *= alpha;
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+          const float p = s[u] == -INFINITY ? 0.f : exp2f(s[u] - mn);
+          ps += p;
+#pragma unroll
+          for (int i = 0; i < VEC; i++) o[i] = fmaf(p, vv[u][i], o[i]);
+        }
+        ps = warp_sum(cc == 0 ? ps : 0.f);
+        lsum = lsum * alpha + ps;
+        m = mn;
+      }
+    }
+    __syncthreads();  // every warp is done with buffer c & 1
+    if (threadIdx.x == 0 && c + 2 < nchunks) {
+      issue(c + 2);
+      issued = c + 3;
+    }
+  }
+  // reduce the output chunks over the RPW rows of the warp
+#pragma unroll
+  for (int o2 = CH; o2 < 32; o2 <<= 1)
+#pragma unroll
+    for (int i = 0; i < VEC; i++) o[i] += __shfl_xor_sync(0xffffffffu, o[i], o2);
+  if (active && !abort_flag && rr == 0) {
+    const float inv = 1.0f / lsum;
+#pragma unroll
+    for (int i = 0; i < VEC; i++) o[i] *= inv;
+    st16(reinterpret_cast<T *>(a.out) + (long)tok * a.ldo + a.col0 + head * D + cc * VEC, o);
+  }
+  // copies still in flight after an abort land before the CTA exits
+  if (threadIdx.x == 0 && abort_flag) {
+    for (int c = consumed; c < issued; c++) {
+      const uint64_t t0 = tcda::gtimer();
+      while (!tcda::try_wait(tcda::smem_u32(&bars[c & 1]), (c >> 1) & 1) &&
+             tcda::gtimer() - t0 < 2000000000ull) {
+      }
+    }
+  }
+}
+
 }  // namespace dreamer

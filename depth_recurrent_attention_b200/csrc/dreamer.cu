@@ -42,6 +42,8 @@ struct dreamer_handle {
   int nsplit = 1;
   int *pidx = nullptr, *eidx = nullptr, *counts = nullptr, *ecnt = nullptr, *eoffs = nullptr;
   int *etiles_a = nullptr, *etiles_b = nullptr, *ecursor = nullptr, *erows = nullptr;
+  int *einv = nullptr;           // [T k] sorted position of each routed slot
+  void *Ybuf = nullptr;          // [T k + 128][h] expert outputs in sorted order
   int *pcnt = nullptr, *poffs = nullptr, *ptiles_a = nullptr, *ptiles_b = nullptr;
   int *pcursor = nullptr, *prows = nullptr, *pinv = nullptr;
   int *err = nullptr;
@@ -346,6 +348,8 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     DALLOC(h->etiles_b, (E + 1) * sizeof(int));
     DALLOC(h->ecursor, E * sizeof(int));
     DALLOC(h->erows, Tk * sizeof(int));
+    DALLOC(h->einv, Tk * sizeof(int));
+    DALLOC(h->Ybuf, (size_t)(Tk + 128) * hd * es);
     DALLOC(h->pcnt, (G + 1) * sizeof(int));
     DALLOC(h->poffs, (G + 1) * sizeof(int));
     DALLOC(h->ptiles_a, (G + 1) * sizeof(int));
@@ -450,9 +454,41 @@ static void launch_attn(const AttnArgs &a, int d, cudaStream_t s) {
   }
 }
 
+// depth attention, one CTA per token streaming its depth history through shared memory
+template <typename T>
+static void launch_da_bulk(const RowsArgs &r, int d, cudaStream_t s) {
+  DaBulkArgs a{};
+  a.n_tok = r.n_q; a.H = r.H; a.h = r.h; a.L = r.L; a.l = r.l;
+  const long row_bytes = 2L * r.h * sizeof(T);
+  int chunk = (int)((50 * 1024) / row_bytes);
+  if (chunk < 1) chunk = 1;
+  if (chunk > r.l + 1) chunk = r.l + 1;
+  a.chunk = chunk;
+  a.q = r.q; a.kv = r.kv; a.out = r.out; a.ldo = r.ldo; a.col0 = r.col0; a.err = r.err;
+  const int smem = (int)(2 * chunk * row_bytes);
+  const int threads = 32 * r.H;
+  auto go = [&](void (*kern)(DaBulkArgs)) {
+    // set for the kernel launched (the four head sizes share one pointer type)
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    ++g_launches;
+    kern<<<a.n_tok, threads, smem, s>>>(a);
+  };
+  switch (d) {
+    case 16: go(da_bulk_kernel<T, 16>); break;
+    case 32: go(da_bulk_kernel<T, 32>); break;
+    case 64: go(da_bulk_kernel<T, 64>); break;
+    default: go(da_bulk_kernel<T, 128>); break;
+  }
+}
+
 // depth attention (mode 0) or split decode attention + merge (mode 2)
 template <typename T>
 static void launch_rows(const RowsArgs &a, int d, cudaStream_t s) {
+  if (a.mode == 0 && a.H <= 32 && 2L * a.h * (long)sizeof(T) <= 50 * 1024) {
+    launch_da_bulk<T>(a, d, s);
+    return;
+  }
   const long warps = (long)a.n_q * a.H * (a.mode == 2 ? a.nsplit : 1);
   const int blocks = cdiv(warps, 8);
   switch (d) {
@@ -506,10 +542,34 @@ static void route_rows(dreamer_handle *h, int mode, int l, const void *X, int n,
   topk_kernel<<<cdiv(n, 8), 256, 0, s>>>(t);
 }
 
+static void trace_depth(dreamer_handle *h, const dreamer_trace *tr, int l, int n, bool prefill,
+                        cudaStream_t s) {
+  if (!tr) return;
+  const dreamer_config &c = h->cfg;
+  const size_t es = h->esz, hd = c.hidden, k = c.top_k;
+  const size_t off = (size_t)l * n;
+  if (tr->xhat) cudaMemcpyAsync((char *)tr->xhat + off * hd * es, h->xh, n * hd * es, cudaMemcpyDeviceToDevice, s);
+  if (tr->y) cudaMemcpyAsync((char *)tr->y + off * hd * es, h->y, n * hd * es, cudaMemcpyDeviceToDevice, s);
+  if (tr->idx) cudaMemcpyAsync(tr->idx + off * k, h->eidx, n * k * sizeof(int), cudaMemcpyDeviceToDevice, s);
+  if (tr->w) cudaMemcpyAsync(tr->w + off * k, h->ew, n * k * sizeof(float), cudaMemcpyDeviceToDevice, s);
+  if (prefill && tr->sa_k)
+    cudaMemcpy2DAsync((char *)tr->sa_k + off * hd * es, hd * es, (char *)h->qkv_sa + hd * es,
+                      3 * hd * es, hd * es, n, cudaMemcpyDeviceToDevice, s);
+  if (prefill && tr->sa_v)
+    cudaMemcpy2DAsync((char *)tr->sa_v + off * hd * es, hd * es, (char *)h->qkv_sa + 2 * hd * es,
+                      3 * hd * es, hd * es, n, cudaMemcpyDeviceToDevice, s);
+  if (c.n_proj_experts > 0) {
+    if (tr->pidx) cudaMemcpyAsync(tr->pidx + off, h->pidx, n * sizeof(int), cudaMemcpyDeviceToDevice, s);
+    if (tr->psig) cudaMemcpyAsync(tr->psig + off, h->psig, n * sizeof(float), cudaMemcpyDeviceToDevice, s);
+  }
+}
+
 struct DepthIO {
   int mode;               // 0 prefill, 1 decode
   int n_tok;
   const void *x_in;       // first depth only
+  void *x_out;            // written by the last depth's combine
+  const dreamer_trace *tr;
   void *da_kv;
   void *k_cache, *v_cache;
   const int *cache_len;
@@ -517,20 +577,23 @@ struct DepthIO {
 
 // One depth step for all n_tok tokens.
 template <typename T>
-static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, cudaStream_t s) {
+static void run_depth(dreamer_handle *h, int l, bool first, bool last, const DepthIO &io,
+                      cudaStream_t s) {
   const dreamer_config &c = h->cfg;
   const int hd = c.hidden, d = c.head_dim, L = c.depth, E = c.n_experts, k = c.top_k;
   const int m = c.expert_hidden, P = c.n_proj_experts, G = P > 0 ? P : 1;
   const int n = io.n_tok;
   const bool tc = h->use_tc && c.dtype == 1;
 
-  // 1. RMSNorm of the residual stream (x_0 on the first depth, else the fp32 accumulator)
+  // 1. RMSNorm of the residual stream on the first depth of the call (later depths get x^
+  // from the previous depth's fused combine + norm)
   mark(h, s, DREAMER_STAGE_NORM);
-  LAUNCHED(1);
+  if (first) {
   ++g_launches;
   rmsnorm_kernel<T><<<cdiv(n, 8), 256, 0, s>>>(first ? (const T *)io.x_in : nullptr,
                                                first ? nullptr : h->acc, (const T *)h->g,
                                                (T *)h->xh, h->inv_rms, n, hd, c.rms_eps);
+  }
   // 2. projection router and token grouping (linear-MoE QKV/O)
   const int *prow = nullptr;
   const float *psig = nullptr;
@@ -667,7 +730,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
                                  h->ecursor);
   ++g_launches;
   scatter_kernel<<<cdiv((long)n * k, 256), 256, 0, s>>>(h->eidx, n * k, h->ecursor, h->erows,
-                                                         nullptr);
+                                                         h->einv);
   // 7. expert FFNs: H = SiLU(X W1_e), acc[token] += w * H W2_e
   mark(h, s, DREAMER_STAGE_EXPERTS);
   LAUNCHED(2);
@@ -682,8 +745,22 @@ static void run_depth(dreamer_handle *h, int l, bool first, const DepthIO &io, c
     dn.N = hd; dn.K = m; dn.G = E; dn.M = n * k; dn.goffs = h->eoffs; dn.tile_offs = h->etiles_a;
     dn.arow = nullptr; dn.arow_div = 1; dn.A = h->Hbuf; dn.lda = m; dn.B = h->w2_t; dn.ldb = m;
     dn.bgstride = (long)m * hd;
-    gemm_simt<T, T, 16>(dn, etiles, EpiDown{hd, k, h->erows, h->ew, h->acc}, s);
+    gemm_simt<T, T, 16>(dn, etiles, EpiDownStore<T>{hd, (T *)h->Ybuf}, s);
   }
+  // per-depth dumps (before the combine replaces x^ with the next depth's)
+  trace_depth(h, io.tr, l, n, io.mode == 0, s);
+  // 8. x_{l+1} = y + sum_s w_s Y_s, then the next depth's RMSNorm (or the call's output)
+  mark(h, s, DREAMER_STAGE_FINISH);
+  const int cb = cdiv(n, 8);
+  ++g_launches;
+  if (hd <= 2048)
+    combine_norm_kernel<T, 64><<<cb, 256, 0, s>>>(h->acc, (const T *)h->Ybuf, h->einv, h->ew, k,
+                                                  (const T *)h->g, (T *)h->xh, h->inv_rms,
+                                                  last ? (T *)io.x_out : nullptr, n, hd, c.rms_eps);
+  else
+    combine_norm_kernel<T, 128><<<cb, 256, 0, s>>>(h->acc, (const T *)h->Ybuf, h->einv, h->ew, k,
+                                                   (const T *)h->g, (T *)h->xh, h->inv_rms,
+                                                   last ? (T *)io.x_out : nullptr, n, hd, c.rms_eps);
 }
 
 // The device error flag is copied to pinned host memory at the end of every call; the next
@@ -710,28 +787,6 @@ static int check_dev_error_sync(dreamer_handle *h) {
     return dev_error_code(e);
   }
   return DREAMER_OK;
-}
-
-static void trace_depth(dreamer_handle *h, const dreamer_trace *tr, int l, int n, bool prefill,
-                        cudaStream_t s) {
-  if (!tr) return;
-  const dreamer_config &c = h->cfg;
-  const size_t es = h->esz, hd = c.hidden, k = c.top_k;
-  const size_t off = (size_t)l * n;
-  if (tr->xhat) cudaMemcpyAsync((char *)tr->xhat + off * hd * es, h->xh, n * hd * es, cudaMemcpyDeviceToDevice, s);
-  if (tr->y) cudaMemcpyAsync((char *)tr->y + off * hd * es, h->y, n * hd * es, cudaMemcpyDeviceToDevice, s);
-  if (tr->idx) cudaMemcpyAsync(tr->idx + off * k, h->eidx, n * k * sizeof(int), cudaMemcpyDeviceToDevice, s);
-  if (tr->w) cudaMemcpyAsync(tr->w + off * k, h->ew, n * k * sizeof(float), cudaMemcpyDeviceToDevice, s);
-  if (prefill && tr->sa_k)
-    cudaMemcpy2DAsync((char *)tr->sa_k + off * hd * es, hd * es, (char *)h->qkv_sa + hd * es,
-                      3 * hd * es, hd * es, n, cudaMemcpyDeviceToDevice, s);
-  if (prefill && tr->sa_v)
-    cudaMemcpy2DAsync((char *)tr->sa_v + off * hd * es, hd * es, (char *)h->qkv_sa + 2 * hd * es,
-                      3 * hd * es, hd * es, n, cudaMemcpyDeviceToDevice, s);
-  if (c.n_proj_experts > 0) {
-    if (tr->pidx) cudaMemcpyAsync(tr->pidx + off, h->pidx, n * sizeof(int), cudaMemcpyDeviceToDevice, s);
-    if (tr->psig) cudaMemcpyAsync(tr->psig + off, h->psig, n * sizeof(float), cudaMemcpyDeviceToDevice, s);
-  }
 }
 
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
@@ -825,18 +880,10 @@ static int forward_impl(dreamer_handle *h, const void *x_in, void *x_out, int l0
   const int n = c.batch * c.seq;
   CK(cudaMemsetAsync(h->counts, 0, (size_t)c.depth * c.n_experts * sizeof(int), s));
   DepthIO io{};
-  io.mode = 0; io.n_tok = n; io.x_in = x_in; io.da_kv = da_kv ? da_kv : h->da_kv_int;
-  for (int l = l0; l < l1; l++) {
-    run_depth<T>(h, l, l == l0, io, s);
-    trace_depth(h, tr, l, n, true, s);
-  }
-  mark(h, s, DREAMER_STAGE_FINISH);
-  if (l1 > l0) {
-    LAUNCHED(1);
-    long tot = (long)n * c.hidden;
-    ++g_launches;
-    finish_kernel<T><<<cdiv(tot / 8, 256), 256, 0, s>>>(h->acc, (T *)x_out, tot);
-  } else if (x_out != x_in) {
+  io.mode = 0; io.n_tok = n; io.x_in = x_in; io.x_out = x_out; io.tr = tr;
+  io.da_kv = da_kv ? da_kv : h->da_kv_int;
+  for (int l = l0; l < l1; l++) run_depth<T>(h, l, l == l0, l == l1 - 1, io, s);
+  if (l1 == l0 && x_out != x_in) {
     CK(cudaMemcpyAsync(x_out, x_in, (size_t)n * c.hidden * h->esz, cudaMemcpyDeviceToDevice, s));
   }
   CK(cudaMemcpyAsync(h->err_host, h->err, sizeof(int), cudaMemcpyDeviceToHost, s));
@@ -879,17 +926,10 @@ static int decode_impl(dreamer_handle *h, const void *x_new, void *kc, void *vc,
   const int n = c.batch;
   CK(cudaMemsetAsync(h->counts, 0, (size_t)c.depth * c.n_experts * sizeof(int), s));
   DepthIO io{};
-  io.mode = 1; io.n_tok = n; io.x_in = x_new; io.da_kv = h->da_kv_int;
+  io.mode = 1; io.n_tok = n; io.x_in = x_new; io.x_out = x_out; io.tr = tr;
+  io.da_kv = h->da_kv_int;
   io.k_cache = kc; io.v_cache = vc; io.cache_len = len;
-  for (int l = 0; l < c.depth; l++) {
-    run_depth<T>(h, l, l == 0, io, s);
-    trace_depth(h, tr, l, n, false, s);
-  }
-  mark(h, s, DREAMER_STAGE_FINISH);
-  LAUNCHED(1);
-  long tot = (long)n * c.hidden;
-  ++g_launches;
-  finish_kernel<T><<<cdiv(tot / 8, 256), 256, 0, s>>>(h->acc, (T *)x_out, tot);
+  for (int l = 0; l < c.depth; l++) run_depth<T>(h, l, l == 0, l == c.depth - 1, io, s);
   CK(cudaMemcpyAsync(h->err_host, h->err, sizeof(int), cudaMemcpyDeviceToHost, s));
   mark(h, s, DREAMER_N_STAGES);
   CK(cudaGetLastError());

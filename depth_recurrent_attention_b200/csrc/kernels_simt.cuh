@@ -164,6 +164,19 @@ struct EpiDown {
   }
 };
 
+// Expert down-projection epilogue, store form: the routed row's expert output Y (sorted row
+// r) is written once in dtype; the weighted sum over a token's k rows happens in
+// combine_norm_kernel (no atomics, fixed summation order).
+template <typename T> struct EpiDownStore {
+  int h;
+  T *Y;  // [rows][h], expert-sorted order
+  template <int SEG>
+  __device__ __forceinline__ void operator()(int r, int token, int g, int n0, float *v) const {
+#pragma unroll
+    for (int i = 0; i < SEG; i += 8) store8(Y + (long)r * h + n0 + i, v + i);
+  }
+};
+
 // Plain fp32 store of columns < N (router queries and scores).
 struct EpiStoreF32 {
   float *C;
@@ -316,6 +329,63 @@ __global__ void rmsnorm_kernel(const T *x_in, const float *acc, const T *gain, T
     load8(gain + c, gv);
 #pragma unroll
     for (int j = 0; j < 8; j++) o[j] = gv[j] * v[j] * r;
+    store8(xh + (long)warp * h + c, o);
+  }
+}
+
+// Combine, residual and RMSNorm fused (one warp per token): x_{l+1} = y + sum_s w_s Y_s over
+// the token's k routed rows (papernotes "Key design 2": the expert outputs mixed by the
+// normalised routing weights; fixed order s = 0..k-1), kept in fp32 in acc; then either the
+// next depth's x^ = g x / rms(x) and 1/rms (RMSNorm on the residual stream, "Overall
+// framework"), or, after the last depth, the output x_L rounded to dtype.
+template <typename T, int MAXV>
+__global__ void __launch_bounds__(256) combine_norm_kernel(float *acc, const T *Y, const int *pos,
+                                                          const float *wts, int k, const T *gain,
+                                                          T *xh, float *inv_rms, T *x_out,
+                                                          int n_tok, int h, float eps) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= n_tok) return;
+  float xv[MAXV];  // this lane's 8-element chunks of the row, in fp32
+  float ss = 0.f;
+  long prow[16];
+  float pw[16];
+  for (int s = 0; s < k; s++) {
+    prow[s] = (long)pos[(long)warp * k + s] * h;
+    pw[s] = wts[(long)warp * k + s];
+  }
+#pragma unroll
+  for (int ci = 0; ci < MAXV / 8; ci++) {
+    const int c = ci * 256 + lane * 8;
+    if (c >= h) break;
+    float x[8];
+    load8(acc + (long)warp * h + c, x);
+    for (int s = 0; s < k; s++) {
+      float yv[8];
+      load8(Y + prow[s] + c, yv);
+#pragma unroll
+      for (int j = 0; j < 8; j++) x[j] = fmaf(pw[s], yv[j], x[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+      xv[ci * 8 + j] = x[j];
+      ss += x[j] * x[j];
+    }
+    if (x_out) store8(x_out + (long)warp * h + c, x);
+    else store8(acc + (long)warp * h + c, x);
+  }
+  if (x_out) return;
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / (float)h + eps);
+  if (lane == 0) inv_rms[warp] = r;
+#pragma unroll
+  for (int ci = 0; ci < MAXV / 8; ci++) {
+    const int c = ci * 256 + lane * 8;
+    if (c >= h) break;
+    float gv[8], o[8];
+    load8(gain + c, gv);
+#pragma unroll
+    for (int j = 0; j < 8; j++) o[j] = gv[j] * xv[ci * 8 + j] * r;
     store8(xh + (long)warp * h + c, o);
   }
 }

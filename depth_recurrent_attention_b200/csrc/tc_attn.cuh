@@ -248,24 +248,35 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(smem_u32(&s_full[t]), j & 1, abort_flag, a.err)) { ok = false; break; }
         tc_fence_after();
         const bool diag = (j == qt);
-        float mx = -INFINITY;
+        // pass 1: row max of the raw scores (the scale is positive: applied to the max)
+        float mraw = -INFINITY;
+        if (!diag) {
 #pragma unroll
-        for (int c = 0; c < 128; c += 32) {
-          float sv[32];
-          tmem_ld32(sbuf + c, sv);
+          for (int c = 0; c < 128; c += 32) {
+            float sv[32];
+            tmem_ld32(sbuf + c, sv);
 #pragma unroll
-          for (int i = 0; i < 32; i++) {
-            const bool masked = diag && (j * 128 + c + i) > qi;
-            if (!masked) mx = fmaxf(mx, sv[i] * a.scale_log2);
+            for (int i = 0; i < 32; i++) mraw = fmaxf(mraw, sv[i]);
+          }
+        } else {
+          const int lim = qi - j * 128;  // last visible key of this row inside the block
+#pragma unroll
+          for (int c = 0; c < 128; c += 32) {
+            float sv[32];
+            tmem_ld32(sbuf + c, sv);
+#pragma unroll
+            for (int i = 0; i < 32; i++)
+              if (c + i <= lim) mraw = fmaxf(mraw, sv[i]);
           }
         }
+        const float mx = mraw * a.scale_log2;
         // lazy rescale: move the reference max only when the row max grows by more than 8
         float m_new = m_ref, alpha = 1.f;
         if (j == 0) {
           m_new = mx;
         } else if (mx > m_ref + 8.f) {
           m_new = mx;
-          alpha = exp2f(m_ref - mx);
+          alpha = ex2(m_ref - mx);
         }
         if (j > 0) {
           // P_t(j-1) V was consumed and O_t holds every earlier block
@@ -282,8 +293,10 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
         }
-        // pass 2: P = exp2(s - m_new) as bf16, K-major SW128 (key chunk kc at kc * TILE,
+        // pass 2: P = 2^(s * scale - m) as bf16, K-major SW128 (key chunk kc at kc * TILE,
         // 16-byte unit u of the row at ((u ^ (row & 7)) << 4))
+        const float nm = -m_new;
+        const int lim = diag ? qi - j * 128 : 127;
         float rs = 0.f;
 #pragma unroll
         for (int c = 0; c < 128; c += 32) {
@@ -291,10 +304,9 @@ __global__ void __launch_bounds__(384, 1)
           tmem_ld32(sbuf + c, sv);
 #pragma unroll
           for (int i = 0; i < 32; i++) {
-            const bool masked = diag && (j * 128 + c + i) > qi;
-            const float p = masked ? 0.f : exp2f(sv[i] * a.scale_log2 - m_new);
-            sv[i] = p;
-            rs += p;
+            const float p = ex2(fmaf(sv[i], a.scale_log2, nm));
+            sv[i] = (c + i <= lim) ? p : 0.f;
+            rs += sv[i];
           }
           const int kc = c >> 6;
 #pragma unroll

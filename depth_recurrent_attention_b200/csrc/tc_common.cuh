@@ -164,6 +164,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
   for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
 }
 
+// 2^x with the hardware approximation (MUFU.EX2, flush to zero); used for softmax weights that
+// are stored in bf16 afterwards.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Shared-memory matrix descriptor of a K-major tile written by TMA with a swizzle of
 // `sw_bytes` (32, 64 or 128) = the byte width of one row of the tile: rows at sw_bytes pitch,
 // 8-row groups every 8 * sw_bytes bytes (stride byte offset), leading byte offset 16

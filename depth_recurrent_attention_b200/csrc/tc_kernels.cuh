@@ -100,16 +100,24 @@ struct EpiTopK {
   template <int SEG>
   __device__ __forceinline__ void row_apply(State &s, int r, int token, int g, int n0,
                                             const float *vals) const {
+    // candidates against the current k-th entry first (straight-line), then a rolled
+    // insertion for the few that qualify (keeps the code small and the warp convergent)
+    float vb[SEG];
+    unsigned mask = 0;
 #pragma unroll
     for (int i = 0; i < SEG; i++) {
-      const int e = n0 + i;
-      float z = vals[i] * zscale;
-      float v = z + bias[e];
+      float v = vals[i] * zscale + bias[n0 + i];
       if (v != v) v = -INFINITY;
-      if (!better(v, e, s.v[KT - 1], s.e[KT - 1])) continue;
-      int ce = e;
-      float cv = v, cz = z;
-#pragma unroll
+      vb[i] = v;
+      if (better(v, n0 + i, s.v[KT - 1], s.e[KT - 1])) mask |= 1u << i;
+    }
+    while (mask) {
+      const int i = __ffs(mask) - 1;
+      mask &= mask - 1;
+      float cv = vb[i], cz = vals[i] * zscale;
+      int ce = n0 + i;
+      if (!better(cv, ce, s.v[KT - 1], s.e[KT - 1])) continue;
+#pragma unroll 1
       for (int j = 0; j < KT; j++) {  // insertion by compare-and-swap down the sorted list
         if (better(cv, ce, s.v[j], s.e[j])) {
           const float tv = s.v[j], tz = s.z[j];
@@ -426,7 +434,7 @@ static bool tc_expert(dreamer_handle *h, const void *X, int n, cudaStream_t s) {
   CUtensorMap tau, tbu, tad, tbd;
   long mtu, mtd;
   EpiUp<bf16> eu{m, (bf16 *)h->Hbuf};
-  EpiDownVec ed{hd, k, h->erows, h->ew, h->acc};
+  EpiDownStore<bf16> ed{hd, (bf16 *)h->Ybuf};
   switch (m) {
     case 16:
       if (!tc_prepare<16, 64>(h, up, h->etiles_b, rows, tu, tau, tbu, mtu) ||
