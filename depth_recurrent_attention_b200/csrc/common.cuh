@@ -43,6 +43,28 @@ __device__ __forceinline__ void store8(bf16 *p, const float *v) {
   *reinterpret_cast<uint4 *>(p) = u;
 }
 
+// 4 consecutive elements <-> float[4]
+__device__ __forceinline__ void load4(const float *p, float *o) {
+  float4 a = *reinterpret_cast<const float4 *>(p);
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+}
+__device__ __forceinline__ void load4(const bf16 *p, float *o) {
+  uint2 u = *reinterpret_cast<const uint2 *>(p);
+  const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+  float2 f0 = __bfloat1622float2(h2[0]), f1 = __bfloat1622float2(h2[1]);
+  o[0] = f0.x; o[1] = f0.y; o[2] = f1.x; o[3] = f1.y;
+}
+__device__ __forceinline__ void store4(float *p, const float *v) {
+  *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void store4(bf16 *p, const float *v) {
+  uint2 u;
+  __nv_bfloat162 *h2 = reinterpret_cast<__nv_bfloat162 *>(&u);
+  h2[0] = __floats2bfloat162_rn(v[0], v[1]);
+  h2[1] = __floats2bfloat162_rn(v[2], v[3]);
+  *reinterpret_cast<uint2 *>(p) = u;
+}
+
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -49,6 +49,7 @@ struct dreamer_handle {
   int *err = nullptr;
   void *k3 = nullptr;            // [E][3 d_r] bf16: router keys repeated for split scores
   int num_sms = 148;
+  int qkv_perm = 0;  // q_SA / k_SA columns of the fused QKV weight in EpiQKV perm order
   int use_tc = 1;  // bf16 contractions on tcgen05 (0: CUDA cores, for cross-checks)
   std::vector<void *> allocs;
   int *err_host = nullptr;       // pinned copy of the device error flag (async)
@@ -297,6 +298,11 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     // W_qkv [G][h][6h] (+ shared) -> [G][6h][h]; W_o [G][2h][h] -> [G][h][2h]
     tr(w->w_qkv, P > 0 ? w->w_qkv_shared : nullptr, h->wqkv_t, hd, 6 * hd, G, s);
     tr(w->w_o, P > 0 ? w->w_o_shared : nullptr, h->wo_t, 2 * hd, hd, G, s);
+    if (c.dtype == 1 && d == 128) {  // RoPE partners 32 columns apart (EpiQKV perm order)
+      h->qkv_perm = 1;
+      ++g_launches;
+      perm_qk_rows_kernel<bf16><<<4 * 148, 256, 0, s>>>((bf16 *)h->wqkv_t, hd, G);
+    }
     tr(w->w_qE, nullptr, h->wqE_t, hd, dr, 1, s);
     tr(w->w1, nullptr, h->w1_t, hd, m, E, s);     // [E][h][m] -> [E][m][h]
     tr(w->w2, nullptr, h->w2_t, m, hd, E, s);     // [E][m][h] -> [E][h][m]
@@ -539,7 +545,7 @@ static void route_rows(dreamer_handle *h, int mode, int l, const void *X, int n,
   t.bias = mode == 0 ? h->bias : nullptr;
   t.idx = idx; t.w = wout; t.counts_a = counts_a; t.counts_b = counts_b;
   ++g_launches;
-  topk_kernel<<<cdiv(n, 8), 256, 0, s>>>(t);
+  launch_topk(t, s);
 }
 
 static void trace_depth(dreamer_handle *h, const dreamer_trace *tr, int l, int n, bool prefill,
@@ -623,6 +629,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
 
   EpiQKV<T> eq{};
   eq.h = hd; eq.d = d; eq.L = L; eq.l = l; eq.S = c.seq; eq.mode = io.mode; eq.col_lo = 0;
+  eq.perm = h->qkv_perm;
   eq.psig = psig; eq.rope_tok = h->rope_tok; eq.rope_dep = h->rope_dep;
   eq.qkv_sa = (T *)h->qkv_sa; eq.q_da = (T *)h->q_da; eq.da_kv = (T *)io.da_kv;
   eq.k_cache = (T *)io.k_cache; eq.v_cache = (T *)io.v_cache; eq.cache_len = io.cache_len;

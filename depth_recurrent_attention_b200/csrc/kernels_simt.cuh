@@ -15,10 +15,16 @@ namespace dreamer {
 // QKV projection epilogue: scale by the projection weight sigma (linear MoE), apply token
 // RoPE to q_SA/k_SA and depth RoPE to q_DA/k_DA, and scatter into the attention layouts.
 // (papernotes "Key design 1": depth RoPE with a reversed half; "Key design 3": sigma x W~.)
+//
+// Column order.  With perm set (head dim 128 on the tensor-core path) the q_SA and k_SA
+// columns of each head come out of the GEMM in the order [0,32) [64,96) [32,64) [96,128), so
+// that rotate-half partners (i, i + 64) sit 32 columns apart like every other RoPE pair;
+// unperm() maps a computed column back to its head column.
 template <typename T> struct EpiQKV {
   int h, d, L, l, S;
   int mode;                  // 0 prefill (position = token % S), 1 decode (position = cache_len[b])
   int col_lo;                // first column of the fused projection this GEMM computes
+  int perm;                  // q_SA / k_SA column order as above
   const float *psig;         // [T] or null (dense)
   const float2 *rope_tok;    // [max_pos][d/2]
   const float2 *rope_dep;    // [L][d/2]
@@ -30,28 +36,167 @@ template <typename T> struct EpiQKV {
   int B, cap;
   int *err;                  // device error flag
 
+  __device__ __forceinline__ static int unperm(int c) {  // c in [0, 128)
+    const int q = c >> 5;
+    return q == 1 ? c + 32 : (q == 2 ? c - 32 : c);
+  }
+
+  // Destination of (token, column nc of the full [6h] projection in head order), or null when
+  // a decode cache slot is out of range (reported by the caller).
+  __device__ __forceinline__ T *dest(int token, int nc) const {
+    const int blk = nc / h, head = (nc % h) / d, hc = nc % h;
+    if (blk <= 2) {
+      if (mode == 0 || blk == 0) return qkv_sa + (long)token * 3 * h + blk * h + hc;
+      const int pos = cache_len[token];
+      if (pos < 0 || pos >= cap) return nullptr;
+      T *base = (blk == 1) ? k_cache : v_cache;
+      return base + ((((long)l * B + token) * (h / d) + head) * cap + pos) * d + (hc % d);
+    }
+    if (blk == 3) return q_da + (long)token * h + hc;
+    return da_kv + (((long)token * L + l) * 2 + (blk - 4)) * h + hc;
+  }
+
+  __device__ __forceinline__ int position(int token) const {  // -1: outside the cache
+    if (mode == 0) return token % S;
+    const int p = cache_len[token];
+    return (p < 0 || p >= cap) ? -1 : p;
+  }
+
+  // Row layout (SEG = d columns of one head, in computed order): sigma only; the rotations
+  // run in the coalesced layout.
   template <int SEG>
-  __device__ __forceinline__ void operator()(int r, int token, int g, int n0, float *v) const {
-    static_assert(SEG % 16 == 0, "segment");
-    const int nc = n0 + col_lo;        // column of the full [6h] projection
-    const int blk = nc / h;            // 0 qSA 1 kSA 2 vSA 3 qDA 4 kDA 5 vDA
-    const int head = (nc % h) / d;
-    const int hc = nc % h;             // column inside the block
+  __device__ __forceinline__ void transform(int r, int token, int g, int n0, float *v) const {
     if (psig) {
       const float s = psig[token];
 #pragma unroll
       for (int i = 0; i < SEG; i++) v[i] *= s;
     }
-    if (mode == 1 && blk <= 2) {
-      const int p = cache_len[token];
-      if (p < 0 || p >= cap) {  // slot outside the cache: report, write nothing
+  }
+
+  // Coalesced layout: a pass of 64 columns [c64, c64 + 64) inside one head; the lane holds
+  // columns col..col+3 (v[i][0..3]) and col+32..col+35 (v[i][4..7]) of rows r[i].
+  static constexpr bool STAGED = true;
+  template <int NR, int NV>
+  __device__ __forceinline__ void store_rows(const int *r, const int *tok, int g, int col,
+                                             const float (*v)[NV]) const {
+    static_assert(NV == 8, "QKV passes are 64 columns wide");
+    const int nc = col + col_lo;
+    const int blk = nc / h, hc = nc % h;
+    const int hb = blk * h + hc - hc % d;   // first column of the head
+    const int cin = hc % d;                 // computed column inside the head (cin % 64 < 32)
+    if (blk <= 1) {
+      // token RoPE: head columns o and o + d/2, frequency o
+      const int o = perm ? unperm(cin) : cin;
+#pragma unroll
+      for (int i = 0; i < NR; i++) {
+        if (r[i] < 0) continue;
+        const int pos = position(tok[i]);
+        if (pos < 0) {
+          raise_dev_error(err, DEV_BAD_INDEX);
+          continue;
+        }
+        const float4 *cs = reinterpret_cast<const float4 *>(rope_tok + (long)pos * (d / 2) + o);
+        const float4 c01 = cs[0], c23 = cs[1];
+        const float cc[4] = {c01.x, c01.z, c23.x, c23.z}, sn[4] = {c01.y, c01.w, c23.y, c23.w};
+        float a[4], b[4];
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          a[j] = v[i][j] * cc[j] - v[i][4 + j] * sn[j];
+          b[j] = v[i][4 + j] * cc[j] + v[i][j] * sn[j];
+        }
+        T *da = dest(tok[i], hb + o);
+        if (da) {
+          store4(da, a);
+          store4(da + d / 2, b);
+        }
+      }
+      return;
+    }
+    if (blk == 3 || blk == 4) {
+      // depth RoPE: two halves of d/2 (positions l and L-1-l), rotate-half inside each
+      const float2 *tab = rope_dep + (long)l * (d / 2);
+      float w[NR][8];
+      if (d == 128) {
+        // the pass is one half; columns col and col + 32 are partners, frequency cin % 32
+        const int half = cin >> 6, f = cin & 31;
+        const float4 *cs = reinterpret_cast<const float4 *>(tab + half * 32 + f);
+        const float4 c01 = cs[0], c23 = cs[1];
+        const float cc[4] = {c01.x, c01.z, c23.x, c23.z}, sn[4] = {c01.y, c01.w, c23.y, c23.w};
+#pragma unroll
+        for (int i = 0; i < NR; i++)
+#pragma unroll
+          for (int j = 0; j < 4; j++) {
+            w[i][j] = v[i][j] * cc[j] - v[i][4 + j] * sn[j];
+            w[i][4 + j] = v[i][4 + j] * cc[j] + v[i][j] * sn[j];
+          }
+      } else {
+        // d = 64: the pass is the head; columns col (half 0) and col + 32 (half 1) each pair
+        // with the column 16 away, held by lane ^ 4
+        const int f = cin & 15;
+        const bool first = (cin & 31) < 16;
+        const float4 *c0 = reinterpret_cast<const float4 *>(tab + f);
+        const float4 *c1 = reinterpret_cast<const float4 *>(tab + 16 + f);
+        const float4 a01 = c0[0], a23 = c0[1], b01 = c1[0], b23 = c1[1];
+        const float ca[4] = {a01.x, a01.z, a23.x, a23.z}, sa[4] = {a01.y, a01.w, a23.y, a23.w};
+        const float cb[4] = {b01.x, b01.z, b23.x, b23.z}, sb[4] = {b01.y, b01.w, b23.y, b23.w};
+        const float sg = first ? -1.f : 1.f;
+#pragma unroll
+        for (int i = 0; i < NR; i++)
+#pragma unroll
+          for (int j = 0; j < 4; j++) {
+            const float pa = __shfl_xor_sync(0xffffffffu, v[i][j], 4);
+            const float pb = __shfl_xor_sync(0xffffffffu, v[i][4 + j], 4);
+            w[i][j] = v[i][j] * ca[j] + sg * pa * sa[j];
+            w[i][4 + j] = v[i][4 + j] * cb[j] + sg * pb * sb[j];
+          }
+      }
+#pragma unroll
+      for (int i = 0; i < NR; i++) {
+        if (r[i] < 0) continue;
+        T *dst = dest(tok[i], hb + cin);
+        store4(dst, w[i]);
+        store4(dst + 32, w[i] + 4);
+      }
+      return;
+    }
+#pragma unroll
+    for (int i = 0; i < NR; i++) {  // v_SA, v_DA: as they are
+      if (r[i] < 0) continue;
+      T *dst = dest(tok[i], hb + cin);
+      if (!dst) {
         raise_dev_error(err, DEV_BAD_INDEX);
-        return;
+        continue;
+      }
+      store4(dst, v[i]);
+      store4(dst + 32, v[i] + 4);
+    }
+  }
+
+  // CUDA-core engine: one row's SEG = d columns of one head at once, in computed order.
+  template <int SEG>
+  __device__ __forceinline__ void operator()(int r, int token, int g, int n0, float *v) const {
+    static_assert(SEG % 16 == 0, "segment");
+    const int nc = n0 + col_lo;        // column of the full [6h] projection
+    const int blk = nc / h;            // 0 qSA 1 kSA 2 vSA 3 qDA 4 kDA 5 vDA
+    if (psig) {
+      const float s = psig[token];
+#pragma unroll
+      for (int i = 0; i < SEG; i++) v[i] *= s;
+    }
+    if (SEG == 128 && perm && blk <= 1) {  // back to head order (the permutation swaps
+#pragma unroll                             // the middle two 32-column blocks)
+      for (int i = 32; i < 64; i++) {
+        const float t = v[i];
+        v[i] = v[i + 32];
+        v[i + 32] = t;
       }
     }
+    if (mode == 1 && blk <= 2 && position(token) < 0) {  // slot outside the cache
+      raise_dev_error(err, DEV_BAD_INDEX);
+      return;
+    }
     if (blk <= 1) {  // token RoPE, rotate-half over d (pair i, i + d/2)
-      const int pos = mode == 0 ? (token % S) : cache_len[token];
-      const float2 *cs = rope_tok + (long)pos * (d / 2);
+      const float2 *cs = rope_tok + (long)position(token) * (d / 2);
 #pragma unroll
       for (int i = 0; i < SEG / 2; i++) {
         float c = cs[i].x, s = cs[i].y;
@@ -73,20 +218,8 @@ template <typename T> struct EpiQKV {
         }
       }
     }
-    T *dst;
-    if (blk <= 2) {
-      if (mode == 0 || blk == 0) {
-        dst = qkv_sa + (long)token * 3 * h + blk * h + hc;
-      } else {
-        const int pos = cache_len[token];
-        T *base = (blk == 1) ? k_cache : v_cache;
-        dst = base + ((((long)l * B + token) * (h / d) + head) * cap + pos) * d;
-      }
-    } else if (blk == 3) {
-      dst = q_da + (long)token * h + hc;
-    } else {
-      dst = da_kv + (((long)token * L + l) * 2 + (blk - 4)) * h + hc;
-    }
+    T *dst = dest(token, n0 + col_lo);
+    if (!dst) return;
 #pragma unroll
     for (int i = 0; i < SEG; i += 8) store8(dst + i, v + i);
   }
@@ -132,6 +265,46 @@ template <typename T> struct EpiO {
       store8(ap, o);
     }
   }
+
+  static constexpr bool STAGED = true;
+  template <int SEG>
+  __device__ __forceinline__ void transform(int, int, int, int, float *) const {}
+  // Coalesced layout (NV values a lane and row: 4 at col, and with NV = 8 four more at
+  // col + 32); all residual loads are issued before the first store.
+  template <int NR, int NV>
+  __device__ __forceinline__ void store_rows(const int *r, const int *tok, int g, int col,
+                                             const float (*v)[NV]) const {
+    float gv[NV];
+#pragma unroll
+    for (int hh = 0; hh < NV / 4; hh++) {
+      if (res_mode != 2) load4(gain + col + 32 * hh, gv + 4 * hh);
+      else gv[4 * hh] = gv[4 * hh + 1] = gv[4 * hh + 2] = gv[4 * hh + 3] = 1.f;
+    }
+    float xr[NR][NV];
+#pragma unroll
+    for (int i = 0; i < NR; i++) {
+      if (r[i] < 0) continue;
+#pragma unroll
+      for (int hh = 0; hh < NV / 4; hh++) {
+        if (res_mode == 0) load4(xin + (long)tok[i] * h + col + 32 * hh, xr[i] + 4 * hh);
+        else load4(acc + (long)tok[i] * h + col + 32 * hh, xr[i] + 4 * hh);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NR; i++) {
+      if (r[i] < 0) continue;
+      const float s = psig ? psig[tok[i]] : 1.0f;
+      const float ir = res_mode == 2 ? 1.f : inv_rms[tok[i]];
+      float o[NV];
+#pragma unroll
+      for (int j = 0; j < NV; j++) o[j] = (res_mode == 2 ? xr[i][j] : gv[j] * xr[i][j] * ir) + s * v[i][j];
+#pragma unroll
+      for (int hh = 0; hh < NV / 4; hh++) {
+        if (y) store4(y + (long)tok[i] * h + col + 32 * hh, o + 4 * hh);
+        store4(acc + (long)tok[i] * h + col + 32 * hh, o + 4 * hh);
+      }
+    }
+  }
 };
 
 // Expert up-projection epilogue: H[r] = SiLU(X W1_e) (papernotes "Key design 2": each
@@ -145,6 +318,21 @@ template <typename T> struct EpiUp {
     for (int i = 0; i < SEG; i++) v[i] = v[i] / (1.0f + __expf(-v[i]));
 #pragma unroll
     for (int i = 0; i < SEG; i += 8) store8(H + (long)r * m + n0 + i, v + i);
+  }
+  static constexpr bool STAGED = true;
+  template <int SEG>
+  __device__ __forceinline__ void transform(int, int, int, int, float *v) const {
+#pragma unroll
+    for (int i = 0; i < SEG; i++) v[i] = v[i] / (1.0f + __expf(-v[i]));
+  }
+  template <int NR, int NV>
+  __device__ __forceinline__ void store_rows(const int *r, const int *, int, int col,
+                                             const float (*v)[NV]) const {
+#pragma unroll
+    for (int i = 0; i < NR; i++)
+      if (r[i] >= 0)
+#pragma unroll
+        for (int hh = 0; hh < NV / 4; hh++) store4(H + (long)r[i] * m + col + 32 * hh, v[i] + 4 * hh);
   }
 };
 
@@ -175,6 +363,18 @@ template <typename T> struct EpiDownStore {
 #pragma unroll
     for (int i = 0; i < SEG; i += 8) store8(Y + (long)r * h + n0 + i, v + i);
   }
+  static constexpr bool STAGED = true;
+  template <int SEG>
+  __device__ __forceinline__ void transform(int, int, int, int, float *) const {}
+  template <int NR, int NV>
+  __device__ __forceinline__ void store_rows(const int *r, const int *, int, int col,
+                                             const float (*v)[NV]) const {
+#pragma unroll
+    for (int i = 0; i < NR; i++)
+      if (r[i] >= 0)
+#pragma unroll
+        for (int hh = 0; hh < NV / 4; hh++) store4(Y + (long)r[i] * h + col + 32 * hh, v[i] + 4 * hh);
+  }
 };
 
 // Plain fp32 store of columns < N (router queries and scores).
@@ -187,6 +387,26 @@ struct EpiStoreF32 {
 #pragma unroll
     for (int i = 0; i < SEG; i++)
       if (n0 + i < N) C[(long)r * ldc + n0 + i] = v[i];
+  }
+  static constexpr bool STAGED = true;
+  template <int SEG>
+  __device__ __forceinline__ void transform(int, int, int, int, float *) const {}
+  template <int NR, int NV>
+  __device__ __forceinline__ void store_rows(const int *r, const int *, int, int col,
+                                             const float (*v)[NV]) const {
+#pragma unroll
+    for (int i = 0; i < NR; i++) {
+      if (r[i] < 0) continue;
+#pragma unroll
+      for (int hh = 0; hh < NV / 4; hh++) {
+        const int c0 = col + 32 * hh;
+        float *p = C + (long)r[i] * ldc + c0;
+        if (c0 + 4 <= N && (ldc & 3) == 0) store4(p, v[i] + 4 * hh);
+        else
+          for (int j = 0; j < 4; j++)
+            if (c0 + j < N) p[j] = v[i][4 * hh + j];
+      }
+    }
   }
 };
 
@@ -535,56 +755,69 @@ __device__ __forceinline__ bool better(float v1, int e1, float v2, int e2) {
   return v1 > v2 || (v1 == v2 && e1 < e2);
 }
 
+// One warp per token.  Lane j scans the experts e = j (mod 32) and keeps its best KT (biased
+// score, index) pairs in registers, sorted, inserting by a fully unrolled compare-and-swap
+// pass (no dynamically indexed arrays, so nothing spills to local memory); then k rounds of a
+// warp argmax over the lanes' heads, the winning lane shifting its list up.  KT >= k.
+template <int KT>
 __global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
-  constexpr int KMAX = 16;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= a.n_tok) return;
   const float *zr = a.z + (long)warp * a.ldz;
-  float lv[KMAX];
-  int le[KMAX];
+  float lv[KT], lz[KT];
+  int le[KT];
 #pragma unroll
-  for (int i = 0; i < KMAX; i++) {
+  for (int i = 0; i < KT; i++) {
     lv[i] = -INFINITY;
+    lz[i] = 0.f;
     le[i] = 0x7fffffff;
   }
   const int k = a.k;
+#pragma unroll 4
   for (int e = lane; e < a.E; e += 32) {
-    float v = zr[e] * a.zscale + (a.bias ? a.bias[e] : 0.f);
+    const float z = zr[e] * a.zscale;
+    float v = z + (a.bias ? a.bias[e] : 0.f);
     if (v != v) v = -INFINITY;  // a NaN score ranks last; indices stay valid
-    if (!better(v, e, lv[k - 1], le[k - 1])) continue;
-    // insert keeping descending order
-    int p = k - 1;
-    while (p > 0 && better(v, e, lv[p - 1], le[p - 1])) {
-      lv[p] = lv[p - 1];
-      le[p] = le[p - 1];
-      p--;
+    if (!better(v, e, lv[KT - 1], le[KT - 1])) continue;
+    float cz = z;
+    int ce = e;
+#pragma unroll
+    for (int j = 0; j < KT; j++) {
+      if (better(v, ce, lv[j], le[j])) {
+        const float tv = lv[j], tz = lz[j];
+        const int te = le[j];
+        lv[j] = v; lz[j] = cz; le[j] = ce;
+        v = tv; cz = tz; ce = te;
+      }
     }
-    lv[p] = v;
-    le[p] = e;
   }
-  int head = 0;
   float wsum = 0.f;
   int myidx = 0;
   float myz = 0.f;
   for (int s = 0; s < k; s++) {
-    float v = head < k ? lv[head] : -INFINITY;
-    int e = head < k ? le[head] : 0x7fffffff;
-    // warp argmax with lower-index tie break
-    float bv = v;
-    int be = e;
+    float bv = lv[0];
+    int be = le[0];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
       if (better(ov, oe, bv, be)) {
         bv = ov;
         be = oe;
       }
     }
-    if (be == e && head < k) head++;
-    const float zv = zr[be] * a.zscale;
-    const float sg = 1.0f / (1.0f + __expf(-zv));
+    const bool win = le[0] == be;
+    const int src = __ffs(__ballot_sync(0xffffffffu, win)) - 1;
+    const float zw = __shfl_sync(0xffffffffu, lz[0], src);
+    if (win) {
+#pragma unroll
+      for (int j = 0; j + 1 < KT; j++) {
+        lv[j] = lv[j + 1]; lz[j] = lz[j + 1]; le[j] = le[j + 1];
+      }
+      lv[KT - 1] = -INFINITY; le[KT - 1] = 0x7fffffff;
+    }
+    const float sg = 1.0f / (1.0f + __expf(-zw));
     wsum += sg;
     if (lane == s) {
       myidx = be;
@@ -597,6 +830,15 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
     if (a.counts_a) atomicAdd(a.counts_a + myidx, 1);
     if (a.counts_b) atomicAdd(a.counts_b + myidx, 1);
   }
+}
+
+// Launch with the smallest list length that holds k (k <= 16).
+inline void launch_topk(const TopkArgs &t, cudaStream_t s) {
+  const int blocks = (t.n_tok + 7) / 8;
+  if (t.k <= 2) topk_kernel<2><<<blocks, 256, 0, s>>>(t);
+  else if (t.k <= 4) topk_kernel<4><<<blocks, 256, 0, s>>>(t);
+  else if (t.k <= 8) topk_kernel<8><<<blocks, 256, 0, s>>>(t);
+  else topk_kernel<16><<<blocks, 256, 0, s>>>(t);
 }
 
 // =======================================================================================
@@ -715,6 +957,30 @@ __global__ void __launch_bounds__(1024) bias_update_kernel(const int *counts, in
 // =======================================================================================
 // dst[g][j][i] = src[g][i][j] (+ sh[i][j]), rounded to T once (absorption, papernotes
 // "Key design 3": W~ = W_p + W_shared folded after training).
+// Column order of the tensor-core QKV GEMM for head dim 128: in the transposed weight
+// [G][6h][h], swap rows [32, 64) and [64, 96) of every 128-row head of q_SA and k_SA (the
+// EpiQKV perm order).  One thread per swapped element pair.
+template <typename T>
+__global__ void perm_qk_rows_kernel(T *w, int h, int G) {
+  const int nh = h / 128;
+  const long total = (long)G * 2 * nh * 32 * h;
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long)gridDim.x * blockDim.x) {
+    const int k = (int)(i % h);
+    long t = i / h;
+    const int r = (int)(t % 32);
+    t /= 32;
+    const int head = (int)(t % nh);
+    t /= nh;
+    const int blk = (int)(t % 2), g = (int)(t / 2);
+    T *base = w + ((long)g * 6 * h + blk * h + head * 128) * h;
+    T *a = base + (long)(32 + r) * h + k, *b = base + (long)(64 + r) * h + k;
+    const T x = *a;
+    *a = *b;
+    *b = x;
+  }
+}
+
 template <typename T>
 __global__ void transpose_absorb_kernel(const T *src, const T *sh, T *dst, int rows, int cols,
                                         int G) {

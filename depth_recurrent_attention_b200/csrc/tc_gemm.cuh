@@ -7,12 +7,15 @@
 //   warp 1      TMEM allocator + single-thread MMA issuer (tcgen05.mma, commit to barriers)
 //   warps 2-5   epilogue: tcgen05.ld of the 128 x BN accumulator, row r per thread, then the
 //               caller's epilogue functor on column segments of SEG values
-//   warps 6-9   (GATHER only) A producers: 16-byte cp.async of gathered rows into the
-//               128B-swizzled layout TMA would have written
+//   warps 6-7   (GATHER only) A producers: 16-byte cp.async of gathered rows into the
+//               128B-swizzled layout TMA would have written (two warps keep the block at
+//               8 warps, so the epilogue may use up to 255 registers a thread)
 // Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap the MMAs of
 // tile i+1.  Every wait is bounded (tc::mbar_wait); on expiry the CTA winds down and the
 // device error flag is set.
 #pragma once
+#include <type_traits>
+
 #include "tc_common.cuh"
 
 namespace dreamer {
@@ -54,13 +57,24 @@ __device__ __forceinline__ bool tc_tile_rows(const TcGemmArgs &a, int mt, int &g
   return m0 < m1;
 }
 
-template <int BN, int BK, int STAGES, bool GATHER>
+// Epilogues that declare STAGED = true get the coalesced store path: each epilogue warp
+// passes its 32 rows x up to 64 columns through shared memory so that a row's columns are
+// spread over 8 lanes (transform<SEG> runs first in the row-per-thread layout, then
+// store_rows<NIT, NV> in the coalesced one).
+template <class E, class = void> struct EpiStaged { static constexpr bool value = false; };
+template <class E> struct EpiStaged<E, std::void_t<decltype(E::STAGED)>> {
+  static constexpr bool value = E::STAGED;
+};
+
+template <int BN, int BK, int STAGES, bool GATHER, bool STAGED = false>
 struct TcGemmCfg {
   static constexpr int A_BYTES = 128 * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int THREADS = GATHER ? 320 : 192;
+  static constexpr int THREADS = GATHER ? 256 : 192;
+  static constexpr int STG_BYTES = STAGED ? 4 * 32 * 64 * 4 : 0;  // 4 warps x 32 x 64 fp32
   // at least 120 KB so that a second CTA never shares the SM (and its 512 TMEM columns)
-  static constexpr int SMEM_USED = STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*bars*/;
+  static constexpr int SMEM_USED =
+      STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*bars*/ + STG_BYTES;
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static_assert(SMEM_USED <= 227 * 1024, "shared memory");
   static constexpr uint32_t IDESC = idesc_bf16_m128(BN);
@@ -76,7 +90,8 @@ template <int BN, int BK, int STAGES, bool GATHER, int SEG, class Epi, bool ROWP
 __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    TcGemmArgs a, Epi epi) {
-  using C = TcGemmCfg<BN, BK, STAGES, GATHER>;
+  constexpr bool STAGED = EpiStaged<Epi>::value && !ROWPASS;
+  using C = TcGemmCfg<BN, BK, STAGES, GATHER, STAGED>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
@@ -85,6 +100,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
   uint64_t *full = bars, *empty = bars + STAGES, *tfull = bars + 2 * STAGES, *tempty = tfull + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  float *stage_buf = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NT = a.N / BN;
@@ -106,7 +122,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; s++) {
-      mbar_init(smem_u32(&full[s]), GATHER ? 1 + 128 : 1);
+      mbar_init(smem_u32(&full[s]), GATHER ? 1 + 64 : 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
     for (int i = 0; i < 2; i++) {
@@ -210,18 +226,74 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
       if constexpr (ROWPASS) {
         if (nt == 0) epi.row_begin(st);
       }
-#pragma unroll 1
-      for (int sg = 0; sg < BN / SEG; sg++) {
-        float v[SEG];
-        if (SEG >= 32) {
+      if constexpr (STAGED) {
+        // Passes of PW = min(SEG, 64) columns.  With PW = 64 lane j of a row holds columns
+        // 4j..4j+3 and 32+4j..32+4j+3 (NV = 8), so rotate-half partners 32 apart meet in
+        // one lane; 8 lanes cover a row, 4 rows a step.  PW = 32: 4 columns a lane (NV = 4).
+        // PW = 16: 4 lanes a row, 8 rows a step.
+        constexpr int PW = SEG < 64 ? SEG : 64;
+        constexpr int CPR = PW / 4;                 // 16-byte chunks per staged row
+        constexpr int LPR = PW == 16 ? 4 : 8;       // lanes per row in the coalesced phase
+        constexpr int NV = PW == 64 ? 8 : 4;        // values per lane and row
+        constexpr int RPI = 32 / LPR;               // rows per step
+        constexpr int NIT = 32 / RPI;               // steps per pass
+        constexpr int SW = CPR >= 8 ? 7 : CPR - 1;  // chunk swizzle mask
+        float *stg = stage_buf + q * 32 * 64;
+        const int cj = lane % LPR;
+        int crow[NIT], ctok[NIT];
 #pragma unroll
-          for (int c = 0; c < SEG; c += 32) tmem_ld32(base + sg * SEG + c, v + c);
-        } else {
-          tmem_ld16(base + sg * SEG, v);
+        for (int i = 0; i < NIT; i++) {
+          const int rr = m0 + q * 32 + i * RPI + lane / LPR;
+          crow[i] = rr < m1 ? rr : -1;
+          ctok[i] = rr < m1 ? (a.arow ? a.arow[rr] / a.arow_div : rr) : 0;
         }
-        if (valid) {
-          if constexpr (ROWPASS) epi.template row_apply<SEG>(st, r, token, g, n0 + sg * SEG, v);
-          else epi.template operator()<SEG>(r, token, g, n0 + sg * SEG, v);
+#pragma unroll 1
+        for (int sg = 0; sg < BN / SEG; sg++) {
+          float v[SEG];
+          if (SEG >= 32) {
+#pragma unroll
+            for (int c = 0; c < SEG; c += 32) tmem_ld32(base + sg * SEG + c, v + c);
+          } else {
+            tmem_ld16(base + sg * SEG, v);
+          }
+          if (valid) epi.template transform<SEG>(r, token, g, n0 + sg * SEG, v);
+#pragma unroll
+          for (int c = 0; c < SEG; c += PW) {
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < CPR; j++)
+              *reinterpret_cast<float4 *>(stg + lane * PW + ((j ^ (lane & SW)) << 2)) =
+                  make_float4(v[c + 4 * j], v[c + 4 * j + 1], v[c + 4 * j + 2], v[c + 4 * j + 3]);
+            __syncwarp();
+            float cv[NIT][NV];
+#pragma unroll
+            for (int i = 0; i < NIT; i++) {
+              const int rl = i * RPI + lane / LPR;
+#pragma unroll
+              for (int hh = 0; hh < NV / 4; hh++) {
+                const int ch = cj + hh * 8;
+                const float4 t4 = *reinterpret_cast<const float4 *>(stg + rl * PW + ((ch ^ (rl & SW)) << 2));
+                cv[i][4 * hh] = t4.x; cv[i][4 * hh + 1] = t4.y;
+                cv[i][4 * hh + 2] = t4.z; cv[i][4 * hh + 3] = t4.w;
+              }
+            }
+            epi.template store_rows<NIT, NV>(crow, ctok, g, n0 + sg * SEG + c + cj * 4, cv);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int sg = 0; sg < BN / SEG; sg++) {
+          float v[SEG];
+          if (SEG >= 32) {
+#pragma unroll
+            for (int c = 0; c < SEG; c += 32) tmem_ld32(base + sg * SEG + c, v + c);
+          } else {
+            tmem_ld16(base + sg * SEG, v);
+          }
+          if (valid) {
+            if constexpr (ROWPASS) epi.template row_apply<SEG>(st, r, token, g, n0 + sg * SEG, v);
+            else epi.template operator()<SEG>(r, token, g, n0 + sg * SEG, v);
+          }
         }
       }
       tc_fence_before();
@@ -232,9 +304,9 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
     }
   } else if (GATHER) {
     // ------------------------------------------------------------- gathered A producers
-    const int tid = threadIdx.x - 192;  // 0..127
+    const int tid = threadIdx.x - 192;  // 0..63
     const int c = tid & 7;              // 16-byte chunk of the 128-byte row slice
-    const int rsub = tid >> 3;          // 0..15
+    const int rsub = tid >> 3;          // 0..7
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
@@ -242,11 +314,11 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
       int g, m0, m1;
       const int mt = t / NT;
       tc_tile_rows(a, mt, g, m0, m1);
-      const bf16 *src[8];
-      uint32_t bytes[8];
+      const bf16 *src[16];
+      uint32_t bytes[16];
 #pragma unroll
-      for (int p = 0; p < 8; p++) {
-        const int rr = p * 16 + rsub, r = m0 + rr;
+      for (int p = 0; p < 16; p++) {
+        const int rr = p * 8 + rsub, r = m0 + rr;
         const bool v = r < m1;
         src[p] = a.A + (v ? (long)(a.arow[r] / a.arow_div) * a.lda : 0) + c * 8;
         bytes[p] = v ? 16u : 0u;
@@ -255,8 +327,8 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
         if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag, a.err)) { ok = false; break; }
         const uint32_t dst0 = smem_u32(sA + s * C::A_BYTES);
 #pragma unroll
-        for (int p = 0; p < 8; p++) {
-          const int rr = p * 16 + rsub;
+        for (int p = 0; p < 16; p++) {
+          const int rr = p * 8 + rsub;
           cp_async16(dst0 + rr * 128 + ((c ^ (rr & 7)) << 4), src[p] + kb * 64, bytes[p]);
         }
         cp_async_arrive(smem_u32(&full[s]));

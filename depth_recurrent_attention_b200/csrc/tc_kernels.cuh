@@ -100,8 +100,9 @@ struct EpiTopK {
   template <int SEG>
   __device__ __forceinline__ void row_apply(State &s, int r, int token, int g, int n0,
                                             const float *vals) const {
-    // candidates against the current k-th entry first (straight-line), then a rolled
-    // insertion for the few that qualify (keeps the code small and the warp convergent)
+    // candidates against the current k-th entry first (straight-line), then one insertion
+    // per qualifying candidate, picked out of the registers by a select chain (a dynamically
+    // indexed array would live in local memory) and placed by an unrolled compare-and-swap
     float vb[SEG];
     unsigned mask = 0;
 #pragma unroll
@@ -114,10 +115,16 @@ struct EpiTopK {
     while (mask) {
       const int i = __ffs(mask) - 1;
       mask &= mask - 1;
-      float cv = vb[i], cz = vals[i] * zscale;
+      float cv = 0.f, cz = 0.f;
+#pragma unroll
+      for (int j = 0; j < SEG; j++)
+        if (j == i) {
+          cv = vb[j];
+          cz = vals[j] * zscale;
+        }
       int ce = n0 + i;
       if (!better(cv, ce, s.v[KT - 1], s.e[KT - 1])) continue;
-#pragma unroll 1
+#pragma unroll
       for (int j = 0; j < KT; j++) {  // insertion by compare-and-swap down the sorted list
         if (better(cv, ce, s.v[j], s.e[j])) {
           const float tv = s.v[j], tz = s.z[j];
@@ -239,7 +246,8 @@ static void tc_destroy(dreamer_handle *h) {}
 template <int BN, int BK, int ST, bool GATHER, int SEG, class Epi, bool ROWPASS = false>
 static void tc_launch(dreamer_handle *h, const dreamer::tc::TcGemmArgs &a, const CUtensorMap &ta,
                       const CUtensorMap &tb, long max_tiles, const Epi &epi, cudaStream_t s) {
-  using Cfg = dreamer::tc::TcGemmCfg<BN, BK, ST, GATHER>;
+  using Cfg = dreamer::tc::TcGemmCfg<BN, BK, ST, GATHER,
+                                     dreamer::tc::EpiStaged<Epi>::value && !ROWPASS>;
   auto kern = dreamer::tc::tc_gemm_kernel<BN, BK, ST, GATHER, SEG, Epi, ROWPASS>;
   if (ROWPASS) max_tiles /= (a.N / BN);  // one unit of work per row tile
   static bool attr_set = false;
@@ -285,6 +293,18 @@ static bool tc_gemm_ok(dreamer_handle *h, const dreamer::GemmArgs &a) {
   return a.N % 256 == 0 && a.K % 64 == 0 && (d == 64 || d == 128);
 }
 
+// N tile of the projection GEMMs: the wider tile reads A fewer times, the narrower one
+// spreads a small problem over more SMs; take the one with the shorter critical path
+// (waves of tiles x tile width plus a fixed per-tile cost of about 32 columns).
+static int tc_pick_bn(dreamer_handle *h, const dreamer::GemmArgs &a) {
+  const long mt = (a.M + 127) / 128 + (a.goffs ? a.G : 0);
+  auto cost = [&](int bn) {
+    const long tiles = mt * (a.N / bn);
+    return ((tiles + h->num_sms - 1) / h->num_sms) * (bn + 32);
+  };
+  return (a.N % 256 == 0 && cost(256) <= cost(128)) ? 256 : 128;
+}
+
 template <typename T>
 static bool tc_gemm_qkv(dreamer_handle *h, const dreamer::GemmArgs &a, const dreamer::EpiQKV<T> &e,
                         cudaStream_t s) {
@@ -293,14 +313,17 @@ static bool tc_gemm_qkv(dreamer_handle *h, const dreamer::GemmArgs &a, const dre
     CUtensorMap ta, tb;
     long mt;
     const int *tiles = h->ptiles_b;
-    if (!tc_prepare<256, 64>(h, a, tiles, a.M, t, ta, tb, mt)) return false;
     const bool gather = a.arow != nullptr;
-    if (h->cfg.head_dim == 64) {
+    // 64-column segments: the staged epilogue rotates pairs 32 columns apart (head dim 64,
+    // or 128 in perm order)
+    if (tc_pick_bn(h, a) == 256) {
+      if (!tc_prepare<256, 64>(h, a, tiles, a.M, t, ta, tb, mt)) return false;
       if (gather) tc_launch<256, 64, 4, true, 64>(h, t, ta, tb, mt, e, s);
       else tc_launch<256, 64, 4, false, 64>(h, t, ta, tb, mt, e, s);
     } else {
-      if (gather) tc_launch<256, 64, 4, true, 128>(h, t, ta, tb, mt, e, s);
-      else tc_launch<256, 64, 4, false, 128>(h, t, ta, tb, mt, e, s);
+      if (!tc_prepare<128, 64>(h, a, tiles, a.M, t, ta, tb, mt)) return false;
+      if (gather) tc_launch<128, 64, 6, true, 64>(h, t, ta, tb, mt, e, s);
+      else tc_launch<128, 64, 6, false, 64>(h, t, ta, tb, mt, e, s);
     }
     return true;
   }
@@ -314,9 +337,15 @@ static bool tc_gemm_o(dreamer_handle *h, const dreamer::GemmArgs &a, const dream
     dreamer::tc::TcGemmArgs t{};
     CUtensorMap ta, tb;
     long mt;
-    if (!tc_prepare<256, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
-    if (a.arow) tc_launch<256, 64, 4, true, 32>(h, t, ta, tb, mt, e, s);
-    else tc_launch<256, 64, 4, false, 32>(h, t, ta, tb, mt, e, s);
+    if (tc_pick_bn(h, a) == 256) {
+      if (!tc_prepare<256, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
+      if (a.arow) tc_launch<256, 64, 4, true, 64>(h, t, ta, tb, mt, e, s);
+      else tc_launch<256, 64, 4, false, 64>(h, t, ta, tb, mt, e, s);
+    } else {
+      if (!tc_prepare<128, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
+      if (a.arow) tc_launch<128, 64, 6, true, 64>(h, t, ta, tb, mt, e, s);
+      else tc_launch<128, 64, 6, false, 64>(h, t, ta, tb, mt, e, s);
+    }
     return true;
   }
   return false;
@@ -374,13 +403,13 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
     default:
       break;
   }
-  tc_launch<256, 64, 4, false, 32>(h, t2, ta2, tb2, mt2, EpiStoreF32{h->zbuf, h->ldz, E}, s);
+  tc_launch<256, 64, 4, false, 64>(h, t2, ta2, tb2, mt2, EpiStoreF32{h->zbuf, h->ldz, E}, s);
   TopkArgs k{};
   k.n_tok = n; k.E = E; k.k = c.top_k; k.mode = 0;
   k.z = h->zbuf; k.ldz = h->ldz; k.zscale = 1.0f / sqrtf((float)dr);
   k.bias = h->bias; k.idx = idx; k.w = w; k.counts_a = counts_a; k.counts_b = counts_b;
   ++g_launches;
-  topk_kernel<<<(n + 7) / 8, 256, 0, s>>>(k);
+  launch_topk(k, s);
   return true;
 }
 
@@ -441,21 +470,21 @@ static bool tc_expert(dreamer_handle *h, const void *X, int n, cudaStream_t s) {
           !tc_prepare<256, 16>(h, dn, h->etiles_b, rows + 128, td, tad, tbd, mtd))
         return false;
       tc_launch<16, 64, 8, true, 16>(h, tu, tau, tbu, mtu, eu, s);
-      tc_launch<256, 16, 8, false, 32>(h, td, tad, tbd, mtd, ed, s);
+      tc_launch<256, 16, 8, false, 64>(h, td, tad, tbd, mtd, ed, s);
       return true;
     case 32:
       if (!tc_prepare<32, 64>(h, up, h->etiles_b, rows, tu, tau, tbu, mtu) ||
           !tc_prepare<256, 32>(h, dn, h->etiles_b, rows + 128, td, tad, tbd, mtd))
         return false;
-      tc_launch<32, 64, 8, true, 16>(h, tu, tau, tbu, mtu, eu, s);
-      tc_launch<256, 32, 6, false, 32>(h, td, tad, tbd, mtd, ed, s);
+      tc_launch<32, 64, 8, true, 32>(h, tu, tau, tbu, mtu, eu, s);
+      tc_launch<256, 32, 6, false, 64>(h, td, tad, tbd, mtd, ed, s);
       return true;
     default:
       if (!tc_prepare<64, 64>(h, up, h->etiles_b, rows, tu, tau, tbu, mtu) ||
           !tc_prepare<256, 64>(h, dn, h->etiles_b, rows + 128, td, tad, tbd, mtd))
         return false;
-      tc_launch<64, 64, 8, true, 16>(h, tu, tau, tbu, mtu, eu, s);
-      tc_launch<256, 64, 4, false, 32>(h, td, tad, tbd, mtd, ed, s);
+      tc_launch<64, 64, 8, true, 64>(h, tu, tau, tbu, mtu, eu, s);
+      tc_launch<256, 64, 4, false, 64>(h, td, tad, tbd, mtd, ed, s);
       return true;
   }
 }

@@ -230,7 +230,11 @@ def test_small_free_running_drift_reported(cuda):
 @pytest.mark.parametrize("kw", [dict(n_experts=4, top_k=4, depth=4),
                                 dict(n_experts=8, top_k=8, depth=3, n_proj_experts=1),
                                 dict(n_experts=4, top_k=4, depth=3, variant=1),
-                                dict(n_experts=4, top_k=4, depth=3, variant=2)])
+                                dict(n_experts=4, top_k=4, depth=3, variant=2),
+                                # head dim 128: q/k columns in the permuted GEMM order
+                                dict(n_experts=4, top_k=4, depth=3, n_heads=4, head_dim=128),
+                                dict(n_experts=8, top_k=8, depth=2, n_heads=4, head_dim=128,
+                                     n_proj_experts=1)])
 def test_small_flip_free_all_depths_bf16(cuda, kw):
     torch = _torch()
     cfg = configs.SMALL.with_(**kw)
@@ -275,6 +279,7 @@ def flip_free(cfg):
     ("small", [300, 1, 77, 299], {}),
     ("small", [300, 1, 77, 299], dict(n_experts=4, top_k=4, depth=4)),
     ("small", [40, 0, 17], dict(n_experts=4, top_k=4, depth=3, n_proj_experts=1)),
+    ("small", [300, 1, 77, 299], dict(n_experts=4, top_k=4, depth=3, n_heads=4, head_dim=128)),
 ])
 def test_decode_step(cuda, base, lens, kw):
     torch = _torch()
