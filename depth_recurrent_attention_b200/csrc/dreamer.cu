@@ -545,7 +545,7 @@ static void route_rows(dreamer_handle *h, int mode, int l, const void *X, int n,
   t.bias = mode == 0 ? h->bias : nullptr;
   t.idx = idx; t.w = wout; t.counts_a = counts_a; t.counts_b = counts_b;
   ++g_launches;
-  launch_topk(t, s);
+  launch_topk(t, h->num_sms, s);
 }
 
 static void trace_depth(dreamer_handle *h, const dreamer_trace *tr, int l, int n, bool prefill,

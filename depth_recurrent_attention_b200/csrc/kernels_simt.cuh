@@ -73,29 +73,46 @@ template <typename T> struct EpiQKV {
     }
   }
 
-  // Coalesced layout: a pass of 64 columns [c64, c64 + 64) inside one head; the lane holds
-  // columns col..col+3 (v[i][0..3]) and col+32..col+35 (v[i][4..7]) of rows r[i].
+  // Coalesced layout: a pass of 64 columns inside one head; the lane holds columns col..col+3
+  // (v[i][0..3]) and col+32..col+35 (v[i][4..7]) of rows r[i]; ax[i] is the row's position
+  // (-1: decode slot outside the cache).
   static constexpr bool STAGED = true;
+  using Aux = int;
+  __device__ __forceinline__ int row_aux(int r, int token) const {
+    return r < 0 ? 0 : position(token);
+  }
   template <int NR, int NV>
-  __device__ __forceinline__ void store_rows(const int *r, const int *tok, int g, int col,
-                                             const float (*v)[NV]) const {
+  __device__ __forceinline__ void store_rows(const int *r, const int *tok, const int *ax, int g,
+                                             int col, const float (*v)[NV]) const {
     static_assert(NV == 8, "QKV passes are 64 columns wide");
     const int nc = col + col_lo;
     const int blk = nc / h, hc = nc % h;
-    const int hb = blk * h + hc - hc % d;   // first column of the head
     const int cin = hc % d;                 // computed column inside the head (cin % 64 < 32)
+    const int hd0 = hc - cin;               // first column of the head inside the block
+    // token-strided destinations (everything but the decode caches): base + token * stride
+    T *base = nullptr;
+    long stride = 0;
+    const bool cache = mode == 1 && (blk == 1 || blk == 2);
+    if (blk <= 2) { base = qkv_sa + blk * h + hd0; stride = 3L * h; }
+    else if (blk == 3) { base = q_da + hd0; stride = h; }
+    else { base = da_kv + ((long)l * 2 + (blk - 4)) * h + hd0; stride = 2L * L * h; }
+    auto row_dst = [&](int i) -> T * {  // head base of row i, or null
+      if (!cache) return base + (long)tok[i] * stride;
+      if (ax[i] < 0) return nullptr;
+      T *cb = blk == 1 ? k_cache : v_cache;
+      return cb + ((((long)l * B + tok[i]) * (h / d) + hd0 / d) * cap + ax[i]) * d;
+    };
     if (blk <= 1) {
       // token RoPE: head columns o and o + d/2, frequency o
       const int o = perm ? unperm(cin) : cin;
 #pragma unroll
       for (int i = 0; i < NR; i++) {
         if (r[i] < 0) continue;
-        const int pos = position(tok[i]);
-        if (pos < 0) {
+        if (ax[i] < 0) {
           raise_dev_error(err, DEV_BAD_INDEX);
           continue;
         }
-        const float4 *cs = reinterpret_cast<const float4 *>(rope_tok + (long)pos * (d / 2) + o);
+        const float4 *cs = reinterpret_cast<const float4 *>(rope_tok + (long)ax[i] * (d / 2) + o);
         const float4 c01 = cs[0], c23 = cs[1];
         const float cc[4] = {c01.x, c01.z, c23.x, c23.z}, sn[4] = {c01.y, c01.w, c23.y, c23.w};
         float a[4], b[4];
@@ -104,11 +121,9 @@ template <typename T> struct EpiQKV {
           a[j] = v[i][j] * cc[j] - v[i][4 + j] * sn[j];
           b[j] = v[i][4 + j] * cc[j] + v[i][j] * sn[j];
         }
-        T *da = dest(tok[i], hb + o);
-        if (da) {
-          store4(da, a);
-          store4(da + d / 2, b);
-        }
+        T *dst = row_dst(i);
+        store4(dst + o, a);
+        store4(dst + o + d / 2, b);
       }
       return;
     }
@@ -153,7 +168,7 @@ template <typename T> struct EpiQKV {
 #pragma unroll
       for (int i = 0; i < NR; i++) {
         if (r[i] < 0) continue;
-        T *dst = dest(tok[i], hb + cin);
+        T *dst = base + (long)tok[i] * stride + cin;
         store4(dst, w[i]);
         store4(dst + 32, w[i] + 4);
       }
@@ -162,13 +177,13 @@ template <typename T> struct EpiQKV {
 #pragma unroll
     for (int i = 0; i < NR; i++) {  // v_SA, v_DA: as they are
       if (r[i] < 0) continue;
-      T *dst = dest(tok[i], hb + cin);
+      T *dst = row_dst(i);
       if (!dst) {
         raise_dev_error(err, DEV_BAD_INDEX);
         continue;
       }
-      store4(dst, v[i]);
-      store4(dst + 32, v[i] + 4);
+      store4(dst + cin, v[i]);
+      store4(dst + cin + 32, v[i] + 4);
     }
   }
 
@@ -269,11 +284,18 @@ template <typename T> struct EpiO {
   static constexpr bool STAGED = true;
   template <int SEG>
   __device__ __forceinline__ void transform(int, int, int, int, float *) const {}
+  struct Aux {
+    float s, ir;  // sigma and 1/rms of the row's token
+  };
+  __device__ __forceinline__ Aux row_aux(int r, int token) const {
+    if (r < 0) return Aux{0.f, 0.f};
+    return Aux{psig ? psig[token] : 1.0f, res_mode == 2 ? 1.f : inv_rms[token]};
+  }
   // Coalesced layout (NV values a lane and row: 4 at col, and with NV = 8 four more at
   // col + 32); all residual loads are issued before the first store.
   template <int NR, int NV>
-  __device__ __forceinline__ void store_rows(const int *r, const int *tok, int g, int col,
-                                             const float (*v)[NV]) const {
+  __device__ __forceinline__ void store_rows(const int *r, const int *tok, const Aux *ax, int g,
+                                             int col, const float (*v)[NV]) const {
     float gv[NV];
 #pragma unroll
     for (int hh = 0; hh < NV / 4; hh++) {
@@ -293,8 +315,7 @@ template <typename T> struct EpiO {
 #pragma unroll
     for (int i = 0; i < NR; i++) {
       if (r[i] < 0) continue;
-      const float s = psig ? psig[tok[i]] : 1.0f;
-      const float ir = res_mode == 2 ? 1.f : inv_rms[tok[i]];
+      const float s = ax[i].s, ir = ax[i].ir;
       float o[NV];
 #pragma unroll
       for (int j = 0; j < NV; j++) o[j] = (res_mode == 2 ? xr[i][j] : gv[j] * xr[i][j] * ir) + s * v[i][j];
@@ -318,21 +339,6 @@ template <typename T> struct EpiUp {
     for (int i = 0; i < SEG; i++) v[i] = v[i] / (1.0f + __expf(-v[i]));
 #pragma unroll
     for (int i = 0; i < SEG; i += 8) store8(H + (long)r * m + n0 + i, v + i);
-  }
-  static constexpr bool STAGED = true;
-  template <int SEG>
-  __device__ __forceinline__ void transform(int, int, int, int, float *v) const {
-#pragma unroll
-    for (int i = 0; i < SEG; i++) v[i] = v[i] / (1.0f + __expf(-v[i]));
-  }
-  template <int NR, int NV>
-  __device__ __forceinline__ void store_rows(const int *r, const int *, int, int col,
-                                             const float (*v)[NV]) const {
-#pragma unroll
-    for (int i = 0; i < NR; i++)
-      if (r[i] >= 0)
-#pragma unroll
-        for (int hh = 0; hh < NV / 4; hh++) store4(H + (long)r[i] * m + col + 32 * hh, v[i] + 4 * hh);
   }
 };
 
@@ -363,18 +369,6 @@ template <typename T> struct EpiDownStore {
 #pragma unroll
     for (int i = 0; i < SEG; i += 8) store8(Y + (long)r * h + n0 + i, v + i);
   }
-  static constexpr bool STAGED = true;
-  template <int SEG>
-  __device__ __forceinline__ void transform(int, int, int, int, float *) const {}
-  template <int NR, int NV>
-  __device__ __forceinline__ void store_rows(const int *r, const int *, int, int col,
-                                             const float (*v)[NV]) const {
-#pragma unroll
-    for (int i = 0; i < NR; i++)
-      if (r[i] >= 0)
-#pragma unroll
-        for (int hh = 0; hh < NV / 4; hh++) store4(Y + (long)r[i] * h + col + 32 * hh, v[i] + 4 * hh);
-  }
 };
 
 // Plain fp32 store of columns < N (router queries and scores).
@@ -384,28 +378,14 @@ struct EpiStoreF32 {
   int N;
   template <int SEG>
   __device__ __forceinline__ void operator()(int r, int token, int g, int n0, float *v) const {
+    float *p = C + (long)r * ldc + n0;
+    if (n0 + SEG <= N && (ldc & 3) == 0) {
 #pragma unroll
-    for (int i = 0; i < SEG; i++)
-      if (n0 + i < N) C[(long)r * ldc + n0 + i] = v[i];
-  }
-  static constexpr bool STAGED = true;
-  template <int SEG>
-  __device__ __forceinline__ void transform(int, int, int, int, float *) const {}
-  template <int NR, int NV>
-  __device__ __forceinline__ void store_rows(const int *r, const int *, int, int col,
-                                             const float (*v)[NV]) const {
+      for (int i = 0; i < SEG; i += 4) store4(p + i, v + i);
+    } else {
 #pragma unroll
-    for (int i = 0; i < NR; i++) {
-      if (r[i] < 0) continue;
-#pragma unroll
-      for (int hh = 0; hh < NV / 4; hh++) {
-        const int c0 = col + 32 * hh;
-        float *p = C + (long)r[i] * ldc + c0;
-        if (c0 + 4 <= N && (ldc & 3) == 0) store4(p, v[i] + 4 * hh);
-        else
-          for (int j = 0; j < 4; j++)
-            if (c0 + j < N) p[j] = v[i][4 * hh + j];
-      }
+      for (int i = 0; i < SEG; i++)
+        if (n0 + i < N) p[i] = v[i];
     }
   }
 };
@@ -755,90 +735,87 @@ __device__ __forceinline__ bool better(float v1, int e1, float v2, int e2) {
   return v1 > v2 || (v1 == v2 && e1 < e2);
 }
 
-// One warp per token.  Lane j scans the experts e = j (mod 32) and keeps its best KT (biased
-// score, index) pairs in registers, sorted, inserting by a fully unrolled compare-and-swap
-// pass (no dynamically indexed arrays, so nothing spills to local memory); then k rounds of a
-// warp argmax over the lanes' heads, the winning lane shifting its list up.  KT >= k.
-template <int KT>
+// Top-k by warps.  A warp keeps its running top k (k <= 32) distributed over its lanes, lane j
+// holding the j-th best (biased score, expert, raw score) pair; it reads 32 candidates at a
+// time and inserts the ones that beat entry k-1, each by a ballot for the insertion position
+// and a one-lane shift (no per-lane arrays, nothing in local memory).  WPT warps share a
+// token: each scans a slice of the experts, then warp 0 merges the others' lists.  Ties go
+// to the lower expert index; a NaN score ranks last.  Writes the experts in descending order
+// of biased score, w = sigmoid(raw) normalised over the k (mode 0) or as it is (mode 1), and
+// counts each pick into the histograms.
+template <int WPT>
 __global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= a.n_tok) return;
-  const float *zr = a.z + (long)warp * a.ldz;
-  float lv[KT], lz[KT];
-  int le[KT];
-#pragma unroll
-  for (int i = 0; i < KT; i++) {
-    lv[i] = -INFINITY;
-    lz[i] = 0.f;
-    le[i] = 0x7fffffff;
-  }
+  constexpr unsigned FULL = 0xffffffffu;
+  constexpr int NONE = 0x7fffffff;
+  __shared__ float mv[WPT][32], mz[WPT][32];
+  __shared__ int me[WPT][32];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int tok = WPT == 1 ? blockIdx.x * 8 + wib : blockIdx.x;
+  if (tok >= a.n_tok) return;  // whole warp (WPT 1) or whole block (WPT > 1)
   const int k = a.k;
-#pragma unroll 4
-  for (int e = lane; e < a.E; e += 32) {
-    const float z = zr[e] * a.zscale;
-    float v = z + (a.bias ? a.bias[e] : 0.f);
-    if (v != v) v = -INFINITY;  // a NaN score ranks last; indices stay valid
-    if (!better(v, e, lv[KT - 1], le[KT - 1])) continue;
-    float cz = z;
-    int ce = e;
-#pragma unroll
-    for (int j = 0; j < KT; j++) {
-      if (better(v, ce, lv[j], le[j])) {
-        const float tv = lv[j], tz = lz[j];
-        const int te = le[j];
-        lv[j] = v; lz[j] = cz; le[j] = ce;
-        v = tv; cz = tz; ce = te;
-      }
+  const float *zr = a.z + (long)tok * a.ldz;
+  float lv = -INFINITY, lz = 0.f;
+  int le = NONE;
+  float tv = -INFINITY;
+  int te = NONE;
+  auto insert = [&](float cv, int ce, float cz) {
+    const int pos = __popc(__ballot_sync(FULL, lane < k && better(lv, le, cv, ce)));
+    const float uv = __shfl_up_sync(FULL, lv, 1), uz = __shfl_up_sync(FULL, lz, 1);
+    const int ue = __shfl_up_sync(FULL, le, 1);
+    if (lane > pos) {
+      lv = uv; lz = uz; le = ue;
+    } else if (lane == pos) {
+      lv = cv; lz = cz; le = ce;
     }
+    tv = __shfl_sync(FULL, lv, k - 1);
+    te = __shfl_sync(FULL, le, k - 1);
+  };
+  auto offer = [&](float v, int e, float z) {  // one candidate a lane (e == NONE: none)
+    unsigned m = __ballot_sync(FULL, e != NONE && better(v, e, tv, te));
+    while (m) {
+      const int src = __ffs(m) - 1;
+      m &= m - 1;
+      const float cv = __shfl_sync(FULL, v, src), cz = __shfl_sync(FULL, z, src);
+      const int ce = __shfl_sync(FULL, e, src);
+      if (better(cv, ce, tv, te)) insert(cv, ce, cz);
+    }
+  };
+  const int per = (a.E + WPT - 1) / WPT;
+  const int e0 = WPT > 1 ? wib * per : 0, e1 = WPT > 1 ? min(a.E, e0 + per) : a.E;
+  for (int b = e0; b < e1; b += 32) {
+    const int e = b + lane;
+    float z = 0.f, v = -INFINITY;
+    int ce = NONE;
+    if (e < e1) {
+      z = zr[e] * a.zscale;
+      v = z + (a.bias ? a.bias[e] : 0.f);
+      if (v != v) v = -INFINITY;
+      ce = e;
+    }
+    offer(v, ce, z);
   }
-  float wsum = 0.f;
-  int myidx = 0;
-  float myz = 0.f;
-  for (int s = 0; s < k; s++) {
-    float bv = lv[0];
-    int be = le[0];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (better(ov, oe, bv, be)) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    const bool win = le[0] == be;
-    const int src = __ffs(__ballot_sync(0xffffffffu, win)) - 1;
-    const float zw = __shfl_sync(0xffffffffu, lz[0], src);
-    if (win) {
-#pragma unroll
-      for (int j = 0; j + 1 < KT; j++) {
-        lv[j] = lv[j + 1]; lz[j] = lz[j + 1]; le[j] = le[j + 1];
-      }
-      lv[KT - 1] = -INFINITY; le[KT - 1] = 0x7fffffff;
-    }
-    const float sg = 1.0f / (1.0f + __expf(-zw));
-    wsum += sg;
-    if (lane == s) {
-      myidx = be;
-      myz = sg;
-    }
+  if (WPT > 1) {
+    mv[wib][lane] = lane < k ? lv : -INFINITY;
+    me[wib][lane] = lane < k ? le : NONE;
+    mz[wib][lane] = lz;
+    __syncthreads();
+    if (wib != 0) return;
+    for (int w = 1; w < WPT; w++) offer(mv[w][lane], me[w][lane], mz[w][lane]);
   }
+  const float sg = lane < k ? 1.0f / (1.0f + __expf(-lz)) : 0.f;
+  const float ssum = warp_sum(sg);
   if (lane < k) {
-    a.idx[(long)warp * k + lane] = myidx;
-    a.w[(long)warp * k + lane] = (a.mode == 0) ? myz / wsum : myz;
-    if (a.counts_a) atomicAdd(a.counts_a + myidx, 1);
-    if (a.counts_b) atomicAdd(a.counts_b + myidx, 1);
+    a.idx[(long)tok * k + lane] = le;
+    a.w[(long)tok * k + lane] = (a.mode == 0) ? sg / ssum : sg;
+    if (a.counts_a) atomicAdd(a.counts_a + le, 1);
+    if (a.counts_b) atomicAdd(a.counts_b + le, 1);
   }
 }
 
-// Launch with the smallest list length that holds k (k <= 16).
-inline void launch_topk(const TopkArgs &t, cudaStream_t s) {
-  const int blocks = (t.n_tok + 7) / 8;
-  if (t.k <= 2) topk_kernel<2><<<blocks, 256, 0, s>>>(t);
-  else if (t.k <= 4) topk_kernel<4><<<blocks, 256, 0, s>>>(t);
-  else if (t.k <= 8) topk_kernel<8><<<blocks, 256, 0, s>>>(t);
-  else topk_kernel<16><<<blocks, 256, 0, s>>>(t);
+// Eight warps a token when there are too few tokens to fill the GPU with one warp each.
+inline void launch_topk(const TopkArgs &t, int num_sms, cudaStream_t s) {
+  if ((long)t.n_tok * 4 < (long)num_sms * 32) topk_kernel<8><<<t.n_tok, 256, 0, s>>>(t);
+  else topk_kernel<1><<<(t.n_tok + 7) / 8, 256, 0, s>>>(t);
 }
 
 // =======================================================================================

@@ -60,7 +60,8 @@ __device__ __forceinline__ bool tc_tile_rows(const TcGemmArgs &a, int mt, int &g
 // Epilogues that declare STAGED = true get the coalesced store path: each epilogue warp
 // passes its 32 rows x up to 64 columns through shared memory so that a row's columns are
 // spread over 8 lanes (transform<SEG> runs first in the row-per-thread layout, then
-// store_rows<NIT, NV> in the coalesced one).
+// store_rows<NIT, NV> in the coalesced one, with Epi::Aux values from row_aux(r, token)
+// looked up once per tile for each of the lane's rows).
 template <class E, class = void> struct EpiStaged { static constexpr bool value = false; };
 template <class E> struct EpiStaged<E, std::void_t<decltype(E::STAGED)>> {
   static constexpr bool value = E::STAGED;
@@ -241,14 +242,16 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
         float *stg = stage_buf + q * 32 * 64;
         const int cj = lane % LPR;
         int crow[NIT], ctok[NIT];
+        typename Epi::Aux caux[NIT];  // per-row values the epilogue looks up once per tile
 #pragma unroll
         for (int i = 0; i < NIT; i++) {
           const int rr = m0 + q * 32 + i * RPI + lane / LPR;
           crow[i] = rr < m1 ? rr : -1;
           ctok[i] = rr < m1 ? (a.arow ? a.arow[rr] / a.arow_div : rr) : 0;
+          caux[i] = epi.row_aux(crow[i], ctok[i]);
         }
 #pragma unroll 1
-        for (int sg = 0; sg < BN / SEG; sg++) {
+        for (int sg = 0; sg < BN / SEG && m0 + q * 32 < m1; sg++) {
           float v[SEG];
           if (SEG >= 32) {
 #pragma unroll
@@ -277,12 +280,12 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
                 cv[i][4 * hh + 2] = t4.z; cv[i][4 * hh + 3] = t4.w;
               }
             }
-            epi.template store_rows<NIT, NV>(crow, ctok, g, n0 + sg * SEG + c + cj * 4, cv);
+            epi.template store_rows<NIT, NV>(crow, ctok, caux, g, n0 + sg * SEG + c + cj * 4, cv);
           }
         }
       } else {
 #pragma unroll 1
-        for (int sg = 0; sg < BN / SEG; sg++) {
+        for (int sg = 0; sg < BN / SEG && m0 + q * 32 < m1; sg++) {  // skip warps with no rows
           float v[SEG];
           if (SEG >= 32) {
 #pragma unroll

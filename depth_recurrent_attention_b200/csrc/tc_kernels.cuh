@@ -409,7 +409,7 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
   k.z = h->zbuf; k.ldz = h->ldz; k.zscale = 1.0f / sqrtf((float)dr);
   k.bias = h->bias; k.idx = idx; k.w = w; k.counts_a = counts_a; k.counts_b = counts_b;
   ++g_launches;
-  launch_topk(k, s);
+  launch_topk(k, h->num_sms, s);
   return true;
 }
 
