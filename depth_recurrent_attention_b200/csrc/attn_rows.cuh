@@ -45,6 +45,8 @@ struct RowsArgs {
 
 template <typename T, int D, int U>
 __global__ void __launch_bounds__(256) attn_rows_kernel(RowsArgs a) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int VEC = VecOf<T>::N;
   constexpr int CH = D / VEC;
   static_assert(CH >= 1 && CH <= 32 && (32 % CH) == 0, "chunking");
@@ -165,6 +167,8 @@ __global__ void __launch_bounds__(256) attn_rows_kernel(RowsArgs a) {
 // Merge the split partials of decode attention: o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) attn_merge_kernel(RowsArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= a.n_q * a.H) return;
@@ -246,6 +250,8 @@ struct DaBulkArgs {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ __align__(8) uint64_t bars[2];
   __shared__ int abort_flag;

@@ -78,6 +78,17 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// Programmatic dependent launch.  Every kernel of the library calls pdl_wait() before its
+// first global memory access (and before any early return), so it may be launched while the
+// previous kernel on its stream is still draining; pdl_trigger() lets the next kernel's blocks
+// be scheduled.  Kernels that allocate TMEM trigger only after their allocation, so a
+// dependent block can never take the columns a running block still needs.  Both are no-ops
+// for a kernel launched without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Device-side error codes written into the handle's flag word (first writer wins).
 enum DevErr : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_INDEX = 2 };
 __device__ __forceinline__ void raise_dev_error(int *flag, int code) {

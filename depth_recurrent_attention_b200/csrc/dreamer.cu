@@ -7,6 +7,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <utility>
 #include <vector>
 
 #include "../../include/dreamer.h"
@@ -56,6 +57,8 @@ struct dreamer_handle {
   cudaStream_t side = nullptr;   // second stream: DA runs beside SA
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   int use_graph = 1;
+  int use_pdl = 1;               // programmatic dependent launch between kernels of a stream
+  bool pdl_ok[2] = {false, false};  // main / side stream: the last operation was a kernel
   struct GraphEntry {
     int kind;                    // 0 forward, 1 decode
     const void *key[5];
@@ -140,6 +143,44 @@ static int dalloc(dreamer_handle *h, void **p, size_t bytes) {
 static inline int cdiv(long a, long b) { return (int)((a + b - 1) / b); }
 // kernels launched by this thread through the library (read as deltas around each call)
 static thread_local uint64_t g_launches = 0;
+
+// ---- kernel launches with programmatic dependent launch -------------------------------
+// A kernel may start while the previous operation on its stream is still running only if that
+// operation is a kernel (whose completion its pdl_wait() then waits for).  pdl_take() answers
+// that for the stream and records that a kernel is now last; pdl_break() records any other
+// operation (copy, memset, event wait).  Off while stages are timed by events.
+static bool pdl_take(dreamer_handle *h, cudaStream_t s) {
+  bool &ok = h->pdl_ok[s == h->side ? 1 : 0];
+  const bool r = ok && h->use_pdl && !h->prof;
+  ok = true;
+  return r;
+}
+static void pdl_break(dreamer_handle *h, cudaStream_t s) { h->pdl_ok[s == h->side ? 1 : 0] = false; }
+
+template <typename... P, typename... A>
+static void launch_k(dreamer_handle *h, void (*kern)(P...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t s, A &&...args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl_take(h, s) ? 1 : 0;
+  ++g_launches;
+  cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+
+// top-k: eight warps a token when there are too few tokens to fill the GPU with one warp each
+static void launch_topk(dreamer_handle *h, const TopkArgs &t, cudaStream_t s) {
+  if ((long)t.n_tok * 4 < (long)h->num_sms * 32)
+    launch_k(h, topk_kernel<8>, dim3(t.n_tok), dim3(256), 0, s, t);
+  else
+    launch_k(h, topk_kernel<1>, dim3((t.n_tok + 7) / 8), dim3(256), 0, s, t);
+}
 
 #include "tc_kernels.cuh"
 
@@ -277,6 +318,7 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     const long T = h->T;
     if (const char *ev = getenv("DREAMER_NO_TC")) h->use_tc = atoi(ev) ? 0 : 1;
     if (const char *ev = getenv("DREAMER_NO_GRAPH")) h->use_graph = atoi(ev) ? 0 : 1;
+    if (const char *ev = getenv("DREAMER_NO_PDL")) h->use_pdl = atoi(ev) ? 0 : 1;
     CK(cudaHostAlloc((void **)&h->err_host, sizeof(int), cudaHostAllocDefault));
     *h->err_host = 0;
     CK(cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
@@ -462,7 +504,7 @@ static void launch_attn(const AttnArgs &a, int d, cudaStream_t s) {
 
 // depth attention, one CTA per token streaming its depth history through shared memory
 template <typename T>
-static void launch_da_bulk(const RowsArgs &r, int d, cudaStream_t s) {
+static void launch_da_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStream_t s) {
   DaBulkArgs a{};
   a.n_tok = r.n_q; a.H = r.H; a.h = r.h; a.L = r.L; a.l = r.l;
   const long row_bytes = 2L * r.h * sizeof(T);
@@ -477,8 +519,7 @@ static void launch_da_bulk(const RowsArgs &r, int d, cudaStream_t s) {
     // set for the kernel launched (the four head sizes share one pointer type)
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    ++g_launches;
-    kern<<<a.n_tok, threads, smem, s>>>(a);
+    launch_k(h, kern, dim3(a.n_tok), dim3(threads), smem, s, a);
   };
   switch (d) {
     case 16: go(da_bulk_kernel<T, 16>); break;
@@ -490,26 +531,26 @@ static void launch_da_bulk(const RowsArgs &r, int d, cudaStream_t s) {
 
 // depth attention (mode 0) or split decode attention + merge (mode 2)
 template <typename T>
-static void launch_rows(const RowsArgs &a, int d, cudaStream_t s) {
+static void launch_rows(dreamer_handle *h, const RowsArgs &a, int d, cudaStream_t s) {
   if (a.mode == 0 && a.H <= 32 && 2L * a.h * (long)sizeof(T) <= 50 * 1024) {
-    launch_da_bulk<T>(a, d, s);
+    launch_da_bulk<T>(h, a, d, s);
     return;
   }
   const long warps = (long)a.n_q * a.H * (a.mode == 2 ? a.nsplit : 1);
   const int blocks = cdiv(warps, 8);
   switch (d) {
-    case 16: ++g_launches; attn_rows_kernel<T, 16, 4><<<blocks, 256, 0, s>>>(a); break;
-    case 32: ++g_launches; attn_rows_kernel<T, 32, 4><<<blocks, 256, 0, s>>>(a); break;
-    case 64: ++g_launches; attn_rows_kernel<T, 64, 4><<<blocks, 256, 0, s>>>(a); break;
-    default: ++g_launches; attn_rows_kernel<T, 128, 4><<<blocks, 256, 0, s>>>(a); break;
+    case 16: launch_k(h, attn_rows_kernel<T, 16, 4>, dim3(blocks), dim3(256), 0, s, a); break;
+    case 32: launch_k(h, attn_rows_kernel<T, 32, 4>, dim3(blocks), dim3(256), 0, s, a); break;
+    case 64: launch_k(h, attn_rows_kernel<T, 64, 4>, dim3(blocks), dim3(256), 0, s, a); break;
+    default: launch_k(h, attn_rows_kernel<T, 128, 4>, dim3(blocks), dim3(256), 0, s, a); break;
   }
   if (a.mode == 2) {
     const int mb = cdiv((long)a.n_q * a.H, 8);
     switch (d) {
-      case 16: ++g_launches; attn_merge_kernel<T, 16><<<mb, 256, 0, s>>>(a); break;
-      case 32: ++g_launches; attn_merge_kernel<T, 32><<<mb, 256, 0, s>>>(a); break;
-      case 64: ++g_launches; attn_merge_kernel<T, 64><<<mb, 256, 0, s>>>(a); break;
-      default: ++g_launches; attn_merge_kernel<T, 128><<<mb, 256, 0, s>>>(a); break;
+      case 16: launch_k(h, attn_merge_kernel<T, 16>, dim3(mb), dim3(256), 0, s, a); break;
+      case 32: launch_k(h, attn_merge_kernel<T, 32>, dim3(mb), dim3(256), 0, s, a); break;
+      case 64: launch_k(h, attn_merge_kernel<T, 64>, dim3(mb), dim3(256), 0, s, a); break;
+      default: launch_k(h, attn_merge_kernel<T, 128>, dim3(mb), dim3(256), 0, s, a); break;
     }
   }
 }
@@ -544,13 +585,13 @@ static void route_rows(dreamer_handle *h, int mode, int l, const void *X, int n,
   t.z = h->zbuf; t.ldz = ldz; t.zscale = 1.0f / sqrtf((float)dr);
   t.bias = mode == 0 ? h->bias : nullptr;
   t.idx = idx; t.w = wout; t.counts_a = counts_a; t.counts_b = counts_b;
-  ++g_launches;
-  launch_topk(t, h->num_sms, s);
+  launch_topk(h, t, s);
 }
 
 static void trace_depth(dreamer_handle *h, const dreamer_trace *tr, int l, int n, bool prefill,
                         cudaStream_t s) {
   if (!tr) return;
+  pdl_break(h, s);
   const dreamer_config &c = h->cfg;
   const size_t es = h->esz, hd = c.hidden, k = c.top_k;
   const size_t off = (size_t)l * n;
@@ -594,12 +635,9 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   // 1. RMSNorm of the residual stream on the first depth of the call (later depths get x^
   // from the previous depth's fused combine + norm)
   mark(h, s, DREAMER_STAGE_NORM);
-  if (first) {
-  ++g_launches;
-  rmsnorm_kernel<T><<<cdiv(n, 8), 256, 0, s>>>(first ? (const T *)io.x_in : nullptr,
-                                               first ? nullptr : h->acc, (const T *)h->g,
-                                               (T *)h->xh, h->inv_rms, n, hd, c.rms_eps);
-  }
+  if (first)
+    launch_k(h, rmsnorm_kernel<T>, dim3(cdiv(n, 8)), dim3(256), 0, s, (const T *)io.x_in,
+             (const float *)nullptr, (const T *)h->g, (T *)h->xh, h->inv_rms, n, hd, c.rms_eps);
   // 2. projection router and token grouping (linear-MoE QKV/O)
   const int *prow = nullptr;
   const float *psig = nullptr;
@@ -607,13 +645,13 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     mark(h, s, DREAMER_STAGE_PROJ_ROUTE);
     LAUNCHED(2);
     cudaMemsetAsync(h->pcnt, 0, (G + 1) * sizeof(int), s);
+    pdl_break(h, s);
     if (!(tc && tc_proj_route(h, l, h->xh, n, s)))
       route_rows<T>(h, 1, l, h->xh, n, h->pidx, h->psig, nullptr, h->pcnt, s);
-    ++g_launches;
-    scan_kernel<<<1, 1024, 0, s>>>(h->pcnt, G, h->poffs, h->ptiles_a, 64, h->ptiles_b, 128,
-                                   h->pcursor);
-    ++g_launches;
-    scatter_kernel<<<cdiv(n, 256), 256, 0, s>>>(h->pidx, n, h->pcursor, h->prows, h->pinv);
+    launch_k(h, scan_kernel, dim3(1), dim3(1024), 0, s, (const int *)h->pcnt, G, h->poffs,
+             h->ptiles_a, 64, h->ptiles_b, 128, h->pcursor);
+    launch_k(h, scatter_kernel, dim3(cdiv(n, 256)), dim3(256), 0, s, (const int *)h->pidx, n,
+             h->pcursor, h->prows, h->pinv);
     prow = h->prows;
     psig = h->psig;
   }
@@ -655,7 +693,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   // kernel for float32 prefill
   auto run_sa = [&](cudaStream_t st) {
     if (io.mode == 1) {
-      launch_rows<T>(sd, d, st);
+      launch_rows<T>(h, sd, d, st);
       return;
     }
     if (!(tc && tc_sa_ok(h) && tc_sa(h, st))) launch_attn<T>(sa, d, st);
@@ -696,7 +734,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     qkv_gemm(h->xh, 3 * hd, 3 * hd);
     mark(h, s, DREAMER_STAGE_DA);
     LAUNCHED(1);
-    launch_rows<T>(da, d, s);
+    launch_rows<T>(h, da, d, s);
     o_gemm((const T *)h->attn + hd, hd, hd, res_xhat, h->u);   // u = x^ + DA part (acc = u)
     qkv_gemm(h->u, 0, 3 * hd);
     mark(h, s, DREAMER_STAGE_SA);
@@ -712,16 +750,20 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     LAUNCHED(io.mode == 1 ? 3 : 2);
     if (h->prof) {
       mark(h, s, DREAMER_STAGE_DA);
-      launch_rows<T>(da, d, s);
+      launch_rows<T>(h, da, d, s);
     } else {
       cudaEventRecord(h->ev_fork, s);
       cudaStreamWaitEvent(h->side, h->ev_fork, 0);
-      launch_rows<T>(da, d, h->side);
+      pdl_break(h, h->side);
+      launch_rows<T>(h, da, d, h->side);
       cudaEventRecord(h->ev_join, h->side);
     }
     mark(h, s, DREAMER_STAGE_SA);
     run_sa(s);
-    if (!h->prof) cudaStreamWaitEvent(s, h->ev_join, 0);
+    if (!h->prof) {
+      cudaStreamWaitEvent(s, h->ev_join, 0);
+      pdl_break(h, s);
+    }
     // 5. O projection, residual y = x^ + DA + SA
     o_gemm(h->attn, 0, 2 * hd, res_xhat, h->y);
   }
@@ -730,14 +772,13 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   mark(h, s, DREAMER_STAGE_EA_ROUTE);
   LAUNCHED(5);
   cudaMemsetAsync(h->ecnt, 0, E * sizeof(int), s);
+  pdl_break(h, s);
   route_rows<T>(h, 0, l, ein, n, h->eidx, h->ew, h->counts + (size_t)l * E, h->ecnt, s);
   mark(h, s, DREAMER_STAGE_PERMUTE);
-  ++g_launches;
-  scan_kernel<<<1, 1024, 0, s>>>(h->ecnt, E, h->eoffs, h->etiles_a, 64, h->etiles_b, 128,
-                                 h->ecursor);
-  ++g_launches;
-  scatter_kernel<<<cdiv((long)n * k, 256), 256, 0, s>>>(h->eidx, n * k, h->ecursor, h->erows,
-                                                         h->einv);
+  launch_k(h, scan_kernel, dim3(1), dim3(1024), 0, s, (const int *)h->ecnt, E, h->eoffs,
+           h->etiles_a, 64, h->etiles_b, 128, h->ecursor);
+  launch_k(h, scatter_kernel, dim3(cdiv((long)n * k, 256)), dim3(256), 0, s,
+           (const int *)h->eidx, n * k, h->ecursor, h->erows, h->einv);
   // 7. expert FFNs: H = SiLU(X W1_e), acc[token] += w * H W2_e
   mark(h, s, DREAMER_STAGE_EXPERTS);
   LAUNCHED(2);
@@ -759,15 +800,10 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   // 8. x_{l+1} = y + sum_s w_s Y_s, then the next depth's RMSNorm (or the call's output)
   mark(h, s, DREAMER_STAGE_FINISH);
   const int cb = cdiv(n, 8);
-  ++g_launches;
-  if (hd <= 2048)
-    combine_norm_kernel<T, 64><<<cb, 256, 0, s>>>(h->acc, (const T *)h->Ybuf, h->einv, h->ew, k,
-                                                  (const T *)h->g, (T *)h->xh, h->inv_rms,
-                                                  last ? (T *)io.x_out : nullptr, n, hd, c.rms_eps);
-  else
-    combine_norm_kernel<T, 128><<<cb, 256, 0, s>>>(h->acc, (const T *)h->Ybuf, h->einv, h->ew, k,
-                                                   (const T *)h->g, (T *)h->xh, h->inv_rms,
-                                                   last ? (T *)io.x_out : nullptr, n, hd, c.rms_eps);
+  auto combine = hd <= 2048 ? combine_norm_kernel<T, 64> : combine_norm_kernel<T, 128>;
+  launch_k(h, combine, dim3(cb), dim3(256), 0, s, h->acc, (const T *)h->Ybuf,
+           (const int *)h->einv, (const float *)h->ew, k, (const T *)h->g, (T *)h->xh,
+           h->inv_rms, last ? (T *)io.x_out : (T *)nullptr, n, hd, c.rms_eps);
 }
 
 // The device error flag is copied to pinned host memory at the end of every call; the next
@@ -886,6 +922,8 @@ static int forward_impl(dreamer_handle *h, const void *x_in, void *x_out, int l0
   const dreamer_config &c = h->cfg;
   const int n = c.batch * c.seq;
   CK(cudaMemsetAsync(h->counts, 0, (size_t)c.depth * c.n_experts * sizeof(int), s));
+  pdl_break(h, s);
+  pdl_break(h, h->side);
   DepthIO io{};
   io.mode = 0; io.n_tok = n; io.x_in = x_in; io.x_out = x_out; io.tr = tr;
   io.da_kv = da_kv ? da_kv : h->da_kv_int;
@@ -932,6 +970,8 @@ static int decode_impl(dreamer_handle *h, const void *x_new, void *kc, void *vc,
   const dreamer_config &c = h->cfg;
   const int n = c.batch;
   CK(cudaMemsetAsync(h->counts, 0, (size_t)c.depth * c.n_experts * sizeof(int), s));
+  pdl_break(h, s);
+  pdl_break(h, h->side);
   DepthIO io{};
   io.mode = 1; io.n_tok = n; io.x_in = x_new; io.x_out = x_out; io.tr = tr;
   io.da_kv = h->da_kv_int;
@@ -993,6 +1033,7 @@ extern "C" int dreamer_route_experts(dreamer_handle *h, int depth, const void *y
   if (n_tokens == 0) return DREAMER_OK;
   cudaStream_t s = (cudaStream_t)stream;
   if (counts) CK(cudaMemsetAsync(counts, 0, h->cfg.n_experts * sizeof(int), s));
+  pdl_break(h, s);  // the caller's stream: whatever ran last is not ours
   if (h->cfg.dtype == 0)
     route_rows<float>(h, 0, depth, y, n_tokens, idx, w, counts, nullptr, s);
   else

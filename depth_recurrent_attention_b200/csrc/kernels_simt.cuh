@@ -431,6 +431,8 @@ __device__ __forceinline__ bool gemm_tile_coords(const GemmArgs &a, int tile, in
 
 template <typename TA, typename TB, int SEG, class Epi>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a, Epi epi) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int BM = 64, BN = 128, BK = 16;
   __shared__ float As[BK][BM + 4];
   __shared__ float Bs[BK][BN + 4];
@@ -508,6 +510,8 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a, Epi epi) {
 template <typename T>
 __global__ void rmsnorm_kernel(const T *x_in, const float *acc, const T *gain, T *xh,
                                float *inv_rms, int n_tok, int h, float eps) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= n_tok) return;
@@ -543,6 +547,8 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(float *acc, const T *
                                                           const float *wts, int k, const T *gain,
                                                           T *xh, float *inv_rms, T *x_out,
                                                           int n_tok, int h, float eps) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= n_tok) return;
@@ -590,16 +596,6 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(float *acc, const T *
   }
 }
 
-// Final residual: x_L = dtype(acc).
-template <typename T>
-__global__ void finish_kernel(const float *acc, T *x_out, long n) {
-  long i = ((long)blockIdx.x * blockDim.x + threadIdx.x) * 8;
-  if (i >= n) return;
-  float v[8];
-  load8(acc + i, v);
-  store8(x_out + i, v);
-}
-
 // =======================================================================================
 // Attention of one query row over a run of keys (R4: scale 1/sqrt(d), fp32 softmax).
 // One warp per (query, head).  Keys are processed 32 at a time: lane j scores key j of the
@@ -628,6 +624,8 @@ struct AttnArgs {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256) attn_warp_kernel(AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= a.n_q * a.H) return;
@@ -745,6 +743,8 @@ __device__ __forceinline__ bool better(float v1, int e1, float v2, int e2) {
 // counts each pick into the histograms.
 template <int WPT>
 __global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
+  pdl_wait();
+  pdl_trigger();
   constexpr unsigned FULL = 0xffffffffu;
   constexpr int NONE = 0x7fffffff;
   __shared__ float mv[WPT][32], mz[WPT][32];
@@ -812,12 +812,6 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
   }
 }
 
-// Eight warps a token when there are too few tokens to fill the GPU with one warp each.
-inline void launch_topk(const TopkArgs &t, int num_sms, cudaStream_t s) {
-  if ((long)t.n_tok * 4 < (long)num_sms * 32) topk_kernel<8><<<t.n_tok, 256, 0, s>>>(t);
-  else topk_kernel<1><<<(t.n_tok + 7) / 8, 256, 0, s>>>(t);
-}
-
 // =======================================================================================
 // Counting sort of routed slots by expert (the permutation feeding the grouped GEMMs).
 // scan: offs = exclusive prefix of cnt; tile_offs = exclusive prefix of ceil(cnt/BM) for
@@ -826,6 +820,8 @@ inline void launch_topk(const TopkArgs &t, int num_sms, cudaStream_t s) {
 __global__ void __launch_bounds__(1024) scan_kernel(const int *cnt, int G, int *offs,
                                                     int *tiles_a, int bm_a, int *tiles_b,
                                                     int bm_b, int *cursor) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int s0[1024], s1[1024], s2[1024];
   const int tid = threadIdx.x;
   const int per = (G + 1023) / 1024;
@@ -876,6 +872,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *cnt, int G, int *
 
 // rows[offs[e] + rank] = slot for every slot (token*k + j) routed to e.
 __global__ void scatter_kernel(const int *idx, int n, int *cursor, int *rows, int *inv) {
+  pdl_wait();
+  pdl_trigger();
   int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   int p = atomicAdd(cursor + idx[i], 1);
@@ -890,6 +888,8 @@ __global__ void scatter_kernel(const int *idx, int n, int *cursor, int *rows, in
 __global__ void __launch_bounds__(1024) bias_update_kernel(const int *counts, int L, int E,
                                                            float lambda, float *bias,
                                                            float *bias_out) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int sm[];  // [pow2 >= E] sorted copy, then [E] totals
   int n2 = 1;
   while (n2 < E) n2 <<= 1;

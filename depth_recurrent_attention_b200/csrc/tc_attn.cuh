@@ -134,6 +134,8 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();     // inputs of the previous kernel are visible from here on
+  pdl_trigger();  // after the TMEM allocation (see pdl_trigger)
   // TMEM columns: S_A 0..127, S_B 128..255, O_A 256.., O_B 256 + D..
   const uint32_t tS = tmem, tO = tmem + 256;
 
@@ -390,16 +392,14 @@ static bool tc_sa(dreamer_handle *h, cudaStream_t s) {
       cudaFuncSetAttribute(tc::tc_sa_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SaCfg<64>::SMEM);
       set = true;
     }
-    ++g_launches;
-    tc::tc_sa_kernel<64><<<grid, 384, tc::SaCfg<64>::SMEM, s>>>(tm, a);
+    launch_k(h, tc::tc_sa_kernel<64>, dim3(grid), dim3(384), tc::SaCfg<64>::SMEM, s, tm, a);
   } else {
     static bool set = false;
     if (!set) {
       cudaFuncSetAttribute(tc::tc_sa_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SaCfg<128>::SMEM);
       set = true;
     }
-    ++g_launches;
-    tc::tc_sa_kernel<128><<<grid, 384, tc::SaCfg<128>::SMEM, s>>>(tm, a);
+    launch_k(h, tc::tc_sa_kernel<128>, dim3(grid), dim3(384), tc::SaCfg<128>::SMEM, s, tm, a);
   }
   return true;
 }

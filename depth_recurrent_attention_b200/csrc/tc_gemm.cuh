@@ -105,8 +105,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NT = a.N / BN;
-  const int mtiles = a.goffs ? a.tiles[a.G] : (a.M + 127) / 128;
-  const int total = mtiles * NT;
+  int mtiles = 0, total = 0;  // read after pdl_wait: the tile table may come from the last kernel
   const int KB = a.K / BK;
   // the i-th tile of this CTA (identical sequence in every role); false past the last one
   auto tile_at = [&](int i, int &mt, int &nt) -> bool {
@@ -143,6 +142,10 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();     // inputs of the previous kernel are visible from here on
+  pdl_trigger();  // after the TMEM allocation (see pdl_trigger)
+  mtiles = a.goffs ? a.tiles[a.G] : (a.M + 127) / 128;
+  total = mtiles * NT;
 
   if (warp == 0) {
     // ------------------------------------------------------------- TMA producer

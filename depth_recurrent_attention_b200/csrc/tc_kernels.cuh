@@ -257,8 +257,7 @@ static void tc_launch(dreamer_handle *h, const dreamer::tc::TcGemmArgs &a, const
   }
   long grid = max_tiles < h->num_sms ? max_tiles : h->num_sms;
   if (grid < 1) grid = 1;
-  ++g_launches;
-  kern<<<(int)grid, Cfg::THREADS, Cfg::SMEM, s>>>(ta, tb, a, epi);
+  launch_k(h, kern, dim3((unsigned)grid), dim3(Cfg::THREADS), Cfg::SMEM, s, ta, tb, a, epi);
 }
 
 // Build engine arguments and tensor maps from the generic GEMM description.  B rows of group
@@ -408,8 +407,7 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
   k.n_tok = n; k.E = E; k.k = c.top_k; k.mode = 0;
   k.z = h->zbuf; k.ldz = h->ldz; k.zscale = 1.0f / sqrtf((float)dr);
   k.bias = h->bias; k.idx = idx; k.w = w; k.counts_a = counts_a; k.counts_b = counts_b;
-  ++g_launches;
-  launch_topk(k, h->num_sms, s);
+  launch_topk(h, k, s);
   return true;
 }
 
