@@ -1,4 +1,4 @@
-// Attention of one query row over a run of key/value rows, HBM-bound form (bf16 / fp32).
+// Attention of one query row over a run of key/value rows, HBM-bound forms (bf16 / fp32).
 // Used for depth attention (the token's own depth states 0..l; papernotes "Key design 1":
 // DA looks back over the token's earlier depth states) and for decode attention over the
 // per-depth SA cache (split over key ranges, then merged).
@@ -54,37 +54,12 @@ __global__ void __launch_bounds__(256) attn_rows_kernel(RowsArgs a) {
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int c = lane % CH, r = lane / CH;
-  const int splits = a.mode == 2 ? a.nsplit : 1;
-  if (gw >= a.n_q * a.H * splits) return;
-  const int sp = gw % splits;
-  const int qh = gw / splits;
-  const int qi = qh / a.H, head = qh % a.H;
-
-  const T *Kb, *Vb;
-  long ldk;
-  int j0, j1;
-  if (a.mode == 0) {
-    const T *base = reinterpret_cast<const T *>(a.kv);
-    Kb = base + ((long)qi * a.L * 2) * a.h + head * D;
-    Vb = Kb + a.h;
-    ldk = 2L * a.h;
-    j0 = 0;
-    j1 = a.l + 1;
-  } else {
-    const int len = a.cache_len[qi];
-    if (len < 0 || len >= a.cap) {  // slot outside the cache: report, attend to nothing
-      if (lane == 0) raise_dev_error(a.err, DEV_BAD_INDEX);
-      return;
-    }
-    const long off = ((((long)a.l * a.B + qi) * a.H + head) * a.cap) * D;
-    Kb = reinterpret_cast<const T *>(a.kv) + off;
-    Vb = reinterpret_cast<const T *>(a.vc) + off;
-    ldk = D;
-    const int nk = len + 1;
-    const int per = (nk + splits - 1) / splits;
-    j0 = sp * per;
-    j1 = min(nk, j0 + per);
-  }
+  if (gw >= a.n_q * a.H) return;
+  const int qi = gw / a.H, head = gw % a.H;
+  const T *Kb = reinterpret_cast<const T *>(a.kv) + ((long)qi * a.L * 2) * a.h + head * D;
+  const T *Vb = Kb + a.h;
+  const long ldk = 2L * a.h;
+  const int j0 = 0, j1 = a.l + 1;
   float q[VEC];
   ld16(reinterpret_cast<const T *>(a.q) + (long)qi * a.ldq + head * D + c * VEC, q);
   const float sl2 = 1.4426950408889634f * rsqrtf((float)D);
@@ -144,23 +119,11 @@ __global__ void __launch_bounds__(256) attn_rows_kernel(RowsArgs a) {
   for (int o2 = CH; o2 < 32; o2 <<= 1)
 #pragma unroll
     for (int i = 0; i < VEC; i++) o[i] += __shfl_xor_sync(0xffffffffu, o[i], o2);
-  if (a.mode == 0) {
-    if (r == 0) {
-      const float inv = 1.0f / lsum;
+  if (r == 0) {
+    const float inv = 1.0f / lsum;
 #pragma unroll
-      for (int i = 0; i < VEC; i++) o[i] *= inv;
-      st16(reinterpret_cast<T *>(a.out) + (long)qi * a.ldo + a.col0 + head * D + c * VEC, o);
-    }
-  } else {
-    float *pp = a.part + ((long)qh * splits + sp) * (D + 2);
-    if (r == 0) {
-#pragma unroll
-      for (int i = 0; i < VEC; i++) pp[c * VEC + i] = o[i];
-    }
-    if (lane == 0) {
-      pp[D] = m;
-      pp[D + 1] = lsum;
-    }
+    for (int i = 0; i < VEC; i++) o[i] *= inv;
+    st16(reinterpret_cast<T *>(a.out) + (long)qi * a.ldo + a.col0 + head * D + c * VEC, o);
   }
 }
 
@@ -321,9 +284,8 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
         }
       }
     }
-    if (abort_flag) break;
-    consumed = c + 1;
-    const T *bk = buf[c & 1];
+    if (!abort_flag) consumed = c + 1;
+    const T *bk = buf[c & 1];  // on a timeout the pass below reads stale data; nothing is stored
     const int nr = min(a.chunk, nrow - c * a.chunk);
     if (active) {
       for (int g = 0; g < nr; g += U * RPW) {
@@ -375,6 +337,7 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
       }
     }
     __syncthreads();  // every warp is done with buffer c & 1
+    if (abort_flag) break;  // read after the barrier: the same decision in every thread
     if (threadIdx.x == 0 && c + 2 < nchunks) {
       issue(c + 2);
       issued = c + 3;
@@ -396,6 +359,221 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
     for (int c = consumed; c < issued; c++) {
       const uint64_t t0 = tcda::gtimer();
       while (!tcda::try_wait(tcda::smem_u32(&bars[c & 1]), (c >> 1) & 1) &&
+             tcda::gtimer() - t0 < 2000000000ull) {
+      }
+    }
+  }
+}
+
+
+// =======================================================================================
+// Decode attention over the per-depth SA cache, streamed: one CTA per (sequence, head, key
+// range).  The range's keys and values are two contiguous runs of the [L][B][H][cap][D]
+// caches, so thread 0 streams them into shared memory with 1-D bulk copies, NST chunks in
+// flight; the four warps take interleaved groups of rows of each chunk (row-group layout as
+// above) with their own online softmax, and the CTA folds the four (m, l, o) into one partial
+// for attn_merge_kernel.  Every chunk wait is bounded; the decision to stop is taken after a
+// block barrier so all threads take it together.
+// =======================================================================================
+struct DecBulkArgs {
+  int B, H, L, l, cap, nsplit, chunk;  // chunk: keys per shared-memory stage
+  const void *q;                       // [B][ldq], head at column head * D
+  long ldq;
+  const void *kc, *vc;                 // [L][B][H][cap][D]
+  const int *cache_len;                // [B]
+  float *part;                         // [B][H][nsplit][D + 2] partial (o, m, l)
+  int *err;
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128) dec_bulk_kernel(DecBulkArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int NST = 4, NW = 4;
+  constexpr int VEC = VecOf<T>::N;
+  constexpr int CH = D / VEC;
+  constexpr int RPW = 32 / CH;
+  constexpr int U = 2;
+  extern __shared__ __align__(128) uint8_t dsm[];
+  __shared__ __align__(8) uint64_t bars[NST];
+  __shared__ int abort_flag;
+  __shared__ float wm[NW], wl[NW];
+  __shared__ __align__(16) float wo[NW][D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sp = blockIdx.x % a.nsplit, bh = blockIdx.x / a.nsplit;
+  const int b = bh / a.H, head = bh % a.H;
+  float *pp = a.part + ((long)bh * a.nsplit + sp) * (D + 2);
+  const int len = a.cache_len[b];
+  if (len < 0 || len >= a.cap) {  // slot outside the cache: report, attend to nothing
+    if (threadIdx.x == 0) {
+      raise_dev_error(a.err, DEV_BAD_INDEX);
+      pp[D] = -INFINITY;
+      pp[D + 1] = 0.f;
+    }
+    return;
+  }
+  const int nk = len + 1;
+  const int per = (nk + a.nsplit - 1) / a.nsplit;
+  const int j0 = sp * per, j1 = min(nk, j0 + per);
+  if (j0 >= j1) {  // empty range
+    if (threadIdx.x == 0) {
+      pp[D] = -INFINITY;
+      pp[D + 1] = 0.f;
+    }
+    return;
+  }
+  const long off = ((((long)a.l * a.B + b) * a.H + head) * a.cap + j0) * D;
+  const T *Ks = reinterpret_cast<const T *>(a.kc) + off;
+  const T *Vs = reinterpret_cast<const T *>(a.vc) + off;
+  const int nrow = j1 - j0;
+  const int nch = (nrow + a.chunk - 1) / a.chunk;
+  const uint32_t cbytes = (uint32_t)(a.chunk * D * sizeof(T));
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NST; i++)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tcda::smem_u32(&bars[i])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    abort_flag = 0;
+  }
+  __syncthreads();
+  auto issue = [&](int c) {
+    const int st = c % NST;
+    const int nr = min(a.chunk, nrow - c * a.chunk);
+    const uint32_t bytes = (uint32_t)(nr * D * sizeof(T));
+    const uint32_t bar = tcda::smem_u32(&bars[st]);
+    asm volatile("{\n\t.reg .b64 s;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 s, [%0], %1;\n\t}" ::"r"(bar),
+                 "r"(2 * bytes)
+                 : "memory");
+    uint8_t *dst = dsm + (size_t)st * 2 * cbytes;
+    tcda::bulk_load(tcda::smem_u32(dst), Ks + (long)c * a.chunk * D, bytes, bar);
+    tcda::bulk_load(tcda::smem_u32(dst + cbytes), Vs + (long)c * a.chunk * D, bytes, bar);
+  };
+  int issued = 0;
+  if (threadIdx.x == 0) {
+    for (; issued < NST && issued < nch; issued++) issue(issued);
+  }
+  const int cc = lane % CH, rr = lane / CH;
+  float q[VEC], o[VEC];
+  const float sl2 = 1.4426950408889634f * rsqrtf((float)D);
+  ld16(reinterpret_cast<const T *>(a.q) + (long)b * a.ldq + head * D + cc * VEC, q);
+#pragma unroll
+  for (int i = 0; i < VEC; i++) {
+    q[i] *= sl2;
+    o[i] = 0.f;
+  }
+  float m = -INFINITY, lsum = 0.f;
+  int consumed = 0;
+  for (int c = 0; c < nch; c++) {
+    const int st = c % NST;
+    const uint32_t bar = tcda::smem_u32(&bars[st]);
+    const uint32_t par = (uint32_t)((c / NST) & 1);
+    if (!tcda::try_wait(bar, par)) {
+      const uint64_t t0 = tcda::gtimer();
+      while (!tcda::try_wait(bar, par)) {
+        if (abort_flag) break;
+        if (tcda::gtimer() - t0 > 2000000000ull) {
+          abort_flag = 1;
+          raise_dev_error(a.err, DEV_TIMEOUT);
+          break;
+        }
+      }
+    }
+    if (!abort_flag) consumed = c + 1;
+    const T *sk = reinterpret_cast<const T *>(dsm + (size_t)st * 2 * cbytes);
+    const T *sv = reinterpret_cast<const T *>(dsm + (size_t)st * 2 * cbytes + cbytes);
+    const int nr = min(a.chunk, nrow - c * a.chunk);
+    for (int g = warp * RPW; g < nr; g += NW * RPW * U) {
+      float s[U], vv[U][VEC];
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const int j = g + u * NW * RPW + rr;
+        s[u] = -INFINITY;
+        if (j < nr) {
+          float kv[VEC];
+          ld16(sk + (long)j * D + cc * VEC, kv);
+          ld16(sv + (long)j * D + cc * VEC, vv[u]);
+          float p = 0.f;
+#pragma unroll
+          for (int i = 0; i < VEC; i++) p = fmaf(q[i], kv[i], p);
+          s[u] = p;
+        } else {
+#pragma unroll
+          for (int i = 0; i < VEC; i++) vv[u][i] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        float p = s[u] == -INFINITY ? 0.f : s[u];
+#pragma unroll
+        for (int o2 = 1; o2 < CH; o2 <<= 1) p += __shfl_xor_sync(0xffffffffu, p, o2);
+        if (s[u] != -INFINITY) s[u] = p;
+      }
+      float gm = s[0];
+#pragma unroll
+      for (int u = 1; u < U; u++) gm = fmaxf(gm, s[u]);
+      gm = warp_max(gm);
+      const float mn = fmaxf(m, gm);
+      const float alpha = exp2f(m - mn);
+      float ps = 0.f;
+#pragma unroll
+      for (int i = 0; i < VEC; i++) o[i] *= alpha;
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const float p = s[u] == -INFINITY ? 0.f : exp2f(s[u] - mn);
+        ps += p;
+#pragma unroll
+        for (int i = 0; i < VEC; i++) o[i] = fmaf(p, vv[u][i], o[i]);
+      }
+      ps = warp_sum(cc == 0 ? ps : 0.f);
+      lsum = lsum * alpha + ps;
+      m = mn;
+    }
+    __syncthreads();        // stage st is free again
+    if (abort_flag) break;  // read after the barrier: the same decision in every thread
+    if (threadIdx.x == 0 && issued < nch) {
+      issue(issued);
+      issued++;
+    }
+  }
+#pragma unroll
+  for (int o2 = CH; o2 < 32; o2 <<= 1)
+#pragma unroll
+    for (int i = 0; i < VEC; i++) o[i] += __shfl_xor_sync(0xffffffffu, o[i], o2);
+  if (rr == 0) {
+#pragma unroll
+    for (int i = 0; i < VEC; i++) wo[warp][cc * VEC + i] = o[i];
+  }
+  if (lane == 0) {
+    wm[warp] = m;
+    wl[warp] = lsum;
+  }
+  __syncthreads();
+  if (!abort_flag) {
+    float M = wm[0];
+#pragma unroll
+    for (int w = 1; w < NW; w++) M = fmaxf(M, wm[w]);
+    float f[NW];
+    float den = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; w++) {
+      f[w] = wm[w] == -INFINITY ? 0.f : exp2f(wm[w] - M);
+      den += f[w] * wl[w];
+    }
+    for (int dd = threadIdx.x; dd < D; dd += blockDim.x) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; w++) acc = fmaf(f[w], wo[w][dd], acc);
+      pp[dd] = acc;
+    }
+    if (threadIdx.x == 0) {
+      pp[D] = M;
+      pp[D + 1] = den;
+    }
+  }
+  // copies still in flight after an abort land before the CTA exits
+  if (threadIdx.x == 0 && abort_flag) {
+    for (int c = consumed; c < issued; c++) {
+      const uint64_t t0 = tcda::gtimer();
+      while (!tcda::try_wait(tcda::smem_u32(&bars[c % NST]), (uint32_t)((c / NST) & 1)) &&
              tcda::gtimer() - t0 < 2000000000ull) {
       }
     }

@@ -316,6 +316,12 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     h->ldzp = round8(P > 0 ? P : 1);
     const size_t es = h->esz;
     const long T = h->T;
+    {
+      int dev = 0, sms = 0;
+      if (cudaGetDevice(&dev) == cudaSuccess &&
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+        h->num_sms = sms;
+    }
     if (const char *ev = getenv("DREAMER_NO_TC")) h->use_tc = atoi(ev) ? 0 : 1;
     if (const char *ev = getenv("DREAMER_NO_GRAPH")) h->use_graph = atoi(ev) ? 0 : 1;
     if (const char *ev = getenv("DREAMER_NO_PDL")) h->use_pdl = atoi(ev) ? 0 : 1;
@@ -407,8 +413,13 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     DALLOC(h->pinv, T * sizeof(int));
     DALLOC(h->err, sizeof(int));
     if (c.max_cache_len > 0) {
-      h->nsplit = (c.max_cache_len + 255) / 256;
-      if (h->nsplit > 64) h->nsplit = 64;
+      // key ranges per (sequence, head): about ten waves of three CTAs per SM, at least 16
+      // keys a range, at most 64 ranges
+      const long pairs = (long)c.batch * c.n_heads;
+      long ns = (30L * h->num_sms + pairs - 1) / pairs;
+      const long by_len = (c.max_cache_len + 1 + 15) / 16;
+      if (ns > by_len) ns = by_len;
+      h->nsplit = (int)(ns < 1 ? 1 : ns > 64 ? 64 : ns);
       DALLOC(h->part, (size_t)c.batch * c.n_heads * h->nsplit * (d + 2) * sizeof(float));
     }
     CK(cudaMemset(h->err, 0, sizeof(int)));
@@ -529,6 +540,30 @@ static void launch_da_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStre
   }
 }
 
+// decode attention over the SA cache: streamed key ranges, then the merge of the partials
+template <typename T>
+static void launch_dec_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStream_t s) {
+  DecBulkArgs a{};
+  a.B = r.B; a.H = r.H; a.L = r.L; a.l = r.l; a.cap = r.cap; a.nsplit = r.nsplit;
+  int chunk = (int)(8192 / (d * (long)sizeof(T)));  // 8 KB of keys (and of values) a stage
+  a.chunk = chunk > 256 ? 256 : chunk;
+  a.q = r.q; a.ldq = r.ldq; a.kc = r.kv; a.vc = r.vc; a.cache_len = r.cache_len;
+  a.part = r.part; a.err = r.err;
+  const int smem = (int)(4 * 2 * (long)a.chunk * d * sizeof(T));
+  const dim3 grid((unsigned)(r.B * r.H * r.nsplit));
+  auto go = [&](void (*kern)(DecBulkArgs)) {
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    launch_k(h, kern, grid, dim3(128), smem, s, a);
+  };
+  switch (d) {
+    case 16: go(dec_bulk_kernel<T, 16>); break;
+    case 32: go(dec_bulk_kernel<T, 32>); break;
+    case 64: go(dec_bulk_kernel<T, 64>); break;
+    default: go(dec_bulk_kernel<T, 128>); break;
+  }
+}
+
 // depth attention (mode 0) or split decode attention + merge (mode 2)
 template <typename T>
 static void launch_rows(dreamer_handle *h, const RowsArgs &a, int d, cudaStream_t s) {
@@ -536,13 +571,17 @@ static void launch_rows(dreamer_handle *h, const RowsArgs &a, int d, cudaStream_
     launch_da_bulk<T>(h, a, d, s);
     return;
   }
-  const long warps = (long)a.n_q * a.H * (a.mode == 2 ? a.nsplit : 1);
-  const int blocks = cdiv(warps, 8);
-  switch (d) {
-    case 16: launch_k(h, attn_rows_kernel<T, 16, 4>, dim3(blocks), dim3(256), 0, s, a); break;
-    case 32: launch_k(h, attn_rows_kernel<T, 32, 4>, dim3(blocks), dim3(256), 0, s, a); break;
-    case 64: launch_k(h, attn_rows_kernel<T, 64, 4>, dim3(blocks), dim3(256), 0, s, a); break;
-    default: launch_k(h, attn_rows_kernel<T, 128, 4>, dim3(blocks), dim3(256), 0, s, a); break;
+  if (a.mode == 2) {
+    launch_dec_bulk<T>(h, a, d, s);
+  } else {
+    const long warps = (long)a.n_q * a.H;
+    const int blocks = cdiv(warps, 8);
+    switch (d) {
+      case 16: launch_k(h, attn_rows_kernel<T, 16, 4>, dim3(blocks), dim3(256), 0, s, a); break;
+      case 32: launch_k(h, attn_rows_kernel<T, 32, 4>, dim3(blocks), dim3(256), 0, s, a); break;
+      case 64: launch_k(h, attn_rows_kernel<T, 64, 4>, dim3(blocks), dim3(256), 0, s, a); break;
+      default: launch_k(h, attn_rows_kernel<T, 128, 4>, dim3(blocks), dim3(256), 0, s, a); break;
+    }
   }
   if (a.mode == 2) {
     const int mb = cdiv((long)a.n_q * a.H, 8);
