@@ -157,21 +157,38 @@ static bool pdl_take(dreamer_handle *h, cudaStream_t s) {
 }
 static void pdl_break(dreamer_handle *h, cudaStream_t s) { h->pdl_ok[s == h->side ? 1 : 0] = false; }
 
+// launch_kc: with thread-block clusters of `cluster` CTAs along x
 template <typename... P, typename... A>
-static void launch_k(dreamer_handle *h, void (*kern)(P...), dim3 grid, dim3 block, size_t smem,
-                     cudaStream_t s, A &&...args) {
+static void launch_kc(dreamer_handle *h, int cluster, void (*kern)(P...), dim3 grid, dim3 block,
+                      size_t smem, cudaStream_t s, A &&...args) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute at[2];
+  int na = 0;
+  if (pdl_take(h, s)) {
+    at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[na].val.programmaticStreamSerializationAllowed = 1;
+    na++;
+  }
+  if (cluster > 1) {
+    at[na].id = cudaLaunchAttributeClusterDimension;
+    at[na].val.clusterDim.x = cluster;
+    at[na].val.clusterDim.y = 1;
+    at[na].val.clusterDim.z = 1;
+    na++;
+  }
   cfg.attrs = at;
-  cfg.numAttrs = pdl_take(h, s) ? 1 : 0;
+  cfg.numAttrs = na;
   ++g_launches;
   cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+template <typename... P, typename... A>
+static void launch_k(dreamer_handle *h, void (*kern)(P...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t s, A &&...args) {
+  launch_kc(h, 1, kern, grid, block, smem, s, std::forward<A>(args)...);
 }
 
 // top-k: eight warps a token when there are too few tokens to fill the GPU with one warp each
@@ -611,6 +628,20 @@ static void route_rows(dreamer_handle *h, int mode, int l, const void *X, int n,
   const int ldz = mode == 0 ? h->ldz : h->ldzp;
   const void *Wq = mode == 0 ? h->wqE_t : h->wqP_t;
   const float *krot = (mode == 0 ? h->kE_rot : h->kP_rot) + (size_t)l * E * dr;
+  if (mode == 0 && (long)n * 4 < (long)h->num_sms * 32 && (dr == 32 || dr == 64 || dr == 128) &&
+      hd % 8 == 0) {
+    // few tokens: query, scores and top-k in one kernel, a cluster of CTAs a token
+    TopkArgs t{};
+    t.n_tok = n; t.E = E; t.k = c.top_k; t.mode = 0;
+    t.zscale = 1.0f / sqrtf((float)dr); t.bias = h->bias;
+    t.idx = idx; t.w = wout; t.counts_a = counts_a; t.counts_b = counts_b;
+    const int ncl = E >= 1024 ? 8 : (E >= 256 ? 4 : 1);
+    auto kern = dr == 32 ? route_cluster_kernel<T, 32>
+                         : (dr == 64 ? route_cluster_kernel<T, 64> : route_cluster_kernel<T, 128>);
+    launch_kc(h, ncl, kern, dim3(n * ncl), dim3(256), 0, s, (const T *)X, hd, (const T *)Wq,
+              (const T *)h->kE_raw, (const float2 *)(h->rope_dr + (size_t)l * (dr / 2)), t);
+    return;
+  }
   if (mode == 0 && h->use_tc && c.dtype == 1 && tc_route_ok(h) &&
       tc_route(h, l, X, n, idx, wout, counts_a, counts_b, s))
     return;
@@ -808,20 +839,30 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   }
   // 6. expert attention routing on y (fully parallel layout: on x^)
   const void *ein = c.variant == 2 ? h->xh : h->y;
+  // few rows per expert (decode): every routed row computes its own expert FFN, unsorted
+  const bool by_rows = (long)n * k < 8L * E && (m == 16 || m == 32 || m == 64) &&
+                       hd <= 2048 && hd % 8 == 0;
   mark(h, s, DREAMER_STAGE_EA_ROUTE);
-  LAUNCHED(5);
-  cudaMemsetAsync(h->ecnt, 0, E * sizeof(int), s);
-  pdl_break(h, s);
-  route_rows<T>(h, 0, l, ein, n, h->eidx, h->ew, h->counts + (size_t)l * E, h->ecnt, s);
-  mark(h, s, DREAMER_STAGE_PERMUTE);
-  launch_k(h, scan_kernel, dim3(1), dim3(1024), 0, s, (const int *)h->ecnt, E, h->eoffs,
-           h->etiles_a, 64, h->etiles_b, 128, h->ecursor);
-  launch_k(h, scatter_kernel, dim3(cdiv((long)n * k, 256)), dim3(256), 0, s,
-           (const int *)h->eidx, n * k, h->ecursor, h->erows, h->einv);
+  if (by_rows) {
+    route_rows<T>(h, 0, l, ein, n, h->eidx, h->ew, h->counts + (size_t)l * E, nullptr, s);
+  } else {
+    cudaMemsetAsync(h->ecnt, 0, E * sizeof(int), s);
+    pdl_break(h, s);
+    route_rows<T>(h, 0, l, ein, n, h->eidx, h->ew, h->counts + (size_t)l * E, h->ecnt, s);
+    mark(h, s, DREAMER_STAGE_PERMUTE);
+    launch_k(h, scan_kernel, dim3(1), dim3(1024), 0, s, (const int *)h->ecnt, E, h->eoffs,
+             h->etiles_a, 64, h->etiles_b, 128, h->ecursor);
+    launch_k(h, scatter_kernel, dim3(cdiv((long)n * k, 256)), dim3(256), 0, s,
+             (const int *)h->eidx, n * k, h->ecursor, h->erows, h->einv);
+  }
   // 7. expert FFNs: H = SiLU(X W1_e), acc[token] += w * H W2_e
   mark(h, s, DREAMER_STAGE_EXPERTS);
-  LAUNCHED(2);
-  if (!(tc && tc_expert_ok(h) && tc_expert(h, ein, n, s))) {
+  if (by_rows) {
+    auto kern = m == 16 ? expert_rows_kernel<T, 16>
+                        : (m == 32 ? expert_rows_kernel<T, 32> : expert_rows_kernel<T, 64>);
+    launch_k(h, kern, dim3(n * k), dim3(256), 0, s, (const T *)ein, (const int *)h->eidx,
+             n * k, k, hd, (const T *)h->w1_t, (const T *)h->w2_t, (T *)h->Ybuf);
+  } else if (!(tc && tc_expert_ok(h) && tc_expert(h, ein, n, s))) {
     const int etiles = cdiv((long)n * k, 64) + E;
     GemmArgs up{};
     up.N = m; up.K = hd; up.G = E; up.M = n * k; up.goffs = h->eoffs; up.tile_offs = h->etiles_a;
@@ -841,7 +882,8 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   const int cb = cdiv(n, 8);
   auto combine = hd <= 2048 ? combine_norm_kernel<T, 64> : combine_norm_kernel<T, 128>;
   launch_k(h, combine, dim3(cb), dim3(256), 0, s, h->acc, (const T *)h->Ybuf,
-           (const int *)h->einv, (const float *)h->ew, k, (const T *)h->g, (T *)h->xh,
+           by_rows ? (const int *)nullptr : (const int *)h->einv, (const float *)h->ew, k,
+           (const T *)h->g, (T *)h->xh,
            h->inv_rms, last ? (T *)io.x_out : (T *)nullptr, n, hd, c.rms_eps);
 }
 

@@ -2,6 +2,8 @@
 // the parts of the bfloat16 mode that are not dense contractions (norm, depth attention,
 // routing top-k, permutation, decode attention).
 #pragma once
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
 namespace dreamer {
@@ -537,6 +539,62 @@ __global__ void rmsnorm_kernel(const T *x_in, const float *acc, const T *gain, T
   }
 }
 
+// Expert FFN of single routed rows, for batches with few rows per expert (decode): one CTA
+// per routed slot (token t, slot s) computes Y[t k + s] = SiLU(x_t W1_e) W2_e for its expert
+// e (papernotes "Key design 2": each expert is a small SiLU FFN), reading the expert's two
+// weight blocks once; no sorting by expert is needed.  The hidden activations are rounded to
+// dtype as the grouped path stores them.  w1t: [E][M][h], w2t: [E][h][M] (K contiguous).
+template <typename T, int M>
+__global__ void __launch_bounds__(256) expert_rows_kernel(const T *X, const int *eidx,
+                                                          int nslots, int k, int h,
+                                                          const T *w1t, const T *w2t, T *Y) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int XC = 8;  // 16-byte x chunks a lane keeps (h <= 2048)
+  __shared__ float hs[M];
+  const int slot = blockIdx.x;
+  if (slot >= nslots) return;
+  const int e = eidx[slot], tok = slot / k;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const T *x = X + (long)tok * h;
+  const T *W1 = w1t + (long)e * M * h;
+  const T *W2 = w2t + (long)e * h * M;
+  float xr[XC][8];
+#pragma unroll
+  for (int t = 0; t < XC; t++) {
+    const int i = t * 256 + lane * 8;
+    if (i < h) load8(x + i, xr[t]);
+  }
+  for (int j = warp; j < M; j += 8) {  // up: one hidden unit a warp at a time
+    float a = 0.f;
+#pragma unroll
+    for (int t = 0; t < XC; t++) {
+      const int i = t * 256 + lane * 8;
+      if (i < h) {
+        float wv[8];
+        load8(W1 + (long)j * h + i, wv);
+#pragma unroll
+        for (int q = 0; q < 8; q++) a = fmaf(xr[t][q], wv[q], a);
+      }
+    }
+    a = warp_sum(a);
+    if (lane == 0) hs[j] = to_f(from_f<T>(a / (1.0f + __expf(-a))));
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < h; c += blockDim.x) {  // down: one output column a thread
+    const T *w = W2 + (long)c * M;
+    float a = 0.f;
+#pragma unroll
+    for (int j = 0; j < M; j += 8) {
+      float wv[8];
+      load8(w + j, wv);
+#pragma unroll
+      for (int q = 0; q < 8; q++) a = fmaf(hs[j + q], wv[q], a);
+    }
+    Y[(long)slot * h + c] = from_f<T>(a);
+  }
+}
+
 // Combine, residual and RMSNorm fused (one warp per token): x_{l+1} = y + sum_s w_s Y_s over
 // the token's k routed rows (papernotes "Key design 2": the expert outputs mixed by the
 // normalised routing weights; fixed order s = 0..k-1), kept in fp32 in acc; then either the
@@ -554,12 +612,7 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(float *acc, const T *
   if (warp >= n_tok) return;
   float xv[MAXV];  // this lane's 8-element chunks of the row, in fp32
   float ss = 0.f;
-  long prow[16];
-  float pw[16];
-  for (int s = 0; s < k; s++) {
-    prow[s] = (long)pos[(long)warp * k + s] * h;
-    pw[s] = wts[(long)warp * k + s];
-  }
+  const long slot0 = (long)warp * k;
 #pragma unroll
   for (int ci = 0; ci < MAXV / 8; ci++) {
     const int c = ci * 256 + lane * 8;
@@ -567,10 +620,13 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(float *acc, const T *
     float x[8];
     load8(acc + (long)warp * h + c, x);
     for (int s = 0; s < k; s++) {
+      // row of slot s in Y: its sorted position, or the slot itself (pos == null)
+      const long pr = (pos ? (long)pos[slot0 + s] : slot0 + s) * h;
+      const float pw = wts[slot0 + s];
       float yv[8];
-      load8(Y + prow[s] + c, yv);
+      load8(Y + pr + c, yv);
 #pragma unroll
-      for (int j = 0; j < 8; j++) x[j] = fmaf(pw[s], yv[j], x[j]);
+      for (int j = 0; j < 8; j++) x[j] = fmaf(pw, yv[j], x[j]);
     }
 #pragma unroll
     for (int j = 0; j < 8; j++) {
@@ -733,32 +789,24 @@ __device__ __forceinline__ bool better(float v1, int e1, float v2, int e2) {
   return v1 > v2 || (v1 == v2 && e1 < e2);
 }
 
-// Top-k by warps.  A warp keeps its running top k (k <= 32) distributed over its lanes, lane j
-// holding the j-th best (biased score, expert, raw score) pair; it reads 32 candidates at a
-// time and inserts the ones that beat entry k-1, each by a ballot for the insertion position
-// and a one-lane shift (no per-lane arrays, nothing in local memory).  WPT warps share a
-// token: each scans a slice of the experts, then warp 0 merges the others' lists.  Ties go
-// to the lower expert index; a NaN score ranks last.  Writes the experts in descending order
-// of biased score, w = sigmoid(raw) normalised over the k (mode 0) or as it is (mode 1), and
-// counts each pick into the histograms.
-template <int WPT>
-__global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
-  pdl_wait();
-  pdl_trigger();
-  constexpr unsigned FULL = 0xffffffffu;
-  constexpr int NONE = 0x7fffffff;
-  __shared__ float mv[WPT][32], mz[WPT][32];
-  __shared__ int me[WPT][32];
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int tok = WPT == 1 ? blockIdx.x * 8 + wib : blockIdx.x;
-  if (tok >= a.n_tok) return;  // whole warp (WPT 1) or whole block (WPT > 1)
-  const int k = a.k;
-  const float *zr = a.z + (long)tok * a.ldz;
-  float lv = -INFINITY, lz = 0.f;
-  int le = NONE;
-  float tv = -INFINITY;
-  int te = NONE;
-  auto insert = [&](float cv, int ce, float cz) {
+// Running top k (k <= 32) of one warp, distributed over its lanes: lane j holds the j-th best
+// (biased score v, expert e, raw score z).  The first 32 candidates are sorted by a warp
+// bitonic network; later ones that beat entry k-1 are inserted by a ballot for the position and
+// a one-lane shift.  No per-lane arrays, nothing in local memory.  Order: higher v first, the
+// lower expert index on ties; a NaN score ranks last.
+struct WarpTopK {
+  static constexpr unsigned FULL = 0xffffffffu;
+  static constexpr int NONE = 0x7fffffff;
+  int k, lane;
+  bool started = false;
+  float lv = -INFINITY, lz = 0.f, tv = -INFINITY;
+  int le = NONE, te = NONE;
+  __device__ WarpTopK(int k_, int lane_) : k(k_), lane(lane_) {}
+  __device__ __forceinline__ void threshold() {
+    tv = __shfl_sync(FULL, lv, k - 1);
+    te = __shfl_sync(FULL, le, k - 1);
+  }
+  __device__ __forceinline__ void insert(float cv, int ce, float cz) {
     const int pos = __popc(__ballot_sync(FULL, lane < k && better(lv, le, cv, ce)));
     const float uv = __shfl_up_sync(FULL, lv, 1), uz = __shfl_up_sync(FULL, lz, 1);
     const int ue = __shfl_up_sync(FULL, le, 1);
@@ -767,10 +815,36 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
     } else if (lane == pos) {
       lv = cv; lz = cz; le = ce;
     }
-    tv = __shfl_sync(FULL, lv, k - 1);
-    te = __shfl_sync(FULL, le, k - 1);
-  };
-  auto offer = [&](float v, int e, float z) {  // one candidate a lane (e == NONE: none)
+    threshold();
+  }
+  // the first batch: sort the warp's 32 candidates (descending) and keep the best k
+  __device__ __forceinline__ void start(float v, int e, float z) {
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const float ov = __shfl_xor_sync(FULL, v, stride), oz = __shfl_xor_sync(FULL, z, stride);
+        const int oe = __shfl_xor_sync(FULL, e, stride);
+        const bool desc = (lane & size) == 0 || size == 32;
+        const bool lower = (lane & stride) == 0;
+        const bool mine = better(v, e, ov, oe);
+        if ((lower == desc) != mine) {
+          v = ov; e = oe; z = oz;
+        }
+      }
+    }
+    lv = lane < k ? v : -INFINITY;
+    le = lane < k ? e : NONE;
+    lz = z;
+    started = true;
+    threshold();
+  }
+  // one candidate a lane (e == NONE: none); warp-uniform call
+  __device__ __forceinline__ void offer(float v, int e, float z) {
+    if (!started) {
+      start(v, e, z);
+      return;
+    }
     unsigned m = __ballot_sync(FULL, e != NONE && better(v, e, tv, te));
     while (m) {
       const int src = __ffs(m) - 1;
@@ -779,36 +853,183 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
       const int ce = __shfl_sync(FULL, e, src);
       if (better(cv, ce, tv, te)) insert(cv, ce, cz);
     }
-  };
+  }
+  // the candidate of expert e with raw score z (already scaled)
+  __device__ __forceinline__ void offer_score(float z, int e, bool valid, const float *bias) {
+    float v = -INFINITY;
+    if (valid) {
+      v = z + (bias ? bias[e] : 0.f);
+      if (v != v) v = -INFINITY;
+    }
+    offer(v, valid ? e : NONE, z);
+  }
+};
+
+// Lanes < k of a warp write the k picks (descending), their weights (sigmoid of the raw score,
+// normalised over the k in mode 0) and count them.
+__device__ __forceinline__ void emit_topk(int lane, int k, float v, int e, float z, long tok,
+                                          int mode, int *idx, float *w, int *ca, int *cb) {
+  const float sg = lane < k ? 1.0f / (1.0f + __expf(-z)) : 0.f;
+  const float ssum = warp_sum(sg);
+  if (lane < k) {
+    idx[tok * k + lane] = e;
+    w[tok * k + lane] = mode == 0 ? sg / ssum : sg;
+    if (ca) atomicAdd(ca + e, 1);
+    if (cb) atomicAdd(cb + e, 1);
+  }
+}
+
+// Top k of n listed candidates (n <= 256, distinct experts, NONE = empty) by rank counting:
+// the threads of the block each rank one entry against all n (no serial chain) and write the
+// k best to out[rank].  Ends with a block barrier.
+__device__ __forceinline__ void rank_select(const float *sv, const int *se, const float *sz,
+                                            int n, int k, float *ov, int *oe, float *oz) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const float v = sv[i];
+    const int e = se[i];
+    if (e == WarpTopK::NONE) continue;
+    int r = 0;
+    for (int j = 0; j < n; j++) r += (se[j] != WarpTopK::NONE && better(sv[j], se[j], v, e)) ? 1 : 0;
+    if (r < k) {
+      ov[r] = v;
+      oe[r] = e;
+      oz[r] = sz[i];
+    }
+  }
+  __syncthreads();
+}
+
+// Top-k of stored scores z (one token's row of E), WPT warps a token; each warp scans a slice
+// of the experts 32 at a time, then the block ranks the WPT lists.
+template <int WPT>
+__global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float mv[WPT * 32], mz[WPT * 32], fv[32], fz[32];
+  __shared__ int me[WPT * 32], fe[32];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int tok = WPT == 1 ? blockIdx.x * 8 + wib : blockIdx.x;
+  if (tok >= a.n_tok) return;  // whole warp (WPT 1) or whole block (WPT > 1)
+  const float *zr = a.z + (long)tok * a.ldz;
+  WarpTopK t(a.k, lane);
   const int per = (a.E + WPT - 1) / WPT;
   const int e0 = WPT > 1 ? wib * per : 0, e1 = WPT > 1 ? min(a.E, e0 + per) : a.E;
   for (int b = e0; b < e1; b += 32) {
     const int e = b + lane;
-    float z = 0.f, v = -INFINITY;
-    int ce = NONE;
-    if (e < e1) {
-      z = zr[e] * a.zscale;
-      v = z + (a.bias ? a.bias[e] : 0.f);
-      if (v != v) v = -INFINITY;
-      ce = e;
+    t.offer_score(e < e1 ? zr[e] * a.zscale : 0.f, e, e < e1, a.bias);
+  }
+  if (WPT == 1) {
+    emit_topk(lane, a.k, t.lv, t.le, t.lz, tok, a.mode, a.idx, a.w, a.counts_a, a.counts_b);
+    return;
+  }
+  mv[wib * 32 + lane] = lane < a.k ? t.lv : -INFINITY;
+  me[wib * 32 + lane] = lane < a.k ? t.le : WarpTopK::NONE;
+  mz[wib * 32 + lane] = t.lz;
+  __syncthreads();
+  rank_select(mv, me, mz, WPT * 32, a.k, fv, fe, fz);
+  if (wib == 0)
+    emit_topk(lane, a.k, fv[lane], fe[lane], fz[lane], tok, a.mode, a.idx, a.w, a.counts_a,
+              a.counts_b);
+}
+
+// Routing of few tokens (decode): a cluster of NCL CTAs per token (papernotes "Key design 2":
+// router query, sigmoid scores against depth-RoPE'd expert keys, biased top-k).  Each CTA
+// computes DR/NCL entries of the query q = y W_q (fp32), the cluster gathers q through
+// distributed shared memory and turns it back by the depth rotation (q . R_l k = R_l^T q . k),
+// each CTA scores its slice of the experts against the unrotated keys and ranks its warps'
+// lists, and CTA 0 ranks the NCL lists read from its peers' shared memory.  wqt: W_q
+// transposed [d_r][h]; kraw: [E][d_r]; rope: the router dim's depth-RoPE row of this depth.
+template <typename T, int DR>
+__global__ void __launch_bounds__(256) route_cluster_kernel(const T *y, int h, const T *wqt,
+                                                            const T *kraw, const float2 *rope,
+                                                            TopkArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const int ncl = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int tok = blockIdx.x / ncl;  // the same for the whole cluster
+  __shared__ __align__(16) float qpart[DR], qv[DR];
+  __shared__ float mv[256], mz[256], fv[32], fz[32];
+  __shared__ int me[256], fe[32];
+  const bool live = tok < a.n_tok;
+  const int qn = DR / ncl;
+  if (live) {
+    const T *yr = y + (long)tok * h;
+    for (int j = rank * qn + wib; j < (rank + 1) * qn; j += 8) {
+      float acc = 0.f;
+      for (int i = lane * 8; i < h; i += 256) {
+        float yv[8], wv[8];
+        load8(yr + i, yv);
+        load8(wqt + (long)j * h + i, wv);
+#pragma unroll
+        for (int u = 0; u < 8; u++) acc = fmaf(yv[u], wv[u], acc);
+      }
+      acc = warp_sum(acc);
+      if (lane == 0) qpart[j] = acc;
     }
-    offer(v, ce, z);
   }
-  if (WPT > 1) {
-    mv[wib][lane] = lane < k ? lv : -INFINITY;
-    me[wib][lane] = lane < k ? le : NONE;
-    mz[wib][lane] = lz;
+  cl.sync();
+  if (threadIdx.x < DR) qv[threadIdx.x] = *cl.map_shared_rank(qpart + threadIdx.x, threadIdx.x / qn);
+  __syncthreads();
+  if (threadIdx.x < DR / 2) {  // R_l^T: pairs (i, i + d_r/4) inside each half
+    const int q4 = DR / 4, half = threadIdx.x / q4, i = threadIdx.x % q4;
+    const int ia = half * (DR / 2) + i, ib = ia + q4;
+    const float c = rope[half * q4 + i].x, sn = rope[half * q4 + i].y;
+    const float va = qv[ia], vb = qv[ib];
+    qv[ia] = va * c + vb * sn;
+    qv[ib] = vb * c - va * sn;
+  }
+  __syncthreads();
+  WarpTopK t(a.k, lane);
+  if (live) {
+    float q[DR];
+#pragma unroll
+    for (int j = 0; j < DR; j++) q[j] = qv[j];
+    const int per_cta = (a.E + ncl - 1) / ncl;
+    const int c0 = rank * per_cta, c1 = min(a.E, c0 + per_cta);
+    const int per_w = (c1 - c0 + 7) / 8;
+    const int e0 = c0 + wib * per_w, e1 = min(c1, e0 + per_w);
+    for (int b = e0; b < e1; b += 32) {
+      const int e = b + lane;
+      float z = 0.f;
+      if (e < e1) {
+        const T *kr = kraw + (long)e * DR;
+#pragma unroll
+        for (int j = 0; j < DR; j += 8) {
+          float kv[8];
+          load8(kr + j, kv);
+#pragma unroll
+          for (int u = 0; u < 8; u++) z = fmaf(q[j + u], kv[u], z);
+        }
+      }
+      t.offer_score(z * a.zscale, e, e < e1, a.bias);
+    }
+  }
+  mv[wib * 32 + lane] = lane < a.k ? t.lv : -INFINITY;
+  me[wib * 32 + lane] = lane < a.k ? t.le : WarpTopK::NONE;
+  mz[wib * 32 + lane] = t.lz;
+  if (threadIdx.x < 32) fe[threadIdx.x] = WarpTopK::NONE;
+  __syncthreads();
+  rank_select(mv, me, mz, 256, a.k, fv, fe, fz);  // this CTA's best k in fv/fe/fz
+  cl.sync();
+  if (rank == 0) {  // gather the cluster's lists and rank them again
+    for (int i = threadIdx.x; i < ncl * 32; i += blockDim.x) {
+      const int r = i / 32, j = i % 32;
+      const bool in = j < a.k;
+      mv[i] = in ? *cl.map_shared_rank(fv + j, r) : -INFINITY;
+      me[i] = in ? *cl.map_shared_rank(fe + j, r) : WarpTopK::NONE;
+      mz[i] = in ? *cl.map_shared_rank(fz + j, r) : 0.f;
+    }
+  }
+  cl.sync();  // peers' lists read; they may exit
+  if (rank == 0) {
     __syncthreads();
-    if (wib != 0) return;
-    for (int w = 1; w < WPT; w++) offer(mv[w][lane], me[w][lane], mz[w][lane]);
-  }
-  const float sg = lane < k ? 1.0f / (1.0f + __expf(-lz)) : 0.f;
-  const float ssum = warp_sum(sg);
-  if (lane < k) {
-    a.idx[(long)tok * k + lane] = le;
-    a.w[(long)tok * k + lane] = (a.mode == 0) ? sg / ssum : sg;
-    if (a.counts_a) atomicAdd(a.counts_a + le, 1);
-    if (a.counts_b) atomicAdd(a.counts_b + le, 1);
+    rank_select(mv, me, mz, ncl * 32, a.k, fv, fe, fz);
+    if (live && wib == 0)
+      emit_topk(lane, a.k, fv[lane], fe[lane], fz[lane], tok, a.mode, a.idx, a.w, a.counts_a,
+                a.counts_b);
   }
 }
 
