@@ -370,8 +370,8 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
 // Decode attention over the per-depth SA cache, streamed: one CTA per (sequence, head, key
 // range).  The range's keys and values are two contiguous runs of the [L][B][H][cap][D]
 // caches, so thread 0 streams them into shared memory with 1-D bulk copies, NST chunks in
-// flight; the four warps take interleaved groups of rows of each chunk (row-group layout as
-// above) with their own online softmax, and the CTA folds the four (m, l, o) into one partial
+// flight; the eight warps take interleaved groups of rows of each chunk (row-group layout as
+// above) with their own online softmax, and the CTA folds the eight (m, l, o) into one partial
 // for attn_merge_kernel.  Every chunk wait is bounded; the decision to stop is taken after a
 // block barrier so all threads take it together.
 // =======================================================================================
@@ -386,10 +386,10 @@ struct DecBulkArgs {
 };
 
 template <typename T, int D>
-__global__ void __launch_bounds__(128) dec_bulk_kernel(DecBulkArgs a) {
+__global__ void __launch_bounds__(256) dec_bulk_kernel(DecBulkArgs a) {
   pdl_wait();
   pdl_trigger();
-  constexpr int NST = 4, NW = 4;
+  constexpr int NST = 4, NW = 8;
   constexpr int VEC = VecOf<T>::N;
   constexpr int CH = D / VEC;
   constexpr int RPW = 32 / CH;

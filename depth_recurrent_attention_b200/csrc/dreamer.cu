@@ -571,7 +571,7 @@ static void launch_dec_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStr
   auto go = [&](void (*kern)(DecBulkArgs)) {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    launch_k(h, kern, grid, dim3(128), smem, s, a);
+    launch_k(h, kern, grid, dim3(256), smem, s, a);
   };
   switch (d) {
     case 16: go(dec_bulk_kernel<T, 16>); break;

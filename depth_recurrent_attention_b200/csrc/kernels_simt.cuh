@@ -879,21 +879,32 @@ __device__ __forceinline__ void emit_topk(int lane, int k, float v, int e, float
   }
 }
 
-// Top k of n listed candidates (n <= 256, distinct experts, NONE = empty) by rank counting:
-// the threads of the block each rank one entry against all n (no serial chain) and write the
-// k best to out[rank].  Ends with a block barrier.
-__device__ __forceinline__ void rank_select(const float *sv, const int *se, const float *sz,
-                                            int n, int k, float *ov, int *oe, float *oz) {
+// Candidates as one ordered 64-bit key: larger key = better (higher biased score, then the
+// lower expert index); 0 = no candidate.  -0 counts as +0, as in better().
+__device__ __forceinline__ unsigned long long topk_key(float v, int e) {
+  if (e == WarpTopK::NONE) return 0ull;
+  if (v == 0.f) v = 0.f;
+  unsigned u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)u << 32) | (unsigned)(~e);
+}
+__device__ __forceinline__ int topk_key_expert(unsigned long long key) {
+  return (int)(~(unsigned)(key & 0xffffffffull));
+}
+
+// Top k of n listed candidates (keys, raw scores; distinct experts) by rank counting: the
+// threads of the block each rank one entry against all n (no serial chain) and write the k
+// best to out[rank].  Ends with a block barrier.
+__device__ __forceinline__ void rank_select(const unsigned long long *key, const float *z, int n,
+                                            int k, unsigned long long *okey, float *oz) {
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const float v = sv[i];
-    const int e = se[i];
-    if (e == WarpTopK::NONE) continue;
+    const unsigned long long ki = key[i];
+    if (ki == 0ull) continue;
     int r = 0;
-    for (int j = 0; j < n; j++) r += (se[j] != WarpTopK::NONE && better(sv[j], se[j], v, e)) ? 1 : 0;
+    for (int j = 0; j < n; j++) r += key[j] > ki ? 1 : 0;
     if (r < k) {
-      ov[r] = v;
-      oe[r] = e;
-      oz[r] = sz[i];
+      okey[r] = ki;
+      oz[r] = z[i];
     }
   }
   __syncthreads();
@@ -905,8 +916,8 @@ template <int WPT>
 __global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float mv[WPT * 32], mz[WPT * 32], fv[32], fz[32];
-  __shared__ int me[WPT * 32], fe[32];
+  __shared__ unsigned long long mk[WPT * 32], fk[32];
+  __shared__ float mz[WPT * 32], fz[32];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int tok = WPT == 1 ? blockIdx.x * 8 + wib : blockIdx.x;
   if (tok >= a.n_tok) return;  // whole warp (WPT 1) or whole block (WPT > 1)
@@ -922,14 +933,15 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
     emit_topk(lane, a.k, t.lv, t.le, t.lz, tok, a.mode, a.idx, a.w, a.counts_a, a.counts_b);
     return;
   }
-  mv[wib * 32 + lane] = lane < a.k ? t.lv : -INFINITY;
-  me[wib * 32 + lane] = lane < a.k ? t.le : WarpTopK::NONE;
-  mz[wib * 32 + lane] = t.lz;
+  if (lane < a.k) {  // the warps' lists, compacted
+    mk[wib * a.k + lane] = topk_key(t.lv, t.le);
+    mz[wib * a.k + lane] = t.lz;
+  }
   __syncthreads();
-  rank_select(mv, me, mz, WPT * 32, a.k, fv, fe, fz);
+  rank_select(mk, mz, WPT * a.k, a.k, fk, fz);
   if (wib == 0)
-    emit_topk(lane, a.k, fv[lane], fe[lane], fz[lane], tok, a.mode, a.idx, a.w, a.counts_a,
-              a.counts_b);
+    emit_topk(lane, a.k, 0.f, lane < a.k ? topk_key_expert(fk[lane]) : 0, fz[lane], tok, a.mode,
+              a.idx, a.w, a.counts_a, a.counts_b);
 }
 
 // Routing of few tokens (decode): a cluster of NCL CTAs per token (papernotes "Key design 2":
@@ -951,8 +963,8 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(const T *y, int h, c
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int tok = blockIdx.x / ncl;  // the same for the whole cluster
   __shared__ __align__(16) float qpart[DR], qv[DR];
-  __shared__ float mv[256], mz[256], fv[32], fz[32];
-  __shared__ int me[256], fe[32];
+  __shared__ unsigned long long mk[256], fk[32];
+  __shared__ float mz[256], fz[32];
   const bool live = tok < a.n_tok;
   const int qn = DR / ncl;
   if (live) {
@@ -1007,29 +1019,28 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(const T *y, int h, c
       t.offer_score(z * a.zscale, e, e < e1, a.bias);
     }
   }
-  mv[wib * 32 + lane] = lane < a.k ? t.lv : -INFINITY;
-  me[wib * 32 + lane] = lane < a.k ? t.le : WarpTopK::NONE;
-  mz[wib * 32 + lane] = t.lz;
-  if (threadIdx.x < 32) fe[threadIdx.x] = WarpTopK::NONE;
+  if (lane < a.k) {  // the warps' lists, compacted
+    mk[wib * a.k + lane] = topk_key(t.lv, t.le);
+    mz[wib * a.k + lane] = t.lz;
+  }
+  if (threadIdx.x < 32) fk[threadIdx.x] = 0ull;
   __syncthreads();
-  rank_select(mv, me, mz, 256, a.k, fv, fe, fz);  // this CTA's best k in fv/fe/fz
+  rank_select(mk, mz, 8 * a.k, a.k, fk, fz);  // this CTA's best k in fk / fz
   cl.sync();
   if (rank == 0) {  // gather the cluster's lists and rank them again
-    for (int i = threadIdx.x; i < ncl * 32; i += blockDim.x) {
-      const int r = i / 32, j = i % 32;
-      const bool in = j < a.k;
-      mv[i] = in ? *cl.map_shared_rank(fv + j, r) : -INFINITY;
-      me[i] = in ? *cl.map_shared_rank(fe + j, r) : WarpTopK::NONE;
-      mz[i] = in ? *cl.map_shared_rank(fz + j, r) : 0.f;
+    for (int i = threadIdx.x; i < ncl * a.k; i += blockDim.x) {
+      const int r = i / a.k, j = i % a.k;
+      mk[i] = *cl.map_shared_rank(fk + j, r);
+      mz[i] = *cl.map_shared_rank(fz + j, r);
     }
   }
   cl.sync();  // peers' lists read; they may exit
   if (rank == 0) {
     __syncthreads();
-    rank_select(mv, me, mz, ncl * 32, a.k, fv, fe, fz);
+    rank_select(mk, mz, ncl * a.k, a.k, fk, fz);
     if (live && wib == 0)
-      emit_topk(lane, a.k, fv[lane], fe[lane], fz[lane], tok, a.mode, a.idx, a.w, a.counts_a,
-                a.counts_b);
+      emit_topk(lane, a.k, 0.f, lane < a.k ? topk_key_expert(fk[lane]) : 0, fz[lane], tok,
+                a.mode, a.idx, a.w, a.counts_a, a.counts_b);
   }
 }
 
