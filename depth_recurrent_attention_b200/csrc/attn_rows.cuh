@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
   const int nrow = a.l + 1;
   const long row_el = 2L * a.h;                        // elements of one depth row (K then V)
   const uint32_t chunk_bytes = (uint32_t)(a.chunk * row_el * sizeof(T));
-  T *buf[2] = {reinterpret_cast<T *>(dsm), reinterpret_cast<T *>(dsm + chunk_bytes)};
+  auto buf = [&](int i) { return reinterpret_cast<T *>(dsm + (size_t)i * chunk_bytes); };
   const T *src = reinterpret_cast<const T *>(a.kv) + (long)tok * a.L * row_el;
   const int nchunks = (nrow + a.chunk - 1) / a.chunk;
   if (threadIdx.x == 0) {
@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
                  "r"(bytes)
                  : "memory");
-    tcda::bulk_load(tcda::smem_u32(buf[c & 1]), src + (long)r0 * row_el, bytes, bar);
+    tcda::bulk_load(tcda::smem_u32(buf(c & 1)), src + (long)r0 * row_el, bytes, bar);
   };
   int issued = 0;  // chunks issued (thread 0's count)
   if (threadIdx.x == 0) {
@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
       }
     }
     if (!abort_flag) consumed = c + 1;
-    const T *bk = buf[c & 1];  // on a timeout the pass below reads stale data; nothing is stored
+    const T *bk = buf(c & 1);  // on a timeout the pass below reads stale data; nothing is stored
     const int nr = min(a.chunk, nrow - c * a.chunk);
     if (active) {
       for (int g = 0; g < nr; g += U * RPW) {

@@ -49,6 +49,7 @@ struct dreamer_handle {
   int *pcursor = nullptr, *prows = nullptr, *pinv = nullptr;
   int *err = nullptr;
   void *k3 = nullptr;            // [E][3 d_r] bf16: router keys repeated for split scores
+  void *kEt = nullptr;           // [d_r][E] bf16: router keys transposed (CUDA-core scores)
   int num_sms = 148;
   int qkv_perm = 0;  // q_SA / k_SA columns of the fused QKV weight in EpiQKV perm order
   int use_tc = 1;  // bf16 contractions on tcgen05 (0: CUDA cores, for cross-checks)
@@ -413,19 +414,19 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     DALLOC(h->ew, Tk * sizeof(float));
     DALLOC(h->eidx, Tk * sizeof(int));
     DALLOC(h->counts, (size_t)L * E * sizeof(int));
-    DALLOC(h->ecnt, E * sizeof(int));
+    DALLOC(h->ecnt, 2 * E * sizeof(int));  // counts | rank counters, zero between depths
+    h->ecursor = h->ecnt + E;
     DALLOC(h->eoffs, (E + 1) * sizeof(int));
     DALLOC(h->etiles_a, (E + 1) * sizeof(int));
     DALLOC(h->etiles_b, (E + 1) * sizeof(int));
-    DALLOC(h->ecursor, E * sizeof(int));
     DALLOC(h->erows, Tk * sizeof(int));
     DALLOC(h->einv, Tk * sizeof(int));
     DALLOC(h->Ybuf, (size_t)(Tk + 128) * hd * es);
-    DALLOC(h->pcnt, (G + 1) * sizeof(int));
+    DALLOC(h->pcnt, 2 * (G + 1) * sizeof(int));  // counts | rank counters
+    h->pcursor = h->pcnt + G + 1;
     DALLOC(h->poffs, (G + 1) * sizeof(int));
     DALLOC(h->ptiles_a, (G + 1) * sizeof(int));
     DALLOC(h->ptiles_b, (G + 1) * sizeof(int));
-    DALLOC(h->pcursor, (G + 1) * sizeof(int));
     DALLOC(h->prows, T * sizeof(int));
     DALLOC(h->pinv, T * sizeof(int));
     DALLOC(h->err, sizeof(int));
@@ -441,6 +442,8 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     }
     CK(cudaMemset(h->err, 0, sizeof(int)));
     CK(cudaMemset(h->counts, 0, (size_t)L * E * sizeof(int)));
+    CK(cudaMemset(h->ecnt, 0, 2 * E * sizeof(int)));
+    CK(cudaMemset(h->pcnt, 0, 2 * (G + 1) * sizeof(int)));
     int r3 = tc_init(h);
     if (r3) return r3;
     CK(cudaDeviceSynchronize());
@@ -714,14 +717,12 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   if (P > 0) {
     mark(h, s, DREAMER_STAGE_PROJ_ROUTE);
     LAUNCHED(2);
-    cudaMemsetAsync(h->pcnt, 0, (G + 1) * sizeof(int), s);
-    pdl_break(h, s);
+    // pcnt / pcursor are zero here: cleared at init and by every depth's combine kernel
     if (!(tc && tc_proj_route(h, l, h->xh, n, s)))
       route_rows<T>(h, 1, l, h->xh, n, h->pidx, h->psig, nullptr, h->pcnt, s);
-    launch_k(h, scan_kernel, dim3(1), dim3(1024), 0, s, (const int *)h->pcnt, G, h->poffs,
-             h->ptiles_a, 64, h->ptiles_b, 128, h->pcursor);
-    launch_k(h, scatter_kernel, dim3(cdiv(n, 256)), dim3(256), 0, s, (const int *)h->pidx, n,
-             h->pcursor, h->prows, h->pinv);
+    launch_k(h, permute_kernel, dim3(cdiv(n, 1024)), dim3(1024), (size_t)(G + 1) * sizeof(int), s,
+             (const int *)h->pcnt, G, (const int *)h->pidx, n, h->poffs, h->ptiles_a, 64,
+             h->ptiles_b, 128, h->pcursor, h->prows, h->pinv);
     prow = h->prows;
     psig = h->psig;
   }
@@ -846,14 +847,19 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   if (by_rows) {
     route_rows<T>(h, 0, l, ein, n, h->eidx, h->ew, h->counts + (size_t)l * E, nullptr, s);
   } else {
-    cudaMemsetAsync(h->ecnt, 0, E * sizeof(int), s);
-    pdl_break(h, s);
+    // ecnt / ecursor are zero here: cleared at init and by every depth's combine kernel
     route_rows<T>(h, 0, l, ein, n, h->eidx, h->ew, h->counts + (size_t)l * E, h->ecnt, s);
     mark(h, s, DREAMER_STAGE_PERMUTE);
-    launch_k(h, scan_kernel, dim3(1), dim3(1024), 0, s, (const int *)h->ecnt, E, h->eoffs,
-             h->etiles_a, 64, h->etiles_b, 128, h->ecursor);
-    launch_k(h, scatter_kernel, dim3(cdiv((long)n * k, 256)), dim3(256), 0, s,
-             (const int *)h->eidx, n * k, h->ecursor, h->erows, h->einv);
+    if (E <= 8192) {
+      launch_k(h, permute_kernel, dim3(cdiv((long)n * k, 1024)), dim3(1024),
+               (size_t)(E + 1) * sizeof(int), s, (const int *)h->ecnt, E, (const int *)h->eidx,
+               n * k, h->eoffs, h->etiles_a, 64, h->etiles_b, 128, h->ecursor, h->erows, h->einv);
+    } else {
+      launch_k(h, scan_kernel, dim3(1), dim3(1024), 0, s, (const int *)h->ecnt, E, h->eoffs,
+               h->etiles_a, 64, h->etiles_b, 128, h->ecursor);
+      launch_k(h, scatter_kernel, dim3(cdiv((long)n * k, 256)), dim3(256), 0, s,
+               (const int *)h->eidx, n * k, h->ecursor, h->erows, h->einv);
+    }
   }
   // 7. expert FFNs: H = SiLU(X W1_e), acc[token] += w * H W2_e
   mark(h, s, DREAMER_STAGE_EXPERTS);
@@ -884,7 +890,8 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   launch_k(h, combine, dim3(cb), dim3(256), 0, s, h->acc, (const T *)h->Ybuf,
            by_rows ? (const int *)nullptr : (const int *)h->einv, (const float *)h->ew, k,
            (const T *)h->g, (T *)h->xh,
-           h->inv_rms, last ? (T *)io.x_out : (T *)nullptr, n, hd, c.rms_eps);
+           h->inv_rms, last ? (T *)io.x_out : (T *)nullptr, n, hd, c.rms_eps, h->ecnt, 2 * E,
+           h->pcnt, P > 0 ? 2 * (G + 1) : 0);
 }
 
 // The device error flag is copied to pinned host memory at the end of every call; the next
@@ -1003,6 +1010,10 @@ static int forward_impl(dreamer_handle *h, const void *x_in, void *x_out, int l0
   const dreamer_config &c = h->cfg;
   const int n = c.batch * c.seq;
   CK(cudaMemsetAsync(h->counts, 0, (size_t)c.depth * c.n_experts * sizeof(int), s));
+  // grouping counters: zero between depths by construction; cleared here as well so that a
+  // call after a failed one starts clean
+  CK(cudaMemsetAsync(h->ecnt, 0, 2 * (size_t)c.n_experts * sizeof(int), s));
+  CK(cudaMemsetAsync(h->pcnt, 0, 2 * (size_t)((c.n_proj_experts > 0 ? c.n_proj_experts : 1) + 1) * sizeof(int), s));
   pdl_break(h, s);
   pdl_break(h, h->side);
   DepthIO io{};
@@ -1051,6 +1062,10 @@ static int decode_impl(dreamer_handle *h, const void *x_new, void *kc, void *vc,
   const dreamer_config &c = h->cfg;
   const int n = c.batch;
   CK(cudaMemsetAsync(h->counts, 0, (size_t)c.depth * c.n_experts * sizeof(int), s));
+  // grouping counters: zero between depths by construction; cleared here as well so that a
+  // call after a failed one starts clean
+  CK(cudaMemsetAsync(h->ecnt, 0, 2 * (size_t)c.n_experts * sizeof(int), s));
+  CK(cudaMemsetAsync(h->pcnt, 0, 2 * (size_t)((c.n_proj_experts > 0 ? c.n_proj_experts : 1) + 1) * sizeof(int), s));
   pdl_break(h, s);
   pdl_break(h, h->side);
   DepthIO io{};

@@ -604,9 +604,16 @@ template <typename T, int MAXV>
 __global__ void __launch_bounds__(256) combine_norm_kernel(float *acc, const T *Y, const int *pos,
                                                           const float *wts, int k, const T *gain,
                                                           T *xh, float *inv_rms, T *x_out,
-                                                          int n_tok, int h, float eps) {
+                                                          int n_tok, int h, float eps,
+                                                          int *zero_a, int na, int *zero_b,
+                                                          int nb) {
   pdl_wait();
   pdl_trigger();
+  {  // the depth's grouping counters, cleared for the next depth (nothing reads them now)
+    const int t = blockIdx.x * blockDim.x + threadIdx.x, nt = gridDim.x * blockDim.x;
+    for (int i = t; i < na; i += nt) zero_a[i] = 0;
+    for (int i = t; i < nb; i += nt) zero_b[i] = 0;
+  }
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= n_tok) return;
@@ -944,6 +951,50 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
               a.idx, a.w, a.counts_a, a.counts_b);
 }
 
+// Scores and top-k from a stored router query, one warp per token: q arrives as the three
+// bf16 parts q_hi + q_mid + q_lo of R_l^T q (the split the tensor-core query GEMM writes), the
+// keys unrotated and transposed [d_r][E]; lane j scores experts b + 2j and b + 2j + 1 of each
+// batch of 64 (one 128-byte row read a key dimension, shared through L1 by the block's warps),
+// z_e = q . k_e in fp32, then the warp top-k.  For batches too short to fill the GPU with
+// fused score tiles.  E even.
+template <int DR>
+__global__ void __launch_bounds__(256) route_q_topk_kernel(const bf16 *qs3, const bf16 *kt,
+                                                           TopkArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int tok = blockIdx.x * 8 + wib;
+  if (tok >= a.n_tok) return;
+  float q[DR];
+  const bf16 *qr = qs3 + (long)tok * 3 * DR;
+#pragma unroll
+  for (int j = 0; j < DR; j += 8) {
+    float hi[8], mid[8], lo[8];
+    load8(qr + j, hi);
+    load8(qr + DR + j, mid);
+    load8(qr + 2 * DR + j, lo);
+#pragma unroll
+    for (int u = 0; u < 8; u++) q[j + u] = (hi[u] + mid[u]) + lo[u];
+  }
+  WarpTopK t(a.k, lane);
+  for (int b = 0; b < a.E; b += 64) {
+    const int e = b + 2 * lane;
+    float z0 = 0.f, z1 = 0.f;
+    if (e < a.E) {
+#pragma unroll
+      for (int j = 0; j < DR; j++) {
+        const float2 f =
+            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(kt + (long)j * a.E + e));
+        z0 = fmaf(q[j], f.x, z0);
+        z1 = fmaf(q[j], f.y, z1);
+      }
+    }
+    t.offer_score(z0 * a.zscale, e, e < a.E, a.bias);
+    t.offer_score(z1 * a.zscale, e + 1, e + 1 < a.E, a.bias);
+  }
+  emit_topk(lane, a.k, t.lv, t.le, t.lz, tok, a.mode, a.idx, a.w, a.counts_a, a.counts_b);
+}
+
 // Routing of few tokens (decode): a cluster of NCL CTAs per token (papernotes "Key design 2":
 // router query, sigmoid scores against depth-RoPE'd expert keys, biased top-k).  Each CTA
 // computes DR/NCL entries of the query q = y W_q (fp32), the cluster gathers q through
@@ -1099,6 +1150,77 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *cnt, int G, int *
     offs[G] = s0[1023];
     tiles_a[G] = s1[1023];
     if (tiles_b) tiles_b[G] = s2[1023];
+  }
+}
+
+// Counting sort in one kernel (G <= 8192 groups): every CTA scans the group counts into its
+// shared memory (exclusive prefix), CTA 0 also publishes offs and the row-tile prefixes for
+// the grouped GEMMs, and each thread places one item: rows[offs[g] + rank] = i, inv[i] = that
+// position, the rank within the group taken from ctr[g] (zero on entry; the order inside a
+// group is not fixed, every row is computed on its own).
+__global__ void __launch_bounds__(1024) permute_kernel(const int *cnt, int G, const int *idx,
+                                                       int n, int *offs, int *tiles_a, int bm_a,
+                                                       int *tiles_b, int bm_b, int *ctr, int *rows,
+                                                       int *inv) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ int so[];  // [G + 1]
+  __shared__ int s0[1024], s1[1024], s2[1024];
+  const int tid = threadIdx.x;
+  const bool pub = blockIdx.x == 0;
+  const int per = (G + 1023) / 1024;
+  int a0 = 0, a1 = 0, a2 = 0;
+  for (int i = 0; i < per; i++) {
+    const int g = tid * per + i;
+    if (g < G) {
+      const int c = cnt[g];
+      a0 += c;
+      a1 += (c + bm_a - 1) / bm_a;
+      a2 += (c + bm_b - 1) / bm_b;
+    }
+  }
+  s0[tid] = a0;
+  s1[tid] = a1;
+  s2[tid] = a2;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {
+    const int v0 = tid >= o ? s0[tid - o] : 0;
+    const int v1 = tid >= o ? s1[tid - o] : 0;
+    const int v2 = tid >= o ? s2[tid - o] : 0;
+    __syncthreads();
+    s0[tid] += v0;
+    s1[tid] += v1;
+    s2[tid] += v2;
+    __syncthreads();
+  }
+  int b0 = tid ? s0[tid - 1] : 0, b1 = tid ? s1[tid - 1] : 0, b2 = tid ? s2[tid - 1] : 0;
+  for (int i = 0; i < per; i++) {
+    const int g = tid * per + i;
+    if (g < G) {
+      const int c = cnt[g];
+      so[g] = b0;
+      if (pub) {
+        offs[g] = b0;
+        tiles_a[g] = b1;
+        if (tiles_b) tiles_b[g] = b2;
+      }
+      b0 += c;
+      b1 += (c + bm_a - 1) / bm_a;
+      b2 += (c + bm_b - 1) / bm_b;
+    }
+  }
+  if (tid == 1023 && pub) {
+    offs[G] = s0[1023];
+    tiles_a[G] = s1[1023];
+    if (tiles_b) tiles_b[G] = s2[1023];
+  }
+  __syncthreads();
+  const int i = blockIdx.x * 1024 + tid;
+  if (i < n) {
+    const int g = idx[i];
+    const int p = so[g] + atomicAdd(ctr + g, 1);
+    rows[p] = i;
+    if (inv) inv[i] = p;
   }
 }
 

@@ -237,6 +237,12 @@ static int tc_init(dreamer_handle *h) {
       if (cudaMemcpy2D((char *)h->k3 + i * dr * 2, 3 * dr * 2, h->kE_raw, dr * 2, dr * 2, E,
                        cudaMemcpyDeviceToDevice) != cudaSuccess)
         return DREAMER_ERR_CUDA;
+    // [d_r][E]: the keys transposed, so that a warp scoring 64 experts reads 128-byte rows
+    if (dalloc(h, &h->kEt, (size_t)E * dr * 2)) return DREAMER_ERR_OOM;
+    dreamer::transpose_absorb_kernel<dreamer::bf16>
+        <<<dim3((dr + 31) / 32, (E + 31) / 32, 1), dim3(32, 8)>>>(
+            (const dreamer::bf16 *)h->kE_raw, nullptr, (dreamer::bf16 *)h->kEt, E, dr, 1);
+    if (cudaGetLastError() != cudaSuccess) return DREAMER_ERR_CUDA;
   }
   return tc_attn_init(h);
 }
@@ -383,8 +389,8 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
   }
   const float zs = 1.0f / sqrtf((float)dr);
   // The fused top-k gives each 128-row tile to one CTA for all E columns: worth it only when
-  // there are enough row tiles to fill the GPU; otherwise scores go through memory and the
-  // warp top-k spreads the rows over every SM.
+  // there are enough row tiles to fill the GPU; otherwise a warp per token scores its row from
+  // the split query on the CUDA cores, which spreads the rows over every SM.
   const int k_fused = (n + 127) / 128 >= h->num_sms / 2 ? c.top_k : 0;
   switch (k_fused) {  // top-k fused into the score GEMM
     case 4:
@@ -402,12 +408,13 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
     default:
       break;
   }
-  tc_launch<256, 64, 4, false, 64>(h, t2, ta2, tb2, mt2, EpiStoreF32{h->zbuf, h->ldz, E}, s);
+  // scores straight from the split query, one warp a token (tc_route_ok: d_r is 64 or 128)
   TopkArgs k{};
-  k.n_tok = n; k.E = E; k.k = c.top_k; k.mode = 0;
-  k.z = h->zbuf; k.ldz = h->ldz; k.zscale = 1.0f / sqrtf((float)dr);
+  k.n_tok = n; k.E = E; k.k = c.top_k; k.mode = 0; k.zscale = zs;
   k.bias = h->bias; k.idx = idx; k.w = w; k.counts_a = counts_a; k.counts_b = counts_b;
-  launch_topk(h, k, s);
+  auto kern = dr == 64 ? route_q_topk_kernel<64> : route_q_topk_kernel<128>;
+  launch_k(h, kern, dim3((n + 7) / 8), dim3(256), 0, s, (const bf16 *)h->qsplit,
+           (const bf16 *)h->kEt, k);
   return true;
 }
 
