@@ -160,12 +160,36 @@ class ClockSampler:
 # ----------------------------------------------------------------------------------------
 # our arm
 
+# ----------------------------------------------------------------------------------------
+# multi-rank host logic (one replica per GPU; tested on CPU with gloo ranks)
+
+def rank_seed(cfg, rank: int) -> int:
+    """Seed of rank `rank`'s input batch: every rank draws its own batch, weights are shared."""
+    return cfg.seed + 1000 * rank
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The slowest rank's time: all-reduce MAX (no-op on one rank)."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(cfg, world: int, ms_per_step: float):
+    """(units of the whole job per step, whole-job units/s): all ranks' units over the
+    slowest rank's step time."""
+    units = cfg.units * world
+    return units, units / (ms_per_step / 1e3)
+
+
 def device_setup(cfg, torch, rank):
     W = inputs.device_weights(cfg)
     X = inputs.device_inputs(cfg)
     if rank:
-        # each rank draws its own batch (the next seed), weights are shared
-        X = {s.name: inputs.device_tensor(s, cfg.seed + 1000 * rank) for s in inputs.input_specs(cfg)}
+        X = {s.name: inputs.device_tensor(s, rank_seed(cfg, rank)) for s in inputs.input_specs(cfg)}
     return W, X
 
 
@@ -215,14 +239,9 @@ def run_ours(args, cfg, rank, world, torch, dist):
     barrier()
     launches = model.stats(reset=True)["launches"]
     ms_steps = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms_total = float(sum(ms_steps))
-    if dist is not None:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(float(sum(ms_steps)), dist, dev)
     ms_step = ms_total / args.steps
-    units = cfg.units * world
-    value = units / (ms_step / 1e3)
+    units, value = job_value(cfg, world, ms_step)
     clocks = clk.summary()
 
     # ---- per-stage device times (same workload, profiling events on, separate run)
@@ -277,11 +296,7 @@ def run_ours(args, cfg, rank, world, torch, dist):
             host_out.copy_(x_out, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
-        ms_e2e = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1), dist, dev)
         nbytes = x_in.numel() * x_in.element_size()
         e2e = {"value": units / (ms_e2e / args.steps / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
@@ -301,11 +316,7 @@ def run_ours(args, cfg, rank, world, torch, dist):
             host_out.copy_(x_out, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
-        ms_e2e = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1), dist, dev)
         nbytes = x_in.numel() * x_in.element_size()
         e2e = {"value": units / (ms_e2e / args.steps / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
