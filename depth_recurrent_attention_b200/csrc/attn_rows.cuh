@@ -166,12 +166,14 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(RowsArgs a) {
 
 
 // =======================================================================================
-// Depth attention, one CTA per token: the token's depth KV rows 0..l for all heads are one
-// contiguous run of the [T][L][2][h] buffer ((l + 1) * 2h elements), so thread 0 streams it
-// into shared memory with 1-D bulk TMA copies in chunks of CHUNK depths (two buffers), and
-// warp `head` attends over its head's slice of every row: score over d with a warp sum,
-// online softmax across rows, output chunk per lane (papernotes "Key design 1": DA attends
-// over the same token's states at depths 0..l).
+// Depth attention as one stream per CTA: a token's depth KV rows 0..l for all heads are one
+// contiguous run of the [T][L][2][h] buffer ((l + 1) * 2h elements).  A CTA takes the tokens
+// blockIdx.x, blockIdx.x + gridDim.x, ... and cuts each run into chunks of CHUNK depths; the
+// (token, chunk) items form one sequence that thread 0 streams into an NB-deep ring of
+// shared-memory buffers with 1-D bulk copies (the token's query row rides with its first
+// chunk), so the copies of the next token overlap the arithmetic of this one.  Warp `head`
+// attends over its head's slice of every row in the row-group layout of the kernels above
+// (papernotes "Key design 1": DA attends over the same token's states at depths 0..l).
 // =======================================================================================
 namespace tcda {
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -215,42 +217,47 @@ template <typename T, int D>
 __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
   pdl_wait();
   pdl_trigger();
+  constexpr int NB = 2;
   extern __shared__ __align__(128) uint8_t dsm[];
-  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ __align__(8) uint64_t bars[NB];
   __shared__ int abort_flag;
-  const int tok = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nrow = a.l + 1;
+  const int nch = (nrow + a.chunk - 1) / a.chunk;
   const long row_el = 2L * a.h;                        // elements of one depth row (K then V)
   const uint32_t chunk_bytes = (uint32_t)(a.chunk * row_el * sizeof(T));
-  auto buf = [&](int i) { return reinterpret_cast<T *>(dsm + (size_t)i * chunk_bytes); };
-  const T *src = reinterpret_cast<const T *>(a.kv) + (long)tok * a.L * row_el;
-  const int nchunks = (nrow + a.chunk - 1) / a.chunk;
+  const uint32_t q_bytes = (uint32_t)(a.h * sizeof(T));
+  const int ntok = a.n_tok > (int)blockIdx.x ? (a.n_tok - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int nitems = ntok * nch;
+  if (nitems == 0) return;  // the whole CTA
+  auto kv_slot = [&](int b) { return dsm + (size_t)b * chunk_bytes; };
+  auto q_slot = [&](int b) { return dsm + (size_t)NB * chunk_bytes + (size_t)b * q_bytes; };
   if (threadIdx.x == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tcda::smem_u32(&bars[0])) : "memory");
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tcda::smem_u32(&bars[1])) : "memory");
+    for (int i = 0; i < NB; i++)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tcda::smem_u32(&bars[i])) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     abort_flag = 0;
   }
   __syncthreads();
-  auto issue = [&](int c) {
+  auto issue = [&](int j) {
+    const int b = j % NB, c = j % nch;
+    const int tok = (int)blockIdx.x + (j / nch) * (int)gridDim.x;
     const int r0 = c * a.chunk, nr = min(a.chunk, nrow - r0);
-    const uint32_t bytes = (uint32_t)(nr * row_el * sizeof(T));
-    const uint32_t bar = tcda::smem_u32(&bars[c & 1]);
+    const uint32_t kvb = (uint32_t)(nr * row_el * sizeof(T));
+    const uint32_t bar = tcda::smem_u32(&bars[b]);
+    const uint32_t total = kvb + (c == 0 ? q_bytes : 0u);
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
-                 "r"(bytes)
+                 "r"(total)
                  : "memory");
-    tcda::bulk_load(tcda::smem_u32(buf(c & 1)), src + (long)r0 * row_el, bytes, bar);
+    tcda::bulk_load(tcda::smem_u32(kv_slot(b)),
+                    reinterpret_cast<const T *>(a.kv) + ((long)tok * a.L + r0) * row_el, kvb, bar);
+    if (c == 0)
+      tcda::bulk_load(tcda::smem_u32(q_slot(b)), reinterpret_cast<const T *>(a.q) + (long)tok * a.h,
+                      q_bytes, bar);
   };
-  int issued = 0;  // chunks issued (thread 0's count)
-  if (threadIdx.x == 0) {
-    issue(0);
-    issued = 1;
-    if (nchunks > 1) {
-      issue(1);
-      issued = 2;
-    }
-  }
+  int issued = 0;  // items issued (thread 0's count)
+  if (threadIdx.x == 0)
+    for (; issued < NB && issued < nitems; issued++) issue(issued);
   // row-group layout: CH lanes of 16 bytes cover a row, RPW rows per warp step
   constexpr int VEC = VecOf<T>::N;
   constexpr int CH = D / VEC;
@@ -259,21 +266,15 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
   const int cc = lane % CH, rr = lane / CH;
   const int head = warp;
   const bool active = head < a.H;
-  float q[VEC], o[VEC];
   const float sl2 = 1.4426950408889634f * rsqrtf((float)D);
-  if (active) ld16(reinterpret_cast<const T *>(a.q) + (long)tok * a.h + head * D + cc * VEC, q);
-#pragma unroll
-  for (int i = 0; i < VEC; i++) {
-    q[i] = active ? q[i] * sl2 : 0.f;
-    o[i] = 0.f;
-  }
+  float q[VEC], o[VEC];
   float m = -INFINITY, lsum = 0.f;
   int consumed = 0;
-  for (int c = 0; c < nchunks; c++) {
-    // wait for chunk c (bounded; on expiry every thread leaves the loop)
-    const uint32_t bar = tcda::smem_u32(&bars[c & 1]);
-    const uint32_t par = (c >> 1) & 1;
-    if (!tcda::try_wait(bar, par)) {
+  for (int j = 0; j < nitems; j++) {
+    const int b = j % NB, c = j % nch;
+    const uint32_t bar = tcda::smem_u32(&bars[b]);
+    const uint32_t par = (uint32_t)((j / NB) & 1);
+    if (!tcda::try_wait(bar, par)) {  // bounded; on expiry every thread stops after the barrier
       const uint64_t t0 = tcda::gtimer();
       while (!tcda::try_wait(bar, par)) {
         if (abort_flag) break;
@@ -284,19 +285,29 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
         }
       }
     }
-    if (!abort_flag) consumed = c + 1;
-    const T *bk = buf(c & 1);  // on a timeout the pass below reads stale data; nothing is stored
+    if (!abort_flag) consumed = j + 1;
+    const T *bk = reinterpret_cast<const T *>(kv_slot(b));  // stale after a timeout; nothing is stored then
     const int nr = min(a.chunk, nrow - c * a.chunk);
     if (active) {
+      if (c == 0) {  // a new token: its query, a fresh softmax
+        ld16(reinterpret_cast<const T *>(q_slot(b)) + head * D + cc * VEC, q);
+#pragma unroll
+        for (int i = 0; i < VEC; i++) {
+          q[i] *= sl2;
+          o[i] = 0.f;
+        }
+        m = -INFINITY;
+        lsum = 0.f;
+      }
       for (int g = 0; g < nr; g += U * RPW) {
         float s[U], vv[U][VEC];
 #pragma unroll
         for (int u = 0; u < U; u++) {
-          const int j = g + u * RPW + rr;
+          const int jr = g + u * RPW + rr;
           s[u] = -INFINITY;
-          if (j < nr) {
+          if (jr < nr) {
             float kv[VEC];
-            const T *kr = bk + (long)j * row_el + head * D + cc * VEC;
+            const T *kr = bk + (long)jr * row_el + head * D + cc * VEC;
             ld16(kr, kv);
             ld16(kr + a.h, vv[u]);
             float p = 0.f;
@@ -335,36 +346,40 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
         lsum = lsum * alpha + ps;
         m = mn;
       }
+      if (c == nch - 1) {  // the token's last chunk: fold the RPW rows, normalise, store
+        float of[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; i++) of[i] = o[i];
+#pragma unroll
+        for (int o2 = CH; o2 < 32; o2 <<= 1)
+#pragma unroll
+          for (int i = 0; i < VEC; i++) of[i] += __shfl_xor_sync(0xffffffffu, of[i], o2);
+        if (rr == 0 && !abort_flag) {
+          const int tok = (int)blockIdx.x + (j / nch) * (int)gridDim.x;
+          const float inv = 1.0f / lsum;
+#pragma unroll
+          for (int i = 0; i < VEC; i++) of[i] *= inv;
+          st16(reinterpret_cast<T *>(a.out) + (long)tok * a.ldo + a.col0 + head * D + cc * VEC, of);
+        }
+      }
     }
-    __syncthreads();  // every warp is done with buffer c & 1
+    __syncthreads();        // buffer b is free again
     if (abort_flag) break;  // read after the barrier: the same decision in every thread
-    if (threadIdx.x == 0 && c + 2 < nchunks) {
-      issue(c + 2);
-      issued = c + 3;
+    if (threadIdx.x == 0 && issued < nitems) {
+      issue(issued);
+      issued++;
     }
-  }
-  // reduce the output chunks over the RPW rows of the warp
-#pragma unroll
-  for (int o2 = CH; o2 < 32; o2 <<= 1)
-#pragma unroll
-    for (int i = 0; i < VEC; i++) o[i] += __shfl_xor_sync(0xffffffffu, o[i], o2);
-  if (active && !abort_flag && rr == 0) {
-    const float inv = 1.0f / lsum;
-#pragma unroll
-    for (int i = 0; i < VEC; i++) o[i] *= inv;
-    st16(reinterpret_cast<T *>(a.out) + (long)tok * a.ldo + a.col0 + head * D + cc * VEC, o);
   }
   // copies still in flight after an abort land before the CTA exits
   if (threadIdx.x == 0 && abort_flag) {
-    for (int c = consumed; c < issued; c++) {
+    for (int j = consumed; j < issued; j++) {
       const uint64_t t0 = tcda::gtimer();
-      while (!tcda::try_wait(tcda::smem_u32(&bars[c & 1]), (c >> 1) & 1) &&
+      while (!tcda::try_wait(tcda::smem_u32(&bars[j % NB]), (uint32_t)((j / NB) & 1)) &&
              tcda::gtimer() - t0 < 2000000000ull) {
       }
     }
   }
 }
-
 
 // =======================================================================================
 // Decode attention over the per-depth SA cache, streamed: one CTA per (sequence, head, key

@@ -534,23 +534,31 @@ static void launch_attn(const AttnArgs &a, int d, cudaStream_t s) {
 }
 
 // depth attention, one CTA per token streaming its depth history through shared memory
+// depth attention: as many CTAs as fit on the GPU, each streaming its tokens' depth runs
 template <typename T>
 static void launch_da_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStream_t s) {
   DaBulkArgs a{};
   a.n_tok = r.n_q; a.H = r.H; a.h = r.h; a.L = r.L; a.l = r.l;
   const long row_bytes = 2L * r.h * sizeof(T);
-  int chunk = (int)((50 * 1024) / row_bytes);
+  int chunk = (int)((48 * 1024) / row_bytes);
   if (chunk < 1) chunk = 1;
   if (chunk > r.l + 1) chunk = r.l + 1;
   a.chunk = chunk;
   a.q = r.q; a.kv = r.kv; a.out = r.out; a.ldo = r.ldo; a.col0 = r.col0; a.err = r.err;
-  const int smem = (int)(2 * chunk * row_bytes);
+  const int smem = (int)(2 * (chunk * row_bytes + r.h * (long)sizeof(T)));
   const int threads = 32 * r.H;
+  int per_sm = (227 * 1024) / smem;
+  if (per_sm > 2048 / threads) per_sm = 2048 / threads;
+  if (per_sm > 8) per_sm = 8;
+  if (per_sm < 1) per_sm = 1;
+  long grid = (long)h->num_sms * per_sm;
+  if (grid > a.n_tok) grid = a.n_tok;
+  if (grid < 1) grid = 1;
   auto go = [&](void (*kern)(DaBulkArgs)) {
     // set for the kernel launched (the four head sizes share one pointer type)
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    launch_k(h, kern, dim3(a.n_tok), dim3(threads), smem, s, a);
+    launch_k(h, kern, dim3((unsigned)grid), dim3(threads), smem, s, a);
   };
   switch (d) {
     case 16: go(da_bulk_kernel<T, 16>); break;
@@ -587,7 +595,7 @@ static void launch_dec_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStr
 // depth attention (mode 0) or split decode attention + merge (mode 2)
 template <typename T>
 static void launch_rows(dreamer_handle *h, const RowsArgs &a, int d, cudaStream_t s) {
-  if (a.mode == 0 && a.H <= 32 && 2L * a.h * (long)sizeof(T) <= 50 * 1024) {
+  if (a.mode == 0 && a.H <= 32 && 2L * a.h * (long)sizeof(T) <= 48 * 1024) {
     launch_da_bulk<T>(h, a, d, s);
     return;
   }
