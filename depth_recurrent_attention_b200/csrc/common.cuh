@@ -65,6 +65,11 @@ __device__ __forceinline__ void store4(bf16 *p, const float *v) {
   *reinterpret_cast<uint2 *>(p) = u;
 }
 
+// L2 prefetch of the 128-byte line holding p
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -83,6 +83,17 @@ template <typename T> struct EpiQKV {
   __device__ __forceinline__ int row_aux(int r, int token) const {
     return r < 0 ? 0 : position(token);
   }
+  // the token-RoPE table rows of the tile's rows, into L2 while the tile's MMAs run
+  template <int NR>
+  __device__ __forceinline__ void prefetch(const int *r, const int *, const int *ax, int n0,
+                                           int bn, int cj, int lpr) const {
+    if ((n0 + col_lo) / h > 1) return;
+    const int lines = (d / 2) * 8 / 128;
+#pragma unroll
+    for (int i = 0; i < NR; i++)
+      if (r[i] >= 0 && ax[i] >= 0 && cj < lines)
+        prefetch_l2(reinterpret_cast<const char *>(rope_tok + (long)ax[i] * (d / 2)) + cj * 128);
+  }
   template <int NR, int NV>
   __device__ __forceinline__ void store_rows(const int *r, const int *tok, const int *ax, int g,
                                              int col, const float (*v)[NV]) const {
@@ -292,6 +303,20 @@ template <typename T> struct EpiO {
   __device__ __forceinline__ Aux row_aux(int r, int token) const {
     if (r < 0) return Aux{0.f, 0.f};
     return Aux{psig ? psig[token] : 1.0f, res_mode == 2 ? 1.f : inv_rms[token]};
+  }
+  // the residual rows of the tile, into L2 while the tile's MMAs run
+  template <int NR>
+  __device__ __forceinline__ void prefetch(const int *r, const int *tok, const Aux *, int n0,
+                                           int bn, int cj, int lpr) const {
+    const bool from_x = res_mode == 0;
+    const int lines = bn * (from_x ? (int)sizeof(T) : 4) / 128;
+#pragma unroll
+    for (int i = 0; i < NR; i++) {
+      if (r[i] < 0) continue;
+      const char *row = from_x ? reinterpret_cast<const char *>(xin + (long)tok[i] * h + n0)
+                               : reinterpret_cast<const char *>(acc + (long)tok[i] * h + n0);
+      for (int ln = cj; ln < lines; ln += lpr) prefetch_l2(row + ln * 128);
+    }
   }
   // Coalesced layout (NV values a lane and row: 4 at col, and with NV = 8 four more at
   // col + 32); all residual loads are issued before the first store.

@@ -218,8 +218,6 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
     for (int it = 0; tile_at(it, mt, nt); it++) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
-      if (!mbar_wait(smem_u32(&tfull[acc]), aph, abort_flag, a.err)) break;
-      tc_fence_after();
       int g, m0, m1;
       const int n0 = nt * BN;
       tc_tile_rows(a, mt, g, m0, m1);
@@ -227,9 +225,6 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
       const bool valid = r < m1;
       const int token = valid ? (a.arow ? a.arow[r] / a.arow_div : r) : 0;
       const uint32_t base = tmem + acc * BN + ((uint32_t)(q * 32) << 16);
-      if constexpr (ROWPASS) {
-        if (nt == 0) epi.row_begin(st);
-      }
       if constexpr (STAGED) {
         // Passes of PW = min(SEG, 64) columns.  With PW = 64 lane j of a row holds columns
         // 4j..4j+3 and 32+4j..32+4j+3 (NV = 8), so rotate-half partners 32 apart meet in
@@ -244,8 +239,10 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
         constexpr int SW = CPR >= 8 ? 7 : CPR - 1;  // chunk swizzle mask
         float *stg = stage_buf + q * 32 * 64;
         const int cj = lane % LPR;
+        // the lane's rows, their per-row values and an L2 prefetch of the tile's inputs, all
+        // while the MMAs of this tile are still running
         int crow[NIT], ctok[NIT];
-        typename Epi::Aux caux[NIT];  // per-row values the epilogue looks up once per tile
+        typename Epi::Aux caux[NIT];
 #pragma unroll
         for (int i = 0; i < NIT; i++) {
           const int rr = m0 + q * 32 + i * RPI + lane / LPR;
@@ -253,6 +250,9 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
           ctok[i] = rr < m1 ? (a.arow ? a.arow[rr] / a.arow_div : rr) : 0;
           caux[i] = epi.row_aux(crow[i], ctok[i]);
         }
+        epi.template prefetch<NIT>(crow, ctok, caux, n0, BN, cj, LPR);
+        if (!mbar_wait(smem_u32(&tfull[acc]), aph, abort_flag, a.err)) break;
+        tc_fence_after();
 #pragma unroll 1
         for (int sg = 0; sg < BN / SEG && m0 + q * 32 < m1; sg++) {
           float v[SEG];
@@ -287,6 +287,11 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
           }
         }
       } else {
+        if (!mbar_wait(smem_u32(&tfull[acc]), aph, abort_flag, a.err)) break;
+        tc_fence_after();
+        if constexpr (ROWPASS) {
+          if (nt == 0) epi.row_begin(st);
+        }
 #pragma unroll 1
         for (int sg = 0; sg < BN / SEG && m0 + q * 32 < m1; sg++) {  // skip warps with no rows
           float v[SEG];
