@@ -319,7 +319,7 @@ template <typename T> struct EpiO {
     }
   }
   // Coalesced layout (NV values a lane and row: 4 at col, and with NV = 8 four more at
-  // col + 32); all residual loads are issued before the first store.
+  // col + 32); rows in pairs, each pair's residual loads issued before its stores.
   template <int NR, int NV>
   __device__ __forceinline__ void store_rows(const int *r, const int *tok, const Aux *ax, int g,
                                              int col, const float (*v)[NV]) const {
@@ -329,27 +329,34 @@ template <typename T> struct EpiO {
       if (res_mode != 2) load4(gain + col + 32 * hh, gv + 4 * hh);
       else gv[4 * hh] = gv[4 * hh + 1] = gv[4 * hh + 2] = gv[4 * hh + 3] = 1.f;
     }
-    float xr[NR][NV];
+    constexpr int GR = NR < 2 ? NR : 2;
 #pragma unroll
-    for (int i = 0; i < NR; i++) {
-      if (r[i] < 0) continue;
+    for (int i0 = 0; i0 < NR; i0 += GR) {
+      float xr[GR][NV];
 #pragma unroll
-      for (int hh = 0; hh < NV / 4; hh++) {
-        if (res_mode == 0) load4(xin + (long)tok[i] * h + col + 32 * hh, xr[i] + 4 * hh);
-        else load4(acc + (long)tok[i] * h + col + 32 * hh, xr[i] + 4 * hh);
+      for (int i = 0; i < GR; i++) {
+        if (r[i0 + i] < 0) continue;
+#pragma unroll
+        for (int hh = 0; hh < NV / 4; hh++) {
+          const long off = (long)tok[i0 + i] * h + col + 32 * hh;
+          if (res_mode == 0) load4(xin + off, xr[i] + 4 * hh);
+          else load4(acc + off, xr[i] + 4 * hh);
+        }
       }
-    }
 #pragma unroll
-    for (int i = 0; i < NR; i++) {
-      if (r[i] < 0) continue;
-      const float s = ax[i].s, ir = ax[i].ir;
-      float o[NV];
+      for (int i = 0; i < GR; i++) {
+        if (r[i0 + i] < 0) continue;
+        const float s = ax[i0 + i].s, ir = ax[i0 + i].ir;
+        float o[NV];
 #pragma unroll
-      for (int j = 0; j < NV; j++) o[j] = (res_mode == 2 ? xr[i][j] : gv[j] * xr[i][j] * ir) + s * v[i][j];
+        for (int j = 0; j < NV; j++)
+          o[j] = (res_mode == 2 ? xr[i][j] : gv[j] * xr[i][j] * ir) + s * v[i0 + i][j];
 #pragma unroll
-      for (int hh = 0; hh < NV / 4; hh++) {
-        if (y) store4(y + (long)tok[i] * h + col + 32 * hh, o + 4 * hh);
-        store4(acc + (long)tok[i] * h + col + 32 * hh, o + 4 * hh);
+        for (int hh = 0; hh < NV / 4; hh++) {
+          const long off = (long)tok[i0 + i] * h + col + 32 * hh;
+          if (y) store4(y + off, o + 4 * hh);
+          store4(acc + off, o + 4 * hh);
+        }
       }
     }
   }

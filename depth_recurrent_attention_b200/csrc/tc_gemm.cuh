@@ -67,12 +67,14 @@ template <class E> struct EpiStaged<E, std::void_t<decltype(E::STAGED)>> {
   static constexpr bool value = E::STAGED;
 };
 
-template <int BN, int BK, int STAGES, bool GATHER, bool STAGED = false>
+template <int BN, int BK, int STAGES, bool GATHER, bool STAGED = false, int EW_ = 4>
 struct TcGemmCfg {
   static constexpr int A_BYTES = 128 * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int THREADS = GATHER ? 256 : 192;
-  static constexpr int STG_BYTES = STAGED ? 4 * 32 * 64 * 4 : 0;  // 4 warps x 32 x 64 fp32
+  static constexpr int EW = STAGED ? EW_ : 4;  // epilogue warps: 4, or 8 (two per TMEM lane quarter)
+  static_assert(EW == 4 || EW == 8, "epilogue warps");
+  static constexpr int THREADS = 64 + 32 * EW + (GATHER ? 64 : 0);
+  static constexpr int STG_BYTES = STAGED ? EW * 32 * 64 * 4 : 0;  // EW warps x 32 x 64 fp32
   // at least 120 KB so that a second CTA never shares the SM (and its 512 TMEM columns)
   static constexpr int SMEM_USED =
       STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*bars*/ + STG_BYTES;
@@ -87,12 +89,14 @@ struct TcGemmCfg {
 // ROWPASS: a CTA takes row tiles mt = blockIdx.x, blockIdx.x + gridDim.x, ... and runs all
 // N tiles of each in order, so the epilogue can carry per-row state across the N tiles
 // (Epi::State with row_begin / row_apply / row_end); otherwise tiles are strided over CTAs.
-template <int BN, int BK, int STAGES, bool GATHER, int SEG, class Epi, bool ROWPASS = false>
-__global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
+template <int BN, int BK, int STAGES, bool GATHER, int SEG, class Epi, bool ROWPASS = false,
+          int EW = 4>
+__global__ void __launch_bounds__(
+    TcGemmCfg<BN, BK, STAGES, GATHER, EpiStaged<Epi>::value && !ROWPASS, EW>::THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    TcGemmArgs a, Epi epi) {
   constexpr bool STAGED = EpiStaged<Epi>::value && !ROWPASS;
-  using C = TcGemmCfg<BN, BK, STAGES, GATHER, STAGED>;
+  using C = TcGemmCfg<BN, BK, STAGES, GATHER, STAGED, EW>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
@@ -127,7 +131,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
     }
     for (int i = 0; i < 2; i++) {
       mbar_init(smem_u32(&tfull[i]), 1);
-      mbar_init(smem_u32(&tempty[i]), 128);
+      mbar_init(smem_u32(&tempty[i]), 32 * C::EW);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -209,9 +213,10 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
         if (ok) mma_commit(smem_u32(&tfull[acc]));
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + C::EW) {
     // ------------------------------------------------------------- epilogue
-    const int q = warp & 3;
+    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    const int half = (warp - 2) >> 2;       // which of the quarter's warps (staged: 0 or 1)
     const int row = q * 32 + lane;
     int mt, nt;
     typename EpiState<Epi, ROWPASS>::type st;
@@ -237,7 +242,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
         constexpr int RPI = 32 / LPR;               // rows per step
         constexpr int NIT = 32 / RPI;               // steps per pass
         constexpr int SW = CPR >= 8 ? 7 : CPR - 1;  // chunk swizzle mask
-        float *stg = stage_buf + q * 32 * 64;
+        float *stg = stage_buf + (warp - 2) * 32 * 64;
         const int cj = lane % LPR;
         // the lane's rows, their per-row values and an L2 prefetch of the tile's inputs, all
         // while the MMAs of this tile are still running
@@ -250,41 +255,41 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
           ctok[i] = rr < m1 ? (a.arow ? a.arow[rr] / a.arow_div : rr) : 0;
           caux[i] = epi.row_aux(crow[i], ctok[i]);
         }
-        epi.template prefetch<NIT>(crow, ctok, caux, n0, BN, cj, LPR);
+        constexpr int NPW = C::EW / 4;  // warps sharing a lane quarter; they split the passes
+        epi.template prefetch<NIT>(crow, ctok, caux, n0, BN, cj + half * LPR, LPR * NPW);
         if (!mbar_wait(smem_u32(&tfull[acc]), aph, abort_flag, a.err)) break;
         tc_fence_after();
+        // passes of PW columns; pass p of the tile belongs to warp half p % NPW
 #pragma unroll 1
-        for (int sg = 0; sg < BN / SEG && m0 + q * 32 < m1; sg++) {
-          float v[SEG];
-          if (SEG >= 32) {
+        for (int p = half; p < BN / PW && m0 + q * 32 < m1; p += NPW) {
+          const int c0 = p * PW;
+          __syncwarp();
 #pragma unroll
-            for (int c = 0; c < SEG; c += 32) tmem_ld32(base + sg * SEG + c, v + c);
-          } else {
-            tmem_ld16(base + sg * SEG, v);
+          for (int c = 0; c < PW; c += 32) {  // TMEM -> row-layout transform -> shared memory
+            constexpr int W = PW < 32 ? PW : 32;
+            float v[W];
+            if (W == 32) tmem_ld32(base + c0 + c, v);
+            else tmem_ld16(base + c0 + c, v);
+            if (valid) epi.template transform<W>(r, token, g, n0 + c0 + c, v);
+#pragma unroll
+            for (int j = 0; j < W / 4; j++)
+              *reinterpret_cast<float4 *>(stg + lane * PW + (((c / 4 + j) ^ (lane & SW)) << 2)) =
+                  make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
           }
-          if (valid) epi.template transform<SEG>(r, token, g, n0 + sg * SEG, v);
+          __syncwarp();
+          float cv[NIT][NV];
 #pragma unroll
-          for (int c = 0; c < SEG; c += PW) {
-            __syncwarp();
+          for (int i = 0; i < NIT; i++) {
+            const int rl = i * RPI + lane / LPR;
 #pragma unroll
-            for (int j = 0; j < CPR; j++)
-              *reinterpret_cast<float4 *>(stg + lane * PW + ((j ^ (lane & SW)) << 2)) =
-                  make_float4(v[c + 4 * j], v[c + 4 * j + 1], v[c + 4 * j + 2], v[c + 4 * j + 3]);
-            __syncwarp();
-            float cv[NIT][NV];
-#pragma unroll
-            for (int i = 0; i < NIT; i++) {
-              const int rl = i * RPI + lane / LPR;
-#pragma unroll
-              for (int hh = 0; hh < NV / 4; hh++) {
-                const int ch = cj + hh * 8;
-                const float4 t4 = *reinterpret_cast<const float4 *>(stg + rl * PW + ((ch ^ (rl & SW)) << 2));
-                cv[i][4 * hh] = t4.x; cv[i][4 * hh + 1] = t4.y;
-                cv[i][4 * hh + 2] = t4.z; cv[i][4 * hh + 3] = t4.w;
-              }
+            for (int hh = 0; hh < NV / 4; hh++) {
+              const int ch = cj + hh * 8;
+              const float4 t4 = *reinterpret_cast<const float4 *>(stg + rl * PW + ((ch ^ (rl & SW)) << 2));
+              cv[i][4 * hh] = t4.x; cv[i][4 * hh + 1] = t4.y;
+              cv[i][4 * hh + 2] = t4.z; cv[i][4 * hh + 3] = t4.w;
             }
-            epi.template store_rows<NIT, NV>(crow, ctok, caux, g, n0 + sg * SEG + c + cj * 4, cv);
           }
+          epi.template store_rows<NIT, NV>(crow, ctok, caux, g, n0 + c0 + cj * 4, cv);
         }
       } else {
         if (!mbar_wait(smem_u32(&tfull[acc]), aph, abort_flag, a.err)) break;
@@ -315,7 +320,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, BK, STAGES, GATHER>::THREADS, 1)
     }
   } else if (GATHER) {
     // ------------------------------------------------------------- gathered A producers
-    const int tid = threadIdx.x - 192;  // 0..63
+    const int tid = threadIdx.x - (64 + 32 * C::EW);  // 0..63
     const int c = tid & 7;              // 16-byte chunk of the 128-byte row slice
     const int rsub = tid >> 3;          // 0..7
     int s = 0;

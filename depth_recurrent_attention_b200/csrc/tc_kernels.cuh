@@ -249,12 +249,13 @@ static int tc_init(dreamer_handle *h) {
 
 static void tc_destroy(dreamer_handle *h) {}
 
-template <int BN, int BK, int ST, bool GATHER, int SEG, class Epi, bool ROWPASS = false>
+template <int BN, int BK, int ST, bool GATHER, int SEG, class Epi, bool ROWPASS = false,
+          int EW = 4>
 static void tc_launch(dreamer_handle *h, const dreamer::tc::TcGemmArgs &a, const CUtensorMap &ta,
                       const CUtensorMap &tb, long max_tiles, const Epi &epi, cudaStream_t s) {
   using Cfg = dreamer::tc::TcGemmCfg<BN, BK, ST, GATHER,
-                                     dreamer::tc::EpiStaged<Epi>::value && !ROWPASS>;
-  auto kern = dreamer::tc::tc_gemm_kernel<BN, BK, ST, GATHER, SEG, Epi, ROWPASS>;
+                                     dreamer::tc::EpiStaged<Epi>::value && !ROWPASS, EW>;
+  auto kern = dreamer::tc::tc_gemm_kernel<BN, BK, ST, GATHER, SEG, Epi, ROWPASS, EW>;
   if (ROWPASS) max_tiles /= (a.N / BN);  // one unit of work per row tile
   static bool attr_set = false;
   if (!attr_set) {
@@ -320,15 +321,27 @@ static bool tc_gemm_qkv(dreamer_handle *h, const dreamer::GemmArgs &a, const dre
     const int *tiles = h->ptiles_b;
     const bool gather = a.arow != nullptr;
     // 64-column segments: the staged epilogue rotates pairs 32 columns apart (head dim 64,
-    // or 128 in perm order)
+    // or 128 in perm order).  Short K leaves little MMA time per tile to hide the epilogue
+    // behind: eight epilogue warps then, at one stage less of operand ring.
+    const bool ew8 = a.K <= 1024;
     if (tc_pick_bn(h, a) == 256) {
       if (!tc_prepare<256, 64>(h, a, tiles, a.M, t, ta, tb, mt)) return false;
-      if (gather) tc_launch<256, 64, 4, true, 64>(h, t, ta, tb, mt, e, s);
-      else tc_launch<256, 64, 4, false, 64>(h, t, ta, tb, mt, e, s);
+      if (ew8) {
+        if (gather) tc_launch<256, 64, 3, true, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        else tc_launch<256, 64, 3, false, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
+      } else {
+        if (gather) tc_launch<256, 64, 4, true, 64>(h, t, ta, tb, mt, e, s);
+        else tc_launch<256, 64, 4, false, 64>(h, t, ta, tb, mt, e, s);
+      }
     } else {
       if (!tc_prepare<128, 64>(h, a, tiles, a.M, t, ta, tb, mt)) return false;
-      if (gather) tc_launch<128, 64, 6, true, 64>(h, t, ta, tb, mt, e, s);
-      else tc_launch<128, 64, 6, false, 64>(h, t, ta, tb, mt, e, s);
+      if (ew8) {
+        if (gather) tc_launch<128, 64, 5, true, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        else tc_launch<128, 64, 5, false, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
+      } else {
+        if (gather) tc_launch<128, 64, 6, true, 64>(h, t, ta, tb, mt, e, s);
+        else tc_launch<128, 64, 6, false, 64>(h, t, ta, tb, mt, e, s);
+      }
     }
     return true;
   }
@@ -342,14 +355,25 @@ static bool tc_gemm_o(dreamer_handle *h, const dreamer::GemmArgs &a, const dream
     dreamer::tc::TcGemmArgs t{};
     CUtensorMap ta, tb;
     long mt;
+    const bool ew8 = a.K <= 1024;  // as for the QKV projection
     if (tc_pick_bn(h, a) == 256) {
       if (!tc_prepare<256, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
-      if (a.arow) tc_launch<256, 64, 4, true, 64>(h, t, ta, tb, mt, e, s);
-      else tc_launch<256, 64, 4, false, 64>(h, t, ta, tb, mt, e, s);
+      if (ew8) {
+        if (a.arow) tc_launch<256, 64, 3, true, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        else tc_launch<256, 64, 3, false, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
+      } else {
+        if (a.arow) tc_launch<256, 64, 4, true, 64>(h, t, ta, tb, mt, e, s);
+        else tc_launch<256, 64, 4, false, 64>(h, t, ta, tb, mt, e, s);
+      }
     } else {
       if (!tc_prepare<128, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
-      if (a.arow) tc_launch<128, 64, 6, true, 64>(h, t, ta, tb, mt, e, s);
-      else tc_launch<128, 64, 6, false, 64>(h, t, ta, tb, mt, e, s);
+      if (ew8) {
+        if (a.arow) tc_launch<128, 64, 5, true, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        else tc_launch<128, 64, 5, false, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
+      } else {
+        if (a.arow) tc_launch<128, 64, 6, true, 64>(h, t, ta, tb, mt, e, s);
+        else tc_launch<128, 64, 6, false, 64>(h, t, ta, tb, mt, e, s);
+      }
     }
     return true;
   }
