@@ -36,7 +36,9 @@ class DreamerConfig:
     cache_len: int = 0  # decode: past tokens per sequence
     rope_base: float = 10000.0
     rms_eps: float = 1e-6
-    variant: int = 0    # block layout: 0 DA||SA then EA (default), 1 serial, 2 fully parallel
+    variant: int = 0    # block layout: 0 DA||SA then EA (default), 1 serial, 2 fully parallel,
+                        # 3 without depth attention (the DR-without-DA comparison arm)
+    da_window: int = 0  # 0: DA over all earlier depths; W > 0: over the last W depths
 
     @property
     def tokens(self) -> int:

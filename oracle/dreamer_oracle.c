@@ -330,6 +330,15 @@ static const float *wsel(const float *base, int P, long per, int p) {
 }
 
 /* ------------------------------------------------------------------------------------ */
+/* First depth that depth attention at depth l reads: 0 (all earlier depths, R2), or the
+ * first of the last W depths with a sliding window (the pages' sparse-DA outlook); -1 when
+ * the layout has no depth attention (variant 3).                                        */
+static int da_first(const orc_cfg *c, int l) {
+  if (c->variant == 3) return -1;
+  if (c->da_window > 0 && l + 1 > c->da_window) return l + 1 - c->da_window;
+  return 0;
+}
+
 /* prefill forward                                                                       */
 
 static int forward_impl(const orc_cfg *c, const orc_weights *W, const float *x_in, int l0,
@@ -392,37 +401,40 @@ static int forward_impl(const orc_cfg *c, const orc_weights *W, const float *x_i
       }
     }
 
-    /* depth attention over depths 0..l of the same token (R2) */
+    /* depth attention over depths j0..l of the same token (R2; j0 > 0 with a window) */
+    const int j0 = da_first(c, l);
 #pragma omp parallel for schedule(dynamic, 4)
     for (long t = 0; t < T; t++) {
       double probs[1024];
       for (int hd = 0; hd < H; hd++) {
         const double *q = q_da + t * h + hd * d;
         double *o = a_da + t * h + hd * d;
-        if (!da_loops) {
+        if (j0 < 0) {  /* no depth attention */
+          for (int i = 0; i < d; i++) o[i] = 0.0;
+        } else if (!da_loops) {
           /* reshape view (notes, "Key design 1"; gist, "Methodology"): the b*s tokens are
            * the batch, the depth index is the sequence; the token's query sits at depth
            * position l and attends over its own depth sequence 0..l.                    */
-          const double *Kseq = da_kv + ((t * L) * 2 + 0) * h + hd * d;
-          const double *Vseq = da_kv + ((t * L) * 2 + 1) * h + hd * d;
-          orc_attend(q, Kseq, Vseq, l + 1, d, 2L * h, o, probs);
+          const double *Kseq = da_kv + ((t * L + j0) * 2 + 0) * h + hd * d;
+          const double *Vseq = da_kv + ((t * L + j0) * 2 + 1) * h + hd * d;
+          orc_attend(q, Kseq, Vseq, l + 1 - j0, d, 2L * h, o, probs);
         } else {
-          /* explicit loops over depths j = 0..l */
+          /* explicit loops over depths j = j0..l */
           double sc[1024], mx = -INFINITY, Z = 0.0;
-          for (int j = 0; j <= l; j++) {
+          for (int j = j0; j <= l; j++) {
             double s = 0.0;
             for (int i = 0; i < d; i++)
               s += q[i] * da_kv[((t * L + j) * 2 + 0) * h + hd * d + i];
             sc[j] = s / sqrt((double)d);
             if (sc[j] > mx) mx = sc[j];
           }
-          for (int j = 0; j <= l; j++) {
+          for (int j = j0; j <= l; j++) {
             sc[j] = exp(sc[j] - mx);
             Z += sc[j];
           }
           for (int i = 0; i < d; i++) {
             double acc = 0.0;
-            for (int j = 0; j <= l; j++)
+            for (int j = j0; j <= l; j++)
               acc += (sc[j] / Z) * da_kv[((t * L + j) * 2 + 1) * h + hd * d + i];
             o[i] = acc;
           }
@@ -599,11 +611,15 @@ int orc_step_tokens(const orc_cfg *c, const orc_weights *W, int l, const float *
       for (int i = 0; i < 2 * h; i++)
         dkv[(long)j * 2 * h + i] = da_hist[((long)s * L + j) * 2 * h + i];
     for (int i = 0; i < 2 * h; i++) dkv[(long)l * 2 * h + i] = qkvd[h + i];
+    const int j0 = da_first(c, l);
     for (int hd = 0; hd < H; hd++) {
       orc_attend(qs + hd * d, kv + hd * d, kv + h + hd * d, (int)t + 1, d, 2L * h,
                  cat + hd * d, probs);
-      orc_attend(qkvd + hd * d, dkv + hd * d, dkv + h + hd * d, l + 1, d, 2L * h,
-                 cat + h + hd * d, probs);
+      if (j0 < 0)
+        for (int i = 0; i < d; i++) cat[h + hd * d + i] = 0.0;
+      else
+        orc_attend(qkvd + hd * d, dkv + (long)j0 * 2 * h + hd * d, dkv + (long)j0 * 2 * h + h + hd * d,
+                   l + 1 - j0, d, 2L * h, cat + h + hd * d, probs);
     }
     const float *Wo = wsel(W->w_o, P, perO, pst[t]);
     proj(cat, 2 * h, Wo, P > 0 ? W->w_o_sh : NULL, h, 0, 0, h, sig[t], tmp);
@@ -680,9 +696,15 @@ int orc_decode_seq(const orc_cfg *c, const orc_weights *W, const float *x_new, d
       orc_depth_rope(qkv + 4 * h + hd * d, d, l, L, c->rope_base);
     }
     for (int i = 0; i < 2 * h; i++) dkv[(long)l * 2 * h + i] = qkv[4 * h + i];
-    for (int hd = 0; hd < H; hd++)
-      orc_attend(qkv + 3 * h + hd * d, dkv + hd * d, dkv + h + hd * d, l + 1, d, 2L * h,
-                 cat + h + hd * d, probs);
+    const int j0 = da_first(c, l);
+    for (int hd = 0; hd < H; hd++) {
+      if (j0 < 0)
+        for (int i = 0; i < d; i++) cat[h + hd * d + i] = 0.0;
+      else
+        orc_attend(qkv + 3 * h + hd * d, dkv + (long)j0 * 2 * h + hd * d,
+                   dkv + (long)j0 * 2 * h + h + hd * d, l + 1 - j0, d, 2L * h,
+                   cat + h + hd * d, probs);
+    }
     if (c->variant == 1) {
       proj(cat + h, h, Wo, Wos, h, h, 0, h, sg, tmp);
       for (int i = 0; i < h; i++) u[i] = xh[i] + tmp[i];

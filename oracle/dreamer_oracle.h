@@ -35,9 +35,12 @@ typedef struct {
   int E, k, m, dr; /* experts, top-k, expert hidden, router key dim                    */
   int P;           /* projection experts (0 = dense QKV/O)                            */
   double rope_base, eps;
-  int variant;     /* block layout: 0 DA||SA then EA; 1 serial DA->SA->EA; 2 all parallel */
+  int variant;     /* block layout: 0 DA||SA then EA; 1 serial DA->SA->EA; 2 all parallel;
+                      3 no depth attention (the DR-without-DA comparison arm) */
   int route_bf16;  /* 1: routing decisions read their input rounded to bf16, the precision
                       the bf16 kernels store it in (the decision itself stays float64)     */
+  int da_window;   /* 0: DA over depths 0..l; W > 0: over the last W depths max(0,l-W+1)..l
+                      (sliding-window depth attention)                                   */
 } orc_cfg;
 
 typedef struct {

@@ -26,7 +26,7 @@ i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
 class OrcCfg(C.Structure):
     _fields_ = [(n, C.c_int) for n in ("B", "S", "h", "H", "d", "L", "E", "k", "m", "dr", "P")] + \
                [("rope_base", C.c_double), ("eps", C.c_double), ("variant", C.c_int),
-                ("route_bf16", C.c_int)]
+                ("route_bf16", C.c_int), ("da_window", C.c_int)]
 
 
 _WNAMES = ("g", "w_qkv", "w_qkv_sh", "w_o", "w_o_sh", "w_qP", "k_P", "w_qE", "k_E", "bias",
@@ -94,7 +94,7 @@ class Oracle:
         self.c = OrcCfg(cfg.batch, cfg.seq, cfg.hidden, cfg.n_heads, cfg.head_dim, cfg.depth,
                         cfg.n_experts, cfg.top_k, cfg.expert_hidden, cfg.router_dim,
                         cfg.n_proj_experts, float(cfg.rope_base), float(cfg.rms_eps),
-                        int(cfg.variant), int(rb))
+                        int(cfg.variant), int(rb), int(getattr(cfg, "da_window", 0)))
         self._keep = {}
         ptrs = {}
         alias = {"w_qkv_sh": "w_qkv_shared", "w_o_sh": "w_o_shared"}

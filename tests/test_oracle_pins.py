@@ -459,3 +459,98 @@ def test_route_on_bf16_input_changes_only_near_ties():
     assert np.array_equal(a["y"], b["y"])                      # states are untouched
     same = np.all(np.sort(a["idx"][0], 1) == np.sort(b["idx"][0], 1), axis=1)
     assert np.all(same | (a["margin"][0] < 0.05))
+
+
+# ---------------------------------------------------------------------------------------
+# Sliding-window depth attention and the layout without DA (the pages' comparison arms and
+# sparse-DA outlook): window W reads depths max(0, l-W+1)..l; variant 3 has no DA at all.
+
+def test_window_covering_all_depths_is_full_da():
+    cfg = tiny_cfg(depth=4)
+    W = inputs.host_weights(cfg)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    full = O.Oracle(cfg, W, threads=2).forward(x0)
+    for win in (4, 9):
+        r = O.Oracle(cfg.with_(da_window=win), W, threads=2).forward(x0)
+        assert np.array_equal(r["x_out"], full["x_out"])
+    short = O.Oracle(cfg.with_(da_window=2), W, threads=2).forward(x0)
+    assert not np.allclose(short["x_out"], full["x_out"])  # depths 2, 3 lose history
+
+
+def test_window_one_returns_the_depths_own_value_closed_form():
+    # W = 1: softmax over one depth is 1, so DA = v_DA(x^_l) at every depth.  SA rows of
+    # W_O zero, DA rows identity, experts off: x_{l+1} = x^_l + x^_l W_v, iterated.
+    cfg = tiny_cfg(depth=3, n_experts=2, top_k=1, da_window=1)
+    W = rand_weights(cfg, seed=5)
+    h = cfg.hidden
+    W["w_o"] = np.zeros_like(W["w_o"])
+    W["w_o"][0, h:, :] = np.eye(h, dtype=np.float32)
+    W["w2"] = np.zeros_like(W["w2"])
+    x0 = inputs.host_inputs(cfg)["x0"]
+    r = O.Oracle(cfg, W, threads=1).forward(x0)
+    x = x0.astype(np.float64)
+    wv = W["w_qkv"][0][:, 5 * h:6 * h].astype(np.float64)
+    for _ in range(cfg.depth):
+        xh = x / np.sqrt(np.mean(x ** 2, 1, keepdims=True) + cfg.rms_eps)
+        x = xh + xh @ wv
+    assert np.allclose(r["x_out"], x, rtol=1e-12, atol=1e-12)
+
+
+def test_window_ignores_depths_before_it():
+    # one step at depth 3 with W = 2 reads the history rows of depths 2 (and its own 3)
+    cfg = tiny_cfg(batch=1, seq=6, depth=5, da_window=2)
+    W = rand_weights(cfg, seed=9)
+    x = inputs.extra_normal(cfg, 1101, (cfg.seq, cfg.hidden), 1.0, dtype="fp32")
+    hist = inputs.extra_normal(cfg, 1102, (2, cfg.depth, 2, cfg.hidden), 1.0, dtype="fp32")
+    hist = hist.astype(np.float64)
+    pos = np.array([1, 5], np.int32)
+    o = O.Oracle(cfg, W, threads=1)
+    base = o.step_tokens(3, x, hist, pos)["x_out"]
+    h2 = hist.copy()
+    h2[:, 0:2] += 3.0                                   # depths 0, 1: outside the window
+    assert np.array_equal(o.step_tokens(3, x, h2, pos)["x_out"], base)
+    h3 = hist.copy()
+    h3[:, 2] += 3.0                                     # depth 2: inside
+    assert not np.allclose(o.step_tokens(3, x, h3, pos)["x_out"], base)
+    full = O.Oracle(cfg.with_(da_window=0), W, threads=1)
+    assert not np.allclose(full.step_tokens(3, x, h2, pos)["x_out"],
+                           full.step_tokens(3, x, hist, pos)["x_out"])
+
+
+def test_window_reshape_equals_explicit_loops():
+    cfg = tiny_cfg(depth=4, da_window=2)
+    W = inputs.host_weights(cfg)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    o = O.Oracle(cfg, W, threads=2)
+    a, b = o.forward(x0), o.forward(x0, da_loops=True)
+    assert np.allclose(a["x_out"], b["x_out"], rtol=1e-12, atol=1e-12)
+
+
+def _zero_da_rows(cfg, W):
+    W2 = dict(W)
+    W2["w_o"] = W["w_o"].copy()
+    W2["w_o"][:, cfg.hidden:, :] = 0.0
+    return W2
+
+
+def test_no_da_layout_equals_zeroed_da_rows():
+    # without DA, y = x^ + SA W_O[SA rows]: the same as the default layout whose W_O rows
+    # for a_DA are zero (adding exact zeros), in forward, one-step and decode form
+    cfg = tiny_cfg(depth=3)
+    W = inputs.host_weights(cfg)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    nda = O.Oracle(cfg.with_(variant=3), W, threads=2)
+    ref = O.Oracle(cfg, _zero_da_rows(cfg, W), threads=2)
+    a, b = nda.forward(x0), ref.forward(x0)
+    assert np.array_equal(a["x_out"], b["x_out"]) and np.array_equal(a["idx"], b["idx"])
+    full = O.Oracle(cfg, W, threads=2).forward(x0)
+    assert not np.allclose(a["x_out"], full["x_out"])
+    dc = configs.TINY.with_(batch=1, seq=1, cache_len=8, depth=3)
+    Wd = inputs.host_weights(dc)
+    H, d = dc.n_heads, dc.head_dim
+    kc = RNG.standard_normal((dc.depth, H, 9, d))
+    vc = RNG.standard_normal((dc.depth, H, 9, d))
+    xn = inputs.host_inputs(dc)["x0"][0]
+    r1 = O.Oracle(dc.with_(variant=3), Wd, threads=1).decode_seq(xn, kc.copy(), vc.copy(), 5)
+    r2 = O.Oracle(dc, _zero_da_rows(dc, Wd), threads=1).decode_seq(xn, kc.copy(), vc.copy(), 5)
+    assert np.array_equal(r1["x_out"], r2["x_out"])
