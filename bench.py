@@ -67,19 +67,23 @@ def algorithmic(cfg, counts=None):
         f0, b0 = st.get(name, (0.0, 0.0))
         st[name] = (f0 + fl, b0 + by)
 
+    no_da = cfg.variant == 3
+    nq = 3 if no_da else 6                                        # projection widths / h
     for l in range(L):
         add("norm", 0.0, T * h * (es + es))                      # x in, x^ out
         if P > 0:
             add("proj_route", 2.0 * T * h * dr + 2.0 * T * P * dr, T * h * es)
-        add("qkv", 2.0 * T * h * 6 * h, T * h * es + G * 6 * h * h * es + T * 6 * h * es)
-        ctx = (l + 1)
-        add("da", 4.0 * T * h * ctx, T * h * es + T * 2 * h * es * l + T * h * es)
+        add("qkv", 2.0 * T * h * nq * h, T * h * es + G * nq * h * h * es + T * nq * h * es)
+        if not no_da:
+            ctx = l + 1 if cfg.da_window <= 0 else min(l + 1, cfg.da_window)
+            add("da", 4.0 * T * h * ctx, T * h * es + T * 2 * h * es * (ctx - 1) + T * h * es)
         if cfg.is_decode:
             n_ctx = cfg.cache_len + 1
             add("sa", 4.0 * T * h * n_ctx, 2.0 * T * h * es * n_ctx + 2 * T * h * es)
         else:
             add("sa", 4.0 * h * b * s * (s + 1) / 2, 4.0 * T * h * es)
-        add("o_proj", 2.0 * T * 2 * h * h, T * 2 * h * es + G * 2 * h * h * es + T * h * (es + 4))
+        ko = 1 if no_da else 2                                    # O contraction width / h
+        add("o_proj", 2.0 * T * ko * h * h, T * ko * h * es + G * ko * h * h * es + T * h * (es + 4))
         add("ea_route", 2.0 * T * h * dr + 2.0 * T * E * dr, T * h * es + h * dr * es + E * dr * es)
         touched = E
         if counts is not None:
@@ -352,6 +356,10 @@ def workload_name(cfg):
            f"L={cfg.depth} E={cfg.n_experts} k={cfg.top_k} m={cfg.expert_hidden} P={cfg.n_proj_experts}"
     if cfg.is_decode:
         base += f" decode cache={cfg.cache_len}"
+    if cfg.variant:
+        base += {1: " serial DA->SA->EA", 2: " fully parallel", 3: " without DA"}[cfg.variant]
+    if cfg.da_window:
+        base += f" DA window {cfg.da_window}"
     return base
 
 
@@ -426,7 +434,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="small", choices=["small", "medium", "large", "decode"])
+    ap.add_argument("--config", default="small", choices=sorted(configs.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     cfg = configs.CONFIGS[args.config]

@@ -82,4 +82,8 @@ LARGE = DreamerConfig("large", batch=2, seq=8192, hidden=2048, n_heads=16, head_
                       depth=64, n_experts=2048, top_k=8, expert_hidden=64, router_dim=128,
                       n_proj_experts=16, dtype="bf16", seed=4, bias_range=0.1)
 
-CONFIGS = {c.name: c for c in (TINY, SMALL, MEDIUM, DECODE, LARGE)}
+# the comparison arms and the sparse-DA outlook on the large shapes: DR without depth
+# attention (variant 3) and depth attention over the last 8 depths
+LARGE_NODA = LARGE.with_(name="large-noda", variant=3)
+LARGE_W8 = LARGE.with_(name="large-w8", da_window=8)
+CONFIGS = {c.name: c for c in (TINY, SMALL, MEDIUM, DECODE, LARGE, LARGE_NODA, LARGE_W8)}

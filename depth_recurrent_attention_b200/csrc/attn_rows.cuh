@@ -30,6 +30,7 @@ __device__ __forceinline__ void st16(float *p, const float *v) {
 struct RowsArgs {
   int mode;            // 0 depth attention, 2 decode attention (split)
   int n_q, H, h, L, l;
+  int r0;              // mode 0: first depth attended (0, or l-W+1 with a window of W)
   const void *q;       // [n_q][ldq], head at column head * D
   long ldq;
   const void *kv;      // mode 0: da_kv [T][L][2][h]; mode 2: k cache [L][B][H][cap][D]
@@ -59,7 +60,7 @@ __global__ void __launch_bounds__(256) attn_rows_kernel(RowsArgs a) {
   const T *Kb = reinterpret_cast<const T *>(a.kv) + ((long)qi * a.L * 2) * a.h + head * D;
   const T *Vb = Kb + a.h;
   const long ldk = 2L * a.h;
-  const int j0 = 0, j1 = a.l + 1;
+  const int j0 = a.r0, j1 = a.l + 1;
   float q[VEC];
   ld16(reinterpret_cast<const T *>(a.q) + (long)qi * a.ldq + head * D + c * VEC, q);
   const float sl2 = 1.4426950408889634f * rsqrtf((float)D);
@@ -205,6 +206,7 @@ __device__ __forceinline__ uint64_t gtimer() {
 
 struct DaBulkArgs {
   int n_tok, H, h, L, l, chunk;  // chunk: depths per shared-memory buffer
+  int r0;                        // first depth attended (0, or l-W+1 with a window of W)
   const void *q;                 // q_DA [T][h]
   const void *kv;                // [T][L][2][h]
   void *out;                     // attn [T][ldo], DA part at column col0
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
   __shared__ __align__(8) uint64_t bars[NB];
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nrow = a.l + 1;
+  const int nrow = a.l + 1 - a.r0;                     // depths r0..l
   const int nch = (nrow + a.chunk - 1) / a.chunk;
   const long row_el = 2L * a.h;                        // elements of one depth row (K then V)
   const uint32_t chunk_bytes = (uint32_t)(a.chunk * row_el * sizeof(T));
@@ -250,7 +252,8 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
                  "r"(total)
                  : "memory");
     tcda::bulk_load(tcda::smem_u32(kv_slot(b)),
-                    reinterpret_cast<const T *>(a.kv) + ((long)tok * a.L + r0) * row_el, kvb, bar);
+                    reinterpret_cast<const T *>(a.kv) + ((long)tok * a.L + a.r0 + r0) * row_el,
+                    kvb, bar);
     if (c == 0)
       tcda::bulk_load(tcda::smem_u32(q_slot(b)), reinterpret_cast<const T *>(a.q) + (long)tok * a.h,
                       q_bytes, bar);

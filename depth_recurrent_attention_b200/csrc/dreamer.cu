@@ -225,7 +225,7 @@ static int validate(const dreamer_config *c) {
   if (c->top_k < 1 || c->top_k > c->n_experts) return DREAMER_ERR_ARG;
   if (c->dtype != 0 && c->dtype != 1) return DREAMER_ERR_ARG;
   if (c->n_proj_experts < 0 || c->max_cache_len < 0) return DREAMER_ERR_ARG;
-  if (c->variant < 0 || c->variant > 2) return DREAMER_ERR_ARG;
+  if (c->variant < 0 || c->variant > 3 || c->da_window < 0) return DREAMER_ERR_ARG;
   if (!(c->rope_base > 0.f) || !(c->rms_eps >= 0.f)) return DREAMER_ERR_ARG;
   const int d = c->head_dim;
   if (d != 16 && d != 32 && d != 64 && d != 128) return DREAMER_ERR_UNSUPPORTED;
@@ -404,7 +404,7 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     DALLOC(h->y, T * hd * es);
     DALLOC(h->acc, T * hd * sizeof(float));
     DALLOC(h->inv_rms, T * sizeof(float));
-    DALLOC(h->da_kv_int, (size_t)T * L * 2 * hd * es);
+    if (c.variant != 3) DALLOC(h->da_kv_int, (size_t)T * L * 2 * hd * es);
     DALLOC(h->Hbuf, (Tk + 128) * m * es);
     DALLOC(h->qsplit, T * 3 * dr * 2);
     DALLOC(h->zbuf, (size_t)T * (h->ldz > h->ldzp ? h->ldz : h->ldzp) * sizeof(float));
@@ -538,11 +538,11 @@ static void launch_attn(const AttnArgs &a, int d, cudaStream_t s) {
 template <typename T>
 static void launch_da_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStream_t s) {
   DaBulkArgs a{};
-  a.n_tok = r.n_q; a.H = r.H; a.h = r.h; a.L = r.L; a.l = r.l;
+  a.n_tok = r.n_q; a.H = r.H; a.h = r.h; a.L = r.L; a.l = r.l; a.r0 = r.r0;
   const long row_bytes = 2L * r.h * sizeof(T);
   int chunk = (int)((48 * 1024) / row_bytes);
   if (chunk < 1) chunk = 1;
-  if (chunk > r.l + 1) chunk = r.l + 1;
+  if (chunk > r.l + 1 - r.r0) chunk = r.l + 1 - r.r0;
   a.chunk = chunk;
   a.q = r.q; a.kv = r.kv; a.out = r.out; a.ldo = r.ldo; a.col0 = r.col0; a.err = r.err;
   const int smem = (int)(2 * (chunk * row_bytes + r.h * (long)sizeof(T)));
@@ -754,6 +754,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
 
   RowsArgs da{};
   da.mode = 0; da.n_q = n; da.H = c.n_heads; da.h = hd; da.L = L; da.l = l;
+  da.r0 = (c.da_window > 0 && l + 1 > c.da_window) ? l + 1 - c.da_window : 0;
   da.q = h->q_da; da.ldq = hd; da.kv = io.da_kv;
   da.out = h->attn; da.ldo = 2 * hd; da.col0 = hd; da.err = h->err;
   RowsArgs sd{};  // decode: attention over the per-depth SA cache, split over key ranges
@@ -808,7 +809,14 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     gemm_simt<T, T, 16>(a, ptiles, eo, s);
   };
 
-  if (c.variant == 1) {
+  if (c.variant == 3) {
+    // without depth attention (the DR-without-DA arm): the SA columns of the projection
+    // only, y = x^ + SA W_O[SA rows]
+    qkv_gemm(h->xh, 0, 3 * hd);
+    mark(h, s, DREAMER_STAGE_SA);
+    run_sa(s);
+    o_gemm(h->attn, 0, hd, res_xhat, h->y);
+  } else if (c.variant == 1) {
     // serial DA -> SA -> EA: DA on x^, then SA on u = x^ + DA-part of O, then EA
     qkv_gemm(h->xh, 3 * hd, 3 * hd);
     mark(h, s, DREAMER_STAGE_DA);
@@ -1043,7 +1051,7 @@ extern "C" int dreamer_core_forward(dreamer_handle *h, const void *x_in, void *x
   if (!h || !x_in || !x_out) return DREAMER_ERR_ARG;
   const dreamer_config &c = h->cfg;
   if (depth_begin < 0 || depth_end > c.depth || depth_begin > depth_end) return DREAMER_ERR_ARG;
-  if (!da_kv && depth_begin != 0) return DREAMER_ERR_ARG;
+  if (!da_kv && depth_begin != 0 && c.variant != 3) return DREAMER_ERR_ARG;
   if (!aligned16(x_in) || !aligned16(x_out) || (da_kv && !aligned16(da_kv))) return DREAMER_ERR_ARG;
   int e = check_dev_error(h);
   if (e) return e;

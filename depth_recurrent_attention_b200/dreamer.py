@@ -32,7 +32,7 @@ class ConfigC(C.Structure):
         "batch", "seq", "hidden", "n_heads", "head_dim", "depth", "n_experts", "top_k",
         "expert_hidden", "router_dim", "n_proj_experts", "dtype")] + \
         [("rope_base", C.c_float), ("rms_eps", C.c_float), ("max_cache_len", C.c_int),
-         ("variant", C.c_int)]
+         ("variant", C.c_int), ("da_window", C.c_int)]
 
 
 WEIGHT_FIELDS = ("rms_gain", "w_qkv", "w_qkv_shared", "w_o", "w_o_shared", "w_qP", "k_P",
@@ -111,7 +111,8 @@ def config_c(cfg: DreamerConfig) -> ConfigC:
     return ConfigC(cfg.batch, cfg.seq, cfg.hidden, cfg.n_heads, cfg.head_dim, cfg.depth,
                    cfg.n_experts, cfg.top_k, cfg.expert_hidden, cfg.router_dim,
                    cfg.n_proj_experts, 0 if cfg.dtype == "fp32" else 1, cfg.rope_base,
-                   cfg.rms_eps, (cfg.cache_len + 1) if cfg.is_decode else 0, cfg.variant)
+                   cfg.rms_eps, (cfg.cache_len + 1) if cfg.is_decode else 0, cfg.variant,
+                   cfg.da_window)
 
 
 class Dreamer:
@@ -215,3 +216,38 @@ class Dreamer:
         return dict(launches=int(st.launches),
                     ms={n: float(st.ms[i]) for i, n in enumerate(STAGES)},
                     count={n: int(st.count[i]) for i, n in enumerate(STAGES)})
+
+
+class LayeredStack:
+    """The layered (LA) comparison arm: L distinct layers, each the Dreamer block without depth
+    attention (SA, then expert attention), layer l with its own weights.  Built from one
+    handle per layer (configuration `variant` 3); layer l runs depth l of its handle, so the
+    expert keys take the depth-RoPE of their layer index and each handle counts its own row
+    of the route histogram.  weights: a list of L device weight dicts."""
+
+    def __init__(self, cfg: DreamerConfig, weights: list, stream=None):
+        if cfg.variant != 3:
+            raise ValueError("the layered arm has no depth attention: use variant 3")
+        if len(weights) != cfg.depth:
+            raise ValueError("one weight set per layer")
+        self.cfg = cfg
+        self.layers = [Dreamer(cfg, w, stream=stream) for w in weights]
+        self._tmp = None
+
+    def forward(self, x_in, x_out=None, stream=None):
+        x = x_in
+        if self._tmp is None or self._tmp[0].shape != x_in.shape or self._tmp[0].dtype != x_in.dtype:
+            self._tmp = (torch.empty_like(x_in), torch.empty_like(x_in))
+        if x_out is None:
+            x_out = torch.empty_like(x_in)
+        L = self.cfg.depth
+        for l, layer in enumerate(self.layers):
+            dst = x_out if l == L - 1 else self._tmp[l % 2]
+            layer.forward(x, x_out=dst, depth_begin=l, depth_end=l + 1, stream=stream)
+            x = dst
+        return x_out
+
+    def close(self):
+        for layer in self.layers:
+            layer.close()
+        self.layers = []

@@ -65,7 +65,10 @@ typedef struct {
   float rms_eps;      /* 1e-6                                                             */
   int max_cache_len;  /* decode: SA cache capacity per sequence (0 = no decode)           */
   int variant;        /* block layout ([notes] ablation table): 0 DA||SA then EA (default),
-                         1 serial DA->SA->EA, 2 fully parallel DA+SA+EA                   */
+                         1 serial DA->SA->EA, 2 fully parallel DA+SA+EA, 3 without depth
+                         attention (the pages' DR-without-DA comparison arm: y = x^ + SA)  */
+  int da_window;      /* 0: DA at depth l over depths 0..l; W > 0: over the last W depths
+                         max(0, l-W+1)..l (sliding-window depth attention)                */
 } dreamer_config;
 
 typedef struct {

@@ -47,10 +47,12 @@ def trace_buffers(cfg, n_tok, with_sa=False):
 # ---------------------------------------------------------------------------------------
 # tiny, float32, free-running end to end
 
-@pytest.mark.parametrize("variant", [0, 1, 2])
-def test_tiny_forward_fp32(cuda, variant):
+@pytest.mark.parametrize("kw", [dict(variant=0), dict(variant=1), dict(variant=2),
+                                # without depth attention; sliding-window depth attention
+                                dict(variant=3), dict(da_window=2), dict(variant=1, da_window=1)])
+def test_tiny_forward_fp32(cuda, kw):
     torch = _torch()
-    cfg = configs.TINY.with_(variant=variant)
+    cfg = configs.TINY.with_(**kw)
     W = inputs.host_weights(cfg)
     x0 = inputs.host_inputs(cfg)["x0"]
     ref = O.Oracle(cfg, W).forward(x0)
@@ -234,7 +236,9 @@ def test_small_free_running_drift_reported(cuda):
                                 # head dim 128: q/k columns in the permuted GEMM order
                                 dict(n_experts=4, top_k=4, depth=3, n_heads=4, head_dim=128),
                                 dict(n_experts=8, top_k=8, depth=2, n_heads=4, head_dim=128,
-                                     n_proj_experts=1)])
+                                     n_proj_experts=1),
+                                dict(n_experts=4, top_k=4, depth=4, da_window=2),
+                                dict(n_experts=4, top_k=4, depth=3, variant=3)])
 def test_small_flip_free_all_depths_bf16(cuda, kw):
     torch = _torch()
     cfg = configs.SMALL.with_(**kw)
@@ -280,6 +284,8 @@ def flip_free(cfg):
     ("small", [300, 1, 77, 299], dict(n_experts=4, top_k=4, depth=4)),
     ("small", [40, 0, 17], dict(n_experts=4, top_k=4, depth=3, n_proj_experts=1)),
     ("small", [300, 1, 77, 299], dict(n_experts=4, top_k=4, depth=3, n_heads=4, head_dim=128)),
+    ("small", [300, 1, 77, 299], dict(n_experts=4, top_k=4, depth=4, da_window=2)),
+    ("tiny", [12, 5, 0], dict(variant=3)),
 ])
 def test_decode_step(cuda, base, lens, kw):
     torch = _torch()
@@ -386,3 +392,31 @@ def test_device_generator_matches_host(cuda):
         dev = t.float().view(-1)[:n].cpu().numpy()
         mism = int((host != dev).sum())
         assert mism <= max(1, n // 1_000_000), (spec.name, mism)
+
+
+# ---------------------------------------------------------------------------------------
+# the layered comparison arm: L distinct layers without depth attention
+
+@pytest.mark.parametrize("base,kw", [("tiny", {}), ("small", dict(n_experts=4, top_k=4, depth=3))])
+def test_layered_stack(cuda, base, kw):
+    torch = _torch()
+    from depth_recurrent_attention_b200.dreamer import LayeredStack
+    cfg = configs.CONFIGS[base].with_(variant=3, **kw)
+    Ws = [inputs.host_weights(cfg.with_(seed=cfg.seed + 100 * l)) for l in range(cfg.depth)]
+    x0 = inputs.host_inputs(cfg)["x0"]
+    stack = LayeredStack(cfg, [upload(cfg, W) for W in Ws])
+    out = stack.forward(inputs.to_device(x0, cfg.dtype))
+    torch.cuda.synchronize()
+    # the oracle layer by layer; the residual leaves each call rounded to dtype (R15)
+    x = x0
+    for l in range(cfg.depth):
+        r = O.Oracle(cfg, PY.deployed_weights(cfg, Ws[l])).forward(x, l, l + 1)
+        x = inputs.round_to(r["x_out"], cfg.dtype)
+        got = stack.layers[l].route_counts(on_host=True).numpy()[l]
+        assert np.array_equal(got, r["counts"][l])
+    bf = cfg.dtype == "bf16"
+    if bf:
+        PY.check_drift(PY.to_np(out), x, "layered x_L", gate_abs=False)
+    else:
+        PY.check_hidden(PY.to_np(out), x, False, "layered x_L")
+    stack.close()
