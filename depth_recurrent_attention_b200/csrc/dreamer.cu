@@ -1154,6 +1154,25 @@ extern "C" int dreamer_route_experts(dreamer_handle *h, int depth, const void *y
   return DREAMER_OK;
 }
 
+extern "C" int dreamer_route_balance(dreamer_handle *h, int depth, float *lorenz, float *gini,
+                                     dreamer_stream stream) {
+  if (!h || !gini) return DREAMER_ERR_ARG;
+  const int E = h->cfg.n_experts, L = h->cfg.depth;
+  if (depth >= L) return DREAMER_ERR_ARG;
+  if (E > 8192) return DREAMER_ERR_UNSUPPORTED;
+  int n2 = 1;
+  while (n2 < E) n2 <<= 1;
+  const size_t smem = (size_t)n2 * sizeof(int);
+  if (smem > 48 * 1024)
+    CK(cudaFuncSetAttribute(balance_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  cudaStream_t s = (cudaStream_t)stream;
+  pdl_break(h, s);
+  launch_k(h, balance_kernel, dim3(1), dim3(1024), smem, s, (const int *)h->counts, L, E, depth,
+           lorenz, gini);
+  CK(cudaGetLastError());
+  return DREAMER_OK;
+}
+
 extern "C" int dreamer_bias_update(dreamer_handle *h, float lambda, float *bias_out,
                                    dreamer_stream stream) {
   if (!h) return DREAMER_ERR_ARG;

@@ -1368,4 +1368,80 @@ __global__ void transpose_absorb_kernel(const T *src, const T *sh, T *dst, int r
   }
 }
 
+// =======================================================================================
+// Balance summary of the route counts (f2 of the bias balance): the Lorenz curve of the
+// per-expert totals N_e (sorted ascending, cumulative share at 0, 1/E, .., 1) and the Gini
+// coefficient from it, G = 1 - (1/E) sum_i (L_{i-1} + L_i).  N_e = counts[depth][e], or the
+// sum over depths for depth < 0.  One block; bitonic sort in shared memory; sums in double.
+// All-zero counts give the diagonal and G = 0.
+// =======================================================================================
+__global__ void __launch_bounds__(1024) balance_kernel(const int *counts, int L, int E,
+                                                       int depth, float *lorenz, float *gini) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ int srt[];  // [pow2 >= E]
+  __shared__ double part[1024];
+  const int tid = threadIdx.x;
+  int n2 = 1;
+  while (n2 < E) n2 <<= 1;
+  for (int e = tid; e < n2; e += blockDim.x) {
+    int v = 0x7fffffff;
+    if (e < E) {
+      if (depth >= 0) {
+        v = counts[(long)depth * E + e];
+      } else {
+        v = 0;
+        for (int l = 0; l < L; l++) v += counts[(long)l * E + e];
+      }
+    }
+    srt[e] = v;
+  }
+  __syncthreads();
+  for (int size = 2; size <= n2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < n2; i += blockDim.x) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool up = (i & size) == 0;
+          const int x = srt[i], y = srt[j];
+          if ((x > y) == up) {
+            srt[i] = y;
+            srt[j] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // prefix sums: thread tid owns sorted entries [i0, i0 + per)
+  const int per = (E + 1023) / 1024, i0 = tid * per;
+  double loc = 0.0;
+  for (int i = i0; i < i0 + per && i < E; i++) loc += (double)srt[i];
+  part[tid] = loc;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {
+    const double v = tid >= o ? part[tid - o] : 0.0;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
+  }
+  const double total = part[1023];
+  double acc = tid ? part[tid - 1] : 0.0, tsum = 0.0;
+  for (int i = i0; i < i0 + per && i < E; i++) {
+    const double prev = acc;
+    acc += (double)srt[i];
+    if (lorenz) lorenz[i + 1] = total > 0.0 ? (float)(acc / total) : (float)(i + 1) / (float)E;
+    tsum += prev + acc;
+  }
+  if (tid == 0 && lorenz) lorenz[0] = 0.f;
+  __syncthreads();
+  part[tid] = tsum;
+  __syncthreads();
+  for (int o = 512; o > 0; o >>= 1) {
+    if (tid < o) part[tid] += part[tid + o];
+    __syncthreads();
+  }
+  if (tid == 0) *gini = total > 0.0 ? (float)(1.0 - part[0] / ((double)E * total)) : 0.f;
+}
+
 }  // namespace dreamer

@@ -74,6 +74,7 @@ def lib():
         L.dreamer_route_counts.argtypes = [vp, vp, i, vp]
         L.dreamer_route_experts.argtypes = [vp, i, vp, i, vp, vp, vp, vp]
         L.dreamer_bias_update.argtypes = [vp, C.c_float, vp, vp]
+        L.dreamer_route_balance.argtypes = [vp, i, vp, vp, vp]
         L.dreamer_set_profiling.argtypes = [vp, i]
         L.dreamer_get_stats.argtypes = [vp, C.POINTER(StatsC), i]
         L.dreamer_destroy.argtypes = [vp]
@@ -177,6 +178,15 @@ class Dreamer:
                                          C.byref(tr) if tr is not None else None,
                                          _stream(stream)), "dreamer_decode_step")
         return x_out
+
+    def route_balance(self, depth: int = -1, stream=None):
+        """(Gini coefficient, Lorenz curve [E+1]) of the last call's route counts (depth < 0:
+        summed over depths), as device tensors."""
+        lor = torch.empty(self.cfg.n_experts + 1, dtype=torch.float32, device="cuda")
+        g = torch.empty(1, dtype=torch.float32, device="cuda")
+        _check(lib().dreamer_route_balance(self.h, int(depth), _ptr(lor), _ptr(g),
+                                           _stream(stream)), "dreamer_route_balance")
+        return g, lor
 
     def route_counts(self, on_host: bool = True, stream=None):
         cfg = self.cfg

@@ -186,6 +186,15 @@ int dreamer_route_experts_noalloc(const dreamer_config *cfg, int depth, const vo
 int dreamer_bias_update(dreamer_handle *h, float lambda, float *bias_out,
                         dreamer_stream stream);
 
+/* Balance summary of the expert route counts N of the last call ([notes] "Key design 2":
+ * the bias keeps expert use balanced; this measures how balanced): N_e = counts of depth
+ * `depth`, or summed over depths for depth < 0.  Writes the Lorenz curve of N (sorted
+ * ascending, cumulative share at e/E for e = 0..E; [E+1] float32, device, may be NULL) and
+ * the Gini coefficient G = 1 - (1/E) sum_e (L_{e-1} + L_e) ([1] float32, device).  E up to
+ * 8192 (DREAMER_ERR_UNSUPPORTED beyond).  Asynchronous on `stream`.                        */
+int dreamer_route_balance(dreamer_handle *h, int depth, float *lorenz, float *gini,
+                          dreamer_stream stream);
+
 /* Instrumentation.  Stages of the depth step, in launch order: */
 enum {
   DREAMER_STAGE_NORM = 0,     /* RMSNorm of the residual stream                          */

@@ -268,3 +268,18 @@ def bias_update(counts, lam, bias):
     b = np.array(bias, np.float64)
     lib().orc_bias_update(L, E, counts, float(lam), b)
     return b
+
+
+def gini_lorenz(counts):
+    """Balance of expert use (papernotes "Key design 2": the bias keeps experts balanced):
+    Lorenz curve of the per-expert counts (sorted ascending, cumulative share at e/E for
+    e = 0..E) and the Gini coefficient by its definition, the mean absolute difference over
+    all pairs divided by twice the mean.  All-zero counts: the diagonal and 0."""
+    x = np.sort(np.asarray(counts, np.float64).ravel())
+    E = x.size
+    tot = x.sum()
+    if tot <= 0:
+        return 0.0, np.arange(E + 1) / E
+    lorenz = np.concatenate([[0.0], np.cumsum(x) / tot])
+    g = np.abs(x[:, None] - x[None, :]).sum() / (2.0 * E * E * (tot / E))
+    return float(g), lorenz

@@ -420,3 +420,27 @@ def test_layered_stack(cuda, base, kw):
     else:
         PY.check_hidden(PY.to_np(out), x, False, "layered x_L")
     stack.close()
+
+
+# ---------------------------------------------------------------------------------------
+# balance summary of the route counts (Gini, Lorenz) against the oracle's definition
+
+def test_route_balance(cuda):
+    torch = _torch()
+    cfg = configs.SMALL.with_(depth=2)
+    W = inputs.host_weights(cfg)
+    dev = make_handle(cfg, W)
+    g0, lor0 = dev.route_balance(-1)                  # no call yet: all-zero counts
+    torch.cuda.synchronize()
+    assert g0.item() == 0.0
+    assert np.allclose(lor0.cpu().numpy(), np.arange(cfg.n_experts + 1) / cfg.n_experts)
+    dev.forward(inputs.to_device(inputs.host_inputs(cfg)["x0"], cfg.dtype))
+    counts = dev.route_counts(on_host=True).numpy()
+    for depth in (-1, 0, 1):
+        g, lor = dev.route_balance(depth)
+        torch.cuda.synchronize()
+        n = counts.sum(0) if depth < 0 else counts[depth]
+        gr, lr = O.gini_lorenz(n)
+        assert abs(g.item() - gr) < 1e-5, (depth, g.item(), gr)
+        assert np.allclose(lor.cpu().numpy(), lr, atol=1e-6)
+    dev.close()

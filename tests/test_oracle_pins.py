@@ -554,3 +554,30 @@ def test_no_da_layout_equals_zeroed_da_rows():
     r1 = O.Oracle(dc.with_(variant=3), Wd, threads=1).decode_seq(xn, kc.copy(), vc.copy(), 5)
     r2 = O.Oracle(dc, _zero_da_rows(dc, Wd), threads=1).decode_seq(xn, kc.copy(), vc.copy(), 5)
     assert np.array_equal(r1["x_out"], r2["x_out"])
+
+
+# ---------------------------------------------------------------------------------------
+# Balance summary of the route counts (f2): Gini and Lorenz
+
+def test_gini_lorenz_closed_forms():
+    g, lor = O.gini_lorenz(np.full(16, 7))
+    assert g == 0.0 and np.allclose(lor, np.arange(17) / 16)        # perfect equality
+    one = np.zeros(16)
+    one[5] = 40
+    g, lor = O.gini_lorenz(one)
+    assert g == pytest.approx(1 - 1 / 16) and lor[15] == 0 and lor[16] == 1   # one expert
+    g, lor = O.gini_lorenz([1, 3])                                   # |1-3|*2 / (2*4*2)
+    assert g == pytest.approx(0.25) and np.allclose(lor, [0, 0.25, 1])
+    g, _ = O.gini_lorenz(np.zeros(8))
+    assert g == 0.0
+
+
+def test_gini_equals_one_minus_twice_lorenz_area():
+    # the pairwise definition and the area under the Lorenz curve agree (trapezoid rule on
+    # the piecewise-linear curve is exact)
+    for n in (5, 64, 300):
+        x = RNG.integers(0, 50, n)
+        g, lor = O.gini_lorenz(x)
+        area = np.sum((lor[1:] + lor[:-1]) / 2) / n
+        assert g == pytest.approx(1 - 2 * area, abs=1e-12)
+        assert np.all(np.diff(lor) >= 0) and np.all(np.diff(lor, 2) >= -1e-15)  # convex
