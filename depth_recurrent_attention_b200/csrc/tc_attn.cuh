@@ -298,17 +298,25 @@ __global__ void __launch_bounds__(384, 1)
         // pass 2: P = 2^(s * scale - m) as bf16, K-major SW128 (key chunk kc at kc * TILE,
         // 16-byte unit u of the row at ((u ^ (row & 7)) << 4))
         const float nm = -m_new;
-        const int lim = diag ? qi - j * 128 : 127;
+        const int lim = qi - j * 128;  // diagonal block: last visible key of the row
         float rs = 0.f;
 #pragma unroll
         for (int c = 0; c < 128; c += 32) {
           float sv[32];
           tmem_ld32(sbuf + c, sv);
+          if (!diag) {  // every key visible: no mask in the hot loop
 #pragma unroll
-          for (int i = 0; i < 32; i++) {
-            const float p = ex2(fmaf(sv[i], a.scale_log2, nm));
-            sv[i] = (c + i <= lim) ? p : 0.f;
-            rs += sv[i];
+            for (int i = 0; i < 32; i++) {
+              sv[i] = ex2(fmaf(sv[i], a.scale_log2, nm));
+              rs += sv[i];
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; i++) {
+              const float p = ex2(fmaf(sv[i], a.scale_log2, nm));
+              sv[i] = (c + i <= lim) ? p : 0.f;
+              rs += sv[i];
+            }
           }
           const int kc = c >> 6;
 #pragma unroll
