@@ -103,14 +103,23 @@ struct EpiTopK {
     // candidates against the current k-th entry first (straight-line), then one insertion
     // per qualifying candidate, picked out of the registers by a select chain (a dynamically
     // indexed array would live in local memory) and placed by an unrolled compare-and-swap
+    // A row's columns arrive in increasing order, so once the list is full a candidate can
+    // only tie entry KT-1 with a larger index and lose: "v > v[KT-1]" is the exact test then.
     float vb[SEG];
     unsigned mask = 0;
+    const float tv = s.v[KT - 1];
+    const bool open = s.e[KT - 1] == 0x7fffffff;  // the list is not full yet
+    const float4 *b4 = reinterpret_cast<const float4 *>(bias + n0);
 #pragma unroll
-    for (int i = 0; i < SEG; i++) {
-      float v = vals[i] * zscale + bias[n0 + i];
-      if (v != v) v = -INFINITY;
-      vb[i] = v;
-      if (better(v, n0 + i, s.v[KT - 1], s.e[KT - 1])) mask |= 1u << i;
+    for (int i = 0; i < SEG; i += 4) {
+      const float4 bq = b4[i / 4];
+      const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+      for (int u = 0; u < 4; u++) {
+        const float v = fmaxf(fmaf(vals[i + u], zscale, bb[u]), -INFINITY);  // NaN ranks last
+        vb[i + u] = v;
+        if (open || v > tv) mask |= 1u << (i + u);
+      }
     }
     while (mask) {
       const int i = __ffs(mask) - 1;
