@@ -164,6 +164,16 @@ class ClockSampler:
 # ----------------------------------------------------------------------------------------
 # our arm
 
+def measured_traffic(workload: str, stage: str):
+    """DRAM bytes (read + write) per launch of the stage's kernel from the committed ncu
+    summary (profiles/dram_traffic.json), or None where none was taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            return json.load(f).get(workload, {}).get(stage)
+    except Exception:
+        return None
+
+
 # ----------------------------------------------------------------------------------------
 # multi-rank host logic (one replica per GPU; tested on CPU with gloo ranks)
 
@@ -278,7 +288,8 @@ def run_ours(args, cfg, rank, world, torch, dist):
         achieved = by / t_dom / 1e9
         roof = dict(bound="hbm", achieved=achieved, peak=pk["hbm"], unit="GB/s",
                     frac=achieved / pk["hbm"])
-    roof.update(kernel=dominant, launches_per_step=launches_per_fwd, traffic=None,
+    roof.update(kernel=dominant, launches_per_step=launches_per_fwd,
+                traffic=measured_traffic(cfg.name, dominant),
                 peak_source=pk["source"] + " (MEASURED_PEAKS.json burst figure)")
 
     # ---- end to end through the public API with host buffers
