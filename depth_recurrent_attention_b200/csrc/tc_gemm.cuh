@@ -67,14 +67,18 @@ template <class E> struct EpiStaged<E, std::void_t<decltype(E::STAGED)>> {
   static constexpr bool value = E::STAGED;
 };
 
-template <int BN, int BK, int STAGES, bool GATHER, bool STAGED = false, int EW_ = 4>
+template <int BN, int BK, int STAGES, bool GATHER, bool STAGED = false, int EW_ = 4,
+          bool ROWPASS = false>
 struct TcGemmCfg {
   static constexpr int A_BYTES = 128 * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int EW = STAGED ? EW_ : 4;  // epilogue warps: 4, or 8 (two per TMEM lane quarter)
+  static constexpr int EW = EW_;  // epilogue warps: 4, or 8 (two per TMEM lane quarter)
   static_assert(EW == 4 || EW == 8, "epilogue warps");
   static constexpr int THREADS = 64 + 32 * EW + (GATHER ? 64 : 0);
-  static constexpr int STG_BYTES = STAGED ? EW * 32 * 64 * 4 : 0;  // EW warps x 32 x 64 fp32
+  // staged epilogues: EW warps x 32 rows x 64 fp32; row-pass epilogues with two warps a lane
+  // quarter: one exchange list of up to 16 (value, raw score, index) a row
+  static constexpr int STG_BYTES =
+      STAGED ? EW * 32 * 64 * 4 : ((ROWPASS && EW == 8) ? 128 * 16 * 12 : 0);
   // at least 120 KB so that a second CTA never shares the SM (and its 512 TMEM columns)
   static constexpr int SMEM_USED =
       STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*bars*/ + STG_BYTES;
@@ -92,18 +96,19 @@ struct TcGemmCfg {
 template <int BN, int BK, int STAGES, bool GATHER, int SEG, class Epi, bool ROWPASS = false,
           int EW = 4>
 __global__ void __launch_bounds__(
-    TcGemmCfg<BN, BK, STAGES, GATHER, EpiStaged<Epi>::value && !ROWPASS, EW>::THREADS, 1)
+    TcGemmCfg<BN, BK, STAGES, GATHER, EpiStaged<Epi>::value && !ROWPASS, EW, ROWPASS>::THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    TcGemmArgs a, Epi epi) {
   constexpr bool STAGED = EpiStaged<Epi>::value && !ROWPASS;
-  using C = TcGemmCfg<BN, BK, STAGES, GATHER, STAGED, EW>;
+  using C = TcGemmCfg<BN, BK, STAGES, GATHER, STAGED, EW, ROWPASS>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
   uint8_t *sB = smem + STAGES * C::A_BYTES;
   uint64_t *bars = reinterpret_cast<uint64_t *>(sB + STAGES * C::B_BYTES);
   uint64_t *full = bars, *empty = bars + STAGES, *tfull = bars + 2 * STAGES, *tempty = tfull + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  uint64_t *xfull = tempty + 2, *xempty = xfull + 4;  // row-pass list exchange, per lane quarter
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xempty + 4);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   float *stage_buf = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + 256);
 
@@ -132,6 +137,10 @@ __global__ void __launch_bounds__(
     for (int i = 0; i < 2; i++) {
       mbar_init(smem_u32(&tfull[i]), 1);
       mbar_init(smem_u32(&tempty[i]), 32 * C::EW);
+    }
+    for (int i = 0; i < 4; i++) {
+      mbar_init(smem_u32(&xfull[i]), 32);
+      mbar_init(smem_u32(&xempty[i]), 32);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -216,10 +225,11 @@ __global__ void __launch_bounds__(
   } else if (warp < 2 + C::EW) {
     // ------------------------------------------------------------- epilogue
     const int q = warp & 3;                 // TMEM lane quarter of this warp
-    const int half = (warp - 2) >> 2;       // which of the quarter's warps (staged: 0 or 1)
+    const int half = (warp - 2) >> 2;       // which of the quarter's warps (0, or 1 with 8)
     const int row = q * 32 + lane;
     int mt, nt;
     typename EpiState<Epi, ROWPASS>::type st;
+    int rb = 0;  // row blocks finished (row-pass exchange phase)
     for (int it = 0; tile_at(it, mt, nt); it++) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
@@ -297,8 +307,9 @@ __global__ void __launch_bounds__(
         if constexpr (ROWPASS) {
           if (nt == 0) epi.row_begin(st);
         }
+        // segments of SEG columns; with eight epilogue warps segment sg belongs to half sg % 2
 #pragma unroll 1
-        for (int sg = 0; sg < BN / SEG && m0 + q * 32 < m1; sg++) {  // skip warps with no rows
+        for (int sg = half; sg < BN / SEG && m0 + q * 32 < m1; sg += C::EW / 4) {  // skip warps with no rows
           float v[SEG];
           if (SEG >= 32) {
 #pragma unroll
@@ -315,7 +326,18 @@ __global__ void __launch_bounds__(
       tc_fence_before();
       mbar_arrive(smem_u32(&tempty[acc]));
       if constexpr (ROWPASS) {
-        if (nt == NT - 1 && valid) epi.row_end(st, r, token);
+        if (nt == NT - 1) {
+          if constexpr (C::EW == 8) {
+            // the quarter's two warps hold lists over alternate segments: half 1 hands its
+            // list over, half 0 merges and finishes the row
+            epi.row_end_pair(st, r, token, valid, half, q * 32 + lane,
+                             reinterpret_cast<uint8_t *>(stage_buf), xfull + q, xempty + q, rb,
+                             abort_flag, a.err);
+            rb++;
+          } else if (valid) {
+            epi.row_end(st, r, token);
+          }
+        }
       }
     }
   } else if (GATHER) {

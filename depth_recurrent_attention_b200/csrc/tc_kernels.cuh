@@ -144,6 +144,47 @@ struct EpiTopK {
       }
     }
   }
+  // Two warps a lane quarter: half 1 writes its list for row slot `slot` (0..127) into xb
+  // and arrives on xfull; half 0 waits for it (bounded), inserts it into its own list (sorted,
+  // so the first entry that does not qualify ends the merge), frees the slot through xempty
+  // and writes the row.  rb: row blocks this pair finished before.
+  __device__ __forceinline__ void row_end_pair(State &s, int r, int token, bool valid, int half,
+                                               int slot, uint8_t *xb, uint64_t *xfull,
+                                               uint64_t *xempty, int rb, volatile int *abort_flag,
+                                               int *err) const {
+    float *xv = reinterpret_cast<float *>(xb) + slot * KT;
+    float *xz = reinterpret_cast<float *>(xb) + 128 * KT + slot * KT;
+    int *xe = reinterpret_cast<int *>(reinterpret_cast<float *>(xb) + 256 * KT) + slot * KT;
+    if (half == 1) {
+      if (rb > 0 && !tc::mbar_wait(tc::smem_u32(xempty), (rb - 1) & 1, abort_flag, err)) return;
+#pragma unroll
+      for (int i = 0; i < KT; i++) {
+        xv[i] = s.v[i];
+        xz[i] = s.z[i];
+        xe[i] = s.e[i];
+      }
+      tc::mbar_arrive(tc::smem_u32(xfull));
+      return;
+    }
+    if (!tc::mbar_wait(tc::smem_u32(xfull), rb & 1, abort_flag, err)) return;
+#pragma unroll 1
+    for (int i = 0; i < KT; i++) {
+      float cv = xv[i], cz = xz[i];
+      int ce = xe[i];
+      if (!better(cv, ce, s.v[KT - 1], s.e[KT - 1])) break;
+#pragma unroll
+      for (int j = 0; j < KT; j++) {
+        if (better(cv, ce, s.v[j], s.e[j])) {
+          const float tv = s.v[j], tz = s.z[j];
+          const int te = s.e[j];
+          s.v[j] = cv; s.z[j] = cz; s.e[j] = ce;
+          cv = tv; cz = tz; ce = te;
+        }
+      }
+    }
+    tc::mbar_arrive(tc::smem_u32(xempty));
+    if (valid) row_end(s, r, token);
+  }
   __device__ __forceinline__ void row_end(State &s, int r, int token) const {
     float sg[KT], sum = 0.f;
 #pragma unroll
@@ -263,7 +304,7 @@ template <int BN, int BK, int ST, bool GATHER, int SEG, class Epi, bool ROWPASS 
 static void tc_launch(dreamer_handle *h, const dreamer::tc::TcGemmArgs &a, const CUtensorMap &ta,
                       const CUtensorMap &tb, long max_tiles, const Epi &epi, cudaStream_t s) {
   using Cfg = dreamer::tc::TcGemmCfg<BN, BK, ST, GATHER,
-                                     dreamer::tc::EpiStaged<Epi>::value && !ROWPASS, EW>;
+                                     dreamer::tc::EpiStaged<Epi>::value && !ROWPASS, EW, ROWPASS>;
   auto kern = dreamer::tc::tc_gemm_kernel<BN, BK, ST, GATHER, SEG, Epi, ROWPASS, EW>;
   if (ROWPASS) max_tiles /= (a.N / BN);  // one unit of work per row tile
   static bool attr_set = false;
@@ -427,11 +468,11 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
   const int k_fused = (n + 127) / 128 >= h->num_sms / 2 ? c.top_k : 0;
   switch (k_fused) {  // top-k fused into the score GEMM
     case 4:
-      tc_launch<256, 64, 4, false, 32, EpiTopK<4>, true>(
+      tc_launch<256, 64, 4, false, 32, EpiTopK<4>, true, 8>(
           h, t2, ta2, tb2, mt2, EpiTopK<4>{E, zs, h->bias, idx, w, counts_a, counts_b}, s);
       return true;
     case 8:
-      tc_launch<256, 64, 4, false, 32, EpiTopK<8>, true>(
+      tc_launch<256, 64, 4, false, 32, EpiTopK<8>, true, 8>(
           h, t2, ta2, tb2, mt2, EpiTopK<8>{E, zs, h->bias, idx, w, counts_a, counts_b}, s);
       return true;
     case 16:
