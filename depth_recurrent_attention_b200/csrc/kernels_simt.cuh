@@ -985,10 +985,10 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
 
 // Scores and top-k from a stored router query, one warp per token: q arrives as the three
 // bf16 parts q_hi + q_mid + q_lo of R_l^T q (the split the tensor-core query GEMM writes), the
-// keys unrotated and transposed [d_r][E]; lane j scores experts b + 2j and b + 2j + 1 of each
-// batch of 64 (one 128-byte row read a key dimension, shared through L1 by the block's warps),
-// z_e = q . k_e in fp32, then the warp top-k.  For batches too short to fill the GPU with
-// fused score tiles.  E even.
+// keys unrotated and transposed [d_r][E]; lane j scores experts b + 4j .. b + 4j + 3 of each
+// batch of 128 (one 256-byte row read a key dimension, shared through L1 by the block's warps;
+// four independent sums a lane), z_e = q . k_e in fp32, then the warp top-k.  For batches too
+// short to fill the GPU with fused score tiles.  E a multiple of 4.
 template <int DR>
 __global__ void __launch_bounds__(256) route_q_topk_kernel(const bf16 *qs3, const bf16 *kt,
                                                            TopkArgs a) {
@@ -1009,20 +1009,23 @@ __global__ void __launch_bounds__(256) route_q_topk_kernel(const bf16 *qs3, cons
     for (int u = 0; u < 8; u++) q[j + u] = (hi[u] + mid[u]) + lo[u];
   }
   WarpTopK t(a.k, lane);
-  for (int b = 0; b < a.E; b += 64) {
-    const int e = b + 2 * lane;
-    float z0 = 0.f, z1 = 0.f;
+  for (int b = 0; b < a.E; b += 128) {
+    const int e = b + 4 * lane;
+    float z[4] = {0.f, 0.f, 0.f, 0.f};
     if (e < a.E) {
 #pragma unroll
       for (int j = 0; j < DR; j++) {
-        const float2 f =
-            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(kt + (long)j * a.E + e));
-        z0 = fmaf(q[j], f.x, z0);
-        z1 = fmaf(q[j], f.y, z1);
+        const uint2 u = *reinterpret_cast<const uint2 *>(kt + (long)j * a.E + e);
+        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+        const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+        z[0] = fmaf(q[j], f0.x, z[0]);
+        z[1] = fmaf(q[j], f0.y, z[1]);
+        z[2] = fmaf(q[j], f1.x, z[2]);
+        z[3] = fmaf(q[j], f1.y, z[3]);
       }
     }
-    t.offer_score(z0 * a.zscale, e, e < a.E, a.bias);
-    t.offer_score(z1 * a.zscale, e + 1, e + 1 < a.E, a.bias);
+#pragma unroll
+    for (int u = 0; u < 4; u++) t.offer_score(z[u] * a.zscale, e + u, e + u < a.E, a.bias);
   }
   emit_topk(lane, a.k, t.lv, t.le, t.lz, tok, a.mode, a.idx, a.w, a.counts_a, a.counts_b);
 }
@@ -1197,8 +1200,8 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int *cnt, int G, co
   pdl_wait();
   pdl_trigger();
   extern __shared__ int so[];  // [G + 1]
-  __shared__ int s0[1024], s1[1024], s2[1024];
-  const int tid = threadIdx.x;
+  __shared__ int w0[32], w1[32], w2[32];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const bool pub = blockIdx.x == 0;
   const int per = (G + 1023) / 1024;
   int a0 = 0, a1 = 0, a2 = 0;
@@ -1211,21 +1214,44 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int *cnt, int G, co
       a2 += (c + bm_b - 1) / bm_b;
     }
   }
-  s0[tid] = a0;
-  s1[tid] = a1;
-  s2[tid] = a2;
-  __syncthreads();
-  for (int o = 1; o < 1024; o <<= 1) {
-    const int v0 = tid >= o ? s0[tid - o] : 0;
-    const int v1 = tid >= o ? s1[tid - o] : 0;
-    const int v2 = tid >= o ? s2[tid - o] : 0;
-    __syncthreads();
-    s0[tid] += v0;
-    s1[tid] += v1;
-    s2[tid] += v2;
-    __syncthreads();
+  // exclusive prefix of the three per-thread sums: warp shuffles, then the warp totals
+  int i0 = a0, i1 = a1, i2 = a2;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v0 = __shfl_up_sync(0xffffffffu, i0, o), v1 = __shfl_up_sync(0xffffffffu, i1, o);
+    const int v2 = __shfl_up_sync(0xffffffffu, i2, o);
+    if (lane >= o) {
+      i0 += v0;
+      i1 += v1;
+      i2 += v2;
+    }
   }
-  int b0 = tid ? s0[tid - 1] : 0, b1 = tid ? s1[tid - 1] : 0, b2 = tid ? s2[tid - 1] : 0;
+  if (lane == 31) {
+    w0[wid] = i0;
+    w1[wid] = i1;
+    w2[wid] = i2;
+  }
+  __syncthreads();
+  if (wid == 0) {
+    int t0 = w0[lane], t1 = w1[lane], t2 = w2[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v0 = __shfl_up_sync(0xffffffffu, t0, o), v1 = __shfl_up_sync(0xffffffffu, t1, o);
+      const int v2 = __shfl_up_sync(0xffffffffu, t2, o);
+      if (lane >= o) {
+        t0 += v0;
+        t1 += v1;
+        t2 += v2;
+      }
+    }
+    w0[lane] = t0;  // inclusive prefix of the warp totals
+    w1[lane] = t1;
+    w2[lane] = t2;
+  }
+  __syncthreads();
+  int b0 = i0 - a0 + (wid ? w0[wid - 1] : 0);
+  int b1 = i1 - a1 + (wid ? w1[wid - 1] : 0);
+  int b2 = i2 - a2 + (wid ? w2[wid - 1] : 0);
   for (int i = 0; i < per; i++) {
     const int g = tid * per + i;
     if (g < G) {
@@ -1242,9 +1268,9 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int *cnt, int G, co
     }
   }
   if (tid == 1023 && pub) {
-    offs[G] = s0[1023];
-    tiles_a[G] = s1[1023];
-    if (tiles_b) tiles_b[G] = s2[1023];
+    offs[G] = w0[31];
+    tiles_a[G] = w1[31];
+    if (tiles_b) tiles_b[G] = w2[31];
   }
   __syncthreads();
   const int i = blockIdx.x * 1024 + tid;

@@ -349,16 +349,19 @@ static bool tc_gemm_ok(dreamer_handle *h, const dreamer::GemmArgs &a) {
   return a.N % 256 == 0 && a.K % 64 == 0 && (d == 64 || d == 128);
 }
 
-// N tile of the projection GEMMs: the wider tile reads A fewer times, the narrower one
-// spreads a small problem over more SMs; take the one with the shorter critical path
-// (waves of tiles x tile width plus a fixed per-tile cost of about 32 columns).
+// N tile of the projection GEMMs (64, 128 or 256): the wider tile reads A fewer times, the
+// narrower one spreads a small problem over more SMs; take the one with the shorter critical
+// path (waves of tiles x tile width plus a fixed per-tile cost of about 32 columns).
 static int tc_pick_bn(dreamer_handle *h, const dreamer::GemmArgs &a) {
   const long mt = (a.M + 127) / 128 + (a.goffs ? a.G : 0);
   auto cost = [&](int bn) {
     const long tiles = mt * (a.N / bn);
     return ((tiles + h->num_sms - 1) / h->num_sms) * (bn + 32);
   };
-  return (a.N % 256 == 0 && cost(256) <= cost(128)) ? 256 : 128;
+  int best = 128;
+  if (a.N % 256 == 0 && cost(256) <= cost(best)) best = 256;
+  if (cost(64) < cost(best)) best = 64;  // few tiles: narrower ones reach more SMs
+  return best;
 }
 
 template <typename T>
@@ -374,7 +377,12 @@ static bool tc_gemm_qkv(dreamer_handle *h, const dreamer::GemmArgs &a, const dre
     // or 128 in perm order).  Short K leaves little MMA time per tile to hide the epilogue
     // behind: eight epilogue warps then, at one stage less of operand ring.
     const bool ew8 = a.K <= 1024;
-    if (tc_pick_bn(h, a) == 256) {
+    const int bn = tc_pick_bn(h, a);
+    if (bn == 64) {  // one 64-column pass a tile: four epilogue warps, eight stages
+      if (!tc_prepare<64, 64>(h, a, tiles, a.M, t, ta, tb, mt)) return false;
+      if (gather) tc_launch<64, 64, 8, true, 64>(h, t, ta, tb, mt, e, s);
+      else tc_launch<64, 64, 8, false, 64>(h, t, ta, tb, mt, e, s);
+    } else if (bn == 256) {
       if (!tc_prepare<256, 64>(h, a, tiles, a.M, t, ta, tb, mt)) return false;
       if (ew8) {
         if (gather) tc_launch<256, 64, 3, true, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
@@ -406,7 +414,12 @@ static bool tc_gemm_o(dreamer_handle *h, const dreamer::GemmArgs &a, const dream
     CUtensorMap ta, tb;
     long mt;
     const bool ew8 = a.K <= 1024;  // as for the QKV projection
-    if (tc_pick_bn(h, a) == 256) {
+    const int bn = tc_pick_bn(h, a);
+    if (bn == 64) {
+      if (!tc_prepare<64, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
+      if (a.arow) tc_launch<64, 64, 8, true, 64>(h, t, ta, tb, mt, e, s);
+      else tc_launch<64, 64, 8, false, 64>(h, t, ta, tb, mt, e, s);
+    } else if (bn == 256) {
       if (!tc_prepare<256, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
       if (ew8) {
         if (a.arow) tc_launch<256, 64, 3, true, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
