@@ -96,8 +96,6 @@ static void mark(dreamer_handle *h, cudaStream_t s, int stage) {
   h->ev_stage[h->ev_used] = stage;
   h->ev_used++;
 }
-// kernels launched by this thread through the library (read as deltas around each call)
-#define LAUNCHED(n) ((void)0)
 
 static void accumulate_marks(dreamer_handle *h, const std::vector<cudaEvent_t> &evs,
                              const std::vector<int> &stages) {
@@ -724,7 +722,6 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   const float *psig = nullptr;
   if (P > 0) {
     mark(h, s, DREAMER_STAGE_PROJ_ROUTE);
-    LAUNCHED(2);
     // pcnt / pcursor are zero here: cleared at init and by every depth's combine kernel
     if (!(tc && tc_proj_route(h, l, h->xh, n, s)))
       route_rows<T>(h, 1, l, h->xh, n, h->pidx, h->psig, nullptr, h->pcnt, s);
@@ -781,7 +778,6 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   auto qkv_gemm = [&](const void *A, int col0, int ncols) {
     // columns [col0, col0 + ncols) of the fused QKV projection
     mark(h, s, DREAMER_STAGE_QKV);
-    LAUNCHED(1);
     GemmArgs a = grouped(ncols, hd, A, hd, (const T *)h->wqkv_t + (size_t)col0 * hd,
                          (long)6 * hd * hd);
     EpiQKV<T> e2 = eq;
@@ -800,7 +796,6 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   auto o_gemm = [&](const void *A, int row0, int nrows, int res_mode, void *yout) {
     // O projection over input rows [row0, row0 + nrows) of W_O ([a_SA | a_DA] order)
     mark(h, s, DREAMER_STAGE_O);
-    LAUNCHED(1);
     GemmArgs a = grouped(hd, nrows, A, 2 * hd, (const T *)h->wo_t + row0, (long)2 * hd * hd);
     a.ldb = 2 * hd;
     EpiO<T> eo{hd, psig, res_mode, (const T *)io.x_in, h->inv_rms, (const T *)h->g,
@@ -820,12 +815,10 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     // serial DA -> SA -> EA: DA on x^, then SA on u = x^ + DA-part of O, then EA
     qkv_gemm(h->xh, 3 * hd, 3 * hd);
     mark(h, s, DREAMER_STAGE_DA);
-    LAUNCHED(1);
     launch_rows<T>(h, da, d, s);
     o_gemm((const T *)h->attn + hd, hd, hd, res_xhat, h->u);   // u = x^ + DA part (acc = u)
     qkv_gemm(h->u, 0, 3 * hd);
     mark(h, s, DREAMER_STAGE_SA);
-    LAUNCHED(io.mode == 1 ? 2 : 1);
     run_sa(s);
     o_gemm(h->attn, 0, hd, 2, h->y);                            // y = u + SA part
   } else {
@@ -834,7 +827,6 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     // 4. DA || SA (papernotes "Key design 1": run in parallel for throughput).  DA runs
     // on the side stream beside SA (two branches of the captured graph); with stage
     // profiling on they run one after the other so each stage's time is its own.
-    LAUNCHED(io.mode == 1 ? 3 : 2);
     if (h->prof) {
       mark(h, s, DREAMER_STAGE_DA);
       launch_rows<T>(h, da, d, s);

@@ -376,22 +376,6 @@ template <typename T> struct EpiUp {
   }
 };
 
-// Expert down-projection epilogue: acc[token] += w_slot * (H W2_e).
-struct EpiDown {
-  int h, k;
-  const int *rows;    // sorted row -> token*k + slot
-  const float *wts;   // [T][k]
-  float *acc;         // [T][h]
-  template <int SEG>
-  __device__ __forceinline__ void operator()(int r, int token, int g, int n0, float *v) const {
-    const int slot = rows[r];
-    const float w = wts[slot];
-    float *dst = acc + (long)(slot / k) * h + n0;
-#pragma unroll
-    for (int i = 0; i < SEG; i++) atomicAdd(dst + i, w * v[i]);
-  }
-};
-
 // Expert down-projection epilogue, store form: the routed row's expert output Y (sorted row
 // r) is written once in dtype; the weighted sum over a token's k rows happens in
 // combine_norm_kernel (no atomics, fixed summation order).

@@ -49,25 +49,6 @@ struct EpiRouterQ {
   }
 };
 
-// Expert down-projection epilogue with 16-byte vector reductions: acc[token] += w (H W2_e).
-struct EpiDownVec {
-  int h, k;
-  const int *rows;
-  const float *wts;
-  float *acc;
-  template <int SEG>
-  __device__ __forceinline__ void operator()(int r, int token, int g, int n0, float *v) const {
-    const int slot = rows[r];
-    const float w = wts[slot];
-    float *dst = acc + (long)(slot / k) * h + n0;
-#pragma unroll
-    for (int i = 0; i < SEG; i += 4)
-      asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + i),
-                   "f"(w * v[i]), "f"(w * v[i + 1]), "f"(w * v[i + 2]), "f"(w * v[i + 3])
-                   : "memory");
-  }
-};
-
 // Expert-attention top-k fused into the score GEMM (row-pass epilogue): each thread owns one
 // token's row, walks all E scores tile by tile and keeps its best KT by z + b (lower expert
 // index on exact ties) in registers (papernotes "Key design 2": sigma(x) = norm(TopK(
