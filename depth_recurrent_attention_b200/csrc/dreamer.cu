@@ -545,17 +545,18 @@ static void launch_da_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStre
   a.q = r.q; a.kv = r.kv; a.out = r.out; a.ldo = r.ldo; a.col0 = r.col0; a.err = r.err;
   const int smem = (int)(2 * (chunk * row_bytes + r.h * (long)sizeof(T)));
   const int threads = 32 * r.H;
-  int per_sm = (227 * 1024) / smem;
-  if (per_sm > 2048 / threads) per_sm = 2048 / threads;
-  if (per_sm > 8) per_sm = 8;
-  if (per_sm < 1) per_sm = 1;
-  long grid = (long)h->num_sms * per_sm;
-  if (grid > a.n_tok) grid = a.n_tok;
-  if (grid < 1) grid = 1;
   auto go = [&](void (*kern)(DaBulkArgs)) {
     // set for the kernel launched (the four head sizes share one pointer type)
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // persistent: as many CTAs as are resident at once (registers, shared memory, threads)
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    long grid = (long)h->num_sms * per_sm;
+    if (grid > a.n_tok) grid = a.n_tok;
+    if (grid < 1) grid = 1;
     launch_k(h, kern, dim3((unsigned)grid), dim3(threads), smem, s, a);
   };
   switch (d) {
