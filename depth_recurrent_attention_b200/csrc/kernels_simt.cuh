@@ -967,51 +967,91 @@ __global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
               a.idx, a.w, a.counts_a, a.counts_b);
 }
 
-// Scores and top-k from a stored router query, one warp per token: q arrives as the three
-// bf16 parts q_hi + q_mid + q_lo of R_l^T q (the split the tensor-core query GEMM writes), the
-// keys unrotated and transposed [d_r][E]; lane j scores experts b + 4j .. b + 4j + 3 of each
-// batch of 128 (one 256-byte row read a key dimension, shared through L1 by the block's warps;
-// four independent sums a lane), z_e = q . k_e in fp32, then the warp top-k.  For batches too
-// short to fill the GPU with fused score tiles.  E a multiple of 4.
-template <int DR>
-__global__ void __launch_bounds__(256) route_q_topk_kernel(const bf16 *qs3, const bf16 *kt,
+// Scores and top-k from a stored router query, WPT warps a token: q arrives as the three bf16
+// parts q_hi + q_mid + q_lo of R_l^T q (the split the tensor-core query GEMM writes), the
+// keys unrotated and transposed [d_r][E].  The token's warps sum the parts once into shared
+// memory; warp w of the token then scores the experts of its slice [w E/WPT, (w+1) E/WPT),
+// lane j taking experts b + 4j .. b + 4j + 3 of each batch of 128 (one 256-byte row read a key
+// dimension, shared through L1 by the block's warps; four independent sums a lane),
+// z_e = q . k_e in fp32 summed in dimension order, and keeps the slice's top k; the token's
+// first warp ranks the WPT lists.  For batches too short to fill the GPU with fused score
+// tiles.  E a multiple of 4 WPT.
+template <int DR, int WPT>
+__global__ void __launch_bounds__(256, 3) route_q_topk_kernel(const bf16 *qs3, const bf16 *kt,
                                                            TopkArgs a) {
   pdl_wait();
   pdl_trigger();
+  constexpr int TPB = 8 / WPT;  // tokens a block
+  __shared__ __align__(16) float qsh[TPB][DR];
+  __shared__ unsigned long long mk[TPB][WPT * 32], ok[TPB][32];
+  __shared__ float mz[TPB][WPT * 32], oz[TPB][32];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int tok = blockIdx.x * 8 + wib;
-  if (tok >= a.n_tok) return;
-  float q[DR];
-  const bf16 *qr = qs3 + (long)tok * 3 * DR;
-#pragma unroll
-  for (int j = 0; j < DR; j += 8) {
-    float hi[8], mid[8], lo[8];
-    load8(qr + j, hi);
-    load8(qr + DR + j, mid);
-    load8(qr + 2 * DR + j, lo);
-#pragma unroll
-    for (int u = 0; u < 8; u++) q[j + u] = (hi[u] + mid[u]) + lo[u];
-  }
-  WarpTopK t(a.k, lane);
-  for (int b = 0; b < a.E; b += 128) {
-    const int e = b + 4 * lane;
-    float z[4] = {0.f, 0.f, 0.f, 0.f};
-    if (e < a.E) {
-#pragma unroll
-      for (int j = 0; j < DR; j++) {
-        const uint2 u = *reinterpret_cast<const uint2 *>(kt + (long)j * a.E + e);
-        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-        const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-        z[0] = fmaf(q[j], f0.x, z[0]);
-        z[1] = fmaf(q[j], f0.y, z[1]);
-        z[2] = fmaf(q[j], f1.x, z[2]);
-        z[3] = fmaf(q[j], f1.y, z[3]);
-      }
+  const int g = wib / WPT, w = wib % WPT;  // token of the block, warp of the token
+  const long tok = (long)blockIdx.x * TPB + g;
+  const bool live = tok < a.n_tok;
+  for (int j = w * 32 + lane; j < DR; j += WPT * 32) {
+    float v = 0.f;
+    if (live) {
+      const bf16 *qr = qs3 + tok * 3 * DR + j;
+      v = (to_f(qr[0]) + to_f(qr[DR])) + to_f(qr[2 * DR]);
     }
-#pragma unroll
-    for (int u = 0; u < 4; u++) t.offer_score(z[u] * a.zscale, e + u, e + u < a.E, a.bias);
+    qsh[g][j] = v;
   }
-  emit_topk(lane, a.k, t.lv, t.le, t.lz, tok, a.mode, a.idx, a.w, a.counts_a, a.counts_b);
+  __syncthreads();
+  WarpTopK t(a.k, lane);
+  if (live) {
+    const int per = a.E / WPT, e0 = w * per, e1 = e0 + per;
+    for (int b = e0; b < e1; b += 128) {
+      const int e = b + 4 * lane;
+      float z[4] = {0.f, 0.f, 0.f, 0.f};
+      if (e < e1) {
+        const bf16 *kc = kt + e;
+#pragma unroll
+        for (int j = 0; j < DR; j += 4) {
+          const float4 q4 = *reinterpret_cast<const float4 *>(&qsh[g][j]);
+          const float qj[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+          for (int jj = 0; jj < 4; jj++) {
+            const uint2 u = *reinterpret_cast<const uint2 *>(kc + (long)(j + jj) * a.E);
+            const float2 f0 =
+                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+            const float2 f1 =
+                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+            z[0] = fmaf(qj[jj], f0.x, z[0]);
+            z[1] = fmaf(qj[jj], f0.y, z[1]);
+            z[2] = fmaf(qj[jj], f1.x, z[2]);
+            z[3] = fmaf(qj[jj], f1.y, z[3]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; u++) t.offer_score(z[u] * a.zscale, e + u, e + u < e1, a.bias);
+    }
+  }
+  if (WPT == 1) {
+    if (live) emit_topk(lane, a.k, t.lv, t.le, t.lz, tok, a.mode, a.idx, a.w, a.counts_a, a.counts_b);
+    return;
+  }
+  if (lane < a.k) {  // the warps' lists, compacted
+    mk[g][w * a.k + lane] = topk_key(t.lv, t.le);
+    mz[g][w * a.k + lane] = t.lz;
+  }
+  __syncthreads();
+  if (w != 0 || !live) return;
+  const int nc = WPT * a.k;  // rank every listed candidate against all (distinct experts)
+  for (int i = lane; i < nc; i += 32) {
+    const unsigned long long ki = mk[g][i];
+    if (ki == 0ull) continue;
+    int r = 0;
+    for (int c = 0; c < nc; c++) r += mk[g][c] > ki ? 1 : 0;
+    if (r < a.k) {
+      ok[g][r] = ki;
+      oz[g][r] = mz[g][i];
+    }
+  }
+  __syncwarp();
+  emit_topk(lane, a.k, 0.f, lane < a.k ? topk_key_expert(ok[g][lane]) : 0,
+            lane < a.k ? oz[g][lane] : 0.f, tok, a.mode, a.idx, a.w, a.counts_a, a.counts_b);
 }
 
 // Routing of few tokens (decode): a cluster of NCL CTAs per token (papernotes "Key design 2":

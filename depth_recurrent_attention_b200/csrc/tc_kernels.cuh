@@ -480,9 +480,10 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
   TopkArgs k{};
   k.n_tok = n; k.E = E; k.k = c.top_k; k.mode = 0; k.zscale = zs;
   k.bias = h->bias; k.idx = idx; k.w = w; k.counts_a = counts_a; k.counts_b = counts_b;
-  auto kern = dr == 64 ? route_q_topk_kernel<64> : route_q_topk_kernel<128>;
-  launch_k(h, kern, dim3((n + 7) / 8), dim3(256), 0, s, (const bf16 *)h->qsplit,
-           (const bf16 *)h->kEt, k);
+  constexpr int WPT = 2;  // warps a token, four tokens a block
+  auto kern = dr == 64 ? route_q_topk_kernel<64, WPT> : route_q_topk_kernel<128, WPT>;
+  launch_k(h, kern, dim3((n + 8 / WPT - 1) / (8 / WPT)), dim3(256), 0, s,
+           (const bf16 *)h->qsplit, (const bf16 *)h->kEt, k);
   return true;
 }
 
