@@ -116,8 +116,17 @@ template <typename T> struct EpiQKV {
       return cb + ((((long)l * B + tok[i]) * (h / d) + hd0 / d) * cap + ax[i]) * d;
     };
     if (blk <= 1) {
-      // token RoPE: head columns o and o + d/2, frequency o
+      // token RoPE: head columns o and o + d/2, frequency o; every row's table entries are
+      // requested before the first store (one memory round trip a pass)
       const int o = perm ? unperm(cin) : cin;
+      float4 t01[NR], t23[NR];
+#pragma unroll
+      for (int i = 0; i < NR; i++) {
+        const float4 *cs = reinterpret_cast<const float4 *>(
+            rope_tok + (long)(r[i] >= 0 && ax[i] >= 0 ? ax[i] : 0) * (d / 2) + o);
+        t01[i] = __ldg(cs);
+        t23[i] = __ldg(cs + 1);
+      }
 #pragma unroll
       for (int i = 0; i < NR; i++) {
         if (r[i] < 0) continue;
@@ -125,8 +134,7 @@ template <typename T> struct EpiQKV {
           raise_dev_error(err, DEV_BAD_INDEX);
           continue;
         }
-        const float4 *cs = reinterpret_cast<const float4 *>(rope_tok + (long)ax[i] * (d / 2) + o);
-        const float4 c01 = cs[0], c23 = cs[1];
+        const float4 c01 = t01[i], c23 = t23[i];
         const float cc[4] = {c01.x, c01.z, c23.x, c23.z}, sn[4] = {c01.y, c01.w, c23.y, c23.w};
         float a[4], b[4];
 #pragma unroll
@@ -319,7 +327,7 @@ template <typename T> struct EpiO {
     }
   }
   // Coalesced layout (NV values a lane and row: 4 at col, and with NV = 8 four more at
-  // col + 32); rows in pairs, each pair's residual loads issued before its stores.
+  // col + 32); every row's residual loads are issued before the first store.
   template <int NR, int NV>
   __device__ __forceinline__ void store_rows(const int *r, const int *tok, const Aux *ax, int g,
                                              int col, const float (*v)[NV]) const {
@@ -329,7 +337,7 @@ template <typename T> struct EpiO {
       if (res_mode != 2) load4(gain + col + 32 * hh, gv + 4 * hh);
       else gv[4 * hh] = gv[4 * hh + 1] = gv[4 * hh + 2] = gv[4 * hh + 3] = 1.f;
     }
-    constexpr int GR = NR < 2 ? NR : 2;
+    constexpr int GR = NR;
 #pragma unroll
     for (int i0 = 0; i0 < NR; i0 += GR) {
       float xr[GR][NV];
