@@ -5,6 +5,7 @@
 #include <cuda.h>
 
 #include "tc_attn.cuh"
+#include "tc_ffn.cuh"
 #include "tc_gemm.cuh"
 
 namespace dreamer {
@@ -518,7 +519,23 @@ static bool tc_expert_ok(dreamer_handle *h) {
   return g_encode_tiled && (m == 16 || m == 32 || m == 64) && c.hidden % 256 == 0;
 }
 
-static bool tc_expert(dreamer_handle *h, const void *X, int n, cudaStream_t s) {
+template <int M, int ST>
+static void tc_ffn_launch(dreamer_handle *h, const CUtensorMap &t1, const CUtensorMap &t2,
+                          const dreamer::tc::TcFfnArgs &a, long max_tiles, cudaStream_t s) {
+  using Cfg = dreamer::tc::TcFfnCfg<M, ST>;
+  auto kern = dreamer::tc::tc_ffn_kernel<M, ST>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    attr_set = true;
+  }
+  long grid = max_tiles < h->num_sms ? max_tiles : h->num_sms;
+  if (grid < 1) grid = 1;
+  launch_k(h, kern, dim3((unsigned)grid), dim3(Cfg::THREADS), Cfg::SMEM, s, t1, t2, a);
+}
+
+// Two grouped GEMMs: H = SiLU(X_gathered W1_e) stored in sorted order, then Y = H W2_e.
+static bool tc_expert_two(dreamer_handle *h, const void *X, int n, cudaStream_t s) {
   using namespace dreamer;
   const dreamer_config &c = h->cfg;
   const int hd = c.hidden, m = c.expert_hidden, k = c.top_k, E = c.n_experts;
@@ -560,5 +577,32 @@ static bool tc_expert(dreamer_handle *h, const void *X, int n, cudaStream_t s) {
       tc_launch<64, 64, 8, true, 64>(h, tu, tau, tbu, mtu, eu, s);
       tc_launch<256, 64, 4, false, 64>(h, td, tad, tbd, mtd, ed, s);
       return true;
+  }
+}
+
+// Expert FFNs of the routed rows (sorted by expert).  With about a full 128-row tile per expert
+// or more, one fused kernel keeps H on chip (H = SiLU(X W1_e), Y = H W2_e stored in sorted
+// order for the combine); with fewer rows per expert the tiles are mostly padding and the two
+// grouped GEMMs, each spread over all SMs on its own tiling, finish sooner.
+static bool tc_expert(dreamer_handle *h, const void *X, int n, cudaStream_t s) {
+  using namespace dreamer;
+  const dreamer_config &c = h->cfg;
+  const int hd = c.hidden, m = c.expert_hidden, k = c.top_k, E = c.n_experts;
+  const long rows = (long)n * k;
+  if (rows < 96L * E) return tc_expert_two(h, X, n, s);
+  if (((uintptr_t)X & 15) || (hd * 2) % 16) return false;
+  CUtensorMap t1, t2;  // W1^T [E m][h] in blocks of m x 64; W2^T [E h][m] in chunks of 256 x m
+  if (!make_tmap(&t1, h->w1_t, hd, (uint64_t)E * m, (uint64_t)hd * 2, 64, m) ||
+      !make_tmap(&t2, h->w2_t, m, (uint64_t)E * hd, (uint64_t)m * 2, m, 256))
+    return false;
+  tc::TcFfnArgs a{};
+  a.H = hd; a.G = E; a.M = (int)rows; a.goffs = h->eoffs; a.tiles = h->etiles_b;
+  a.arow = h->erows; a.arow_div = k; a.X = (const bf16 *)X; a.ldx = hd;
+  a.Y = (bf16 *)h->Ybuf; a.err = h->err;
+  const long max_tiles = (rows + 127) / 128 + E;
+  switch (m) {
+    case 16: tc_ffn_launch<16, 6>(h, t1, t2, a, max_tiles, s); return true;
+    case 32: tc_ffn_launch<32, 6>(h, t1, t2, a, max_tiles, s); return true;
+    default: tc_ffn_launch<64, 5>(h, t1, t2, a, max_tiles, s); return true;
   }
 }

@@ -188,6 +188,19 @@ def test_small_linear_moe_step_bf16(cuda):
         run_step_and_compare(cfg, W, dev, l, orc=orc)
 
 
+@pytest.mark.parametrize("m", [16, 32])
+def test_small_expert_sizes_bf16(cuda, m):
+    """Expert hidden sizes 16 and 32 (the fused expert FFN with 32- and 64-byte H rows), about
+    32 routed rows per expert, so most tiles are partial."""
+    cfg = configs.SMALL.with_(expert_hidden=m, depth=2)
+    W = inputs.host_weights(cfg)
+    dev = make_handle(cfg, W)
+    orc = O.Oracle(cfg, W)
+    for l in (0, 1):
+        flips, n = run_step_and_compare(cfg, W, dev, l, orc=orc)
+        assert flips <= 0.05 * n
+
+
 @pytest.mark.parametrize("variant", [1, 2])
 def test_small_layout_variants_bf16(cuda, variant):
     cfg = configs.SMALL.with_(variant=variant, depth=3)
@@ -238,7 +251,10 @@ def test_small_free_running_drift_reported(cuda):
                                 dict(n_experts=8, top_k=8, depth=2, n_heads=4, head_dim=128,
                                      n_proj_experts=1),
                                 dict(n_experts=4, top_k=4, depth=4, da_window=2),
-                                dict(n_experts=4, top_k=4, depth=3, variant=3)])
+                                dict(n_experts=4, top_k=4, depth=3, variant=3),
+                                # expert FFN with 32- and 64-byte H rows, full tiles
+                                dict(n_experts=4, top_k=4, depth=2, expert_hidden=16),
+                                dict(n_experts=4, top_k=4, depth=2, expert_hidden=32)])
 def test_small_flip_free_all_depths_bf16(cuda, kw):
     torch = _torch()
     cfg = configs.SMALL.with_(**kw)
