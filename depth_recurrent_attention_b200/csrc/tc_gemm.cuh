@@ -6,10 +6,11 @@
 //   warp 0      TMA producer: B tile (and A tile unless rows are gathered) per stage
 //   warp 1      TMEM allocator + single-thread MMA issuer (tcgen05.mma, commit to barriers)
 //   warps 2-5   epilogue: tcgen05.ld of the 128 x BN accumulator, row r per thread, then the
-//               caller's epilogue functor on column segments of SEG values
-//   warps 6-7   (GATHER only) A producers: 16-byte cp.async of gathered rows into the
-//               128B-swizzled layout TMA would have written (two warps keep the block at
-//               8 warps, so the epilogue may use up to 255 registers a thread)
+//               caller's epilogue functor on column segments of SEG values (EW = 8: warps
+//               2-9, two per TMEM lane quarter, splitting the segments or column passes)
+//   next 2      (GATHER only) A producers: 16-byte cp.async of gathered rows into the
+//               128B-swizzled layout TMA would have written (with four epilogue warps the
+//               block stays at 8 warps, so the epilogue may use up to 255 registers a thread)
 // Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap the MMAs of
 // tile i+1.  Every wait is bounded (tc::mbar_wait); on expiry the CTA winds down and the
 // device error flag is set.
