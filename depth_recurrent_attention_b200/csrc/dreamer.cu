@@ -1166,19 +1166,29 @@ extern "C" int dreamer_route_balance(dreamer_handle *h, int depth, float *lorenz
   return DREAMER_OK;
 }
 
-extern "C" int dreamer_bias_update(dreamer_handle *h, float lambda, float *bias_out,
-                                   dreamer_stream stream) {
-  if (!h) return DREAMER_ERR_ARG;
+static int launch_bias_update(dreamer_handle *h, const int *counts, int rows, float lambda,
+                              float *bias_out, cudaStream_t s) {
   const int E = h->cfg.n_experts;
   int n2 = 1;
   while (n2 < E) n2 <<= 1;
   const size_t smem = (size_t)(n2 + E) * sizeof(int);
   if (smem > 200 * 1024) return DREAMER_ERR_UNSUPPORTED;
-  cudaStream_t s = (cudaStream_t)stream;
   if (smem > 48 * 1024)
     CK(cudaFuncSetAttribute(bias_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   ++g_launches;
-  bias_update_kernel<<<1, 1024, smem, s>>>(h->counts, h->cfg.depth, E, lambda, h->bias, bias_out);
+  bias_update_kernel<<<1, 1024, smem, s>>>(counts, rows, E, lambda, h->bias, bias_out);
   CK(cudaGetLastError());
   return DREAMER_OK;
+}
+
+extern "C" int dreamer_bias_update(dreamer_handle *h, float lambda, float *bias_out,
+                                   dreamer_stream stream) {
+  if (!h) return DREAMER_ERR_ARG;
+  return launch_bias_update(h, h->counts, h->cfg.depth, lambda, bias_out, (cudaStream_t)stream);
+}
+
+extern "C" int dreamer_bias_update_counts(dreamer_handle *h, float lambda, const int32_t *counts,
+                                          int n_rows, float *bias_out, dreamer_stream stream) {
+  if (!h || !counts || n_rows < 1) return DREAMER_ERR_ARG;
+  return launch_bias_update(h, counts, n_rows, lambda, bias_out, (cudaStream_t)stream);
 }

@@ -74,6 +74,7 @@ def lib():
         L.dreamer_route_counts.argtypes = [vp, vp, i, vp]
         L.dreamer_route_experts.argtypes = [vp, i, vp, i, vp, vp, vp, vp]
         L.dreamer_bias_update.argtypes = [vp, C.c_float, vp, vp]
+        L.dreamer_bias_update_counts.argtypes = [vp, C.c_float, vp, i, vp, vp]
         L.dreamer_route_balance.argtypes = [vp, i, vp, vp, vp]
         L.dreamer_set_profiling.argtypes = [vp, i]
         L.dreamer_get_stats.argtypes = [vp, C.POINTER(StatsC), i]
@@ -83,6 +84,7 @@ def lib():
         L.dreamer_strerror.restype = C.c_char_p
         for f in ("dreamer_init", "dreamer_core_forward", "dreamer_decode_step",
                   "dreamer_route_counts", "dreamer_route_experts", "dreamer_bias_update",
+                  "dreamer_bias_update_counts", "dreamer_route_balance",
                   "dreamer_set_profiling", "dreamer_get_stats"):
             getattr(L, f).restype = i
         _lib = L
@@ -211,10 +213,22 @@ class Dreamer:
                "dreamer_route_experts")
         return idx, w, counts
 
-    def bias_update(self, lam: float, stream=None):
+    def bias_update(self, lam: float, counts=None, stream=None):
+        """b_e += lam * sign(median(N) - N_e) on the handle's bias; returns the new bias.
+        N = the last call's route counts summed over depths, or, when `counts` is given (a
+        CUDA int32 tensor [R][E] or [E], e.g. the counts of all replicas from
+        allreduce_route_counts), those summed over their rows."""
         out = torch.empty(self.cfg.n_experts, dtype=torch.float32, device="cuda")
-        _check(lib().dreamer_bias_update(self.h, float(lam), _ptr(out), _stream(stream)),
-               "dreamer_bias_update")
+        if counts is None:
+            _check(lib().dreamer_bias_update(self.h, float(lam), _ptr(out), _stream(stream)),
+                   "dreamer_bias_update")
+            return out
+        c = counts.reshape(-1, self.cfg.n_experts)
+        if c.dtype != torch.int32 or not c.is_cuda or not c.is_contiguous():
+            raise ValueError("counts: a contiguous CUDA int32 tensor [R][E] or [E]")
+        _check(lib().dreamer_bias_update_counts(self.h, float(lam), _ptr(c), int(c.shape[0]),
+                                                _ptr(out), _stream(stream)),
+               "dreamer_bias_update_counts")
         return out
 
     def set_profiling(self, enable: bool):
@@ -226,6 +240,18 @@ class Dreamer:
         return dict(launches=int(st.launches),
                     ms={n: float(st.ms[i]) for i, n in enumerate(STAGES)},
                     count={n: int(st.count[i]) for i, n in enumerate(STAGES)})
+
+
+def allreduce_route_counts(counts, group=None):
+    """Sum route counts ([L][E] int32, from Dreamer.route_counts) over the ranks of `group` in
+    place and return them: the one exchange of data-parallel replicas, after which every
+    replica's bias update (Dreamer.bias_update(lam, counts=...)) sees the global expert use.
+    NCCL for CUDA tensors (NVLink), gloo for CPU ones; a no-op without a process group of
+    more than one rank."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(counts, op=dist.ReduceOp.SUM, group=group)
+    return counts
 
 
 class LayeredStack:

@@ -186,6 +186,14 @@ int dreamer_route_experts_noalloc(const dreamer_config *cfg, int depth, const vo
 int dreamer_bias_update(dreamer_handle *h, float lambda, float *bias_out,
                         dreamer_stream stream);
 
+/* The same update from caller-given counts: counts [n_rows][E] int32, device pointer (read
+ * only), N_e = sum over the rows.  With data-parallel replicas (one handle per GPU, each
+ * routing its own batch) the counts are the [L][E] output of dreamer_route_counts summed over
+ * the replicas by one all-reduce, so every replica applies the same update to its bias.
+ * DREAMER_ERR_ARG for a NULL handle or counts or n_rows < 1.                              */
+int dreamer_bias_update_counts(dreamer_handle *h, float lambda, const int32_t *counts,
+                               int n_rows, float *bias_out, dreamer_stream stream);
+
 /* Balance summary of the expert route counts N of the last call ([notes] "Key design 2":
  * the bias keeps expert use balanced; this measures how balanced): N_e = counts of depth
  * `depth`, or summed over depths for depth < 0.  Writes the Lorenz curve of N (sorted

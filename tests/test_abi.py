@@ -50,6 +50,16 @@ def test_strerror_without_gpu(built):
     assert lib.dreamer_strerror(-5) == b"device wait timed out"
 
 
+def test_argument_errors_without_gpu(built):
+    """Entry points reject a NULL handle before touching the device (through the binding's
+    argument types)."""
+    from depth_recurrent_attention_b200.dreamer import ERR_ARG, lib
+    L = lib()
+    assert L.dreamer_bias_update_counts(None, ctypes.c_float(0.01), None, 1, None, None) == ERR_ARG
+    assert L.dreamer_bias_update(None, ctypes.c_float(0.01), None, None) == ERR_ARG
+    assert L.dreamer_route_balance(None, -1, None, None, None) == ERR_ARG
+
+
 def test_product_does_not_reference_the_oracle():
     for dirpath, _, files in os.walk(PKG):
         for f in files:

@@ -366,6 +366,24 @@ def test_bias_update_matches_oracle(cuda):
     assert np.allclose(new_b, ref, atol=1e-7)
 
 
+def test_bias_update_from_replica_counts(cuda):
+    """The update from given counts (this handle's route counts plus another replica's,
+    summed as the all-reduce would) matches the oracle's update from the same counts."""
+    torch = _torch()
+    cfg = configs.TINY
+    W = inputs.host_weights(cfg)
+    dev = make_handle(cfg, W)
+    dev.forward(inputs.to_device(inputs.host_inputs(cfg)["x0"], "fp32"))
+    counts = dev.route_counts(on_host=False)
+    rng = np.random.default_rng(7)
+    other = rng.integers(0, 9, size=tuple(counts.shape)).astype(np.int32)
+    total = counts + torch.from_numpy(other).to(counts.device)
+    new_b = dev.bias_update(0.01, counts=total).cpu().numpy()
+    ref = O.bias_update(np.ascontiguousarray(total.cpu().numpy()), 0.01,
+                        W["bias"].astype(np.float64))
+    assert np.allclose(new_b, ref, atol=1e-7)
+
+
 def test_errors_are_returned_not_faulted(cuda):
     torch = _torch()
     from depth_recurrent_attention_b200.dreamer import Dreamer, DreamerError, ERR_ARG, \

@@ -4,7 +4,9 @@ bench.py runs one full replica per GPU; nothing crosses ranks on the data path. 
 ranks share is host logic, checked here without a GPU: the timed region is the slowest
 rank's (all-reduce MAX), the job's value counts every rank's units over that time, each
 rank draws its own input batch from its own seed while the weights are identical, and the
-ranks leave the process group cleanly.
+ranks leave the process group cleanly.  The one exchange of the replicas, the all-reduce of
+the [L][E] route counts before a bias-balance update, runs here on CPU tensors: every rank
+gets the sum and computes the same update from it.
 """
 import os
 import socket
@@ -21,7 +23,18 @@ def _free_port():
         return s.getsockname()[1]
 
 
+def _rank_counts(cfg, rank):
+    """A rank's [L][E] route counts: each depth routes T k slots, spread unevenly."""
+    rng = np.random.default_rng(100 + rank)
+    c = np.zeros((cfg.depth, cfg.n_experts), np.int32)
+    for l in range(cfg.depth):
+        e = rng.integers(0, cfg.n_experts, cfg.tokens * cfg.top_k)
+        np.add.at(c[l], e, 1)
+    return c
+
+
 def _worker(rank, world, port, out_q):
+    import sys
     import torch
     import torch.distributed as dist
     os.environ["MASTER_ADDR"] = "127.0.0.1"
@@ -38,7 +51,16 @@ def _worker(rank, world, port, out_q):
     spec = inputs.input_specs(cfg)[0]
     x = inputs.draw(spec, bench.rank_seed(cfg, rank), 0, 4096)
     w = inputs.draw(inputs.weight_specs(cfg)[0], cfg.seed, 0, 4096)
-    out_q.put((rank, m, units, value, float(np.sum(x)), float(np.sum(w))))
+    # route counts of this rank's batch, summed over the ranks, then the bias update from them
+    from depth_recurrent_attention_b200.dreamer import allreduce_route_counts
+    sys.path.insert(0, os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                                    "oracle"))
+    import oracle as O
+    counts = allreduce_route_counts(torch.from_numpy(_rank_counts(cfg, rank)))
+    bias0 = inputs.host_weights(configs.TINY)["bias"].astype(np.float64)
+    tiny_counts = counts[:configs.TINY.depth, :configs.TINY.n_experts].numpy()
+    new_b = O.bias_update(np.ascontiguousarray(tiny_counts), 0.01, bias0)
+    out_q.put((rank, m, units, value, float(np.sum(x)), float(np.sum(w)), counts.numpy(), new_b))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -60,12 +82,16 @@ def test_two_gloo_ranks():
         assert p.exitcode == 0
     cfg = configs.SMALL
     for r in range(2):
-        _, m, units, value, _, _ = res[r]
+        _, m, units, value, _, _, _, _ = res[r]
         assert m == 14.0                                   # max over ranks
         assert units == 2 * cfg.units                      # whole-job units
         assert value == pytest.approx(2 * cfg.units / (14.0 / 4 / 1e3))
     assert res[0][4] != res[1][4]                          # each rank its own batch
     assert res[0][5] == res[1][5]                          # shared weights
+    total = _rank_counts(cfg, 0) + _rank_counts(cfg, 1)
+    for r in range(2):                                     # the all-reduced route counts
+        assert np.array_equal(res[r][6], total)
+    assert np.array_equal(res[0][7], res[1][7])            # the same bias update everywhere
 
 
 def test_single_rank_helpers():
