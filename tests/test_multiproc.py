@@ -101,3 +101,8 @@ def test_single_rank_helpers():
     units, value = bench.job_value(cfg, 1, 2.0)
     assert units == cfg.units and value == pytest.approx(cfg.units / 2e-3)
     assert bench.rank_seed(cfg, 0) == cfg.seed and bench.rank_seed(cfg, 3) != cfg.seed
+    # without a process group the count exchange leaves the counts as they are
+    import torch
+    from depth_recurrent_attention_b200.dreamer import allreduce_route_counts
+    c = torch.arange(12, dtype=torch.int32).reshape(3, 4)
+    assert torch.equal(allreduce_route_counts(c.clone()), c)
