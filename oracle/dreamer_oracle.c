@@ -783,3 +783,22 @@ int orc_route(const orc_cfg *c, const orc_weights *W, int l, const float *y, int
   free(krotE);
   return 0;
 }
+
+/* Projection router alone on given normalised states (R12): x^ [T][h] at depth l ->
+ * p* [T], sigma [T], margin z_P[p*] - runner-up [T] (margin may be NULL).             */
+int orc_proj_route(const orc_cfg *c, const orc_weights *W, int l, const float *xh, int T,
+                   int32_t *pstar, double *sigma, double *pmargin) {
+  const int h = c->h, dr = c->dr, P = c->P;
+  if (P < 1 || P > 256 || l < 0 || l >= c->L || dr > 1024) return -1;
+  double *krotP = (double *)xcalloc((size_t)P * dr, sizeof(double));
+  rotate_keys(W->k_P, P, dr, l, c->L, c->rope_base, krotP);
+#pragma omp parallel for schedule(dynamic, 8)
+  for (long t = 0; t < T; t++) {
+    double *xd = (double *)xcalloc((size_t)h, sizeof(double));
+    for (int i = 0; i < h; i++) xd[i] = (double)xh[t * h + i];
+    proj_route(c, W, krotP, xd, &pstar[t], &sigma[t], pmargin ? &pmargin[t] : NULL);
+    free(xd);
+  }
+  free(krotP);
+  return 0;
+}

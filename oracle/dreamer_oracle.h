@@ -109,6 +109,11 @@ int orc_decode_seq(const orc_cfg *c, const orc_weights *W, const float *x_new, d
 int orc_route(const orc_cfg *c, const orc_weights *W, int l, const float *y, int T,
               int32_t *idx, double *w, double *margin, double *zsel, int32_t *counts);
 
+/* Projection router alone on given states (R12): x^ [T][h] at depth l -> p* [T],
+ * sigma [T], margin [T] (z_P of p* minus the runner-up; may be NULL).  P > 0 only.    */
+int orc_proj_route(const orc_cfg *c, const orc_weights *W, int l, const float *xh, int T,
+                   int32_t *pstar, double *sigma, double *pmargin);
+
 /* Building blocks exposed for the pins. */
 void orc_rmsnorm(int h, const double *x, const float *g, double eps, double *out);
 void orc_rope(double *v, int n, double pos, double base);

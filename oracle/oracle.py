@@ -57,6 +57,7 @@ def lib():
                                       f64p, vp]
         L.orc_decode_seq.argtypes = [vp, vp, f32p, f64p, f64p, C.c_int, C.c_int, f64p, vp]
         L.orc_route.argtypes = [vp, vp, C.c_int, f32p, C.c_int, i32p, f64p, vp, vp, vp]
+        L.orc_proj_route.argtypes = [vp, vp, C.c_int, f32p, C.c_int, i32p, f64p, vp]
         L.orc_rmsnorm.argtypes = [C.c_int, f64p, f32p, C.c_double, f64p]
         L.orc_rope.argtypes = [f64p, C.c_int, C.c_double, C.c_double]
         L.orc_depth_rope.argtypes = [f64p, C.c_int, C.c_int, C.c_int, C.c_double]
@@ -67,7 +68,7 @@ def lib():
         L.orc_expert.argtypes = [C.c_int, C.c_int, f64p, f32p, f32p, f64p]
         L.orc_bias_update.argtypes = [C.c_int, C.c_int, i32p, C.c_double, f64p]
         for f in ("orc_forward", "orc_forward_da_loops", "orc_step_tokens", "orc_decode_seq",
-                  "orc_route"):
+                  "orc_route", "orc_proj_route"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -200,6 +201,19 @@ class Oracle:
         if rc != 0:
             raise RuntimeError(f"orc_route failed: {rc}")
         return dict(idx=idx, w=w, margin=margin, zsel=zsel, counts=counts)
+
+    def proj_route(self, l: int, xh) -> dict:
+        """Projection router alone on normalised states x^ [T][h] at depth l (P > 0)."""
+        xh = _f32(xh)
+        T = xh.shape[0]
+        pidx = np.zeros(T, np.int32)
+        psig = np.zeros(T)
+        pmargin = np.zeros(T)
+        rc = lib().orc_proj_route(C.byref(self.c), C.byref(self.W), l, xh, T, pidx, psig,
+                                  pmargin.ctypes.data)
+        if rc != 0:
+            raise RuntimeError(f"orc_proj_route failed: {rc}")
+        return dict(pidx=pidx, psig=psig, pmargin=pmargin)
 
 
 # -- building blocks (for the pins) ------------------------------------------------------

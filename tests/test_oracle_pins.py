@@ -219,23 +219,29 @@ def test_expert_ffn_scalar_case():
 
 def _closed_form_single_token(cfg, W, x0):
     """L = 1, s = 1, E = k: SA over one key returns v_SA, DA at depth 0 returns v_DA,
-    all experts are picked.  Everything reduces to plain matrix products."""
+    all experts are picked.  Everything reduces to plain matrix products.  With P projection
+    experts each token takes p* = argmax_p z_P (numpy's argmax: the first of equal maxima)
+    and runs sigma (W_p* + W_shared) with sigma = sigmoid(z_P[p*]) (papernotes "Key design
+    3": sigma x W + max(sigma^) x W_shared, the router shared by QKV and O).  Returns
+    (x_out, p*, sigma)."""
     h, dr = cfg.hidden, cfg.router_dim
     f = lambda a: np.asarray(a, np.float64)
     x = f(x0)
+    T = x.shape[0]
     xh = x / np.sqrt(np.mean(x ** 2, axis=-1, keepdims=True) + cfg.rms_eps) * f(W["g"])
     P = cfg.n_proj_experts
     if P > 0:
-        # single projection expert: p* = 0, sigma = sigmoid(q_P . k~_P / sqrt(d_r))
-        kP = O.depth_rope(f(W["k_P"][0]), 0, 1)
-        z = (xh @ f(W["w_qP"])) @ kP / np.sqrt(dr)
-        sig = (1 / (1 + np.exp(-z)))[:, None]
-        Wqkv = sig[:, :, None] * (f(W["w_qkv"][0]) + f(W["w_qkv_shared"]))[None]
-        Wo = sig[:, :, None] * (f(W["w_o"][0]) + f(W["w_o_shared"]))[None]
+        # at L = 1 the depth RoPE of depth 0 rotates both halves by position 0: the identity
+        kP = np.stack([O.depth_rope(f(k), 0, 1) for k in W["k_P"]])       # [P][d_r]
+        zP = (xh @ f(W["w_qP"])) @ kP.T / np.sqrt(dr)                     # [T][P]
+        pstar = np.argmax(zP, axis=1)
+        sig = 1 / (1 + np.exp(-zP[np.arange(T), pstar]))
+        Wqkv = sig[:, None, None] * (f(W["w_qkv"])[pstar] + f(W["w_qkv_shared"])[None])
+        Wo = sig[:, None, None] * (f(W["w_o"])[pstar] + f(W["w_o_shared"])[None])
         qkv = np.einsum("ti,tij->tj", xh, Wqkv)
     else:
         qkv = xh @ f(W["w_qkv"][0])
-        Wo = None
+        Wo, pstar, sig = None, np.zeros(T, int), np.ones(T)
     v_sa, v_da = qkv[:, 2 * h:3 * h], qkv[:, 5 * h:6 * h]
     cat = np.concatenate([v_sa, v_da], axis=1)
     o = np.einsum("ti,tij->tj", cat, Wo) if Wo is not None else cat @ f(W["w_o"][0])
@@ -248,7 +254,7 @@ def _closed_form_single_token(cfg, W, x0):
     for e in range(cfg.n_experts):
         u = y @ f(W["w1"][e])
         out += w[:, e:e + 1] * ((u / (1 + np.exp(-u))) @ f(W["w2"][e]))
-    return out
+    return out, pstar, sig
 
 
 @pytest.mark.parametrize("P", [0, 1])
@@ -257,8 +263,64 @@ def test_block_reduces_to_closed_form(P):
     W = rand_weights(cfg, seed=11)
     x0 = inputs.host_inputs(cfg)["x0"]
     r = O.Oracle(cfg, W, threads=1).forward(x0)
-    ref = _closed_form_single_token(cfg, W, x0)
+    ref, _, _ = _closed_form_single_token(cfg, W, x0)
     assert np.allclose(r["x_out"], ref, rtol=1e-11, atol=1e-11)
+
+
+def test_block_with_three_projection_experts_closed_form():
+    """P = 3 projection experts with distinct QKV/O matrices; the keys are built so that the
+    six tokens pick all three experts (token t aligns with expert t mod 3) and the argmin
+    differs from the argmax for every token.  The oracle's p*, sigma, margin and output
+    must equal the numpy chain; so an argmin for the argmax, a wrong expert offset into the
+    stacked matrices, or a sigma from another expert's score fails here."""
+    P = 3
+    cfg = tiny_cfg(batch=6, seq=1, depth=1, n_experts=3, top_k=3, n_proj_experts=P)
+    W = dict(rand_weights(cfg, seed=12))
+    x0 = inputs.host_inputs(cfg)["x0"]
+    f = lambda a: np.asarray(a, np.float64)
+    x = f(x0)
+    xh = x / np.sqrt(np.mean(x ** 2, axis=-1, keepdims=True) + cfg.rms_eps)
+    q = xh @ f(W["w_qP"])
+    W["k_P"] = np.stack([3.0 * q[p] / np.linalg.norm(q[p]) for p in range(P)]).astype(np.float32)
+    # the stacked expert matrices differ from one another
+    for name in ("w_qkv", "w_o"):
+        for a in range(P):
+            for b in range(a + 1, P):
+                assert np.abs(W[name][a] - W[name][b]).max() > 0.1
+    ref, pstar, sig = _closed_form_single_token(cfg, W, x0)
+    kP = f(W["k_P"])
+    zP = q @ kP.T / np.sqrt(cfg.router_dim)
+    assert sorted(set(pstar.tolist())) == [0, 1, 2], pstar
+    assert np.all(np.argmin(zP, axis=1) != pstar)
+    r = O.Oracle(cfg, W, threads=1).forward(x0)
+    assert np.array_equal(r["pidx"][0], pstar)
+    assert np.allclose(r["psig"][0], sig, rtol=1e-12, atol=0)
+    second = np.sort(zP, axis=1)[:, -2]
+    assert np.allclose(r["pmargin"][0], zP.max(1) - second, rtol=1e-10, atol=1e-12)
+    assert np.allclose(r["x_out"], ref, rtol=1e-11, atol=1e-11)
+    # the router alone (the entry the GPU parity tests route the device's x^ with)
+    pr = O.Oracle(cfg, W, threads=1).proj_route(0, xh.astype(np.float32))
+    xh32 = f(xh.astype(np.float32))
+    z32 = (xh32 @ f(W["w_qP"])) @ kP.T / np.sqrt(cfg.router_dim)
+    assert np.array_equal(pr["pidx"], np.argmax(z32, axis=1))
+    assert np.allclose(pr["psig"], 1 / (1 + np.exp(-z32.max(1))), rtol=1e-12, atol=0)
+
+
+def test_projection_router_rotates_keys_by_the_depth():
+    """At depth l of L the projection keys carry the depth RoPE of l (reading R12, the same
+    form as expert attention): the router alone equals argmax over (x^ W_qP) . R_l k_p."""
+    cfg = tiny_cfg(batch=4, seq=2, depth=3, n_proj_experts=5)
+    W = rand_weights(cfg, seed=13)
+    xh = RNG.normal(size=(cfg.tokens, cfg.hidden)).astype(np.float32)
+    f = lambda a: np.asarray(a, np.float64)
+    q = f(xh) @ f(W["w_qP"])
+    for l in range(cfg.depth):
+        kP = np.stack([O.depth_rope(f(k), l, cfg.depth) for k in W["k_P"]])
+        z = q @ kP.T / np.sqrt(cfg.router_dim)
+        r = O.Oracle(cfg, W, threads=1).proj_route(l, xh)
+        assert np.array_equal(r["pidx"], np.argmax(z, axis=1))
+        assert np.allclose(r["psig"], 1 / (1 + np.exp(-z.max(1))), rtol=1e-12, atol=0)
+        assert np.allclose(r["pmargin"], z.max(1) - np.sort(z, axis=1)[:, -2], rtol=1e-9, atol=1e-12)
 
 
 def test_da_reshape_equals_explicit_loops():
