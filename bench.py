@@ -5,7 +5,10 @@ Metric: token-depth-steps per second (one unit = one token through one depth ste
 full L-depth forward, bf16, and its fraction of the roofline
 T_roof = max(F_alg / tensor peak, B_alg / HBM peak) with both peaks measured on this machine.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config small|medium|large|decode]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config large|medium|small|decode|...]
+
+The default workload is the large one (b 2, s 8192, h 2048, 16x128 heads, L 64, E 2048,
+k 8, m 64, 16 linear-MoE projection experts): the largest that runs on one GPU.
   python bench.py --impl reference ...     # the CPU oracle, timed on the host cores
 
 N > 1 runs one replica per GPU (torchrun, one rank per GPU): sequences are independent,
@@ -49,13 +52,17 @@ def peaks():
 
 
 def algorithmic(cfg, counts=None):
-    """Per-stage algorithmic FLOPs and HBM bytes of one full forward (or decode step).
-
-    FLOPs: every multiply-add of a contraction counted twice (SA causal half only, the router
-    at its plain 2 h d_r + 2 E d_r per token).  Bytes: weights read once per depth (routed
-    experts only: those the run's route counts touch), activations read and written once,
-    DA keys/values written once and re-read for every later depth, SA keys/values (prefill)
-    written and read once, the decode cache read once.  bf16 = 2 bytes."""
+    """Per-stage algorithmic FLOPs and HBM bytes of one full forward (or decode step), by the
+    accounting of the roofline: every multiply-add of a contraction counted twice at tensor
+    rate (SA over the causal half only; routers 2 h d_r + 2 E d_r per token; non-tensor math
+    not counted); bytes with perfect on-chip reuse inside a depth step and none across depths:
+    weights once per depth (every projection expert; only the routed experts the run's own
+    route counts touch), the residual x read and written once a depth, the DA keys/values
+    written once (4h bytes a token) and re-read by every later depth (4h l), the SA keys/values
+    written and read once (prefill) or the decode cache read once (4h per cached token).
+    Bytes are attributed to the stage that moves them: qkv (x^ in, projection weights, DA and
+    SA K/V out), da (earlier depths' K/V), sa (K/V in or the cache), o_proj and routers (their
+    weights), experts (touched expert weights), finish (x out).  2-byte bf16 values."""
     b, s, h, L = cfg.batch, cfg.seq, cfg.hidden, cfg.depth
     E, k, m, dr, P = cfg.n_experts, cfg.top_k, cfg.expert_hidden, cfg.router_dim, cfg.n_proj_experts
     T = cfg.tokens
@@ -69,27 +76,27 @@ def algorithmic(cfg, counts=None):
 
     no_da = cfg.variant == 3
     nq = 3 if no_da else 6                                        # projection widths / h
+    ko = 1 if no_da else 2                                        # O contraction width / h
     for l in range(L):
-        add("norm", 0.0, T * h * (es + es))                      # x in, x^ out
         if P > 0:
-            add("proj_route", 2.0 * T * h * dr + 2.0 * T * P * dr, T * h * es)
-        add("qkv", 2.0 * T * h * nq * h, T * h * es + G * nq * h * h * es + T * nq * h * es)
+            add("proj_route", 2.0 * T * h * dr + 2.0 * T * P * dr, (h * dr + P * dr) * es)
+        kv_out = (0 if no_da else 2 * T * h * es) + 2 * T * h * es   # DA and SA keys/values
+        add("qkv", 2.0 * T * h * nq * h, T * h * es + G * nq * h * h * es + kv_out)
         if not no_da:
             ctx = l + 1 if cfg.da_window <= 0 else min(l + 1, cfg.da_window)
-            add("da", 4.0 * T * h * ctx, T * h * es + T * 2 * h * es * (ctx - 1) + T * h * es)
+            add("da", 4.0 * T * h * ctx, 2.0 * T * h * es * (ctx - 1))
         if cfg.is_decode:
             n_ctx = cfg.cache_len + 1
-            add("sa", 4.0 * T * h * n_ctx, 2.0 * T * h * es * n_ctx + 2 * T * h * es)
+            add("sa", 4.0 * T * h * n_ctx, 2.0 * T * h * es * cfg.cache_len)
         else:
-            add("sa", 4.0 * h * b * s * (s + 1) / 2, 4.0 * T * h * es)
-        ko = 1 if no_da else 2                                    # O contraction width / h
-        add("o_proj", 2.0 * T * ko * h * h, T * ko * h * es + G * ko * h * h * es + T * h * (es + 4))
-        add("ea_route", 2.0 * T * h * dr + 2.0 * T * E * dr, T * h * es + h * dr * es + E * dr * es)
+            add("sa", 4.0 * h * b * s * (s + 1) / 2, 2.0 * T * h * es)
+        add("o_proj", 2.0 * T * ko * h * h, G * ko * h * h * es)
+        add("ea_route", 2.0 * T * h * dr + 2.0 * T * E * dr, (h * dr + E * dr) * es)
         touched = E
         if counts is not None:
             touched = int((np.asarray(counts)[l] > 0).sum())
-        add("experts", 4.0 * T * k * h * m,
-            2.0 * touched * h * m * es + T * h * es + T * h * 4 * 2)
+        add("experts", 4.0 * T * k * h * m, 2.0 * touched * h * m * es)
+        add("finish", 0.0, T * h * es)
     tot_f = sum(v[0] for v in st.values())
     tot_b = sum(v[1] for v in st.values())
     return st, tot_f, tot_b
@@ -99,6 +106,8 @@ def algorithmic(cfg, counts=None):
 # clocks sampled during the timed region
 
 class ClockSampler:
+    PERIOD_MS = 100
+    MIN_SAMPLES = 10   # fewer samples than this over the timed region: flagged as too short
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -114,7 +123,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -156,9 +165,12 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4)
                           if r[5 + i].lower() in ("active", "1")})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+        out = {"sm_mhz": statistics.median(sm) if sm else None,
+               "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+               "samples": len(rows), "period_ms": self.PERIOD_MS}
+        if len(rows) < self.MIN_SAMPLES:
+            out["too_short"] = True   # the median says little about the timed kernels' clock
+        return out
 
 
 # ----------------------------------------------------------------------------------------
@@ -273,9 +285,9 @@ def run_ours(args, cfg, rank, world, torch, dist):
     for name, ms in st["ms"].items():
         n = max(st["count"][name], 1)
         per_stage[name] = ms / max(args.steps, 1)
-    # the dominant kernel: the slowest stage that is a single kernel launch per depth
-    single = [k for k in ("qkv", "da", "sa", "o_proj", "finish") if per_stage.get(k, 0) > 0]
-    dominant = max(single or per_stage, key=lambda k: per_stage[k])
+    # the dominant stage: the slowest of all stages of the depth step
+    timed = [k for k in per_stage if per_stage[k] > 0 and k in stage_alg]
+    dominant = max(timed, key=lambda k: per_stage[k])
     fl, by = stage_alg.get(dominant, (0.0, 0.0))
     t_dom = per_stage[dominant] / 1e3  # s per forward
     bound_tensor = fl / (pk["tc"] * 1e12) > by / (pk["hbm"] * 1e9)
@@ -288,7 +300,8 @@ def run_ours(args, cfg, rank, world, torch, dist):
         achieved = by / t_dom / 1e9
         roof = dict(bound="hbm", achieved=achieved, peak=pk["hbm"], unit="GB/s",
                     frac=achieved / pk["hbm"])
-    roof.update(kernel=dominant, launches_per_step=launches_per_fwd,
+    roof.update(kernel=dominant, kernels=STAGE_KERNELS.get(dominant, dominant),
+                launches_per_step=launches_per_fwd,
                 traffic=measured_traffic(cfg.name, dominant),
                 peak_source=pk["source"] + " (MEASURED_PEAKS.json burst figure)")
 
@@ -343,14 +356,7 @@ def run_ours(args, cfg, rank, world, torch, dist):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
         "data": "synthetic (seeded N(0,1) inputs, N(0,1/fan_in) weights)",
-        "config": {"workload": workload_name(cfg), "global_batch": cfg.batch * world,
-                   "seq_len": cfg.seq, "depth": cfg.depth, "hidden": cfg.hidden,
-                   "heads": f"{cfg.n_heads}x{cfg.head_dim}", "experts": cfg.n_experts,
-                   "top_k": cfg.top_k, "expert_hidden": cfg.expert_hidden,
-                   "proj_experts": cfg.n_proj_experts,
-                   "units_per_step": cfg.units * world, "parallelism": f"dp{world} (replicas)",
-                   "l2": "flushed before every timed step (256 MB write, not timed)",
-                   "resident_bytes_per_gpu": resident},
+        "config": dict(config_dict(cfg, world), resident_bytes_per_gpu=resident),
         "roofline": roof,
         "roofline_step": {"t_roof_ms": t_roof * 1e3, "t_meas_ms": ms_step,
                           "frac": t_roof * 1e3 / ms_step, "F_alg": F, "B_alg": B,
@@ -362,6 +368,31 @@ def run_ours(args, cfg, rank, world, torch, dist):
         "clocks": clocks,
     }
     return out, model
+
+
+# kernels of each stage (bf16 path)
+STAGE_KERNELS = {
+    "qkv": "tc_gemm_kernel<EpiQKV>", "o_proj": "tc_gemm_kernel<EpiO>",
+    "sa": "tc_sa_kernel (prefill) / dec_bulk_kernel + attn_merge_kernel (decode)",
+    "da": "da_bulk_kernel", "proj_route": "tc_gemm_kernel<EpiProjRoute> + permute_kernel",
+    "ea_route": "tc_gemm_kernel<EpiRouterQ> + tc_gemm_kernel<EpiTopK> or route_q_topk_kernel "
+                "(decode: route_cluster_kernel)",
+    "permute": "permute_kernel",
+    "experts": "tc_gemm_kernel<EpiUp> + tc_gemm_kernel<EpiDownStore>, or tc_ffn_kernel "
+               "(decode: expert_rows_kernel)",
+    "finish": "combine_norm_kernel", "norm": "rmsnorm_kernel",
+}
+
+
+def config_dict(cfg, world=1):
+    """The `config` object of the JSON line (both arms)."""
+    return {"workload": workload_name(cfg), "global_batch": cfg.batch * world,
+            "seq_len": cfg.seq, "depth": cfg.depth, "hidden": cfg.hidden,
+            "heads": f"{cfg.n_heads}x{cfg.head_dim}", "experts": cfg.n_experts,
+            "top_k": cfg.top_k, "expert_hidden": cfg.expert_hidden,
+            "proj_experts": cfg.n_proj_experts, "units_per_step": cfg.units * world,
+            "parallelism": f"dp{world} (replicas)",
+            "l2": "flushed before every timed step (256 MB write, not timed)"}
 
 
 def workload_name(cfg):
@@ -379,60 +410,70 @@ def workload_name(cfg):
 # ----------------------------------------------------------------------------------------
 # the oracle on the host cores (cpu_baseline leg and the --impl reference arm)
 
-def oracle_sample(cfg, seconds_hint=20.0, threads=None):
-    """Time the oracle on a bounded sample of the workload: one sequence (or, for decode,
-    one sequence's step) through a few depths; returns units/s and a description."""
-    sys.path.insert(0, os.path.join(ROOT, "oracle"))
-    import oracle as O
-    threads = threads or os.cpu_count() or 1
-    W = inputs.host_weights(cfg)
-    if cfg.is_decode:
-        one = cfg.with_(batch=1)
-        o = O.Oracle(one, W, threads=threads)
-        L, H, d = cfg.depth, cfg.n_heads, cfg.head_dim
-        cap = cfg.cache_len + 1
-        spec_k = [s for s in inputs.input_specs(cfg) if s.name == "k_cache"][0]
-        kc = np.zeros((L, H, cap, d))
-        vc = np.zeros((L, H, cap, d))
-        x = inputs.host_inputs(one)["x0"][0] if False else inputs.draw(
-            [s for s in inputs.input_specs(cfg) if s.name == "x0"][0], cfg.seed, 0, cfg.hidden)
+class OracleSampler:
+    """The oracle on the host cores (all of them, OpenMP), on a bounded sample of the
+    workload: for prefill the first S' <= 1024 tokens of one sequence (causal SA makes them an
+    exact part of the workload) through its first depths, for decode one sequence's whole
+    step.  Weights are drawn once; sample() returns (units/s, description)."""
+
+    def __init__(self, cfg, threads=None):
+        sys.path.insert(0, os.path.join(ROOT, "oracle"))
+        import oracle as O
+        self.cfg = cfg
+        self.threads = threads or os.cpu_count() or 1
+        W = inputs.host_weights(cfg)
+        self.one = cfg.with_(batch=1) if cfg.is_decode else cfg.with_(batch=1, seq=min(cfg.seq, 1024))
+        self.o = O.Oracle(self.one, W, threads=self.threads)
+
+    def sample(self, seconds_hint=20.0):
+        cfg, one, o = self.cfg, self.one, self.o
+        if cfg.is_decode:
+            L, H, d = cfg.depth, cfg.n_heads, cfg.head_dim
+            cap = cfg.cache_len + 1
+            kc = np.zeros((L, H, cap, d))
+            vc = np.zeros((L, H, cap, d))
+            x = inputs.draw([s for s in inputs.input_specs(cfg) if s.name == "x0"][0], cfg.seed,
+                            0, cfg.hidden)
+            t0 = time.perf_counter()
+            o.decode_seq(x, kc, vc, cfg.cache_len)
+            dt = time.perf_counter() - t0
+            return cfg.depth / dt, f"one sequence's decode step (all {cfg.depth} depths, " \
+                                   f"cache {cfg.cache_len}, zero cache contents)"
+        x = inputs.host_inputs(one)["x0"]
         t0 = time.perf_counter()
-        o.decode_seq(x, kc, vc, cfg.cache_len)
+        depths = 0
+        da = np.zeros((one.tokens, cfg.depth, 2, cfg.hidden))
+        while depths < cfg.depth:
+            r = o.forward(x, depths, depths + 1, da_kv=da, trace=False)
+            x = inputs.round_to(r["x_out"], cfg.dtype)
+            da = r["da_kv"]
+            depths += 1
+            if time.perf_counter() - t0 > seconds_hint:
+                break
         dt = time.perf_counter() - t0
-        return 1 * cfg.depth / dt, f"one sequence's decode step (all {cfg.depth} depths, cache " \
-                                   f"{cfg.cache_len}), zero cache contents", threads
-    # prefill: one sequence of S tokens, first depths until ~seconds_hint
-    one = cfg.with_(batch=1)
-    o = O.Oracle(one, W, threads=threads)
-    x = inputs.host_inputs(one)["x0"]
-    t0 = time.perf_counter()
-    depths = 0
-    da = np.zeros((one.tokens, cfg.depth, 2, cfg.hidden))
-    while depths < cfg.depth:
-        r = o.forward(x, depths, depths + 1, da_kv=da, trace=False)
-        x = r["x_out"].astype(np.float32)
-        da = r["da_kv"]
-        depths += 1
-        if time.perf_counter() - t0 > seconds_hint:
-            break
-    dt = time.perf_counter() - t0
-    return one.tokens * depths / dt, f"one sequence ({one.tokens} tokens) through depths " \
-                                     f"0..{depths - 1} of {cfg.depth}", threads
+        return one.tokens * depths / dt, f"the first {one.tokens} of {cfg.seq} tokens of one " \
+                                         f"sequence through depths 0..{depths - 1} of {cfg.depth}"
 
 
 def run_reference(args, cfg):
-    v, sample, cores = oracle_sample(cfg, seconds_hint=max(5.0, 20.0 / max(args.steps, 1)))
-    vals = [v]
-    for _ in range(max(args.steps, 1) - 1):
-        vv, _, _ = oracle_sample(cfg, seconds_hint=max(5.0, 20.0 / max(args.steps, 1)))
-        vals.append(vv)
+    """The reference arm: the oracle, as it stands, on the host cores; each of the K timed steps
+    is one bounded sample of the workload (W untimed warm-up samples first)."""
+    smp = OracleSampler(cfg)
+    hint = max(2.0, 60.0 / max(args.steps + args.warmup, 1))
+    for _ in range(args.warmup):
+        smp.sample(seconds_hint=hint)
+    vals = []
+    for _ in range(max(args.steps, 1)):
+        v, sample = smp.sample(seconds_hint=hint)
+        vals.append(v)
+    cores = smp.threads
     value = statistics.median(vals)
     return {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": workload_name(cfg)},
+        "config": config_dict(cfg, 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -447,7 +488,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="small", choices=sorted(configs.CONFIGS))
+    ap.add_argument("--config", default="large", choices=sorted(configs.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     cfg = configs.CONFIGS[args.config]
@@ -473,9 +514,10 @@ def main():
     out, model = run_ours(args, cfg, rank, world, torch, dist)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            v, sample, cores = oracle_sample(cfg)
-            out["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                   "sample": sample}
+            smp = OracleSampler(cfg)
+            v, sample = smp.sample()
+            out["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": smp.threads,
+                                   "kind": "oracle", "sample": sample}
         print(json.dumps(out))
     model.close()
     if dist is not None:

@@ -1,5 +1,6 @@
-"""Build libdreamer.so (the product) and libdreamer_inputs.so (seeded input generator) for
-sm_100a with nvcc, in-tree."""
+"""Build libdreamer.so (the product), libdreamer_inputs.so (seeded input generator) and
+libdreamer_testhooks.so (test infrastructure: the product's sources with the timeout-test hook
+and a 20 ms device wait limit) for sm_100a with nvcc, in-tree."""
 import os
 import subprocess
 import sys
@@ -38,6 +39,15 @@ def build(force: bool = False, verbose: bool = False) -> list:
             print(" ".join(cmd))
         subprocess.run(cmd, check=True)
     outs.append(lib)
+    hooks = os.path.join(HERE, "libdreamer_testhooks.so")
+    if force or not _newer(hooks, deps):
+        cmd = ["nvcc", *ARCH, *FLAGS, "-DDREAMER_TEST_HOOKS",
+               "-DDREAMER_WAIT_LIMIT_NS=20000000ull", "-o", hooks,
+               os.path.join(CSRC, "dreamer.cu"), os.path.join(CSRC, "route_noalloc.cu")]
+        if verbose:
+            print(" ".join(cmd))
+        subprocess.run(cmd, check=True)
+    outs.append(hooks)
     gen = os.path.join(HERE, "libdreamer_inputs.so")
     src = os.path.join(CSRC, "inputs_gen.cu")
     if force or not _newer(gen, [src]):

@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
       const uint64_t t0 = tcda::gtimer();
       while (!tcda::try_wait(bar, par)) {
         if (abort_flag) break;
-        if (tcda::gtimer() - t0 > 2000000000ull) {
+        if (tcda::gtimer() - t0 > DREAMER_WAIT_LIMIT_NS) {
           abort_flag = 1;
           raise_dev_error(a.err, DEV_TIMEOUT);
           break;
@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
     for (int j = consumed; j < issued; j++) {
       const uint64_t t0 = tcda::gtimer();
       while (!tcda::try_wait(tcda::smem_u32(&bars[j % NB]), (uint32_t)((j / NB) & 1)) &&
-             tcda::gtimer() - t0 < 2000000000ull) {
+             tcda::gtimer() - t0 < DREAMER_WAIT_LIMIT_NS) {
       }
     }
   }
@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(256) dec_bulk_kernel(DecBulkArgs a) {
       const uint64_t t0 = tcda::gtimer();
       while (!tcda::try_wait(bar, par)) {
         if (abort_flag) break;
-        if (tcda::gtimer() - t0 > 2000000000ull) {
+        if (tcda::gtimer() - t0 > DREAMER_WAIT_LIMIT_NS) {
           abort_flag = 1;
           raise_dev_error(a.err, DEV_TIMEOUT);
           break;
@@ -592,7 +592,7 @@ __global__ void __launch_bounds__(256) dec_bulk_kernel(DecBulkArgs a) {
     for (int c = consumed; c < issued; c++) {
       const uint64_t t0 = tcda::gtimer();
       while (!tcda::try_wait(tcda::smem_u32(&bars[c % NST]), (uint32_t)((c / NST) & 1)) &&
-             tcda::gtimer() - t0 < 2000000000ull) {
+             tcda::gtimer() - t0 < DREAMER_WAIT_LIMIT_NS) {
       }
     }
   }

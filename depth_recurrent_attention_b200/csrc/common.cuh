@@ -72,6 +72,14 @@ __device__ __forceinline__ void prefetch_l2(const void *p) {
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
 
+// Routing weights w_s = sigmoid(z_s) / sum_j sigmoid(z_j) over a token's picks, formed as
+// exp(ls_s - m) / sum_j exp(ls_j - m) from ls = log sigmoid(z) = min(z, 0) - log(1 + e^-|z|)
+// and m = max_j ls_j: the same ratio, finite for every finite z (sigmoids that underflow to
+// 0 would give 0/0).
+__device__ __forceinline__ float log_sigmoidf_(float z) {
+  return fminf(z, 0.f) - log1pf(expf(-fabsf(z)));
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -96,6 +104,13 @@ __device__ __forceinline__ void pdl_trigger() {
 
 // Device-side error codes written into the handle's flag word (first writer wins).
 enum DevErr : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_INDEX = 2 };
+
+// Limit of every bounded device wait (an mbarrier phase, copies in flight), in nanoseconds of
+// %globaltimer; on expiry a kernel sets DEV_TIMEOUT and winds down.  The test-hook build
+// shortens it so that its timeout test ends quickly.
+#ifndef DREAMER_WAIT_LIMIT_NS
+#define DREAMER_WAIT_LIMIT_NS 2000000000ull
+#endif
 __device__ __forceinline__ void raise_dev_error(int *flag, int code) {
   if (flag) atomicCAS(flag, 0, code);
 }

@@ -52,7 +52,11 @@ struct dreamer_handle {
   void *kEt = nullptr;           // [d_r][E] bf16: router keys transposed (CUDA-core scores)
   int num_sms = 148;
   int qkv_perm = 0;  // q_SA / k_SA columns of the fused QKV weight in EpiQKV perm order
-  int use_tc = 1;  // bf16 contractions on tcgen05 (0: CUDA cores, for cross-checks)
+  int prefill_ok = 1;  // bf16: the prefill shapes are ones the tcgen05 kernels take
+#ifdef DREAMER_TEST_HOOKS
+  int inject_skip = 0;  // the next QKV GEMM's TMA producer issues no loads (timeout test)
+#endif
+  int path_err = 0;    // a bf16 step found no kernel for its shape while enqueuing (a bug)
   std::vector<void *> allocs;
   int *err_host = nullptr;       // pinned copy of the device error flag (async)
   cudaStream_t side = nullptr;   // second stream: DA runs beside SA
@@ -66,7 +70,7 @@ struct dreamer_handle {
     int l0, l1, prof;
     int captured;                // 0: seen once (ran directly), 1: graph ready
     cudaGraphExec_t exec;
-    uint64_t launches;
+    uint64_t launches, launches_tc, launches_simt;
     std::vector<cudaEvent_t> evs;
     std::vector<int> stages;
     uint64_t last_use;
@@ -74,7 +78,7 @@ struct dreamer_handle {
   std::vector<GraphEntry> graphs;
   uint64_t use_clock = 0;
   // instrumentation
-  uint64_t launches = 0;
+  uint64_t launches = 0, launches_tc = 0, launches_simt = 0;
   int prof = 0;
   std::vector<cudaEvent_t> ev;
   std::vector<int> ev_stage;
@@ -140,8 +144,11 @@ static int dalloc(dreamer_handle *h, void **p, size_t bytes) {
   } while (0)
 
 static inline int cdiv(long a, long b) { return (int)((a + b - 1) / b); }
-// kernels launched by this thread through the library (read as deltas around each call)
+// kernels launched by this thread through the library (read as deltas around each call):
+// all of them, the tcgen05 ones, and the generic CUDA-core GEMM / attention / top-k kernels
 static thread_local uint64_t g_launches = 0;
+static thread_local uint64_t g_launches_tc = 0;
+static thread_local uint64_t g_launches_simt = 0;
 
 // ---- kernel launches with programmatic dependent launch -------------------------------
 // A kernel may start while the previous operation on its stream is still running only if that
@@ -192,6 +199,7 @@ static void launch_k(dreamer_handle *h, void (*kern)(P...), dim3 grid, dim3 bloc
 
 // top-k: eight warps a token when there are too few tokens to fill the GPU with one warp each
 static void launch_topk(dreamer_handle *h, const TopkArgs &t, cudaStream_t s) {
+  ++g_launches_simt;
   if ((long)t.n_tok * 4 < (long)h->num_sms * 32)
     launch_k(h, topk_kernel<8>, dim3(t.n_tok), dim3(256), 0, s, t);
   else
@@ -230,7 +238,17 @@ static int validate(const dreamer_config *c) {
   if (c->top_k > 16 || c->n_experts > 65536 || c->n_proj_experts > 64) return DREAMER_ERR_UNSUPPORTED;
   if (c->expert_hidden % 16 || c->router_dim % 16 || c->router_dim > 256 || c->hidden % 64)
     return DREAMER_ERR_UNSUPPORTED;
-  if (c->depth > 1024) return DREAMER_ERR_UNSUPPORTED;
+  if (c->depth > 1024 || c->hidden > 4096) return DREAMER_ERR_UNSUPPORTED;
+  if (c->dtype == 1) {
+    // bf16 runs only on the tcgen05 kernels and the purpose-built streaming kernels: shapes
+    // they do not take are refused here instead of being routed to CUDA-core fallbacks
+    if (d != 64 && d != 128) return DREAMER_ERR_UNSUPPORTED;             // GEMM / flash SA
+    if (c->hidden % 256 || c->n_heads > 32) return DREAMER_ERR_UNSUPPORTED;  // N tiles; DA CTA
+    const int m = c->expert_hidden;
+    if (m != 16 && m != 32 && m != 64) return DREAMER_ERR_UNSUPPORTED;     // expert FFN
+    if (c->router_dim != 64 && c->router_dim != 128) return DREAMER_ERR_UNSUPPORTED;
+    if (c->n_experts % 4) return DREAMER_ERR_UNSUPPORTED;                  // router scorer
+  }
   return DREAMER_OK;
 }
 
@@ -326,6 +344,7 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     const int hd = c.hidden, E = c.n_experts, m = c.expert_hidden, dr = c.router_dim;
     const int P = c.n_proj_experts, G = P > 0 ? P : 1, L = c.depth, d = c.head_dim;
     h->esz = c.dtype == 0 ? 4 : 2;
+    h->prefill_ok = c.dtype == 0 || c.seq % 128 == 0;  // bf16 flash SA: 128-token query tiles
     h->T = c.batch * c.seq > c.batch ? c.batch * c.seq : c.batch;
     h->max_pos = c.seq > c.max_cache_len ? c.seq : c.max_cache_len;
     h->ldz = round8(E);
@@ -338,7 +357,6 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
           cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
         h->num_sms = sms;
     }
-    if (const char *ev = getenv("DREAMER_NO_TC")) h->use_tc = atoi(ev) ? 0 : 1;
     if (const char *ev = getenv("DREAMER_NO_GRAPH")) h->use_graph = atoi(ev) ? 0 : 1;
     if (const char *ev = getenv("DREAMER_NO_PDL")) h->use_pdl = atoi(ev) ? 0 : 1;
     CK(cudaHostAlloc((void **)&h->err_host, sizeof(int), cudaHostAllocDefault));
@@ -471,12 +489,16 @@ extern "C" int dreamer_get_stats(dreamer_handle *h, dreamer_stats *out, int rese
   }
   h->ev_used = 0;
   out->launches = h->launches;
+  out->launches_tc = h->launches_tc;
+  out->launches_simt = h->launches_simt;
   for (int i = 0; i < DREAMER_N_STAGES; i++) {
     out->ms[i] = h->stage_ms[i];
     out->count[i] = h->stage_count[i];
   }
   if (reset) {
     h->launches = 0;
+    h->launches_tc = 0;
+    h->launches_simt = 0;
     for (int i = 0; i < DREAMER_N_STAGES; i++) {
       h->stage_ms[i] = 0;
       h->stage_count[i] = 0;
@@ -508,6 +530,7 @@ template <typename TA, typename TB, int SEG, class Epi>
 static void gemm_simt(const GemmArgs &a, int max_tiles, const Epi &epi, cudaStream_t s) {
   dim3 grid(max_tiles, cdiv(a.N, 128));
   ++g_launches;
+  ++g_launches_simt;
   gemm_simt_kernel<TA, TB, SEG, Epi><<<grid, 256, 0, s>>>(a, epi);
 }
 
@@ -523,6 +546,7 @@ template <typename T>
 static void launch_attn(const AttnArgs &a, int d, cudaStream_t s) {
   const int warps = a.n_q * a.H;
   const int blocks = cdiv(warps, 8);
+  ++g_launches_simt;
   switch (d) {
     case 16: ++g_launches; attn_warp_kernel<T, 16><<<blocks, 256, 0, s>>>(a); break;
     case 32: ++g_launches; attn_warp_kernel<T, 32><<<blocks, 256, 0, s>>>(a); break;
@@ -600,9 +624,13 @@ static void launch_rows(dreamer_handle *h, const RowsArgs &a, int d, cudaStream_
   }
   if (a.mode == 2) {
     launch_dec_bulk<T>(h, a, d, s);
+  } else if (sizeof(T) == 2) {
+    h->path_err = 1;  // bf16 depth attention is the bulk-copy kernel only
+    return;
   } else {
     const long warps = (long)a.n_q * a.H;
     const int blocks = cdiv(warps, 8);
+    ++g_launches_simt;
     switch (d) {
       case 16: launch_k(h, attn_rows_kernel<T, 16, 4>, dim3(blocks), dim3(256), 0, s, a); break;
       case 32: launch_k(h, attn_rows_kernel<T, 32, 4>, dim3(blocks), dim3(256), 0, s, a); break;
@@ -652,10 +680,12 @@ static void route_rows(dreamer_handle *h, int mode, int l, const void *X, int n,
               (const T *)h->kE_raw, (const float2 *)(h->rope_dr + (size_t)l * (dr / 2)), t);
     return;
   }
-  if (mode == 0 && h->use_tc && c.dtype == 1 && tc_route_ok(h) &&
-      tc_route(h, l, X, n, idx, wout, counts_a, counts_b, s))
+  if (c.dtype == 1) {
+    // bf16: query GEMM on tcgen05, then the fused top-k score GEMM or the warp scorer
+    if (!(mode == 0 && tc_route(h, l, X, n, idx, wout, counts_a, counts_b, s))) h->path_err = 1;
     return;
-  // q = X W_q (fp32 accumulation), z = q . k~ (fp32), on CUDA cores
+  }
+  // float32: q = X W_q (fp32 accumulation), z = q . k~ (fp32), on CUDA cores
   GemmArgs a = dense_args(n, dr, hd, X, hd, Wq, hd);
   gemm_simt<T, T, 8>(a, cdiv(n, 64), EpiStoreF32{h->qbuf, dr, dr}, s);
   GemmArgs b = dense_args(n, E, dr, h->qbuf, dr, krot, dr);
@@ -689,6 +719,16 @@ static void trace_depth(dreamer_handle *h, const dreamer_trace *tr, int l, int n
     if (tr->pidx) cudaMemcpyAsync(tr->pidx + off, h->pidx, n * sizeof(int), cudaMemcpyDeviceToDevice, s);
     if (tr->psig) cudaMemcpyAsync(tr->psig + off, h->psig, n * sizeof(float), cudaMemcpyDeviceToDevice, s);
   }
+  // the residual accumulator holds y_l in float32 between the O projection and the combine
+  if (tr->y_f32) cudaMemcpyAsync(tr->y_f32 + off * hd, h->acc, n * hd * sizeof(float), cudaMemcpyDeviceToDevice, s);
+}
+
+// after the combine: the accumulator holds x_{l+1} in float32
+static void trace_next(dreamer_handle *h, const dreamer_trace *tr, int l, int n, cudaStream_t s) {
+  if (!tr || !tr->x_f32) return;
+  pdl_break(h, s);
+  const size_t hd = h->cfg.hidden, off = (size_t)l * n;
+  cudaMemcpyAsync(tr->x_f32 + off * hd, h->acc, n * hd * sizeof(float), cudaMemcpyDeviceToDevice, s);
 }
 
 struct DepthIO {
@@ -710,7 +750,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   const int hd = c.hidden, d = c.head_dim, L = c.depth, E = c.n_experts, k = c.top_k;
   const int m = c.expert_hidden, P = c.n_proj_experts, G = P > 0 ? P : 1;
   const int n = io.n_tok;
-  const bool tc = h->use_tc && c.dtype == 1;
+  const bool tc = c.dtype == 1;  // bf16: tcgen05 and streaming kernels only
 
   // 1. RMSNorm of the residual stream on the first depth of the call (later depths get x^
   // from the previous depth's fused combine + norm)
@@ -724,8 +764,10 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   if (P > 0) {
     mark(h, s, DREAMER_STAGE_PROJ_ROUTE);
     // pcnt / pcursor are zero here: cleared at init and by every depth's combine kernel
-    if (!(tc && tc_proj_route(h, l, h->xh, n, s)))
+    if (!tc)
       route_rows<T>(h, 1, l, h->xh, n, h->pidx, h->psig, nullptr, h->pcnt, s);
+    else if (!tc_proj_route(h, l, h->xh, n, s))
+      h->path_err = 1;
     launch_k(h, permute_kernel, dim3(cdiv(n, 1024)), dim3(1024), (size_t)(G + 1) * sizeof(int), s,
              (const int *)h->pcnt, G, (const int *)h->pidx, n, h->poffs, h->ptiles_a, 64,
              h->ptiles_b, 128, h->pcursor, h->prows, h->pinv);
@@ -774,7 +816,10 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
       launch_rows<T>(h, sd, d, st);
       return;
     }
-    if (!(tc && tc_sa_ok(h) && tc_sa(h, st))) launch_attn<T>(sa, d, st);
+    if (!tc)
+      launch_attn<T>(sa, d, st);
+    else if (!(tc_sa_ok(h) && tc_sa(h, st)))
+      h->path_err = 1;
   };
   auto qkv_gemm = [&](const void *A, int col0, int ncols) {
     // columns [col0, col0 + ncols) of the fused QKV projection
@@ -783,7 +828,10 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
                          (long)6 * hd * hd);
     EpiQKV<T> e2 = eq;
     e2.col_lo = col0;
-    if (tc && tc_gemm_ok(h, a) && tc_gemm_qkv(h, a, e2, s)) return;
+    if (tc) {
+      if (!(tc_gemm_ok(h, a) && tc_gemm_qkv(h, a, e2, s))) h->path_err = 1;
+      return;
+    }
     switch (d) {
       case 16: gemm_qkv<T, 16>(h, a, ptiles, e2, s); break;
       case 32: gemm_qkv<T, 32>(h, a, ptiles, e2, s); break;
@@ -801,7 +849,10 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     a.ldb = 2 * hd;
     EpiO<T> eo{hd, psig, res_mode, (const T *)io.x_in, h->inv_rms, (const T *)h->g,
                (T *)yout, h->acc};
-    if (tc && tc_gemm_ok(h, a) && tc_gemm_o(h, a, eo, s)) return;
+    if (tc) {
+      if (!(tc_gemm_ok(h, a) && tc_gemm_o(h, a, eo, s))) h->path_err = 1;
+      return;
+    }
     gemm_simt<T, T, 16>(a, ptiles, eo, s);
   };
 
@@ -877,7 +928,9 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
                         : (m == 32 ? expert_rows_kernel<T, 32> : expert_rows_kernel<T, 64>);
     launch_k(h, kern, dim3(n * k), dim3(256), 0, s, (const T *)ein, (const int *)h->eidx,
              n * k, k, hd, (const T *)h->w1_t, (const T *)h->w2_t, (T *)h->Ybuf);
-  } else if (!(tc && tc_expert_ok(h) && tc_expert(h, ein, n, s))) {
+  } else if (tc) {
+    if (!(tc_expert_ok(h) && tc_expert(h, ein, n, s))) h->path_err = 1;
+  } else {
     const int etiles = cdiv((long)n * k, 64) + E;
     GemmArgs up{};
     up.N = m; up.K = hd; up.G = E; up.M = n * k; up.goffs = h->eoffs; up.tile_offs = h->etiles_a;
@@ -901,6 +954,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
            (const T *)h->g, (T *)h->xh,
            h->inv_rms, last ? (T *)io.x_out : (T *)nullptr, n, hd, c.rms_eps, h->ecnt, 2 * E,
            h->pcnt, P > 0 ? 2 * (G + 1) : 0);
+  trace_next(h, io.tr, l, n, s);
 }
 
 // The device error flag is copied to pinned host memory at the end of every call; the next
@@ -941,6 +995,9 @@ template <class F>
 static int run_graphed(dreamer_handle *h, int kind, const void *const key[5], int l0, int l1,
                        cudaStream_t s, F &&enqueue) {
   if (!h->use_graph) return enqueue();
+#ifdef DREAMER_TEST_HOOKS
+  if (h->inject_skip) return enqueue();  // an injected call runs directly, never from a graph
+#endif
   dreamer_handle::GraphEntry *e = nullptr;
   for (auto &g : h->graphs)
     if (g.kind == kind && g.l0 == l0 && g.l1 == l1 && g.prof == h->prof &&
@@ -969,7 +1026,7 @@ static int run_graphed(dreamer_handle *h, int kind, const void *const key[5], in
   e->last_use = ++h->use_clock;
   if (!e->captured) {
     const size_t ev0 = h->ev_used;
-    const uint64_t l_before = g_launches;
+    const uint64_t l_before = g_launches, tc_before = g_launches_tc, simt_before = g_launches_simt;
     cudaGraph_t graph = nullptr;
     if (cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
       cudaGetLastError();
@@ -978,9 +1035,12 @@ static int run_graphed(dreamer_handle *h, int kind, const void *const key[5], in
     int rc = enqueue();
     cudaError_t ce = cudaStreamEndCapture(s, &graph);
     const uint64_t n_launch = g_launches - l_before;
-    g_launches = l_before;  // captured kernels run when the graph is launched
+    const uint64_t n_tc = g_launches_tc - tc_before, n_simt = g_launches_simt - simt_before;
+    // captured kernels run when the graph is launched
+    g_launches = l_before;
+    g_launches_tc = tc_before;
+    g_launches_simt = simt_before;
     if (rc != DREAMER_OK || ce != cudaSuccess || !graph) {
-      g_launches = l_before;
       if (graph) cudaGraphDestroy(graph);
       cudaGetLastError();
       h->ev_used = ev0;
@@ -997,6 +1057,8 @@ static int run_graphed(dreamer_handle *h, int kind, const void *const key[5], in
     }
     e->captured = 1;
     e->launches = n_launch;
+    e->launches_tc = n_tc;
+    e->launches_simt = n_simt;
     // the graph records into the events its marks captured: they now belong to it
     e->evs.assign(h->ev.begin() + ev0, h->ev.begin() + h->ev_used);
     e->stages.assign(h->ev_stage.begin() + ev0, h->ev_stage.begin() + h->ev_used);
@@ -1006,6 +1068,8 @@ static int run_graphed(dreamer_handle *h, int kind, const void *const key[5], in
   }
   CK(cudaGraphLaunch(e->exec, s));
   g_launches += e->launches;
+  g_launches_tc += e->launches_tc;
+  g_launches_simt += e->launches_simt;
   if (e->prof && !e->evs.empty()) {
     CK(cudaStreamSynchronize(s));
     accumulate_marks(h, e->evs, e->stages);
@@ -1028,7 +1092,9 @@ static int forward_impl(dreamer_handle *h, const void *x_in, void *x_out, int l0
   DepthIO io{};
   io.mode = 0; io.n_tok = n; io.x_in = x_in; io.x_out = x_out; io.tr = tr;
   io.da_kv = da_kv ? da_kv : h->da_kv_int;
+  h->path_err = 0;
   for (int l = l0; l < l1; l++) run_depth<T>(h, l, l == l0, l == l1 - 1, io, s);
+  if (h->path_err) return DREAMER_ERR_UNSUPPORTED;
   if (l1 == l0 && x_out != x_in) {
     CK(cudaMemcpyAsync(x_out, x_in, (size_t)n * c.hidden * h->esz, cudaMemcpyDeviceToDevice, s));
   }
@@ -1046,6 +1112,7 @@ extern "C" int dreamer_core_forward(dreamer_handle *h, const void *x_in, void *x
   if (depth_begin < 0 || depth_end > c.depth || depth_begin > depth_end) return DREAMER_ERR_ARG;
   if (!da_kv && depth_begin != 0 && c.variant != 3) return DREAMER_ERR_ARG;
   if (!aligned16(x_in) || !aligned16(x_out) || (da_kv && !aligned16(da_kv))) return DREAMER_ERR_ARG;
+  if (!h->prefill_ok) return DREAMER_ERR_UNSUPPORTED;
   int e = check_dev_error(h);
   if (e) return e;
   cudaStream_t s = (cudaStream_t)stream;
@@ -1053,7 +1120,7 @@ extern "C" int dreamer_core_forward(dreamer_handle *h, const void *x_in, void *x
     return c.dtype == 0 ? forward_impl<float>(h, x_in, x_out, depth_begin, depth_end, da_kv, trace, s)
                         : forward_impl<bf16>(h, x_in, x_out, depth_begin, depth_end, da_kv, trace, s);
   };
-  const uint64_t l0c = g_launches;
+  const uint64_t l0c = g_launches, l0tc = g_launches_tc, l0simt = g_launches_simt;
   int rc;
   if (trace) {
     rc = enqueue();
@@ -1062,6 +1129,8 @@ extern "C" int dreamer_core_forward(dreamer_handle *h, const void *x_in, void *x
     rc = run_graphed(h, 0, key, depth_begin, depth_end, s, enqueue);
   }
   h->launches += g_launches - l0c;
+  h->launches_tc += g_launches_tc - l0tc;
+  h->launches_simt += g_launches_simt - l0simt;
   return rc;
 }
 
@@ -1081,7 +1150,9 @@ static int decode_impl(dreamer_handle *h, const void *x_new, void *kc, void *vc,
   io.mode = 1; io.n_tok = n; io.x_in = x_new; io.x_out = x_out; io.tr = tr;
   io.da_kv = h->da_kv_int;
   io.k_cache = kc; io.v_cache = vc; io.cache_len = len;
+  h->path_err = 0;
   for (int l = 0; l < c.depth; l++) run_depth<T>(h, l, l == 0, l == c.depth - 1, io, s);
+  if (h->path_err) return DREAMER_ERR_UNSUPPORTED;
   CK(cudaMemcpyAsync(h->err_host, h->err, sizeof(int), cudaMemcpyDeviceToHost, s));
   mark(h, s, DREAMER_N_STAGES);
   CK(cudaGetLastError());
@@ -1103,7 +1174,7 @@ extern "C" int dreamer_decode_step(dreamer_handle *h, const void *x_new, void *k
                ? decode_impl<float>(h, x_new, k_cache, v_cache, cache_len, x_out, trace, s)
                : decode_impl<bf16>(h, x_new, k_cache, v_cache, cache_len, x_out, trace, s);
   };
-  const uint64_t l0c = g_launches;
+  const uint64_t l0c = g_launches, l0tc = g_launches_tc, l0simt = g_launches_simt;
   int rc;
   if (trace) {
     rc = enqueue();
@@ -1112,6 +1183,8 @@ extern "C" int dreamer_decode_step(dreamer_handle *h, const void *x_new, void *k
     rc = run_graphed(h, 1, key, 0, h->cfg.depth, s, enqueue);
   }
   h->launches += g_launches - l0c;
+  h->launches_tc += g_launches_tc - l0tc;
+  h->launches_simt += g_launches_simt - l0simt;
   return rc;
 }
 
@@ -1139,10 +1212,12 @@ extern "C" int dreamer_route_experts(dreamer_handle *h, int depth, const void *y
   cudaStream_t s = (cudaStream_t)stream;
   if (counts) CK(cudaMemsetAsync(counts, 0, h->cfg.n_experts * sizeof(int), s));
   pdl_break(h, s);  // the caller's stream: whatever ran last is not ours
+  h->path_err = 0;
   if (h->cfg.dtype == 0)
     route_rows<float>(h, 0, depth, y, n_tokens, idx, w, counts, nullptr, s);
   else
     route_rows<bf16>(h, 0, depth, y, n_tokens, idx, w, counts, nullptr, s);
+  if (h->path_err) return DREAMER_ERR_UNSUPPORTED;
   CK(cudaGetLastError());
   return DREAMER_OK;
 }
@@ -1186,6 +1261,17 @@ extern "C" int dreamer_bias_update(dreamer_handle *h, float lambda, float *bias_
   if (!h) return DREAMER_ERR_ARG;
   return launch_bias_update(h, h->counts, h->cfg.depth, lambda, bias_out, (cudaStream_t)stream);
 }
+
+#ifdef DREAMER_TEST_HOOKS
+// Test-hook build only (not in libdreamer.so): what = 1 makes the TMA producer of the next
+// call's first QKV projection GEMM issue no loads, so that its MMA issuer's bounded wait
+// expires; the call's error then surfaces as DREAMER_ERR_TIMEOUT.
+extern "C" int dreamer_test_inject(dreamer_handle *h, int what) {
+  if (!h || what < 0 || what > 1) return DREAMER_ERR_ARG;
+  h->inject_skip = what;
+  return DREAMER_OK;
+}
+#endif
 
 extern "C" int dreamer_bias_update_counts(dreamer_handle *h, float lambda, const int32_t *counts,
                                           int n_rows, float *bias_out, dreamer_stream stream) {

@@ -664,8 +664,9 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(float *acc, const T *
       xv[ci * 8 + j] = x[j];
       ss += x[j] * x[j];
     }
+    // the accumulator always keeps x_{l+1} in fp32 (the last depth also stores it rounded)
     if (x_out) store8(x_out + (long)warp * h + c, x);
-    else store8(acc + (long)warp * h + c, x);
+    store8(acc + (long)warp * h + c, x);
   }
   if (x_out) return;
   ss = warp_sum(ss);
@@ -900,11 +901,14 @@ struct WarpTopK {
 // normalised over the k in mode 0) and count them.
 __device__ __forceinline__ void emit_topk(int lane, int k, float v, int e, float z, long tok,
                                           int mode, int *idx, float *w, int *ca, int *cb) {
-  const float sg = lane < k ? 1.0f / (1.0f + __expf(-z)) : 0.f;
-  const float ssum = warp_sum(sg);
+  // mode 0: normalised routing weights (stable form); mode 1: the projection weight sigmoid(z)
+  const float ls = lane < k ? log_sigmoidf_(z) : -INFINITY;
+  const float m = warp_max(ls);
+  const float ex = lane < k ? expf(ls - m) : 0.f;
+  const float ssum = warp_sum(ex);
   if (lane < k) {
     idx[tok * k + lane] = e;
-    w[tok * k + lane] = mode == 0 ? sg / ssum : sg;
+    w[tok * k + lane] = mode == 0 ? ex / ssum : 1.0f / (1.0f + expf(-z));
     if (ca) atomicAdd(ca + e, 1);
     if (cb) atomicAdd(cb + e, 1);
   }

@@ -13,7 +13,10 @@
 // it keeps the previous call's contents, so calls that overlap on the GPU (two streams, or two
 // host threads) race on it: serialise them.  The first call on a device looks up the array's
 // device address (cudaGetSymbolAddress) and caches it; make that first call before any stream
-// capture on that device.
+// capture on that device.  The cached address belongs to the CUDA context current at that
+// first call: it is keyed by device and context, so a new context on the device (after
+// cudaDeviceReset, or another context made current) looks the address up again.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -30,20 +33,42 @@ static __device__ __align__(256) float g_route_scratch[ROUTE_NOALLOC_SCRATCH_FLO
 
 constexpr int MAX_DEVICES = 64;
 static float *g_scratch_addr[MAX_DEVICES] = {nullptr};
+static void *g_scratch_ctx[MAX_DEVICES] = {nullptr};  // context the cached address belongs to
 static std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device (looked up once per device; in
-// host code the symbol name is only a host-side stand-in and must never reach a kernel).
+// The CUDA context current on this thread (driver entry point through the runtime, so the
+// library needs no link against the driver library); NULL if it cannot be read.
+static void *current_context() {
+  typedef CUresult (*PFN_ctx_t)(CUcontext *);
+  static PFN_ctx_t fn = nullptr;
+  static bool looked = false;
+  if (!looked) {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_ctx_t)f;
+    looked = true;
+  }
+  CUcontext c = nullptr;
+  if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+  return (void *)c;
+}
+
+// Device address of the scratch array on the current device and context (looked up once per
+// device and context; in host code the symbol name is only a host-side stand-in and must never
+// reach a kernel).
 static int scratch_on_current_device(float **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DREAMER_ERR_CUDA;
   if (dev < 0 || dev >= MAX_DEVICES) return DREAMER_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  if (!g_scratch_addr[dev] || current_context() != g_scratch_ctx[dev]) {
     void *p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
     if (e != cudaSuccess || !p) return DREAMER_ERR_CUDA;
     g_scratch_addr[dev] = static_cast<float *>(p);
+    g_scratch_ctx[dev] = current_context();  // current now: the lookup initialised it
   }
   *out = g_scratch_addr[dev];
   return DREAMER_OK;
@@ -131,7 +156,7 @@ __global__ void __launch_bounds__(256) route_noalloc_kernel(const T *y, int n, i
     le[p] = e;
   }
   int head = 0, my_e = 0;
-  float my_s = 0.f, ssum = 0.f;
+  float my_z = 0.f;
   for (int s = 0; s < k; s++) {
     float bv = head < k ? lv[head] : -INFINITY;
     int be = head < k ? le[head] : 0x7fffffff;
@@ -146,20 +171,24 @@ __global__ void __launch_bounds__(256) route_noalloc_kernel(const T *y, int n, i
       }
     }
     if (be == mine && head < k) head++;
-    // sigmoid of the unbiased score of the pick
+    // the unbiased score of the pick; lane s keeps pick s
     const float *kr = keys + (long)be * DR;
     float z = 0.f;
     for (int i = 0; i < DR; i++) z = fmaf(qs[wid][i], kr[i], z);
-    const float sg = 1.0f / (1.0f + __expf(-z * scale));
-    ssum += sg;
     if (lane == s) {
       my_e = be;
-      my_s = sg;
+      my_z = z * scale;
     }
   }
+  // w = sigmoid(z) / sum over the picks, in the stable form exp(ls - max ls) / sum exp(...)
+  // with ls = log sigmoid(z): no 0/0 when every pick's sigmoid underflows
+  const float ls = lane < k ? dreamer::log_sigmoidf_(my_z) : -INFINITY;
+  const float m = dreamer::warp_max(ls);
+  const float ex = lane < k ? expf(ls - m) : 0.f;
+  const float ssum = dreamer::warp_sum(ex);
   if (lane < k) {
     idx[(long)t * k + lane] = my_e;
-    w[(long)t * k + lane] = my_s / ssum;
+    w[(long)t * k + lane] = ex / ssum;
     if (counts) atomicAdd(counts + my_e, 1);
   }
 }

@@ -394,6 +394,7 @@ static bool tc_sa(dreamer_handle *h, cudaStream_t s) {
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
   a.err = h->err;
   const int grid = a.bh * a.n_pairs;
+  ++g_launches_tc;
   if (d == 64) {
     static bool set = false;
     if (!set) {

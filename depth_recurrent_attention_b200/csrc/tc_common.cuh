@@ -49,10 +49,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase of `parity` to complete, for at most ~2 s.  On expiry set the CTA's
-// abort word and the device error flag and return false; every role polls `abort` so the
-// CTA winds down instead of hanging.
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+// Wait for the phase of `parity` to complete, for at most DREAMER_WAIT_LIMIT_NS (2 s).  On
+// expiry set the CTA's abort word and the device error flag and return false; every role
+// polls `abort` so the CTA winds down instead of hanging.
+constexpr uint64_t WAIT_LIMIT_NS = DREAMER_WAIT_LIMIT_NS;
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
                                           int *err) {
   if (mbar_try_wait(bar, parity)) return true;

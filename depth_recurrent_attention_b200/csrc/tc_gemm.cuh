@@ -32,6 +32,7 @@ struct TcGemmArgs {
   long lda;
   int b_group_rows, b_row0;
   int *err;
+  int skip_loads;     // test-hook build only: the TMA producer issues no loads (0 otherwise)
 };
 
 // per-row epilogue state: Epi::State for row-pass epilogues, nothing otherwise
@@ -170,6 +171,10 @@ __global__ void __launch_bounds__(
       for (int i = 0; i < STAGES; i++) issued_ph[i] = -1;
       bool ok = true;
       int mt, nt;
+#ifdef DREAMER_TEST_HOOKS
+      // the timeout test: no operand ever arrives, so the MMA issuer's bounded wait expires
+      if (a.skip_loads) ok = false;
+#endif
       for (int i = 0; ok && tile_at(i, mt, nt); i++) {
         int g, m0, m1;
         const int n0 = nt * BN;

@@ -168,10 +168,16 @@ struct EpiTopK {
     if (valid) row_end(s, r, token);
   }
   __device__ __forceinline__ void row_end(State &s, int r, int token) const {
-    float sg[KT], sum = 0.f;
+    // normalised sigmoid weights in the stable form (log_sigmoidf_)
+    float sg[KT], m = -INFINITY, sum = 0.f;
 #pragma unroll
     for (int i = 0; i < KT; i++) {
-      sg[i] = 1.0f / (1.0f + __expf(-s.z[i]));
+      sg[i] = log_sigmoidf_(s.z[i]);
+      m = fmaxf(m, sg[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < KT; i++) {
+      sg[i] = expf(sg[i] - m);
       sum += sg[i];
     }
     const float inv = 1.0f / sum;
@@ -296,6 +302,7 @@ static void tc_launch(dreamer_handle *h, const dreamer::tc::TcGemmArgs &a, const
   }
   long grid = max_tiles < h->num_sms ? max_tiles : h->num_sms;
   if (grid < 1) grid = 1;
+  ++g_launches_tc;
   launch_k(h, kern, dim3((unsigned)grid), dim3(Cfg::THREADS), Cfg::SMEM, s, ta, tb, a, epi);
 }
 
@@ -360,12 +367,22 @@ static bool tc_gemm_qkv(dreamer_handle *h, const dreamer::GemmArgs &a, const dre
     // behind: eight epilogue warps then, at one stage less of operand ring.
     const bool ew8 = a.K <= 1024;
     const int bn = tc_pick_bn(h, a);
+#ifdef DREAMER_TEST_HOOKS
+    const int skip = h->inject_skip;
+    h->inject_skip = 0;
+#endif
     if (bn == 64) {  // one 64-column pass a tile: four epilogue warps, eight stages
       if (!tc_prepare<64, 64>(h, a, tiles, a.M, t, ta, tb, mt)) return false;
+#ifdef DREAMER_TEST_HOOKS
+      t.skip_loads = skip;
+#endif
       if (gather) tc_launch<64, 64, 8, true, 64>(h, t, ta, tb, mt, e, s);
       else tc_launch<64, 64, 8, false, 64>(h, t, ta, tb, mt, e, s);
     } else if (bn == 256) {
       if (!tc_prepare<256, 64>(h, a, tiles, a.M, t, ta, tb, mt)) return false;
+#ifdef DREAMER_TEST_HOOKS
+      t.skip_loads = skip;
+#endif
       if (ew8) {
         if (gather) tc_launch<256, 64, 3, true, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
         else tc_launch<256, 64, 3, false, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
@@ -375,6 +392,9 @@ static bool tc_gemm_qkv(dreamer_handle *h, const dreamer::GemmArgs &a, const dre
       }
     } else {
       if (!tc_prepare<128, 64>(h, a, tiles, a.M, t, ta, tb, mt)) return false;
+#ifdef DREAMER_TEST_HOOKS
+      t.skip_loads = skip;
+#endif
       if (ew8) {
         if (gather) tc_launch<128, 64, 5, true, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
         else tc_launch<128, 64, 5, false, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
@@ -425,17 +445,12 @@ static bool tc_gemm_o(dreamer_handle *h, const dreamer::GemmArgs &a, const dream
   return false;
 }
 
-static bool tc_route_ok(dreamer_handle *h) {
-  const dreamer_config &c = h->cfg;
-  return g_encode_tiled && h->k3 && c.n_experts % 256 == 0 &&
-         (c.router_dim == 64 || c.router_dim == 128) && c.hidden % 64 == 0;
-}
-
 static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, float *w,
                      int *counts_a, int *counts_b, cudaStream_t s) {
   using namespace dreamer;
   const dreamer_config &c = h->cfg;
   const int dr = c.router_dim, hd = c.hidden, E = c.n_experts;
+  if (!g_encode_tiled || !h->k3 || !(dr == 64 || dr == 128) || hd % 64 || E % 4) return false;
   // q = X W_qE, turned back by the depth rotation and split into hi/mid/lo bf16
   GemmArgs qa{};
   qa.N = dr; qa.K = hd; qa.G = 1; qa.M = n; qa.arow_div = 1;
@@ -448,7 +463,12 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
   GemmArgs za{};
   za.N = E; za.K = 3 * dr; za.G = 1; za.M = n; za.arow_div = 1;
   za.A = h->qsplit; za.lda = 3 * dr; za.B = h->k3; za.ldb = 3 * dr; za.bgstride = 0;
-  if (!tc_prepare<256, 64>(h, za, nullptr, n, t2, ta2, tb2, mt2)) return false;
+  // The fused top-k gives each 128-row tile to one CTA for all E columns: worth it only when
+  // there are enough row tiles to fill the GPU; otherwise a warp per token scores its row from
+  // the split query on the CUDA cores, which spreads the rows over every SM.
+  int k_fused = (n + 127) / 128 >= h->num_sms / 2 && E % 256 == 0 ? c.top_k : 0;
+  if (k_fused != 4 && k_fused != 8 && k_fused != 16) k_fused = 0;
+  if (k_fused && !tc_prepare<256, 64>(h, za, nullptr, n, t2, ta2, tb2, mt2)) return false;
   if (dr == 64) {
     if (!tc_prepare<64, 64>(h, qa, nullptr, n, t, ta, tb, mt)) return false;
     tc_launch<64, 64, 6, false, 64>(h, t, ta, tb, mt, eq, s);
@@ -457,10 +477,6 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
     tc_launch<128, 64, 6, false, 128>(h, t, ta, tb, mt, eq, s);
   }
   const float zs = 1.0f / sqrtf((float)dr);
-  // The fused top-k gives each 128-row tile to one CTA for all E columns: worth it only when
-  // there are enough row tiles to fill the GPU; otherwise a warp per token scores its row from
-  // the split query on the CUDA cores, which spreads the rows over every SM.
-  const int k_fused = (n + 127) / 128 >= h->num_sms / 2 ? c.top_k : 0;
   switch (k_fused) {  // top-k fused into the score GEMM
     case 4:
       tc_launch<256, 64, 4, false, 32, EpiTopK<4>, true, 8>(
@@ -477,14 +493,20 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
     default:
       break;
   }
-  // scores straight from the split query, one warp a token (tc_route_ok: d_r is 64 or 128)
+  // scores straight from the split query: two warps a token, four tokens a block (each warp's
+  // expert slice a multiple of 4), or one warp a token when E is not a multiple of 8
   TopkArgs k{};
   k.n_tok = n; k.E = E; k.k = c.top_k; k.mode = 0; k.zscale = zs;
   k.bias = h->bias; k.idx = idx; k.w = w; k.counts_a = counts_a; k.counts_b = counts_b;
-  constexpr int WPT = 2;  // warps a token, four tokens a block
-  auto kern = dr == 64 ? route_q_topk_kernel<64, WPT> : route_q_topk_kernel<128, WPT>;
-  launch_k(h, kern, dim3((n + 8 / WPT - 1) / (8 / WPT)), dim3(256), 0, s,
-           (const bf16 *)h->qsplit, (const bf16 *)h->kEt, k);
+  if (E % 8 == 0) {
+    auto kern = dr == 64 ? route_q_topk_kernel<64, 2> : route_q_topk_kernel<128, 2>;
+    launch_k(h, kern, dim3((n + 3) / 4), dim3(256), 0, s, (const bf16 *)h->qsplit,
+             (const bf16 *)h->kEt, k);
+  } else {
+    auto kern = dr == 64 ? route_q_topk_kernel<64, 1> : route_q_topk_kernel<128, 1>;
+    launch_k(h, kern, dim3((n + 7) / 8), dim3(256), 0, s, (const bf16 *)h->qsplit,
+             (const bf16 *)h->kEt, k);
+  }
   return true;
 }
 
@@ -531,6 +553,7 @@ static void tc_ffn_launch(dreamer_handle *h, const CUtensorMap &t1, const CUtens
   }
   long grid = max_tiles < h->num_sms ? max_tiles : h->num_sms;
   if (grid < 1) grid = 1;
+  ++g_launches_tc;
   launch_k(h, kern, dim3((unsigned)grid), dim3(Cfg::THREADS), Cfg::SMEM, s, t1, t2, a);
 }
 

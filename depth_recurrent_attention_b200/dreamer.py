@@ -15,7 +15,10 @@ from .configs import DreamerConfig
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdreamer.so")
-_lib = None
+# test infrastructure only: the same sources with the timeout-test hook (dreamer_test_inject)
+# and a 20 ms device wait limit
+TESTHOOKS_PATH = os.path.join(_HERE, "libdreamer_testhooks.so")
+_libs = {}
 
 OK = 0
 ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_OOM, ERR_TIMEOUT, ERR_STATE = -1, -2, -3, -4, -5, -6
@@ -51,22 +54,22 @@ STAGES = ("norm", "proj_route", "qkv", "da", "sa", "o_proj", "ea_route", "permut
 
 class StatsC(C.Structure):
     _fields_ = [("launches", C.c_uint64), ("ms", C.c_double * len(STAGES)),
-                ("count", C.c_uint64 * len(STAGES))]
+                ("count", C.c_uint64 * len(STAGES)), ("launches_tc", C.c_uint64),
+                ("launches_simt", C.c_uint64)]
 
 
-TRACE_FIELDS = ("xhat", "y", "idx", "w", "sa_k", "sa_v", "pidx", "psig")
+TRACE_FIELDS = ("xhat", "y", "idx", "w", "sa_k", "sa_v", "pidx", "psig", "y_f32", "x_f32")
 
 
 class TraceC(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in TRACE_FIELDS]
 
 
-def lib():
-    global _lib
-    if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} not built: run __graft_entry__.build()")
-        L = C.CDLL(LIB_PATH)
+def lib(path: str = LIB_PATH):
+    if path not in _libs:
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} not built: run __graft_entry__.build()")
+        L = C.CDLL(path)
         vp, i = C.c_void_p, C.c_int
         L.dreamer_init.argtypes = [C.POINTER(ConfigC), C.POINTER(WeightsC), vp, C.POINTER(vp)]
         L.dreamer_core_forward.argtypes = [vp, vp, vp, i, i, vp, vp, vp]
@@ -87,8 +90,11 @@ def lib():
                   "dreamer_bias_update_counts", "dreamer_route_balance",
                   "dreamer_set_profiling", "dreamer_get_stats"):
             getattr(L, f).restype = i
-        _lib = L
-    return _lib
+        if hasattr(L, "dreamer_test_inject"):
+            L.dreamer_test_inject.argtypes = [vp, i]
+            L.dreamer_test_inject.restype = i
+        _libs[path] = L
+    return _libs[path]
 
 
 def _ptr(t):
@@ -125,8 +131,10 @@ class Dreamer:
     k_E, bias, w1, w2 and, with projection experts, w_qkv_shared, w_o_shared, w_qP, k_P).
     """
 
-    def __init__(self, cfg: DreamerConfig, weights: dict, stream=None, max_cache_len=None):
+    def __init__(self, cfg: DreamerConfig, weights: dict, stream=None, max_cache_len=None,
+                 lib_path: str = LIB_PATH):
         self.cfg = cfg
+        self.L = lib(lib_path)
         self.cc = config_c(cfg)
         if max_cache_len is not None:
             self.cc.max_cache_len = int(max_cache_len)
@@ -137,12 +145,12 @@ class Dreamer:
             ptrs[f] = _ptr(t) if t is not None else None
         self.wc = WeightsC(**ptrs)
         self.h = C.c_void_p()
-        _check(lib().dreamer_init(C.byref(self.cc), C.byref(self.wc), _stream(stream),
+        _check(self.L.dreamer_init(C.byref(self.cc), C.byref(self.wc), _stream(stream),
                                   C.byref(self.h)), "dreamer_init")
 
     def close(self):
         if self.h:
-            lib().dreamer_destroy(self.h)
+            self.L.dreamer_destroy(self.h)
             self.h = C.c_void_p()
 
     def __del__(self):
@@ -164,7 +172,7 @@ class Dreamer:
         if x_out is None:
             x_out = torch.empty_like(x_in)
         tr = self._trace(trace)
-        _check(lib().dreamer_core_forward(self.h, _ptr(x_in), _ptr(x_out), int(depth_begin),
+        _check(self.L.dreamer_core_forward(self.h, _ptr(x_in), _ptr(x_out), int(depth_begin),
                                           int(depth_end), _ptr(da_kv),
                                           C.byref(tr) if tr is not None else None,
                                           _stream(stream)), "dreamer_core_forward")
@@ -175,7 +183,7 @@ class Dreamer:
         if x_out is None:
             x_out = torch.empty_like(x_new)
         tr = self._trace(trace)
-        _check(lib().dreamer_decode_step(self.h, _ptr(x_new), _ptr(k_cache), _ptr(v_cache),
+        _check(self.L.dreamer_decode_step(self.h, _ptr(x_new), _ptr(k_cache), _ptr(v_cache),
                                          _ptr(cache_len), _ptr(x_out),
                                          C.byref(tr) if tr is not None else None,
                                          _stream(stream)), "dreamer_decode_step")
@@ -186,7 +194,7 @@ class Dreamer:
         summed over depths), as device tensors."""
         lor = torch.empty(self.cfg.n_experts + 1, dtype=torch.float32, device="cuda")
         g = torch.empty(1, dtype=torch.float32, device="cuda")
-        _check(lib().dreamer_route_balance(self.h, int(depth), _ptr(lor), _ptr(g),
+        _check(self.L.dreamer_route_balance(self.h, int(depth), _ptr(lor), _ptr(g),
                                            _stream(stream)), "dreamer_route_balance")
         return g, lor
 
@@ -194,11 +202,11 @@ class Dreamer:
         cfg = self.cfg
         if on_host:
             out = torch.zeros((cfg.depth, cfg.n_experts), dtype=torch.int32)
-            _check(lib().dreamer_route_counts(self.h, C.c_void_p(out.data_ptr()), 1,
+            _check(self.L.dreamer_route_counts(self.h, C.c_void_p(out.data_ptr()), 1,
                                               _stream(stream)), "dreamer_route_counts")
             return out
         out = torch.zeros((cfg.depth, cfg.n_experts), dtype=torch.int32, device="cuda")
-        _check(lib().dreamer_route_counts(self.h, _ptr(out), 0, _stream(stream)),
+        _check(self.L.dreamer_route_counts(self.h, _ptr(out), 0, _stream(stream)),
                "dreamer_route_counts")
         return out
 
@@ -208,7 +216,7 @@ class Dreamer:
         idx = torch.empty((n, cfg.top_k), dtype=torch.int32, device=y.device)
         w = torch.empty((n, cfg.top_k), dtype=torch.float32, device=y.device)
         counts = torch.empty(cfg.n_experts, dtype=torch.int32, device=y.device)
-        _check(lib().dreamer_route_experts(self.h, int(depth), _ptr(y), int(n), _ptr(idx),
+        _check(self.L.dreamer_route_experts(self.h, int(depth), _ptr(y), int(n), _ptr(idx),
                                            _ptr(w), _ptr(counts), _stream(stream)),
                "dreamer_route_experts")
         return idx, w, counts
@@ -220,24 +228,30 @@ class Dreamer:
         allreduce_route_counts), those summed over their rows."""
         out = torch.empty(self.cfg.n_experts, dtype=torch.float32, device="cuda")
         if counts is None:
-            _check(lib().dreamer_bias_update(self.h, float(lam), _ptr(out), _stream(stream)),
+            _check(self.L.dreamer_bias_update(self.h, float(lam), _ptr(out), _stream(stream)),
                    "dreamer_bias_update")
             return out
         c = counts.reshape(-1, self.cfg.n_experts)
         if c.dtype != torch.int32 or not c.is_cuda or not c.is_contiguous():
             raise ValueError("counts: a contiguous CUDA int32 tensor [R][E] or [E]")
-        _check(lib().dreamer_bias_update_counts(self.h, float(lam), _ptr(c), int(c.shape[0]),
+        _check(self.L.dreamer_bias_update_counts(self.h, float(lam), _ptr(c), int(c.shape[0]),
                                                 _ptr(out), _stream(stream)),
                "dreamer_bias_update_counts")
         return out
 
     def set_profiling(self, enable: bool):
-        _check(lib().dreamer_set_profiling(self.h, int(bool(enable))), "dreamer_set_profiling")
+        _check(self.L.dreamer_set_profiling(self.h, int(bool(enable))), "dreamer_set_profiling")
+
+    def test_inject(self, what: int):
+        """Test-hook library only: what = 1 makes the next call's first QKV GEMM load no
+        operands, so that its bounded wait expires (DREAMER_ERR_TIMEOUT)."""
+        _check(self.L.dreamer_test_inject(self.h, int(what)), "dreamer_test_inject")
 
     def stats(self, reset: bool = True) -> dict:
         st = StatsC()
-        _check(lib().dreamer_get_stats(self.h, C.byref(st), int(bool(reset))), "dreamer_get_stats")
-        return dict(launches=int(st.launches),
+        _check(self.L.dreamer_get_stats(self.h, C.byref(st), int(bool(reset))), "dreamer_get_stats")
+        return dict(launches=int(st.launches), launches_tc=int(st.launches_tc),
+                    launches_simt=int(st.launches_simt),
                     ms={n: float(st.ms[i]) for i, n in enumerate(STAGES)},
                     count={n: int(st.count[i]) for i, n in enumerate(STAGES)})
 

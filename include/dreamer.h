@@ -100,7 +100,19 @@ typedef struct {
   void *sa_v;      /* [L][T][h] dtype: SA values (forward only)                            */
   int32_t *pidx;   /* [L][T]: projection expert p* (P > 0)                                 */
   float *psig;     /* [L][T]: projection weight sigma (P > 0)                              */
+  float *y_f32;    /* [L][T][h] float32: y_l as the residual stream carries it, before its
+                      rounding to dtype (in bf16 mode `y` above is this value rounded)     */
+  float *x_f32;    /* [L][T][h] float32: x_{l+1} = y_l + expert attention, before rounding
+                      (the last depth's x_out is this value rounded to dtype)              */
 } dreamer_trace;
+
+/* Shapes the bfloat16 path takes (every contraction and attention on the tcgen05 tensor
+ * cores or in the purpose-built streaming kernels; there is no CUDA-core fallback):
+ * head_dim 64 or 128, hidden a multiple of 256 and at most 2048 where rows are few per expert
+ * (decode), n_heads <= 32, expert_hidden 16, 32 or 64, router_dim 64 or 128, n_experts a
+ * multiple of 4; dreamer_core_forward also needs seq a multiple of 128.  dreamer_init returns
+ * DREAMER_ERR_UNSUPPORTED for any other bf16 shape (dreamer_core_forward on a handle whose seq
+ * is not a multiple of 128 returns it too).  float32 mode runs every shape on CUDA cores.  */
 
 /* Create a handle: validates the configuration, copies the weights (device pointers) into
  * handle-owned buffers in the kernels' layouts, absorbs the shared projection expert into
@@ -172,8 +184,10 @@ int dreamer_route_experts(dreamer_handle *h, int depth, const void *y, int n_tok
  * DREAMER_ERR_UNSUPPORTED before anything runs.  Every GPU that loads the library keeps the
  * array until the process exits.  All calls share it and it keeps the last call's contents,
  * so calls that overlap on the GPU (other streams, other host threads) race: serialise them.
- * The first call on a device looks up the array's device address and caches it; make that
- * first call before any stream capture on the device.                                      */
+ * The first call on a device looks up the array's device address and caches it (per device
+ * and CUDA context: a new context, e.g. after cudaDeviceReset, looks it up again); make that
+ * first call before any stream capture on the device.  Routing weights are formed in a form
+ * that stays finite when every pick's sigmoid underflows.                                  */
 int dreamer_route_experts_noalloc(const dreamer_config *cfg, int depth, const void *y,
                                   int n_tokens, const void *w_qE, const void *k_E,
                                   const float *bias_E, int32_t *idx, float *w,
@@ -221,6 +235,10 @@ typedef struct {
   uint64_t launches;                 /* kernels launched by the library since the reset    */
   double ms[DREAMER_N_STAGES];       /* device time per stage (profiling enabled only)     */
   uint64_t count[DREAMER_N_STAGES];  /* timed stage executions                             */
+  uint64_t launches_tc;              /* of `launches`: tcgen05 kernels (GEMM engine, flash
+                                        SA, fused expert FFN)                              */
+  uint64_t launches_simt;            /* of `launches`: the generic CUDA-core GEMM, attention
+                                        and top-k kernels of float32 mode (0 in bf16 mode)   */
 } dreamer_stats;
 
 /* Enable (1) or disable (0) per-stage CUDA-event timing on the streams of later calls.

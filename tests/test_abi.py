@@ -68,3 +68,34 @@ def test_product_does_not_reference_the_oracle():
                 assert "oracle" not in txt.lower() or f == "inputs.py", f
     lib_txt = open(os.path.join(PKG, "dreamer.py")).read()
     assert "import oracle" not in lib_txt
+
+
+@pytest.mark.parametrize("kw,bf16_code", [
+    ({}, "ARG"),                                        # valid shapes: fails only at the weights
+    (dict(n_heads=16, head_dim=32), "UNSUPPORTED"),     # no tcgen05 GEMM / flash SA for d = 32
+    (dict(expert_hidden=48), "UNSUPPORTED"),            # expert FFN kernels: m 16, 32 or 64
+    (dict(router_dim=32), "UNSUPPORTED"),               # router: d_r 64 or 128
+    (dict(hidden=384, n_heads=6), "UNSUPPORTED"),       # N tiles of 256 columns
+    (dict(n_experts=6, top_k=2), "UNSUPPORTED"),        # router scorer: E a multiple of 4
+    (dict(n_heads=64, head_dim=64, hidden=4096), "UNSUPPORTED"),  # DA: a warp per head, <= 32
+])
+def test_bf16_shapes_without_a_tcgen05_kernel_are_refused(built, kw, bf16_code):
+    """bfloat16 mode has no CUDA-core fallback: dreamer_init refuses a shape its kernels do not
+    take (before any device call), while float32 mode takes it (and fails only at the NULL
+    weights here)."""
+    import depth_recurrent_attention_b200.dreamer as D
+    from depth_recurrent_attention_b200 import configs
+    cfg = configs.SMALL.with_(**kw)
+    h = ctypes.c_void_p()
+    rc = D.lib().dreamer_init(ctypes.byref(D.config_c(cfg)), None, None, ctypes.byref(h))
+    assert rc == getattr(D, "ERR_" + bf16_code), (kw, rc)
+    rc32 = D.lib().dreamer_init(ctypes.byref(D.config_c(cfg.with_(dtype="fp32"))), None, None,
+                                ctypes.byref(h))
+    assert rc32 == D.ERR_ARG, (kw, rc32)
+
+
+def test_only_the_test_hook_library_exports_the_injection(built):
+    """dreamer_test_inject (the timeout test's hook) exists in the test-hook build only."""
+    from depth_recurrent_attention_b200 import dreamer as D
+    assert not hasattr(ctypes.CDLL(D.LIB_PATH), "dreamer_test_inject")
+    assert hasattr(ctypes.CDLL(D.TESTHOOKS_PATH), "dreamer_test_inject")

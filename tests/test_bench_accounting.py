@@ -1,6 +1,6 @@
 """The algorithmic FLOP and byte counts behind the bench line's roofline fractions, pinned to
-numbers worked out by hand for the small workload (b 4, s 512, h 512, 8x64, L 8, E 256, k 4,
-m 64, d_r 64, bf16)."""
+hand counts and to the workload table of the roofline accounting (small 0.55 GB, medium
+16.6 GB, large 442 GB: perfect on-chip reuse inside a depth step, none across depths)."""
 import os
 import sys
 
@@ -22,20 +22,35 @@ from depth_recurrent_attention_b200 import configs  # noqa: E402
 SMALL_FLOPS = 8 * (6_442_450_944 + 1_075_838_976 + 2_147_483_648 + 201_326_592
                    + 1_073_741_824) + 150_994_944
 
-# per depth (2-byte values): norm 4 T h = 4 194 304; QKV T h 2 + 6h h 2 + T 6h 2 = 17 825 792;
-# SA 8 T h = 8 388 608; O T 2h 2 + 2h h 2 + T h (2 + 4) = 11 534 336;
-# EA T h 2 + h d_r 2 + E d_r 2 = 2 195 456; FFN (all 256 experts) 2 E h m 2 + T h 2 + 8 T h =
-# 44 040 192.  DA over all depths: 8 (T h 2 + T h 2) + T 2h 2 (0 + 1 + ... + 7) = 150 994 944
-SMALL_BYTES = 8 * (4_194_304 + 17_825_792 + 8_388_608 + 11_534_336 + 2_195_456
-                   + 44_040_192) + 150_994_944
+# per depth (2-byte values, T = 2048, h = 512):
+#   residual x read and written        4 T h     =  4 194 304
+#   DA keys/values written             4 T h     =  4 194 304
+#   SA keys/values written and read    8 T h     =  8 388 608
+#   QKV and O weights                  (6 + 2) h^2 2 = 4 194 304
+#   router query and keys              (h + E) d_r 2 =    98 304
+#   expert weights (all 256 touched)   2 E h m 2     = 33 554 432
+# DA re-reads of earlier depths: 4 T h (0 + 1 + ... + 7) = 117 440 512
+SMALL_BYTES = 8 * (4_194_304 + 4_194_304 + 8_388_608 + 4_194_304 + 98_304
+                   + 33_554_432) + 117_440_512
 
 
 def test_small_totals_match_the_hand_count():
     st, f, b = bench.algorithmic(configs.SMALL)
     assert f == SMALL_FLOPS == 87_677_730_816
-    assert b == SMALL_BYTES == 856_424_448
+    assert b == SMALL_BYTES == 554_434_560
     assert st["qkv"][0] == 8 * 6_442_450_944
-    assert st["da"] == (150_994_944, 150_994_944)
+    assert st["da"] == (150_994_944, 117_440_512)
+
+
+def test_workload_table_totals():
+    """The roofline table's byte totals: medium 16.6 GB (DA 9.1), large 442 GB (DA 279)."""
+    _, f, b = bench.algorithmic(configs.MEDIUM)
+    assert round(b / 1e9, 1) == 16.6 and round(f / 1e12, 2) == 5.89
+    st, f, b = bench.algorithmic(configs.LARGE)
+    assert round(b / 1e9) == 442 and round(f / 1e12, 1) == 111.9
+    T, h, L = configs.LARGE.tokens, configs.LARGE.hidden, configs.LARGE.depth
+    da_bytes = st["da"][1] + 4 * T * h * L           # re-reads + the writes (in the qkv stage)
+    assert round(da_bytes / 1e9) == 279
 
 
 def test_untouched_experts_drop_their_weight_bytes():
@@ -52,13 +67,15 @@ def test_untouched_experts_drop_their_weight_bytes():
 def test_da_window_and_no_da_arms():
     cfg = configs.SMALL
     T, h = cfg.tokens, cfg.hidden
-    # window 2: depths attend to min(l + 1, 2) states, 1 + 2 * 7 = 15 in all
+    # window 2: depths attend to min(l + 1, 2) states, 1 + 2 * 7 = 15 in all; one earlier
+    # depth re-read by each of depths 1..7
     st, _, _ = bench.algorithmic(cfg.with_(da_window=2))
     assert st["da"][0] == 4.0 * T * h * 15
-    assert st["da"][1] == 8 * 2 * T * h * 2 + 2 * T * h * 2 * 7
-    # without DA: half-width projections, no DA stage
-    st, f, _ = bench.algorithmic(cfg.with_(variant=3))
+    assert st["da"][1] == 2 * T * h * 2 * 7
+    # without DA: half-width projections, no DA stage, no DA keys/values written
+    st, f, b = bench.algorithmic(cfg.with_(variant=3))
     assert "da" not in st
     assert st["qkv"][0] == 8 * 2.0 * T * h * 3 * h
     assert st["o_proj"][0] == 8 * 2.0 * T * h * h
     assert f == SMALL_FLOPS - 150_994_944 - 8 * (3_221_225_472 + 1_073_741_824)
+    assert b == SMALL_BYTES - 117_440_512 - 8 * (4_194_304 + 4 * h * h * 2)

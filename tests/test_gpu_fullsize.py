@@ -37,6 +37,9 @@ def host_rows(sp, seed, row0, nrows):
 
 
 def step_check(cfg, dev, W, l, seq, pos, orc):
+    """One depth over every token on seeded inputs; the routing of every token gated on the
+    device's own router inputs (strict 1e-5 rule, exact counts), the float32 states of the
+    sampled tokens against the oracle's step, the stored bf16 values as their exact rounding."""
     torch = _torch()
     T, L, h = cfg.tokens, cfg.depth, cfg.hidden
     xs = spec("x_l", (T, h), 1000 + l)
@@ -44,11 +47,30 @@ def step_check(cfg, dev, W, l, seq, pos, orc):
     x = inputs.device_tensor(xs, cfg.seed)
     hist = inputs.device_tensor(hs, cfg.seed)
     tr = dict(y=torch.empty((L, T, h), dtype=torch.bfloat16, device="cuda"),
-              idx=torch.empty((L, T, cfg.top_k), dtype=torch.int32, device="cuda"))
+              y_f32=torch.empty((L, T, h), dtype=torch.float32, device="cuda"),
+              x_f32=torch.empty((L, T, h), dtype=torch.float32, device="cuda"),
+              idx=torch.empty((L, T, cfg.top_k), dtype=torch.int32, device="cuda"),
+              w=torch.empty((L, T, cfg.top_k), dtype=torch.float32, device="cuda"))
     if cfg.n_proj_experts:
+        tr["xhat"] = torch.empty((L, T, h), dtype=torch.bfloat16, device="cuda")
         tr["pidx"] = torch.empty((L, T), dtype=torch.int32, device="cuda")
+        tr["psig"] = torch.empty((L, T), dtype=torch.float32, device="cuda")
     out = dev.forward(x, depth_begin=l, depth_end=l + 1, da_kv=hist, trace=tr)
     torch.cuda.synchronize()
+    # routing of every token, on the device's own y (and x^ for the projection router)
+    y_all = PY.to_np(tr["y"][l])
+    counts = dev.route_counts(on_host=True).numpy()[l]
+    PY.gate_router_on_device_input(cfg, W, orc, l, y_all, tr["idx"][l].cpu().numpy(),
+                                   PY.to_np(tr["w"][l]), counts, what=cfg.name)
+    if cfg.n_proj_experts:
+        gp_all = tr["pidx"][l].cpu().numpy()
+        PY.gate_proj_router_on_device_input(cfg, orc, l, PY.to_np(tr["xhat"][l]), gp_all,
+                                            PY.to_np(tr["psig"][l]), what=cfg.name)
+    # the stored bf16 states are the exact rounding of the float32 ones (all tokens)
+    assert np.array_equal(PY.rn_bf16(PY.to_np(tr["y_f32"][l])), y_all)
+    assert np.array_equal(PY.rn_bf16(PY.to_np(tr["x_f32"][l])), PY.to_np(out))
+    del y_all
+    # the sampled tokens against the oracle's step with the sequence's whole context
     S = cfg.seq
     tk = seq * S + np.asarray(pos)
     x_seq = host_rows(xs, cfg.seed, seq * S, int(max(pos)) + 1)
@@ -57,19 +79,18 @@ def step_check(cfg, dev, W, l, seq, pos, orc):
         hist_h[:, j] = 0.0
     r = orc.step_tokens(l, x_seq, hist_h, np.asarray(pos, np.int32))
     if cfg.n_proj_experts:
-        gp = tr["pidx"][l, tk].cpu().numpy()
-        assert np.all((gp == r["pidx"]) | (r["pmargin"] <= 1e-3))
-        keep = gp == r["pidx"]
+        keep = PY.proj_same_as_forward(cfg, W, l, gp_all[tk], r["pidx"], r["pmargin"],
+                                       PY.to_np(tr["xhat"][l, tk]), r["xhat"])
     else:
         keep = np.ones(len(tk), bool)
     gy = PY.to_np(tr["y"][l, tk])
-    PY.check_hidden(gy[keep], r["y"][keep], True, f"y depth {l}")
+    PY.check_hidden(gy[keep], r["y"][keep], True, f"y depth {l}",
+                    f32=PY.to_np(tr["y_f32"][l, tk])[keep])
     same, flips = PY.check_routing(cfg, W, l, tr["idx"][l, tk].cpu().numpy()[keep],
                                    r["idx"][keep], r["margin"][keep], gy[keep], r["y"][keep])
     gx = PY.to_np(out[tk])
-    PY.check_hidden(gx[keep][same], r["x_out"][keep][same], True, f"x depth {l}")
-    # the depth KV written for depth l (post depth-RoPE key, value) of the sampled tokens is
-    # checked through y (DA output); the rest of the buffer is untouched
+    PY.check_hidden(gx[keep][same], r["x_out"][keep][same], True, f"x depth {l}",
+                    f32=PY.to_np(tr["x_f32"][l, tk])[keep][same])
     return flips
 
 
@@ -118,14 +139,26 @@ def decode_run(cfg, seqs):
     lens = torch.full((cfg.batch,), cfg.cache_len, dtype=torch.int32, device="cuda")
     L, k = cfg.depth, cfg.top_k
     tr = dict(y=torch.empty((L, cfg.batch, cfg.hidden), dtype=torch.bfloat16, device="cuda"),
-              idx=torch.empty((L, cfg.batch, k), dtype=torch.int32, device="cuda"))
+              y_f32=torch.empty((L, cfg.batch, cfg.hidden), dtype=torch.float32, device="cuda"),
+              x_f32=torch.empty((L, cfg.batch, cfg.hidden), dtype=torch.float32, device="cuda"),
+              idx=torch.empty((L, cfg.batch, k), dtype=torch.int32, device="cuda"),
+              w=torch.empty((L, cfg.batch, k), dtype=torch.float32, device="cuda"))
     out = dev.decode_step(X["x0"], X["k_cache"], X["v_cache"], lens, trace=tr)
     torch.cuda.synchronize()
     kslot = PY.to_np(X["k_cache"][:, :, :, cfg.cache_len])   # [L][B][H][d]
-    res = dict(out=PY.to_np(out), y=PY.to_np(tr["y"]), idx=tr["idx"].cpu().numpy(), kslot=kslot)
+    res = dict(out=PY.to_np(out), y=PY.to_np(tr["y"]), idx=tr["idx"].cpu().numpy(), kslot=kslot,
+               y_f32=PY.to_np(tr["y_f32"]), x_f32=PY.to_np(tr["x_f32"]), w=PY.to_np(tr["w"]),
+               counts=dev.route_counts(on_host=True).numpy())
     del X
     dev.close()
     W = inputs.host_weights(cfg)
+    # every depth's routing of all sequences, on the states the device routed
+    orc_all = O.Oracle(cfg, PY.deployed_weights(cfg, W))
+    for l in range(L):
+        PY.gate_router_on_device_input(cfg, W, orc_all, l, res["y"][l], res["idx"][l],
+                                       res["w"][l], res["counts"][l], what=cfg.name)
+    assert np.array_equal(PY.rn_bf16(res["y_f32"]), res["y"])
+    assert np.array_equal(PY.rn_bf16(res["x_f32"][L - 1]), res["out"])
     o = O.Oracle(cfg.with_(batch=1), PY.deployed_weights(cfg, W))
     sp = {s.name: s for s in inputs.input_specs(cfg)}
     H, d, cap = cfg.n_heads, cfg.head_dim, cfg.cache_len + 1
@@ -144,13 +177,14 @@ def decode_run(cfg, seqs):
 
 
 def test_fullsize_decode_first_depth(cuda):
-    """Real routing: depth 0 is compared token by token (later depths of a free-running bf16
-    decode follow routing flips); the full routing decision at every depth is covered by the
-    strict router test."""
+    """Real routing: the routing of every depth is gated on the states the device routed;
+    depth 0's states are compared token by token with the oracle's decode (later depths of a
+    free-running bf16 decode follow routing flips at near ties)."""
     cfg = configs.DECODE
     res, refs, W = decode_run(cfg, (0, 37))
     for b, (r, kslot) in refs.items():
-        PY.check_hidden(res["y"][0, b], r["y"][0], True, f"y depth 0 seq {b}")
+        PY.check_hidden(res["y"][0, b], r["y"][0], True, f"y depth 0 seq {b}",
+                        f32=res["y_f32"][0, b])
         PY.check_hidden(res["kslot"][0, b], kslot[0], True, f"k slot depth 0 seq {b}")
         PY.check_routing(cfg, W, 0, res["idx"][0, b:b + 1], r["idx"][0:1], r["margin"][0:1],
                          res["y"][0, b:b + 1], r["y"][0:1])
@@ -163,7 +197,9 @@ def test_fullsize_decode_flip_free_all_depths(cuda):
     res, refs, W = decode_run(cfg, (0, 63))
     for b, (r, kslot) in refs.items():
         for l in range(cfg.depth):
-            PY.check_drift(res["y"][l, b], r["y"][l], f"y depth {l} seq {b}", gate_abs=(l == 0))
+            PY.check_drift(res["y"][l, b], r["y"][l], f"y depth {l} seq {b}", gate_abs=(l == 0),
+                           f32=res["y_f32"][l, b])
         PY.check_drift(res["kslot"][:, b], kslot, f"k slots seq {b}", gate_abs=False)
-        e, rl = PY.check_drift(res["out"][b], r["x_out"], f"x_out seq {b}", gate_abs=False)
+        e, rl = PY.check_drift(res["out"][b], r["x_out"], f"x_out seq {b}", gate_abs=False,
+                               f32=res["x_f32"][cfg.depth - 1, b])
         print(f"decode flip-free seq {b}: x_out max-abs {e:.3g} rel-L2 {rl:.3g}")
