@@ -83,7 +83,11 @@ LARGE = DreamerConfig("large", batch=2, seq=8192, hidden=2048, n_heads=16, head_
                       n_proj_experts=16, dtype="bf16", seed=4, bias_range=0.1)
 
 # the comparison arms and the sparse-DA outlook on the large shapes: DR without depth
-# attention (variant 3) and depth attention over the last 8 depths
+# attention (variant 3) and depth attention over the last 8 depths; the pages' other block
+# layouts: serial DA -> SA -> EA (variant 1) and fully parallel DA + SA + EA (variant 2)
 LARGE_NODA = LARGE.with_(name="large-noda", variant=3)
 LARGE_W8 = LARGE.with_(name="large-w8", da_window=8)
-CONFIGS = {c.name: c for c in (TINY, SMALL, MEDIUM, DECODE, LARGE, LARGE_NODA, LARGE_W8)}
+LARGE_SERIAL = LARGE.with_(name="large-serial", variant=1)
+LARGE_PARALLEL = LARGE.with_(name="large-parallel", variant=2)
+CONFIGS = {c.name: c for c in (TINY, SMALL, MEDIUM, DECODE, LARGE, LARGE_NODA, LARGE_W8,
+                               LARGE_SERIAL, LARGE_PARALLEL)}

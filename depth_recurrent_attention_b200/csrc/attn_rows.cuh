@@ -215,11 +215,12 @@ struct DaBulkArgs {
   int *err;
 };
 
-template <typename T, int D>
+// NB chunk buffers: 2 (two CTAs share an SM) or 4 (a CTA owns its SM: the launch beside SA
+// gives depth attention a set of whole SMs, and more chunks in flight per SM).
+template <typename T, int D, int NB>
 __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
   pdl_wait();
   pdl_trigger();
-  constexpr int NB = 2;
   extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ __align__(8) uint64_t bars[NB];
   __shared__ int abort_flag;
@@ -363,6 +364,240 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
 #pragma unroll
           for (int i = 0; i < VEC; i++) of[i] *= inv;
           st16(reinterpret_cast<T *>(a.out) + (long)tok * a.ldo + a.col0 + head * D + cc * VEC, of);
+        }
+      }
+    }
+    __syncthreads();        // buffer b is free again
+    if (abort_flag) break;  // read after the barrier: the same decision in every thread
+    if (threadIdx.x == 0 && issued < nitems) {
+      issue(issued);
+      issued++;
+    }
+  }
+  // copies still in flight after an abort land before the CTA exits
+  if (threadIdx.x == 0 && abort_flag) {
+    for (int j = consumed; j < issued; j++) {
+      const uint64_t t0 = tcda::gtimer();
+      while (!tcda::try_wait(tcda::smem_u32(&bars[j % NB]), (uint32_t)((j / NB) & 1)) &&
+             tcda::gtimer() - t0 < DREAMER_WAIT_LIMIT_NS) {
+      }
+    }
+  }
+}
+
+// =======================================================================================
+// Depth attention for bf16 and head dims 64 / 128, fewer instructions per streamed byte: the
+// same (token, chunk) stream of bulk copies as da_bulk_kernel (three buffers, one CTA an SM),
+// with the rows of a chunk taken in batches of 8.  A warp (one head) splits a row into CH =
+// D / 8 lanes of 8 elements and its 32 lanes into G = 32 / CH groups; lane (g, c) forms the
+// partial dot products of its chunk c with the NR = 8 / G rows of group g, and one transposed
+// butterfly (log2 NR halving exchanges, then plain ones) leaves every row's full score in
+// CH / NR lanes with NR - 1 + log2(CH / NR) shuffles for the batch instead of log2(CH) a row.
+// Products and accumulations use the packed FP32 pair instructions (fma.rn.f32x2), bf16
+// values widen to fp32 by a shift or a mask.  One online-softmax update a batch (max and sum
+// by warp shuffles); each lane then fetches the NR weights of its group's rows and
+// accumulates the V rows into its 8 output elements; the G groups' partial outputs are
+// summed at the token's last chunk.  (papernotes "Key design 1": attention over the token's
+// own states at depths 0..l.)
+// =======================================================================================
+namespace tcda {
+// packed fp32 pairs: {lo, hi} in one 64-bit register
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 up2(uint64_t v) {
+  float2 f;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
+  return f;
+}
+// two bf16 of one 32-bit word as an fp32 pair (low element, high element)
+__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xffff0000u));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float ex2a(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+}  // namespace tcda
+
+template <int D>
+__global__ void __launch_bounds__(1024) da_fast_kernel(DaBulkArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int NB = 3;
+  constexpr int CH = D / 8, G = 32 / CH, NR = 8 / G, DUP = CH / NR;
+  static_assert(D == 64 || D == 128, "head dim");
+  extern __shared__ __align__(128) uint8_t dsm[];
+  __shared__ __align__(8) uint64_t bars[NB];
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nrow = a.l + 1 - a.r0;                     // depths r0..l
+  const int nch = (nrow + a.chunk - 1) / a.chunk;
+  const long row_el = 2L * a.h;                        // elements of one depth row (K then V)
+  const uint32_t chunk_bytes = (uint32_t)(a.chunk * row_el * sizeof(bf16));
+  const uint32_t q_bytes = (uint32_t)(a.h * sizeof(bf16));
+  const int ntok = a.n_tok > (int)blockIdx.x ? (a.n_tok - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int nitems = ntok * nch;
+  if (nitems == 0) return;  // the whole CTA
+  auto kv_slot = [&](int b) { return dsm + (size_t)b * chunk_bytes; };
+  auto q_slot = [&](int b) { return dsm + (size_t)NB * chunk_bytes + (size_t)b * q_bytes; };
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NB; i++)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tcda::smem_u32(&bars[i])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    abort_flag = 0;
+  }
+  __syncthreads();
+  auto issue = [&](int j) {
+    const int b = j % NB, c = j % nch;
+    const int tok = (int)blockIdx.x + (j / nch) * (int)gridDim.x;
+    const int r0 = c * a.chunk, nr = min(a.chunk, nrow - r0);
+    const uint32_t kvb = (uint32_t)(nr * row_el * sizeof(bf16));
+    const uint32_t bar = tcda::smem_u32(&bars[b]);
+    const uint32_t total = kvb + (c == 0 ? q_bytes : 0u);
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+                 "r"(total)
+                 : "memory");
+    tcda::bulk_load(tcda::smem_u32(kv_slot(b)),
+                    reinterpret_cast<const bf16 *>(a.kv) + ((long)tok * a.L + a.r0 + r0) * row_el,
+                    kvb, bar);
+    if (c == 0)
+      tcda::bulk_load(tcda::smem_u32(q_slot(b)), reinterpret_cast<const bf16 *>(a.q) + (long)tok * a.h,
+                      q_bytes, bar);
+  };
+  int issued = 0;  // items issued (thread 0's count)
+  if (threadIdx.x == 0)
+    for (; issued < NB && issued < nitems; issued++) issue(issued);
+  const int cc = lane % CH, g = lane / CH;
+  const int myrow = g * NR + cc / DUP;                 // the batch row whose score this lane ends with
+  const int head = warp;
+  const bool active = head < a.H;
+  const float sl2 = 1.4426950408889634f * rsqrtf((float)D);
+  uint64_t q2[4], o2[4];
+  float m = -INFINITY, lsum = 0.f;
+  int consumed = 0;
+  for (int j = 0; j < nitems; j++) {
+    const int b = j % NB, c = j % nch;
+    const uint32_t bar = tcda::smem_u32(&bars[b]);
+    const uint32_t par = (uint32_t)((j / NB) & 1);
+    if (!tcda::try_wait(bar, par)) {  // bounded; on expiry every thread stops after the barrier
+      const uint64_t t0 = tcda::gtimer();
+      while (!tcda::try_wait(bar, par)) {
+        if (abort_flag) break;
+        if (tcda::gtimer() - t0 > DREAMER_WAIT_LIMIT_NS) {
+          abort_flag = 1;
+          raise_dev_error(a.err, DEV_TIMEOUT);
+          break;
+        }
+      }
+    }
+    if (!abort_flag) consumed = j + 1;
+    // stale after a timeout; nothing is stored then
+    const uint8_t *bk = kv_slot(b) + (size_t)(head * D + cc * 8) * sizeof(bf16);
+    const uint32_t vofs = (uint32_t)(a.h * sizeof(bf16));
+    const uint32_t rstride = (uint32_t)(row_el * sizeof(bf16));
+    const int nr = min(a.chunk, nrow - c * a.chunk);
+    if (active) {
+      if (c == 0) {  // a new token: its query, a fresh softmax
+        const uint4 qw = *reinterpret_cast<const uint4 *>(q_slot(b) + (size_t)(head * D + cc * 8) * sizeof(bf16));
+        q2[0] = tcda::bf2_to_f2(qw.x); q2[1] = tcda::bf2_to_f2(qw.y);
+        q2[2] = tcda::bf2_to_f2(qw.z); q2[3] = tcda::bf2_to_f2(qw.w);
+#pragma unroll
+        for (int w = 0; w < 4; w++) o2[w] = 0ull;
+        m = -INFINITY;
+        lsum = 0.f;
+      }
+#pragma unroll 1
+      for (int b0 = 0; b0 < nr; b0 += 8) {
+        // partial dot products of this lane's 8 elements with the NR rows of its group
+        float v[NR];
+#pragma unroll
+        for (int i = 0; i < NR; i++) {
+          const int r = b0 + g * NR + i;
+          v[i] = 0.f;
+          if (r < nr) {
+            const uint4 kw = *reinterpret_cast<const uint4 *>(bk + (size_t)r * rstride);
+            uint64_t acc = tcda::mul2(q2[0], tcda::bf2_to_f2(kw.x));
+            acc = tcda::fma2(q2[1], tcda::bf2_to_f2(kw.y), acc);
+            acc = tcda::fma2(q2[2], tcda::bf2_to_f2(kw.z), acc);
+            acc = tcda::fma2(q2[3], tcda::bf2_to_f2(kw.w), acc);
+            const float2 f = tcda::up2(acc);
+            v[i] = f.x + f.y;
+          }
+        }
+        // transposed butterfly: halving exchanges over the lanes of a row, then plain ones
+#pragma unroll
+        for (int st = 0; (NR >> st) > 1; st++) {
+          const int mk = CH >> (st + 1), half = NR >> (st + 1);
+          const bool upper = (lane & mk) != 0;
+#pragma unroll
+          for (int i = 0; i < half; i++) {
+            const float send = upper ? v[i] : v[i + half];
+            const float keep = upper ? v[i + half] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, mk);
+          }
+        }
+#pragma unroll
+        for (int mk = DUP / 2; mk >= 1; mk >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], mk);
+        // online softmax over the batch (scores in log2 units)
+        const bool valid = b0 + myrow < nr;
+        const float x = valid ? v[0] * sl2 : -INFINITY;
+        const float mn = fmaxf(m, warp_max(x));
+        const float alpha = tcda::ex2a(m - mn);
+        const float p = valid ? tcda::ex2a(x - mn) : 0.f;
+        lsum = lsum * alpha + warp_sum(p) * (1.0f / DUP);
+        m = mn;
+        const uint64_t al2 = tcda::pk2(alpha, alpha);
+#pragma unroll
+        for (int w = 0; w < 4; w++) o2[w] = tcda::mul2(o2[w], al2);
+        // the weights of this group's rows, then their V rows into the 8 output elements
+#pragma unroll
+        for (int i = 0; i < NR; i++) {
+          const float pi = __shfl_sync(0xffffffffu, p, g * CH + i * DUP);
+          const int r = b0 + g * NR + i;
+          if (r < nr) {
+            const uint4 vw = *reinterpret_cast<const uint4 *>(bk + (size_t)r * rstride + vofs);
+            const uint64_t p2 = tcda::pk2(pi, pi);
+            o2[0] = tcda::fma2(p2, tcda::bf2_to_f2(vw.x), o2[0]);
+            o2[1] = tcda::fma2(p2, tcda::bf2_to_f2(vw.y), o2[1]);
+            o2[2] = tcda::fma2(p2, tcda::bf2_to_f2(vw.z), o2[2]);
+            o2[3] = tcda::fma2(p2, tcda::bf2_to_f2(vw.w), o2[3]);
+          }
+        }
+      }
+      if (c == nch - 1) {  // the token's last chunk: sum the groups, normalise, store
+        float of[8];
+#pragma unroll
+        for (int w = 0; w < 4; w++) {
+          const float2 f = tcda::up2(o2[w]);
+          of[2 * w] = f.x;
+          of[2 * w + 1] = f.y;
+        }
+#pragma unroll
+        for (int mk = CH; mk < 32; mk <<= 1)
+#pragma unroll
+          for (int i = 0; i < 8; i++) of[i] += __shfl_xor_sync(0xffffffffu, of[i], mk);
+        if (g == 0 && !abort_flag) {
+          const int tok = (int)blockIdx.x + (j / nch) * (int)gridDim.x;
+          const float inv = 1.0f / lsum;
+#pragma unroll
+          for (int i = 0; i < 8; i++) of[i] *= inv;
+          store8(reinterpret_cast<bf16 *>(a.out) + (long)tok * a.ldo + a.col0 + head * D + cc * 8, of);
         }
       }
     }

@@ -51,6 +51,7 @@ struct dreamer_handle {
   void *k3 = nullptr;            // [E][3 d_r] bf16: router keys repeated for split scores
   void *kEt = nullptr;           // [d_r][E] bf16: router keys transposed (CUDA-core scores)
   int num_sms = 148;
+  int prio_hi = 0;   // the device's most urgent launch priority (depth attention beside SA)
   int qkv_perm = 0;  // q_SA / k_SA columns of the fused QKV weight in EpiQKV perm order
   int prefill_ok = 1;  // bf16: the prefill shapes are ones the tcgen05 kernels take
 #ifdef DREAMER_TEST_HOOKS
@@ -61,9 +62,11 @@ struct dreamer_handle {
   int *err_host = nullptr;       // pinned copy of the device error flag (async)
   cudaStream_t side = nullptr;   // second stream: DA runs beside SA
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  cudaStream_t side2 = nullptr;  // third stream: expert attention beside DA/SA/O (layout 2)
+  cudaEvent_t ev_fork2 = nullptr, ev_join2 = nullptr;
   int use_graph = 1;
   int use_pdl = 1;               // programmatic dependent launch between kernels of a stream
-  bool pdl_ok[2] = {false, false};  // main / side stream: the last operation was a kernel
+  bool pdl_ok[3] = {false, false, false};  // main / side / side2: the last operation was a kernel
   struct GraphEntry {
     int kind;                    // 0 forward, 1 decode
     const void *key[5];
@@ -156,24 +159,33 @@ static thread_local uint64_t g_launches_simt = 0;
 // that for the stream and records that a kernel is now last; pdl_break() records any other
 // operation (copy, memset, event wait).  Off while stages are timed by events.
 static bool pdl_take(dreamer_handle *h, cudaStream_t s) {
-  bool &ok = h->pdl_ok[s == h->side ? 1 : 0];
+  bool &ok = h->pdl_ok[s == h->side ? 1 : (s == h->side2 ? 2 : 0)];
   const bool r = ok && h->use_pdl && !h->prof;
   ok = true;
   return r;
 }
-static void pdl_break(dreamer_handle *h, cudaStream_t s) { h->pdl_ok[s == h->side ? 1 : 0] = false; }
+static void pdl_break(dreamer_handle *h, cudaStream_t s) {
+  h->pdl_ok[s == h->side ? 1 : (s == h->side2 ? 2 : 0)] = false;
+}
 
-// launch_kc: with thread-block clusters of `cluster` CTAs along x
+// launch_kx: with thread-block clusters of `cluster` CTAs along x and, for prio != 0, the
+// launch priority prio (lower = more urgent: its CTAs are placed before pending CTAs of
+// kernels launched with the default priority)
 template <typename... P, typename... A>
-static void launch_kc(dreamer_handle *h, int cluster, void (*kern)(P...), dim3 grid, dim3 block,
-                      size_t smem, cudaStream_t s, A &&...args) {
+static void launch_kx(dreamer_handle *h, int cluster, int prio, void (*kern)(P...), dim3 grid,
+                      dim3 block, size_t smem, cudaStream_t s, A &&...args) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute at[2];
+  cudaLaunchAttribute at[3];
   int na = 0;
+  if (prio != 0) {
+    at[na].id = cudaLaunchAttributePriority;
+    at[na].val.priority = prio;
+    na++;
+  }
   if (pdl_take(h, s)) {
     at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[na].val.programmaticStreamSerializationAllowed = 1;
@@ -190,6 +202,11 @@ static void launch_kc(dreamer_handle *h, int cluster, void (*kern)(P...), dim3 g
   cfg.numAttrs = na;
   ++g_launches;
   cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+template <typename... P, typename... A>
+static void launch_kc(dreamer_handle *h, int cluster, void (*kern)(P...), dim3 grid, dim3 block,
+                      size_t smem, cudaStream_t s, A &&...args) {
+  launch_kx(h, cluster, 0, kern, grid, block, smem, s, std::forward<A>(args)...);
 }
 template <typename... P, typename... A>
 static void launch_k(dreamer_handle *h, void (*kern)(P...), dim3 grid, dim3 block, size_t smem,
@@ -359,11 +376,18 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     }
     if (const char *ev = getenv("DREAMER_NO_GRAPH")) h->use_graph = atoi(ev) ? 0 : 1;
     if (const char *ev = getenv("DREAMER_NO_PDL")) h->use_pdl = atoi(ev) ? 0 : 1;
+    {
+      int least = 0, greatest = 0;
+      if (cudaDeviceGetStreamPriorityRange(&least, &greatest) == cudaSuccess) h->prio_hi = greatest;
+    }
     CK(cudaHostAlloc((void **)&h->err_host, sizeof(int), cudaHostAllocDefault));
     *h->err_host = 0;
     CK(cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
     CK(cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
     CK(cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming));
+    CK(cudaStreamCreateWithFlags(&h->side2, cudaStreamNonBlocking));
+    CK(cudaEventCreateWithFlags(&h->ev_fork2, cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&h->ev_join2, cudaEventDisableTiming));
     // ---- weights
     DALLOC(h->g, hd * es);
     CK(cudaMemcpyAsync(h->g, w->rms_gain, hd * es, cudaMemcpyDeviceToDevice, s));
@@ -519,6 +543,9 @@ extern "C" void dreamer_destroy(dreamer_handle *h) {
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
   if (h->ev_join) cudaEventDestroy(h->ev_join);
   if (h->side) cudaStreamDestroy(h->side);
+  if (h->ev_fork2) cudaEventDestroy(h->ev_fork2);
+  if (h->ev_join2) cudaEventDestroy(h->ev_join2);
+  if (h->side2) cudaStreamDestroy(h->side2);
   if (h->err_host) cudaFreeHost(h->err_host);
   for (void *p : h->allocs) cudaFree(p);
   delete h;
@@ -555,10 +582,13 @@ static void launch_attn(const AttnArgs &a, int d, cudaStream_t s) {
   }
 }
 
-// depth attention, one CTA per token streaming its depth history through shared memory
-// depth attention: as many CTAs as fit on the GPU, each streaming its tokens' depth runs
+// Depth attention: persistent CTAs, each streaming its tokens' depth runs through shared
+// memory.  sms = 0: as many CTAs as are resident at once on the whole GPU (two buffers, two
+// CTAs an SM).  sms > 0 (beside SA): sms CTAs that each own an SM (four buffers, at least
+// 116 KB of shared memory so that no other CTA fits beside), launched at the most urgent
+// priority so that they take their SMs before SA's pending CTAs.
 template <typename T>
-static void launch_da_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStream_t s) {
+static void launch_da_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStream_t s, int sms) {
   DaBulkArgs a{};
   a.n_tok = r.n_q; a.H = r.H; a.h = r.h; a.L = r.L; a.l = r.l; a.r0 = r.r0;
   const long row_bytes = 2L * r.h * sizeof(T);
@@ -567,27 +597,53 @@ static void launch_da_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStre
   if (chunk > r.l + 1 - r.r0) chunk = r.l + 1 - r.r0;
   a.chunk = chunk;
   a.q = r.q; a.kv = r.kv; a.out = r.out; a.ldo = r.ldo; a.col0 = r.col0; a.err = r.err;
-  const int smem = (int)(2 * (chunk * row_bytes + r.h * (long)sizeof(T)));
+  const bool own = sms > 0;
+  const int nb = own ? 4 : 2;
+  int smem = (int)(nb * (chunk * row_bytes + r.h * (long)sizeof(T)));
+  if (own && smem < 116 * 1024) smem = 116 * 1024;
   const int threads = 32 * r.H;
   auto go = [&](void (*kern)(DaBulkArgs)) {
-    // set for the kernel launched (the four head sizes share one pointer type)
+    // set for the kernel launched (the head sizes share one pointer type)
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    // persistent: as many CTAs as are resident at once (registers, shared memory, threads)
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess ||
-        per_sm < 1)
-      per_sm = 1;
-    long grid = (long)h->num_sms * per_sm;
+    long grid;
+    if (own) {
+      grid = sms;
+    } else {  // as many CTAs as are resident at once (registers, shared memory, threads)
+      int per_sm = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess ||
+          per_sm < 1)
+        per_sm = 1;
+      grid = (long)h->num_sms * per_sm;
+    }
     if (grid > a.n_tok) grid = a.n_tok;
     if (grid < 1) grid = 1;
-    launch_k(h, kern, dim3((unsigned)grid), dim3(threads), smem, s, a);
+    launch_kx(h, 1, own ? h->prio_hi : 0, kern, dim3((unsigned)grid), dim3(threads), smem, s, a);
   };
-  switch (d) {
-    case 16: go(da_bulk_kernel<T, 16>); break;
-    case 32: go(da_bulk_kernel<T, 32>); break;
-    case 64: go(da_bulk_kernel<T, 64>); break;
-    default: go(da_bulk_kernel<T, 128>); break;
+  if (sizeof(T) == 2 && (d == 64 || d == 128)) {
+    // bf16, head dim 64 / 128: batches of 8 rows, chunks of a multiple of 8 rows (about
+    // 64 KB), three buffers
+    int c8 = (int)((64 * 1024) / row_bytes) / 8 * 8;
+    if (c8 < 8) c8 = 8;
+    a.chunk = c8 < r.l + 1 - r.r0 ? c8 : r.l + 1 - r.r0;
+    smem = (int)(3 * (a.chunk * row_bytes + r.h * (long)sizeof(T)));
+    if (own && smem < 116 * 1024) smem = 116 * 1024;
+    if (d == 64) go(da_fast_kernel<64>);
+    else go(da_fast_kernel<128>);
+  } else if (own) {
+    switch (d) {
+      case 16: go(da_bulk_kernel<T, 16, 4>); break;
+      case 32: go(da_bulk_kernel<T, 32, 4>); break;
+      case 64: go(da_bulk_kernel<T, 64, 4>); break;
+      default: go(da_bulk_kernel<T, 128, 4>); break;
+    }
+  } else {
+    switch (d) {
+      case 16: go(da_bulk_kernel<T, 16, 2>); break;
+      case 32: go(da_bulk_kernel<T, 32, 2>); break;
+      case 64: go(da_bulk_kernel<T, 64, 2>); break;
+      default: go(da_bulk_kernel<T, 128, 2>); break;
+    }
   }
 }
 
@@ -617,9 +673,10 @@ static void launch_dec_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStr
 
 // depth attention (mode 0) or split decode attention + merge (mode 2)
 template <typename T>
-static void launch_rows(dreamer_handle *h, const RowsArgs &a, int d, cudaStream_t s) {
+static void launch_rows(dreamer_handle *h, const RowsArgs &a, int d, cudaStream_t s,
+                        int da_sms = 0) {
   if (a.mode == 0 && a.H <= 32 && 2L * a.h * (long)sizeof(T) <= 48 * 1024) {
-    launch_da_bulk<T>(h, a, d, s);
+    launch_da_bulk<T>(h, a, d, s, da_sms);
     return;
   }
   if (a.mode == 2) {
@@ -647,6 +704,35 @@ static void launch_rows(dreamer_handle *h, const RowsArgs &a, int d, cudaStream_
       default: launch_k(h, attn_merge_kernel<T, 128>, dim3(mb), dim3(256), 0, s, a); break;
     }
   }
+}
+
+// SMs depth attention gets when it runs beside causal SA in a prefill depth step (papernotes
+// "Key design 1": DA and SA computed in parallel).  Both kernels fill whole SMs, so run side
+// by side at full width they would take turns; instead DA takes n SMs of its own and SA the
+// rest.  n balances DA's streamed K/V bytes on n SMs against SA's tensor-core work on the
+// other SMs, from per-SM rates measured on B200: DA about DA_BYTES_SM bytes/s an SM, up to
+// DA_BYTES_ALL over the whole chip; flash SA about SA_FLOPS_SM_D128 (head dim 128) or
+// SA_FLOPS_SM_D64 flop/s an SM.  0 when the split does not pay (DA then runs at full width).
+static constexpr double DA_BYTES_SM = 26e9, DA_BYTES_ALL = 4.7e12;
+static constexpr double SA_FLOPS_SM_D128 = 5.3e12, SA_FLOPS_SM_D64 = 2.5e12;
+static int da_beside_sa_sms(const dreamer_handle *h, int l, int r0) {
+  const dreamer_config &c = h->cfg;
+  const double hd = c.hidden, T = (double)c.batch * c.seq;
+  const double bytes = T * (double)(l + 1 - r0) * 4.0 * hd;  // the depths' bf16 K and V rows
+  const double flops = 2.0 * hd * c.batch * (double)c.seq * (c.seq + 1.0);  // causal half
+  const double r_sa = c.head_dim == 128 ? SA_FLOPS_SM_D128 : SA_FLOPS_SM_D64;
+  const int S = h->num_sms;
+  double best = 1e30;
+  int bn = 0;
+  for (int n = 8; n <= S - 8; n++) {
+    const double t = fmax(bytes / fmin(n * DA_BYTES_SM, DA_BYTES_ALL), flops / ((S - n) * r_sa));
+    if (t < best) {
+      best = t;
+      bn = n;
+    }
+  }
+  const double apart = bytes / DA_BYTES_ALL + flops / (S * r_sa);
+  return best < 0.9 * apart ? bn : 0;
 }
 
 template <typename T, int SEG>
@@ -758,6 +844,66 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   if (first)
     launch_k(h, rmsnorm_kernel<T>, dim3(cdiv(n, 8)), dim3(256), 0, s, (const T *)io.x_in,
              (const float *)nullptr, (const T *)h->g, (T *)h->xh, h->inv_rms, n, hd, c.rms_eps);
+  // Expert attention (steps 6-7 below): routing on y (fully parallel layout: on x^), token
+  // grouping and the expert FFNs, enqueued on stream st.  Defined here so that the fully
+  // parallel layout can start it first, on a stream of its own.
+  const void *ein = c.variant == 2 ? h->xh : h->y;
+  // few rows per expert (decode): every routed row computes its own expert FFN, unsorted
+  const bool by_rows = (long)n * k < 8L * E && (m == 16 || m == 32 || m == 64) &&
+                       hd <= 2048 && hd % 8 == 0;
+  auto run_ea = [&](cudaStream_t st) {
+    mark(h, s, DREAMER_STAGE_EA_ROUTE);
+    if (by_rows) {
+      route_rows<T>(h, 0, l, ein, n, h->eidx, h->ew, h->counts + (size_t)l * E, nullptr, st);
+    } else {
+      // ecnt / ecursor are zero here: cleared at init and by every depth's combine kernel
+      route_rows<T>(h, 0, l, ein, n, h->eidx, h->ew, h->counts + (size_t)l * E, h->ecnt, st);
+      mark(h, s, DREAMER_STAGE_PERMUTE);
+      if (E <= 8192) {
+        launch_k(h, permute_kernel, dim3(cdiv((long)n * k, 1024)), dim3(1024),
+                 (size_t)(E + 1) * sizeof(int), st, (const int *)h->ecnt, E, (const int *)h->eidx,
+                 n * k, h->eoffs, h->etiles_a, 64, h->etiles_b, 128, h->ecursor, h->erows, h->einv);
+      } else {
+        launch_k(h, scan_kernel, dim3(1), dim3(1024), 0, st, (const int *)h->ecnt, E, h->eoffs,
+                 h->etiles_a, 64, h->etiles_b, 128, h->ecursor);
+        launch_k(h, scatter_kernel, dim3(cdiv((long)n * k, 256)), dim3(256), 0, st,
+                 (const int *)h->eidx, n * k, h->ecursor, h->erows, h->einv);
+      }
+    }
+    // 7. expert FFNs: H = SiLU(X W1_e), acc[token] += w * H W2_e
+    mark(h, s, DREAMER_STAGE_EXPERTS);
+    if (by_rows) {
+      auto kern = m == 16 ? expert_rows_kernel<T, 16>
+                          : (m == 32 ? expert_rows_kernel<T, 32> : expert_rows_kernel<T, 64>);
+      launch_k(h, kern, dim3(n * k), dim3(256), 0, st, (const T *)ein, (const int *)h->eidx,
+               n * k, k, hd, (const T *)h->w1_t, (const T *)h->w2_t, (T *)h->Ybuf);
+    } else if (tc) {
+      if (!(tc_expert_ok(h) && tc_expert(h, ein, n, st))) h->path_err = 1;
+    } else {
+      const int etiles = cdiv((long)n * k, 64) + E;
+      GemmArgs up{};
+      up.N = m; up.K = hd; up.G = E; up.M = n * k; up.goffs = h->eoffs; up.tile_offs = h->etiles_a;
+      up.arow = h->erows; up.arow_div = k; up.A = ein; up.lda = hd; up.B = h->w1_t; up.ldb = hd;
+      up.bgstride = (long)m * hd;
+      gemm_simt<T, T, 16>(up, etiles, EpiUp<T>{m, (T *)h->Hbuf}, st);
+      GemmArgs dn{};
+      dn.N = hd; dn.K = m; dn.G = E; dn.M = n * k; dn.goffs = h->eoffs; dn.tile_offs = h->etiles_a;
+      dn.arow = nullptr; dn.arow_div = 1; dn.A = h->Hbuf; dn.lda = m; dn.B = h->w2_t; dn.ldb = m;
+      dn.bgstride = (long)m * hd;
+      gemm_simt<T, T, 16>(dn, etiles, EpiDownStore<T>{hd, (T *)h->Ybuf}, st);
+    }
+  };
+  // the fully parallel layout ([notes] ablation table): expert attention reads x^ only, so
+  // with bf16 it runs on a third stream beside the projections, DA, SA and O (one more branch
+  // of the captured graph), joined before the combine; with stage profiling on it runs in line
+  const bool ea_beside = c.variant == 2 && c.dtype == 1 && !h->prof;
+  if (ea_beside) {
+    cudaEventRecord(h->ev_fork2, s);
+    cudaStreamWaitEvent(h->side2, h->ev_fork2, 0);
+    pdl_break(h, h->side2);
+    run_ea(h->side2);
+    cudaEventRecord(h->ev_join2, h->side2);
+  }
   // 2. projection router and token grouping (linear-MoE QKV/O)
   const int *prow = nullptr;
   const float *psig = nullptr;
@@ -877,19 +1023,24 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     // 3. fused QKV projection with RoPE / depth RoPE epilogue, DA KV write
     qkv_gemm(h->xh, 0, 6 * hd);
     // 4. DA || SA (papernotes "Key design 1": run in parallel for throughput).  DA runs
-    // on the side stream beside SA (two branches of the captured graph); with stage
-    // profiling on they run one after the other so each stage's time is its own.
+    // on the side stream beside SA (two branches of the captured graph), on SMs of its own
+    // where that pays; with stage profiling on they run one after the other (same launch
+    // shapes) so each stage's time is its own.
+    const int da_sms = io.mode == 0 && c.dtype == 1 ? da_beside_sa_sms(h, l, da.r0) : 0;
     if (h->prof) {
       mark(h, s, DREAMER_STAGE_DA);
-      launch_rows<T>(h, da, d, s);
+      launch_rows<T>(h, da, d, s, da_sms);
     } else {
       cudaEventRecord(h->ev_fork, s);
       cudaStreamWaitEvent(h->side, h->ev_fork, 0);
       pdl_break(h, h->side);
-      launch_rows<T>(h, da, d, h->side);
+      launch_rows<T>(h, da, d, h->side, da_sms);
       cudaEventRecord(h->ev_join, h->side);
     }
     mark(h, s, DREAMER_STAGE_SA);
+    // with DA on its own SMs, SA starts after the projection has completed, as DA does, so that
+    // DA's urgent CTAs are placed first (no early launch of SA's CTAs into the projection's tail)
+    if (da_sms > 0) pdl_break(h, s);
     run_sa(s);
     if (!h->prof) {
       cudaStreamWaitEvent(s, h->ev_join, 0);
@@ -898,50 +1049,12 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     // 5. O projection, residual y = x^ + DA + SA
     o_gemm(h->attn, 0, 2 * hd, res_xhat, h->y);
   }
-  // 6. expert attention routing on y (fully parallel layout: on x^)
-  const void *ein = c.variant == 2 ? h->xh : h->y;
-  // few rows per expert (decode): every routed row computes its own expert FFN, unsorted
-  const bool by_rows = (long)n * k < 8L * E && (m == 16 || m == 32 || m == 64) &&
-                       hd <= 2048 && hd % 8 == 0;
-  mark(h, s, DREAMER_STAGE_EA_ROUTE);
-  if (by_rows) {
-    route_rows<T>(h, 0, l, ein, n, h->eidx, h->ew, h->counts + (size_t)l * E, nullptr, s);
+  // 6-7. expert attention in line, or the join of its own stream
+  if (!ea_beside) {
+    run_ea(s);
   } else {
-    // ecnt / ecursor are zero here: cleared at init and by every depth's combine kernel
-    route_rows<T>(h, 0, l, ein, n, h->eidx, h->ew, h->counts + (size_t)l * E, h->ecnt, s);
-    mark(h, s, DREAMER_STAGE_PERMUTE);
-    if (E <= 8192) {
-      launch_k(h, permute_kernel, dim3(cdiv((long)n * k, 1024)), dim3(1024),
-               (size_t)(E + 1) * sizeof(int), s, (const int *)h->ecnt, E, (const int *)h->eidx,
-               n * k, h->eoffs, h->etiles_a, 64, h->etiles_b, 128, h->ecursor, h->erows, h->einv);
-    } else {
-      launch_k(h, scan_kernel, dim3(1), dim3(1024), 0, s, (const int *)h->ecnt, E, h->eoffs,
-               h->etiles_a, 64, h->etiles_b, 128, h->ecursor);
-      launch_k(h, scatter_kernel, dim3(cdiv((long)n * k, 256)), dim3(256), 0, s,
-               (const int *)h->eidx, n * k, h->ecursor, h->erows, h->einv);
-    }
-  }
-  // 7. expert FFNs: H = SiLU(X W1_e), acc[token] += w * H W2_e
-  mark(h, s, DREAMER_STAGE_EXPERTS);
-  if (by_rows) {
-    auto kern = m == 16 ? expert_rows_kernel<T, 16>
-                        : (m == 32 ? expert_rows_kernel<T, 32> : expert_rows_kernel<T, 64>);
-    launch_k(h, kern, dim3(n * k), dim3(256), 0, s, (const T *)ein, (const int *)h->eidx,
-             n * k, k, hd, (const T *)h->w1_t, (const T *)h->w2_t, (T *)h->Ybuf);
-  } else if (tc) {
-    if (!(tc_expert_ok(h) && tc_expert(h, ein, n, s))) h->path_err = 1;
-  } else {
-    const int etiles = cdiv((long)n * k, 64) + E;
-    GemmArgs up{};
-    up.N = m; up.K = hd; up.G = E; up.M = n * k; up.goffs = h->eoffs; up.tile_offs = h->etiles_a;
-    up.arow = h->erows; up.arow_div = k; up.A = ein; up.lda = hd; up.B = h->w1_t; up.ldb = hd;
-    up.bgstride = (long)m * hd;
-    gemm_simt<T, T, 16>(up, etiles, EpiUp<T>{m, (T *)h->Hbuf}, s);
-    GemmArgs dn{};
-    dn.N = hd; dn.K = m; dn.G = E; dn.M = n * k; dn.goffs = h->eoffs; dn.tile_offs = h->etiles_a;
-    dn.arow = nullptr; dn.arow_div = 1; dn.A = h->Hbuf; dn.lda = m; dn.B = h->w2_t; dn.ldb = m;
-    dn.bgstride = (long)m * hd;
-    gemm_simt<T, T, 16>(dn, etiles, EpiDownStore<T>{hd, (T *)h->Ybuf}, s);
+    cudaStreamWaitEvent(s, h->ev_join2, 0);
+    pdl_break(h, s);
   }
   // per-depth dumps (before the combine replaces x^ with the next depth's)
   trace_depth(h, io.tr, l, n, io.mode == 0, s);
@@ -1089,6 +1202,7 @@ static int forward_impl(dreamer_handle *h, const void *x_in, void *x_out, int l0
   CK(cudaMemsetAsync(h->pcnt, 0, 2 * (size_t)((c.n_proj_experts > 0 ? c.n_proj_experts : 1) + 1) * sizeof(int), s));
   pdl_break(h, s);
   pdl_break(h, h->side);
+  pdl_break(h, h->side2);
   DepthIO io{};
   io.mode = 0; io.n_tok = n; io.x_in = x_in; io.x_out = x_out; io.tr = tr;
   io.da_kv = da_kv ? da_kv : h->da_kv_int;
@@ -1146,6 +1260,7 @@ static int decode_impl(dreamer_handle *h, const void *x_new, void *kc, void *vc,
   CK(cudaMemsetAsync(h->pcnt, 0, 2 * (size_t)((c.n_proj_experts > 0 ? c.n_proj_experts : 1) + 1) * sizeof(int), s));
   pdl_break(h, s);
   pdl_break(h, h->side);
+  pdl_break(h, h->side2);
   DepthIO io{};
   io.mode = 1; io.n_tok = n; io.x_in = x_new; io.x_out = x_out; io.tr = tr;
   io.da_kv = h->da_kv_int;

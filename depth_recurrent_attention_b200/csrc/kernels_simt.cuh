@@ -388,6 +388,7 @@ template <typename T> struct EpiUp {
 // r) is written once in dtype; the weighted sum over a token's k rows happens in
 // combine_norm_kernel (no atomics, fixed summation order).
 template <typename T> struct EpiDownStore {
+  static constexpr bool TMA_STORE = true;  // tcgen05 engine: tile stores through a tensor map
   int h;
   T *Y;  // [rows][h], expert-sorted order
   template <int SEG>

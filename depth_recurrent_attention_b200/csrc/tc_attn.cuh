@@ -9,11 +9,16 @@
 //   warp 1      TMEM allocator + MMA issuer: S_A(j), S_B(j) = Q K_j^T into one TMEM buffer
 //               per tile, then O_t += P_t(j-1) V_(j-1) for both tiles (one block behind, so the
 //               tensor core computes block j's scores while the softmax works on j-1)
-//   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B (one query row per thread):
-//               pass 1 over S for the row max, pass 2 writes P = exp2(s - m_ref) as bf16 into
-//               the swizzled K-major operand in shared memory and sums it.  O lives in TMEM and
-//               is only rescaled when the running max grows by more than 2^8 (P stays <= 256),
-//               so most blocks need no O traffic at all; the last step divides O by the sum.
+//   warps 3-10  softmax, one query row per thread: tile A on warps 4, 5, 6, 3 and tile B on
+//               warps 8, 9, 10, 7 (a warp reads the TMEM lanes of its warp index mod 4), 11
+//               warps in all so that a thread may hold a row of 128 scores in registers:
+//               the row's 128 scores come out of TMEM in one batch of loads (S is released to
+//               the next QK^T right away), then the row max, and P = exp2(s - m_ref) written
+//               as bf16 into the swizzled K-major operand in shared memory and summed (a
+//               quarter of the exponentials on the FMA pipe, the rest on MUFU).  O lives in
+//               TMEM and is only rescaled when the running max grows by more than 2^8 (P stays
+//               <= 256), so most blocks need no O traffic at all; the last step divides O by
+//               the sum.
 // V is consumed in its natural [key][d] layout as an MN-major B operand.
 #pragma once
 #include "tc_common.cuh"
@@ -76,7 +81,7 @@ struct SaCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(352, 1)
     tc_sa_kernel(const __grid_constant__ CUtensorMap tm, SaArgs a) {
   using C = SaCfg<D>;
   constexpr int CH = C::CH, KST = C::KST, VST = C::VST;
@@ -231,9 +236,9 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (ok) issue_pv(nb - 1);
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------- softmax (tile A: warps 4-7, B: 8-11)
-    const int t = (warp - 4) >> 2;
+  } else if (warp >= 3) {
+    // ------------------------------------------------- softmax (tile A: warps 3-6, B: 7-10)
+    const int t = warp < 7 ? 0 : 1;
     const int nbt = t == 0 ? nbA : nbB;
     const int qt = t == 0 ? qtA : qtB;
     if (nbt > 0) {
@@ -250,26 +255,26 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(smem_u32(&s_full[t]), j & 1, abort_flag, a.err)) { ok = false; break; }
         tc_fence_after();
         const bool diag = (j == qt);
-        // pass 1: row max of the raw scores (the scale is positive: applied to the max)
+        const int lim = qi - j * 128;  // diagonal block: last visible key of the row
+        // the row's 128 scores into registers with four loads in flight, then S is free for
+        // the next block's QK^T while this block's softmax runs
+        float sv[128];
+#pragma unroll
+        for (int c = 0; c < 128; c += 32) tmem_ld32_async(sbuf + c, sv + c);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 128; c += 32) tmem_ld_fence(sv + c);
+        tc_fence_before();
+        mbar_arrive(smem_u32(&s_free[t]));
+        // row max of the raw scores (the scale is positive: applied to the max)
         float mraw = -INFINITY;
         if (!diag) {
 #pragma unroll
-          for (int c = 0; c < 128; c += 32) {
-            float sv[32];
-            tmem_ld32(sbuf + c, sv);
-#pragma unroll
-            for (int i = 0; i < 32; i++) mraw = fmaxf(mraw, sv[i]);
-          }
+          for (int i = 0; i < 128; i++) mraw = fmaxf(mraw, sv[i]);
         } else {
-          const int lim = qi - j * 128;  // last visible key of this row inside the block
 #pragma unroll
-          for (int c = 0; c < 128; c += 32) {
-            float sv[32];
-            tmem_ld32(sbuf + c, sv);
-#pragma unroll
-            for (int i = 0; i < 32; i++)
-              if (c + i <= lim) mraw = fmaxf(mraw, sv[i]);
-          }
+          for (int i = 0; i < 128; i++)
+            if (i <= lim) mraw = fmaxf(mraw, sv[i]);
         }
         const float mx = mraw * a.scale_log2;
         // lazy rescale: move the reference max only when the row max grows by more than 8
@@ -280,58 +285,45 @@ __global__ void __launch_bounds__(384, 1)
           m_new = mx;
           alpha = ex2(m_ref - mx);
         }
+        // P_t(j-1) V was consumed: its P buffer is free and O_t holds every earlier block
         if (j > 0) {
-          // P_t(j-1) V was consumed and O_t holds every earlier block
           if (!mbar_wait(smem_u32(&pv_done[t]), (j - 1) & 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-            for (int c = 0; c < D; c += 32) {
-              float ov[32];
-              tmem_ld32(obuf + c, ov);
-#pragma unroll
-              for (int i = 0; i < 32; i++) ov[i] *= alpha;
-              tmem_st32(obuf + c, ov);
-            }
-          }
         }
-        // pass 2: P = 2^(s * scale - m) as bf16, K-major SW128 (key chunk kc at kc * TILE,
-        // 16-byte unit u of the row at ((u ^ (row & 7)) << 4))
+        // P = 2^(s * scale - m) as bf16, K-major SW128 (key chunk kc at kc * TILE, 16-byte unit
+        // u of the row at ((u ^ (row & 7)) << 4)), summed; one 32-key chunk in four on the FMA
+        // pipe (ex2_poly), the rest on the MUFU unit
         const float nm = -m_new;
-        const int lim = qi - j * 128;  // diagonal block: last visible key of the row
         float rs = 0.f;
 #pragma unroll
-        for (int c = 0; c < 128; c += 32) {
-          float sv[32];
-          tmem_ld32(sbuf + c, sv);
-          if (!diag) {  // every key visible: no mask in the hot loop
+        for (int u8 = 0; u8 < 16; u8++) {
+          const int kc = u8 >> 3, u = u8 & 7;
+          float p[8];
 #pragma unroll
-            for (int i = 0; i < 32; i++) {
-              sv[i] = ex2(fmaf(sv[i], a.scale_log2, nm));
-              rs += sv[i];
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; i++) {
-              const float p = ex2(fmaf(sv[i], a.scale_log2, nm));
-              sv[i] = (c + i <= lim) ? p : 0.f;
-              rs += sv[i];
-            }
+          for (int e = 0; e < 8; e++) {
+            const int i = u8 * 8 + e;
+            const float x = fmaf(sv[i], a.scale_log2, nm);
+            p[e] = (i >= 32 && i < 64) ? ex2_poly(x) : ex2(x);
+            if (diag && i > lim) p[e] = 0.f;
+            rs += p[e];
           }
-          const int kc = c >> 6;
+          uint4 pk;
+          __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&pk);
 #pragma unroll
-          for (int uu = 0; uu < 4; uu++) {
-            const int u = ((c & 63) >> 3) + uu;
-            uint4 pk;
-            __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&pk);
+          for (int e = 0; e < 4; e++) p2[e] = __floats2bfloat162_rn(p[2 * e], p[2 * e + 1]);
+          *reinterpret_cast<uint4 *>(prow + kc * C::TILE + ((u ^ (row & 7)) << 4)) = pk;
+        }
+        // O rescaled before P_t(j) V accumulates into it (issued after p_full below)
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int c = 0; c < D; c += 32) {
+            float ov[32];
+            tmem_ld32(obuf + c, ov);
 #pragma unroll
-            for (int e = 0; e < 4; e++)
-              p2[e] = __floats2bfloat162_rn(sv[uu * 8 + 2 * e], sv[uu * 8 + 2 * e + 1]);
-            *reinterpret_cast<uint4 *>(prow + kc * C::TILE + ((u ^ (row & 7)) << 4)) = pk;
+            for (int i = 0; i < 32; i++) ov[i] *= alpha;
+            tmem_st32(obuf + c, ov);
           }
         }
-        tc_fence_before();
-        mbar_arrive(smem_u32(&s_free[t]));
         l = l * alpha + rs;
         m_ref = m_new;
         fence_proxy_async();
@@ -401,14 +393,14 @@ static bool tc_sa(dreamer_handle *h, cudaStream_t s) {
       cudaFuncSetAttribute(tc::tc_sa_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SaCfg<64>::SMEM);
       set = true;
     }
-    launch_k(h, tc::tc_sa_kernel<64>, dim3(grid), dim3(384), tc::SaCfg<64>::SMEM, s, tm, a);
+    launch_k(h, tc::tc_sa_kernel<64>, dim3(grid), dim3(352), tc::SaCfg<64>::SMEM, s, tm, a);
   } else {
     static bool set = false;
     if (!set) {
       cudaFuncSetAttribute(tc::tc_sa_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SaCfg<128>::SMEM);
       set = true;
     }
-    launch_k(h, tc::tc_sa_kernel<128>, dim3(grid), dim3(384), tc::SaCfg<128>::SMEM, s, tm, a);
+    launch_k(h, tc::tc_sa_kernel<128>, dim3(grid), dim3(352), tc::SaCfg<128>::SMEM, s, tm, a);
   }
   return true;
 }

@@ -5,7 +5,9 @@
 //             -> rounded to bf16 into shared memory, in the K-major swizzled layout that
 //                tcgen05.mma reads (the layout TMA writes for a box m elements wide)
 //   phase 2   Y_rows = H W2_e in chunks of 256 output columns, K = m, each chunk stored in
-//             dtype to Y[sorted row]
+//             dtype to Y[sorted row]: an epilogue warp whose 32 rows all belong to the tile
+//             writes its 32 x 64 blocks into shared-memory boxes and stores them with TMA
+//             (tensor map tmY); the warp holding the expert's last rows stores row by row
 // H never leaves the SM.  Rounding points are those of the two-GEMM form (H in bf16, Y in
 // bf16), so the result is the same.
 //
@@ -44,8 +46,9 @@ struct TcFfnCfg {
   static constexpr int B2_BYTES = 256 * M * 2;   // W2_e^T chunk: 256 rows x M K
   static constexpr int H_BYTES = 128 * M * 2;
   static constexpr int THREADS = 256;
-  static constexpr int SMEM_USED =
-      STAGES * (A_BYTES + B1_BYTES) + 2 * B2_BYTES + H_BYTES + 1024 /*align*/ + 256 /*bars*/;
+  static constexpr int BOX_BYTES = 4 * 2 * 4096;  // two 32 x 64 bf16 boxes per epilogue warp
+  static constexpr int SMEM_USED = STAGES * (A_BYTES + B1_BYTES) + 2 * B2_BYTES + H_BYTES +
+                                   1024 /*align*/ + 1024 /*bars*/ + BOX_BYTES;
   // at least 120 KB so that a second CTA never shares the SM (and its 512 TMEM columns)
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static_assert(SMEM_USED <= 227 * 1024, "shared memory");
@@ -78,7 +81,7 @@ __device__ __forceinline__ int ffn_swz(int r, int c) {
 template <int M, int STAGES>
 __global__ void __launch_bounds__(256, 1)
     tc_ffn_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
-                  TcFfnArgs a) {
+                  const __grid_constant__ CUtensorMap tmY, TcFfnArgs a) {
   using C = TcFfnCfg<M, STAGES>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -93,6 +96,7 @@ __global__ void __launch_bounds__(256, 1)
   uint64_t *hready = rempty + 2, *hfree = hready + 1;        // H in shared memory
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(hfree + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  uint8_t *sbox = reinterpret_cast<uint8_t *>(bars) + 1024;  // 1024-byte aligned store boxes
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KB = a.H / 64, NC = a.H / 256;
@@ -114,6 +118,7 @@ __global__ void __launch_bounds__(256, 1)
     fence_mbar_init();
     prefetch_tmap(&tmW1);
     prefetch_tmap(&tmW2);
+    prefetch_tmap(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -230,7 +235,7 @@ __global__ void __launch_bounds__(256, 1)
     // ------------------------------------------------------------- epilogue
     const int qq = warp & 3;  // TMEM lane quarter
     const int row = qq * 32 + lane;
-    int j = 0, it = 0;
+    int j = 0, it = 0, nbox = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < total; t += gridDim.x, it++) {
       int g, m0, m1;
@@ -271,19 +276,41 @@ __global__ void __launch_bounds__(256, 1)
         tc_fence_after();
         const uint32_t base = tmem + rg * 256 + ((uint32_t)(qq * 32) << 16);
         bf16 *yr = a.Y + (long)r * a.H + c * 256;
+        const bool full_warp = m0 + qq * 32 + 31 < m1;
 #pragma unroll 1
-        for (int sg = 0; sg < 256; sg += 32) {
-          float v[32];
+        for (int sg = 0; sg < 256; sg += 64) {
+          float v[64];
           tmem_ld32(base + sg, v);
-          if (valid) {
+          tmem_ld32(base + sg + 32, v + 32);
+          if (full_warp) {
+            uint8_t *box = sbox + ((warp - 2) * 2 + (nbox & 1)) * 4096;
+            if (lane == 0) bulk_wait_read<1>();  // this box's store of two passes ago has read it
+            __syncwarp();
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) store8(yr + sg + i, v + i);
+            for (int q = 0; q < 8; q++) {  // 16-byte chunk q of the row at (q ^ (lane & 7))
+              uint4 pk;
+              __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&pk);
+#pragma unroll
+              for (int e = 0; e < 4; e++) p2[e] = __floats2bfloat162_rn(v[8 * q + 2 * e], v[8 * q + 2 * e + 1]);
+              *reinterpret_cast<uint4 *>(box + lane * 128 + ((q ^ (lane & 7)) << 4)) = pk;
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, smem_u32(box), c * 256 + sg, m0 + qq * 32);
+              bulk_commit();
+            }
+            nbox++;
+          } else if (valid) {
+#pragma unroll
+            for (int i = 0; i < 64; i += 8) store8(yr + sg + i, v + i);
           }
         }
         tc_fence_before();
         mbar_arrive(smem_u32(&rempty[rg]));
       }
     }
+    if (lane == 0) bulk_wait_all();  // every tile store of this warp has landed
   } else {
     // ------------------------------------------------------------- gathered X rows
     const int tid = threadIdx.x - 192;  // 0..63

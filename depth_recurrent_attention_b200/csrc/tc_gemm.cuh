@@ -68,9 +68,18 @@ template <class E, class = void> struct EpiStaged { static constexpr bool value 
 template <class E> struct EpiStaged<E, std::void_t<decltype(E::STAGED)>> {
   static constexpr bool value = E::STAGED;
 };
+// Epilogues that declare TMA_STORE = true store plain bf16 rows [r][n] through a TMA tensor
+// map (tmC, box 64 columns x 32 rows, 128-byte swizzle): each epilogue warp whose 32 rows are
+// all valid writes its 32 x 64 block into a double-buffered shared-memory box and one lane
+// issues the tile store; the warp that holds a group's last rows stores them one by one with
+// the functor (rows past the group belong to the next group's tile).
+template <class E, class = void> struct EpiTma { static constexpr bool value = false; };
+template <class E> struct EpiTma<E, std::void_t<decltype(E::TMA_STORE)>> {
+  static constexpr bool value = E::TMA_STORE;
+};
 
 template <int BN, int BK, int STAGES, bool GATHER, bool STAGED = false, int EW_ = 4,
-          bool ROWPASS = false>
+          bool ROWPASS = false, bool TMAST = false>
 struct TcGemmCfg {
   static constexpr int A_BYTES = 128 * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
@@ -79,8 +88,10 @@ struct TcGemmCfg {
   static constexpr int THREADS = 64 + 32 * EW + (GATHER ? 64 : 0);
   // staged epilogues: EW warps x 32 rows x 64 fp32; row-pass epilogues with two warps a lane
   // quarter: one exchange list of up to 16 (value, raw score, index) a row
+  // TMA-store epilogues: two 4 KB boxes a warp, 1024-byte aligned after the barrier block
   static constexpr int STG_BYTES =
-      STAGED ? EW * 32 * 64 * 4 : ((ROWPASS && EW == 8) ? 128 * 16 * 12 : 0);
+      STAGED ? EW * 32 * 64 * 4
+             : ((ROWPASS && EW == 8) ? 128 * 16 * 12 : (TMAST ? 768 + EW * 2 * 4096 : 0));
   // at least 120 KB so that a second CTA never shares the SM (and its 512 TMEM columns)
   static constexpr int SMEM_USED =
       STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*bars*/ + STG_BYTES;
@@ -98,11 +109,14 @@ struct TcGemmCfg {
 template <int BN, int BK, int STAGES, bool GATHER, int SEG, class Epi, bool ROWPASS = false,
           int EW = 4>
 __global__ void __launch_bounds__(
-    TcGemmCfg<BN, BK, STAGES, GATHER, EpiStaged<Epi>::value && !ROWPASS, EW, ROWPASS>::THREADS, 1)
+    TcGemmCfg<BN, BK, STAGES, GATHER, EpiStaged<Epi>::value && !ROWPASS, EW, ROWPASS,
+              EpiTma<Epi>::value>::THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   TcGemmArgs a, Epi epi) {
+                   const __grid_constant__ CUtensorMap tmC, TcGemmArgs a, Epi epi) {
   constexpr bool STAGED = EpiStaged<Epi>::value && !ROWPASS;
-  using C = TcGemmCfg<BN, BK, STAGES, GATHER, STAGED, EW, ROWPASS>;
+  constexpr bool TMAST = EpiTma<Epi>::value && !STAGED && !ROWPASS;
+  static_assert(!TMAST || SEG == 64, "TMA-store epilogue: 64-column segments");
+  using C = TcGemmCfg<BN, BK, STAGES, GATHER, STAGED, EW, ROWPASS, TMAST>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
@@ -113,6 +127,7 @@ __global__ void __launch_bounds__(
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xempty + 4);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   float *stage_buf = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + 256);
+  uint8_t *tma_box = reinterpret_cast<uint8_t *>(bars) + 1024;  // TMAST: 1024-byte aligned
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NT = a.N / BN;
@@ -148,6 +163,7 @@ __global__ void __launch_bounds__(
     fence_mbar_init();
     prefetch_tmap(&tmB);
     if (!GATHER) prefetch_tmap(&tmA);
+    if (TMAST) prefetch_tmap(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -236,6 +252,7 @@ __global__ void __launch_bounds__(
     int mt, nt;
     typename EpiState<Epi, ROWPASS>::type st;
     int rb = 0;  // row blocks finished (row-pass exchange phase)
+    int nbox = 0;  // TMAST: tile stores issued by this warp (alternating shared-memory boxes)
     for (int it = 0; tile_at(it, mt, nt); it++) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
@@ -307,6 +324,39 @@ __global__ void __launch_bounds__(
           }
           epi.template store_rows<NIT, NV>(crow, ctok, caux, g, n0 + c0 + cj * 4, cv);
         }
+      } else if constexpr (TMAST) {
+        if (!mbar_wait(smem_u32(&tfull[acc]), aph, abort_flag, a.err)) break;
+        tc_fence_after();
+        const bool full_warp = m0 + q * 32 + 31 < m1;
+#pragma unroll 1
+        for (int sg = half; sg < BN / 64 && m0 + q * 32 < m1; sg += C::EW / 4) {
+          float v[64];
+          tmem_ld32(base + sg * 64, v);
+          tmem_ld32(base + sg * 64 + 32, v + 32);
+          if (full_warp) {
+            uint8_t *box = tma_box + ((warp - 2) * 2 + (nbox & 1)) * 4096;
+            if (lane == 0) bulk_wait_read<1>();  // this box's store of two passes ago has read it
+            __syncwarp();
+            // row `lane` of the box: 16-byte chunk c at (c ^ (lane & 7)), the 128-byte swizzle
+#pragma unroll
+            for (int c = 0; c < 8; c++) {
+              uint4 pk;
+              __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&pk);
+#pragma unroll
+              for (int j = 0; j < 4; j++) p2[j] = __floats2bfloat162_rn(v[8 * c + 2 * j], v[8 * c + 2 * j + 1]);
+              *reinterpret_cast<uint4 *>(box + lane * 128 + ((c ^ (lane & 7)) << 4)) = pk;
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmC, smem_u32(box), n0 + sg * 64, m0 + q * 32);
+              bulk_commit();
+            }
+            nbox++;
+          } else if (valid) {
+            epi.template operator()<64>(r, token, g, n0 + sg * 64, v);
+          }
+        }
       } else {
         if (!mbar_wait(smem_u32(&tfull[acc]), aph, abort_flag, a.err)) break;
         tc_fence_after();
@@ -345,6 +395,9 @@ __global__ void __launch_bounds__(
           }
         }
       }
+    }
+    if constexpr (TMAST) {
+      if (lane == 0) bulk_wait_all();  // every tile store of this warp has landed
     }
   } else if (GATHER) {
     // ------------------------------------------------------------- gathered A producers

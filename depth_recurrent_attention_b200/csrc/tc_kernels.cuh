@@ -290,9 +290,11 @@ static void tc_destroy(dreamer_handle *h) {}
 template <int BN, int BK, int ST, bool GATHER, int SEG, class Epi, bool ROWPASS = false,
           int EW = 4>
 static void tc_launch(dreamer_handle *h, const dreamer::tc::TcGemmArgs &a, const CUtensorMap &ta,
-                      const CUtensorMap &tb, long max_tiles, const Epi &epi, cudaStream_t s) {
-  using Cfg = dreamer::tc::TcGemmCfg<BN, BK, ST, GATHER,
-                                     dreamer::tc::EpiStaged<Epi>::value && !ROWPASS, EW, ROWPASS>;
+                      const CUtensorMap &tb, long max_tiles, const Epi &epi, cudaStream_t s,
+                      const CUtensorMap *tc = nullptr) {
+  constexpr bool STG = dreamer::tc::EpiStaged<Epi>::value && !ROWPASS;
+  using Cfg = dreamer::tc::TcGemmCfg<BN, BK, ST, GATHER, STG, EW, ROWPASS,
+                                     dreamer::tc::EpiTma<Epi>::value && !STG && !ROWPASS>;
   auto kern = dreamer::tc::tc_gemm_kernel<BN, BK, ST, GATHER, SEG, Epi, ROWPASS, EW>;
   if (ROWPASS) max_tiles /= (a.N / BN);  // one unit of work per row tile
   static bool attr_set = false;
@@ -303,7 +305,8 @@ static void tc_launch(dreamer_handle *h, const dreamer::tc::TcGemmArgs &a, const
   long grid = max_tiles < h->num_sms ? max_tiles : h->num_sms;
   if (grid < 1) grid = 1;
   ++g_launches_tc;
-  launch_k(h, kern, dim3((unsigned)grid), dim3(Cfg::THREADS), Cfg::SMEM, s, ta, tb, a, epi);
+  launch_k(h, kern, dim3((unsigned)grid), dim3(Cfg::THREADS), Cfg::SMEM, s, ta, tb,
+           tc ? *tc : tb, a, epi);
 }
 
 // Build engine arguments and tensor maps from the generic GEMM description.  B rows of group
@@ -543,7 +546,8 @@ static bool tc_expert_ok(dreamer_handle *h) {
 
 template <int M, int ST>
 static void tc_ffn_launch(dreamer_handle *h, const CUtensorMap &t1, const CUtensorMap &t2,
-                          const dreamer::tc::TcFfnArgs &a, long max_tiles, cudaStream_t s) {
+                          const CUtensorMap &ty, const dreamer::tc::TcFfnArgs &a,
+                          long max_tiles, cudaStream_t s) {
   using Cfg = dreamer::tc::TcFfnCfg<M, ST>;
   auto kern = dreamer::tc::tc_ffn_kernel<M, ST>;
   static bool attr_set = false;
@@ -554,7 +558,7 @@ static void tc_ffn_launch(dreamer_handle *h, const CUtensorMap &t1, const CUtens
   long grid = max_tiles < h->num_sms ? max_tiles : h->num_sms;
   if (grid < 1) grid = 1;
   ++g_launches_tc;
-  launch_k(h, kern, dim3((unsigned)grid), dim3(Cfg::THREADS), Cfg::SMEM, s, t1, t2, a);
+  launch_k(h, kern, dim3((unsigned)grid), dim3(Cfg::THREADS), Cfg::SMEM, s, t1, t2, ty, a);
 }
 
 // Two grouped GEMMs: H = SiLU(X_gathered W1_e) stored in sorted order, then Y = H W2_e.
@@ -574,31 +578,33 @@ static bool tc_expert_two(dreamer_handle *h, const void *X, int n, cudaStream_t 
   dn.arow = nullptr; dn.arow_div = 1; dn.A = h->Hbuf; dn.lda = m; dn.B = h->w2_t; dn.ldb = m;
   dn.bgstride = (long)m * hd;
   tc::TcGemmArgs tu{}, td{};
-  CUtensorMap tau, tbu, tad, tbd;
+  CUtensorMap tau, tbu, tad, tbd, tyd;
   long mtu, mtd;
   EpiUp<bf16> eu{m, (bf16 *)h->Hbuf};
   EpiDownStore<bf16> ed{hd, (bf16 *)h->Ybuf};
+  // Y [T k + 128][h]: the down-projection's tile stores (32 rows x 64 columns a box)
+  if (!make_tmap(&tyd, h->Ybuf, hd, (uint64_t)rows + 128, (uint64_t)hd * 2, 64, 32)) return false;
   switch (m) {
     case 16:
       if (!tc_prepare<16, 64>(h, up, h->etiles_b, rows, tu, tau, tbu, mtu) ||
           !tc_prepare<256, 16>(h, dn, h->etiles_b, rows + 128, td, tad, tbd, mtd))
         return false;
       tc_launch<16, 64, 8, true, 16>(h, tu, tau, tbu, mtu, eu, s);
-      tc_launch<256, 16, 8, false, 64>(h, td, tad, tbd, mtd, ed, s);
+      tc_launch<256, 16, 8, false, 64>(h, td, tad, tbd, mtd, ed, s, &tyd);
       return true;
     case 32:
       if (!tc_prepare<32, 64>(h, up, h->etiles_b, rows, tu, tau, tbu, mtu) ||
           !tc_prepare<256, 32>(h, dn, h->etiles_b, rows + 128, td, tad, tbd, mtd))
         return false;
       tc_launch<32, 64, 8, true, 32>(h, tu, tau, tbu, mtu, eu, s);
-      tc_launch<256, 32, 6, false, 64>(h, td, tad, tbd, mtd, ed, s);
+      tc_launch<256, 32, 6, false, 64>(h, td, tad, tbd, mtd, ed, s, &tyd);
       return true;
     default:
       if (!tc_prepare<64, 64>(h, up, h->etiles_b, rows, tu, tau, tbu, mtu) ||
           !tc_prepare<256, 64>(h, dn, h->etiles_b, rows + 128, td, tad, tbd, mtd))
         return false;
       tc_launch<64, 64, 8, true, 64>(h, tu, tau, tbu, mtu, eu, s);
-      tc_launch<256, 64, 4, false, 64>(h, td, tad, tbd, mtd, ed, s);
+      tc_launch<256, 64, 4, false, 64>(h, td, tad, tbd, mtd, ed, s, &tyd);
       return true;
   }
 }
@@ -614,9 +620,12 @@ static bool tc_expert(dreamer_handle *h, const void *X, int n, cudaStream_t s) {
   const long rows = (long)n * k;
   if (rows < 96L * E) return tc_expert_two(h, X, n, s);
   if (((uintptr_t)X & 15) || (hd * 2) % 16) return false;
-  CUtensorMap t1, t2;  // W1^T [E m][h] in blocks of m x 64; W2^T [E h][m] in chunks of 256 x m
+  // W1^T [E m][h] in blocks of m x 64; W2^T [E h][m] in chunks of 256 x m; Y [T k + 128][h]
+  // in 32 x 64 store boxes
+  CUtensorMap t1, t2, ty;
   if (!make_tmap(&t1, h->w1_t, hd, (uint64_t)E * m, (uint64_t)hd * 2, 64, m) ||
-      !make_tmap(&t2, h->w2_t, m, (uint64_t)E * hd, (uint64_t)m * 2, m, 256))
+      !make_tmap(&t2, h->w2_t, m, (uint64_t)E * hd, (uint64_t)m * 2, m, 256) ||
+      !make_tmap(&ty, h->Ybuf, hd, (uint64_t)rows + 128, (uint64_t)hd * 2, 64, 32))
     return false;
   tc::TcFfnArgs a{};
   a.H = hd; a.G = E; a.M = (int)rows; a.goffs = h->eoffs; a.tiles = h->etiles_b;
@@ -624,8 +633,8 @@ static bool tc_expert(dreamer_handle *h, const void *X, int n, cudaStream_t s) {
   a.Y = (bf16 *)h->Ybuf; a.err = h->err;
   const long max_tiles = (rows + 127) / 128 + E;
   switch (m) {
-    case 16: tc_ffn_launch<16, 6>(h, t1, t2, a, max_tiles, s); return true;
-    case 32: tc_ffn_launch<32, 6>(h, t1, t2, a, max_tiles, s); return true;
-    default: tc_ffn_launch<64, 5>(h, t1, t2, a, max_tiles, s); return true;
+    case 16: tc_ffn_launch<16, 6>(h, t1, t2, ty, a, max_tiles, s); return true;
+    case 32: tc_ffn_launch<32, 6>(h, t1, t2, ty, a, max_tiles, s); return true;
+    default: tc_ffn_launch<64, 4>(h, t1, t2, ty, a, max_tiles, s); return true;
   }
 }
