@@ -44,6 +44,8 @@ struct dreamer_handle {
   int *pidx = nullptr, *eidx = nullptr, *counts = nullptr, *ecnt = nullptr, *eoffs = nullptr;
   int *etiles_a = nullptr, *etiles_b = nullptr, *ecursor = nullptr, *erows = nullptr;
   int *einv = nullptr;           // [T k] sorted position of each routed slot
+  int2 *etab = nullptr;          // 128-row tiles of the expert groups (written by the sort)
+  int2 *ptab = nullptr;          // 128-row tiles of the projection groups
   void *Ybuf = nullptr;          // [T k + 128][h] expert outputs in sorted order
   int *pcnt = nullptr, *poffs = nullptr, *ptiles_a = nullptr, *ptiles_b = nullptr;
   int *pcursor = nullptr, *prows = nullptr, *pinv = nullptr;
@@ -256,6 +258,8 @@ static int validate(const dreamer_config *c) {
   if (c->expert_hidden % 16 || c->router_dim % 16 || c->router_dim > 256 || c->hidden % 64)
     return DREAMER_ERR_UNSUPPORTED;
   if (c->depth > 1024 || c->hidden > 4096) return DREAMER_ERR_UNSUPPORTED;
+  // routed rows (tokens x k) are indexed with 24 bits in the grouping tables
+  if ((long)c->batch * c->seq * c->top_k >= (1L << 24)) return DREAMER_ERR_UNSUPPORTED;
   if (c->dtype == 1) {
     // bf16 runs only on the tcgen05 kernels and the purpose-built streaming kernels: shapes
     // they do not take are refused here instead of being routed to CUDA-core fallbacks
@@ -461,6 +465,8 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     DALLOC(h->etiles_b, (E + 1) * sizeof(int));
     DALLOC(h->erows, Tk * sizeof(int));
     DALLOC(h->einv, Tk * sizeof(int));
+    DALLOC(h->etab, (Tk / 128 + E + 2) * sizeof(int2));
+    DALLOC(h->ptab, (T / 128 + G + 2) * sizeof(int2));
     DALLOC(h->Ybuf, (size_t)(Tk + 128) * hd * es);
     DALLOC(h->pcnt, 2 * (G + 1) * sizeof(int));  // counts | rank counters
     h->pcursor = h->pcnt + G + 1;
@@ -603,9 +609,9 @@ static void launch_da_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStre
   if (own && smem < 116 * 1024) smem = 116 * 1024;
   const int threads = 32 * r.H;
   auto go = [&](void (*kern)(DaBulkArgs)) {
-    // set for the kernel launched (the head sizes share one pointer type)
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // the largest dynamic shared memory any launch of the kernel asks for: a call captured
+    // into a graph holds launches of several depths, each with its own size
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
     long grid;
     if (own) {
       grid = sms;
@@ -862,7 +868,8 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
       if (E <= 8192) {
         launch_k(h, permute_kernel, dim3(cdiv((long)n * k, 1024)), dim3(1024),
                  (size_t)(E + 1) * sizeof(int), st, (const int *)h->ecnt, E, (const int *)h->eidx,
-                 n * k, h->eoffs, h->etiles_a, 64, h->etiles_b, 128, h->ecursor, h->erows, h->einv);
+                 n * k, h->eoffs, h->etiles_a, 64, h->etiles_b, 128, h->ecursor, h->erows, h->einv,
+                 h->etab);
       } else {
         launch_k(h, scan_kernel, dim3(1), dim3(1024), 0, st, (const int *)h->ecnt, E, h->eoffs,
                  h->etiles_a, 64, h->etiles_b, 128, h->ecursor);
@@ -916,7 +923,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
       h->path_err = 1;
     launch_k(h, permute_kernel, dim3(cdiv(n, 1024)), dim3(1024), (size_t)(G + 1) * sizeof(int), s,
              (const int *)h->pcnt, G, (const int *)h->pidx, n, h->poffs, h->ptiles_a, 64,
-             h->ptiles_b, 128, h->pcursor, h->prows, h->pinv);
+             h->ptiles_b, 128, h->pcursor, h->prows, h->pinv, h->ptab);
     prow = h->prows;
     psig = h->psig;
   }
@@ -1060,13 +1067,15 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   trace_depth(h, io.tr, l, n, io.mode == 0, s);
   // 8. x_{l+1} = y + sum_s w_s Y_s, then the next depth's RMSNorm (or the call's output)
   mark(h, s, DREAMER_STAGE_FINISH);
-  const int cb = cdiv(n, 8);
-  auto combine = hd <= 2048 ? combine_norm_kernel<T, 64> : combine_norm_kernel<T, 128>;
-  launch_k(h, combine, dim3(cb), dim3(256), 0, s, h->acc, (const T *)h->Ybuf,
-           by_rows ? (const int *)nullptr : (const int *)h->einv, (const float *)h->ew, k,
-           (const T *)h->g, (T *)h->xh,
-           h->inv_rms, last ? (T *)io.x_out : (T *)nullptr, n, hd, c.rms_eps, h->ecnt, 2 * E,
-           h->pcnt, P > 0 ? 2 * (G + 1) : 0);
+  {
+    const int cb = cdiv(n, 8);
+    auto combine = hd <= 2048 ? combine_norm_kernel<T, 64> : combine_norm_kernel<T, 128>;
+    launch_k(h, combine, dim3(cb), dim3(256), 0, s, h->acc, (const T *)h->Ybuf,
+             by_rows ? (const int *)nullptr : (const int *)h->einv, (const float *)h->ew, k,
+             (const T *)h->g, (T *)h->xh,
+             h->inv_rms, last ? (T *)io.x_out : (T *)nullptr, n, hd, c.rms_eps, h->ecnt, 2 * E,
+             h->pcnt, P > 0 ? 2 * (G + 1) : 0);
+  }
   trace_next(h, io.tr, l, n, s);
 }
 

@@ -626,7 +626,7 @@ __global__ void __launch_bounds__(256) expert_rows_kernel(const T *X, const int 
 // next depth's x^ = g x / rms(x) and 1/rms (RMSNorm on the residual stream, "Overall
 // framework"), or, after the last depth, the output x_L rounded to dtype.
 template <typename T, int MAXV>
-__global__ void __launch_bounds__(256) combine_norm_kernel(float *acc, const T *Y, const int *pos,
+__global__ void __launch_bounds__(256, 4) combine_norm_kernel(float *acc, const T *Y, const int *pos,
                                                           const float *wts, int k, const T *gain,
                                                           T *xh, float *inv_rms, T *x_out,
                                                           int n_tok, int h, float eps,
@@ -642,45 +642,63 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(float *acc, const T *
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= n_tok) return;
-  float xv[MAXV];  // this lane's 8-element chunks of the row, in fp32
-  float ss = 0.f;
+  // slot s's row in Y (its sorted position, or the slot itself when pos == null) and weight,
+  // held by lane s (k <= 16) and passed round by shuffles
   const long slot0 = (long)warp * k;
-#pragma unroll
+  long my_row = 0;
+  float my_w = 0.f;
+  if (lane < k) {
+    my_row = (pos ? (long)pos[slot0 + lane] : slot0 + lane) * h;
+    my_w = wts[slot0 + lane];
+  }
+  float ss = 0.f;
+#pragma unroll 1
   for (int ci = 0; ci < MAXV / 8; ci++) {
+    if (ci * 256 >= h) break;  // uniform across the warp
     const int c = ci * 256 + lane * 8;
-    if (c >= h) break;
+    const bool on = c < h;
     float x[8];
-    load8(acc + (long)warp * h + c, x);
-    for (int s = 0; s < k; s++) {
-      // row of slot s in Y: its sorted position, or the slot itself (pos == null)
-      const long pr = (pos ? (long)pos[slot0 + s] : slot0 + s) * h;
-      const float pw = wts[slot0 + s];
-      float yv[8];
-      load8(Y + pr + c, yv);
+    if (on) load8(acc + (long)warp * h + c, x);
+    // four slot rows requested before any is used; the sum runs over s = 0..k-1 in order
+    for (int s0 = 0; s0 < k; s0 += 4) {
+      float yv[4][8];
 #pragma unroll
-      for (int j = 0; j < 8; j++) x[j] = fmaf(pw, yv[j], x[j]);
-    }
+      for (int u = 0; u < 4; u++) {
+        const long pr = __shfl_sync(0xffffffffu, my_row, (s0 + u) & 31);
+        if (on && s0 + u < k) load8(Y + pr + c, yv[u]);
+      }
 #pragma unroll
-    for (int j = 0; j < 8; j++) {
-      xv[ci * 8 + j] = x[j];
-      ss += x[j] * x[j];
+      for (int u = 0; u < 4; u++) {
+        const float pw = __shfl_sync(0xffffffffu, my_w, (s0 + u) & 31);
+        if (on && s0 + u < k) {
+#pragma unroll
+          for (int j = 0; j < 8; j++) x[j] = fmaf(pw, yv[u][j], x[j]);
+        }
+      }
     }
-    // the accumulator always keeps x_{l+1} in fp32 (the last depth also stores it rounded)
-    if (x_out) store8(x_out + (long)warp * h + c, x);
-    store8(acc + (long)warp * h + c, x);
+    if (on) {
+#pragma unroll
+      for (int j = 0; j < 8; j++) ss += x[j] * x[j];
+      // the accumulator always keeps x_{l+1} in fp32 (the last depth also stores it rounded)
+      if (x_out) store8(x_out + (long)warp * h + c, x);
+      store8(acc + (long)warp * h + c, x);
+    }
   }
   if (x_out) return;
   ss = warp_sum(ss);
   const float r = rsqrtf(ss / (float)h + eps);
   if (lane == 0) inv_rms[warp] = r;
-#pragma unroll
+  // the next depth's x^ from the row just stored (this thread's own writes, still in L1/L2):
+  // the row is not kept in registers, so more warps fit on an SM to hide the slot loads
+#pragma unroll 1
   for (int ci = 0; ci < MAXV / 8; ci++) {
     const int c = ci * 256 + lane * 8;
     if (c >= h) break;
-    float gv[8], o[8];
+    float gv[8], xr[8], o[8];
     load8(gain + c, gv);
+    load8(acc + (long)warp * h + c, xr);
 #pragma unroll
-    for (int j = 0; j < 8; j++) o[j] = gv[j] * xv[ci * 8 + j] * r;
+    for (int j = 0; j < 8; j++) o[j] = gv[j] * xr[j] * r;
     store8(xh + (long)warp * h + c, o);
   }
 }
@@ -1233,7 +1251,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *cnt, int G, int *
 __global__ void __launch_bounds__(1024) permute_kernel(const int *cnt, int G, const int *idx,
                                                        int n, int *offs, int *tiles_a, int bm_a,
                                                        int *tiles_b, int bm_b, int *ctr, int *rows,
-                                                       int *inv) {
+                                                       int *inv, int2 *ttab_b) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ int so[];  // [G + 1]
@@ -1298,6 +1316,13 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int *cnt, int G, co
         offs[g] = b0;
         tiles_a[g] = b1;
         if (tiles_b) tiles_b[g] = b2;
+        // the group's bm_b-row tiles: (group, first row | rows << 24), so a GEMM finds a tile's
+        // rows with one load instead of a search over the tile offsets
+        if (ttab_b)
+          for (int t = 0; t * bm_b < c; t++) {
+            const int r0 = b0 + t * bm_b, nr = min(bm_b, c - t * bm_b);
+            ttab_b[b2 + t] = make_int2(g, (int)((unsigned)r0 | ((unsigned)nr << 24)));
+          }
       }
       b0 += c;
       b1 += (c + bm_a - 1) / bm_a;

@@ -36,6 +36,7 @@ struct TcFfnArgs {
   long ldx;
   bf16 *Y;             // [rows][H], expert-sorted order
   int *err;
+  const int2 *ttab;    // [tiles] (expert, first row | rows << 24) of each tile, or null
 };
 
 template <int M, int STAGES>
@@ -58,6 +59,13 @@ struct TcFfnCfg {
 
 __device__ __forceinline__ void ffn_tile_rows(const TcFfnArgs &a, int mt, int &g, int &m0,
                                               int &m1) {
+  if (a.ttab) {
+    const int2 e = a.ttab[mt];
+    g = e.x;
+    m0 = e.y & 0xffffff;
+    m1 = m0 + ((unsigned)e.y >> 24);
+    return;
+  }
   int lo = 0, hi = a.G - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;

@@ -33,6 +33,7 @@ struct TcGemmArgs {
   int b_group_rows, b_row0;
   int *err;
   int skip_loads;     // test-hook build only: the TMA producer issues no loads (0 otherwise)
+  const int2 *ttab;   // [tiles] (group, first row | rows << 24) of each 128-row tile, or null
 };
 
 // per-row epilogue state: Epi::State for row-pass epilogues, nothing otherwise
@@ -40,8 +41,16 @@ struct NoEpiState {};
 template <class Epi, bool ROWPASS> struct EpiState { using type = NoEpiState; };
 template <class Epi> struct EpiState<Epi, true> { using type = typename Epi::State; };
 
+// group and rows of a tile from its table entry
+__device__ __forceinline__ bool tc_tile_unpack(int2 e, int &g, int &m0, int &m1) {
+  g = e.x;
+  m0 = e.y & 0xffffff;
+  m1 = m0 + ((unsigned)e.y >> 24);
+  return m0 < m1;
+}
 __device__ __forceinline__ bool tc_tile_rows(const TcGemmArgs &a, int mt, int &g, int &m0,
                                              int &m1) {
+  if (a.goffs && a.ttab) return tc_tile_unpack(a.ttab[mt], g, m0, m1);
   if (!a.goffs) {
     g = 0;
     m0 = mt * 128;
@@ -191,10 +200,22 @@ __global__ void __launch_bounds__(
       // the timeout test: no operand ever arrives, so the MMA issuer's bounded wait expires
       if (a.skip_loads) ok = false;
 #endif
+      // grouped rows: each tile's table entry requested two tiles ahead, so a tile of a single
+      // K block does not wait a memory round trip before its loads are issued
+      const bool tab = a.goffs && a.ttab;
+      auto entry = [&](int i) -> int2 {
+        int m_, n_;
+        return (tab && tile_at(i, m_, n_)) ? a.ttab[m_] : make_int2(0, 0);
+      };
+      int2 e1 = entry(0), e2 = entry(1);
       for (int i = 0; ok && tile_at(i, mt, nt); i++) {
         int g, m0, m1;
         const int n0 = nt * BN;
-        tc_tile_rows(a, mt, g, m0, m1);
+        const int2 e0 = e1;
+        e1 = e2;
+        e2 = entry(i + 2);
+        if (tab) tc_tile_unpack(e0, g, m0, m1);
+        else tc_tile_rows(a, mt, g, m0, m1);
         const int brow = g * a.b_group_rows + a.b_row0 + n0;
         for (int kb = 0; kb < KB; kb++) {
           if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag, a.err)) { ok = false; break; }

@@ -331,6 +331,11 @@ static bool tc_prepare(dreamer_handle *h, const dreamer::GemmArgs &a, const int 
   t.A = (const dreamer::bf16 *)a.A; t.lda = a.lda;
   t.b_group_rows = (int)bgr; t.b_row0 = 0;
   t.err = h->err;
+  // 128-row tile table of the grouping (written by the counting sort; the expert one only
+  // when the sort ran in one kernel)
+  t.ttab = nullptr;
+  if (a.goffs && tiles == h->etiles_b && h->cfg.n_experts <= 8192) t.ttab = h->etab;
+  if (a.goffs && tiles == h->ptiles_b) t.ttab = h->ptab;
   max_tiles = ((a.M + 127) / 128 + (a.goffs ? a.G : 0)) * (long)(a.N / BN);
   return true;
 }
@@ -631,6 +636,7 @@ static bool tc_expert(dreamer_handle *h, const void *X, int n, cudaStream_t s) {
   a.H = hd; a.G = E; a.M = (int)rows; a.goffs = h->eoffs; a.tiles = h->etiles_b;
   a.arow = h->erows; a.arow_div = k; a.X = (const bf16 *)X; a.ldx = hd;
   a.Y = (bf16 *)h->Ybuf; a.err = h->err;
+  a.ttab = E <= 8192 ? h->etab : nullptr;
   const long max_tiles = (rows + 127) / 128 + E;
   switch (m) {
     case 16: tc_ffn_launch<16, 6>(h, t1, t2, ty, a, max_tiles, s); return true;
