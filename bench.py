@@ -374,7 +374,7 @@ def run_ours(args, cfg, rank, world, torch, dist):
 STAGE_KERNELS = {
     "qkv": "tc_gemm_kernel<EpiQKV>", "o_proj": "tc_gemm_kernel<EpiO>",
     "sa": "tc_sa_kernel (prefill) / dec_bulk_kernel + attn_merge_kernel (decode)",
-    "da": "da_bulk_kernel", "proj_route": "tc_gemm_kernel<EpiProjRoute> + permute_kernel",
+    "da": "da_fast_kernel", "proj_route": "tc_gemm_kernel<EpiProjRoute> + permute_kernel",
     "ea_route": "tc_gemm_kernel<EpiRouterQ> + tc_gemm_kernel<EpiTopK> or route_q_topk_kernel "
                 "(decode: route_cluster_kernel)",
     "permute": "permute_kernel",

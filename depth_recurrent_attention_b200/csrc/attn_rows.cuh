@@ -42,6 +42,7 @@ struct RowsArgs {
   long ldo;
   int col0;
   float *part;         // mode 2: [n_q][H][nsplit][D + 2] partial (o, m, l)
+  const int *out_rows; // mode 0: output row of token t (grouped projections), or null: t
 };
 
 template <typename T, int D, int U>
@@ -213,6 +214,7 @@ struct DaBulkArgs {
   long ldo;
   int col0;
   int *err;
+  const int *out_rows;           // output row of token t (grouped projections), or null: t
 };
 
 // NB chunk buffers: 2 (two CTAs share an SM) or 4 (a CTA owns its SM: the launch beside SA
@@ -363,7 +365,8 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
           const float inv = 1.0f / lsum;
 #pragma unroll
           for (int i = 0; i < VEC; i++) of[i] *= inv;
-          st16(reinterpret_cast<T *>(a.out) + (long)tok * a.ldo + a.col0 + head * D + cc * VEC, of);
+          const long orow = a.out_rows ? a.out_rows[tok] : tok;
+          st16(reinterpret_cast<T *>(a.out) + orow * a.ldo + a.col0 + head * D + cc * VEC, of);
         }
       }
     }
@@ -597,7 +600,8 @@ __global__ void __launch_bounds__(1024) da_fast_kernel(DaBulkArgs a) {
           const float inv = 1.0f / lsum;
 #pragma unroll
           for (int i = 0; i < 8; i++) of[i] *= inv;
-          store8(reinterpret_cast<bf16 *>(a.out) + (long)tok * a.ldo + a.col0 + head * D + cc * 8, of);
+          const long orow = a.out_rows ? a.out_rows[tok] : tok;
+          store8(reinterpret_cast<bf16 *>(a.out) + orow * a.ldo + a.col0 + head * D + cc * 8, of);
         }
       }
     }

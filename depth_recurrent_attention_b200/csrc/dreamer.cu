@@ -37,6 +37,7 @@ struct dreamer_handle {
   // workspace
   void *xh = nullptr, *qkv_sa = nullptr, *q_da = nullptr, *attn = nullptr, *y = nullptr;
   void *u = nullptr, *da_kv_int = nullptr, *Hbuf = nullptr, *qsplit = nullptr;
+  void *xh_sorted = nullptr;     // x^ in the projection experts' group order (P > 0)
   float *acc = nullptr, *zbuf = nullptr, *qbuf = nullptr, *psig = nullptr, *ew = nullptr;
   float *inv_rms = nullptr;      // [T] 1/rms of the current depth's residual
   float *part = nullptr;         // decode attention split partials [B][H][nsplit][d + 2]
@@ -442,6 +443,7 @@ extern "C" int dreamer_init(const dreamer_config *cfg, const dreamer_weights *w,
     const long Tk = T * c.top_k;
     DALLOC(h->xh, T * hd * es);
     DALLOC(h->u, T * hd * es);
+    if (P > 0) DALLOC(h->xh_sorted, T * hd * es);
     DALLOC(h->qkv_sa, T * 3 * hd * es);
     DALLOC(h->q_da, T * hd * es);
     DALLOC(h->attn, T * 2 * hd * es);
@@ -603,6 +605,7 @@ static void launch_da_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStre
   if (chunk > r.l + 1 - r.r0) chunk = r.l + 1 - r.r0;
   a.chunk = chunk;
   a.q = r.q; a.kv = r.kv; a.out = r.out; a.ldo = r.ldo; a.col0 = r.col0; a.err = r.err;
+  a.out_rows = r.out_rows;
   const bool own = sms > 0;
   const int nb = own ? 4 : 2;
   int smem = (int)(nb * (chunk * row_bytes + r.h * (long)sizeof(T)));
@@ -911,9 +914,13 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     run_ea(h->side2);
     cudaEventRecord(h->ev_join2, h->side2);
   }
-  // 2. projection router and token grouping (linear-MoE QKV/O)
+  // 2. projection router and token grouping (linear-MoE QKV/O).  In bf16 prefill (not the
+  // serial layout) the grouped projections read their A rows in group order with TMA: x^ is
+  // gathered into that order once, and SA and DA write their outputs at the tokens' sorted
+  // rows, so that the O projection reads them in order too.
   const int *prow = nullptr;
   const float *psig = nullptr;
+  const bool sorted = P > 0 && tc && io.mode == 0 && c.variant != 1;
   if (P > 0) {
     mark(h, s, DREAMER_STAGE_PROJ_ROUTE);
     // pcnt / pcursor are zero here: cleared at init and by every depth's combine kernel
@@ -926,6 +933,13 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
              h->ptiles_b, 128, h->pcursor, h->prows, h->pinv, h->ptab);
     prow = h->prows;
     psig = h->psig;
+    if (sorted) {
+      const long chunks = (long)n * (hd / 8);
+      launch_k(h, gather_rows_kernel, dim3((unsigned)cdiv(chunks, 256) < 4u * h->num_sms
+                                               ? (unsigned)cdiv(chunks, 256) : 4u * h->num_sms),
+               dim3(256), 0, s, (const bf16 *)h->xh, (const int *)h->prows, (bf16 *)h->xh_sorted,
+               n, hd);
+    }
   }
   auto grouped = [&](int N, int K, const void *A, long lda, const void *B, long bgs) {
     GemmArgs a{};
@@ -933,6 +947,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     a.goffs = P > 0 ? h->poffs : nullptr;
     a.tile_offs = P > 0 ? h->ptiles_a : nullptr;
     a.arow = prow; a.arow_div = 1; a.A = A; a.lda = lda; a.B = B; a.ldb = K; a.bgstride = bgs;
+    a.a_sorted = sorted ? 1 : 0;
     return a;
   };
   const int ptiles = cdiv(n, 64) + (P > 0 ? G : 0);
@@ -950,6 +965,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   da.r0 = (c.da_window > 0 && l + 1 > c.da_window) ? l + 1 - c.da_window : 0;
   da.q = h->q_da; da.ldq = hd; da.kv = io.da_kv;
   da.out = h->attn; da.ldo = 2 * hd; da.col0 = hd; da.err = h->err;
+  da.out_rows = sorted ? h->pinv : nullptr;
   RowsArgs sd{};  // decode: attention over the per-depth SA cache, split over key ranges
   sd.mode = 2; sd.n_q = n; sd.H = c.n_heads; sd.h = hd; sd.L = L; sd.l = l;
   sd.q = h->qkv_sa; sd.ldq = 3 * hd; sd.kv = io.k_cache; sd.vc = io.v_cache;
@@ -971,7 +987,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     }
     if (!tc)
       launch_attn<T>(sa, d, st);
-    else if (!(tc_sa_ok(h) && tc_sa(h, st)))
+    else if (!(tc_sa_ok(h) && tc_sa(h, st, sorted ? h->pinv : nullptr)))
       h->path_err = 1;
   };
   auto qkv_gemm = [&](const void *A, int col0, int ncols) {
@@ -1012,7 +1028,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   if (c.variant == 3) {
     // without depth attention (the DR-without-DA arm): the SA columns of the projection
     // only, y = x^ + SA W_O[SA rows]
-    qkv_gemm(h->xh, 0, 3 * hd);
+    qkv_gemm(sorted ? h->xh_sorted : h->xh, 0, 3 * hd);
     mark(h, s, DREAMER_STAGE_SA);
     run_sa(s);
     o_gemm(h->attn, 0, hd, res_xhat, h->y);
@@ -1028,7 +1044,7 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     o_gemm(h->attn, 0, hd, 2, h->y);                            // y = u + SA part
   } else {
     // 3. fused QKV projection with RoPE / depth RoPE epilogue, DA KV write
-    qkv_gemm(h->xh, 0, 6 * hd);
+    qkv_gemm(sorted ? h->xh_sorted : h->xh, 0, 6 * hd);
     // 4. DA || SA (papernotes "Key design 1": run in parallel for throughput).  DA runs
     // on the side stream beside SA (two branches of the captured graph), on SMs of its own
     // where that pays; with stage profiling on they run one after the other (same launch
@@ -1067,7 +1083,15 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
   trace_depth(h, io.tr, l, n, io.mode == 0, s);
   // 8. x_{l+1} = y + sum_s w_s Y_s, then the next depth's RMSNorm (or the call's output)
   mark(h, s, DREAMER_STAGE_FINISH);
-  {
+  if (c.dtype == 1) {  // bf16: a CTA of h / 8 threads per token (h <= 4096, k <= 16)
+    auto kern = k <= 4 ? combine_norm_row_kernel<4>
+                       : (k <= 8 ? combine_norm_row_kernel<8> : combine_norm_row_kernel<16>);
+    launch_k(h, kern, dim3(n), dim3(hd / 8), 0, s, h->acc,
+             (const bf16 *)h->Ybuf, by_rows ? (const int *)nullptr : (const int *)h->einv,
+             (const float *)h->ew, k, (const bf16 *)h->g, (bf16 *)h->xh, h->inv_rms,
+             last ? (bf16 *)io.x_out : (bf16 *)nullptr, n, hd, c.rms_eps, h->ecnt, 2 * E,
+             h->pcnt, P > 0 ? 2 * (G + 1) : 0);
+  } else {
     const int cb = cdiv(n, 8);
     auto combine = hd <= 2048 ? combine_norm_kernel<T, 64> : combine_norm_kernel<T, 128>;
     launch_k(h, combine, dim3(cb), dim3(256), 0, s, h->acc, (const T *)h->Ybuf,

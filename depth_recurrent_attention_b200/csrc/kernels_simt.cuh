@@ -429,6 +429,8 @@ struct GemmArgs {
   const int *tile_offs;   // [G+1] cumulative row tiles (of this engine's BM) or null
   const int *arow;        // sorted row -> source id, or null (identity)
   int arow_div;           // A row = arow[r] / arow_div
+  int a_sorted;           // tcgen05 engine: A is already in sorted-row order (TMA tiles);
+                          // arow then only maps rows to tokens for the epilogue
   const void *A;
   long lda;
   const void *B;
@@ -701,6 +703,74 @@ __global__ void __launch_bounds__(256, 4) combine_norm_kernel(float *acc, const 
     for (int j = 0; j < 8; j++) o[j] = gv[j] * xr[j] * r;
     store8(xh + (long)warp * h + c, o);
   }
+}
+
+// The same combine for bf16 with one CTA per token and h / 8 threads (8 elements each): every
+// thread requests its acc chunk and all k <= KMAX slot chunks (16-byte loads, kept packed)
+// before the first use, so a token costs one memory round trip; the sum over the slots runs in the same
+// fixed order s = 0..k-1, and the row's squares are reduced over the CTA for the next norm.
+template <int KMAX>
+__global__ void __launch_bounds__(512) combine_norm_row_kernel(
+    float *acc, const bf16 *Y, const int *pos, const float *wts, int k, const bf16 *gain,
+    bf16 *xh, float *inv_rms, bf16 *x_out, int n_tok, int h, float eps, int *zero_a, int na,
+    int *zero_b, int nb) {
+  pdl_wait();
+  pdl_trigger();
+  {  // the depth's grouping counters, cleared for the next depth (nothing reads them now)
+    const int t = blockIdx.x * blockDim.x + threadIdx.x, nt = gridDim.x * blockDim.x;
+    for (int i = t; i < na; i += nt) zero_a[i] = 0;
+    for (int i = t; i < nb; i += nt) zero_b[i] = 0;
+  }
+  __shared__ long srow[16];
+  __shared__ float sw[16];
+  __shared__ float red[32];
+  const int tok = blockIdx.x;
+  const long slot0 = (long)tok * k;
+  if (threadIdx.x < k) {
+    srow[threadIdx.x] = (pos ? (long)pos[slot0 + threadIdx.x] : slot0 + threadIdx.x) * h;
+    sw[threadIdx.x] = wts[slot0 + threadIdx.x];
+  }
+  __syncthreads();
+  const int c = threadIdx.x * 8;
+  float x[8];
+  load8(acc + (long)tok * h + c, x);
+  uint4 yv[KMAX];
+#pragma unroll
+  for (int s = 0; s < KMAX; s++)
+    if (s < k) yv[s] = *reinterpret_cast<const uint4 *>(Y + srow[s] + c);
+#pragma unroll
+  for (int s = 0; s < KMAX; s++) {
+    if (s < k) {
+      const float pw = sw[s];
+      const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&yv[s]);
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const float2 f = __bfloat1622float2(h2[i]);
+        x[2 * i] = fmaf(pw, f.x, x[2 * i]);
+        x[2 * i + 1] = fmaf(pw, f.y, x[2 * i + 1]);
+      }
+    }
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; j++) ss += x[j] * x[j];
+  // the accumulator always keeps x_{l+1} in fp32 (the last depth also stores it rounded)
+  if (x_out) store8(x_out + (long)tok * h + c, x);
+  store8(acc + (long)tok * h + c, x);
+  if (x_out) return;  // uniform over the CTA
+  ss = warp_sum(ss);
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  if (lane == 0) red[wid] = ss;
+  __syncthreads();
+  float tot = lane < nw ? red[lane] : 0.f;
+  tot = warp_sum(tot);
+  const float r = rsqrtf(tot / (float)h + eps);
+  if (threadIdx.x == 0) inv_rms[tok] = r;
+  float gv[8], o[8];
+  load8(gain + c, gv);
+#pragma unroll
+  for (int j = 0; j < 8; j++) o[j] = gv[j] * x[j] * r;
+  store8(xh + (long)tok * h + c, o);
 }
 
 // =======================================================================================
@@ -1341,6 +1411,23 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int *cnt, int G, co
     const int p = so[g] + atomicAdd(ctr + g, 1);
     rows[p] = i;
     if (inv) inv[i] = p;
+  }
+}
+
+// dst[r] = src[rows[r]] for r < n, rows of h bf16 (16-byte chunks, grid-stride): the
+// normalised states in the order of the projection experts' groups, so that the grouped QKV
+// projection loads its A tiles with TMA.
+__global__ void gather_rows_kernel(const bf16 *src, const int *rows, bf16 *dst, int n, int h) {
+  pdl_wait();
+  pdl_trigger();
+  const int cpr = h / 8;
+  const long total = (long)n * cpr;
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long)gridDim.x * blockDim.x) {
+    const long r = i / cpr;
+    const int c = (int)(i % cpr) * 8;
+    *reinterpret_cast<uint4 *>(dst + r * h + c) =
+        *reinterpret_cast<const uint4 *>(src + (long)rows[r] * h + c);
   }
 }
 

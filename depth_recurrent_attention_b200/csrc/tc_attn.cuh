@@ -64,6 +64,7 @@ struct SaArgs {
   long ldo;
   float scale_log2;       // log2(e) / sqrt(d)
   int *err;
+  const int *out_rows;    // output row of token t (grouped projections), or null: t
 };
 
 template <int D>
@@ -332,7 +333,8 @@ __global__ void __launch_bounds__(352, 1)
       if (ok && mbar_wait(smem_u32(&pv_done[t]), (nbt - 1) & 1, abort_flag, a.err)) {
         tc_fence_after();
         const float inv = 1.0f / l;
-        bf16 *dst = a.out + (long)(row0 + qi) * a.ldo + head * D;
+        const long orow = a.out_rows ? a.out_rows[row0 + qi] : row0 + qi;
+        bf16 *dst = a.out + orow * a.ldo + head * D;
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
           float ov[32];
@@ -371,7 +373,7 @@ static bool tc_sa_ok(dreamer_handle *h) {
 
 // SA of every (sequence, head, pair of query tiles): q/k/v from qkv_sa [T][3h], output into
 // the SA half of attn [T][2h].
-static bool tc_sa(dreamer_handle *h, cudaStream_t s) {
+static bool tc_sa(dreamer_handle *h, cudaStream_t s, const int *out_rows) {
   using namespace dreamer;
   const dreamer_config &c = h->cfg;
   const int hd = c.hidden, d = c.head_dim;
@@ -385,6 +387,7 @@ static bool tc_sa(dreamer_handle *h, cudaStream_t s) {
   a.out = (bf16 *)h->attn; a.ldo = 2 * hd;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
   a.err = h->err;
+  a.out_rows = out_rows;
   const int grid = a.bh * a.n_pairs;
   ++g_launches_tc;
   if (d == 64) {

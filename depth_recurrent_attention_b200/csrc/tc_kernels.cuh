@@ -316,7 +316,7 @@ static bool tc_prepare(dreamer_handle *h, const dreamer::GemmArgs &a, const int 
                        long a_rows, dreamer::tc::TcGemmArgs &t, CUtensorMap &ta, CUtensorMap &tb,
                        long &max_tiles) {
   if (a.N % BN || a.K % BK) return false;
-  const bool gather = a.arow != nullptr;
+  const bool gather = a.arow != nullptr && !a.a_sorted;
   const long bgr = a.G > 1 ? a.bgstride / a.ldb : 0;
   if (!make_tmap(&tb, a.B, a.K, (uint64_t)((a.G - 1) * bgr + a.N), a.ldb * 2, BK, BN)) return false;
   if (!gather) {
@@ -369,7 +369,7 @@ static bool tc_gemm_qkv(dreamer_handle *h, const dreamer::GemmArgs &a, const dre
     CUtensorMap ta, tb;
     long mt;
     const int *tiles = h->ptiles_b;
-    const bool gather = a.arow != nullptr;
+    const bool gather = a.arow != nullptr && !a.a_sorted;
     // 64-column segments: the staged epilogue rotates pairs 32 columns apart (head dim 64,
     // or 128 in perm order).  Short K leaves little MMA time per tile to hide the epilogue
     // behind: eight epilogue warps then, at one stage less of operand ring.
@@ -427,24 +427,24 @@ static bool tc_gemm_o(dreamer_handle *h, const dreamer::GemmArgs &a, const dream
     const int bn = tc_pick_bn(h, a);
     if (bn == 64) {
       if (!tc_prepare<64, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
-      if (a.arow) tc_launch<64, 64, 8, true, 64>(h, t, ta, tb, mt, e, s);
+      if (a.arow && !a.a_sorted) tc_launch<64, 64, 8, true, 64>(h, t, ta, tb, mt, e, s);
       else tc_launch<64, 64, 8, false, 64>(h, t, ta, tb, mt, e, s);
     } else if (bn == 256) {
       if (!tc_prepare<256, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
       if (ew8) {
-        if (a.arow) tc_launch<256, 64, 3, true, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        if (a.arow && !a.a_sorted) tc_launch<256, 64, 3, true, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
         else tc_launch<256, 64, 3, false, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
       } else {
-        if (a.arow) tc_launch<256, 64, 4, true, 64>(h, t, ta, tb, mt, e, s);
+        if (a.arow && !a.a_sorted) tc_launch<256, 64, 4, true, 64>(h, t, ta, tb, mt, e, s);
         else tc_launch<256, 64, 4, false, 64>(h, t, ta, tb, mt, e, s);
       }
     } else {
       if (!tc_prepare<128, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
       if (ew8) {
-        if (a.arow) tc_launch<128, 64, 5, true, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        if (a.arow && !a.a_sorted) tc_launch<128, 64, 5, true, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
         else tc_launch<128, 64, 5, false, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
       } else {
-        if (a.arow) tc_launch<128, 64, 6, true, 64>(h, t, ta, tb, mt, e, s);
+        if (a.arow && !a.a_sorted) tc_launch<128, 64, 6, true, 64>(h, t, ta, tb, mt, e, s);
         else tc_launch<128, 64, 6, false, 64>(h, t, ta, tb, mt, e, s);
       }
     }
