@@ -267,16 +267,17 @@ __global__ void __launch_bounds__(352, 1)
         for (int c = 0; c < 128; c += 32) tmem_ld_fence(sv + c);
         tc_fence_before();
         mbar_arrive(smem_u32(&s_free[t]));
-        // row max of the raw scores (the scale is positive: applied to the max)
-        float mraw = -INFINITY;
-        if (!diag) {
-#pragma unroll
-          for (int i = 0; i < 128; i++) mraw = fmaxf(mraw, sv[i]);
-        } else {
+        // the diagonal block: keys past the row's own position get -inf (weight 0 below)
+        if (diag) {
 #pragma unroll
           for (int i = 0; i < 128; i++)
-            if (i <= lim) mraw = fmaxf(mraw, sv[i]);
+            if (i > lim) sv[i] = -INFINITY;
         }
+        // row max of the raw scores (the scale is positive: applied to the max), three a step
+        float mraw = max3f(sv[0], sv[1], sv[2]);
+#pragma unroll
+        for (int i = 3; i < 127; i += 2) mraw = max3f(mraw, sv[i], sv[i + 1]);
+        mraw = fmaxf(mraw, sv[127]);
         const float mx = mraw * a.scale_log2;
         // lazy rescale: move the reference max only when the row max grows by more than 8
         float m_new = m_ref, alpha = 1.f;
@@ -292,28 +293,30 @@ __global__ void __launch_bounds__(352, 1)
           tc_fence_after();
         }
         // P = 2^(s * scale - m) as bf16, K-major SW128 (key chunk kc at kc * TILE, 16-byte unit
-        // u of the row at ((u ^ (row & 7)) << 4)), summed; one 32-key chunk in four on the FMA
-        // pipe (ex2_poly), the rest on the MUFU unit
-        const float nm = -m_new;
-        float rs = 0.f;
+        // u of the row at ((u ^ (row & 7)) << 4)), summed.  Scale, offset and sum on packed
+        // fp32 pairs; keys 32..63 of the block on the FMA pipe (ex2_poly) except on the
+        // diagonal (masked keys must give exactly 0), the rest on the MUFU unit.
+        const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), nm2 = f2_pack(-m_new, -m_new);
+        uint64_t rs2 = 0ull;
 #pragma unroll
         for (int u8 = 0; u8 < 16; u8++) {
           const int kc = u8 >> 3, u = u8 & 7;
-          float p[8];
+          uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 8; e++) {
-            const int i = u8 * 8 + e;
-            const float x = fmaf(sv[i], a.scale_log2, nm);
-            p[e] = (i >= 32 && i < 64) ? ex2_poly(x) : ex2(x);
-            if (diag && i > lim) p[e] = 0.f;
-            rs += p[e];
+          for (int e = 0; e < 4; e++) {
+            const int i = u8 * 8 + 2 * e;
+            const float2 x = f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), sc2, nm2));
+            const bool poly = i >= 32 && i < 64 && !diag;
+            const float p0 = poly ? ex2_poly(x.x) : ex2(x.x);
+            const float p1 = poly ? ex2_poly(x.y) : ex2(x.y);
+            rs2 = f2_add(rs2, f2_pack(p0, p1));
+            w[e] = bf2_pack_rn(p0, p1);
           }
-          uint4 pk;
-          __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&pk);
-#pragma unroll
-          for (int e = 0; e < 4; e++) p2[e] = __floats2bfloat162_rn(p[2 * e], p[2 * e + 1]);
-          *reinterpret_cast<uint4 *>(prow + kc * C::TILE + ((u ^ (row & 7)) << 4)) = pk;
+          *reinterpret_cast<uint4 *>(prow + kc * C::TILE + ((u ^ (row & 7)) << 4)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
+        const float2 rsf = f2_unpack(rs2);
+        const float rs = rsf.x + rsf.y;
         // O rescaled before P_t(j) V accumulates into it (issued after p_full below)
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
