@@ -302,8 +302,11 @@ def run_ours(args, cfg, rank, world, torch, dist):
                     frac=achieved / pk["hbm"])
     roof.update(kernel=dominant, kernels=STAGE_KERNELS.get(dominant, dominant),
                 launches_per_step=launches_per_fwd,
-                traffic=measured_traffic(cfg.name, dominant),
-                peak_source=pk["source"] + " (MEASURED_PEAKS.json burst figure)")
+                traffic=None if args.reduced else measured_traffic(cfg.name, dominant),
+                alg_bytes_per_launch=by / launches_per_fwd,
+                peak_source=("measured (MEASURED_PEAKS.json burst figure)" if pk["source"] == "measured"
+                             else "fallback (no MEASURED_PEAKS.json: 6650 GB/s copy, 1590 TFLOP/s "
+                                  "bf16 GEMM burst, an earlier B200 measurement)"))
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -490,8 +493,15 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="large", choices=sorted(configs.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    for k in ("depth", "batch", "seq"):
+        ap.add_argument(f"--{k}", type=int, default=0,
+                        help=f"run the workload with this {k} instead of its own (reduced cases "
+                             "for ncu captures of single kernels); the line's config names it")
     args = ap.parse_args()
     cfg = configs.CONFIGS[args.config]
+    args.reduced = {k: getattr(args, k) for k in ("depth", "batch", "seq") if getattr(args, k)}
+    if args.reduced:
+        cfg = cfg.with_(**args.reduced)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
 

@@ -14,8 +14,9 @@
 //               warps in all so that a thread may hold a row of 128 scores in registers:
 //               the row's 128 scores come out of TMEM in one batch of loads (S is released to
 //               the next QK^T right away), then the row max, and P = exp2(s - m_ref) written
-//               as bf16 into the swizzled K-major operand in shared memory and summed (a
-//               quarter of the exponentials on the FMA pipe, the rest on MUFU).  O lives in
+//               as bf16 into the swizzled K-major operand in shared memory and summed (every
+//               exponential on MUFU: the softmax warps are issue-bound, and a polynomial on
+//               the FMA pipe costs more issue slots than it saves).  O lives in
 //               TMEM and is only rescaled when the running max grows by more than 2^8 (P stays
 //               <= 256), so most blocks need no O traffic at all; the last step divides O by
 //               the sum.
@@ -274,10 +275,15 @@ __global__ void __launch_bounds__(352, 1)
             if (i > lim) sv[i] = -INFINITY;
         }
         // row max of the raw scores (the scale is positive: applied to the max), three a step
-        float mraw = max3f(sv[0], sv[1], sv[2]);
+        // on four independent chains
+        float mc[4] = {sv[0], sv[1], sv[2], sv[3]};
 #pragma unroll
-        for (int i = 3; i < 127; i += 2) mraw = max3f(mraw, sv[i], sv[i + 1]);
-        mraw = fmaxf(mraw, sv[127]);
+        for (int i = 4; i < 124; i += 8)
+#pragma unroll
+          for (int k = 0; k < 4; k++) mc[k] = max3f(mc[k], sv[i + 2 * k], sv[i + 2 * k + 1]);
+        mc[0] = max3f(mc[0], sv[124], sv[125]);
+        mc[1] = max3f(mc[1], sv[126], sv[127]);
+        const float mraw = max3f(mc[0], mc[1], fmaxf(mc[2], mc[3]));
         const float mx = mraw * a.scale_log2;
         // lazy rescale: move the reference max only when the row max grows by more than 8
         float m_new = m_ref, alpha = 1.f;
@@ -294,10 +300,9 @@ __global__ void __launch_bounds__(352, 1)
         }
         // P = 2^(s * scale - m) as bf16, K-major SW128 (key chunk kc at kc * TILE, 16-byte unit
         // u of the row at ((u ^ (row & 7)) << 4)), summed.  Scale, offset and sum on packed
-        // fp32 pairs; keys 32..63 of the block on the FMA pipe (ex2_poly) except on the
-        // diagonal (masked keys must give exactly 0), the rest on the MUFU unit.
+        // fp32 pairs (masked keys: 2^-inf = 0 exactly).
         const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), nm2 = f2_pack(-m_new, -m_new);
-        uint64_t rs2 = 0ull;
+        uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};  // four independent sums of pairs
 #pragma unroll
         for (int u8 = 0; u8 < 16; u8++) {
           const int kc = u8 >> 3, u = u8 & 7;
@@ -306,16 +311,14 @@ __global__ void __launch_bounds__(352, 1)
           for (int e = 0; e < 4; e++) {
             const int i = u8 * 8 + 2 * e;
             const float2 x = f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), sc2, nm2));
-            const bool poly = i >= 32 && i < 64 && !diag;
-            const float p0 = poly ? ex2_poly(x.x) : ex2(x.x);
-            const float p1 = poly ? ex2_poly(x.y) : ex2(x.y);
-            rs2 = f2_add(rs2, f2_pack(p0, p1));
+            const float p0 = ex2(x.x), p1 = ex2(x.y);
+            rs2[e] = f2_add(rs2[e], f2_pack(p0, p1));
             w[e] = bf2_pack_rn(p0, p1);
           }
           *reinterpret_cast<uint4 *>(prow + kc * C::TILE + ((u ^ (row & 7)) << 4)) =
               make_uint4(w[0], w[1], w[2], w[3]);
         }
-        const float2 rsf = f2_unpack(rs2);
+        const float2 rsf = f2_unpack(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])));
         const float rs = rsf.x + rsf.y;
         // O rescaled before P_t(j) V accumulates into it (issued after p_full below)
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {

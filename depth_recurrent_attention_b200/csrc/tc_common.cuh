@@ -211,20 +211,6 @@ __device__ __forceinline__ void tmem_ld_fence(float *v) {
                  "+f"(v[30]), "+f"(v[31]));
 }
 
-// 2^x on the FMA and integer pipes, to share the softmax exponentials with the MUFU unit:
-// Cody-Waite style range reduction x = n + f with n = round(x) (the 1.5 * 2^23 rounding
-// constant) and f in [-1/2, 1/2], 2^f by a cubic fitted to 2^f on that interval by iterated
-// weighted least squares on the relative error (max relative error 7.6e-5, well under the
-// bf16 rounding of the softmax weights that use it), and 2^n added to the exponent bits.
-// x is clamped to >= -126 so the exponent field stays positive.
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0.05516991f, f, 0.24260705f), f, 0.69326091f), f, 0.99992834f);
-  return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
-}
-
 // 2^x with the hardware approximation (MUFU.EX2, flush to zero); used for softmax weights that
 // are stored in bf16 afterwards.
 __device__ __forceinline__ float ex2(float x) {
