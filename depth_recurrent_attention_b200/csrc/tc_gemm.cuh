@@ -8,9 +8,10 @@
 //   warps 2-5   epilogue: tcgen05.ld of the 128 x BN accumulator, row r per thread, then the
 //               caller's epilogue functor on column segments of SEG values (EW = 8: warps
 //               2-9, two per TMEM lane quarter, splitting the segments or column passes)
-//   next 2      (GATHER only) A producers: 16-byte cp.async of gathered rows into the
-//               128B-swizzled layout TMA would have written (with four epilogue warps the
-//               block stays at 8 warps, so the epilogue may use up to 255 registers a thread)
+//   next GATHER (gathered rows only: 2 or 4 warps) A producers: 16-byte cp.async of the
+//               rows into the 128B-swizzled layout TMA would have written (with four epilogue
+//               warps and two gather warps the block stays at 8 warps, so the epilogue may use
+//               up to 255 registers a thread)
 // Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap the MMAs of
 // tile i+1.  Every wait is bounded (tc::mbar_wait); on expiry the CTA winds down and the
 // device error flag is set.
@@ -87,14 +88,15 @@ template <class E> struct EpiTma<E, std::void_t<decltype(E::TMA_STORE)>> {
   static constexpr bool value = E::TMA_STORE;
 };
 
-template <int BN, int BK, int STAGES, bool GATHER, bool STAGED = false, int EW_ = 4,
+template <int BN, int BK, int STAGES, int GATHER, bool STAGED = false, int EW_ = 4,
           bool ROWPASS = false, bool TMAST = false>
 struct TcGemmCfg {
   static constexpr int A_BYTES = 128 * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int EW = EW_;  // epilogue warps: 4, or 8 (two per TMEM lane quarter)
   static_assert(EW == 4 || EW == 8, "epilogue warps");
-  static constexpr int THREADS = 64 + 32 * EW + (GATHER ? 64 : 0);
+  static_assert(GATHER == 0 || GATHER == 2 || GATHER == 4, "gather warps");
+  static constexpr int THREADS = 64 + 32 * EW + 32 * GATHER;
   // staged epilogues: EW warps x 32 rows x 64 fp32; row-pass epilogues with two warps a lane
   // quarter: one exchange list of up to 16 (value, raw score, index) a row
   // TMA-store epilogues: two 4 KB boxes a warp, 1024-byte aligned after the barrier block
@@ -115,7 +117,7 @@ struct TcGemmCfg {
 // ROWPASS: a CTA takes row tiles mt = blockIdx.x, blockIdx.x + gridDim.x, ... and runs all
 // N tiles of each in order, so the epilogue can carry per-row state across the N tiles
 // (Epi::State with row_begin / row_apply / row_end); otherwise tiles are strided over CTAs.
-template <int BN, int BK, int STAGES, bool GATHER, int SEG, class Epi, bool ROWPASS = false,
+template <int BN, int BK, int STAGES, int GATHER, int SEG, class Epi, bool ROWPASS = false,
           int EW = 4>
 __global__ void __launch_bounds__(
     TcGemmCfg<BN, BK, STAGES, GATHER, EpiStaged<Epi>::value && !ROWPASS, EW, ROWPASS,
@@ -157,7 +159,7 @@ __global__ void __launch_bounds__(
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; s++) {
-      mbar_init(smem_u32(&full[s]), GATHER ? 1 + 64 : 1);
+      mbar_init(smem_u32(&full[s]), 1 + 32 * GATHER);
       mbar_init(smem_u32(&empty[s]), 1);
     }
     for (int i = 0; i < 2; i++) {
@@ -422,9 +424,10 @@ __global__ void __launch_bounds__(
     }
   } else if (GATHER) {
     // ------------------------------------------------------------- gathered A producers
-    const int tid = threadIdx.x - (64 + 32 * C::EW);  // 0..63
+    constexpr int GT = 32 * (GATHER > 0 ? GATHER : 2), RSUB = GT / 8, NP = 128 / RSUB;
+    const int tid = threadIdx.x - (64 + 32 * C::EW);  // 0..GT-1
     const int c = tid & 7;              // 16-byte chunk of the 128-byte row slice
-    const int rsub = tid >> 3;          // 0..7
+    const int rsub = tid >> 3;          // 0..RSUB-1
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
@@ -432,11 +435,11 @@ __global__ void __launch_bounds__(
       int g, m0, m1;
       const int mt = t / NT;
       tc_tile_rows(a, mt, g, m0, m1);
-      const bf16 *src[16];
-      uint32_t bytes[16];
+      const bf16 *src[NP];
+      uint32_t bytes[NP];
 #pragma unroll
-      for (int p = 0; p < 16; p++) {
-        const int rr = p * 8 + rsub, r = m0 + rr;
+      for (int p = 0; p < NP; p++) {
+        const int rr = p * RSUB + rsub, r = m0 + rr;
         const bool v = r < m1;
         src[p] = a.A + (v ? (long)(a.arow[r] / a.arow_div) * a.lda : 0) + c * 8;
         bytes[p] = v ? 16u : 0u;
@@ -445,8 +448,8 @@ __global__ void __launch_bounds__(
         if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag, a.err)) { ok = false; break; }
         const uint32_t dst0 = smem_u32(sA + s * C::A_BYTES);
 #pragma unroll
-        for (int p = 0; p < 16; p++) {
-          const int rr = p * 8 + rsub;
+        for (int p = 0; p < NP; p++) {
+          const int rr = p * RSUB + rsub;
           cp_async16(dst0 + rr * 128 + ((c ^ (rr & 7)) << 4), src[p] + kb * 64, bytes[p]);
         }
         cp_async_arrive(smem_u32(&full[s]));

@@ -287,7 +287,7 @@ static int tc_init(dreamer_handle *h) {
 
 static void tc_destroy(dreamer_handle *h) {}
 
-template <int BN, int BK, int ST, bool GATHER, int SEG, class Epi, bool ROWPASS = false,
+template <int BN, int BK, int ST, int GATHER, int SEG, class Epi, bool ROWPASS = false,
           int EW = 4>
 static void tc_launch(dreamer_handle *h, const dreamer::tc::TcGemmArgs &a, const CUtensorMap &ta,
                       const CUtensorMap &tb, long max_tiles, const Epi &epi, cudaStream_t s,
@@ -384,19 +384,19 @@ static bool tc_gemm_qkv(dreamer_handle *h, const dreamer::GemmArgs &a, const dre
 #ifdef DREAMER_TEST_HOOKS
       t.skip_loads = skip;
 #endif
-      if (gather) tc_launch<64, 64, 8, true, 64>(h, t, ta, tb, mt, e, s);
-      else tc_launch<64, 64, 8, false, 64>(h, t, ta, tb, mt, e, s);
+      if (gather) tc_launch<64, 64, 8, 2, 64>(h, t, ta, tb, mt, e, s);
+      else tc_launch<64, 64, 8, 0, 64>(h, t, ta, tb, mt, e, s);
     } else if (bn == 256) {
       if (!tc_prepare<256, 64>(h, a, tiles, a.M, t, ta, tb, mt)) return false;
 #ifdef DREAMER_TEST_HOOKS
       t.skip_loads = skip;
 #endif
       if (ew8) {
-        if (gather) tc_launch<256, 64, 3, true, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
-        else tc_launch<256, 64, 3, false, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        if (gather) tc_launch<256, 64, 3, 2, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        else tc_launch<256, 64, 3, 0, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
       } else {
-        if (gather) tc_launch<256, 64, 4, true, 64>(h, t, ta, tb, mt, e, s);
-        else tc_launch<256, 64, 4, false, 64>(h, t, ta, tb, mt, e, s);
+        if (gather) tc_launch<256, 64, 4, 2, 64>(h, t, ta, tb, mt, e, s);
+        else tc_launch<256, 64, 4, 0, 64>(h, t, ta, tb, mt, e, s);
       }
     } else {
       if (!tc_prepare<128, 64>(h, a, tiles, a.M, t, ta, tb, mt)) return false;
@@ -404,11 +404,11 @@ static bool tc_gemm_qkv(dreamer_handle *h, const dreamer::GemmArgs &a, const dre
       t.skip_loads = skip;
 #endif
       if (ew8) {
-        if (gather) tc_launch<128, 64, 5, true, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
-        else tc_launch<128, 64, 5, false, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        if (gather) tc_launch<128, 64, 5, 2, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        else tc_launch<128, 64, 5, 0, 64, EpiQKV<T>, false, 8>(h, t, ta, tb, mt, e, s);
       } else {
-        if (gather) tc_launch<128, 64, 6, true, 64>(h, t, ta, tb, mt, e, s);
-        else tc_launch<128, 64, 6, false, 64>(h, t, ta, tb, mt, e, s);
+        if (gather) tc_launch<128, 64, 6, 2, 64>(h, t, ta, tb, mt, e, s);
+        else tc_launch<128, 64, 6, 0, 64>(h, t, ta, tb, mt, e, s);
       }
     }
     return true;
@@ -427,25 +427,25 @@ static bool tc_gemm_o(dreamer_handle *h, const dreamer::GemmArgs &a, const dream
     const int bn = tc_pick_bn(h, a);
     if (bn == 64) {
       if (!tc_prepare<64, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
-      if (a.arow && !a.a_sorted) tc_launch<64, 64, 8, true, 64>(h, t, ta, tb, mt, e, s);
-      else tc_launch<64, 64, 8, false, 64>(h, t, ta, tb, mt, e, s);
+      if (a.arow && !a.a_sorted) tc_launch<64, 64, 8, 2, 64>(h, t, ta, tb, mt, e, s);
+      else tc_launch<64, 64, 8, 0, 64>(h, t, ta, tb, mt, e, s);
     } else if (bn == 256) {
       if (!tc_prepare<256, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
       if (ew8) {
-        if (a.arow && !a.a_sorted) tc_launch<256, 64, 3, true, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
-        else tc_launch<256, 64, 3, false, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        if (a.arow && !a.a_sorted) tc_launch<256, 64, 3, 2, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        else tc_launch<256, 64, 3, 0, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
       } else {
-        if (a.arow && !a.a_sorted) tc_launch<256, 64, 4, true, 64>(h, t, ta, tb, mt, e, s);
-        else tc_launch<256, 64, 4, false, 64>(h, t, ta, tb, mt, e, s);
+        if (a.arow && !a.a_sorted) tc_launch<256, 64, 4, 2, 64>(h, t, ta, tb, mt, e, s);
+        else tc_launch<256, 64, 4, 0, 64>(h, t, ta, tb, mt, e, s);
       }
     } else {
       if (!tc_prepare<128, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
       if (ew8) {
-        if (a.arow && !a.a_sorted) tc_launch<128, 64, 5, true, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
-        else tc_launch<128, 64, 5, false, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        if (a.arow && !a.a_sorted) tc_launch<128, 64, 5, 2, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
+        else tc_launch<128, 64, 5, 0, 64, EpiO<T>, false, 8>(h, t, ta, tb, mt, e, s);
       } else {
-        if (a.arow && !a.a_sorted) tc_launch<128, 64, 6, true, 64>(h, t, ta, tb, mt, e, s);
-        else tc_launch<128, 64, 6, false, 64>(h, t, ta, tb, mt, e, s);
+        if (a.arow && !a.a_sorted) tc_launch<128, 64, 6, 2, 64>(h, t, ta, tb, mt, e, s);
+        else tc_launch<128, 64, 6, 0, 64>(h, t, ta, tb, mt, e, s);
       }
     }
     return true;
@@ -479,23 +479,23 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
   if (k_fused && !tc_prepare<256, 64>(h, za, nullptr, n, t2, ta2, tb2, mt2)) return false;
   if (dr == 64) {
     if (!tc_prepare<64, 64>(h, qa, nullptr, n, t, ta, tb, mt)) return false;
-    tc_launch<64, 64, 6, false, 64>(h, t, ta, tb, mt, eq, s);
+    tc_launch<64, 64, 6, 0, 64>(h, t, ta, tb, mt, eq, s);
   } else {
     if (!tc_prepare<128, 64>(h, qa, nullptr, n, t, ta, tb, mt)) return false;
-    tc_launch<128, 64, 6, false, 128>(h, t, ta, tb, mt, eq, s);
+    tc_launch<128, 64, 6, 0, 128>(h, t, ta, tb, mt, eq, s);
   }
   const float zs = 1.0f / sqrtf((float)dr);
   switch (k_fused) {  // top-k fused into the score GEMM
     case 4:
-      tc_launch<256, 64, 4, false, 32, EpiTopK<4>, true, 8>(
+      tc_launch<256, 64, 4, 0, 32, EpiTopK<4>, true, 8>(
           h, t2, ta2, tb2, mt2, EpiTopK<4>{E, zs, h->bias, idx, w, counts_a, counts_b}, s);
       return true;
     case 8:
-      tc_launch<256, 64, 4, false, 32, EpiTopK<8>, true, 8>(
+      tc_launch<256, 64, 4, 0, 32, EpiTopK<8>, true, 8>(
           h, t2, ta2, tb2, mt2, EpiTopK<8>{E, zs, h->bias, idx, w, counts_a, counts_b}, s);
       return true;
     case 16:
-      tc_launch<256, 64, 4, false, 32, EpiTopK<16>, true>(
+      tc_launch<256, 64, 4, 0, 32, EpiTopK<16>, true>(
           h, t2, ta2, tb2, mt2, EpiTopK<16>{E, zs, h->bias, idx, w, counts_a, counts_b}, s);
       return true;
     default:
@@ -535,10 +535,10 @@ static bool tc_proj_route(dreamer_handle *h, int l, const void *X, int n, cudaSt
                  h->psig, h->pcnt};
   if (dr == 64) {
     if (!tc_prepare<64, 64>(h, qa, nullptr, n, t, ta, tb, mt)) return false;
-    tc_launch<64, 64, 6, false, 64>(h, t, ta, tb, mt, e, s);
+    tc_launch<64, 64, 6, 0, 64>(h, t, ta, tb, mt, e, s);
   } else {
     if (!tc_prepare<128, 64>(h, qa, nullptr, n, t, ta, tb, mt)) return false;
-    tc_launch<128, 64, 6, false, 128>(h, t, ta, tb, mt, e, s);
+    tc_launch<128, 64, 6, 0, 128>(h, t, ta, tb, mt, e, s);
   }
   return true;
 }
@@ -566,7 +566,9 @@ static void tc_ffn_launch(dreamer_handle *h, const CUtensorMap &t1, const CUtens
   launch_k(h, kern, dim3((unsigned)grid), dim3(Cfg::THREADS), Cfg::SMEM, s, t1, t2, ty, a);
 }
 
-// Two grouped GEMMs: H = SiLU(X_gathered W1_e) stored in sorted order, then Y = H W2_e.
+// Two grouped GEMMs: H = SiLU(X_gathered W1_e) stored in sorted order, then Y = H W2_e.  The
+// up-projection's rows are gathered by four cp.async warps (its epilogue is light, and with
+// about one short tile per expert the gather is what bounds it).
 static bool tc_expert_two(dreamer_handle *h, const void *X, int n, cudaStream_t s) {
   using namespace dreamer;
   const dreamer_config &c = h->cfg;
@@ -594,22 +596,22 @@ static bool tc_expert_two(dreamer_handle *h, const void *X, int n, cudaStream_t 
       if (!tc_prepare<16, 64>(h, up, h->etiles_b, rows, tu, tau, tbu, mtu) ||
           !tc_prepare<256, 16>(h, dn, h->etiles_b, rows + 128, td, tad, tbd, mtd))
         return false;
-      tc_launch<16, 64, 8, true, 16>(h, tu, tau, tbu, mtu, eu, s);
-      tc_launch<256, 16, 8, false, 64>(h, td, tad, tbd, mtd, ed, s, &tyd);
+      tc_launch<16, 64, 8, 4, 16>(h, tu, tau, tbu, mtu, eu, s);
+      tc_launch<256, 16, 8, 0, 64>(h, td, tad, tbd, mtd, ed, s, &tyd);
       return true;
     case 32:
       if (!tc_prepare<32, 64>(h, up, h->etiles_b, rows, tu, tau, tbu, mtu) ||
           !tc_prepare<256, 32>(h, dn, h->etiles_b, rows + 128, td, tad, tbd, mtd))
         return false;
-      tc_launch<32, 64, 8, true, 32>(h, tu, tau, tbu, mtu, eu, s);
-      tc_launch<256, 32, 6, false, 64>(h, td, tad, tbd, mtd, ed, s, &tyd);
+      tc_launch<32, 64, 8, 4, 32>(h, tu, tau, tbu, mtu, eu, s);
+      tc_launch<256, 32, 6, 0, 64>(h, td, tad, tbd, mtd, ed, s, &tyd);
       return true;
     default:
       if (!tc_prepare<64, 64>(h, up, h->etiles_b, rows, tu, tau, tbu, mtu) ||
           !tc_prepare<256, 64>(h, dn, h->etiles_b, rows + 128, td, tad, tbd, mtd))
         return false;
-      tc_launch<64, 64, 8, true, 64>(h, tu, tau, tbu, mtu, eu, s);
-      tc_launch<256, 64, 4, false, 64>(h, td, tad, tbd, mtd, ed, s, &tyd);
+      tc_launch<64, 64, 8, 4, 64>(h, tu, tau, tbu, mtu, eu, s);
+      tc_launch<256, 64, 4, 0, 64>(h, td, tad, tbd, mtd, ed, s, &tyd);
       return true;
   }
 }
