@@ -1034,6 +1034,134 @@ __device__ __forceinline__ void rank_select(const unsigned long long *key, const
   __syncthreads();
 }
 
+// Top-k of stored raw router scores, one warp a token, E = 32 EPL experts (EPL a multiple of
+// 4, at most 64): lane j holds experts 4j..4j+3 of every 128 (float4 loads) as biased scores
+// v = fma(z, zscale, b) (NaN ranks last).  The k-th largest of the 32 lane maxima is at most
+// the k-th largest v, so only values at or above it can be picks: when there are at most 32
+// such candidates (the usual case) the warp sorts them once (bitonic, by better(): higher v,
+// then the lower index); otherwise it takes k rounds of a warp-wide best.  Either way the
+// picks and their order are those of a full sort.  The weights are emit_topk's, from the
+// picks' scaled raw scores.
+template <int KT, int EPL>
+__global__ void __launch_bounds__(256, 2) topk_rows_kernel(TopkArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  static_assert(EPL % 4 == 0 && EPL <= 64 && KT <= 32, "experts a lane");
+  constexpr unsigned FULL = 0xffffffffu;
+  constexpr int NONE = WarpTopK::NONE, NJ = EPL / 4;
+  extern __shared__ float bsh[];  // bias [E]
+  __shared__ float cvs[8][32];
+  __shared__ int ces[8][32];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < a.E; i += blockDim.x) bsh[i] = a.bias ? a.bias[i] : 0.f;
+  __syncthreads();
+  for (long tok = (long)blockIdx.x * 8 + wib; tok < a.n_tok; tok += (long)gridDim.x * 8) {
+    const float4 *src = reinterpret_cast<const float4 *>(a.z + tok * a.ldz);
+    float v[EPL];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < NJ; j++) {
+      const float4 q = src[j * 32 + lane];
+      const int c = (j * 32 + lane) * 4;
+      v[4 * j] = fmaxf(fmaf(q.x, a.zscale, bsh[c]), -INFINITY);
+      v[4 * j + 1] = fmaxf(fmaf(q.y, a.zscale, bsh[c + 1]), -INFINITY);
+      v[4 * j + 2] = fmaxf(fmaf(q.z, a.zscale, bsh[c + 2]), -INFINITY);
+      v[4 * j + 3] = fmaxf(fmaf(q.w, a.zscale, bsh[c + 3]), -INFINITY);
+      mx = max3f(mx, fmaxf(v[4 * j], v[4 * j + 1]), fmaxf(v[4 * j + 2], v[4 * j + 3]));
+    }
+    // the KT-th largest lane maximum: bitonic sort of the 32 maxima, descending
+    float sm = mx;
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const float o = __shfl_xor_sync(FULL, sm, stride);
+        const bool desc = (lane & size) == 0 || size == 32;
+        const bool lower = (lane & stride) == 0;
+        sm = (lower == desc) ? fmaxf(sm, o) : fminf(sm, o);
+      }
+    }
+    const float tau = __shfl_sync(FULL, sm, KT - 1);
+    int cnt = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; i++) cnt += v[i] >= tau ? 1 : 0;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(FULL, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const int C = __shfl_sync(FULL, incl, 31);
+    float bv = -INFINITY;
+    int be = NONE;
+    if (C <= 32) {
+      int off = incl - cnt;
+#pragma unroll
+      for (int i = 0; i < EPL; i++)
+        if (v[i] >= tau) {
+          cvs[wib][off] = v[i];
+          ces[wib][off] = ((i >> 2) * 32 + lane) * 4 + (i & 3);
+          off++;
+        }
+      __syncwarp();
+      float cv = lane < C ? cvs[wib][lane] : -INFINITY;
+      int ce = lane < C ? ces[wib][lane] : NONE;
+      __syncwarp();  // the lists are read before the next token writes them
+#pragma unroll
+      for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          const float ov = __shfl_xor_sync(FULL, cv, stride);
+          const int oe = __shfl_xor_sync(FULL, ce, stride);
+          const bool desc = (lane & size) == 0 || size == 32;
+          const bool lower = (lane & stride) == 0;
+          if ((lower == desc) != better(cv, ce, ov, oe)) {
+            cv = ov;
+            ce = oe;
+          }
+        }
+      }
+      bv = cv;
+      be = ce;
+    } else {
+      // many values tied at the bound: KT rounds of the warp-wide best not yet taken
+      unsigned long long taken = 0ull;
+#pragma unroll 1
+      for (int t = 0; t < KT; t++) {
+        float lv = -INFINITY;
+        int le = NONE, li = -1;
+#pragma unroll
+        for (int i = 0; i < EPL; i++) {
+          const int e = ((i >> 2) * 32 + lane) * 4 + (i & 3);
+          if (!((taken >> i) & 1ull) && better(v[i], e, lv, le)) {
+            lv = v[i];
+            le = e;
+            li = i;
+          }
+        }
+        float wv = lv;
+        int we = le;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ov = __shfl_xor_sync(FULL, wv, o);
+          const int oe = __shfl_xor_sync(FULL, we, o);
+          if (better(ov, oe, wv, we)) {
+            wv = ov;
+            we = oe;
+          }
+        }
+        if (li >= 0 && we == le) taken |= 1ull << li;  // the owner marks its pick
+        if (lane == t) {
+          bv = wv;
+          be = we;
+        }
+      }
+    }
+    const float z = (lane < KT && be != NONE) ? a.z[tok * a.ldz + be] * a.zscale : 0.f;
+    emit_topk(lane, KT, bv, be, z, tok, 0, a.idx, a.w, a.counts_a, a.counts_b);
+  }
+}
+
 // Top-k of stored scores z (one token's row of E), WPT warps a token; each warp scans a slice
 // of the experts 32 at a time, then the block ranks the WPT lists.
 template <int WPT>

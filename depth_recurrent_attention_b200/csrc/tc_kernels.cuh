@@ -15,6 +15,18 @@ namespace dreamer {
 // the depth rotation of depth l (k_e then enters the contraction exactly as stored, bf16) and
 // split into three bf16 parts hi + mid + lo that carry q to float32 precision; the score
 // contraction against [k | k | k] then runs on the tensor cores with fp32 accumulation.
+// Raw router scores z [n][ldz] in fp32, row r's columns n0.. (read by topk_rows_kernel).
+struct EpiScoreStore {
+  float *z;
+  long ldz;
+  template <int SEG>
+  __device__ __forceinline__ void operator()(int r, int token, int g, int n0, float *v) const {
+    float4 *d = reinterpret_cast<float4 *>(z + (long)r * ldz + n0);
+#pragma unroll
+    for (int i = 0; i < SEG; i += 4) d[i / 4] = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+  }
+};
+
 struct EpiRouterQ {
   int dr;
   const float2 *rope;  // depth-RoPE table row of depth l over d_r dims
@@ -471,9 +483,10 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
   GemmArgs za{};
   za.N = E; za.K = 3 * dr; za.G = 1; za.M = n; za.arow_div = 1;
   za.A = h->qsplit; za.lda = 3 * dr; za.B = h->k3; za.ldb = 3 * dr; za.bgstride = 0;
-  // The fused top-k gives each 128-row tile to one CTA for all E columns: worth it only when
-  // there are enough row tiles to fill the GPU; otherwise a warp per token scores its row from
-  // the split query on the CUDA cores, which spreads the rows over every SM.
+  // Scores on the tensor cores (then the top k of each row, from stored scores or inside the
+  // GEMM's epilogue) only when there are enough 128-row tiles to fill the GPU; otherwise a warp
+  // per token scores its row from the split query on the CUDA cores, which spreads the rows
+  // over every SM.
   int k_fused = (n + 127) / 128 >= h->num_sms / 2 && E % 256 == 0 ? c.top_k : 0;
   if (k_fused != 4 && k_fused != 8 && k_fused != 16) k_fused = 0;
   if (k_fused && !tc_prepare<256, 64>(h, za, nullptr, n, t2, ta2, tb2, mt2)) return false;
@@ -485,6 +498,28 @@ static bool tc_route(dreamer_handle *h, int l, const void *X, int n, int *idx, f
     tc_launch<128, 64, 6, 0, 128>(h, t, ta, tb, mt, eq, s);
   }
   const float zs = 1.0f / sqrtf((float)dr);
+  // Up to 2048 experts: the score GEMM stores z and a warp a token picks the top k of its row
+  // (a few hundred instructions a row); beyond that the top k is kept in the GEMM's epilogue.
+  const int epl = E / 32;
+  if (k_fused && E % 128 == 0 && E <= 2048 && h->ldz == E) {
+    tc_launch<256, 64, 4, 0, 64>(h, t2, ta2, tb2, mt2, EpiScoreStore{h->zbuf, (long)h->ldz}, s);
+    TopkArgs k{};
+    k.n_tok = n; k.E = E; k.k = k_fused; k.mode = 0; k.z = h->zbuf; k.ldz = h->ldz; k.zscale = zs;
+    k.bias = h->bias; k.idx = idx; k.w = w; k.counts_a = counts_a; k.counts_b = counts_b;
+    void (*kern)(TopkArgs) = nullptr;
+#define TOPK_ROWS_CASE(KT)                                                              \
+  if (k_fused == KT)                                                                    \
+    kern = epl == 64 ? topk_rows_kernel<KT, 64> : epl == 32 ? topk_rows_kernel<KT, 32>  \
+         : epl == 16 ? topk_rows_kernel<KT, 16> : topk_rows_kernel<KT, 8>;
+    TOPK_ROWS_CASE(4)
+    TOPK_ROWS_CASE(8)
+    TOPK_ROWS_CASE(16)
+#undef TOPK_ROWS_CASE
+    long grid = ((long)n + 7) / 8;
+    if (grid > 2L * h->num_sms) grid = 2L * h->num_sms;
+    launch_k(h, kern, dim3((unsigned)grid), dim3(256), (size_t)E * sizeof(float), s, k);
+    return true;
+  }
   switch (k_fused) {  // top-k fused into the score GEMM
     case 4:
       tc_launch<256, 64, 4, 0, 32, EpiTopK<4>, true, 8>(
