@@ -15,15 +15,31 @@ namespace dreamer {
 // the depth rotation of depth l (k_e then enters the contraction exactly as stored, bf16) and
 // split into three bf16 parts hi + mid + lo that carry q to float32 precision; the score
 // contraction against [k | k | k] then runs on the tensor cores with fp32 accumulation.
-// Raw router scores z [n][ldz] in fp32, row r's columns n0.. (read by topk_rows_kernel).
+// Raw router scores z [n][ldz] in fp32 (read by topk_rows_kernel), through the staged
+// epilogue: a pass's 32 rows x 64 columns leave the warp as four full 128-byte lines a store.
 struct EpiScoreStore {
   float *z;
   long ldz;
+  static constexpr bool STAGED = true;
+  using Aux = int;
+  __device__ __forceinline__ int row_aux(int, int) const { return 0; }
+  template <int NR>
+  __device__ __forceinline__ void prefetch(const int *, const int *, const int *, int, int, int,
+                                           int) const {}
   template <int SEG>
-  __device__ __forceinline__ void operator()(int r, int token, int g, int n0, float *v) const {
-    float4 *d = reinterpret_cast<float4 *>(z + (long)r * ldz + n0);
+  __device__ __forceinline__ void transform(int, int, int, int, float *) const {}
+  // the lane holds columns col..col+3 (v[i][0..3]) and col+32..col+35 (v[i][4..7]) of rows r[i]
+  template <int NR, int NV>
+  __device__ __forceinline__ void store_rows(const int *r, const int *, const int *, int, int col,
+                                             const float (*v)[NV]) const {
+    static_assert(NV == 8, "passes of 64 columns");
 #pragma unroll
-    for (int i = 0; i < SEG; i += 4) d[i / 4] = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    for (int i = 0; i < NR; i++) {
+      if (r[i] < 0) continue;
+      float *d = z + (long)r[i] * ldz + col;
+      *reinterpret_cast<float4 *>(d) = make_float4(v[i][0], v[i][1], v[i][2], v[i][3]);
+      *reinterpret_cast<float4 *>(d + 32) = make_float4(v[i][4], v[i][5], v[i][6], v[i][7]);
+    }
   }
 };
 
