@@ -35,6 +35,7 @@ struct TcGemmArgs {
   int *err;
   int skip_loads;     // test-hook build only: the TMA producer issues no loads (0 otherwise)
   const int2 *ttab;   // [tiles] (group, first row | rows << 24) of each 128-row tile, or null
+  int mswz;           // row tiles a raster block: the N tiles of mswz row tiles run together
 };
 
 // per-row epilogue state: Epi::State for row-pass epilogues, nothing otherwise
@@ -151,10 +152,24 @@ __global__ void __launch_bounds__(
       nt = i % NT;
       return mt < mtiles;
     }
+    // blocks of mswz row tiles; inside a block the row tile changes fastest, so the CTAs
+    // working at one time share each B tile (and the block's A tiles stay in L2)
     const int t = blockIdx.x + i * gridDim.x;
-    mt = t / NT;
-    nt = t % NT;
-    return t < total;
+    if (a.mswz <= 1) {
+      mt = t / NT;
+      nt = t % NT;
+      return t < total;
+    }
+    if (t >= total) {
+      mt = nt = 0;
+      return false;
+    }
+    const int sw = a.mswz;
+    const int per = sw * NT, blk = t / per, u = t - blk * per;
+    const int rows = min(sw, mtiles - blk * sw);  // >= 1 since t < mtiles * NT
+    nt = u / rows;
+    mt = blk * sw + u % rows;
+    return true;
   };
 
   if (threadIdx.x == 0) {

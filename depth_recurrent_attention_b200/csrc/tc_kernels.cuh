@@ -364,6 +364,9 @@ static bool tc_prepare(dreamer_handle *h, const dreamer::GemmArgs &a, const int 
   t.ttab = nullptr;
   if (a.goffs && tiles == h->etiles_b && h->cfg.n_experts <= 8192) t.ttab = h->etab;
   if (a.goffs && tiles == h->ptiles_b) t.ttab = h->ptab;
+  // projections whose weights (a group's N x K) do not stay in L2 next to the streams around
+  // them: raster blocks of 16 row tiles, so each B tile comes from DRAM about once
+  t.mswz = (tiles != h->etiles_b && a.N / BN >= 8 && 2L * a.N * a.K >= (32L << 20)) ? 16 : 1;
   max_tiles = ((a.M + 127) / 128 + (a.goffs ? a.G : 0)) * (long)(a.N / BN);
   return true;
 }
