@@ -6,20 +6,20 @@
 // share every K/V block (heaviest pairs first):
 //   warp 0      TMA: both Q tiles once, then K_j into a KST-deep ring
 //   warp 2      TMA: V_j into a VST-deep ring
-//   warp 1      TMEM allocator + MMA issuer: S_A(j), S_B(j) = Q K_j^T into one TMEM buffer
-//               per tile, then O_t += P_t(j-1) V_(j-1) for both tiles (one block behind, so the
-//               tensor core computes block j's scores while the softmax works on j-1)
+//   warp 1      TMEM allocator + MMA issuer: S_t(0) = Q_t K_0^T for both tiles; then per
+//               block j and tile t, O_t += P_t(j) V_j with P read from TMEM, and S_t(j+1)
+//               into the same TMEM columns (issued after the P.V, so it runs after it);
+//               tile B's MMAs keep the tensor core busy while tile A's softmax runs and the
+//               other way round
 //   warps 3-10  softmax, one query row per thread: tile A on warps 4, 5, 6, 3 and tile B on
 //               warps 8, 9, 10, 7 (a warp reads the TMEM lanes of its warp index mod 4), 11
 //               warps in all so that a thread may hold a row of 128 scores in registers:
-//               the row's 128 scores come out of TMEM in one batch of loads (S is released to
-//               the next QK^T right away), then the row max, and P = exp2(s - m_ref) written
-//               as bf16 into the swizzled K-major operand in shared memory and summed (every
-//               exponential on MUFU: the softmax warps are issue-bound, and a polynomial on
-//               the FMA pipe costs more issue slots than it saves).  O lives in
-//               TMEM and is only rescaled when the running max grows by more than 2^8 (P stays
-//               <= 256), so most blocks need no O traffic at all; the last step divides O by
-//               the sum.
+//               the row's 128 scores come out of TMEM in one batch of loads, then the row
+//               max, P = exp2(s - m_ref) summed and written as bf16 pairs over the first 64
+//               columns of the tile's S (every exponential on MUFU).  O lives in TMEM and is
+//               only rescaled when the running max grows by more than 2^8 (P stays <= 256),
+//               so most blocks need no O traffic at all; the last step divides O by the sum.
+// TMEM: S_A columns 0..127, S_B 128..255, O_A 256.., O_B 256 + D.. (512 allocated).
 // V is consumed in its natural [key][d] layout as an MN-major B operand.
 #pragma once
 #include "tc_common.cuh"
@@ -57,6 +57,32 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v) {
       : "memory");
 }
 
+// 32 lanes x 32 columns of 32-bit words into TMEM; the wait is a separate tmem_st_wait()
+__device__ __forceinline__ void tmem_st32_nowait(uint32_t taddr, const uint32_t *v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]^T: A (M = 128 rows on the 128 lanes, K packed two bf16 a
+// 32-bit column, the lower K in the low half) read from tensor memory, one thread issues.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 struct SaArgs {
   int S, H, h, n_qt;      // tokens per sequence, heads, hidden, query tiles per sequence
   int n_pairs;            // query-tile pairs per sequence
@@ -72,13 +98,11 @@ template <int D>
 struct SaCfg {
   static constexpr int CH = D / 64;                 // 64-column chunks of a head
   static constexpr int TILE = 128 * 128;            // bytes of one [128 x 64] bf16 chunk
-  static constexpr int KST = D == 64 ? 3 : 2;       // K ring depth
-  static constexpr int VST = D == 64 ? 3 : 1;       // V ring depth
+  static constexpr int KST = D == 64 ? 4 : 3;       // K ring depth
+  static constexpr int VST = D == 64 ? 4 : 2;       // V ring depth
   static constexpr int Q_BYTES = 2 * CH * TILE;     // both query tiles
   static constexpr int KV_BYTES = CH * TILE;        // one K (or V) block
-  static constexpr int P_BYTES = 2 * TILE;          // one tile's P [128 x 128]
-  static constexpr int SMEM =
-      Q_BYTES + (KST + VST) * KV_BYTES + 2 * P_BYTES + 1024 + 256;
+  static constexpr int SMEM = Q_BYTES + (KST + VST) * KV_BYTES + 1024 + 256;
   static_assert(SMEM <= 227 * 1024, "smem");
 };
 
@@ -92,14 +116,12 @@ __global__ void __launch_bounds__(352, 1)
   uint8_t *sQ = smem;
   uint8_t *sK = sQ + C::Q_BYTES;
   uint8_t *sV = sK + KST * C::KV_BYTES;
-  uint8_t *sP = sV + VST * C::KV_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sP + 2 * C::P_BYTES);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sV + VST * C::KV_BYTES);
   uint64_t *q_full = bars;
   uint64_t *k_full = q_full + 1, *k_empty = k_full + KST;
   uint64_t *v_full = k_empty + KST, *v_empty = v_full + VST;
-  uint64_t *s_full = v_empty + VST, *s_free = s_full + 2;
-  uint64_t *p_full = s_free + 2, *pv_done = p_full + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pv_done + 2);
+  uint64_t *s_full = v_empty + VST, *p_full = s_full + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(p_full + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -125,9 +147,7 @@ __global__ void __launch_bounds__(352, 1)
     }
     for (int i = 0; i < 2; i++) {
       mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&s_free[i]), 128);
       mbar_init(smem_u32(&p_full[i]), 128);
-      mbar_init(smem_u32(&pv_done[i]), 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -161,7 +181,7 @@ __global__ void __launch_bounds__(352, 1)
       const int NS = isK ? KST : VST;
       uint64_t *fullb = isK ? k_full : v_full, *emptyb = isK ? k_empty : v_empty;
       uint8_t *ring = isK ? sK : sV;
-      int issued_ph[3] = {-1, -1, -1};
+      int issued_ph[4] = {-1, -1, -1, -1};
       bool ok = true;
       for (int j = 0; j < nb; j++) {
         const int s = j % NS;
@@ -189,54 +209,66 @@ __global__ void __launch_bounds__(352, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer
+    // Per tile t the order is S_t(0), then for each block j: P_t(j) V_j (P read from the S_t
+    // columns in TMEM), S_t(j+1) into the same columns (issued after, so it runs after the
+    // P.V has read them), one commit to s_full[t]: the softmax sees S_t(j+1) and, with it, O_t
+    // holding every block up to j.  Tile B's work fills the tensor core while tile A's
+    // softmax runs, and the other way round.
     if (lane == 0) {
       constexpr uint32_t ID_S = idesc_bf16_m128(128);
       constexpr uint32_t ID_PV = idesc_bf16_m128_bmn(D);
       bool ok = mbar_wait(smem_u32(q_full), 0, abort_flag, a.err);
-      const uint32_t q0 = smem_u32(sQ), p0 = smem_u32(sP);
-      auto issue_pv = [&](int jj) -> bool {
-        const int vs = jj % VST;
-        if (!mbar_wait(smem_u32(&v_full[vs]), (jj / VST) & 1, abort_flag, a.err)) return false;
+      const uint32_t q0 = smem_u32(sQ);
+      auto issue_s = [&](int t, uint32_t k0) {
+        const uint32_t qt0 = q0 + t * CH * C::TILE;
+#pragma unroll
+        for (int k = 0; k < D / 16; k++) {
+          const uint32_t off = (k >> 2) * C::TILE + (k & 3) * 32;
+          mma_bf16(tS + t * 128, desc_k128(qt0 + off), desc_k128(k0 + off), ID_S, k != 0);
+        }
+      };
+      if (ok && mbar_wait(smem_u32(&k_full[0]), 0, abort_flag, a.err)) {
+        tc_fence_after();
+        const uint32_t k0 = smem_u32(sK);
+        issue_s(0, k0);
+        mma_commit(smem_u32(&s_full[0]));
+        if (nbB > 0) {
+          issue_s(1, k0);
+          mma_commit(smem_u32(&s_full[1]));
+        }
+        mma_commit(smem_u32(&k_empty[0]));
+      } else {
+        ok = false;
+      }
+      for (int j = 0; j < nb && ok; j++) {
+        const int vs = j % VST;
+        if (!mbar_wait(smem_u32(&v_full[vs]), (j / VST) & 1, abort_flag, a.err)) break;
         tc_fence_after();
         const uint32_t v0 = smem_u32(sV + vs * C::KV_BYTES);
-        for (int t = 0; t < 2; t++) {
-          if (jj >= (t == 0 ? nbA : nbB)) continue;
-          if (!mbar_wait(smem_u32(&p_full[t]), jj & 1, abort_flag, a.err)) return false;
+        const bool next = j + 1 < nb;
+        const int ks = (j + 1) % KST;
+        uint32_t k1 = 0;
+        if (next) {
+          if (!mbar_wait(smem_u32(&k_full[ks]), ((j + 1) / KST) & 1, abort_flag, a.err)) break;
           tc_fence_after();
-          const uint32_t pt = p0 + t * C::P_BYTES;
-#pragma unroll
-          for (int k = 0; k < 8; k++) {  // 128 keys, 16 per instruction
-            const uint32_t poff = (k >> 2) * C::TILE + (k & 3) * 32;
-            mma_bf16(tO + t * D, desc_k128(pt + poff), desc_mn128(v0 + k * 2048, C::TILE), ID_PV,
-                     (jj | k) != 0);
-          }
-          mma_commit(smem_u32(&pv_done[t]));
+          k1 = smem_u32(sK + ks * C::KV_BYTES);
         }
-        mma_commit(smem_u32(&v_empty[vs]));
-        return true;
-      };
-      for (int j = 0; j < nb && ok; j++) {
-        const int ks = j % KST;
-        if (!mbar_wait(smem_u32(&k_full[ks]), (j / KST) & 1, abort_flag, a.err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t k0 = smem_u32(sK + ks * C::KV_BYTES);
         for (int t = 0; t < 2; t++) {
-          if (j >= (t == 0 ? nbA : nbB)) continue;
-          if (!mbar_wait(smem_u32(&s_free[t]), (j & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
+          const int nbt = t == 0 ? nbA : nbB;
+          if (j >= nbt) continue;
+          if (!mbar_wait(smem_u32(&p_full[t]), j & 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t qt0 = q0 + t * CH * C::TILE;
 #pragma unroll
-          for (int k = 0; k < D / 16; k++) {
-            const uint32_t off = (k >> 2) * C::TILE + (k & 3) * 32;
-            mma_bf16(tS + t * 128, desc_k128(qt0 + off), desc_k128(k0 + off), ID_S, k != 0);
-          }
+          for (int k = 0; k < 8; k++)  // 128 keys, 16 per instruction (8 TMEM columns of P)
+            mma_bf16_ts(tO + t * D, tS + t * 128 + k * 8, desc_mn128(v0 + k * 2048, C::TILE), ID_PV,
+                        (j | k) != 0);
+          if (j + 1 < nbt) issue_s(t, k1);
           mma_commit(smem_u32(&s_full[t]));
         }
         if (!ok) break;
-        mma_commit(smem_u32(&k_empty[ks]));
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        mma_commit(smem_u32(&v_empty[vs]));
+        if (next) mma_commit(smem_u32(&k_empty[ks]));
       }
-      if (ok) issue_pv(nb - 1);
     }
   } else if (warp >= 3) {
     // ------------------------------------------------- softmax (tile A: warps 3-6, B: 7-10)
@@ -250,7 +282,6 @@ __global__ void __launch_bounds__(352, 1)
       const uint32_t lane_off = (uint32_t)(q * 32) << 16;
       const uint32_t sbuf = tS + t * 128 + lane_off;
       const uint32_t obuf = tO + t * D + lane_off;
-      uint8_t *prow = sP + t * C::P_BYTES + row * 128;
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < nbt; j++) {
@@ -258,16 +289,13 @@ __global__ void __launch_bounds__(352, 1)
         tc_fence_after();
         const bool diag = (j == qt);
         const int lim = qi - j * 128;  // diagonal block: last visible key of the row
-        // the row's 128 scores into registers with four loads in flight, then S is free for
-        // the next block's QK^T while this block's softmax runs
+        // the row's 128 scores into registers with four loads in flight
         float sv[128];
 #pragma unroll
         for (int c = 0; c < 128; c += 32) tmem_ld32_async(sbuf + c, sv + c);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 128; c += 32) tmem_ld_fence(sv + c);
-        tc_fence_before();
-        mbar_arrive(smem_u32(&s_free[t]));
         // the diagonal block: keys past the row's own position get -inf (weight 0 below)
         if (diag) {
 #pragma unroll
@@ -293,34 +321,28 @@ __global__ void __launch_bounds__(352, 1)
           m_new = mx;
           alpha = ex2(m_ref - mx);
         }
-        // P_t(j-1) V was consumed: its P buffer is free and O_t holds every earlier block
-        if (j > 0) {
-          if (!mbar_wait(smem_u32(&pv_done[t]), (j - 1) & 1, abort_flag, a.err)) { ok = false; break; }
-          tc_fence_after();
-        }
-        // P = 2^(s * scale - m) as bf16, K-major SW128 (key chunk kc at kc * TILE, 16-byte unit
-        // u of the row at ((u ^ (row & 7)) << 4)), summed.  Scale, offset and sum on packed
-        // fp32 pairs (masked keys: 2^-inf = 0 exactly).
+        // P = 2^(s * scale - m) as bf16 pairs (the lower key in the low half) into the first
+        // 64 columns of this tile's S in TMEM, where the P.V MMA reads it, and summed.  Scale,
+        // offset and sum on packed fp32 pairs (masked keys: 2^-inf = 0 exactly).
         const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), nm2 = f2_pack(-m_new, -m_new);
         uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};  // four independent sums of pairs
 #pragma unroll
-        for (int u8 = 0; u8 < 16; u8++) {
-          const int kc = u8 >> 3, u = u8 & 7;
-          uint32_t w[4];
+        for (int hh = 0; hh < 2; hh++) {
+          uint32_t w[32];
 #pragma unroll
-          for (int e = 0; e < 4; e++) {
-            const int i = u8 * 8 + 2 * e;
+          for (int e = 0; e < 32; e++) {
+            const int i = hh * 64 + 2 * e;
             const float2 x = f2_unpack(f2_fma(f2_pack(sv[i], sv[i + 1]), sc2, nm2));
             const float p0 = ex2(x.x), p1 = ex2(x.y);
-            rs2[e] = f2_add(rs2[e], f2_pack(p0, p1));
+            rs2[e & 3] = f2_add(rs2[e & 3], f2_pack(p0, p1));
             w[e] = bf2_pack_rn(p0, p1);
           }
-          *reinterpret_cast<uint4 *>(prow + kc * C::TILE + ((u ^ (row & 7)) << 4)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+          tmem_st32_nowait(sbuf + hh * 32, w);
         }
         const float2 rsf = f2_unpack(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])));
         const float rs = rsf.x + rsf.y;
-        // O rescaled before P_t(j) V accumulates into it (issued after p_full below)
+        // O rescaled before P_t(j) V accumulates into it (s_full of block j also means that
+        // P_t(j-1) V has completed; P_t(j) V is issued after p_full below)
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
           for (int c = 0; c < D; c += 32) {
@@ -333,10 +355,12 @@ __global__ void __launch_bounds__(352, 1)
         }
         l = l * alpha + rs;
         m_ref = m_new;
-        fence_proxy_async();
+        tmem_st_wait();
+        tc_fence_before();
         mbar_arrive(smem_u32(&p_full[t]));
       }
-      if (ok && mbar_wait(smem_u32(&pv_done[t]), (nbt - 1) & 1, abort_flag, a.err)) {
+      // the commit after the last P.V: O_t is final
+      if (ok && mbar_wait(smem_u32(&s_full[t]), nbt & 1, abort_flag, a.err)) {
         tc_fence_after();
         const float inv = 1.0f / l;
         const long orow = a.out_rows ? a.out_rows[row0 + qi] : row0 + qi;
