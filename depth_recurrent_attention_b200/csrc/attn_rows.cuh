@@ -9,6 +9,7 @@
 // of them, reduces the partial dot products over the CH lanes of a row with shuffles, keeps an
 // online softmax over groups, and reduces the output chunks over the RPW rows at the end.
 #pragma once
+#include <type_traits>
 #include "common.cuh"
 
 namespace dreamer {
@@ -396,12 +397,15 @@ __global__ void __launch_bounds__(1024) da_bulk_kernel(DaBulkArgs a) {
 // partial dot products of its chunk c with the NR = 8 / G rows of group g, and one transposed
 // butterfly (log2 NR halving exchanges, then plain ones) leaves every row's full score in
 // CH / NR lanes with NR - 1 + log2(CH / NR) shuffles for the batch instead of log2(CH) a row.
-// Products and accumulations use the packed FP32 pair instructions (fma.rn.f32x2), bf16
-// values widen to fp32 by a shift or a mask.  One online-softmax update a batch (max and sum
-// by warp shuffles); each lane then fetches the NR weights of its group's rows and
+// The q.k products take the bf16 pairs as they are (fma.rn.f32.bf16: bf16 inputs, fp32
+// accumulate, each product exact); the V accumulation uses packed fp32 pairs
+// (fma.rn.f32x2) with V widened by a shift or a mask.  One online-softmax update a batch (max
+// and sum by warp shuffles); each lane then fetches the NR weights of its group's rows and
 // accumulates the V rows into its 8 output elements; the G groups' partial outputs are
-// summed at the token's last chunk.  (papernotes "Key design 1": attention over the token's
-// own states at depths 0..l.)
+// summed at the token's last chunk.  Batches with all 8 rows present (every one but a
+// chunk's last partial batch) run without per-row checks: the kernel is bound by the
+// instructions a streamed byte costs, and the checks' branches were a sixth of them.
+// (papernotes "Key design 1": attention over the token's own states at depths 0..l.)
 // =======================================================================================
 namespace tcda {
 // packed fp32 pairs: {lo, hi} in one 64-bit register
@@ -416,6 +420,15 @@ __device__ __forceinline__ float2 up2(uint64_t v) {
   return f;
 }
 // two bf16 of one 32-bit word as an fp32 pair (low element, high element)
+// acc + a.lo * b.lo + a.hi * b.hi for bf16 pairs a, b: mixed-precision FMAs (bf16 inputs,
+// fp32 accumulate; each product is exact in fp32)
+__device__ __forceinline__ float dot2_bf16(uint32_t a, uint32_t b, float acc) {
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, al, bl, %0;\n\tfma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(a), "r"(b));
+  return acc;
+}
 __device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xffff0000u));
@@ -491,7 +504,8 @@ __global__ void __launch_bounds__(1024) da_fast_kernel(DaBulkArgs a) {
   const int head = warp;
   const bool active = head < a.H;
   const float sl2 = 1.4426950408889634f * rsqrtf((float)D);
-  uint64_t q2[4], o2[4];
+  uint64_t o2[4];
+  uint32_t qb[4];  // the query slice as bf16 pairs
   float m = -INFINITY, lsum = 0.f;
   int consumed = 0;
   for (int j = 0; j < nitems; j++) {
@@ -518,29 +532,28 @@ __global__ void __launch_bounds__(1024) da_fast_kernel(DaBulkArgs a) {
     if (active) {
       if (c == 0) {  // a new token: its query, a fresh softmax
         const uint4 qw = *reinterpret_cast<const uint4 *>(q_slot(b) + (size_t)(head * D + cc * 8) * sizeof(bf16));
-        q2[0] = tcda::bf2_to_f2(qw.x); q2[1] = tcda::bf2_to_f2(qw.y);
-        q2[2] = tcda::bf2_to_f2(qw.z); q2[3] = tcda::bf2_to_f2(qw.w);
+        qb[0] = qw.x; qb[1] = qw.y; qb[2] = qw.z; qb[3] = qw.w;
 #pragma unroll
         for (int w = 0; w < 4; w++) o2[w] = 0ull;
         m = -INFINITY;
         lsum = 0.f;
       }
-#pragma unroll 1
-      for (int b0 = 0; b0 < nr; b0 += 8) {
+      // one batch of 8 rows; FULL: all 8 rows exist (no per-row checks)
+      auto batch = [&](const int b0, auto full_tag) {
+        constexpr bool FULL = decltype(full_tag)::value;
         // partial dot products of this lane's 8 elements with the NR rows of its group
         float v[NR];
 #pragma unroll
         for (int i = 0; i < NR; i++) {
           const int r = b0 + g * NR + i;
           v[i] = 0.f;
-          if (r < nr) {
+          if (FULL || r < nr) {
             const uint4 kw = *reinterpret_cast<const uint4 *>(bk + (size_t)r * rstride);
-            uint64_t acc = tcda::mul2(q2[0], tcda::bf2_to_f2(kw.x));
-            acc = tcda::fma2(q2[1], tcda::bf2_to_f2(kw.y), acc);
-            acc = tcda::fma2(q2[2], tcda::bf2_to_f2(kw.z), acc);
-            acc = tcda::fma2(q2[3], tcda::bf2_to_f2(kw.w), acc);
-            const float2 f = tcda::up2(acc);
-            v[i] = f.x + f.y;
+            // bf16 products are exact in fp32: no widening of q or k, two fp32 sums
+            float a0 = tcda::dot2_bf16(qb[0], kw.x, 0.f), a1 = tcda::dot2_bf16(qb[1], kw.y, 0.f);
+            a0 = tcda::dot2_bf16(qb[2], kw.z, a0);
+            a1 = tcda::dot2_bf16(qb[3], kw.w, a1);
+            v[i] = a0 + a1;
           }
         }
         // transposed butterfly: halving exchanges over the lanes of a row, then plain ones
@@ -558,7 +571,7 @@ __global__ void __launch_bounds__(1024) da_fast_kernel(DaBulkArgs a) {
 #pragma unroll
         for (int mk = DUP / 2; mk >= 1; mk >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], mk);
         // online softmax over the batch (scores in log2 units)
-        const bool valid = b0 + myrow < nr;
+        const bool valid = FULL || b0 + myrow < nr;
         const float x = valid ? v[0] * sl2 : -INFINITY;
         const float mn = fmaxf(m, warp_max(x));
         const float alpha = tcda::ex2a(m - mn);
@@ -573,7 +586,7 @@ __global__ void __launch_bounds__(1024) da_fast_kernel(DaBulkArgs a) {
         for (int i = 0; i < NR; i++) {
           const float pi = __shfl_sync(0xffffffffu, p, g * CH + i * DUP);
           const int r = b0 + g * NR + i;
-          if (r < nr) {
+          if (FULL || r < nr) {
             const uint4 vw = *reinterpret_cast<const uint4 *>(bk + (size_t)r * rstride + vofs);
             const uint64_t p2 = tcda::pk2(pi, pi);
             o2[0] = tcda::fma2(p2, tcda::bf2_to_f2(vw.x), o2[0]);
@@ -582,7 +595,11 @@ __global__ void __launch_bounds__(1024) da_fast_kernel(DaBulkArgs a) {
             o2[3] = tcda::fma2(p2, tcda::bf2_to_f2(vw.w), o2[3]);
           }
         }
-      }
+      };
+      int b0 = 0;
+#pragma unroll 1
+      for (; b0 + 8 <= nr; b0 += 8) batch(b0, std::true_type{});
+      if (b0 < nr) batch(b0, std::false_type{});
       if (c == nch - 1) {  // the token's last chunk: sum the groups, normalise, store
         float of[8];
 #pragma unroll
