@@ -573,10 +573,18 @@ __global__ void __launch_bounds__(1024) da_fast_kernel(DaBulkArgs a) {
         // online softmax over the batch (scores in log2 units)
         const bool valid = FULL || b0 + myrow < nr;
         const float x = valid ? v[0] * sl2 : -INFINITY;
-        const float mn = fmaxf(m, warp_max(x));
+        // max and sum over the batch's rows: a row's score sits in DUP neighbouring lanes
+        // (bitwise equal), so the exchanges skip the low log2(DUP) lane bits
+        float xm = x;
+#pragma unroll
+        for (int mk = DUP; mk < 32; mk <<= 1) xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, mk));
+        const float mn = fmaxf(m, xm);
         const float alpha = tcda::ex2a(m - mn);
         const float p = valid ? tcda::ex2a(x - mn) : 0.f;
-        lsum = lsum * alpha + warp_sum(p) * (1.0f / DUP);
+        float ps = p;
+#pragma unroll
+        for (int mk = DUP; mk < 32; mk <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, mk);
+        lsum = lsum * alpha + ps;
         m = mn;
         const uint64_t al2 = tcda::pk2(alpha, alpha);
 #pragma unroll
