@@ -743,6 +743,20 @@ __global__ void __launch_bounds__(256) dec_bulk_kernel(DecBulkArgs a) {
     o[i] = 0.f;
   }
   float m = -INFINITY, lsum = 0.f;
+  // bf16 at head dim 64 / 128: depth attention's batch form (8 rows a warp batch, the
+  // transposed butterfly, bf16 q.k products in mixed FMAs, check-free full batches); warp w
+  // takes batches w, w + 8, ... of each chunk with its own online softmax
+  constexpr bool FAST = std::is_same<T, bf16>::value && (D == 64 || D == 128);
+  constexpr int FCH = FAST ? D / 8 : 16, FG = 32 / FCH, FNR = 8 / FG, FDUP = FCH / FNR;
+  const int fg = lane / FCH;
+  const int myrow = fg * FNR + cc / FDUP;
+  uint32_t qb[4] = {0u, 0u, 0u, 0u};
+  uint64_t o2[4] = {0ull, 0ull, 0ull, 0ull};
+  if constexpr (FAST) {
+    const uint4 qw = *reinterpret_cast<const uint4 *>(reinterpret_cast<const bf16 *>(a.q) +
+                                                      (long)b * a.ldq + head * D + cc * 8);
+    qb[0] = qw.x; qb[1] = qw.y; qb[2] = qw.z; qb[3] = qw.w;
+  }
   int consumed = 0;
   for (int c = 0; c < nch; c++) {
     const int st = c % NST;
@@ -763,6 +777,74 @@ __global__ void __launch_bounds__(256) dec_bulk_kernel(DecBulkArgs a) {
     const T *sk = reinterpret_cast<const T *>(dsm + (size_t)st * 2 * cbytes);
     const T *sv = reinterpret_cast<const T *>(dsm + (size_t)st * 2 * cbytes + cbytes);
     const int nr = min(a.chunk, nrow - c * a.chunk);
+    if constexpr (FAST) {
+      const uint8_t *kb = reinterpret_cast<const uint8_t *>(sk) + cc * 16;
+      const uint8_t *vb = reinterpret_cast<const uint8_t *>(sv) + cc * 16;
+      constexpr uint32_t RS = D * 2;  // bytes of a key (value) row
+      auto batch = [&](const int b0, auto full_tag) {
+        constexpr bool FULL = decltype(full_tag)::value;
+        float v[FNR];
+#pragma unroll
+        for (int i = 0; i < FNR; i++) {
+          const int r = b0 + fg * FNR + i;
+          v[i] = 0.f;
+          if (FULL || r < nr) {
+            const uint4 kw = *reinterpret_cast<const uint4 *>(kb + (size_t)r * RS);
+            float a0 = tcda::dot2_bf16(qb[0], kw.x, 0.f), a1 = tcda::dot2_bf16(qb[1], kw.y, 0.f);
+            a0 = tcda::dot2_bf16(qb[2], kw.z, a0);
+            a1 = tcda::dot2_bf16(qb[3], kw.w, a1);
+            v[i] = a0 + a1;
+          }
+        }
+#pragma unroll
+        for (int stp = 0; (FNR >> stp) > 1; stp++) {
+          const int mk = FCH >> (stp + 1), half = FNR >> (stp + 1);
+          const bool upper = (lane & mk) != 0;
+#pragma unroll
+          for (int i = 0; i < half; i++) {
+            const float send = upper ? v[i] : v[i + half];
+            const float keep = upper ? v[i + half] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, mk);
+          }
+        }
+#pragma unroll
+        for (int mk = FDUP / 2; mk >= 1; mk >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], mk);
+        const bool valid = FULL || b0 + myrow < nr;
+        const float x = valid ? v[0] * sl2 : -INFINITY;
+        float xm = x;
+#pragma unroll
+        for (int mk = FDUP; mk < 32; mk <<= 1) xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, mk));
+        const float mn = fmaxf(m, xm);
+        const float alpha = tcda::ex2a(m - mn);
+        const float p = valid ? tcda::ex2a(x - mn) : 0.f;
+        float ps = p;
+#pragma unroll
+        for (int mk = FDUP; mk < 32; mk <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, mk);
+        lsum = lsum * alpha + ps;
+        m = mn;
+        const uint64_t al2 = tcda::pk2(alpha, alpha);
+#pragma unroll
+        for (int w = 0; w < 4; w++) o2[w] = tcda::mul2(o2[w], al2);
+#pragma unroll
+        for (int i = 0; i < FNR; i++) {
+          const float pi = __shfl_sync(0xffffffffu, p, fg * FCH + i * FDUP);
+          const int r = b0 + fg * FNR + i;
+          if (FULL || r < nr) {
+            const uint4 vw = *reinterpret_cast<const uint4 *>(vb + (size_t)r * RS);
+            const uint64_t p2 = tcda::pk2(pi, pi);
+            o2[0] = tcda::fma2(p2, tcda::bf2_to_f2(vw.x), o2[0]);
+            o2[1] = tcda::fma2(p2, tcda::bf2_to_f2(vw.y), o2[1]);
+            o2[2] = tcda::fma2(p2, tcda::bf2_to_f2(vw.z), o2[2]);
+            o2[3] = tcda::fma2(p2, tcda::bf2_to_f2(vw.w), o2[3]);
+          }
+        }
+      };
+#pragma unroll 1
+      for (int b0 = warp * 8; b0 < nr; b0 += NW * 8) {
+        if (b0 + 8 <= nr) batch(b0, std::true_type{});
+        else batch(b0, std::false_type{});
+      }
+    } else
     for (int g = warp * RPW; g < nr; g += NW * RPW * U) {
       float s[U], vv[U][VEC];
 #pragma unroll
@@ -814,6 +896,14 @@ __global__ void __launch_bounds__(256) dec_bulk_kernel(DecBulkArgs a) {
     if (threadIdx.x == 0 && issued < nch) {
       issue(issued);
       issued++;
+    }
+  }
+  if constexpr (FAST) {
+#pragma unroll
+    for (int w = 0; w < 4; w++) {
+      const float2 f = tcda::up2(o2[w]);
+      o[2 * w] = f.x;
+      o[2 * w + 1] = f.y;
     }
   }
 #pragma unroll

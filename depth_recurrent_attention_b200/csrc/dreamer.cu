@@ -662,6 +662,8 @@ static void launch_dec_bulk(dreamer_handle *h, const RowsArgs &r, int d, cudaStr
   DecBulkArgs a{};
   a.B = r.B; a.H = r.H; a.L = r.L; a.l = r.l; a.cap = r.cap; a.nsplit = r.nsplit;
   int chunk = (int)(8192 / (d * (long)sizeof(T)));  // 8 KB of keys (and of values) a stage
+  // bf16 at head dim 64 / 128 takes 8-row batches, one a warp: 64 rows a stage
+  if (sizeof(T) == 2 && (d == 64 || d == 128)) chunk = 64;
   a.chunk = chunk > 256 ? 256 : chunk;
   a.q = r.q; a.ldq = r.ldq; a.kc = r.kv; a.vc = r.vc; a.cache_len = r.cache_len;
   a.part = r.part; a.err = r.err;
