@@ -98,7 +98,7 @@ template <int D>
 struct SaCfg {
   static constexpr int CH = D / 64;                 // 64-column chunks of a head
   static constexpr int TILE = 128 * 128;            // bytes of one [128 x 64] bf16 chunk
-  static constexpr int KST = D == 64 ? 4 : 3;       // K ring depth
+  static constexpr int KST = D == 64 ? 4 : 2;       // K ring depth
   static constexpr int VST = D == 64 ? 4 : 2;       // V ring depth
   static constexpr int Q_BYTES = 2 * CH * TILE;     // both query tiles
   static constexpr int KV_BYTES = CH * TILE;        // one K (or V) block
