@@ -479,9 +479,15 @@ __global__ void __launch_bounds__(1024) da_fast_kernel(DaBulkArgs a) {
     abort_flag = 0;
   }
   __syncthreads();
+  // the issuer's position in the (token, chunk) stream: no run-time divisions a chunk
+  int is_c = 0, is_tok = (int)blockIdx.x;
   auto issue = [&](int j) {
-    const int b = j % NB, c = j % nch;
-    const int tok = (int)blockIdx.x + (j / nch) * (int)gridDim.x;
+    const int b = j % NB, c = is_c;
+    const int tok = is_tok;
+    if (++is_c == nch) {
+      is_c = 0;
+      is_tok += (int)gridDim.x;
+    }
     const int r0 = c * a.chunk, nr = min(a.chunk, nrow - r0);
     const uint32_t kvb = (uint32_t)(nr * row_el * sizeof(bf16));
     const uint32_t bar = tcda::smem_u32(&bars[b]);
@@ -508,8 +514,9 @@ __global__ void __launch_bounds__(1024) da_fast_kernel(DaBulkArgs a) {
   uint32_t qb[4];  // the query slice as bf16 pairs
   float m = -INFINITY, lsum = 0.f;
   int consumed = 0;
+  int c = 0, ctok = (int)blockIdx.x;  // the consumer's (chunk, token) position
   for (int j = 0; j < nitems; j++) {
-    const int b = j % NB, c = j % nch;
+    const int b = j % NB;
     const uint32_t bar = tcda::smem_u32(&bars[b]);
     const uint32_t par = (uint32_t)((j / NB) & 1);
     if (!tcda::try_wait(bar, par)) {  // bounded; on expiry every thread stops after the barrier
@@ -621,7 +628,7 @@ __global__ void __launch_bounds__(1024) da_fast_kernel(DaBulkArgs a) {
 #pragma unroll
           for (int i = 0; i < 8; i++) of[i] += __shfl_xor_sync(0xffffffffu, of[i], mk);
         if (g == 0 && !abort_flag) {
-          const int tok = (int)blockIdx.x + (j / nch) * (int)gridDim.x;
+          const int tok = ctok;
           const float inv = 1.0f / lsum;
 #pragma unroll
           for (int i = 0; i < 8; i++) of[i] *= inv;
@@ -635,6 +642,10 @@ __global__ void __launch_bounds__(1024) da_fast_kernel(DaBulkArgs a) {
     if (threadIdx.x == 0 && issued < nitems) {
       issue(issued);
       issued++;
+    }
+    if (++c == nch) {
+      c = 0;
+      ctok += (int)gridDim.x;
     }
   }
   // copies still in flight after an abort land before the CTA exits
