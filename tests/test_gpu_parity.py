@@ -110,6 +110,34 @@ def test_router_strict(cuda, name, l):
         assert np.array_equal(c, ref["counts"])
 
 
+@pytest.mark.parametrize("pattern", ["all-equal", "every-third"])
+def test_router_exact_ties_on_the_tensor_core_path(cuda, pattern):
+    """Scores tied exactly at the selection bound, on the path that stores the scores and picks
+    a token's top k from them (9728 tokens: enough 128-row tiles for the tensor-core scores;
+    E = 256, k = 4).  Zero router keys make every raw score 0, so the biased score is the bias:
+    all equal (every lane's maximum ties, so the candidates exceed a warp and the k rounds of a
+    warp-wide best run) or 1 on every third expert and 0 elsewhere.  The picks must be the k
+    lowest-index experts among the best, each weighted 1/k."""
+    cfg = configs.SMALL.with_(batch=19)
+    assert cfg.tokens // 128 >= 74
+    W = dict(inputs.host_weights(cfg))
+    E, k = cfg.n_experts, cfg.top_k
+    W["k_E"] = np.zeros_like(W["k_E"])
+    if pattern == "all-equal":
+        W["bias"] = np.zeros(E, np.float32)
+        want = np.arange(k)
+    else:
+        W["bias"] = (np.arange(E) % 3 == 0).astype(np.float32)
+        want = np.arange(0, 3 * k, 3)
+    dev = make_handle(cfg, W)
+    y = inputs.extra_normal(cfg, 3000, (cfg.tokens, cfg.hidden), 1.0)
+    idx, w, counts = dev.route_experts(0, inputs.to_device(y, cfg.dtype))
+    idx, w, counts = idx.cpu().numpy(), PY.to_np(w), counts.cpu().numpy()
+    assert np.array_equal(np.sort(idx, axis=-1), np.broadcast_to(want, idx.shape))
+    assert np.allclose(w, 1.0 / k, atol=1e-6)
+    assert np.array_equal(counts, np.bincount(idx.ravel(), minlength=E))
+
+
 # ---------------------------------------------------------------------------------------
 # small, bf16: one depth at a time from seeded states (every depth)
 
