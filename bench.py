@@ -3,7 +3,9 @@
 
 Metric: token-depth-steps per second (one unit = one token through one depth step) of the
 full L-depth forward, bf16, and its fraction of the roofline
-T_roof = max(F_alg / tensor peak, B_alg / HBM peak) with both peaks measured on this machine.
+T_roof = max(F_alg / tensor peak, B_alg / HBM peak) with both peaks measured on B200: the HBM
+copy bandwidth, and the bf16 GEMM rate sustained under the power cap for a timed loop of a
+second or more (the burst rate for a shorter one; the other one is reported beside it).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config large|medium|small|decode|...]
 
@@ -280,7 +282,14 @@ def run_ours(args, cfg, rank, world, torch, dist):
     counts = model.route_counts(on_host=True).numpy()
     stage_alg, F, B = algorithmic(cfg, counts)
     pk = peaks()
-    t_roof = max(F / (pk["tc"] * 1e12), B / (pk["hbm"] * 1e9))
+    # the tensor peak a kernel is held to: the sustained GEMM figure when the timed region is a
+    # loop of a second or more (the GPU then runs at its power cap, as the sustained figure was
+    # measured), the burst figure for a shorter one; the other figure is reported beside it
+    long_loop = ms_total >= 1000.0
+    tc_peak = pk["tc_sust"] if long_loop else pk["tc"]
+    tc_other = pk["tc"] if long_loop else pk["tc_sust"]
+    t_roof = max(F / (tc_peak * 1e12), B / (pk["hbm"] * 1e9))
+    t_roof_other = max(F / (tc_other * 1e12), B / (pk["hbm"] * 1e9))
     per_stage = {}
     for name, ms in st["ms"].items():
         n = max(st["count"][name], 1)
@@ -290,12 +299,15 @@ def run_ours(args, cfg, rank, world, torch, dist):
     dominant = max(timed, key=lambda k: per_stage[k])
     fl, by = stage_alg.get(dominant, (0.0, 0.0))
     t_dom = per_stage[dominant] / 1e3  # s per forward
-    bound_tensor = fl / (pk["tc"] * 1e12) > by / (pk["hbm"] * 1e9)
+    bound_tensor = fl / (tc_peak * 1e12) > by / (pk["hbm"] * 1e9)
     launches_per_fwd = max(st["count"][dominant] // max(args.steps, 1), 1)
     if bound_tensor:
         achieved = fl / t_dom / 1e12
-        roof = dict(bound="tensor", achieved=achieved, peak=pk["tc"], unit="TFLOP/s",
-                    frac=achieved / pk["tc"])
+        roof = dict(bound="tensor", achieved=achieved, peak=tc_peak, unit="TFLOP/s",
+                    frac=achieved / tc_peak,
+                    peak_kind="sustained" if long_loop else "burst",
+                    other_peak={"kind": "burst" if long_loop else "sustained",
+                                "peak": tc_other, "frac": achieved / tc_other})
     else:
         achieved = by / t_dom / 1e9
         roof = dict(bound="hbm", achieved=achieved, peak=pk["hbm"], unit="GB/s",
@@ -304,9 +316,10 @@ def run_ours(args, cfg, rank, world, torch, dist):
                 launches_per_step=launches_per_fwd,
                 traffic=None if args.reduced else measured_traffic(cfg.name, dominant),
                 alg_bytes_per_launch=by / launches_per_fwd,
-                peak_source=("measured (MEASURED_PEAKS.json burst figure)" if pk["source"] == "measured"
-                             else "fallback (no MEASURED_PEAKS.json: 6650 GB/s copy, 1590 TFLOP/s "
-                                  "bf16 GEMM burst, an earlier B200 measurement)"))
+                peak_source=("measured (MEASURED_PEAKS.json)" if pk["source"] == "measured"
+                             else "fallback (no MEASURED_PEAKS.json: 6650 GB/s copy; bf16 GEMM "
+                                  "1590 TFLOP/s burst, 1400 TFLOP/s sustained under the power "
+                                  "cap; earlier B200 measurements)"))
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -363,8 +376,11 @@ def run_ours(args, cfg, rank, world, torch, dist):
         "roofline": roof,
         "roofline_step": {"t_roof_ms": t_roof * 1e3, "t_meas_ms": ms_step,
                           "frac": t_roof * 1e3 / ms_step, "F_alg": F, "B_alg": B,
-                          "peaks": {"tensor_tflops": pk["tc"], "hbm_gbs": pk["hbm"],
-                                    "source": pk["source"]}},
+                          "peaks": {"tensor_tflops": tc_peak,
+                                    "tensor_kind": "sustained" if long_loop else "burst",
+                                    "hbm_gbs": pk["hbm"], "source": pk["source"]},
+                          "frac_other_tensor_peak": {"tensor_tflops": tc_other,
+                                                     "frac": t_roof_other * 1e3 / ms_step}},
         "stage_ms_per_step": per_stage,
         "e2e": e2e,
         "gpu_launches": launches,
