@@ -577,7 +577,10 @@ __global__ void __launch_bounds__(256) expert_rows_kernel(const T *X, const int 
                                                           const T *w1t, const T *w2t, T *Y) {
   pdl_wait();
   pdl_trigger();
-  constexpr int XC = 8;  // 16-byte x chunks a lane keeps (h <= 2048)
+  constexpr int XC = 8;  // 16-byte x chunks a lane covers (h <= 2048)
+  // the row x in shared memory as fp32 (in registers it would take 64 a thread and cap the
+  // CTAs an SM holds at two)
+  __shared__ __align__(16) float xs[XC * 256];
   __shared__ float hs[M];
   const int slot = blockIdx.x;
   if (slot >= nslots) return;
@@ -586,13 +589,17 @@ __global__ void __launch_bounds__(256) expert_rows_kernel(const T *X, const int 
   const T *x = X + (long)tok * h;
   const T *W1 = w1t + (long)e * M * h;
   const T *W2 = w2t + (long)e * h * M;
-  float xr[XC][8];
-#pragma unroll
-  for (int t = 0; t < XC; t++) {
-    const int i = t * 256 + lane * 8;
-    if (i < h) load8(x + i, xr[t]);
+  for (int i = threadIdx.x * 8; i < h; i += 256 * 8) {
+    float xv[8];
+    load8(x + i, xv);
+    *reinterpret_cast<float4 *>(xs + i) = make_float4(xv[0], xv[1], xv[2], xv[3]);
+    *reinterpret_cast<float4 *>(xs + i + 4) = make_float4(xv[4], xv[5], xv[6], xv[7]);
   }
-  for (int j = warp; j < M; j += 8) {  // up: one hidden unit a warp at a time
+  __syncthreads();
+  // up: one hidden unit a warp at a time, two in flight
+#pragma unroll 2
+  for (int jj = 0; jj < M / 8; jj++) {
+    const int j = warp + 8 * jj;
     float a = 0.f;
 #pragma unroll
     for (int t = 0; t < XC; t++) {
@@ -600,14 +607,19 @@ __global__ void __launch_bounds__(256) expert_rows_kernel(const T *X, const int 
       if (i < h) {
         float wv[8];
         load8(W1 + (long)j * h + i, wv);
-#pragma unroll
-        for (int q = 0; q < 8; q++) a = fmaf(xr[t][q], wv[q], a);
+        const float4 x0 = *reinterpret_cast<const float4 *>(xs + i);
+        const float4 x1 = *reinterpret_cast<const float4 *>(xs + i + 4);
+        a = fmaf(x0.x, wv[0], a); a = fmaf(x0.y, wv[1], a);
+        a = fmaf(x0.z, wv[2], a); a = fmaf(x0.w, wv[3], a);
+        a = fmaf(x1.x, wv[4], a); a = fmaf(x1.y, wv[5], a);
+        a = fmaf(x1.z, wv[6], a); a = fmaf(x1.w, wv[7], a);
       }
     }
     a = warp_sum(a);
     if (lane == 0) hs[j] = to_f(from_f<T>(a / (1.0f + __expf(-a))));
   }
   __syncthreads();
+#pragma unroll 4
   for (int c = threadIdx.x; c < h; c += blockDim.x) {  // down: one output column a thread
     const T *w = W2 + (long)c * M;
     float a = 0.f;
@@ -1291,7 +1303,7 @@ __global__ void __launch_bounds__(256, 3) route_q_topk_kernel(const bf16 *qs3, c
 // lists, and CTA 0 ranks the NCL lists read from its peers' shared memory.  wqt: W_q
 // transposed [d_r][h]; kraw: [E][d_r]; rope: the router dim's depth-RoPE row of this depth.
 template <typename T, int DR>
-__global__ void __launch_bounds__(256) route_cluster_kernel(const T *y, int h, const T *wqt,
+__global__ void __launch_bounds__(256, 4) route_cluster_kernel(const T *y, int h, const T *wqt,
                                                             const T *kraw, const float2 *rope,
                                                             TopkArgs a) {
   pdl_wait();
@@ -1310,6 +1322,7 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(const T *y, int h, c
     const T *yr = y + (long)tok * h;
     for (int j = rank * qn + wib; j < (rank + 1) * qn; j += 8) {
       float acc = 0.f;
+#pragma unroll 4
       for (int i = lane * 8; i < h; i += 256) {
         float yv[8], wv[8];
         load8(yr + i, yv);
@@ -1335,9 +1348,9 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(const T *y, int h, c
   __syncthreads();
   WarpTopK t(a.k, lane);
   if (live) {
-    float q[DR];
-#pragma unroll
-    for (int j = 0; j < DR; j++) q[j] = qv[j];
+    // q stays in shared memory (every lane reads the same words): as registers it would
+    // take DR of them a thread and halve the CTAs an SM holds
+    const float4 *q4 = reinterpret_cast<const float4 *>(qv);
     const int per_cta = (a.E + ncl - 1) / ncl;
     const int c0 = rank * per_cta, c1 = min(a.E, c0 + per_cta);
     const int per_w = (c1 - c0 + 7) / 8;
@@ -1347,12 +1360,15 @@ __global__ void __launch_bounds__(256) route_cluster_kernel(const T *y, int h, c
       float z = 0.f;
       if (e < e1) {
         const T *kr = kraw + (long)e * DR;
-#pragma unroll
+#pragma unroll 4
         for (int j = 0; j < DR; j += 8) {
           float kv[8];
           load8(kr + j, kv);
-#pragma unroll
-          for (int u = 0; u < 8; u++) z = fmaf(q[j + u], kv[u], z);
+          const float4 qa = q4[j / 4], qb = q4[j / 4 + 1];
+          z = fmaf(qa.x, kv[0], z); z = fmaf(qa.y, kv[1], z);
+          z = fmaf(qa.z, kv[2], z); z = fmaf(qa.w, kv[3], z);
+          z = fmaf(qb.x, kv[4], z); z = fmaf(qb.y, kv[5], z);
+          z = fmaf(qb.z, kv[6], z); z = fmaf(qb.w, kv[7], z);
         }
       }
       t.offer_score(z * a.zscale, e, e < e1, a.bias);

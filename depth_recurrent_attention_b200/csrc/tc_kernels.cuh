@@ -380,7 +380,8 @@ static bool tc_gemm_ok(dreamer_handle *h, const dreamer::GemmArgs &a) {
 // N tile of the projection GEMMs (64, 128 or 256): the wider tile reads A fewer times, the
 // narrower one spreads a small problem over more SMs; take the one with the shorter critical
 // path (waves of tiles x tile width plus a fixed per-tile cost of about 32 columns).
-static int tc_pick_bn(dreamer_handle *h, const dreamer::GemmArgs &a) {
+// min_bn: 64 for epilogues that pair columns 32 apart (the QKV RoPE), else 16
+static int tc_pick_bn(dreamer_handle *h, const dreamer::GemmArgs &a, int min_bn = 64) {
   const long mt = (a.M + 127) / 128 + (a.goffs ? a.G : 0);
   auto cost = [&](int bn) {
     const long tiles = mt * (a.N / bn);
@@ -389,6 +390,10 @@ static int tc_pick_bn(dreamer_handle *h, const dreamer::GemmArgs &a) {
   int best = 128;
   if (a.N % 256 == 0 && cost(256) <= cost(best)) best = 256;
   if (cost(64) < cost(best)) best = 64;  // few tiles: narrower ones reach more SMs
+  // a single row tile (decode): every N tile streams its own slice of B, so narrower tiles
+  // put more SMs on the weights
+  if (min_bn <= 32 && a.N % 32 == 0 && cost(32) < cost(best)) best = 32;
+  if (min_bn <= 16 && a.N % 16 == 0 && cost(16) < cost(best)) best = 16;
   return best;
 }
 
@@ -455,8 +460,16 @@ static bool tc_gemm_o(dreamer_handle *h, const dreamer::GemmArgs &a, const dream
     CUtensorMap ta, tb;
     long mt;
     const bool ew8 = a.K <= 1024;  // as for the QKV projection
-    const int bn = tc_pick_bn(h, a);
-    if (bn == 64) {
+    const int bn = tc_pick_bn(h, a, 16);
+    if (bn == 16) {
+      if (!tc_prepare<16, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
+      if (a.arow && !a.a_sorted) tc_launch<16, 64, 8, 2, 16>(h, t, ta, tb, mt, e, s);
+      else tc_launch<16, 64, 8, 0, 16>(h, t, ta, tb, mt, e, s);
+    } else if (bn == 32) {
+      if (!tc_prepare<32, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
+      if (a.arow && !a.a_sorted) tc_launch<32, 64, 8, 2, 32>(h, t, ta, tb, mt, e, s);
+      else tc_launch<32, 64, 8, 0, 32>(h, t, ta, tb, mt, e, s);
+    } else if (bn == 64) {
       if (!tc_prepare<64, 64>(h, a, h->ptiles_b, a.M, t, ta, tb, mt)) return false;
       if (a.arow && !a.a_sorted) tc_launch<64, 64, 8, 2, 64>(h, t, ta, tb, mt, e, s);
       else tc_launch<64, 64, 8, 0, 64>(h, t, ta, tb, mt, e, s);
