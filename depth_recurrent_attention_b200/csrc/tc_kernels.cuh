@@ -377,7 +377,7 @@ static bool tc_gemm_ok(dreamer_handle *h, const dreamer::GemmArgs &a) {
   return a.N % 256 == 0 && a.K % 64 == 0 && (d == 64 || d == 128);
 }
 
-// N tile of the projection GEMMs (64, 128 or 256): the wider tile reads A fewer times, the
+// N tile of the projection GEMMs (16 to 256): the wider tile reads A fewer times, the
 // narrower one spreads a small problem over more SMs; take the one with the shorter critical
 // path (waves of tiles x tile width plus a fixed per-tile cost of about 32 columns).
 // min_bn: 64 for epilogues that pair columns 32 apart (the QKV RoPE), else 16
