@@ -364,6 +364,30 @@ def test_sa_causality_and_single_token():
     assert np.array_equal(a[8:], b[8:])          # other sequence untouched
 
 
+def test_sa_with_zero_keys_is_the_causal_running_mean_of_values():
+    """Sequence attention with every key zero: all scores are 0, so the causal softmax gives
+    each of the keys 0..t the weight 1/(t+1) and position t returns the running mean of v over
+    its own sequence (papernotes "Overall framework": causal attention over time steps;
+    reading R4).  A dropped mask would average over the whole sequence, a wrong limit or a
+    missing normaliser would change the count.  L = 1, the DA rows of W_O and the experts'
+    W2 zero, the SA rows of W_O the identity: x_1 = x^ + running_mean(x^ W_v)."""
+    cfg = tiny_cfg(batch=2, seq=8, depth=1, n_experts=2, top_k=1)
+    W = rand_weights(cfg, seed=11)
+    h, s = cfg.hidden, cfg.seq
+    W["w_qkv"] = W["w_qkv"].copy()
+    W["w_qkv"][0][:, h:2 * h] = 0.0                   # k_SA = 0
+    W["w_o"] = np.zeros_like(W["w_o"])
+    W["w_o"][0, :h, :] = np.eye(h, dtype=np.float32)   # SA rows: identity; DA rows: 0
+    W["w2"] = np.zeros_like(W["w2"])
+    x0 = inputs.host_inputs(cfg)["x0"]
+    r = O.Oracle(cfg, W, threads=1).forward(x0)
+    x = x0.astype(np.float64)
+    xh = x / np.sqrt(np.mean(x ** 2, 1, keepdims=True) + cfg.rms_eps)
+    v = (xh @ W["w_qkv"][0][:, 2 * h:3 * h].astype(np.float64)).reshape(cfg.batch, s, h)
+    run_mean = np.cumsum(v, axis=1) / np.arange(1, s + 1)[None, :, None]
+    assert np.allclose(r["x_out"], xh + run_mean.reshape(-1, h), rtol=1e-12, atol=1e-12)
+
+
 def test_batch_permutation_equivariance():
     cfg = tiny_cfg(batch=3, seq=4, depth=2)
     W = rand_weights(cfg, seed=6)
