@@ -388,6 +388,33 @@ def test_sa_with_zero_keys_is_the_causal_running_mean_of_values():
     assert np.allclose(r["x_out"], xh + run_mean.reshape(-1, h), rtol=1e-12, atol=1e-12)
 
 
+def test_da_with_zero_keys_is_the_running_mean_over_depths():
+    """Depth attention with every key zero: the token's scores over depths 0..l are all 0, so
+    depth l returns the mean of v_DA over depths 0..l, the current one included (papernotes
+    "Key design 1": attention over the token's own earlier depth states; reading R2).  SA rows
+    of W_O and the experts' W2 zero, the DA rows of W_O the identity, L = 4: the recurrence
+    x^_l = RMSNorm(x_l), v_l = x^_l W_v, x_{l+1} = x^_l + mean(v_0..v_l) in closed form.  An
+    exclusive slice, a missing normaliser or a depth read from the wrong slot all fail."""
+    cfg = tiny_cfg(batch=1, seq=4, depth=4, n_experts=2, top_k=1)
+    W = rand_weights(cfg, seed=12)
+    h = cfg.hidden
+    W["w_qkv"] = W["w_qkv"].copy()
+    W["w_qkv"][0][:, 4 * h:5 * h] = 0.0                # k_DA = 0
+    W["w_o"] = np.zeros_like(W["w_o"])
+    W["w_o"][0, h:, :] = np.eye(h, dtype=np.float32)   # DA rows: identity; SA rows: 0
+    W["w2"] = np.zeros_like(W["w2"])
+    x0 = inputs.host_inputs(cfg)["x0"]
+    r = O.Oracle(cfg, W, threads=1).forward(x0)
+    Wv = W["w_qkv"][0][:, 5 * h:6 * h].astype(np.float64)
+    x = x0.astype(np.float64)
+    vs = []
+    for _ in range(cfg.depth):
+        xh = x / np.sqrt(np.mean(x ** 2, 1, keepdims=True) + cfg.rms_eps)
+        vs.append(xh @ Wv)
+        x = xh + np.mean(vs, axis=0)
+    assert np.allclose(r["x_out"], x, rtol=1e-12, atol=1e-12)
+
+
 def test_batch_permutation_equivariance():
     cfg = tiny_cfg(batch=3, seq=4, depth=2)
     W = rand_weights(cfg, seed=6)
