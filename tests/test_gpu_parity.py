@@ -230,6 +230,18 @@ def test_small_expert_sizes_bf16(cuda, m):
         run_step_and_compare(cfg, W, dev, l, orc=orc)
 
 
+def test_short_batch_wide_hidden_bf16(cuda):
+    """256 tokens at h = 2048 (16 heads of 128): the O projection takes 32-column tiles (two
+    row tiles × 64 N tiles), the router its cluster form and the experts their per-row
+    form (about 4 routed rows per expert), all in a prefill step."""
+    cfg = configs.SMALL.with_(batch=2, seq=128, hidden=2048, n_heads=16, head_dim=128, depth=2)
+    W = inputs.host_weights(cfg)
+    dev = make_handle(cfg, W)
+    orc = O.Oracle(cfg, W)
+    for l in (0, 1):
+        run_step_and_compare(cfg, W, dev, l, orc=orc)
+
+
 @pytest.mark.parametrize("variant", [1, 2])
 def test_small_layout_variants_bf16(cuda, variant):
     cfg = configs.SMALL.with_(variant=variant, depth=3)
