@@ -1304,8 +1304,8 @@ __global__ void __launch_bounds__(256, 3) route_q_topk_kernel(const bf16 *qs3, c
 // transposed [d_r][h]; kraw: [E][d_r]; rope: the router dim's depth-RoPE row of this depth.
 template <typename T, int DR>
 __global__ void __launch_bounds__(256, 4) route_cluster_kernel(const T *y, int h, const T *wqt,
-                                                            const T *kraw, const float2 *rope,
-                                                            TopkArgs a) {
+                                                               const T *kraw, const float2 *rope,
+                                                               TopkArgs a) {
   pdl_wait();
   pdl_trigger();
   namespace cg = cooperative_groups;
