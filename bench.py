@@ -53,6 +53,15 @@ def peaks():
         return dict(hbm=6650.0, tc=1590.0, tc_sust=1400.0, source="fallback")
 
 
+def tensor_peaks(pk, timed_ms: float):
+    """(peak held to, the other peak, its kind) in TFLOP/s: the sustained GEMM figure when the
+    timed region is a loop of a second or more (the GPU then runs at its power cap, as the
+    sustained figure was measured), the burst figure for a shorter one."""
+    if timed_ms >= 1000.0:
+        return pk["tc_sust"], pk["tc"], "sustained"
+    return pk["tc"], pk["tc_sust"], "burst"
+
+
 def algorithmic(cfg, counts=None):
     """Per-stage algorithmic FLOPs and HBM bytes of one full forward (or decode step), by the
     accounting of the roofline: every multiply-add of a contraction counted twice at tensor
@@ -282,12 +291,9 @@ def run_ours(args, cfg, rank, world, torch, dist):
     counts = model.route_counts(on_host=True).numpy()
     stage_alg, F, B = algorithmic(cfg, counts)
     pk = peaks()
-    # the tensor peak a kernel is held to: the sustained GEMM figure when the timed region is a
-    # loop of a second or more (the GPU then runs at its power cap, as the sustained figure was
-    # measured), the burst figure for a shorter one; the other figure is reported beside it
-    long_loop = ms_total >= 1000.0
-    tc_peak = pk["tc_sust"] if long_loop else pk["tc"]
-    tc_other = pk["tc"] if long_loop else pk["tc_sust"]
+    # the tensor peak a kernel is held to (tensor_peaks); the other figure is reported beside it
+    tc_peak, tc_other, tc_kind = tensor_peaks(pk, ms_total)
+    long_loop = tc_kind == "sustained"
     t_roof = max(F / (tc_peak * 1e12), B / (pk["hbm"] * 1e9))
     t_roof_other = max(F / (tc_other * 1e12), B / (pk["hbm"] * 1e9))
     per_stage = {}

@@ -79,3 +79,15 @@ def test_da_window_and_no_da_arms():
     assert st["o_proj"][0] == 8 * 2.0 * T * h * h
     assert f == SMALL_FLOPS - 150_994_944 - 8 * (3_221_225_472 + 1_073_741_824)
     assert b == SMALL_BYTES - 117_440_512 - 8 * (4_194_304 + 4 * h * h * 2)
+
+
+def test_tensor_peak_follows_the_length_of_the_timed_loop():
+    """Kernels timed inside a loop of a second or more run at the power cap: they are held to
+    the sustained GEMM rate; shorter loops to the burst rate; the other rate is reported."""
+    pk = dict(hbm=6650.0, tc=1590.0, tc_sust=1400.0, source="fallback")
+    assert bench.tensor_peaks(pk, 2041.0) == (1400.0, 1590.0, "sustained")
+    assert bench.tensor_peaks(pk, 1000.0) == (1400.0, 1590.0, "sustained")
+    assert bench.tensor_peaks(pk, 150.9) == (1590.0, 1400.0, "burst")
+    fb = bench.peaks()
+    if fb["source"] == "fallback":
+        assert (fb["hbm"], fb["tc"], fb["tc_sust"]) == (6650.0, 1590.0, 1400.0)
