@@ -351,6 +351,9 @@ def flip_free(cfg):
     ("small", [300, 1, 77, 299], dict(n_experts=4, top_k=4, depth=3, n_heads=4, head_dim=128)),
     ("small", [300, 1, 77, 299], dict(n_experts=4, top_k=4, depth=4, da_window=2)),
     ("tiny", [12, 5, 0], dict(variant=3)),
+    # one sequence with an empty cache; 130 sequences (two row tiles in the projections)
+    ("small", [0], {}),
+    ("small", [(7 * i) % 61 for i in range(130)], dict(depth=3)),
 ])
 def test_decode_step(cuda, base, lens, kw):
     torch = _torch()
