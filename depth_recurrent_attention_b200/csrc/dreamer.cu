@@ -936,11 +936,12 @@ static void run_depth(dreamer_handle *h, int l, bool first, bool last, const Dep
     prow = h->prows;
     psig = h->psig;
     if (sorted) {
-      const long chunks = (long)n * (hd / 8);
-      launch_k(h, gather_rows_kernel, dim3((unsigned)cdiv(chunks, 256) < 4u * h->num_sms
-                                               ? (unsigned)cdiv(chunks, 256) : 4u * h->num_sms),
-               dim3(256), 0, s, (const bf16 *)h->xh, (const int *)h->prows, (bf16 *)h->xh_sorted,
-               n, hd);
+      // four rows a CTA at a time, a thread a 16-byte chunk of each
+      const int threads = hd / 8 < 32 ? 32 : (hd / 8 > 256 ? 256 : hd / 8);
+      const long groups = cdiv(n, 4);
+      const long cap = 2048L / threads * h->num_sms;  // the CTAs resident at once
+      launch_k(h, gather_rows_kernel, dim3((unsigned)(groups < cap ? groups : cap)), dim3(threads),
+               0, s, (const bf16 *)h->xh, (const int *)h->prows, (bf16 *)h->xh_sorted, n, hd);
     }
   }
   auto grouped = [&](int N, int K, const void *A, long lda, const void *B, long bgs) {

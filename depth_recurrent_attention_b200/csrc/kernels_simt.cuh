@@ -1561,17 +1561,26 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int *cnt, int G, co
 // dst[r] = src[rows[r]] for r < n, rows of h bf16 (16-byte chunks, grid-stride): the
 // normalised states in the order of the projection experts' groups, so that the grouped QKV
 // projection loads its A tiles with TMA.
+// A CTA copies four rows at a time, its threads taking the rows' 16-byte chunks, so a thread
+// keeps four independent loads in flight (one at a time left most of HBM idle).
 __global__ void gather_rows_kernel(const bf16 *src, const int *rows, bf16 *dst, int n, int h) {
   pdl_wait();
   pdl_trigger();
+  constexpr int RB = 4;
   const int cpr = h / 8;
-  const long total = (long)n * cpr;
-  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long)gridDim.x * blockDim.x) {
-    const long r = i / cpr;
-    const int c = (int)(i % cpr) * 8;
-    *reinterpret_cast<uint4 *>(dst + r * h + c) =
-        *reinterpret_cast<const uint4 *>(src + (long)rows[r] * h + c);
+  for (int r0 = blockIdx.x * RB; r0 < n; r0 += gridDim.x * RB) {
+    const bf16 *sr[RB];
+#pragma unroll
+    for (int u = 0; u < RB; u++) sr[u] = r0 + u < n ? src + (long)rows[r0 + u] * h : nullptr;
+    for (int c = threadIdx.x; c < cpr; c += blockDim.x) {
+      uint4 v[RB];
+#pragma unroll
+      for (int u = 0; u < RB; u++)
+        if (sr[u]) v[u] = *reinterpret_cast<const uint4 *>(sr[u] + c * 8);
+#pragma unroll
+      for (int u = 0; u < RB; u++)
+        if (sr[u]) *reinterpret_cast<uint4 *>(dst + (long)(r0 + u) * h + c * 8) = v[u];
+    }
   }
 }
 
