@@ -1558,9 +1558,8 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int *cnt, int G, co
   }
 }
 
-// dst[r] = src[rows[r]] for r < n, rows of h bf16 (16-byte chunks, grid-stride): the
-// normalised states in the order of the projection experts' groups, so that the grouped QKV
-// projection loads its A tiles with TMA.
+// dst[r] = src[rows[r]] for r < n, rows of h bf16: the normalised states in the order of the
+// projection experts' groups, so that the grouped QKV projection loads its A tiles with TMA.
 // A CTA copies four rows at a time, its threads taking the rows' 16-byte chunks, so a thread
 // keeps four independent loads in flight (one at a time left most of HBM idle).
 __global__ void gather_rows_kernel(const bf16 *src, const int *rows, bf16 *dst, int n, int h) {
