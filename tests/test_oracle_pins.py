@@ -388,6 +388,40 @@ def test_sa_with_zero_keys_is_the_causal_running_mean_of_values():
     assert np.allclose(r["x_out"], xh + run_mean.reshape(-1, h), rtol=1e-12, atol=1e-12)
 
 
+def test_sa_rotates_queries_and_keys_by_their_positions_in_the_sequence():
+    """Sequence attention over two tokens with one head of 4 dims, worked by hand: queries and
+    keys turn by their position inside the sequence (rotate-half pairs (0, 2) and (1, 3) at
+    angles p and p / 100, i.e. base 10000 over d = 4: reading R5), so the second token scores
+    the first by (R_1 q_1) . k_0 and itself by q_1 . k_1 (a rotation keeps the dot product);
+    values are not rotated.  SA rows of W_O the identity, DA rows and experts off, L = 1."""
+    cfg = tiny_cfg(batch=1, seq=2, hidden=4, n_heads=1, head_dim=4, depth=1, n_experts=2,
+                   top_k=1, router_dim=4)
+    W = rand_weights(cfg, seed=13)
+    h = cfg.hidden
+    W["w_o"] = np.zeros_like(W["w_o"])
+    W["w_o"][0, :h, :] = np.eye(h, dtype=np.float32)
+    W["w2"] = np.zeros_like(W["w2"])
+    x0 = inputs.host_inputs(cfg)["x0"]
+    r = O.Oracle(cfg, W, threads=1).forward(x0)
+    x = x0.astype(np.float64)
+    xh = x / np.sqrt(np.mean(x ** 2, 1, keepdims=True) + cfg.rms_eps)
+    Wf = W["w_qkv"][0].astype(np.float64)
+    q, k, v = xh @ Wf[:, 0:4], xh @ Wf[:, 4:8], xh @ Wf[:, 8:12]
+
+    def turn(u, p):   # angles p * 1 and p * 0.01 on the pairs (0, 2) and (1, 3)
+        a0, a1 = p * 1.0, p * 0.01
+        return np.array([u[0] * np.cos(a0) - u[2] * np.sin(a0),
+                         u[1] * np.cos(a1) - u[3] * np.sin(a1),
+                         u[0] * np.sin(a0) + u[2] * np.cos(a0),
+                         u[1] * np.sin(a1) + u[3] * np.cos(a1)])
+    s10 = turn(q[1], 1) @ k[0] / 2.0          # k_0 at position 0 is not turned
+    s11 = q[1] @ k[1] / 2.0
+    p0 = 1.0 / (1.0 + np.exp(s11 - s10))
+    a = np.stack([v[0], p0 * v[0] + (1 - p0) * v[1]])
+    assert abs(s10 - q[1] @ k[0] / 2.0) > 1e-3           # the rotation matters here
+    assert np.allclose(r["x_out"], xh + a, rtol=1e-12, atol=1e-12)
+
+
 def test_da_with_zero_keys_is_the_running_mean_over_depths():
     """Depth attention with every key zero: the token's scores over depths 0..l are all 0, so
     depth l returns the mean of v_DA over depths 0..l, the current one included (papernotes
