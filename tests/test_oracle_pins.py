@@ -422,6 +422,39 @@ def test_sa_rotates_queries_and_keys_by_their_positions_in_the_sequence():
     assert np.allclose(r["x_out"], xh + a, rtol=1e-12, atol=1e-12)
 
 
+def test_da_rotates_by_depth_with_the_second_half_reversed_worked_by_hand():
+    """Depth attention of one token over depths 0 and 1 (L = 2) with one head of 4 dims,
+    worked by hand: each half of the head (2 dims, one rotate-half pair at base^0 = 1 rad a
+    step) turns by the depth for the first half and by L - 1 - depth for the second (reading
+    R6, the pages' half-reversed depth RoPE), queries and keys alike; values are not turned.
+    SA rows of W_O and the experts off, DA rows of W_O the identity."""
+    cfg = tiny_cfg(batch=1, seq=1, hidden=4, n_heads=1, head_dim=4, depth=2, n_experts=2,
+                   top_k=1, router_dim=4)
+    W = rand_weights(cfg, seed=14)
+    h = cfg.hidden
+    W["w_o"] = np.zeros_like(W["w_o"])
+    W["w_o"][0, h:, :] = np.eye(h, dtype=np.float32)
+    W["w2"] = np.zeros_like(W["w2"])
+    x0 = inputs.host_inputs(cfg)["x0"]
+    r = O.Oracle(cfg, W, threads=1).forward(x0)
+    Wf = W["w_qkv"][0].astype(np.float64)
+    norm = lambda x: x / np.sqrt(np.mean(x ** 2, 1, keepdims=True) + cfg.rms_eps)
+
+    def turn(u, l):   # first half by l, second half by L - 1 - l (1 rad a step)
+        a, b = float(l), float(cfg.depth - 1 - l)
+        return np.array([u[0] * np.cos(a) - u[1] * np.sin(a), u[0] * np.sin(a) + u[1] * np.cos(a),
+                         u[2] * np.cos(b) - u[3] * np.sin(b), u[2] * np.sin(b) + u[3] * np.cos(b)])
+    xh0 = norm(x0.astype(np.float64))
+    k0, v0 = turn((xh0 @ Wf[:, 16:20])[0], 0), (xh0 @ Wf[:, 20:24])[0]
+    xh1 = norm(xh0 + v0)                      # depth 0 attends to itself only: a_0 = v_0
+    q1, k1, v1 = (xh1 @ Wf[:, 12:16])[0], (xh1 @ Wf[:, 16:20])[0], (xh1 @ Wf[:, 20:24])[0]
+    q1, k1 = turn(q1, 1), turn(k1, 1)
+    s0, s1 = q1 @ k0 / 2.0, q1 @ k1 / 2.0
+    p0 = 1.0 / (1.0 + np.exp(s1 - s0))
+    want = xh1 + p0 * v0 + (1 - p0) * v1
+    assert np.allclose(r["x_out"][0], want[0], rtol=1e-12, atol=1e-12)
+
+
 def test_da_with_zero_keys_is_the_running_mean_over_depths():
     """Depth attention with every key zero: the token's scores over depths 0..l are all 0, so
     depth l returns the mean of v_DA over depths 0..l, the current one included (papernotes
