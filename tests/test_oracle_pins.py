@@ -455,6 +455,41 @@ def test_da_rotates_by_depth_with_the_second_half_reversed_worked_by_hand():
     assert np.allclose(r["x_out"][0], want[0], rtol=1e-12, atol=1e-12)
 
 
+def test_expert_attention_scores_depth_rotated_keys_worked_by_hand():
+    """Expert attention of one token over two depths (L = 2), two experts, top-1, worked by
+    hand: the unrotated query q = y W_qE against each expert key turned by the half-reversed
+    depth rotation of the depth (reading R8: "depth-RoPE'd expert keys"), the pick by z + b
+    (R9), weight 1 (R10), x_{l+1} = y + SiLU(y W1_e) W2_e (R11).  W_O zero, so y_l = x^_l.
+    The seed is one where unrotated keys would pick another expert at both depths."""
+    cfg = tiny_cfg(batch=1, seq=1, hidden=4, n_heads=1, head_dim=4, depth=2, n_experts=2,
+                   top_k=1, router_dim=4, seed=21)
+    W = dict(inputs.host_weights(cfg))
+    W["w_o"] = np.zeros_like(W["w_o"])
+    x0 = inputs.host_inputs(cfg)["x0"]
+    r = O.Oracle(cfg, W, threads=1).forward(x0)
+    f = lambda a: np.asarray(a, np.float64)
+    norm = lambda x: x / np.sqrt(np.mean(x ** 2, 1, keepdims=True) + cfg.rms_eps)
+
+    def turn(u, l):   # first half by l, second half by L - 1 - l (1 rad a step)
+        a, b = float(l), float(cfg.depth - 1 - l)
+        return np.array([u[0] * np.cos(a) - u[1] * np.sin(a), u[0] * np.sin(a) + u[1] * np.cos(a),
+                         u[2] * np.cos(b) - u[3] * np.sin(b), u[2] * np.sin(b) + u[3] * np.cos(b)])
+    x, picks, unrotated = f(x0), [], []
+    for l in range(cfg.depth):
+        y = norm(x)
+        q = (y @ f(W["w_qE"]))[0]
+        z = np.array([q @ turn(f(W["k_E"][e]), l) / 2.0 for e in range(2)])
+        z_plain = np.array([q @ f(W["k_E"][e]) / 2.0 for e in range(2)])
+        e = int(np.argmax(z + f(W["bias"])))
+        picks.append(e)
+        unrotated.append(int(np.argmax(z_plain + f(W["bias"]))))
+        u = y @ f(W["w1"][e])
+        x = y + (u / (1.0 + np.exp(-u))) @ f(W["w2"][e])
+    assert picks != unrotated                              # the rotation decides here
+    assert [int(r["idx"][l][0][0]) for l in range(cfg.depth)] == picks
+    assert np.allclose(r["x_out"], x, rtol=1e-12, atol=1e-12)
+
+
 def test_da_with_zero_keys_is_the_running_mean_over_depths():
     """Depth attention with every key zero: the token's scores over depths 0..l are all 0, so
     depth l returns the mean of v_DA over depths 0..l, the current one included (papernotes
