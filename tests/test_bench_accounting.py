@@ -91,3 +91,20 @@ def test_tensor_peak_follows_the_length_of_the_timed_loop():
     fb = bench.peaks()
     if fb["source"] == "fallback":
         assert (fb["hbm"], fb["tc"], fb["tc_sust"]) == (6650.0, 1590.0, 1400.0)
+
+
+def test_reference_arm_line_on_a_tiny_workload():
+    """The reference arm (the oracle on the host cores) prints the bench line's keys with
+    impl "reference", a positive value, its own cpu_baseline and an e2e entry without copies."""
+    import json
+    import types
+    cfg = configs.TINY
+    args = types.SimpleNamespace(steps=2, warmup=1, gpus=1)
+    line = bench.run_reference(args, cfg)
+    json.dumps(line)
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == bench.UNIT
+    assert line["config"]["workload"].startswith("tiny")
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert "depths 0..3 of 4" in cb["sample"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
