@@ -267,6 +267,19 @@ def test_block_reduces_to_closed_form(P):
     assert np.allclose(r["x_out"], ref, rtol=1e-11, atol=1e-11)
 
 
+def test_block_closed_form_with_a_non_unit_norm_gain():
+    """The same single-token closed form with a random RMSNorm gain g (the configurations all
+    use g = 1): the block's normalised state is g * x / rms(x) wherever it is used (QKV input,
+    residual, projection router)."""
+    cfg = tiny_cfg(batch=3, seq=1, depth=1, n_experts=3, top_k=3, n_proj_experts=1)
+    W = dict(rand_weights(cfg, seed=15))
+    W["g"] = (0.5 + np.random.default_rng(15).random(cfg.hidden)).astype(np.float32)
+    x0 = inputs.host_inputs(cfg)["x0"]
+    r = O.Oracle(cfg, W, threads=1).forward(x0)
+    ref, _, _ = _closed_form_single_token(cfg, W, x0)
+    assert np.allclose(r["x_out"], ref, rtol=1e-11, atol=1e-11)
+
+
 def test_block_with_three_projection_experts_closed_form():
     """P = 3 projection experts with distinct QKV/O matrices; the keys are built so that the
     six tokens pick all three experts (token t aligns with expert t mod 3) and the argmin
