@@ -230,6 +230,19 @@ def test_small_expert_sizes_bf16(cuda, m):
         run_step_and_compare(cfg, W, dev, l, orc=orc)
 
 
+def test_small_random_norm_gain_bf16(cuda):
+    """A random RMSNorm gain (the configurations use g = 1): the first depth's norm, the
+    residual rebuilt in the O epilogue and the combine's norm for the next depth all apply it."""
+    cfg = configs.SMALL.with_(depth=2)
+    W = dict(inputs.host_weights(cfg))
+    g = np.random.default_rng(16).uniform(0.5, 1.5, cfg.hidden).astype(np.float32)
+    W["g"] = inputs.round_to(g, "bf16").astype(np.float32)
+    dev = make_handle(cfg, W)
+    orc = O.Oracle(cfg, W)
+    for l in (0, 1):
+        run_step_and_compare(cfg, W, dev, l, orc=orc)
+
+
 def test_short_batch_wide_hidden_bf16(cuda):
     """256 tokens at h = 2048 (16 heads of 128): the O projection takes 32-column tiles (two
     row tiles × 64 N tiles), the router its cluster form and the experts their per-row
